@@ -1,0 +1,221 @@
+"""ctypes front end of the fp64 OPQ oracle (``opq_oracle.c``).
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline leg are the only callers. The CUDA library never
+imports this package and shares no code with it.
+
+All array arguments are numpy arrays; bf16 tensors travel as their uint16 bit
+patterns. The shared object is built on first use with gcc (``build()``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "opq_oracle.c")
+_BUILD = os.path.join(_HERE, "_build")
+_SO = os.path.join(_BUILD, "liboracle.so")
+_lock = threading.Lock()
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle (plain C99, -O2, OpenMP over rows, no fast-math)."""
+    os.makedirs(_BUILD, exist_ok=True)
+    if force or not os.path.exists(_SO) or os.path.getmtime(_SO) < os.path.getmtime(_SRC):
+        tmp = _SO + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-std=c99", "-O2", "-fno-fast-math", "-fopenmp", "-fPIC",
+                               "-shared", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _SO)
+    return _SO
+
+
+def _bind(path: str):
+    lib = ctypes.CDLL(path)
+    P = ctypes.c_void_p
+    I = ctypes.c_int64
+    D = ctypes.c_double
+    lib.oracle_quantize.argtypes = [P, I, I, I, D, P, P, P, P, P]
+    lib.oracle_quantize.restype = None
+    lib.oracle_dequantize_f64.argtypes = [P, P, P, I, I, D, P]
+    lib.oracle_dequantize_bf16.argtypes = [P, P, P, I, I, D, P]
+    lib.oracle_linear.argtypes = [P, I, I, P, P, P, I, D, P, P]
+    lib.oracle_linear_pairs.argtypes = [P, I, I, P, P, P, I, D, I, P, P, P, P]
+    lib.oracle_snr_db.argtypes = [P, P, I]
+    lib.oracle_snr_db.restype = D
+    lib.oracle_uniform_int4.argtypes = [P, I, I, P]
+    lib.oracle_double_to_bf16.argtypes = [D]
+    lib.oracle_double_to_bf16.restype = ctypes.c_uint16
+    lib.oracle_rounding_mode_ok.restype = ctypes.c_int
+    return lib
+
+
+def _p(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"], "oracle arrays must be C-contiguous"
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _u16(a) -> np.ndarray:
+    """bf16 tensor / uint16 array -> contiguous uint16 bit patterns."""
+    try:
+        import torch
+        if isinstance(a, torch.Tensor):
+            assert a.dtype == torch.bfloat16
+            return np.ascontiguousarray(a.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16))
+    except ImportError:  # pragma: no cover
+        pass
+    a = np.ascontiguousarray(a)
+    assert a.dtype == np.uint16
+    return a
+
+
+class Oracle:
+    """The oracle's entry points bound to one compiled shared object."""
+
+    def __init__(self, so_path: str):
+        self._lib = _bind(so_path)
+        self.path = so_path
+
+    def quantize(self, w, alpha: float, want_ties: bool = False, want_v15: bool = False):
+        """OPQ-quantize bf16 W[N, K] row by row.
+
+        Returns dict(codes uint32[N, K/8], signs uint32[N, K/32], scales float32[N],
+        near_tie uint8[N, K] | None, v15 float64[N, K] | None).
+        """
+        w = _u16(w)
+        N, K = w.shape
+        assert K % 32 == 0
+        lib = self._lib
+        assert lib.oracle_rounding_mode_ok() == 1
+        codes = np.zeros((N, K // 8), np.uint32)
+        signs = np.zeros((N, K // 32), np.uint32)
+        scales = np.zeros((N,), np.float32)
+        ties = np.zeros((N, K), np.uint8) if want_ties else None
+        v15 = np.zeros((N, K), np.float64) if want_v15 else None
+        lib.oracle_quantize(_p(w), N, K, K, float(alpha), _p(codes), _p(signs), _p(scales),
+                            _p(ties) if ties is not None else None,
+                            _p(v15) if v15 is not None else None)
+        return dict(codes=codes, signs=signs, scales=scales, near_tie=ties, v15=v15)
+
+    def dequantize_f64(self, codes, signs, scales, alpha: float) -> np.ndarray:
+        codes = np.ascontiguousarray(codes, np.uint32)
+        signs = np.ascontiguousarray(signs, np.uint32)
+        scales = np.ascontiguousarray(scales, np.float32)
+        N, cw = codes.shape
+        K = cw * 8
+        out = np.zeros((N, K), np.float64)
+        self._lib.oracle_dequantize_f64(_p(codes), _p(signs), _p(scales), N, K, float(alpha), _p(out))
+        return out
+
+    def dequantize_bf16(self, codes, signs, scales, alpha: float) -> np.ndarray:
+        """Returns uint16 bf16 bit patterns [N, K]."""
+        codes = np.ascontiguousarray(codes, np.uint32)
+        signs = np.ascontiguousarray(signs, np.uint32)
+        scales = np.ascontiguousarray(scales, np.float32)
+        N, cw = codes.shape
+        K = cw * 8
+        out = np.zeros((N, K), np.uint16)
+        self._lib.oracle_dequantize_bf16(_p(codes), _p(signs), _p(scales), N, K, float(alpha), _p(out))
+        return out
+
+    def linear(self, x, codes, signs, scales, alpha: float):
+        """y = x @ W'^T in fp64 with its error bound B = |x| @ |W'|^T. Returns (y, B)."""
+        x = _u16(x)
+        M, K = x.shape
+        codes = np.ascontiguousarray(codes, np.uint32)
+        signs = np.ascontiguousarray(signs, np.uint32)
+        scales = np.ascontiguousarray(scales, np.float32)
+        N = codes.shape[0]
+        assert codes.shape[1] * 8 == K
+        y = np.zeros((M, N), np.float64)
+        b = np.zeros((M, N), np.float64)
+        self._lib.oracle_linear(_p(x), M, K, _p(codes), _p(signs), _p(scales), N, float(alpha), _p(y), _p(b))
+        return y, b
+
+    def linear_pairs(self, x, codes, signs, scales, alpha: float, ms, ns):
+        """y[m_i, n_i] and B[m_i, n_i] for the listed output positions."""
+        x = _u16(x)
+        M, K = x.shape
+        codes = np.ascontiguousarray(codes, np.uint32)
+        signs = np.ascontiguousarray(signs, np.uint32)
+        scales = np.ascontiguousarray(scales, np.float32)
+        N = codes.shape[0]
+        ms = np.ascontiguousarray(ms, np.int64)
+        ns = np.ascontiguousarray(ns, np.int64)
+        assert ms.shape == ns.shape
+        assert (ms >= 0).all() and (ms < M).all() and (ns >= 0).all() and (ns < N).all()
+        y = np.zeros(ms.shape, np.float64)
+        b = np.zeros(ms.shape, np.float64)
+        self._lib.oracle_linear_pairs(_p(x), M, K, _p(codes), _p(signs), _p(scales), N, float(alpha),
+                                    ms.size, _p(ms), _p(ns), _p(y), _p(b))
+        return y, b
+
+    def snr_db(self, w, w_rec: np.ndarray) -> float:
+        w = _u16(w)
+        w_rec = np.ascontiguousarray(w_rec, np.float64)
+        assert w.size == w_rec.size
+        return float(self._lib.oracle_snr_db(_p(w), _p(w_rec), w.size))
+
+    def uniform_int4(self, w) -> np.ndarray:
+        w = _u16(w)
+        N, K = w.shape
+        out = np.zeros((N, K), np.float64)
+        self._lib.oracle_uniform_int4(_p(w), N, K, _p(out))
+        return out
+
+    def double_to_bf16(self, v: float) -> int:
+        return int(self._lib.oracle_double_to_bf16(float(v)))
+
+
+_default = None
+
+
+def default() -> Oracle:
+    """The oracle built from ``opq_oracle.c`` (compiled on first use)."""
+    global _default
+    with _lock:
+        if _default is None:
+            _default = Oracle(build())
+    return _default
+
+
+def quantize(*a, **k):
+    return default().quantize(*a, **k)
+
+
+def dequantize_f64(*a, **k):
+    return default().dequantize_f64(*a, **k)
+
+
+def dequantize_bf16(*a, **k):
+    return default().dequantize_bf16(*a, **k)
+
+
+def linear(*a, **k):
+    return default().linear(*a, **k)
+
+
+def linear_pairs(*a, **k):
+    return default().linear_pairs(*a, **k)
+
+
+def snr_db(*a, **k):
+    return default().snr_db(*a, **k)
+
+
+def uniform_int4(*a, **k):
+    return default().uniform_int4(*a, **k)
+
+
+def double_to_bf16(*a, **k):
+    return default().double_to_bf16(*a, **k)
+
+
+def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    """Exact value of bf16 bit patterns (a plain reinterpretation, no arithmetic)."""
+    bits = np.ascontiguousarray(bits, np.uint16)
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)

@@ -1,0 +1,294 @@
+"""Pins that tie the fp64 OPQ oracle to facts fixed outside the oracle itself.
+
+Each ``pin_*`` takes an ``oracle.Oracle`` and raises AssertionError when the
+oracle disagrees with a closed form, an exact-rational evaluation, a
+hand-derived fixture (``tests/golden``), a brute-force search in extended
+precision, or an invariant of the method ("OPQ INT4 Z-Image" model card,
+"OPQ principle": u = |w|/max|w|, v = u^alpha, q = round(15 v),
+w' = sign(w) (q/15)^(1/alpha) max|w|). The mutation test plants mistakes in
+copies of the oracle source and checks that some pin catches each of them.
+"""
+from __future__ import annotations
+
+import os
+from decimal import Decimal, getcontext
+from fractions import Fraction
+
+import numpy as np
+import torch
+
+import workloads
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+# ----------------------------------------------------------------- helpers --
+def bf16_bits(values) -> np.ndarray:
+    """Exact bf16 bit patterns of values that are representable in bf16."""
+    t = torch.tensor(list(values), dtype=torch.float64)
+    b = t.to(torch.float32).to(torch.bfloat16)
+    assert torch.equal(b.to(torch.float64), t), "fixture value not exact in bf16"
+    return b.view(torch.int16).numpy().view(np.uint16).copy()
+
+
+def bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    return (np.asarray(bits, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def unpack_codes(codes: np.ndarray) -> np.ndarray:
+    """uint32 [N, K/8] -> uint8 [N, K] with element 8j+i = nibble i of word j."""
+    N, cw = codes.shape
+    shifts = (4 * np.arange(8, dtype=np.uint32))[None, None, :]
+    return ((codes[:, :, None] >> shifts) & 0xF).reshape(N, cw * 8).astype(np.uint8)
+
+
+def unpack_signs(signs: np.ndarray) -> np.ndarray:
+    N, sw = signs.shape
+    shifts = np.arange(32, dtype=np.uint32)[None, None, :]
+    return ((signs[:, :, None] >> shifts) & 1).reshape(N, sw * 32).astype(np.uint8)
+
+
+def read_golden(name: str):
+    """Blocks of 'key values...' lines; '#' comments; 'block X' starts a block."""
+    blocks, cur = [], {}
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.split("#", 1)[0].strip()
+            if not line:
+                continue
+            key, *vals = line.split()
+            if key == "block":
+                if cur:
+                    blocks.append(cur)
+                cur = {}
+                continue
+            cur[key] = vals
+    if cur:
+        blocks.append(cur)
+    return blocks
+
+
+def tiny_weights() -> np.ndarray:
+    w = workloads.tiny().make_weights("cpu")
+    return w.view(torch.int16).numpy().view(np.uint16).copy()
+
+
+# -------------------------------------------------------------------- pins --
+def pin_golden_fixtures(orc):
+    """Hand-derived rows: exact .5 ties at alpha = 1, bit layout, zero and duplicate-max rows."""
+    for fname in ("alpha1_ties_row.txt", "special_rows.txt"):
+        for blk in read_golden(fname):
+            alpha = float(blk["alpha"][0])
+            w = bf16_bits(float(v) for v in blk["w"])[None, :]
+            r = orc.quantize(w, alpha)
+            want_codes = np.array([int(v, 16) for v in blk["codes"]], np.uint32)
+            want_signs = np.array([int(v, 16) for v in blk["signs"]], np.uint32)
+            assert r["scales"][0] == np.float32(float(blk["scale"][0])), (fname, r["scales"])
+            assert np.array_equal(r["codes"][0], want_codes), (fname, [hex(c) for c in r["codes"][0]])
+            assert np.array_equal(r["signs"][0], want_signs), (fname, [hex(c) for c in r["signs"][0]])
+            if "dequant" in blk:
+                want = bf16_bits(float(v) for v in blk["dequant"])
+                got = orc.dequantize_bf16(r["codes"], r["signs"], r["scales"], alpha)[0]
+                assert np.array_equal(got, want), (fname, got, want)
+
+
+def pin_alpha1_exact_rational(orc):
+    """alpha = 1 reduces to round-half-even(15 |w| / max) in exact rational arithmetic."""
+    w = tiny_weights()[:64]
+    r = orc.quantize(w, 1.0)
+    q = unpack_codes(r["codes"])
+    s = unpack_signs(r["signs"])
+    vals = bits_to_f64(w)
+    for n in range(w.shape[0]):
+        row = [Fraction(float(v)) for v in vals[n]]
+        mx = max(abs(v) for v in row)
+        assert Fraction(float(r["scales"][n])) == mx
+        for k, v in enumerate(row):
+            want = round(15 * abs(v) / mx) if mx != 0 else 0   # Fraction round(): half to even
+            assert q[n, k] == want, (n, k, q[n, k], want)
+            assert s[n, k] == (1 if v < 0 else 0)
+    # dequantize at alpha = 1 is q/15 * max: check against exact rationals rounded once
+    deq = orc.dequantize_f64(r["codes"], r["signs"], r["scales"], 1.0)
+    for n in range(8):
+        mx = Fraction(float(r["scales"][n]))
+        for k in range(w.shape[1]):
+            exact = Fraction(int(q[n, k]), 15) * mx * (-1 if s[n, k] else 1)
+            assert abs(Fraction(deq[n, k]) - exact) <= abs(exact) * Fraction(1, 2 ** 51)
+
+
+def pin_max_zero_monotone(orc):
+    """max element -> q = 15 and w' = +-max bit-exactly; zero -> 0; codes monotone in |w|."""
+    w = tiny_weights()
+    w = w.copy()
+    w[3, :] = 0                       # an all-zero row
+    w[5, 7] = 0x8000                  # a negative zero
+    for alpha in (0.45, 0.73, 1.0):
+        r = orc.quantize(w, alpha)
+        q = unpack_codes(r["codes"])
+        mag = w & 0x7FFF
+        mx = mag.max(axis=1)
+        at_max = mag == mx[:, None]
+        nz = mx > 0
+        assert (q[at_max & nz[:, None]] == 15).all()
+        assert (q[mag == 0] == 0).all()
+        assert (q[~nz] == 0).all() and (r["scales"][~nz] == 0).all()
+        deq = orc.dequantize_bf16(r["codes"], r["signs"], r["scales"], alpha)
+        sel = at_max & nz[:, None]
+        assert np.array_equal(deq[sel], w[sel]), "max element must reconstruct exactly"
+        assert ((deq[mag == 0] & 0x7FFF) == 0).all()
+        for n in range(w.shape[0]):
+            order = np.argsort(mag[n], kind="stable")
+            assert (np.diff(q[n, order].astype(np.int32)) >= 0).all(), "codes not monotone in |w|"
+
+
+def _longdouble_levels(w: np.ndarray, alpha: float):
+    """15 (|w|/max)^alpha in extended precision (x87 long double)."""
+    a = np.abs(bits_to_f64(w)).astype(np.longdouble)
+    mx = a.max(axis=1, keepdims=True)
+    u = np.where(mx > 0, a / np.where(mx > 0, mx, 1), 0)
+    return np.longdouble(15) * np.power(u, np.longdouble(alpha))
+
+
+def pin_bruteforce_nearest_level(orc):
+    """Every entry of the tiny weights: q = argmin_k |15 u^alpha - k| (extended precision, ties even)."""
+    w = tiny_weights()
+    for alpha in (0.45, 0.73, 1.0):
+        v = _longdouble_levels(w, alpha)
+        ks = np.arange(16, dtype=np.longdouble)
+        d = np.abs(v[..., None] - ks)
+        best = np.argmin(d, axis=-1)
+        # a tie between k and k+1 resolves to the even one
+        dmin = np.take_along_axis(d, best[..., None], -1)[..., 0]
+        nxt = np.minimum(best + 1, 15)
+        tie = np.take_along_axis(d, nxt[..., None], -1)[..., 0] == dmin
+        best = np.where(tie & (best % 2 == 1), nxt, best)
+        frac = v - np.floor(v)
+        near = np.abs(frac - np.longdouble(0.5)) <= np.longdouble(1e-6)
+        r = orc.quantize(w, alpha, want_ties=True)
+        q = unpack_codes(r["codes"])
+        bad = (q != best) & ~near
+        assert not bad.any(), (alpha, int(bad.sum()))
+        # the oracle's own near-tie flag marks the same entries
+        assert np.array_equal(r["near_tie"].astype(bool), near), alpha
+
+
+def pin_threshold_identity(orc):
+    """q >= k  <=>  u >= ((k - 1/2)/15)^(1/alpha), checked in 50-digit decimal arithmetic."""
+    getcontext().prec = 50
+    w = tiny_weights()[:16]
+    vals = bits_to_f64(w)
+    for alpha in (0.45, 0.73):
+        r = orc.quantize(w, alpha)
+        q = unpack_codes(r["codes"])
+        inv = Decimal(1) / Decimal(repr(alpha))
+        t = [Decimal(0)] + [((Decimal(2 * k - 1) / Decimal(30)) ** inv) for k in range(1, 16)]
+        for n in range(w.shape[0]):
+            mx = Decimal(abs(vals[n]).max())
+            for kk in range(w.shape[1]):
+                u = Decimal(abs(vals[n, kk])) / mx
+                want = sum(1 for k in range(1, 16) if u >= t[k])
+                assert q[n, kk] == want, (alpha, n, kk, q[n, kk], want)
+
+
+def pin_lut_decimal(orc):
+    """Dequantized magnitudes (q/15)^(1/alpha) * max against 50-digit decimal values."""
+    getcontext().prec = 50
+    for alpha in (0.45, 0.73, 1.0):
+        codes = np.array([[0x76543210, 0xFEDCBA98]], np.uint32)      # q = 0..15
+        signs = np.array([[0x0000AAAA]], np.uint32)                  # odd elements negative
+        codes = np.concatenate([codes, codes], axis=1)
+        scales = np.array([1.0], np.float32)
+        got = orc.dequantize_f64(codes, signs, scales, alpha)[0]
+        inv = Decimal(1) / Decimal(repr(alpha))
+        for k in range(32):
+            q = k % 16
+            mag = (Decimal(q) / Decimal(15)) ** inv if q else Decimal(0)
+            want = -mag if (k < 16 and k % 2 == 1) else mag
+            assert abs(Decimal(got[k]) - want) <= Decimal(2) ** -50, (alpha, k, got[k], want)
+
+
+def pin_roundtrip_idempotent(orc):
+    """quantize(bf16(dequantize(codes))) returns the codes (and signs where q > 0)."""
+    w = tiny_weights()
+    for alpha in (0.45, 0.73, 1.0):
+        r = orc.quantize(w, alpha)
+        deq = orc.dequantize_bf16(r["codes"], r["signs"], r["scales"], alpha)
+        r2 = orc.quantize(deq, alpha)
+        assert np.array_equal(r2["scales"], r["scales"])
+        assert np.array_equal(r2["codes"], r["codes"]), alpha
+        q = unpack_codes(r["codes"])
+        s1, s2 = unpack_signs(r["signs"]), unpack_signs(r2["signs"])
+        assert np.array_equal(s1[q > 0], s2[q > 0])
+
+
+def pin_linear(orc):
+    """y = x W'^T: one-hot rows of x return rows of W'; a BLAS matmul of W' agrees."""
+    x, w = workloads.tiny().make("cpu")
+    M, K = x.shape
+    r = orc.quantize(w, 0.73)
+    wq = orc.dequantize_f64(r["codes"], r["signs"], r["scales"], 0.73)
+    # one-hot activations: 1.0 at column (7 * m) % K
+    onehot = np.zeros((M, K), np.uint16)
+    cols = (7 * np.arange(M)) % K
+    onehot[np.arange(M), cols] = 0x3F80
+    y, b = orc.linear(onehot, r["codes"], r["signs"], r["scales"], 0.73)
+    assert np.array_equal(y, wq[:, cols].T)
+    assert np.array_equal(b, np.abs(wq[:, cols].T))
+    xv = bits_to_f64(x.view(torch.int16).numpy().view(np.uint16))
+    y, b = orc.linear(x, r["codes"], r["signs"], r["scales"], 0.73)
+    ref = xv @ wq.T
+    assert np.abs(y - ref).max() <= 1e-12 * b.max()
+    assert np.allclose(b, np.abs(xv) @ np.abs(wq).T, rtol=1e-12, atol=0)
+    # sampled positions agree with the full product
+    ms = np.array([0, 5, 63, 17]); ns = np.array([0, 255, 100, 3])
+    yp, bp = orc.linear_pairs(x, r["codes"], r["signs"], r["scales"], 0.73, ms, ns)
+    assert np.array_equal(yp, y[ms, ns]) and np.array_equal(bp, b[ms, ns])
+
+
+def pin_bf16_rounding(orc):
+    """double -> bf16 round-to-nearest-even against exact rational rounding."""
+    rng = np.random.default_rng(7)
+    vals = list(rng.standard_normal(2000) * 10.0 ** rng.integers(-30, 30, 2000))
+    # exact ties between neighbours 1 + 2^-7 k, and just off them
+    vals += [1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, -(1.0 + 2.0 ** -8), 1.0 + 2.0 ** -8 + 2.0 ** -40,
+             3.0e38, 3.4e38, 1e-40, 2.0 ** -133, 2.0 ** -134, 3 * 2.0 ** -135, 0.0, -0.0]
+    for v in vals:
+        got = orc.double_to_bf16(v)
+        # reference: nearest bf16 by exhaustive neighbour search on exact rationals
+        f32 = np.float32(v) if abs(v) < 3.4e38 else np.float32(np.sign(v) * 3.4e38)
+        base = int(np.array([f32], np.float32).view(np.uint32)[0] >> 16)
+        cands = [(base + d) & 0xFFFF for d in (-2, -1, 0, 1, 2)]
+        best = None
+        for c in cands:
+            if (c & 0x7FFF) >= 0x7F80:
+                continue
+            cv = float(bits_to_f64(np.array([c], np.uint16))[0])
+            err = abs(Fraction(cv) - Fraction(v))
+            key = (err, (c & 1))  # ties: even mantissa wins
+            if best is None or key < best[0]:
+                best = (key, c)
+        want = best[1]
+        if abs(v) >= (2.0 - 2.0 ** -8) * 2.0 ** 127:   # at or past max + half an ulp: overflow
+            want = 0xFF80 if v < 0 else 0x7F80
+        if v == 0.0:
+            want = 0x8000 if np.signbit(v) else 0
+        assert got == want, (v, hex(got), hex(want))
+
+
+def pin_snr_ordering(orc):
+    """The method's claim, as an inequality: OPQ(alpha<1) beats alpha = 1 and uniform INT4
+    on heavy-tailed weights (a Student-t(4) 512 x 3840 block)."""
+    lin = workloads.Linear("snr", 1, 512, 3840, w_seed=11)
+    w = lin.make_weights("cpu").view(torch.int16).numpy().view(np.uint16).copy()
+    snr = {}
+    for alpha in (0.45, 0.73, 1.0):
+        r = orc.quantize(w, alpha)
+        snr[alpha] = orc.snr_db(w, orc.dequantize_f64(r["codes"], r["signs"], r["scales"], alpha))
+    snr["int4"] = orc.snr_db(w, orc.uniform_int4(w))
+    assert snr[0.73] > snr[1.0] + 2.0, snr
+    assert snr[1.0] > snr["int4"] + 2.0, snr
+
+
+PINS = [pin_golden_fixtures, pin_alpha1_exact_rational, pin_max_zero_monotone,
+        pin_bruteforce_nearest_level, pin_threshold_identity, pin_lut_decimal,
+        pin_roundtrip_idempotent, pin_linear, pin_bf16_rounding, pin_snr_ordering]
