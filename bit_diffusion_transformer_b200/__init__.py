@@ -1,0 +1,151 @@
+"""Python binding of libopq.so: OPQ (Optimal Power Quantization) weights and the
+linear layer that consumes them, on B200 (sm_100a).
+
+The binding only marshals arguments: torch tensors provide device memory and the
+current CUDA stream; every step runs in the library's kernels. There is no CPU
+or PyTorch fallback: if ``libopq.so`` is missing or a tensor is not on a CUDA
+device, the call raises.
+
+Packed weight of W[N, K] (K % 32 == 0):
+  codes  int32 [N, K/8]   element (n, 8j+i) is bits 4i..4i+3 of word j (4-bit magnitude)
+  signs  int32 [N, K/32]  element (n, 32j+i) is bit i of word j (1 = negative)
+  scales float32 [N]      max |w| of row n
+(int32 tensors carry the uint32 words bit for bit.)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libopq.so")
+ALPHA = 0.73
+
+_STATUS = {0: "OPQ_OK", 1: "OPQ_ERR_INVALID_ARG", 2: "OPQ_ERR_UNSUPPORTED_SHAPE", 3: "OPQ_ERR_MISALIGNED",
+           4: "OPQ_ERR_WORKSPACE", 5: "OPQ_ERR_CUDA", 6: "OPQ_ERR_NOT_DEVICE_MEMORY"}
+
+EXPORTS = ["opq_quantize", "opq_dequantize", "opq_linear_workspace_size", "opq_linear", "opq_linear_plan",
+           "opq_device_error", "opq_status_string", "opq_last_cuda_error", "opq_abi_version"]
+
+
+class OPQError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {_STATUS.get(status, status)}")
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH):
+    """Load libopq.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"libopq.so not found at {path}; build it with "
+                          f"`python -m bit_diffusion_transformer_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, I, F, S = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+    lib.opq_quantize.argtypes = [P, I, I, I, F, P, P, P, P]
+    lib.opq_dequantize.argtypes = [P, P, P, I, I, F, P, P]
+    lib.opq_linear_workspace_size.argtypes = [I, I, I, ctypes.POINTER(S)]
+    lib.opq_linear.argtypes = [P, I, I, P, P, P, I, F, P, P, S, P]
+    lib.opq_linear_plan.argtypes = [I, I, I, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int),
+                                    ctypes.POINTER(ctypes.c_int)]
+    lib.opq_device_error.argtypes = [P, ctypes.POINTER(ctypes.c_uint32)]
+    lib.opq_status_string.argtypes = [ctypes.c_int]
+    lib.opq_status_string.restype = ctypes.c_char_p
+    for f in ("opq_quantize", "opq_dequantize", "opq_linear_workspace_size", "opq_linear", "opq_linear_plan",
+              "opq_device_error"):
+        getattr(lib, f).restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise OPQError(status, where)
+
+
+def _ptr(t: torch.Tensor):
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError("opq: tensors must be on a CUDA device")
+        if not t.is_contiguous():
+            raise ValueError("opq: tensors must be contiguous")
+
+
+def quantize(w: torch.Tensor, alpha: float = ALPHA, out=None):
+    """OPQ-quantize bf16 W[N, K] -> (codes, signs, scales)."""
+    assert w.dtype == torch.bfloat16 and w.dim() == 2
+    _need_cuda(w)
+    N, K = w.shape
+    if out is None:
+        codes = torch.empty((N, K // 8), dtype=torch.int32, device=w.device)
+        signs = torch.empty((N, K // 32), dtype=torch.int32, device=w.device)
+        scales = torch.empty((N,), dtype=torch.float32, device=w.device)
+    else:
+        codes, signs, scales = out
+    _check(load().opq_quantize(_ptr(w), N, K, K, float(alpha), _ptr(codes), _ptr(signs), _ptr(scales),
+                               _stream(w.device)), "opq_quantize")
+    return codes, signs, scales
+
+
+def dequantize(codes: torch.Tensor, signs: torch.Tensor, scales: torch.Tensor, alpha: float = ALPHA, out=None):
+    """Packed planes -> bf16 W'[N, K]."""
+    _need_cuda(codes, signs, scales)
+    N, cw = codes.shape
+    K = cw * 8
+    w = out if out is not None else torch.empty((N, K), dtype=torch.bfloat16, device=codes.device)
+    _check(load().opq_dequantize(_ptr(codes), _ptr(signs), _ptr(scales), N, K, float(alpha), _ptr(w),
+                                 _stream(codes.device)), "opq_dequantize")
+    return w
+
+
+def workspace_size(M: int, N: int, K: int) -> int:
+    b = ctypes.c_size_t(0)
+    _check(load().opq_linear_workspace_size(M, N, K, ctypes.byref(b)), "opq_linear_workspace_size")
+    return int(b.value)
+
+
+def plan(M: int, N: int, K: int):
+    """(path, splits, launches) that opq_linear uses for this shape."""
+    p, s, l = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
+    _check(load().opq_linear_plan(M, N, K, ctypes.byref(p), ctypes.byref(s), ctypes.byref(l)), "opq_linear_plan")
+    return p.value, s.value, l.value
+
+
+def linear(x: torch.Tensor, codes: torch.Tensor, signs: torch.Tensor, scales: torch.Tensor,
+           alpha: float = ALPHA, out=None, workspace=None):
+    """y = x @ W'^T for bf16 x[M, K] and a packed W[N, K] -> bf16 y[M, N]."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2
+    _need_cuda(x, codes, signs, scales)
+    M, K = x.shape
+    N = codes.shape[0]
+    y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    need = workspace_size(M, N, K)
+    if need and workspace is None:
+        workspace = torch.empty((need,), dtype=torch.uint8, device=x.device)
+    ws_ptr = _ptr(workspace) if workspace is not None else ctypes.c_void_p(0)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(load().opq_linear(_ptr(x), M, K, _ptr(codes), _ptr(signs), _ptr(scales), N, float(alpha), _ptr(y),
+                             ws_ptr, ws_bytes, _stream(x.device)), "opq_linear")
+    return y
+
+
+def device_error(device=None) -> int:
+    """Read and clear the library's device-side error word (synchronises the current stream)."""
+    v = ctypes.c_uint32(0)
+    _check(load().opq_device_error(_stream(device), ctypes.byref(v)), "opq_device_error")
+    return int(v.value)

@@ -1,0 +1,129 @@
+// opq_bits.h — register-level bit tricks shared by the OPQ kernels.
+//
+// Everything here is __host__ __device__ so that a host-side harness can check
+// it exhaustively without a GPU; on the device PRMT is the hardware byte
+// permute (inline PTX, generic mode with sign replication).
+//
+// Packed format ("OPQ INT4 Z-Image" model card, "Technical details / storage
+// format": 8 magnitudes per uint32, 32 signs per uint32): element 8j+i of a row
+// is nibble i of code word j; element 32j+i is bit i of sign word j.
+#pragma once
+#include <stdint.h>
+
+#if defined(__CUDACC__)
+#define OPQ_HD __host__ __device__ __forceinline__
+#else
+#define OPQ_HD static inline
+#endif
+
+namespace opqbits {
+
+// PRMT, generic mode: output byte i = source byte (sel_i & 7) of {b:a}, or, when
+// sel_i & 8, that byte's top bit replicated over 8 bits. Only sel[15:0] is used.
+OPQ_HD uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+#if defined(__CUDA_ARCH__)
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+    return r;
+#else
+    uint64_t src = ((uint64_t)b << 32) | a;
+    uint32_t r = 0;
+    for (int i = 0; i < 4; ++i) {
+        uint32_t s = (sel >> (4 * i)) & 0xFu;
+        uint32_t byte = (uint32_t)(src >> (8 * (s & 7u))) & 0xFFu;
+        if (s & 8u) byte = (byte & 0x80u) ? 0xFFu : 0x00u;
+        r |= byte << (8 * i);
+    }
+    return r;
+#endif
+}
+
+// ---------------------------------------------------------------------------
+// Quantize: 15 per-row thresholds as bf16 bit patterns, T[1..15] non-decreasing,
+// T[k] = smallest bf16 magnitude m with round-half-even(15 (m/max)^alpha) >= k.
+// P[k] = T[k] * 0x00010001 (the threshold in both 16-bit halves).
+//
+// quant_pair: codes of the two bf16 weights in w2 (low half, high half) by a
+// 4-level binary search done on both halves at once. For a 16-bit half holding
+// 0x8000 | |w| and a threshold t <= 0x8000, the 32-bit subtraction never borrows
+// across halves and bit 15 (bit 31) of the difference is |w| >= t. PRMT turns
+// those bits into 0x0000FFFF / 0xFFFF0000 masks that select the next level's
+// thresholds. Returns q_lo in bits 0..3 and q_hi in bits 16..19.
+// ---------------------------------------------------------------------------
+OPQ_HD uint32_t sel_mask(uint32_t m, uint32_t a, uint32_t b) { return (a & m) | (b & ~m); }
+
+OPQ_HD uint32_t quant_pair(uint32_t w2, const uint32_t (&P)[16]) {
+    const uint32_t M2 = w2 | 0x80008000u;
+    const uint32_t k3 = prmt(M2 - P[8], 0, 0xBB99u);                 // q >= 8
+    const uint32_t t2 = sel_mask(k3, P[12], P[4]);
+    const uint32_t k2 = prmt(M2 - t2, 0, 0xBB99u);                   // q >= 4 + 8c3
+    const uint32_t hi2 = sel_mask(k2, P[14], P[10]);
+    const uint32_t lo2 = sel_mask(k2, P[6], P[2]);
+    const uint32_t t1 = sel_mask(k3, hi2, lo2);
+    const uint32_t k1 = prmt(M2 - t1, 0, 0xBB99u);                   // next level
+    const uint32_t a0 = sel_mask(k1, P[3], P[1]);
+    const uint32_t a1 = sel_mask(k1, P[7], P[5]);
+    const uint32_t a2 = sel_mask(k1, P[11], P[9]);
+    const uint32_t a3 = sel_mask(k1, P[15], P[13]);
+    const uint32_t b0 = sel_mask(k2, a1, a0);
+    const uint32_t b1 = sel_mask(k2, a3, a2);
+    const uint32_t t0 = sel_mask(k3, b1, b0);
+    const uint32_t k0 = prmt(M2 - t0, 0, 0xBB99u);
+    return (k3 & 0x00080008u) | (k2 & 0x00040004u) | (k1 & 0x00020002u) | (k0 & 0x00010001u);
+}
+
+// 8 weights (4 bf16 pairs, elements 0..7) -> one code word, element i in nibble i.
+OPQ_HD uint32_t pack_codes(uint32_t q0, uint32_t q1, uint32_t q2, uint32_t q3) {
+    // q_p holds element 2p in bits 0..3 and element 2p+1 in bits 16..19
+    const uint32_t t0 = q0 | (q0 >> 12), t1 = q1 | (q1 >> 12);
+    const uint32_t t2 = q2 | (q2 >> 12), t3 = q3 | (q3 >> 12);
+    return prmt(prmt(t0, t1, 0x0040u), prmt(t2, t3, 0x0040u), 0x5410u);
+}
+
+// Sign bits (bf16 sign bit set) of 8 weights held as 4 bf16 pairs -> bits 0..7.
+OPQ_HD uint32_t sign_byte(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3) {
+    // gather the high byte of every bf16 (its top bit is the sign), then move the
+    // four top bits to bits 28..31 with one multiply (no carries: the products
+    // of distinct bits land on distinct positions)
+    const uint32_t a = prmt(w0, w1, 0x7531u) & 0x80808080u;   // elements 0..3
+    const uint32_t b = prmt(w2, w3, 0x7531u) & 0x80808080u;   // elements 4..7
+    return ((a * 0x00204081u) >> 28) | (((b * 0x00204081u) >> 28) << 4);
+}
+
+// ---------------------------------------------------------------------------
+// Decode: one code word (8 nibbles) and its 8 sign bits -> 8 bf16 values
+// sign * LUT[q], as 4 packed pairs (element 2p in the low half of out[p]).
+// The 16-entry bf16 table travels as byte planes: L[j] holds the low bytes of
+// entries 4j..4j+3, H[j] their high bytes (every H byte has its top bit clear:
+// the table is non-negative).
+// ---------------------------------------------------------------------------
+struct DecodeTable {
+    uint32_t L[4];
+    uint32_t H[4];
+};
+
+OPQ_HD void decode8(uint32_t c, uint32_t sb, const DecodeTable &T, uint32_t out[4]) {
+    const uint32_t s = c & 0x77777777u;        // low 3 bits of every nibble
+    const uint32_t c4 = c << 4;
+    // nibbles 0..3
+    {
+        const uint32_t m = prmt(c, c4, 0x9D8Cu);   // 0xFF in byte i iff bit 3 of nibble i
+        const uint32_t l = sel_mask(m, prmt(T.L[2], T.L[3], s), prmt(T.L[0], T.L[1], s));
+        const uint32_t sg = ((sb & 0xFu) * 0x10204080u) & 0x80808080u;   // sign i -> bit 8i+7
+        const uint32_t h = sel_mask(m, prmt(T.H[2], T.H[3], s), prmt(T.H[0], T.H[1], s)) | sg;
+        out[0] = prmt(l, h, 0x5140u);
+        out[1] = prmt(l, h, 0x7362u);
+    }
+    // nibbles 4..7
+    {
+        const uint32_t sh = s >> 16;
+        const uint32_t m = prmt(c, c4, 0xBFAEu);
+        const uint32_t l = sel_mask(m, prmt(T.L[2], T.L[3], sh), prmt(T.L[0], T.L[1], sh));
+        const uint32_t sg = (((sb >> 4) & 0xFu) * 0x10204080u) & 0x80808080u;
+        const uint32_t h = sel_mask(m, prmt(T.H[2], T.H[3], sh), prmt(T.H[0], T.H[1], sh)) | sg;
+        out[2] = prmt(l, h, 0x5140u);
+        out[3] = prmt(l, h, 0x7362u);
+    }
+}
+
+}  // namespace opqbits

@@ -1,0 +1,384 @@
+// opq_capi.cu — the C ABI of libopq.so (declared in include/opq.h): argument
+// validation, the alpha-dependent tables, TMA descriptors, kernel selection and
+// launches. The whole library is this one translation unit.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <initializer_list>
+#include <mutex>
+
+#include "opq.h"
+#include "opq_dequantize.cuh"
+#include "opq_linear.cuh"
+#include "opq_quantize.cuh"
+
+namespace {
+
+thread_local int t_last_cuda_error = 0;
+
+constexpr int kPlanSMs = 148;   // B200 SM count; the split-K plan is fixed by shape alone
+
+opq_status cuda_fail(cudaError_t e) {
+    t_last_cuda_error = (int)e;
+    return OPQ_ERR_CUDA;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Tensor pointers: all non-null and 16-byte aligned first, then each must be
+// device-accessible memory (device or managed), so that the cheapest argument
+// error is reported regardless of pointer order.
+opq_status check_ptrs(std::initializer_list<const void *> ptrs) {
+    for (const void *p : ptrs)
+        if (p == nullptr) return OPQ_ERR_INVALID_ARG;
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return OPQ_ERR_MISALIGNED;
+    for (const void *p : ptrs) {
+        cudaPointerAttributes attr;
+        cudaError_t e = cudaPointerGetAttributes(&attr, p);
+        if (e != cudaSuccess) {
+            (void)cudaGetLastError();
+            return OPQ_ERR_NOT_DEVICE_MEMORY;
+        }
+        if (attr.type != cudaMemoryTypeDevice && attr.type != cudaMemoryTypeManaged) return OPQ_ERR_NOT_DEVICE_MEMORY;
+    }
+    return OPQ_OK;
+}
+
+bool alpha_ok(float alpha) { return std::isfinite(alpha) && alpha > 0.0f; }
+
+// fp64 -> bf16 bits, round to nearest even, for the small decode table (host).
+// The value is first truncated to fp32 with a sticky last bit when inexact
+// (round to odd), then rounded to bf16 on the bit pattern.
+uint16_t host_bf16(double v) {
+    float t = (float)v;
+    if (std::fabs((double)t) > std::fabs(v)) t = std::nextafter(t, 0.0f);   // truncate toward zero
+    uint32_t b;
+    std::memcpy(&b, &t, 4);
+    if ((double)t != v) b |= 1u;
+    return (uint16_t)((b + 0x7FFFu + ((b >> 16) & 1u)) >> 16);
+}
+
+struct DeviceInfo {
+    int sms = 0;
+    bool tile_attr = false;
+    bool stream_attr[17] = {false};
+};
+std::mutex g_mu;
+DeviceInfo g_dev[64];
+
+opq_status device_info(DeviceInfo **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (dev < 0 || dev >= 64) return OPQ_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceInfo &d = g_dev[dev];
+    if (d.sms == 0) {
+        e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    *out = &d;
+    return OPQ_OK;
+}
+
+// --------------------------------------------------------------- TMA maps --
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+        else
+            (void)cudaGetLastError();
+    });
+    return fn;
+}
+
+// bf16 [rows, K] row-major, box {64 columns, box_rows}, 128-byte swizzle, zero fill out of bounds.
+opq_status make_x_map(CUtensorMap *map, const void *x, int64_t rows, int64_t K, uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return OPQ_ERR_CUDA;
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    cuuint32_t box[2] = {64u, box_rows};
+    cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(x), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        t_last_cuda_error = (int)r;
+        return OPQ_ERR_CUDA;
+    }
+    return OPQ_OK;
+}
+
+opqbits::DecodeTable decode_table(float alpha) {
+    opqbits::DecodeTable t;
+    const double inv = 1.0 / (double)alpha;
+    uint16_t lut[16];
+    for (int q = 0; q < 16; ++q) lut[q] = host_bf16(std::pow((double)q / 15.0, inv));
+    for (int j = 0; j < 4; ++j) {
+        t.L[j] = 0;
+        t.H[j] = 0;
+        for (int b = 0; b < 4; ++b) {
+            t.L[j] |= (uint32_t)(lut[4 * j + b] & 0xFFu) << (8 * b);
+            t.H[j] |= (uint32_t)(lut[4 * j + b] >> 8) << (8 * b);
+        }
+    }
+    return t;
+}
+
+struct Plan {
+    int path;      // 0 tile, 1 weight streaming
+    int splits;
+    int bx;
+    size_t ws_bytes;
+    int launches;
+};
+
+Plan make_plan(int64_t M, int64_t N, int64_t K) {
+    Plan p{};
+    if (M <= 256) {
+        p.path = 1;
+        p.bx = (int)((M + 15) / 16 * 16);
+        const int64_t tiles = (N + opqk::stream::BW - 1) / opqk::stream::BW;
+        const int64_t nkb = (K + opqk::stream::BK - 1) / opqk::stream::BK;
+        int64_t s = (2 * kPlanSMs + tiles - 1) / tiles;        // about two CTAs per SM
+        const int64_t max_s = nkb / 4 > 1 ? nkb / 4 : 1;       // keep >= 4 k-blocks per slice
+        if (s > max_s) s = max_s;
+        if (s > 16) s = 16;
+        if (s < 1) s = 1;
+        const int64_t per = (nkb + s - 1) / s;
+        s = (nkb + per - 1) / per;                             // no empty slice
+        p.splits = (int)s;
+        p.ws_bytes = s > 1 ? (size_t)s * (size_t)M * (size_t)N * sizeof(float) : 0;
+        p.launches = s > 1 ? 2 : 1;
+    } else {
+        p.path = 0;
+        p.splits = 1;
+        p.bx = 0;
+        p.ws_bytes = 0;
+        p.launches = 1;
+    }
+    return p;
+}
+
+opq_status check_sizes(int64_t N, int64_t K) {
+    if (N < 1 || K < 1) return OPQ_ERR_INVALID_ARG;
+    if (K % 32 != 0) return OPQ_ERR_UNSUPPORTED_SHAPE;
+    if (N > INT32_MAX || K > INT32_MAX) return OPQ_ERR_UNSUPPORTED_SHAPE;
+    return OPQ_OK;
+}
+
+template <int G, int V>
+void launch_quant(const uint16_t *w, int64_t N, int64_t K, int64_t ldw, const opqk::QuantParams &qp,
+                  uint32_t *codes, uint32_t *signs, float *scales, int grid, cudaStream_t st) {
+    opqk::quantize_kernel<G, V><<<grid, 256, 0, st>>>(w, N, K, ldw, qp, codes, signs, scales);
+}
+
+template <int G>
+void dispatch_quant(int vpl, const uint16_t *w, int64_t N, int64_t K, int64_t ldw, const opqk::QuantParams &qp,
+                    uint32_t *codes, uint32_t *signs, float *scales, int grid, cudaStream_t st) {
+    switch (vpl) {
+#define OPQ_Q(V) \
+    case V: launch_quant<G, V>(w, N, K, ldw, qp, codes, signs, scales, grid, st); break;
+        OPQ_Q(1) OPQ_Q(2) OPQ_Q(3) OPQ_Q(4) OPQ_Q(5) OPQ_Q(6) OPQ_Q(7) OPQ_Q(8)
+        OPQ_Q(9) OPQ_Q(10) OPQ_Q(11) OPQ_Q(12) OPQ_Q(13) OPQ_Q(14) OPQ_Q(15) OPQ_Q(16)
+#undef OPQ_Q
+        default: break;
+    }
+}
+
+}  // namespace
+
+extern "C" {
+
+int opq_abi_version(void) { return 1; }
+
+int opq_last_cuda_error(void) { return t_last_cuda_error; }
+
+const char *opq_status_string(opq_status s) {
+    switch (s) {
+        case OPQ_OK: return "OPQ_OK";
+        case OPQ_ERR_INVALID_ARG: return "OPQ_ERR_INVALID_ARG";
+        case OPQ_ERR_UNSUPPORTED_SHAPE: return "OPQ_ERR_UNSUPPORTED_SHAPE";
+        case OPQ_ERR_MISALIGNED: return "OPQ_ERR_MISALIGNED";
+        case OPQ_ERR_WORKSPACE: return "OPQ_ERR_WORKSPACE";
+        case OPQ_ERR_CUDA: return "OPQ_ERR_CUDA";
+        case OPQ_ERR_NOT_DEVICE_MEMORY: return "OPQ_ERR_NOT_DEVICE_MEMORY";
+    }
+    return "OPQ_ERR_UNKNOWN";
+}
+
+opq_status opq_quantize(const uint16_t *w, int64_t N, int64_t K, int64_t ldw, float alpha, uint32_t *codes,
+                        uint32_t *signs, float *scales, void *stream) {
+    opq_status s = check_sizes(N, K);
+    if (s != OPQ_OK) return s;
+    if (K > 32768) return OPQ_ERR_UNSUPPORTED_SHAPE;
+    if (ldw < K || ldw % 8 != 0) return OPQ_ERR_INVALID_ARG;
+    if (!alpha_ok(alpha)) return OPQ_ERR_INVALID_ARG;
+    if ((s = check_ptrs({w, codes, signs, scales})) != OPQ_OK) return s;
+    opqk::QuantParams qp{};
+    const double inv = 1.0 / (double)alpha;
+    qp.t[0] = 0.0;
+    for (int k = 1; k < 16; ++k) qp.t[k] = std::pow(((double)k - 0.5) / 15.0, inv);
+    qp.alpha_is_one = (alpha == 1.0f) ? 1 : 0;
+    DeviceInfo *di = nullptr;
+    if ((s = device_info(&di)) != OPQ_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t nvec = K / 8;
+    if (K <= 4096) {
+        const int vpl = (int)((nvec + 31) / 32);
+        const int64_t blocks = (N + 7) / 8;
+        const int grid = (int)(blocks < (int64_t)di->sms * 8 ? blocks : (int64_t)di->sms * 8);
+        dispatch_quant<1>(vpl, w, N, K, ldw, qp, codes, signs, scales, grid, st);
+    } else {
+        const int vpl = (int)((nvec + 255) / 256);
+        const int64_t blocks = N;
+        const int grid = (int)(blocks < (int64_t)di->sms * 8 ? blocks : (int64_t)di->sms * 8);
+        dispatch_quant<8>(vpl, w, N, K, ldw, qp, codes, signs, scales, grid, st);
+    }
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? OPQ_OK : cuda_fail(e);
+}
+
+opq_status opq_dequantize(const uint32_t *codes, const uint32_t *signs, const float *scales, int64_t N, int64_t K,
+                          float alpha, uint16_t *w_out, void *stream) {
+    opq_status s = check_sizes(N, K);
+    if (s != OPQ_OK) return s;
+    if (!alpha_ok(alpha)) return OPQ_ERR_INVALID_ARG;
+    if ((uint64_t)N * (uint64_t)(K / 8) >= (1ull << 40)) return OPQ_ERR_UNSUPPORTED_SHAPE;
+    if ((s = check_ptrs({codes, signs, scales, w_out})) != OPQ_OK) return s;
+    opqk::DequantParams dp{};
+    const double inv = 1.0 / (double)alpha;
+    for (int q = 0; q < 16; ++q) dp.lut[q] = std::pow((double)q / 15.0, inv);
+    DeviceInfo *di = nullptr;
+    if ((s = device_info(&di)) != OPQ_OK) return s;
+    const uint64_t total = (uint64_t)N * (uint64_t)(K / 8);
+    uint64_t blocks = (total + 255) / 256;
+    const uint64_t cap = (uint64_t)di->sms * 16;
+    if (blocks > cap) blocks = cap;
+    opqk::dequantize_kernel<<<(int)blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        codes, signs, scales, (uint32_t)N, (uint32_t)(K / 8), dp, w_out);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? OPQ_OK : cuda_fail(e);
+}
+
+opq_status opq_linear_workspace_size(int64_t M, int64_t N, int64_t K, size_t *bytes) {
+    if (!bytes) return OPQ_ERR_INVALID_ARG;
+    if (M < 1) return OPQ_ERR_INVALID_ARG;
+    opq_status s = check_sizes(N, K);
+    if (s != OPQ_OK) return s;
+    if (M > INT32_MAX) return OPQ_ERR_UNSUPPORTED_SHAPE;
+    *bytes = make_plan(M, N, K).ws_bytes;
+    return OPQ_OK;
+}
+
+opq_status opq_linear_plan(int64_t M, int64_t N, int64_t K, int *path, int *splits, int *launches) {
+    if (M < 1) return OPQ_ERR_INVALID_ARG;
+    opq_status s = check_sizes(N, K);
+    if (s != OPQ_OK) return s;
+    if (M > INT32_MAX) return OPQ_ERR_UNSUPPORTED_SHAPE;
+    const Plan p = make_plan(M, N, K);
+    if (path) *path = p.path;
+    if (splits) *splits = p.splits;
+    if (launches) *launches = p.launches;
+    return OPQ_OK;
+}
+
+opq_status opq_linear(const uint16_t *x, int64_t M, int64_t K, const uint32_t *codes, const uint32_t *signs,
+                      const float *scales, int64_t N, float alpha, uint16_t *y, void *workspace,
+                      size_t workspace_bytes, void *stream) {
+    if (M < 1) return OPQ_ERR_INVALID_ARG;
+    opq_status s = check_sizes(N, K);
+    if (s != OPQ_OK) return s;
+    if (M > INT32_MAX) return OPQ_ERR_UNSUPPORTED_SHAPE;
+    if (!alpha_ok(alpha)) return OPQ_ERR_INVALID_ARG;
+    if ((s = check_ptrs({x, codes, signs, scales, y})) != OPQ_OK) return s;
+    const Plan plan = make_plan(M, N, K);
+    if (plan.ws_bytes > 0) {
+        if (workspace == nullptr || workspace_bytes < plan.ws_bytes) return OPQ_ERR_WORKSPACE;
+        if ((s = check_ptrs({workspace})) != OPQ_OK) return s;
+    }
+    DeviceInfo *di = nullptr;
+    if ((s = device_info(&di)) != OPQ_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+
+    opqk::LinearArgs a{};
+    a.codes = codes;
+    a.signs = signs;
+    a.scales = scales;
+    a.y = y;
+    a.ws = reinterpret_cast<float *>(workspace);
+    a.M = (int)M;
+    a.N = (int)N;
+    a.K = (int)K;
+    a.splits = plan.splits;
+    a.bx = plan.bx;
+    a.tab = decode_table(alpha);
+
+    cudaError_t e;
+    if (plan.path == 0) {
+        CUtensorMap map;
+        if ((s = make_x_map(&map, x, M, K, opqk::tile::BM)) != OPQ_OK) return s;
+        if (!di->tile_attr) {
+            e = cudaFuncSetAttribute(opqk::linear_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     opqk::tile::SMEM_BYTES);
+            if (e != cudaSuccess) return cuda_fail(e);
+            di->tile_attr = true;
+        }
+        const int64_t tiles = ((M + opqk::tile::BM - 1) / opqk::tile::BM) * ((N + opqk::tile::BN - 1) / opqk::tile::BN);
+        const int grid = (int)(tiles < di->sms ? tiles : di->sms);
+        opqk::linear_tile_kernel<<<grid, opqk::tile::THREADS, opqk::tile::SMEM_BYTES, st>>>(map, a);
+    } else {
+        CUtensorMap map;
+        if ((s = make_x_map(&map, x, M, K, (uint32_t)plan.bx)) != OPQ_OK) return s;
+        const int smem = opqk::stream::smem_bytes(plan.bx);
+        const int key = plan.bx / 16;
+        if (!di->stream_attr[key]) {
+            e = cudaFuncSetAttribute(opqk::linear_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     opqk::stream::smem_bytes(256));
+            if (e != cudaSuccess) return cuda_fail(e);
+            di->stream_attr[key] = true;
+        }
+        dim3 grid((unsigned)((N + opqk::stream::BW - 1) / opqk::stream::BW), (unsigned)plan.splits);
+        opqk::linear_stream_kernel<<<grid, opqk::stream::THREADS, smem, st>>>(map, a);
+        if (plan.splits > 1) {
+            e = cudaGetLastError();
+            if (e != cudaSuccess) return cuda_fail(e);
+            const uint64_t total = (uint64_t)M * (uint64_t)N;
+            uint64_t blocks = (total + 255) / 256;
+            const uint64_t cap = (uint64_t)di->sms * 8;
+            if (blocks > cap) blocks = cap;
+            opqk::splitk_reduce_kernel<<<(int)blocks, 256, 0, st>>>(a.ws, scales, a.M, a.N, a.splits, y);
+        }
+    }
+    e = cudaGetLastError();
+    return e == cudaSuccess ? OPQ_OK : cuda_fail(e);
+}
+
+opq_status opq_device_error(void *stream, uint32_t *err) {
+    if (!err) return OPQ_ERR_INVALID_ARG;
+    cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e);
+    uint32_t v = 0, zero = 0;
+    e = cudaMemcpyFromSymbol(&v, opqdev::g_error, sizeof v);
+    if (e != cudaSuccess) return cuda_fail(e);
+    e = cudaMemcpyToSymbol(opqdev::g_error, &zero, sizeof zero);
+    if (e != cudaSuccess) return cuda_fail(e);
+    *err = v;
+    return OPQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,145 @@
+/*
+ * opq.h — C ABI of the B200 (sm_100a) OPQ library, libopq.so.
+ *
+ * OPQ (Optimal Power Quantization) as described on the "OPQ INT4 Z-Image"
+ * model card: per output row n of a weight matrix W[N, K],
+ *     u = |w| / max_k |w[n, k]|,   v = u^alpha,   q = round(15 v)  (ties to even),
+ *     w' = sign(w) * (q / 15)^(1 / alpha) * max_k |w[n, k]|
+ * ("OPQ principle"), stored as 4-bit magnitudes packed 8 per uint32 and 1-bit
+ * signs packed 32 per uint32 ("Technical details / storage format"), decoded
+ * for inference as sign * (q/15)^(1/alpha) * max ("inference decoding").
+ * This library keeps one fp32 scale (the row's max |w|) per output row where
+ * the card keeps one fp16 max per group of 128.
+ *
+ * Packed format of an N x K weight (K a multiple of 32), all row-major:
+ *   codes  uint32 [N, K/8]   element (n, 8j+i) is bits 4i..4i+3 of codes[n, j]
+ *   signs  uint32 [N, K/32]  element (n, 32j+i) is bit i of signs[n, j]; 1 = negative
+ *   scales float  [N]        max_k |w[n, k]| (exact: a bf16 value)
+ * bf16 tensors are passed as their 16-bit patterns (uint16_t).
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers (cudaMalloc'd or managed memory of
+ *     the current device); host pointers are rejected with
+ *     OPQ_ERR_NOT_DEVICE_MEMORY before anything is launched.
+ *   - Ownership stays with the caller; the library allocates no device memory.
+ *   - Every pointer must be 16-byte aligned (OPQ_ERR_MISALIGNED otherwise).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t, NULL = legacy default
+ *     stream). The return value reports argument errors (checked before any
+ *     launch) and launch errors; execution errors surface at the caller's next
+ *     synchronisation, and device-side wait time-outs are reported by
+ *     opq_device_error().
+ *   - alpha must be finite and > 0. Non-finite weights are accepted without
+ *     trapping; their codes and scales are unspecified.
+ *   - Sizes are int64_t; N, K, M must be >= 1 and K % 32 == 0.
+ */
+#ifndef OPQ_H
+#define OPQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum opq_status {
+    OPQ_OK = 0,
+    OPQ_ERR_INVALID_ARG = 1,        /* null pointer, non-positive size, bad alpha, bad ldw */
+    OPQ_ERR_UNSUPPORTED_SHAPE = 2,  /* K % 32 != 0, or a size beyond the supported range */
+    OPQ_ERR_MISALIGNED = 3,         /* a pointer is not 16-byte aligned */
+    OPQ_ERR_WORKSPACE = 4,          /* workspace missing or smaller than opq_linear_workspace_size */
+    OPQ_ERR_CUDA = 5,               /* a CUDA runtime/driver call failed (see opq_last_cuda_error) */
+    OPQ_ERR_NOT_DEVICE_MEMORY = 6   /* a tensor pointer is not device-accessible memory */
+} opq_status;
+
+/*
+ * opq_quantize — steps "normalise, power transform, quantize, pack" of the
+ * card's "OPQ principle" and "storage format", one output row at a time.
+ *   w       bf16 [N, ldw] device, row-major; columns 0..K-1 of each row are quantized
+ *   N, K    rows (output features) and columns (input features); K % 32 == 0
+ *   ldw     row stride of w in elements, ldw >= K and ldw % 8 == 0
+ *   alpha   the power (the card's optimum for Z-Image is 0.73)
+ *   codes   uint32 [N, K/8] device, written
+ *   signs   uint32 [N, K/32] device, written
+ *   scales  float [N] device, written (max |w| of the row; 0 for an all-zero row,
+ *           whose codes are all 0)
+ * Codes are exactly the round-half-even of 15 (|w|/max)^alpha, decided by
+ * comparing |w| against per-row thresholds max * ((k - 1/2)/15)^(1/alpha)
+ * formed in fp64; the output is deterministic run to run.
+ */
+opq_status opq_quantize(const uint16_t *w, int64_t N, int64_t K, int64_t ldw, float alpha,
+                        uint32_t *codes, uint32_t *signs, float *scales, void *stream);
+
+/*
+ * opq_dequantize — the card's "inference decoding": w' = sign * (q/15)^(1/alpha) * max.
+ *   codes, signs, scales  packed weight as produced by opq_quantize (device)
+ *   N, K                  as for opq_quantize
+ *   alpha                 the power used to quantize
+ *   w_out                 bf16 [N, K] device, row-major, written
+ * The product (q/15)^(1/alpha) * max is formed in fp64 and rounded once to
+ * bf16 (round to nearest even); q = 0 with sign 1 gives -0.0.
+ */
+opq_status opq_dequantize(const uint32_t *codes, const uint32_t *signs, const float *scales,
+                          int64_t N, int64_t K, float alpha, uint16_t *w_out, void *stream);
+
+/*
+ * opq_linear_workspace_size — device scratch bytes opq_linear needs for an
+ * M x K by (N x K)^T product (0 when the chosen kernel needs none).
+ */
+opq_status opq_linear_workspace_size(int64_t M, int64_t N, int64_t K, size_t *bytes);
+
+/*
+ * opq_linear — y = x W'^T with W' decoded from the packed planes (the card's
+ * OPQLinear forward: decode w' = sign * (q/15)^(1/alpha) * max, then matmul).
+ *   x          bf16 [M, K] device, row-major (leading dimension K)
+ *   M, K       activation rows and the reduction length (K % 32 == 0)
+ *   codes, signs, scales   packed W [N, K] (device)
+ *   N          output features
+ *   alpha      the power used to quantize
+ *   y          bf16 [M, N] device, row-major (leading dimension N), written
+ *   workspace  device scratch of at least opq_linear_workspace_size(M, N, K) bytes
+ *              (may be NULL when that size is 0); its contents need no initialisation
+ *              and are garbage afterwards; calls sharing one workspace must not
+ *              overlap on the GPU
+ * Arithmetic: each decoded weight sign * bf16((q/15)^(1/alpha)) enters a bf16
+ * tensor-core product with fp32 accumulation; the row scale is applied to the
+ * fp32 sum, which is then rounded once to bf16. Deterministic: the same inputs
+ * give bitwise-identical y (split-K partial sums are added in a fixed order).
+ */
+opq_status opq_linear(const uint16_t *x, int64_t M, int64_t K, const uint32_t *codes,
+                      const uint32_t *signs, const float *scales, int64_t N, float alpha,
+                      uint16_t *y, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * opq_linear_plan — the kernel opq_linear would use for this shape:
+ *   *path      0 = tile kernel (x rows on the MMA M side), 1 = weight-streaming split-K
+ *              kernel (weight rows on the MMA M side) followed by a fixed-order reduce
+ *   *splits    number of K slices (1 when not split)
+ *   *launches  kernels launched per opq_linear call
+ * Any output pointer may be NULL.
+ */
+opq_status opq_linear_plan(int64_t M, int64_t N, int64_t K, int *path, int *splits, int *launches);
+
+/*
+ * opq_device_error — reads and clears the library's device-side error word on
+ * the current device (synchronises `stream`). 0 = no error; otherwise a bitmask
+ * of OPQ_DEVERR_* recorded by a kernel whose bounded wait on a barrier gave up
+ * (the kernel then returned early and its output is invalid).
+ */
+#define OPQ_DEVERR_WAIT_TIMEOUT 1u
+opq_status opq_device_error(void *stream, uint32_t *err);
+
+/* Human-readable name of a status. */
+const char *opq_status_string(opq_status s);
+
+/* Last CUDA error code (cudaError_t) seen by this thread inside the library, 0 if none. */
+int opq_last_cuda_error(void);
+
+/* ABI version of this header: 1. */
+int opq_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* OPQ_H */

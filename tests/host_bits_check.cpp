@@ -1,0 +1,85 @@
+// Exhaustive host-side check of the kernels' register bit tricks (opq_bits.h)
+// against naive per-element loops. Built and run by tests/test_host_bits.py.
+#include <cstdio>
+#include <cstdlib>
+#include <cstdint>
+#include <random>
+#include <algorithm>
+#include "opq_bits.h"
+
+using namespace opqbits;
+
+static int fails = 0;
+#define CHECK(c, ...) do { if (!(c)) { if (fails < 20) { std::printf(__VA_ARGS__); std::printf("\n"); } ++fails; } } while (0)
+
+int main() {
+    std::mt19937_64 rng(12345);
+    // --- prmt emulation: a few hand-checked cases of the PTX generic mode
+    CHECK(prmt(0x33221100u, 0x77665544u, 0x3210u) == 0x33221100u, "prmt identity");
+    CHECK(prmt(0x33221100u, 0x77665544u, 0x7654u) == 0x77665544u, "prmt upper");
+    CHECK(prmt(0x00008000u, 0u, 0x9999u) == 0xFFFFFFFFu, "prmt sign replicate");
+    CHECK(prmt(0x00007F00u, 0u, 0x9999u) == 0x00000000u, "prmt sign replicate 0");
+    // --- quant_pair: thresholds sorted, <= 0x8000, ties and repeats included
+    for (int trial = 0; trial < 400; ++trial) {
+        uint32_t T[16] = {0};
+        for (int k = 1; k <= 15; ++k) {
+            uint32_t r = (uint32_t)(rng() % 0x8001u);
+            if (trial % 7 == 0) r = (uint32_t)(rng() % 40u) + 0x3F00u;    // crowded thresholds
+            if (trial % 11 == 0 && k > 10) r = 0x8000u;                    // unreachable levels
+            T[k] = r;
+        }
+        std::sort(T + 1, T + 16);
+        if (trial == 0) for (int k = 1; k <= 15; ++k) T[k] = 0x8000u;       // max == 0 row
+        uint32_t P[16];
+        for (int k = 0; k < 16; ++k) P[k] = T[k] * 0x00010001u;
+        const int step = (trial < 8) ? 1 : 37;
+        for (uint32_t m = 0; m < 0x8000u; m += step) {
+            uint32_t m2 = (uint32_t)(rng() & 0x7FFFu);
+            uint32_t s1 = (uint32_t)(rng() & 1u), s2 = (uint32_t)(rng() & 1u);
+            uint32_t w2 = (m | (s1 << 15)) | ((m2 | (s2 << 15)) << 16);
+            uint32_t q2 = quant_pair(w2, P);
+            uint32_t want_lo = 0, want_hi = 0;
+            for (int k = 1; k <= 15; ++k) { want_lo += (m >= T[k]); want_hi += (m2 >= T[k]); }
+            CHECK((q2 & 0xFFFFu) == want_lo && (q2 >> 16) == want_hi,
+                  "quant_pair trial %d m %x m2 %x got %x want %x %x", trial, m, m2, q2, want_lo, want_hi);
+        }
+    }
+    // --- pack_codes / sign_byte
+    for (int trial = 0; trial < 100000; ++trial) {
+        uint32_t q[8], w[4], want_code = 0, want_sb = 0;
+        for (int i = 0; i < 8; ++i) { q[i] = (uint32_t)(rng() & 15u); want_code |= q[i] << (4 * i); }
+        for (int p = 0; p < 4; ++p) w[p] = (uint32_t)rng();
+        for (int i = 0; i < 8; ++i) want_sb |= ((w[i / 2] >> (i % 2 ? 31 : 15)) & 1u) << i;
+        uint32_t code = pack_codes(q[0] | q[1] << 16, q[2] | q[3] << 16, q[4] | q[5] << 16, q[6] | q[7] << 16);
+        CHECK(code == want_code, "pack_codes %x %x", code, want_code);
+        uint32_t sb = sign_byte(w[0], w[1], w[2], w[3]);
+        CHECK(sb == want_sb, "sign_byte %x %x", sb, want_sb);
+    }
+    // --- decode8: random non-negative bf16 tables, every code word pattern class
+    for (int trial = 0; trial < 200; ++trial) {
+        uint16_t lut[16];
+        for (int q = 0; q < 16; ++q) lut[q] = (uint16_t)(rng() & 0x7FFFu);
+        if (trial == 0) lut[0] = 0;
+        DecodeTable T;
+        for (int j = 0; j < 4; ++j) {
+            T.L[j] = 0; T.H[j] = 0;
+            for (int b = 0; b < 4; ++b) {
+                T.L[j] |= (uint32_t)(lut[4 * j + b] & 0xFFu) << (8 * b);
+                T.H[j] |= (uint32_t)(lut[4 * j + b] >> 8) << (8 * b);
+            }
+        }
+        for (int rep = 0; rep < 5000; ++rep) {
+            uint32_t c = (uint32_t)rng(), sb = (uint32_t)(rng() & 0xFFu);
+            uint32_t out[4];
+            decode8(c, sb, T, out);
+            for (int i = 0; i < 8; ++i) {
+                uint32_t q = (c >> (4 * i)) & 15u;
+                uint32_t want = lut[q] | (((sb >> i) & 1u) << 15);
+                uint32_t got = (out[i / 2] >> (16 * (i % 2))) & 0xFFFFu;
+                CHECK(got == want, "decode8 c %x sb %x i %d got %x want %x", c, sb, i, got, want);
+            }
+        }
+    }
+    std::printf("%s fails=%d\n", fails ? "FAIL" : "OK", fails);
+    return fails ? 1 : 0;
+}

@@ -1,0 +1,128 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry point
+that include/opq.h declares, and rejects bad arguments before any launch."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import bit_diffusion_transformer_b200 as opq
+from bit_diffusion_transformer_b200 import build as opq_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "opq.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    opq_build.build()
+    return opq.load()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(opq_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_header_declarations_are_exported(lib):
+    names = declared_functions()
+    assert "opq_quantize" in names and "opq_linear" in names and "opq_dequantize" in names
+    for name in names:
+        assert hasattr(lib, name), f"{name} declared in opq.h but not exported"
+    assert set(names) == set(opq.EXPORTS)
+
+
+def test_version_and_status_strings(lib):
+    assert lib.opq_abi_version() == 1
+    for code, name in [(0, b"OPQ_OK"), (1, b"OPQ_ERR_INVALID_ARG"), (2, b"OPQ_ERR_UNSUPPORTED_SHAPE"),
+                       (3, b"OPQ_ERR_MISALIGNED"), (4, b"OPQ_ERR_WORKSPACE"), (5, b"OPQ_ERR_CUDA"),
+                       (6, b"OPQ_ERR_NOT_DEVICE_MEMORY"), (99, b"OPQ_ERR_UNKNOWN")]:
+        assert lib.opq_status_string(code) == name
+
+
+def _buf(nbytes, offset=0):
+    a = np.zeros(nbytes + 64, np.uint8)
+    base = (-a.ctypes.data) % 16
+    return a, ctypes.c_void_p(a.ctypes.data + base + offset)
+
+
+def test_quantize_argument_errors(lib):
+    keep = []
+    def b(n, off=0):
+        a, p = _buf(n, off)
+        keep.append(a)
+        return p
+    w, c, s, sc = b(256 * 2), b(64), b(16), b(16)
+    q = lib.opq_quantize
+    assert q(None, 4, 32, 32, 0.73, c, s, sc, None) == 1          # null pointer
+    assert q(w, 0, 32, 32, 0.73, c, s, sc, None) == 1             # N = 0
+    assert q(w, 4, 48, 48, 0.73, c, s, sc, None) == 2             # K % 32 != 0
+    assert q(w, 4, 32 * 1025 * 1, 32 * 1025, 0.73, c, s, sc, None) == 2  # K beyond 32768
+    assert q(w, 4, 32, 16, 0.73, c, s, sc, None) == 1             # ldw < K
+    assert q(w, 4, 32, 36, 0.73, c, s, sc, None) == 1             # ldw % 8 != 0
+    for bad in (0.0, -0.5, float("nan"), float("inf")):
+        assert q(w, 4, 32, 32, bad, c, s, sc, None) == 1          # alpha
+    assert q(b(512, 2), 4, 32, 32, 0.73, c, s, sc, None) == 3     # misaligned
+    assert q(w, 4, 32, 32, 0.73, c, s, sc, None) == 6             # host memory, not device memory
+
+
+def test_dequantize_and_linear_argument_errors(lib):
+    keep = []
+    def b(n, off=0):
+        a, p = _buf(n, off)
+        keep.append(a)
+        return p
+    c, s, sc, out = b(64), b(16), b(16), b(512)
+    assert lib.opq_dequantize(c, s, sc, 4, 40, 0.73, out, None) == 2
+    assert lib.opq_dequantize(c, s, sc, 4, 32, 0.0, out, None) == 1
+    assert lib.opq_dequantize(c, None, sc, 4, 32, 0.73, out, None) == 1
+    assert lib.opq_dequantize(c, s, sc, 4, 32, 0.73, out, None) == 6
+    x, y = b(4096), b(4096)
+    L = lib.opq_linear
+    assert L(x, 0, 32, c, s, sc, 4, 0.73, y, None, 0, None) == 1
+    assert L(x, 2, 33, c, s, sc, 4, 0.73, y, None, 0, None) == 2
+    assert L(x, 2, 32, c, s, sc, 0, 0.73, y, None, 0, None) == 1
+    assert L(x, 2, 32, c, s, sc, 4, float("nan"), y, None, 0, None) == 1
+    assert L(x, 2, 32, c, s, sc, 4, 0.73, b(64, 8), None, 0, None) == 3
+    assert L(x, 2, 32, c, s, sc, 4, 0.73, y, None, 0, None) == 6
+
+
+def test_plan_and_workspace_host_logic(lib):
+    # weight streaming for small M, split so that ~2 CTAs per SM exist, no empty slice
+    for M, N, K in [(1, 11520, 3840), (16, 11520, 3840), (64, 11520, 3840), (256, 11520, 3840),
+                    (1, 3840, 3840), (17, 257, 96), (1, 64, 32)]:
+        path, splits, launches = opq.plan(M, N, K)
+        assert path == 1
+        nkb = -(-K // 64)
+        per = -(-nkb // splits)
+        assert (splits - 1) * per < nkb <= splits * per
+        assert launches == (2 if splits > 1 else 1)
+        ws = opq.workspace_size(M, N, K)
+        assert ws == (splits * M * N * 4 if splits > 1 else 0)
+    assert opq.plan(3072, 3840, 3840) == (0, 1, 1)
+    assert opq.workspace_size(3072, 3840, 3840) == 0
+    sz = ctypes.c_size_t(0)
+    assert lib.opq_linear_workspace_size(0, 4, 32, ctypes.byref(sz)) == 1
+    assert lib.opq_linear_workspace_size(4, 4, 40, ctypes.byref(sz)) == 2
+    assert lib.opq_linear_workspace_size(4, 4, 32, None) == 1
+
+
+def test_python_binding_refuses_cpu_tensors():
+    import torch
+    w = torch.zeros(4, 32, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        opq.quantize(w)
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    import importlib
+    mod = importlib.import_module("bit_diffusion_transformer_b200")
+    saved = mod._lib
+    mod._lib = None
+    try:
+        with pytest.raises(ImportError):
+            mod.load(str(tmp_path / "nope.so"))
+    finally:
+        mod._lib = saved
