@@ -27,7 +27,9 @@ _STATUS = {0: "OPQ_OK", 1: "OPQ_ERR_INVALID_ARG", 2: "OPQ_ERR_UNSUPPORTED_SHAPE"
            4: "OPQ_ERR_WORKSPACE", 5: "OPQ_ERR_CUDA", 6: "OPQ_ERR_NOT_DEVICE_MEMORY"}
 
 EXPORTS = ["opq_quantize", "opq_dequantize", "opq_linear_workspace_size", "opq_linear", "opq_linear_plan",
-           "opq_device_error", "opq_status_string", "opq_last_cuda_error", "opq_abi_version"]
+           "opq_linear_noalloc", "opq_device_error", "opq_status_string", "opq_last_cuda_error",
+           "opq_abi_version"]
+NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 
 class OPQError(RuntimeError):
@@ -55,11 +57,12 @@ def load(path: str = LIB_PATH):
     lib.opq_linear.argtypes = [P, I, I, P, P, P, I, F, P, P, S, P]
     lib.opq_linear_plan.argtypes = [I, I, I, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int),
                                     ctypes.POINTER(ctypes.c_int)]
+    lib.opq_linear_noalloc.argtypes = [P, I, I, P, P, P, I, F, P, P]
     lib.opq_device_error.argtypes = [P, ctypes.POINTER(ctypes.c_uint32)]
     lib.opq_status_string.argtypes = [ctypes.c_int]
     lib.opq_status_string.restype = ctypes.c_char_p
     for f in ("opq_quantize", "opq_dequantize", "opq_linear_workspace_size", "opq_linear", "opq_linear_plan",
-              "opq_device_error"):
+              "opq_linear_noalloc", "opq_device_error"):
         getattr(lib, f).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -141,6 +144,21 @@ def linear(x: torch.Tensor, codes: torch.Tensor, signs: torch.Tensor, scales: to
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check(load().opq_linear(_ptr(x), M, K, _ptr(codes), _ptr(signs), _ptr(scales), N, float(alpha), _ptr(y),
                              ws_ptr, ws_bytes, _stream(x.device)), "opq_linear")
+    return y
+
+
+def linear_noalloc(x: torch.Tensor, codes: torch.Tensor, signs: torch.Tensor, scales: torch.Tensor,
+                   alpha: float = ALPHA, out=None):
+    """y = x @ W'^T without a caller workspace: split-K partial sums use the library's
+    static 16 MiB device array (for callers that cannot allocate device memory).
+    Calls that overlap on the GPU race on that array; shapes needing more scratch raise."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2
+    _need_cuda(x, codes, signs, scales)
+    M, K = x.shape
+    N = codes.shape[0]
+    y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _check(load().opq_linear_noalloc(_ptr(x), M, K, _ptr(codes), _ptr(signs), _ptr(scales), N, float(alpha),
+                                     _ptr(y), _stream(x.device)), "opq_linear_noalloc")
     return y
 
 

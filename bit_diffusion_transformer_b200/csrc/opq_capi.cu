@@ -381,4 +381,46 @@ opq_status opq_device_error(void *stream, uint32_t *err) {
     return OPQ_OK;
 }
 
+// ---------------------------------------------------------------------------
+// Allocation-free linear: the split-K scratch lives in a static device array.
+// ---------------------------------------------------------------------------
 }  // extern "C"
+
+namespace {
+// Scratch for opq_linear_noalloc only. In host code `g_noalloc_scratch` names a
+// host-side shadow, not the device array: kernels get the device address looked
+// up with cudaGetSymbolAddress (per device, with that device current).
+static __device__ __align__(256) float g_noalloc_scratch[OPQ_NOALLOC_SCRATCH_BYTES / sizeof(float)];
+
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[64] = {nullptr};
+
+opq_status noalloc_scratch(void **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (dev < 0 || dev >= 64) return OPQ_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail(e);
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return OPQ_OK;
+}
+}  // namespace
+
+extern "C" opq_status opq_linear_noalloc(const uint16_t *x, int64_t M, int64_t K, const uint32_t *codes,
+                                         const uint32_t *signs, const float *scales, int64_t N, float alpha,
+                                         uint16_t *y, void *stream) {
+    size_t need = 0;
+    opq_status s = opq_linear_workspace_size(M, N, K, &need);
+    if (s != OPQ_OK) return s;
+    if (need > (size_t)OPQ_NOALLOC_SCRATCH_BYTES) return OPQ_ERR_WORKSPACE;
+    void *scratch = nullptr;
+    if (need > 0 && (s = noalloc_scratch(&scratch)) != OPQ_OK) return s;
+    return opq_linear(x, M, K, codes, signs, scales, N, alpha, y, scratch,
+                      need > 0 ? (size_t)OPQ_NOALLOC_SCRATCH_BYTES : 0, stream);
+}

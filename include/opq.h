@@ -121,6 +121,32 @@ opq_status opq_linear(const uint16_t *x, int64_t M, int64_t K, const uint32_t *c
 opq_status opq_linear_plan(int64_t M, int64_t N, int64_t K, int *path, int *splits, int *launches);
 
 /*
+ * opq_linear_noalloc — opq_linear without a caller-provided workspace. The paper
+ * has no counterpart; this entry point exists for callers that cannot allocate
+ * device memory themselves: code embedded in a host runtime that owns the GPU's
+ * memory pool and forbids foreign cudaMalloc calls after start-up, or code whose
+ * fixed operator signature has no slot for a scratch buffer.
+ *   Arguments and results are those of opq_linear (x, codes, signs, scales, y are
+ *   still the caller's device buffers); the split-K partial sums go to a static
+ *   device array of OPQ_NOALLOC_SCRATCH_BYTES (16 MiB) inside libopq.so, which
+ *   every GPU that loads the library holds until the process exits.
+ *   - Shapes whose opq_linear_workspace_size exceeds OPQ_NOALLOC_SCRATCH_BYTES are
+ *     rejected with OPQ_ERR_WORKSPACE before anything is launched.
+ *   - The first call on a device looks up the array's device address on that
+ *     device (cudaGetSymbolAddress, with that device current); make that first
+ *     call before any stream capture on the device.
+ *   - All calls share the one array and it keeps the last call's contents. The
+ *     kernels write every partial sum they later read, so nothing needs clearing,
+ *     but calls that overlap on the GPU (different streams, or different host
+ *     threads without ordering) race on the array and give wrong results.
+ *   - No device memory is allocated or freed by this call.
+ */
+#define OPQ_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+opq_status opq_linear_noalloc(const uint16_t *x, int64_t M, int64_t K, const uint32_t *codes,
+                              const uint32_t *signs, const float *scales, int64_t N, float alpha,
+                              uint16_t *y, void *stream);
+
+/*
  * opq_device_error — reads and clears the library's device-side error word on
  * the current device (synchronises `stream`). 0 = no error; otherwise a bitmask
  * of OPQ_DEVERR_* recorded by a kernel whose bounded wait on a barrier gave up
