@@ -143,7 +143,7 @@ def gpu_arm(args, rank, world, local_rank):
     y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     wq = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
     ws_bytes = opq.workspace_size(M, N, K)
-    ws = torch.empty((max(ws_bytes, 16),), dtype=torch.uint8, device=dev)
+    ws = torch.zeros((max(ws_bytes, 16),), dtype=torch.uint8, device=dev)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush = torch.empty((4 * max(l2, 64 << 20),), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -227,7 +227,7 @@ def gpu_arm(args, rank, world, local_rank):
         for m in workloads.SMALL_M_SWEEP:
             xm = workloads.small_m(m).make_x(dev)
             ym = torch.empty((m, qkv.N), dtype=torch.bfloat16, device=dev)
-            wsm = torch.empty((max(opq.workspace_size(m, qkv.N, qkv.K), 16),), dtype=torch.uint8, device=dev)
+            wsm = torch.zeros((max(opq.workspace_size(m, qkv.N, qkv.K), 16),), dtype=torch.uint8, device=dev)
             fn = lambda: opq.linear(xm, *pq, alpha, out=ym, workspace=wsm)
             for _ in range(3):
                 fn()
@@ -370,7 +370,7 @@ def profile_run(args):
     planes = opq.quantize(w, lin.alpha)
     y = torch.empty((lin.M, lin.N), dtype=torch.bfloat16, device=dev)
     wq = torch.empty_like(w)
-    ws = torch.empty((max(opq.workspace_size(lin.M, lin.N, lin.K), 16),), dtype=torch.uint8, device=dev)
+    ws = torch.zeros((max(opq.workspace_size(lin.M, lin.N, lin.K), 16),), dtype=torch.uint8, device=dev)
     fns = {"quantize": lambda: opq.quantize(w, lin.alpha, out=planes),
            "dequantize": lambda: opq.dequantize(*planes, lin.alpha, out=wq)}
     fn = fns.get(args.profile, lambda: opq.linear(x, *planes, lin.alpha, out=y, workspace=ws))

@@ -131,7 +131,10 @@ def plan(M: int, N: int, K: int):
 
 def linear(x: torch.Tensor, codes: torch.Tensor, signs: torch.Tensor, scales: torch.Tensor,
            alpha: float = ALPHA, out=None, workspace=None):
-    """y = x @ W'^T for bf16 x[M, K] and a packed W[N, K] -> bf16 y[M, N]."""
+    """y = x @ W'^T for bf16 x[M, K] and a packed W[N, K] -> bf16 y[M, N].
+
+    ``workspace`` (uint8 device tensor of at least workspace_size(M, N, K) bytes)
+    must be zero-filled before its first use; every call leaves it reusable."""
     assert x.dtype == torch.bfloat16 and x.dim() == 2
     _need_cuda(x, codes, signs, scales)
     M, K = x.shape
@@ -139,7 +142,7 @@ def linear(x: torch.Tensor, codes: torch.Tensor, signs: torch.Tensor, scales: to
     y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     need = workspace_size(M, N, K)
     if need and workspace is None:
-        workspace = torch.empty((need,), dtype=torch.uint8, device=x.device)
+        workspace = torch.zeros((need,), dtype=torch.uint8, device=x.device)   # must start zeroed
     ws_ptr = _ptr(workspace) if workspace is not None else ctypes.c_void_p(0)
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check(load().opq_linear(_ptr(x), M, K, _ptr(codes), _ptr(signs), _ptr(scales), N, float(alpha), _ptr(y),

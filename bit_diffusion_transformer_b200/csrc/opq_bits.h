@@ -126,4 +126,48 @@ OPQ_HD void decode8(uint32_t c, uint32_t sb, const DecodeTable &T, uint32_t out[
     }
 }
 
+// ---------------------------------------------------------------------------
+// Pair-table decode. A 64 KiB shared-memory table holds, for every code byte b
+// (two nibbles = two consecutive weights), the bf16 pair
+//     value(b) = LUT[b & 15] | LUT[b >> 4] << 16
+// and, for every sign byte s (signs of 8 consecutive weights = 4 pairs), a
+// spread word
+//     spread(s) = sum_p  s[2p] << (15 - p)  |  s[2p+1] << (31 - p)
+// so that (spread(s) << p) & 0x80008000 is the sign mask of pair p.
+// Entry b occupies bytes [256 b, 256 b + 256): 32 copies of value(b) at
+// 256 b + 4 lane, then 32 copies of spread(b) at 256 b + 128 + 4 lane; each lane
+// reads its own copy, so the 32 lanes of a warp hit 32 different banks.
+// The byte offset of a lookup is built by one PRMT from the code (or sign) word
+// and a per-lane word holding 4 lane (or 128 + 4 lane) in its low byte.
+// ---------------------------------------------------------------------------
+constexpr uint32_t kPairTableBytes = 256u * 256u;
+
+OPQ_HD uint32_t pair_value(uint32_t b, const uint16_t (&lut)[16]) {
+    return (uint32_t)lut[b & 15u] | ((uint32_t)lut[(b >> 4) & 15u] << 16);
+}
+
+OPQ_HD uint32_t sign_spread(uint32_t s) {
+    uint32_t x = 0;
+    for (int p = 0; p < 4; ++p) {
+        x |= ((s >> (2 * p)) & 1u) << (15 - p);
+        x |= ((s >> (2 * p + 1)) & 1u) << (31 - p);
+    }
+    return x;
+}
+
+// Byte offset of code byte p of c (value part) for the lane whose low byte is in lw.
+OPQ_HD uint32_t pair_offset(uint32_t c, uint32_t lw, uint32_t p) { return prmt(c, lw, 0x5504u | (p << 4)); }
+
+// 8 weights: code word c, sign word sw (byte j holds their signs), values from
+// the table via `load(offset)`. lw = 4 lane, lw2 = 128 + 4 lane.
+template <class Load>
+OPQ_HD void decode8_table(uint32_t c, uint32_t sw, uint32_t j, uint32_t lw, uint32_t lw2, Load load,
+                          uint32_t out[4]) {
+    const uint32_t x = load(prmt(sw, lw2, 0x5504u | (j << 4)));
+    out[0] = load(pair_offset(c, lw, 0)) ^ (x & 0x80008000u);
+    out[1] = load(pair_offset(c, lw, 1)) ^ ((x << 1) & 0x80008000u);
+    out[2] = load(pair_offset(c, lw, 2)) ^ ((x << 2) & 0x80008000u);
+    out[3] = load(pair_offset(c, lw, 3)) ^ ((x << 3) & 0x80008000u);
+}
+
 }  // namespace opqbits

@@ -64,8 +64,7 @@ uint16_t host_bf16(double v) {
 
 struct DeviceInfo {
     int sms = 0;
-    bool tile_attr = false;
-    bool stream_attr[17] = {false};
+    bool linear_attr[17] = {false};
 };
 std::mutex g_mu;
 DeviceInfo g_dev[64];
@@ -123,54 +122,79 @@ opq_status make_x_map(CUtensorMap *map, const void *x, int64_t rows, int64_t K, 
     return OPQ_OK;
 }
 
-opqbits::DecodeTable decode_table(float alpha) {
-    opqbits::DecodeTable t;
+// bf16 (q/15)^(1/alpha) for q = 0..15 (the decoded magnitudes before the row scale)
+void lut_bf16(float alpha, uint16_t (&lut)[16]) {
     const double inv = 1.0 / (double)alpha;
-    uint16_t lut[16];
     for (int q = 0; q < 16; ++q) lut[q] = host_bf16(std::pow((double)q / 15.0, inv));
-    for (int j = 0; j < 4; ++j) {
-        t.L[j] = 0;
-        t.H[j] = 0;
-        for (int b = 0; b < 4; ++b) {
-            t.L[j] |= (uint32_t)(lut[4 * j + b] & 0xFFu) << (8 * b);
-            t.H[j] |= (uint32_t)(lut[4 * j + b] >> 8) << (8 * b);
-        }
+}
+
+// uint32 plane [rows, words] row-major, box {box_words, box_rows}, zero fill. With the
+// 64-byte swizzle (box rows of 64 bytes) 16-byte chunk c of row r lands at c ^ ((r >> 1) & 3).
+opq_status make_u32_map(CUtensorMap *map, const void *p, int64_t rows, int64_t words, uint32_t box_words,
+                        uint32_t box_rows, CUtensorMapSwizzle swizzle) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return OPQ_ERR_CUDA;
+    cuuint64_t dims[2] = {(cuuint64_t)words, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)words * 4};
+    cuuint32_t box[2] = {box_words, box_rows};
+    cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void *>(p), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        t_last_cuda_error = (int)r;
+        return OPQ_ERR_CUDA;
     }
-    return t;
+    return OPQ_OK;
 }
 
 struct Plan {
-    int path;      // 0 tile, 1 weight streaming
-    int splits;
-    int bx;
+    int mode;       // 0 whole tiles, 1 stream-K with a fixed-order fix-up
+    int bx;         // activation rows per tile (the MMA N)
+    int m_tiles, n_tiles, kblocks;
+    int grid;       // CTAs of the linear kernel
+    int runs_max;   // mode 1
+    size_t counter_bytes;   // mode 1: the zero-between-calls arrival counters at the workspace start
     size_t ws_bytes;
     int launches;
 };
 
+// The schedule depends on the shape alone (a fixed 148-CTA budget), so the
+// workspace size and the result bits are the same on every B200.
+// Stream-K arrival counters occupy a fixed region at the start of every
+// workspace (4 per weight tile, at most kCounterTiles tiles), so that no shape's
+// partial sums ever land on counters another shape relies on being zero.
+constexpr int kCounterTiles = 4096;
+constexpr size_t kCounterBytes = (size_t)kCounterTiles * 4u * sizeof(uint32_t);   // 64 KiB
+
 Plan make_plan(int64_t M, int64_t N, int64_t K) {
     Plan p{};
-    if (M <= 256) {
-        p.path = 1;
-        p.bx = (int)((M + 15) / 16 * 16);
-        const int64_t tiles = (N + opqk::stream::BW - 1) / opqk::stream::BW;
-        const int64_t nkb = (K + opqk::stream::BK - 1) / opqk::stream::BK;
-        int64_t s = (2 * kPlanSMs + tiles - 1) / tiles;        // about two CTAs per SM
-        const int64_t max_s = nkb / 4 > 1 ? nkb / 4 : 1;       // keep >= 4 k-blocks per slice
-        if (s > max_s) s = max_s;
-        if (s > 16) s = 16;
-        if (s < 1) s = 1;
-        const int64_t per = (nkb + s - 1) / s;
-        s = (nkb + per - 1) / per;                             // no empty slice
-        p.splits = (int)s;
-        p.ws_bytes = s > 1 ? (size_t)s * (size_t)M * (size_t)N * sizeof(float) : 0;
-        p.launches = s > 1 ? 2 : 1;
+    p.kblocks = (int)((K + 127) / 128);
+    p.n_tiles = (int)((N + 127) / 128);
+    if (M <= 128) {
+        p.bx = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
+        p.m_tiles = 1;
     } else {
-        p.path = 0;
-        p.splits = 1;
-        p.bx = 0;
-        p.ws_bytes = 0;
-        p.launches = 1;
+        p.bx = 256;
+        p.m_tiles = (int)((M + 255) / 256);
     }
+    if (M <= 128 && p.n_tiles <= kCounterTiles) {
+        p.mode = 1;
+        const int64_t U = (int64_t)p.n_tiles * p.kblocks;
+        p.grid = (int)(U < kPlanSMs ? U : kPlanSMs);
+        const int64_t per = (U + p.grid - 1) / p.grid;
+        p.runs_max = (int)((per + p.kblocks - 1) / p.kblocks + 1);
+        p.counter_bytes = kCounterBytes;
+        p.ws_bytes = p.counter_bytes + (size_t)p.grid * (size_t)p.runs_max * (size_t)p.bx * 128u * sizeof(float);
+    } else {
+        p.mode = 0;
+        const int64_t tiles = (int64_t)p.m_tiles * p.n_tiles;
+        p.grid = (int)(tiles < kPlanSMs ? tiles : kPlanSMs);
+        p.runs_max = 1;
+        p.counter_bytes = 0;
+        p.ws_bytes = 0;
+    }
+    p.launches = 1;
     return p;
 }
 
@@ -198,6 +222,21 @@ void dispatch_quant(int vpl, const uint16_t *w, int64_t N, int64_t K, int64_t ld
 #undef OPQ_Q
         default: break;
     }
+}
+
+template <int BX>
+cudaError_t launch_linear(DeviceInfo *di, const Plan &plan, const CUtensorMap &xmap, const CUtensorMap &cmap,
+                          const CUtensorMap &smap, const opqk::LinearArgs &a, cudaStream_t st) {
+    using C = opqk::Cfg<BX>;
+    const int key = BX / 16;
+    if (!di->linear_attr[key]) {
+        cudaError_t e = cudaFuncSetAttribute(opqk::linear_kernel<BX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             C::SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        di->linear_attr[key] = true;
+    }
+    opqk::linear_kernel<BX><<<plan.grid, C::THREADS, C::SMEM_BYTES, st>>>(xmap, cmap, smap, a);
+    return cudaGetLastError();
 }
 
 }  // namespace
@@ -285,14 +324,14 @@ opq_status opq_linear_workspace_size(int64_t M, int64_t N, int64_t K, size_t *by
     return OPQ_OK;
 }
 
-opq_status opq_linear_plan(int64_t M, int64_t N, int64_t K, int *path, int *splits, int *launches) {
+opq_status opq_linear_plan(int64_t M, int64_t N, int64_t K, int *path, int *ctas, int *launches) {
     if (M < 1) return OPQ_ERR_INVALID_ARG;
     opq_status s = check_sizes(N, K);
     if (s != OPQ_OK) return s;
     if (M > INT32_MAX) return OPQ_ERR_UNSUPPORTED_SHAPE;
     const Plan p = make_plan(M, N, K);
-    if (path) *path = p.path;
-    if (splits) *splits = p.splits;
+    if (path) *path = p.mode;
+    if (ctas) *ctas = p.grid;
     if (launches) *launches = p.launches;
     return OPQ_OK;
 }
@@ -316,54 +355,42 @@ opq_status opq_linear(const uint16_t *x, int64_t M, int64_t K, const uint32_t *c
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
 
     opqk::LinearArgs a{};
-    a.codes = codes;
     a.signs = signs;
     a.scales = scales;
     a.y = y;
-    a.ws = reinterpret_cast<float *>(workspace);
+    a.counters = reinterpret_cast<uint32_t *>(workspace);
+    a.ws = plan.ws_bytes ? reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(workspace) + plan.counter_bytes)
+                         : nullptr;
     a.M = (int)M;
     a.N = (int)N;
     a.K = (int)K;
-    a.splits = plan.splits;
-    a.bx = plan.bx;
-    a.tab = decode_table(alpha);
+    a.m_tiles = plan.m_tiles;
+    a.n_tiles = plan.n_tiles;
+    a.kblocks = plan.kblocks;
+    a.mode = plan.mode;
+    a.runs_max = plan.runs_max;
+    lut_bf16(alpha, a.lut);
 
-    cudaError_t e;
-    if (plan.path == 0) {
-        CUtensorMap map;
-        if ((s = make_x_map(&map, x, M, K, opqk::tile::BM)) != OPQ_OK) return s;
-        if (!di->tile_attr) {
-            e = cudaFuncSetAttribute(opqk::linear_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     opqk::tile::SMEM_BYTES);
-            if (e != cudaSuccess) return cuda_fail(e);
-            di->tile_attr = true;
-        }
-        const int64_t tiles = ((M + opqk::tile::BM - 1) / opqk::tile::BM) * ((N + opqk::tile::BN - 1) / opqk::tile::BN);
-        const int grid = (int)(tiles < di->sms ? tiles : di->sms);
-        opqk::linear_tile_kernel<<<grid, opqk::tile::THREADS, opqk::tile::SMEM_BYTES, st>>>(map, a);
+    CUtensorMap xmap, cmap, smap;
+    if ((s = make_x_map(&xmap, x, M, K, (uint32_t)plan.bx)) != OPQ_OK) return s;
+    if ((s = make_u32_map(&cmap, codes, N, K / 8, 16u, 128u, CU_TENSOR_MAP_SWIZZLE_64B)) != OPQ_OK) return s;
+    // the sign plane's rows are 16-byte aligned (a TMA requirement) when K % 128 == 0; otherwise the
+    // kernel copies the sign words with cp.async
+    a.signs_tma = (K % 128 == 0) ? 1 : 0;
+    if (a.signs_tma) {
+        if ((s = make_u32_map(&smap, signs, N, K / 32, 4u, 128u, CU_TENSOR_MAP_SWIZZLE_NONE)) != OPQ_OK) return s;
     } else {
-        CUtensorMap map;
-        if ((s = make_x_map(&map, x, M, K, (uint32_t)plan.bx)) != OPQ_OK) return s;
-        const int smem = opqk::stream::smem_bytes(plan.bx);
-        const int key = plan.bx / 16;
-        if (!di->stream_attr[key]) {
-            e = cudaFuncSetAttribute(opqk::linear_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     opqk::stream::smem_bytes(256));
-            if (e != cudaSuccess) return cuda_fail(e);
-            di->stream_attr[key] = true;
-        }
-        dim3 grid((unsigned)((N + opqk::stream::BW - 1) / opqk::stream::BW), (unsigned)plan.splits);
-        opqk::linear_stream_kernel<<<grid, opqk::stream::THREADS, smem, st>>>(map, a);
-        if (plan.splits > 1) {
-            e = cudaGetLastError();
-            if (e != cudaSuccess) return cuda_fail(e);
-            const uint64_t total = (uint64_t)M * (uint64_t)N;
-            uint64_t blocks = (total + 255) / 256;
-            const uint64_t cap = (uint64_t)di->sms * 8;
-            if (blocks > cap) blocks = cap;
-            opqk::splitk_reduce_kernel<<<(int)blocks, 256, 0, st>>>(a.ws, scales, a.M, a.N, a.splits, y);
-        }
+        smap = cmap;   // not read by the kernel
     }
+    cudaError_t e;
+    switch (plan.bx) {
+        case 16: e = launch_linear<16>(di, plan, xmap, cmap, smap, a, st); break;
+        case 32: e = launch_linear<32>(di, plan, xmap, cmap, smap, a, st); break;
+        case 64: e = launch_linear<64>(di, plan, xmap, cmap, smap, a, st); break;
+        case 128: e = launch_linear<128>(di, plan, xmap, cmap, smap, a, st); break;
+        default: e = launch_linear<256>(di, plan, xmap, cmap, smap, a, st); break;
+    }
+    if (e != cudaSuccess) return cuda_fail(e);
     e = cudaGetLastError();
     return e == cudaSuccess ? OPQ_OK : cuda_fail(e);
 }

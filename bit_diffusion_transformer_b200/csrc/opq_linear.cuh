@@ -2,25 +2,36 @@
 //
 // "OPQ INT4 Z-Image" model card: the OPQLinear forward decodes
 // w = sign * (q/15)^(1/alpha) * max ("inference decoding") and multiplies.
-// Here the row scale max is deferred to the epilogue, so the tensor cores see
-// sign * bf16((q/15)^(1/alpha)) and the fp32 sum is multiplied by scale[n] once.
+// Here the row scale max is deferred to the epilogue: the tensor cores see
+// sign * bf16((q/15)^(1/alpha)) and each fp32 sum is multiplied by scale[n] once.
 //
-// Two kernels, both tcgen05 (5th-generation tensor cores, accumulators in TMEM):
+// One kernel, templated on BX (activation rows per tile, 16..256):
 //
-//  tile kernel (large M): D[128 x 256] = x_tile[128 x K] * W'_tile[256 x K]^T.
-//    x tiles arrive by TMA (128-byte swizzle); W' tiles are decoded by 8 warps
-//    (one weight row per thread) from codes/signs that each thread streams into
-//    its own shared-memory ring with cp.async, and are stored in the same
-//    swizzled K-major layout the MMA reads. One thread issues the MMAs, four
-//    warps drain the double-buffered accumulator (2 x 256 TMEM columns) while
-//    the next tile accumulates. Persistent: one CTA per SM walks the tiles.
+//   D^T[128 x BX] = W'_tile[128 x K] * x_tile[BX x K]^T     (tcgen05, kind::f16)
 //
-//  weight-streaming kernel (small M): the roles swap so that the weights fill
-//    the MMA's 128-row side: D^T[128 x BX] = W'_tile[128 x K] * x[BX x K]^T,
-//    BX = M rounded up to 16. Each CTA decodes one 128-row weight tile over a
-//    slice of K (split-K); fp32 partial sums go to the workspace and a second
-//    kernel adds them in a fixed order, scales and rounds (or, unsplit, the
-//    epilogue writes y directly).
+// Weights sit on the MMA's 128-row side so that each decoded weight meets BX
+// activation rows. Per CTA (one per SM, persistent):
+//   warp 0       raw producer: packed codes of 128 weight rows x 128 K by TMA
+//                (64-byte swizzle), their sign words by cp.async (the sign plane's
+//                row stride need not be 16-byte aligned)
+//   warp 1       TMEM allocation and the single-thread MMA issue; A comes from TMEM
+//   warp 2       x producer: x tiles (BX rows x 64 K, 128-byte swizzle) by TMA, on
+//                its own thread so that neither ring throttles the other
+//   warps 3..10  decoders: two threads per weight row, 32 weights each per 64-K
+//                stage, through the shared-memory pair table (opq_bits.h), written
+//                to TMEM with tcgen05.st as the MMA's A operand; the store of one
+//                stage drains while the next stage is decoded
+//   warps 11..14 epilogue: accumulator TMEM -> registers -> * scale[n] -> bf16 y,
+//                or fp32 partial sums for tiles split across CTAs
+// TMEM columns: [0, 256) eight 64-K A stages; [256, 256 + NACC * BX) accumulators.
+//
+// Work is a list of runs (tile, range of 128-K blocks). Mode 0 gives each CTA
+// whole tiles (tile = blockIdx.x + i * gridDim.x). Mode 1 (stream-K) cuts the
+// flattened (tile, 128-K block) sequence into one contiguous range per CTA; a
+// tile covered by several CTAs leaves fp32 partial sums in the workspace, and
+// the epilogue warp that arrives last on the tile's counter (one per 32-row
+// quarter) adds all partials in CTA order (deterministic), scales, rounds, stores
+// y and resets the counter to zero.
 #pragma once
 #include <cuda_bf16.h>
 
@@ -31,126 +42,236 @@ namespace opqk {
 
 using namespace opqdev;
 
-// ------------------------------------------------------------ cp.async helpers --
-__device__ __forceinline__ void cp_async_16(void *smem_dst, const void *gsrc, uint32_t src_bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)), "l"(gsrc),
-                 "r"(src_bytes)
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
+}
+// a + b as a multiply-add by an opaque 1, so that it issues on the FMA pipe and
+// leaves the integer ALU pipe to the decode's PRMT / LOP3
+__device__ __forceinline__ uint32_t add_fma(uint32_t a, uint32_t b, uint32_t one) {
+    uint32_t r;
+    asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(one), "r"(b));
+    return r;
+}
+
+__device__ __forceinline__ void cp_async_4(uint32_t smem_dst, const void *gsrc, uint32_t src_bytes) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_dst), "l"(gsrc), "r"(src_bytes)
                  : "memory");
 }
-__device__ __forceinline__ void cp_async_4(void *smem_dst, const void *gsrc, uint32_t src_bytes) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(smem_dst)), "l"(gsrc),
-                 "r"(src_bytes)
-                 : "memory");
+// The mbarrier counts one arrival when all of this thread's earlier cp.async copies have landed.
+__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t *bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint32_t (&v)[4]) {
-    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v[0]), "r"(v[1]), "r"(v[2]),
-                 "r"(v[3])
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3])
                  : "memory");
 }
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t *>(&h);
+// tcgen05.st: 32 lanes x 16 consecutive 32-bit columns (thread i -> lane base + i)
+__device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+        "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// tcgen05.ld: 32 lanes x 16 consecutive 32-bit columns
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+
+// Every lane waits (and so acquires); the verdict is made warp-uniform, so a
+// time-out seen by one lane can never leave the others behind at a warp barrier.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity) {
+    const bool ok = mbar_wait(bar, parity);
+    return __all_sync(0xFFFFFFFFu, ok) != 0;
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]^T, kind::f16 (bf16 in, fp32 accumulate), one CTA.
+__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
 }
 
 struct LinearArgs {
-    const uint32_t *codes;
-    const uint32_t *signs;
+    const uint32_t *signs;  // sign plane [N, K/32]
     const float *scales;
     uint16_t *y;
-    float *ws;   // split-K partials [splits, M, N] (weight-streaming kernel only)
+    float *ws;              // mode 1: fp32 partials [grid][runs_max][BX][128]
+    uint32_t *counters;     // mode 1: arrivals per (tile, TMEM lane quarter); zero between calls
+    int signs_tma;          // 1: sign plane rows are 16-byte aligned (K % 128 == 0), load it by TMA
     int M, N, K;
-    int splits;  // weight-streaming kernel
-    int bx;      // weight-streaming kernel: MMA N (x rows per CTA, multiple of 16)
-    opqbits::DecodeTable tab;
+    int m_tiles, n_tiles;
+    int kblocks;            // 128-K blocks per tile
+    int mode;               // 0 whole tiles strided over CTAs, 1 contiguous unit ranges (stream-K)
+    int runs_max;           // mode 1: most runs one CTA can have
+    uint16_t lut[16];       // bf16 (q/15)^(1/alpha)
 };
 
-// Decode one 8-weight chunk and store it as 16 swizzled bytes.
-__device__ __forceinline__ void decode_store(uint32_t code, uint32_t sb, const opqbits::DecodeTable &tab,
-                                             uint32_t dst) {
-    uint32_t o[4];
-    opqbits::decode8(code, sb, tab, o);
-    st_shared_v4(dst, o);
+// Units (tile, 128-K block) of CTA c out of C in stream-K mode: [begin(c), begin(c + 1)).
+__host__ __device__ __forceinline__ int64_t unit_begin(int64_t c, int64_t C, int64_t U) { return (c * U) / C; }
+// The CTA whose range holds unit u.
+__host__ __device__ __forceinline__ int64_t unit_owner(int64_t u, int64_t C, int64_t U) {
+    return ((u + 1) * C - 1) / U;
 }
 
-// ============================================================================
-// Tile kernel (path 0)
-// ============================================================================
-namespace tile {
-constexpr int BM = 128, BN = 256, BK = 64;
-constexpr int STAGES = 3;
-constexpr int RD = 4;                       // per-thread cp.async ring depth
-constexpr int A_BYTES = BM * BK * 2;        // 16 KiB
-constexpr int B_BYTES = BN * BK * 2;        // 32 KiB
-constexpr int RAW_CODE_BYTES = RD * BN * 32;
-constexpr int RAW_SIGN_BYTES = RD * BN * 8;
-constexpr int NUM_DECODE_WARPS = BN / 32;   // one weight row per thread
-constexpr int WARP_TMA = 0, WARP_MMA = 1, WARP_DEC0 = 2;
-constexpr int WARP_EPI0 = WARP_DEC0 + NUM_DECODE_WARPS;  // 10..13
-constexpr int THREADS = (WARP_EPI0 + 4) * 32;             // 448
-constexpr int ACC_COLS = BN;                // fp32 columns per accumulator
-constexpr int TMEM_COLS = 2 * ACC_COLS;     // double-buffered
-// shared memory map (offsets from the 1 KiB-aligned base)
-constexpr int OFF_A = 0;
-constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
-constexpr int OFF_RAWC = OFF_B + STAGES * B_BYTES;
-constexpr int OFF_RAWS = OFF_RAWC + RAW_CODE_BYTES;
-constexpr int OFF_BAR = OFF_RAWS + RAW_SIGN_BYTES;
-constexpr int NUM_BARS = 3 * STAGES + 4 + 1;              // a_full, b_full, empty, acc_full x2, acc_empty x2, drain
-constexpr int OFF_TMEM = OFF_BAR + NUM_BARS * 8;
-constexpr int SMEM_BYTES = OFF_TMEM + 16 + 1024;          // + alignment slack
-static_assert(SMEM_BYTES <= 232448, "tile kernel shared memory");
-constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
-}  // namespace tile
+// The sequence of runs of one CTA; every role walks the same sequence.
+struct RunIter {
+    int mode, tiles, kblocks, grid;
+    int64_t u, u_end;   // mode 1
+    int t_next;         // mode 0
+    int run_idx;
+    __device__ __forceinline__ void init(const LinearArgs &a, int tiles_, int grid_, int cta) {
+        mode = a.mode;
+        tiles = tiles_;
+        kblocks = a.kblocks;
+        grid = grid_;
+        run_idx = 0;
+        t_next = cta;
+        const int64_t U = (int64_t)tiles * kblocks;
+        u = unit_begin(cta, grid_, U);
+        u_end = unit_begin(cta + 1, grid_, U);
+    }
+    // next run: tile, block range [r0, r1), run index j; false at the end
+    __device__ __forceinline__ bool next(int &tile, int &r0, int &r1, int &j) {
+        if (mode == 0) {
+            if (t_next >= tiles) return false;
+            tile = t_next;
+            r0 = 0;
+            r1 = kblocks;
+            t_next += grid;
+        } else {
+            if (u >= u_end) return false;
+            tile = (int)(u / kblocks);
+            r0 = (int)(u - (int64_t)tile * kblocks);
+            const int64_t end = (int64_t)r0 + (u_end - u);
+            r1 = end < (int64_t)kblocks ? (int)end : kblocks;
+            u += r1 - r0;
+        }
+        j = run_idx++;
+        return true;
+    }
+};
 
-__global__ void __launch_bounds__(tile::THREADS, 1)
-    linear_tile_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ LinearArgs args) {
-    using namespace tile;
+template <int BX>
+struct Cfg {
+    static constexpr int BW = 128;                     // weight rows per tile (MMA M)
+    static constexpr int KR = 128;                     // K per raw (codes/signs) stage
+    static constexpr int KA = 64;                      // K per A / x stage
+    static constexpr int RAW_STAGES = BX >= 256 ? 3 : (BX <= 16 ? 6 : 4);
+    static constexpr int A_STAGES = BX >= 256 ? 3 : 4;
+    static constexpr int X_STAGES = BX >= 256 ? 2 : (BX >= 128 ? 3 : (BX >= 64 ? 6 : 10));
+    static constexpr int NACC = 2;                     // accumulators in TMEM, double-buffered
+    static constexpr uint32_t TMEM_COLS = (2 * BX <= 32) ? 32 : (2 * BX <= 64) ? 64 : (2 * BX <= 128) ? 128
+                                                           : (2 * BX <= 256) ? 256 : 512;
+    static constexpr int RAW_CODE_BYTES = BW * KR / 2;    // 8 KiB: [128 rows][16 words], 64-byte swizzle
+    static constexpr int RAW_SIGN_BYTES = BW * KR / 8;    // 2 KiB: [128 rows][4 words]
+    static constexpr int RAW_BYTES = RAW_CODE_BYTES + RAW_SIGN_BYTES;
+    static constexpr int A_BYTES = BW * KA * 2;           // 16 KiB decoded W', 128-byte swizzle, K-major
+    static constexpr int X_BYTES = BX * KA * 2;
+    static constexpr int STAGE_EPI_BYTES = 4 * 2 * 16 * 32 * 2;   // 4 warps x 2 buffers x [16 m][32 n] bf16
+    static constexpr int OFF_TABLE = 0;
+    static constexpr int OFF_RAW = OFF_TABLE + (int)opqbits::kPairTableBytes;
+    static constexpr int OFF_A = OFF_RAW + RAW_STAGES * RAW_BYTES;
+    static constexpr int OFF_X = OFF_A + A_STAGES * A_BYTES;
+    static constexpr int OFF_EPI = OFF_X + X_STAGES * X_BYTES;
+    static constexpr int OFF_BAR = OFF_EPI + STAGE_EPI_BYTES;
+    static constexpr int NUM_BARS = 2 * RAW_STAGES + 2 * X_STAGES + 2 * A_STAGES + 2 * NACC + 1;
+    static constexpr int OFF_TMEM = OFF_BAR + NUM_BARS * 8;
+    static constexpr int SMEM_BYTES = OFF_TMEM + 16 + 1024;
+    static constexpr int WARP_LOAD = 0, WARP_MMA = 1, WARP_XLOAD = 2, WARP_DEC0 = 3, NUM_DEC_WARPS = 16;
+    static constexpr int WARP_EPI0 = WARP_DEC0 + NUM_DEC_WARPS;
+    static constexpr int THREADS = (WARP_EPI0 + 4) * 32;
+    static_assert(SMEM_BYTES <= 232448, "shared memory");
+    static_assert(BX % 16 == 0 && BX >= 16 && BX <= 256, "MMA N");
+    static_assert(RAW_BYTES % 1024 == 0 && A_BYTES % 1024 == 0 && X_BYTES % 1024 == 0, "stage alignment");
+};
+
+template <int BX>
+__global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
+    linear_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_codes,
+                  const __grid_constant__ CUtensorMap tmap_signs, const __grid_constant__ LinearArgs args) {
+    using C = Cfg<BX>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = smem_u32(smem_raw);
     const uint32_t pad = ((raw_base + 1023u) & ~1023u) - raw_base;
     uint8_t *smem = smem_raw + pad;
     const uint32_t sbase = raw_base + pad;
 
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
-    uint64_t *a_full = bars;
-    uint64_t *b_full = bars + STAGES;
-    uint64_t *empty = bars + 2 * STAGES;
-    uint64_t *acc_full = bars + 3 * STAGES;
-    uint64_t *acc_empty = acc_full + 2;
-    uint64_t *drain = acc_empty + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_TMEM);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
+    uint64_t *raw_full = bars;
+    uint64_t *raw_empty = raw_full + C::RAW_STAGES;
+    uint64_t *x_full = raw_empty + C::RAW_STAGES;
+    uint64_t *x_empty = x_full + C::X_STAGES;
+    uint64_t *a_full = x_empty + C::X_STAGES;
+    uint64_t *a_empty = a_full + C::A_STAGES;
+    uint64_t *acc_full = a_empty + C::A_STAGES;
+    uint64_t *acc_empty = acc_full + C::NACC;
+    uint64_t *drain = acc_empty + C::NACC;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_TMEM);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int M = args.M, N = args.N, K = args.K;
-    const int num_m = (M + BM - 1) / BM, num_n = (N + BN - 1) / BN;
-    const int num_tiles = num_m * num_n;
-    const int nkb = (K + BK - 1) / BK;
-    const int my_tiles = (blockIdx.x < num_tiles) ? (num_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    const int tiles = args.m_tiles * args.n_tiles;
+    const bool signs_by_tma = args.signs_tma != 0;
 
+    // ---- pair table: 32 copies of value(b) then 32 copies of spread(b) per entry b
+    for (int e = threadIdx.x; e < 512; e += C::THREADS) {
+        const uint32_t b = (uint32_t)e & 255u;
+        const uint32_t v = e < 256 ? ((uint32_t)args.lut[b & 15u] | ((uint32_t)args.lut[b >> 4] << 16))
+                                   : opqbits::sign_spread(b);
+        const uint32_t dst = sbase + C::OFF_TABLE + b * 256u + (e < 256 ? 0u : 128u);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst + 16u * k), "r"(v) : "memory");
+    }
     if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&a_full[s], 1);
-            mbar_init(&b_full[s], NUM_DECODE_WARPS);
-            mbar_init(&empty[s], 1);
+        for (int s = 0; s < C::RAW_STAGES; ++s) {
+            // the codes' (and signs') expect_tx arrival, plus 32 cp.async arrivals when signs are copied by threads
+            mbar_init(&raw_full[s], signs_by_tma ? 1 : 1 + 32);
+            mbar_init(&raw_empty[s], C::NUM_DEC_WARPS);
         }
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < C::X_STAGES; ++s) {
+            mbar_init(&x_full[s], 1);
+            mbar_init(&x_empty[s], 1);
+        }
+        for (int s = 0; s < C::A_STAGES; ++s) {
+            mbar_init(&a_full[s], C::NUM_DEC_WARPS);
+            mbar_init(&a_empty[s], 1);
+        }
+        for (int s = 0; s < C::NACC; ++s) {
             mbar_init(&acc_full[s], 1);
             mbar_init(&acc_empty[s], 4);
         }
         mbar_init(drain, 1);
         fence_mbar_init();
     }
-    if (warp == WARP_TMA && lane == 0) tma_prefetch_desc(&tmap_x);
-    if (warp == WARP_MMA) {
-        tmem_alloc(tmem_slot, TMEM_COLS);
+    if (warp == C::WARP_LOAD && lane == 0) {
+        tma_prefetch_desc(&tmap_codes);
+        if (signs_by_tma) tma_prefetch_desc(&tmap_signs);
+    }
+    if (warp == C::WARP_XLOAD && lane == 0) tma_prefetch_desc(&tmap_x);
+    if (warp == C::WARP_MMA) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -158,390 +279,309 @@ __global__ void __launch_bounds__(tile::THREADS, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    if (warp == WARP_TMA) {
-        // ------------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0;
-            bool ok = true;
-            int armed = 0;  // loads issued whose completion has not been observed
-            for (int t = 0; t < my_tiles && ok; ++t) {
-                const int tile_id = blockIdx.x + t * gridDim.x;
-                const int m_blk = tile_id % num_m;
-                for (int kb = 0; kb < nkb; ++kb) {
-                    if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
-                    mbar_arrive_expect_tx(&a_full[stage], A_BYTES);
-                    tma_load_2d(smem + OFF_A + stage * A_BYTES, &tmap_x, kb * BK, m_blk * BM, &a_full[stage]);
-                    armed = armed < STAGES ? armed + 1 : STAGES;
-                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+    RunIter it;
+    it.init(args, tiles, gridDim.x, blockIdx.x);
+    int tile, r0, r1, j;
+
+    if (warp == C::WARP_LOAD) {
+        // ----------------------------------------------------------- raw producer
+        const int swd = args.K / 32;        // sign words per row
+        int rs = 0;
+        uint32_t rph = 0;
+        int raw_issued = 0;
+        bool ok = true;
+        while (ok && it.next(tile, r0, r1, j)) {
+            const int n_blk = tile / args.m_tiles;
+            for (int r = r0; r < r1 && ok; ++r) {
+                // lane 0 waits for the stage; the verdict and the ordering reach the other lanes
+                int okw = 1;
+                if (lane == 0) okw = mbar_wait(&raw_empty[rs], rph ^ 1) ? 1 : 0;
+                okw = __shfl_sync(0xFFFFFFFFu, okw, 0);
+                __syncwarp();
+                if (!okw) { ok = false; break; }
+                const uint32_t dst = sbase + C::OFF_RAW + rs * C::RAW_BYTES;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&raw_full[rs], signs_by_tma ? C::RAW_BYTES : C::RAW_CODE_BYTES);
+                    tma_load_2d(smem + C::OFF_RAW + rs * C::RAW_BYTES, &tmap_codes, r * (C::KR / 8), n_blk * C::BW,
+                                &raw_full[rs]);
+                    if (signs_by_tma)
+                        tma_load_2d(smem + C::OFF_RAW + rs * C::RAW_BYTES + C::RAW_CODE_BYTES, &tmap_signs,
+                                    r * (C::KR / 32), n_blk * C::BW, &raw_full[rs]);
                 }
+                if (!signs_by_tma) {
+                    // sign words: 128 rows x 4 words; copy i of lane l is word 32 i + l of the stage
+                    // (consecutive lanes, consecutive banks); out-of-range words read as 0
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int e = i * 32 + lane;
+                        const int row = e >> 2, w = e & 3;
+                        const int n = n_blk * C::BW + row, kw = r * 4 + w;
+                        const bool in = n < args.N && kw < swd;
+                        const uint32_t *src = args.signs + (in ? (size_t)n * swd + kw : 0);
+                        cp_async_4(dst + C::RAW_CODE_BYTES + row * 16 + w * 4, src, in ? 4u : 0u);
+                    }
+                    cp_async_mbar_arrive(&raw_full[rs]);
+                }
+                ++raw_issued;
+                if (++rs == C::RAW_STAGES) { rs = 0; rph ^= 1; }
             }
-            if (!ok) {
-                // let the copies already in flight land before the CTA can exit
-                for (int i = 0; i < armed; ++i) {
-                    if (--stage < 0) { stage = STAGES - 1; phase ^= 1; }
-                    (void)mbar_wait(&a_full[stage], phase);
+        }
+        if (!ok) {
+            // let every copy already issued land before the CTA can exit
+            asm volatile("cp.async.wait_all;" ::: "memory");
+            if (lane == 0) {
+                for (int i = 0; i < raw_issued && i < C::RAW_STAGES; ++i) {
+                    if (--rs < 0) { rs = C::RAW_STAGES - 1; rph ^= 1; }
+                    (void)mbar_wait(&raw_full[rs], rph);
                 }
             }
         }
-    } else if (warp == WARP_MMA) {
-        // ------------------------------------------------------------ MMA issuer
+    } else if (warp == C::WARP_XLOAD) {
+        // ----------------------------------------------------------- x producer
         if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0;
+            int xs = 0;
+            uint32_t xph = 0;
+            int x_issued = 0;
             bool ok = true;
-            for (int t = 0; t < my_tiles && ok; ++t) {
-                const int as = t & 1;
-                const uint32_t aph = (t >> 1) & 1;
-                if (!mbar_wait(&acc_empty[as], aph ^ 1)) { ok = false; break; }
-                tc_fence_after();
-                const uint32_t d_tmem = tmem_base + as * ACC_COLS;
-                for (int kb = 0; kb < nkb; ++kb) {
-                    if (!mbar_wait(&a_full[stage], phase) || !mbar_wait(&b_full[stage], phase)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint64_t adesc = smem_desc_sw128(sbase + OFF_A + stage * A_BYTES);
-                    const uint64_t bdesc = smem_desc_sw128(sbase + OFF_B + stage * B_BYTES);
-#pragma unroll
-                    for (int k = 0; k < BK / 16; ++k)
-                        umma_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, IDESC, (kb | k) != 0 ? 1u : 0u);
-                    umma_commit(&empty[stage]);
-                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+            while (ok && it.next(tile, r0, r1, j)) {
+                const int m_blk = tile % args.m_tiles;
+                for (int r = r0; r < r1 && ok; ++r) {
+                    for (int h = 0; h < C::KR / C::KA; ++h) {
+                        if (!mbar_wait(&x_empty[xs], xph ^ 1)) { ok = false; break; }
+                        mbar_arrive_expect_tx(&x_full[xs], C::X_BYTES);
+                        tma_load_2d(smem + C::OFF_X + xs * C::X_BYTES, &tmap_x, r * C::KR + h * C::KA, m_blk * BX,
+                                    &x_full[xs]);
+                        ++x_issued;
+                        if (++xs == C::X_STAGES) { xs = 0; xph ^= 1; }
+                    }
                 }
-                if (ok) umma_commit(&acc_full[as]);
+            }
+            if (!ok) {
+                for (int i = 0; i < x_issued && i < C::X_STAGES; ++i) {
+                    if (--xs < 0) { xs = C::X_STAGES - 1; xph ^= 1; }
+                    (void)mbar_wait(&x_full[xs], xph);
+                }
+            }
+        }
+    } else if (warp == C::WARP_MMA) {
+        // ----------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            int as = 0, xs = 0, ab = 0;
+            uint32_t aph = 0, xph = 0, abph = 0;
+            bool ok = true;
+            constexpr uint32_t idesc = idesc_bf16_f32(128, BX);
+            while (ok && it.next(tile, r0, r1, j)) {
+                if (!mbar_wait(&acc_empty[ab], abph ^ 1)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + ab * BX;
+                bool first = true;
+                for (int r = r0; r < r1 && ok; ++r) {
+                    for (int h = 0; h < C::KR / C::KA; ++h) {
+                        if (!mbar_wait(&a_full[as], aph) || !mbar_wait(&x_full[xs], xph)) { ok = false; break; }
+                        tc_fence_after();
+                        const uint64_t adesc = smem_desc_sw128(sbase + C::OFF_A + as * C::A_BYTES);
+                        const uint64_t bdesc = smem_desc_sw128(sbase + C::OFF_X + xs * C::X_BYTES);
+#pragma unroll
+                        for (int k = 0; k < C::KA / 16; ++k) {
+                            umma_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, first ? 0u : 1u);
+                            first = false;
+                        }
+                        umma_commit(&a_empty[as]);
+                        umma_commit(&x_empty[xs]);
+                        if (++as == C::A_STAGES) { as = 0; aph ^= 1; }
+                        if (++xs == C::X_STAGES) { xs = 0; xph ^= 1; }
+                    }
+                }
+                if (ok) umma_commit(&acc_full[ab]);
+                if (++ab == C::NACC) { ab = 0; abph ^= 1; }
             }
             // every MMA issued by this thread has completed once `drain` flips
             umma_commit(drain);
             (void)mbar_wait(drain, 0);
         }
-    } else if (warp < WARP_EPI0) {
-        // ------------------------------------------------------------ decoders
-        const int d = threadIdx.x - WARP_DEC0 * 32;   // weight row inside the tile
-        uint8_t *rawc = smem + OFF_RAWC;
-        uint8_t *raws = smem + OFF_RAWS;
-        const int total = my_tiles * nkb;
-        const int cw = K / 8, swd = K / 32;
-        auto issue = [&](int it) {
-            if (it < total) {
-                const int t = it / nkb, kb = it - t * nkb;
-                const int tile_id = blockIdx.x + t * gridDim.x;
-                const int n = (tile_id / num_m) * BN + d;
-                const bool rv = n < N;
-                const uint32_t *crow = args.codes + (size_t)(rv ? n : 0) * cw;
-                const uint32_t *srow = args.signs + (size_t)(rv ? n : 0) * swd;
-                const int slot = it % RD;
-                const bool full = (kb + 1) * BK <= K;   // else only the first 32 columns exist
-                uint8_t *dc = rawc + (slot * BN + d) * 32;
-                uint8_t *ds = raws + (slot * BN + d) * 8;
-                cp_async_16(dc, crow + kb * 8, rv ? 16u : 0u);
-                cp_async_16(dc + 16, crow + kb * 8 + (full ? 4 : 0), (rv && full) ? 16u : 0u);
-                cp_async_4(ds, srow + kb * 2, rv ? 4u : 0u);
-                cp_async_4(ds + 4, srow + kb * 2 + (full ? 1 : 0), (rv && full) ? 4u : 0u);
+    } else if (warp < C::WARP_EPI0) {
+        // ----------------------------------------------------------- decoders
+        // 512 threads; per 64-K stage thread t decodes weight row t / 4, 16-byte
+        // chunks 2 (t % 4) and 2 (t % 4) + 1 (16 weights), stores them swizzled.
+        const int t = threadIdx.x - C::WARP_DEC0 * 32;
+        const int row = t >> 2, cp = (t & 3) * 2;       // first of the thread's two chunks
+        const uint32_t lw = 4u * lane, lw2 = 128u + 4u * lane;
+        const uint32_t tab = sbase + C::OFF_TABLE;
+        uint32_t one = 1;
+        asm volatile("" : "+r"(one));                    // opaque 1 for add_fma
+        auto load = [&](uint32_t off) { return lds_u32(add_fma(off, tab, one)); };
+        // 64-byte swizzle of the codes stage: 16-byte chunk c of row r sits at chunk c ^ ((r >> 1) & 3)
+        const uint32_t sw64 = (uint32_t)((row >> 1) & 3);
+        const uint32_t a_off0 = (uint32_t)row * 128u + ((uint32_t)(cp ^ (row & 7)) << 4);
+        const uint32_t a_off1 = (uint32_t)row * 128u + ((uint32_t)((cp + 1) ^ (row & 7)) << 4);
+        // the decoders need only the number of 128-K blocks this CTA walks
+        int nblocks = 0;
+        while (it.next(tile, r0, r1, j)) nblocks += r1 - r0;
+        int rs = 0, as = 0;
+        uint32_t rph = 0, aph = 0;
+        // raw words of one block: codes of both 64-K halves (2 words each) and their sign words
+        auto fetch = [&](uint2 (&cw)[2], uint32_t (&sw)[2]) -> bool {
+            if (!warp_wait(&raw_full[rs], rph)) return false;
+            const uint32_t rawc = sbase + C::OFF_RAW + rs * C::RAW_BYTES + row * (C::KR / 2);
+            const uint32_t raws = sbase + C::OFF_RAW + rs * C::RAW_BYTES + C::RAW_CODE_BYTES + row * (C::KR / 8);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                // words 8h + cp, 8h + cp + 1 of the row: 16-byte chunk 2h + cp / 4, word cp % 4
+                const uint32_t chunk = ((uint32_t)(2 * h + (cp >> 2))) ^ sw64;
+                asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(cw[h].x), "=r"(cw[h].y)
+                             : "r"(rawc + (chunk << 4) + (uint32_t)(cp & 3) * 4u));
+                sw[h] = lds_u32(raws + (uint32_t)(h * 2 + (cp >> 2)) * 4u);
             }
-            cp_async_commit();
-        };
-#pragma unroll
-        for (int i = 0; i < RD - 1; ++i) issue(i);
-        int stage = 0;
-        uint32_t phase = 0;
-        for (int it = 0; it < total; ++it) {
-            issue(it + RD - 1);
-            cp_async_wait<RD - 1>();
-            const int slot = it % RD;
-            const uint4 c0 = *reinterpret_cast<const uint4 *>(rawc + (slot * BN + d) * 32);
-            const uint4 c1 = *reinterpret_cast<const uint4 *>(rawc + (slot * BN + d) * 32 + 16);
-            const uint2 sg = *reinterpret_cast<const uint2 *>(raws + (slot * BN + d) * 8);
-            if (!mbar_wait(&empty[stage], phase ^ 1)) break;
-            const uint32_t dst = sbase + OFF_B + stage * B_BYTES;
-            decode_store(c0.x, sg.x & 0xFFu, args.tab, dst + sw128_offset(d, 0));
-            decode_store(c0.y, (sg.x >> 8) & 0xFFu, args.tab, dst + sw128_offset(d, 1));
-            decode_store(c0.z, (sg.x >> 16) & 0xFFu, args.tab, dst + sw128_offset(d, 2));
-            decode_store(c0.w, sg.x >> 24, args.tab, dst + sw128_offset(d, 3));
-            decode_store(c1.x, sg.y & 0xFFu, args.tab, dst + sw128_offset(d, 4));
-            decode_store(c1.y, (sg.y >> 8) & 0xFFu, args.tab, dst + sw128_offset(d, 5));
-            decode_store(c1.z, (sg.y >> 16) & 0xFFu, args.tab, dst + sw128_offset(d, 6));
-            decode_store(c1.w, sg.y >> 24, args.tab, dst + sw128_offset(d, 7));
-            fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&b_full[stage]);
-            if (++stage == STAGES) { stage = 0; phase ^= 1; }
+            if (lane == 0) mbar_arrive(&raw_empty[rs]);   // the raw words are in registers now
+            if (++rs == C::RAW_STAGES) { rs = 0; rph ^= 1; }
+            return true;
+        };
+        uint2 ncw[2];
+        uint32_t nsw[2];
+        bool ok = nblocks > 0 ? fetch(ncw, nsw) : true;
+        for (int blk = 0; blk < nblocks && ok; ++blk) {
+            const uint2 cw0 = ncw[0], cw1 = ncw[1];
+            const uint32_t sw0 = nsw[0], sw1 = nsw[1];
+            // all 20 table lookups of this block before any store
+            uint32_t o[4][4];
+            opqbits::decode8_table(cw0.x, sw0, (uint32_t)(cp & 3), lw, lw2, load, o[0]);
+            opqbits::decode8_table(cw0.y, sw0, (uint32_t)((cp & 3) + 1), lw, lw2, load, o[1]);
+            opqbits::decode8_table(cw1.x, sw1, (uint32_t)(cp & 3), lw, lw2, load, o[2]);
+            opqbits::decode8_table(cw1.y, sw1, (uint32_t)((cp & 3) + 1), lw, lw2, load, o[3]);
+            if (blk + 1 < nblocks && !fetch(ncw, nsw)) { ok = false; break; }   // next block's raw words
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                if (!warp_wait(&a_empty[as], aph ^ 1)) { ok = false; break; }
+                const uint32_t abase = sbase + C::OFF_A + as * C::A_BYTES;
+                st_shared_v4(abase + a_off0, o[2 * h]);
+                st_shared_v4(abase + a_off1, o[2 * h + 1]);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&a_full[as]);
+                if (++as == C::A_STAGES) { as = 0; aph ^= 1; }
+            }
         }
-        cp_async_wait_all();
     } else {
-        // ------------------------------------------------------------ epilogue
-        const int q = warp & 3;                 // TMEM lane quarter of this warp
-        const bool vec_ok = (N % 8) == 0;
-        for (int t = 0; t < my_tiles; ++t) {
-            const int tile_id = blockIdx.x + t * gridDim.x;
-            const int m_blk = tile_id % num_m, n_blk = tile_id / num_m;
-            const int as = t & 1;
-            const uint32_t aph = (t >> 1) & 1;
-            if (!mbar_wait(&acc_full[as], aph)) break;
+        // ----------------------------------------------------------- epilogue
+        const int q = warp & 3;
+        const int row = q * 32 + lane;
+        const int64_t U = (int64_t)tiles * args.kblocks;
+        const bool vec_y = (args.N % 8) == 0;
+        // per-warp staging for y: 2 buffers of [16 m][32 n] bf16
+        const uint32_t stage0 = sbase + C::OFF_EPI + (uint32_t)(warp - C::WARP_EPI0) * 2048u;
+        int ab = 0;
+        uint32_t abph = 0;
+        int sb = 0;
+        while (it.next(tile, r0, r1, j)) {
+            const int n_blk = tile / args.m_tiles, m_blk = tile % args.m_tiles;
+            const int n = n_blk * C::BW + row;
+            const int n0 = n_blk * C::BW + q * 32;           // first row of this warp's quarter
+            const bool full = (r0 == 0 && r1 == args.kblocks);
+            const float scale = n < args.N ? __ldg(args.scales + n) : 0.0f;
+            if (!warp_wait(&acc_full[ab], abph)) break;
             tc_fence_after();
-            const int m = m_blk * BM + q * 32 + lane;
-            const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + as * ACC_COLS;
+            const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + ab * BX;
+            float *wsp = full ? nullptr
+                              : args.ws + ((size_t)blockIdx.x * args.runs_max + j) * (size_t)(BX * C::BW);
 #pragma unroll 1
-            for (int cc = 0; cc < BN / 32; ++cc) {
-                uint32_t r[32];
-                tmem_ld_32x32b_x32(taddr + cc * 32, r);
-                const int n0 = n_blk * BN + cc * 32;
-                // lane i holds scale[n0 + i]; shuffles broadcast it to the row owners
-                const float scl = (n0 + lane < N) ? __ldg(args.scales + n0 + lane) : 0.0f;
+            for (int c0 = 0; c0 < BX; c0 += 16) {
+                uint32_t v[16];
+                tmem_ld_32x32b_x16(taddr + c0, v);
                 tmem_ld_wait();
-                uint32_t p[16];
+                if (full) {
+                    const int m0 = m_blk * BX + c0;
+                    if (vec_y && n0 + 32 <= args.N) {
+                        // stage [16 m][32 n] bf16, then each lane stores 32 contiguous bytes of one m row
+                        const uint32_t sbuf = stage0 + (uint32_t)sb * 1024u;
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    p[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * __shfl_sync(0xFFFFFFFFu, scl, 2 * i),
-                                       __uint_as_float(r[2 * i + 1]) * __shfl_sync(0xFFFFFFFFu, scl, 2 * i + 1));
-                if (m < M && n0 < N) {
-                    uint16_t *yrow = args.y + (size_t)m * N;
-                    if (vec_ok && n0 + 32 <= N) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(yrow + n0);
+                        for (int i = 0; i < 16; ++i) {
+                            const __nv_bfloat16 o = __float2bfloat16_rn(__uint_as_float(v[i]) * scale);
+                            asm volatile("st.shared.u16 [%0], %1;" ::"r"(sbuf + (uint32_t)i * 64u + (uint32_t)lane * 2u),
+                                         "h"(*reinterpret_cast<const unsigned short *>(&o)) : "memory");
+                        }
+                        __syncwarp();
+                        const int mi = lane >> 1, hf = lane & 1;
+                        if (m0 + mi < args.M) {
+                            const uint4 w0 = lds_v4(sbuf + (uint32_t)mi * 64u + (uint32_t)hf * 32u);
+                            const uint4 w1 = lds_v4(sbuf + (uint32_t)mi * 64u + (uint32_t)hf * 32u + 16u);
+                            uint4 *dst = reinterpret_cast<uint4 *>(args.y + (size_t)(m0 + mi) * args.N + n0 + hf * 16);
+                            dst[0] = w0;
+                            dst[1] = w1;
+                        }
+                        sb ^= 1;
+                    } else if (n < args.N) {
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) dst[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            if (n0 + i < N) yrow[n0 + i] = (uint16_t)((p[i / 2] >> (16 * (i & 1))) & 0xFFFFu);
+                        for (int i = 0; i < 16; ++i) {
+                            const int m = m0 + i;
+                            if (m < args.M) {
+                                const __nv_bfloat16 o = __float2bfloat16_rn(__uint_as_float(v[i]) * scale);
+                                args.y[(size_t)m * args.N + n] = *reinterpret_cast<const uint16_t *>(&o);
+                            }
+                        }
                     }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) wsp[(size_t)(c0 + i) * C::BW + row] = __uint_as_float(v[i]);
                 }
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[as]);
-        }
-    }
-
-    tc_fence_before();
-    __syncthreads();
-    if (warp == WARP_MMA) {
-        tc_fence_after();
-        tmem_dealloc(tmem_base, TMEM_COLS);
-    }
-}
-
-// ============================================================================
-// Weight-streaming split-K kernel (path 1)
-// ============================================================================
-namespace stream {
-constexpr int BW = 128, BK = 64;            // weight rows per CTA (MMA M), K per stage
-constexpr int STAGES = 4;
-constexpr int RD = 4;
-constexpr int A_BYTES = BW * BK * 2;        // 16 KiB decoded weights per stage
-constexpr int DEC_THREADS = 256;            // two threads per weight row (32 columns each)
-constexpr int WARP_TMA = 0, WARP_MMA = 1, WARP_DEC0 = 2;
-constexpr int THREADS = (WARP_DEC0 + DEC_THREADS / 32) * 32;  // 320
-constexpr int RAW_CODE_BYTES = RD * DEC_THREADS * 16;
-constexpr int RAW_SIGN_BYTES = RD * DEC_THREADS * 4;
-__host__ __device__ constexpr int b_bytes(int bx) { return bx * BK * 2; }
-__host__ __device__ constexpr int off_b() { return STAGES * A_BYTES; }
-__host__ __device__ constexpr int off_rawc(int bx) { return off_b() + STAGES * b_bytes(bx); }
-__host__ __device__ constexpr int off_raws(int bx) { return off_rawc(bx) + RAW_CODE_BYTES; }
-__host__ __device__ constexpr int off_bar(int bx) { return off_raws(bx) + RAW_SIGN_BYTES; }
-constexpr int NUM_BARS = 3 * STAGES + 1 + 1;  // a_full(x), b_full(decoded), empty, acc_full, drain
-__host__ __device__ constexpr int off_tmem(int bx) { return off_bar(bx) + NUM_BARS * 8; }
-__host__ __device__ constexpr int smem_bytes(int bx) { return off_tmem(bx) + 16 + 1024; }
-__host__ __device__ constexpr uint32_t tmem_cols(int bx) {
-    return bx <= 32 ? 32u : bx <= 64 ? 64u : bx <= 128 ? 128u : 256u;
-}
-}  // namespace stream
-
-__global__ void __launch_bounds__(stream::THREADS)
-    linear_stream_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ LinearArgs args) {
-    using namespace stream;
-    extern __shared__ uint8_t smem_raw[];
-    const uint32_t raw_base = smem_u32(smem_raw);
-    const uint32_t pad = ((raw_base + 1023u) & ~1023u) - raw_base;
-    uint8_t *smem = smem_raw + pad;
-    const uint32_t sbase = raw_base + pad;
-    const int bx = args.bx;
-    const int BX_BYTES = b_bytes(bx);
-
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + off_bar(bx));
-    uint64_t *x_full = bars;
-    uint64_t *w_full = bars + STAGES;
-    uint64_t *empty = bars + 2 * STAGES;
-    uint64_t *acc_full = bars + 3 * STAGES;
-    uint64_t *drain = acc_full + 1;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + off_tmem(bx));
-
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int M = args.M, N = args.N, K = args.K;
-    const int nkb_total = (K + BK - 1) / BK;
-    const int split = blockIdx.y;
-    const int kb_per = (nkb_total + args.splits - 1) / args.splits;
-    const int kb_begin = split * kb_per;
-    const int kb_end = min(nkb_total, kb_begin + kb_per);
-    const int nkb = max(0, kb_end - kb_begin);
-    const int n_base = blockIdx.x * BW;
-    const uint32_t ncols = tmem_cols(bx);
-
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&x_full[s], 1);
-            mbar_init(&w_full[s], DEC_THREADS / 32);
-            mbar_init(&empty[s], 1);
-        }
-        mbar_init(acc_full, 1);
-        mbar_init(drain, 1);
-        fence_mbar_init();
-    }
-    if (warp == WARP_TMA && lane == 0) tma_prefetch_desc(&tmap_x);
-    if (warp == WARP_MMA) {
-        tmem_alloc(tmem_slot, ncols);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem_base = *tmem_slot;
-
-    if (warp == WARP_TMA) {
-        if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0;
-            int armed = 0;
-            bool ok = true;
-            for (int i = 0; i < nkb; ++i) {
-                if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
-                mbar_arrive_expect_tx(&x_full[stage], BX_BYTES);
-                tma_load_2d(smem + off_b() + stage * BX_BYTES, &tmap_x, (kb_begin + i) * BK, 0, &x_full[stage]);
-                armed = armed < STAGES ? armed + 1 : STAGES;
-                if (++stage == STAGES) { stage = 0; phase ^= 1; }
-            }
-            if (!ok) {
-                for (int i = 0; i < armed; ++i) {
-                    if (--stage < 0) { stage = STAGES - 1; phase ^= 1; }
-                    (void)mbar_wait(&x_full[stage], phase);
-                }
-            }
-        }
-    } else if (warp == WARP_MMA) {
-        if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0;
-            bool ok = true;
-            const uint32_t idesc = idesc_bf16_f32(BW, bx);
-            for (int i = 0; i < nkb; ++i) {
-                if (!mbar_wait(&w_full[stage], phase) || !mbar_wait(&x_full[stage], phase)) { ok = false; break; }
-                tc_fence_after();
-                const uint64_t adesc = smem_desc_sw128(sbase + stage * A_BYTES);
-                const uint64_t bdesc = smem_desc_sw128(sbase + off_b() + stage * BX_BYTES);
-#pragma unroll
-                for (int k = 0; k < BK / 16; ++k)
-                    umma_bf16(tmem_base, adesc + 2 * k, bdesc + 2 * k, idesc, (i | k) != 0 ? 1u : 0u);
-                umma_commit(&empty[stage]);
-                if (++stage == STAGES) { stage = 0; phase ^= 1; }
-            }
-            if (ok) umma_commit(acc_full);
-            umma_commit(drain);
-            (void)mbar_wait(drain, 0);
-        }
-    } else {
-        // ---------------------------------------------------- decoders, then epilogue
-        const int d = threadIdx.x - WARP_DEC0 * 32;
-        const int r = d >> 1, h = d & 1;          // weight row, column half (32 of 64)
-        const int n = n_base + r;
-        const bool rv = n < N;
-        const int cw = K / 8, swd = K / 32;
-        const uint32_t *crow = args.codes + (size_t)(rv ? n : 0) * cw;
-        const uint32_t *srow = args.signs + (size_t)(rv ? n : 0) * swd;
-        uint8_t *rawc = smem + off_rawc(bx);
-        uint8_t *raws = smem + off_raws(bx);
-        auto issue = [&](int i) {
-            if (i < nkb) {
-                const int kb = kb_begin + i;
-                const bool present = rv && (kb * BK + h * 32) < K;
-                const int slot = i % RD;
-                cp_async_16(rawc + (slot * DEC_THREADS + d) * 16, crow + (present ? kb * 8 + h * 4 : 0),
-                            present ? 16u : 0u);
-                cp_async_4(raws + (slot * DEC_THREADS + d) * 4, srow + (present ? kb * 2 + h : 0),
-                           present ? 4u : 0u);
-            }
-            cp_async_commit();
-        };
-#pragma unroll
-        for (int i = 0; i < RD - 1; ++i) issue(i);
-        int stage = 0;
-        uint32_t phase = 0;
-        bool ok = true;
-        for (int i = 0; i < nkb; ++i) {
-            issue(i + RD - 1);
-            cp_async_wait<RD - 1>();
-            const int slot = i % RD;
-            const uint4 c = *reinterpret_cast<const uint4 *>(rawc + (slot * DEC_THREADS + d) * 16);
-            const uint32_t sg = *reinterpret_cast<const uint32_t *>(raws + (slot * DEC_THREADS + d) * 4);
-            if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
-            const uint32_t dst = sbase + stage * A_BYTES;
-            decode_store(c.x, sg & 0xFFu, args.tab, dst + sw128_offset(r, 4 * h + 0));
-            decode_store(c.y, (sg >> 8) & 0xFFu, args.tab, dst + sw128_offset(r, 4 * h + 1));
-            decode_store(c.z, (sg >> 16) & 0xFFu, args.tab, dst + sw128_offset(r, 4 * h + 2));
-            decode_store(c.w, sg >> 24, args.tab, dst + sw128_offset(r, 4 * h + 3));
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&w_full[stage]);
-            if (++stage == STAGES) { stage = 0; phase ^= 1; }
-        }
-        cp_async_wait_all();
-
-        // epilogue: warps 2..5 hold TMEM lane quarters 2, 3, 0, 1
-        if (ok && warp < WARP_DEC0 + 4 && nkb > 0) {
-            const int q = warp & 3;
-            const int row = q * 32 + lane;
-            const int nn = n_base + row;
-            if (mbar_wait(acc_full, 0)) {
-                tc_fence_after();
-                const float scale = (nn < N) ? __ldg(args.scales + nn) : 0.0f;
-                const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16);
-                for (int c0 = 0; c0 < bx; c0 += 8) {
-                    uint32_t v[8];
-                    tmem_ld_32x32b_x8(taddr + c0, v);
-                    tmem_ld_wait();
-                    if (nn < N) {
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            const int m = c0 + j;
-                            if (m < M) {
-                                const float acc = __uint_as_float(v[j]);
-                                if (args.splits == 1) {
-                                    const __nv_bfloat16 o = __float2bfloat16_rn(acc * scale);
-                                    args.y[(size_t)m * N + nn] = *reinterpret_cast<const uint16_t *>(&o);
-                                } else {
-                                    args.ws[((size_t)split * M + m) * N + nn] = acc;
-                                }
+            if (lane == 0) mbar_arrive(&acc_empty[ab]);
+            if (++ab == C::NACC) { ab = 0; abph ^= 1; }
+            if (!full) {
+                // The last of the tile's CTAs to get here (per lane quarter) adds every
+                // CTA's partial rows in CTA order, so the sum does not depend on timing.
+                const int64_t c_lo = unit_owner((int64_t)tile * args.kblocks, gridDim.x, U);
+                const int64_t c_hi = unit_owner((int64_t)(tile + 1) * args.kblocks - 1, gridDim.x, U);
+                const uint32_t parts = (uint32_t)(c_hi - c_lo + 1);
+                __threadfence();
+                __syncwarp();
+                uint32_t old = 0;
+                if (lane == 0) old = atomicAdd(args.counters + (size_t)tile * 4 + q, 1u);
+                old = __shfl_sync(0xFFFFFFFFu, old, 0);
+                if (old == parts - 1) {
+                    __threadfence();
+                    // lane i (< parts) resolves part i's base; bases are broadcast by shuffles
+                    const float *mybase = nullptr;
+                    if ((uint32_t)lane < parts) {
+                        const int64_t c = c_lo + lane;
+                        const int64_t jj = tile - unit_begin(c, gridDim.x, U) / args.kblocks;
+                        mybase = args.ws + ((size_t)c * args.runs_max + (size_t)jj) * (size_t)(BX * C::BW);
+                    }
+                    // every lane runs the loops (shuffles need all lanes); only rows < N store
+                    for (int col = 0; col < BX; ++col) {
+                        const int m = m_blk * BX + col;
+                        if (m >= args.M) break;
+                        float acc = 0.0f;
+                        for (uint32_t p = 0; p < parts; ++p) {
+                            const float *base;
+                            if (p < 32) {
+                                base = reinterpret_cast<const float *>(
+                                    __shfl_sync(0xFFFFFFFFu, reinterpret_cast<unsigned long long>(mybase), (int)p));
+                            } else {
+                                const int64_t c = c_lo + p;
+                                const int64_t jj = tile - unit_begin(c, gridDim.x, U) / args.kblocks;
+                                base = args.ws + ((size_t)c * args.runs_max + (size_t)jj) * (size_t)(BX * C::BW);
                             }
+                            acc += __ldcg(base + (size_t)col * C::BW + row);
+                        }
+                        if (n < args.N) {
+                            const __nv_bfloat16 o = __float2bfloat16_rn(acc * scale);
+                            args.y[(size_t)m * args.N + n] = *reinterpret_cast<const uint16_t *>(&o);
                         }
                     }
+                    if (lane == 0) atomicExch(args.counters + (size_t)tile * 4 + q, 0u);   // ready for the next call
                 }
             }
-        } else if (nkb == 0 && warp < WARP_DEC0 + 4 && args.splits > 1) {
-            // an empty K slice still owns its partial-sum rows: write zeros
-            const int q = warp & 3;
-            const int nn = n_base + q * 32 + lane;
-            if (nn < N)
-                for (int m = 0; m < M; ++m) args.ws[((size_t)split * M + m) * N + nn] = 0.0f;
         }
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == WARP_MMA) {
+    if (warp == C::WARP_MMA) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, ncols);
-    }
-}
-
-// y[m, n] = bf16(scale[n] * sum_{s = 0..splits-1} ws[s, m, n]), summed in order s = 0, 1, ...
-__global__ void __launch_bounds__(256) splitk_reduce_kernel(const float *__restrict__ ws,
-                                                            const float *__restrict__ scales, int M, int N,
-                                                            int splits, uint16_t *__restrict__ y) {
-    const size_t total = (size_t)M * N;
-    const size_t plane = total;
-    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
-        float acc = ws[i];
-        for (int s = 1; s < splits; ++s) acc += ws[(size_t)s * plane + i];
-        const int n = (int)(i % (size_t)N);
-        const __nv_bfloat16 o = __float2bfloat16_rn(acc * __ldg(scales + n));
-        y[i] = *reinterpret_cast<const uint16_t *>(&o);
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
     }
 }
 

@@ -98,9 +98,11 @@ opq_status opq_linear_workspace_size(int64_t M, int64_t N, int64_t K, size_t *by
  *   alpha      the power used to quantize
  *   y          bf16 [M, N] device, row-major (leading dimension N), written
  *   workspace  device scratch of at least opq_linear_workspace_size(M, N, K) bytes
- *              (may be NULL when that size is 0); its contents need no initialisation
- *              and are garbage afterwards; calls sharing one workspace must not
- *              overlap on the GPU
+ *              (may be NULL when that size is 0). It must be zero-filled before its
+ *              first use (e.g. one cudaMemset after allocation); every completed call
+ *              leaves it valid for the next one (its leading arrival counters back at
+ *              zero), for any shape. Calls sharing one workspace must not overlap on
+ *              the GPU.
  * Arithmetic: each decoded weight sign * bf16((q/15)^(1/alpha)) enters a bf16
  * tensor-core product with fp32 accumulation; the row scale is applied to the
  * fp32 sum, which is then rounded once to bf16. Deterministic: the same inputs
@@ -111,14 +113,16 @@ opq_status opq_linear(const uint16_t *x, int64_t M, int64_t K, const uint32_t *c
                       uint16_t *y, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
- * opq_linear_plan — the kernel opq_linear would use for this shape:
- *   *path      0 = tile kernel (x rows on the MMA M side), 1 = weight-streaming split-K
- *              kernel (weight rows on the MMA M side) followed by a fixed-order reduce
- *   *splits    number of K slices (1 when not split)
+ * opq_linear_plan — the schedule opq_linear uses for this shape (it depends on the
+ * shape alone, so workspace sizes and result bits do not vary between B200s):
+ *   *path      0 = whole 128-weight-row x 256-activation-row tiles, one persistent CTA
+ *              per SM; 1 = stream-K: the (tile, 128-K block) sequence cut into one
+ *              contiguous range per CTA, followed by a fixed-order fix-up kernel
+ *   *ctas      CTAs of the main kernel
  *   *launches  kernels launched per opq_linear call
  * Any output pointer may be NULL.
  */
-opq_status opq_linear_plan(int64_t M, int64_t N, int64_t K, int *path, int *splits, int *launches);
+opq_status opq_linear_plan(int64_t M, int64_t N, int64_t K, int *path, int *ctas, int *launches);
 
 /*
  * opq_linear_noalloc — opq_linear without a caller-provided workspace. The paper
@@ -135,10 +139,11 @@ opq_status opq_linear_plan(int64_t M, int64_t N, int64_t K, int *path, int *spli
  *   - The first call on a device looks up the array's device address on that
  *     device (cudaGetSymbolAddress, with that device current); make that first
  *     call before any stream capture on the device.
- *   - All calls share the one array and it keeps the last call's contents. The
- *     kernels write every partial sum they later read, so nothing needs clearing,
- *     but calls that overlap on the GPU (different streams, or different host
- *     threads without ordering) race on the array and give wrong results.
+ *   - All calls share the one array and it keeps the last call's contents. Its
+ *     leading arrival counters must be zero when a call starts: the array is zero
+ *     when the library loads and every completed call leaves them at zero again.
+ *     Calls that overlap on the GPU (different streams, or different host threads
+ *     without ordering) race on the array and give wrong results.
  *   - No device memory is allocated or freed by this call.
  */
 #define OPQ_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)

@@ -5,6 +5,7 @@
 #include <cstdint>
 #include <random>
 #include <algorithm>
+#include <vector>
 #include "opq_bits.h"
 
 using namespace opqbits;
@@ -77,6 +78,40 @@ int main() {
                 uint32_t want = lut[q] | (((sb >> i) & 1u) << 15);
                 uint32_t got = (out[i / 2] >> (16 * (i % 2))) & 0xFFFFu;
                 CHECK(got == want, "decode8 c %x sb %x i %d got %x want %x", c, sb, i, got, want);
+            }
+        }
+    }
+    // --- pair-table decode: build the 64 KiB table exactly as the kernels lay it out
+    {
+        std::vector<uint32_t> table(kPairTableBytes / 4);
+        for (int trial = 0; trial < 50; ++trial) {
+            uint16_t lut[16];
+            for (int q = 0; q < 16; ++q) lut[q] = (uint16_t)(rng() & 0x7FFFu);
+            if (trial == 0) lut[0] = 0;
+            for (uint32_t b = 0; b < 256; ++b)
+                for (uint32_t r = 0; r < 32; ++r) {
+                    table[(b * 256 + 4 * r) / 4] = pair_value(b, lut);
+                    table[(b * 256 + 128 + 4 * r) / 4] = sign_spread(b);
+                }
+            for (int rep = 0; rep < 20000; ++rep) {
+                const uint32_t lane = (uint32_t)(rng() & 31u);
+                const uint32_t lw = 4 * lane, lw2 = 128 + 4 * lane;
+                uint32_t c = (uint32_t)rng(), sw = (uint32_t)rng(), j = (uint32_t)(rng() & 3u);
+                uint32_t out[4];
+                bool lane_ok = true;
+                auto load = [&](uint32_t off) -> uint32_t {
+                    if (off >= kPairTableBytes || (off & 3u) || ((off % 128u) / 4u) != lane) lane_ok = false;
+                    return table[(off % kPairTableBytes) / 4];
+                };
+                decode8_table(c, sw, j, lw, lw2, load, out);
+                CHECK(lane_ok, "table offset outside the lane's copy");
+                const uint32_t sb = (sw >> (8 * j)) & 0xFFu;
+                for (int i = 0; i < 8; ++i) {
+                    uint32_t q = (c >> (4 * i)) & 15u;
+                    uint32_t want = lut[q] | (((sb >> i) & 1u) << 15);
+                    uint32_t got = (out[i / 2] >> (16 * (i % 2))) & 0xFFFFu;
+                    CHECK(got == want, "decode8_table c %x sw %x j %u i %d got %x want %x", c, sw, j, i, got, want);
+                }
             }
         }
     }

@@ -90,19 +90,24 @@ def test_dequantize_and_linear_argument_errors(lib):
 
 
 def test_plan_and_workspace_host_logic(lib):
-    # weight streaming for small M, split so that ~2 CTAs per SM exist, no empty slice
-    for M, N, K in [(1, 11520, 3840), (16, 11520, 3840), (64, 11520, 3840), (256, 11520, 3840),
+    # small M: stream-K over (128-row weight tile, 128-K block) units on at most 148 CTAs
+    for M, N, K in [(1, 11520, 3840), (16, 11520, 3840), (64, 11520, 3840), (128, 11520, 3840),
                     (1, 3840, 3840), (17, 257, 96), (1, 64, 32)]:
-        path, splits, launches = opq.plan(M, N, K)
-        assert path == 1
-        nkb = -(-K // 64)
-        per = -(-nkb // splits)
-        assert (splits - 1) * per < nkb <= splits * per
-        assert launches == (2 if splits > 1 else 1)
-        ws = opq.workspace_size(M, N, K)
-        assert ws == (splits * M * N * 4 if splits > 1 else 0)
-    assert opq.plan(3072, 3840, 3840) == (0, 1, 1)
-    assert opq.workspace_size(3072, 3840, 3840) == 0
+        path, ctas, launches = opq.plan(M, N, K)
+        assert path == 1 and launches == 1
+        bx = 16 if M <= 16 else 32 if M <= 32 else 64 if M <= 64 else 128
+        units = -(-N // 128) * -(-K // 128)
+        assert ctas == min(148, units)
+        per = -(-units // ctas)
+        runs_max = -(-per // -(-K // 128)) + 1
+        counters = 4096 * 4 * 4        # fixed region: 4 arrival counters for each of up to 4096 weight tiles
+        assert opq.workspace_size(M, N, K) == counters + ctas * runs_max * bx * 128 * 4
+    # large M: whole 128 x 256 tiles, one persistent CTA per SM, no workspace
+    for M, N, K in [(129, 100, 32), (3072, 3840, 3840), (4096, 10240, 3840), (8, 4097 * 128, 64)]:
+        path, ctas, launches = opq.plan(M, N, K)
+        assert path == 0 and launches == 1
+        assert ctas == min(148, -(-M // 256) * -(-N // 128))
+        assert opq.workspace_size(M, N, K) == 0
     sz = ctypes.c_size_t(0)
     assert lib.opq_linear_workspace_size(0, 4, 32, ctypes.byref(sz)) == 1
     assert lib.opq_linear_workspace_size(4, 4, 40, ctypes.byref(sz)) == 2

@@ -261,3 +261,22 @@ def test_full_whole_model_sampled_layers():
         x, w = lin.make("cpu")
         quant_parity(w.to(DEV), lin.alpha, rows=np.arange(0, lin.N, 13))
         linear_parity(x, w, lin.alpha, pairs=800)
+
+
+def test_linear_workspace_reuse_across_shapes():
+    """One zero-filled workspace serves calls of different shapes in a row: every
+    call leaves its arrival counters at zero for the next one."""
+    shapes = [(16, 11520, 3840), (64, 2048, 1024), (1, 3840, 3840), (16, 11520, 3840), (128, 640, 4096)]
+    need = max(opq.workspace_size(*s) for s in shapes)
+    ws = torch.zeros((need,), dtype=torch.uint8, device=DEV)
+    for i, (M, N, K) in enumerate(shapes):
+        lin = workloads.Linear("reuse", M, N, K, w_seed=31 + i, x_seed=37 + i)
+        x, w = lin.make(DEV)
+        planes = opq.quantize(w)
+        y_shared = opq.linear(x, *planes, workspace=ws)
+        y_fresh = opq.linear(x, *planes)
+        assert torch.equal(y_shared, y_fresh), (M, N, K)
+    torch.cuda.synchronize()
+    counters = ws[: 4096 * 4 * 4].view(torch.int32)
+    assert int(counters.abs().sum()) == 0
+    assert opq.device_error() == 0
