@@ -177,34 +177,41 @@ template <int BX>
 struct Cfg {
     static constexpr int BW = 128;                     // weight rows per tile (MMA M)
     static constexpr int KR = 128;                     // K per raw (codes/signs) stage
-    static constexpr int KA = 64;                      // K per A / x stage
-    static constexpr int RAW_STAGES = BX >= 256 ? 3 : (BX <= 16 ? 6 : 4);
-    static constexpr int A_STAGES = BX >= 256 ? 3 : 4;
-    static constexpr int X_STAGES = BX >= 256 ? 2 : (BX >= 128 ? 3 : (BX >= 64 ? 6 : 10));
-    static constexpr int NACC = 2;                     // accumulators in TMEM, double-buffered
-    static constexpr uint32_t TMEM_COLS = (2 * BX <= 32) ? 32 : (2 * BX <= 64) ? 64 : (2 * BX <= 128) ? 128
-                                                           : (2 * BX <= 256) ? 256 : 512;
+    static constexpr int KA = 64;                      // K per A stage (TMEM) and per x stage (smem)
+    static constexpr int RAW_STAGES = BX >= 256 ? 3 : 6;
+    static constexpr int A_STAGES = 8;                 // 32 TMEM columns each (64 K of bf16 pairs)
+    static constexpr int A_COLS = A_STAGES * 32;
+    static constexpr int X_STAGES = BX >= 256 ? 3 : (BX >= 128 ? 4 : (BX >= 64 ? 6 : 10));
+    // independent accumulation chains per tile: consecutive MMAs into one accumulator
+    // serialize on its latency, which dominates when N (= BX) is small; K-step k of a
+    // stage goes to chain k % NCHAIN and the epilogue adds the chains in a fixed order
+    static constexpr int NCHAIN = BX <= 32 ? 4 : (BX <= 64 ? 2 : 1);
+    static constexpr int ACC_COLS = NCHAIN * BX;       // one accumulator buffer (all chains)
+    static constexpr int NACC = (A_COLS + 2 * ACC_COLS <= 512) ? 2 : 1;   // accumulator buffers
+    static constexpr uint32_t TMEM_COLS = 512;
     static constexpr int RAW_CODE_BYTES = BW * KR / 2;    // 8 KiB: [128 rows][16 words], 64-byte swizzle
     static constexpr int RAW_SIGN_BYTES = BW * KR / 8;    // 2 KiB: [128 rows][4 words]
     static constexpr int RAW_BYTES = RAW_CODE_BYTES + RAW_SIGN_BYTES;
-    static constexpr int A_BYTES = BW * KA * 2;           // 16 KiB decoded W', 128-byte swizzle, K-major
     static constexpr int X_BYTES = BX * KA * 2;
     static constexpr int STAGE_EPI_BYTES = 4 * 2 * 16 * 32 * 2;   // 4 warps x 2 buffers x [16 m][32 n] bf16
     static constexpr int OFF_TABLE = 0;
     static constexpr int OFF_RAW = OFF_TABLE + (int)opqbits::kPairTableBytes;
-    static constexpr int OFF_A = OFF_RAW + RAW_STAGES * RAW_BYTES;
-    static constexpr int OFF_X = OFF_A + A_STAGES * A_BYTES;
+    static constexpr int OFF_X = OFF_RAW + RAW_STAGES * RAW_BYTES;
     static constexpr int OFF_EPI = OFF_X + X_STAGES * X_BYTES;
     static constexpr int OFF_BAR = OFF_EPI + STAGE_EPI_BYTES;
     static constexpr int NUM_BARS = 2 * RAW_STAGES + 2 * X_STAGES + 2 * A_STAGES + 2 * NACC + 1;
     static constexpr int OFF_TMEM = OFF_BAR + NUM_BARS * 8;
     static constexpr int SMEM_BYTES = OFF_TMEM + 16 + 1024;
-    static constexpr int WARP_LOAD = 0, WARP_MMA = 1, WARP_XLOAD = 2, WARP_DEC0 = 3, NUM_DEC_WARPS = 16;
+    // decoder groups of 4 warps: group g decodes the CTA's 128-K blocks g, g + G, ...;
+    // thread r of a group owns weight row r (TMEM lane r) and decodes its whole 128-K block row
+    static constexpr int GROUPS = 3;
+    static constexpr int WARP_LOAD = 0, WARP_MMA = 1, WARP_XLOAD = 2, WARP_DEC0 = 3, NUM_DEC_WARPS = 4 * GROUPS;
     static constexpr int WARP_EPI0 = WARP_DEC0 + NUM_DEC_WARPS;
     static constexpr int THREADS = (WARP_EPI0 + 4) * 32;
     static_assert(SMEM_BYTES <= 232448, "shared memory");
     static_assert(BX % 16 == 0 && BX >= 16 && BX <= 256, "MMA N");
-    static_assert(RAW_BYTES % 1024 == 0 && A_BYTES % 1024 == 0 && X_BYTES % 1024 == 0, "stage alignment");
+    static_assert(A_COLS + NACC * ACC_COLS <= 512, "TMEM columns");
+    static_assert(RAW_BYTES % 1024 == 0 && X_BYTES % 1024 == 0, "stage alignment");
 };
 
 template <int BX>
@@ -248,14 +255,14 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
         for (int s = 0; s < C::RAW_STAGES; ++s) {
             // the codes' (and signs') expect_tx arrival, plus 32 cp.async arrivals when signs are copied by threads
             mbar_init(&raw_full[s], signs_by_tma ? 1 : 1 + 32);
-            mbar_init(&raw_empty[s], C::NUM_DEC_WARPS);
+            mbar_init(&raw_empty[s], 4);          // the 4 warps of the group that decodes the block
         }
         for (int s = 0; s < C::X_STAGES; ++s) {
             mbar_init(&x_full[s], 1);
             mbar_init(&x_empty[s], 1);
         }
         for (int s = 0; s < C::A_STAGES; ++s) {
-            mbar_init(&a_full[s], C::NUM_DEC_WARPS);
+            mbar_init(&a_full[s], 4);             // the 4 warps of the decoding group
             mbar_init(&a_empty[s], 1);
         }
         for (int s = 0; s < C::NACC; ++s) {
@@ -373,18 +380,20 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
             while (ok && it.next(tile, r0, r1, j)) {
                 if (!mbar_wait(&acc_empty[ab], abph ^ 1)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + ab * BX;
-                bool first = true;
+                const uint32_t d_tmem = tmem_base + C::A_COLS + ab * C::ACC_COLS;
+                uint32_t fresh = (1u << C::NCHAIN) - 1u;  // chains not yet written in this run
                 for (int r = r0; r < r1 && ok; ++r) {
                     for (int h = 0; h < C::KR / C::KA; ++h) {
                         if (!mbar_wait(&a_full[as], aph) || !mbar_wait(&x_full[xs], xph)) { ok = false; break; }
                         tc_fence_after();
-                        const uint64_t adesc = smem_desc_sw128(sbase + C::OFF_A + as * C::A_BYTES);
+                        const uint32_t a_tmem = tmem_base + as * 32;
                         const uint64_t bdesc = smem_desc_sw128(sbase + C::OFF_X + xs * C::X_BYTES);
 #pragma unroll
                         for (int k = 0; k < C::KA / 16; ++k) {
-                            umma_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, first ? 0u : 1u);
-                            first = false;
+                            const int ch = k % C::NCHAIN;
+                            umma_bf16_ts(d_tmem + ch * BX, a_tmem + 8 * k, bdesc + 2 * k, idesc,
+                                         ((fresh >> ch) & 1u) ? 0u : 1u);
+                            fresh &= ~(1u << ch);
                         }
                         umma_commit(&a_empty[as]);
                         umma_commit(&x_empty[xs]);
@@ -401,65 +410,56 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
         }
     } else if (warp < C::WARP_EPI0) {
         // ----------------------------------------------------------- decoders
-        // 512 threads; per 64-K stage thread t decodes weight row t / 4, 16-byte
-        // chunks 2 (t % 4) and 2 (t % 4) + 1 (16 weights), stores them swizzled.
-        const int t = threadIdx.x - C::WARP_DEC0 * 32;
-        const int row = t >> 2, cp = (t & 3) * 2;       // first of the thread's two chunks
+        const int g = (warp - C::WARP_DEC0) >> 2;        // decoder group
+        const int q = warp & 3;                          // TMEM lane quarter this warp may access
+        const int row = q * 32 + lane;                   // weight row in the tile = TMEM lane
         const uint32_t lw = 4u * lane, lw2 = 128u + 4u * lane;
-        const uint32_t tab = sbase + C::OFF_TABLE;
-        uint32_t one = 1;
-        asm volatile("" : "+r"(one));                    // opaque 1 for add_fma
-        auto load = [&](uint32_t off) { return lds_u32(add_fma(off, tab, one)); };
+        const uint32_t *tabp = reinterpret_cast<const uint32_t *>(smem + C::OFF_TABLE);
+        auto load = [&](uint32_t off) { return tabp[off >> 2]; };
         // 64-byte swizzle of the codes stage: 16-byte chunk c of row r sits at chunk c ^ ((r >> 1) & 3)
         const uint32_t sw64 = (uint32_t)((row >> 1) & 3);
-        const uint32_t a_off0 = (uint32_t)row * 128u + ((uint32_t)(cp ^ (row & 7)) << 4);
-        const uint32_t a_off1 = (uint32_t)row * 128u + ((uint32_t)((cp + 1) ^ (row & 7)) << 4);
-        // the decoders need only the number of 128-K blocks this CTA walks
+        const uint32_t tm_row = tmem_base + ((uint32_t)(q * 32) << 16);
         int nblocks = 0;
         while (it.next(tile, r0, r1, j)) nblocks += r1 - r0;
-        int rs = 0, as = 0;
-        uint32_t rph = 0, aph = 0;
-        // raw words of one block: codes of both 64-K halves (2 words each) and their sign words
-        auto fetch = [&](uint2 (&cw)[2], uint32_t (&sw)[2]) -> bool {
-            if (!warp_wait(&raw_full[rs], rph)) return false;
-            const uint32_t rawc = sbase + C::OFF_RAW + rs * C::RAW_BYTES + row * (C::KR / 2);
-            const uint32_t raws = sbase + C::OFF_RAW + rs * C::RAW_BYTES + C::RAW_CODE_BYTES + row * (C::KR / 8);
+        bool ok = true;
+        for (int blk = g; blk < nblocks && ok; blk += C::GROUPS) {
+            const int rs = blk % C::RAW_STAGES;
+            const uint32_t rph = (uint32_t)(blk / C::RAW_STAGES) & 1u;
+            if (!warp_wait(&raw_full[rs], rph)) { ok = false; break; }
+            const uint8_t *rawc = smem + C::OFF_RAW + rs * C::RAW_BYTES + row * (C::KR / 2);
+            uint32_t cw[16];
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                // words 8h + cp, 8h + cp + 1 of the row: 16-byte chunk 2h + cp / 4, word cp % 4
-                const uint32_t chunk = ((uint32_t)(2 * h + (cp >> 2))) ^ sw64;
-                asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(cw[h].x), "=r"(cw[h].y)
-                             : "r"(rawc + (chunk << 4) + (uint32_t)(cp & 3) * 4u));
-                sw[h] = lds_u32(raws + (uint32_t)(h * 2 + (cp >> 2)) * 4u);
+            for (int c = 0; c < 4; ++c) {
+                const uint4 v = *reinterpret_cast<const uint4 *>(rawc + ((((uint32_t)c) ^ sw64) << 4));
+                cw[4 * c] = v.x; cw[4 * c + 1] = v.y; cw[4 * c + 2] = v.z; cw[4 * c + 3] = v.w;
             }
+            const uint4 sv = *reinterpret_cast<const uint4 *>(smem + C::OFF_RAW + rs * C::RAW_BYTES + C::RAW_CODE_BYTES +
+                                                             row * (C::KR / 8));
+            const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
             __syncwarp();
             if (lane == 0) mbar_arrive(&raw_empty[rs]);   // the raw words are in registers now
-            if (++rs == C::RAW_STAGES) { rs = 0; rph ^= 1; }
-            return true;
-        };
-        uint2 ncw[2];
-        uint32_t nsw[2];
-        bool ok = nblocks > 0 ? fetch(ncw, nsw) : true;
-        for (int blk = 0; blk < nblocks && ok; ++blk) {
-            const uint2 cw0 = ncw[0], cw1 = ncw[1];
-            const uint32_t sw0 = nsw[0], sw1 = nsw[1];
-            // all 20 table lookups of this block before any store
-            uint32_t o[4][4];
-            opqbits::decode8_table(cw0.x, sw0, (uint32_t)(cp & 3), lw, lw2, load, o[0]);
-            opqbits::decode8_table(cw0.y, sw0, (uint32_t)((cp & 3) + 1), lw, lw2, load, o[1]);
-            opqbits::decode8_table(cw1.x, sw1, (uint32_t)(cp & 3), lw, lw2, load, o[2]);
-            opqbits::decode8_table(cw1.y, sw1, (uint32_t)((cp & 3) + 1), lw, lw2, load, o[3]);
-            if (blk + 1 < nblocks && !fetch(ncw, nsw)) { ok = false; break; }   // next block's raw words
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
+            for (int h = 0; h < C::KR / C::KA; ++h) {     // two 64-K A stages per block
+                const int sidx = blk * 2 + h;
+                const int as = sidx % C::A_STAGES;
+                const uint32_t aph = (uint32_t)(sidx / C::A_STAGES) & 1u;
+                uint32_t o[2][16];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int w = 8 * h + i;
+                    uint32_t t4[4];
+                    opqbits::decode8_table(cw[w], sw[w >> 2], (uint32_t)(w & 3), lw, lw2, load, t4);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) o[i >> 2][(i & 3) * 4 + e] = t4[e];
+                }
                 if (!warp_wait(&a_empty[as], aph ^ 1)) { ok = false; break; }
-                const uint32_t abase = sbase + C::OFF_A + as * C::A_BYTES;
-                st_shared_v4(abase + a_off0, o[2 * h]);
-                st_shared_v4(abase + a_off1, o[2 * h + 1]);
-                fence_proxy_async_smem();
+                tc_fence_after();
+                tmem_st_32x32b_x16(tm_row + as * 32, o[0]);
+                tmem_st_32x32b_x16(tm_row + as * 32 + 16, o[1]);
+                tmem_st_wait();
+                tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&a_full[as]);
-                if (++as == C::A_STAGES) { as = 0; aph ^= 1; }
             }
         }
     } else {
@@ -481,13 +481,23 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
             const float scale = n < args.N ? __ldg(args.scales + n) : 0.0f;
             if (!warp_wait(&acc_full[ab], abph)) break;
             tc_fence_after();
-            const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + ab * BX;
+            const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + C::A_COLS + ab * C::ACC_COLS;
             float *wsp = full ? nullptr
                               : args.ws + ((size_t)blockIdx.x * args.runs_max + j) * (size_t)(BX * C::BW);
 #pragma unroll 1
             for (int c0 = 0; c0 < BX; c0 += 16) {
                 uint32_t v[16];
                 tmem_ld_32x32b_x16(taddr + c0, v);
+                if (C::NCHAIN > 1) {
+#pragma unroll
+                    for (int ch = 1; ch < C::NCHAIN; ++ch) {
+                        uint32_t u[16];
+                        tmem_ld_32x32b_x16(taddr + ch * BX + c0, u);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) + __uint_as_float(u[i]));
+                    }
+                }
                 tmem_ld_wait();
                 if (full) {
                     const int m0 = m_blk * BX + c0;
