@@ -178,10 +178,16 @@ struct Cfg {
     static constexpr int BW = 128;                     // weight rows per tile (MMA M)
     static constexpr int KR = 128;                     // K per raw (codes/signs) stage
     static constexpr int KA = 64;                      // K per A stage (TMEM) and per x stage (smem)
-    static constexpr int RAW_STAGES = BX >= 256 ? 3 : 6;
+    static constexpr int RAW_STAGES = BX >= 256 ? 2 : (BX >= 128 ? 4 : 6);
     static constexpr int A_STAGES = 8;                 // 32 TMEM columns each (64 K of bf16 pairs)
+    static constexpr int A_BLOCKS = A_STAGES / 2;      // 128-K blocks of A held in TMEM
     static constexpr int A_COLS = A_STAGES * 32;
-    static constexpr int X_STAGES = BX >= 256 ? 3 : (BX >= 128 ? 4 : (BX >= 64 ? 6 : 10));
+    // x stages hold a whole 128-K block (two 64-K swizzle atoms' worth of columns)
+    static constexpr int X_STAGES = BX >= 256 ? 2 : (BX >= 128 ? 3 : (BX >= 64 ? 4 : (BX >= 32 ? 8 : 10)));
+    // One tcgen05.commit per 128-K block frees both its A slot and its x stage: a commit
+    // stalls the tensor pipe for a few hundred cycles, so there is one per 8 MMAs, not per 4.
+    // Slot b % NDONE of `blk_done` completes when the MMAs of the CTA's block b are done.
+    static constexpr int NDONE = X_STAGES > A_BLOCKS ? X_STAGES : A_BLOCKS;
     // independent accumulation chains per tile: consecutive MMAs into one accumulator
     // serialize on its latency, which dominates when N (= BX) is small; K-step k of a
     // stage goes to chain k % NCHAIN and the epilogue adds the chains in a fixed order
@@ -192,26 +198,37 @@ struct Cfg {
     static constexpr int RAW_CODE_BYTES = BW * KR / 2;    // 8 KiB: [128 rows][16 words], 64-byte swizzle
     static constexpr int RAW_SIGN_BYTES = BW * KR / 8;    // 2 KiB: [128 rows][4 words]
     static constexpr int RAW_BYTES = RAW_CODE_BYTES + RAW_SIGN_BYTES;
-    static constexpr int X_BYTES = BX * KA * 2;
+    static constexpr int X_HALF_BYTES = BX * KA * 2;   // one 64-K half: BX rows x 128 bytes, 128-byte swizzle
+    static constexpr int X_BYTES = 2 * X_HALF_BYTES;
     static constexpr int STAGE_EPI_BYTES = 4 * 2 * 16 * 32 * 2;   // 4 warps x 2 buffers x [16 m][32 n] bf16
     static constexpr int OFF_TABLE = 0;
     static constexpr int OFF_RAW = OFF_TABLE + (int)opqbits::kPairTableBytes;
     static constexpr int OFF_X = OFF_RAW + RAW_STAGES * RAW_BYTES;
     static constexpr int OFF_EPI = OFF_X + X_STAGES * X_BYTES;
     static constexpr int OFF_BAR = OFF_EPI + STAGE_EPI_BYTES;
-    static constexpr int NUM_BARS = 2 * RAW_STAGES + 2 * X_STAGES + 2 * A_STAGES + 2 * NACC + 1;
+    static constexpr int NUM_BARS = 2 * RAW_STAGES + X_STAGES + A_STAGES + NDONE + 2 * NACC + 1;
     static constexpr int OFF_TMEM = OFF_BAR + NUM_BARS * 8;
     static constexpr int SMEM_BYTES = OFF_TMEM + 16 + 1024;
     // decoder groups of 4 warps: group g decodes the CTA's 128-K blocks g, g + G, ...;
     // thread r of a group owns weight row r (TMEM lane r) and decodes its whole 128-K block row
-    static constexpr int GROUPS = 3;
+    static constexpr int GROUPS = BX >= 256 ? 2 : 3;
+    // a group waits on raw stage blk % RAW_STAGES knowing only that its own previous block
+    // (blk - GROUPS) was loaded, so the stage's previous phase (block blk - RAW_STAGES) must
+    // be at least that old for the parity test to be exact
+    static_assert(RAW_STAGES >= GROUPS, "raw ring shorter than the decoder rotation");
     static constexpr int WARP_LOAD = 0, WARP_MMA = 1, WARP_XLOAD = 2, WARP_DEC0 = 3, NUM_DEC_WARPS = 4 * GROUPS;
     static constexpr int WARP_EPI0 = WARP_DEC0 + NUM_DEC_WARPS;
-    static constexpr int THREADS = (WARP_EPI0 + 4) * 32;
+    // One MMA-issuing thread per accumulation chain: a thread issues one tcgen05.mma every
+    // few dozen cycles, far slower than the tensor pipe runs a narrow (N <= 64) MMA, so the
+    // chains are issued from separate warps (warp 1, then warps WARP_ISS1...).
+    static constexpr int NISS = NCHAIN;
+    static constexpr int WARP_ISS1 = WARP_EPI0 + 4;
+    static constexpr int THREADS = (WARP_ISS1 + NISS - 1) * 32;
     static_assert(SMEM_BYTES <= 232448, "shared memory");
     static_assert(BX % 16 == 0 && BX >= 16 && BX <= 256, "MMA N");
     static_assert(A_COLS + NACC * ACC_COLS <= 512, "TMEM columns");
     static_assert(RAW_BYTES % 1024 == 0 && X_BYTES % 1024 == 0, "stage alignment");
+    static_assert(A_STAGES % 2 == 0, "a block is two A half-stages");
 };
 
 template <int BX>
@@ -229,10 +246,9 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
     uint64_t *raw_full = bars;
     uint64_t *raw_empty = raw_full + C::RAW_STAGES;
     uint64_t *x_full = raw_empty + C::RAW_STAGES;
-    uint64_t *x_empty = x_full + C::X_STAGES;
-    uint64_t *a_full = x_empty + C::X_STAGES;
-    uint64_t *a_empty = a_full + C::A_STAGES;
-    uint64_t *acc_full = a_empty + C::A_STAGES;
+    uint64_t *a_full = x_full + C::X_STAGES;
+    uint64_t *blk_done = a_full + C::A_STAGES;
+    uint64_t *acc_full = blk_done + C::NDONE;
     uint64_t *acc_empty = acc_full + C::NACC;
     uint64_t *drain = acc_empty + C::NACC;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_TMEM);
@@ -257,19 +273,14 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
             mbar_init(&raw_full[s], signs_by_tma ? 1 : 1 + 32);
             mbar_init(&raw_empty[s], 4);          // the 4 warps of the group that decodes the block
         }
-        for (int s = 0; s < C::X_STAGES; ++s) {
-            mbar_init(&x_full[s], 1);
-            mbar_init(&x_empty[s], 1);
-        }
-        for (int s = 0; s < C::A_STAGES; ++s) {
-            mbar_init(&a_full[s], 4);             // the 4 warps of the decoding group
-            mbar_init(&a_empty[s], 1);
-        }
+        for (int s = 0; s < C::X_STAGES; ++s) mbar_init(&x_full[s], 1);
+        for (int s = 0; s < C::A_STAGES; ++s) mbar_init(&a_full[s], 4);   // the 4 warps of the decoding group
+        for (int s = 0; s < C::NDONE; ++s) mbar_init(&blk_done[s], C::NISS);   // one commit per issuer
         for (int s = 0; s < C::NACC; ++s) {
-            mbar_init(&acc_full[s], 1);
+            mbar_init(&acc_full[s], C::NISS);
             mbar_init(&acc_empty[s], 4);
         }
-        mbar_init(drain, 1);
+        mbar_init(drain, C::NISS);
         fence_mbar_init();
     }
     if (warp == C::WARP_LOAD && lane == 0) {
@@ -346,60 +357,68 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
     } else if (warp == C::WARP_XLOAD) {
         // ----------------------------------------------------------- x producer
         if (lane == 0) {
-            int xs = 0;
-            uint32_t xph = 0;
-            int x_issued = 0;
+            int b = 0;                 // the CTA's block index
             bool ok = true;
             while (ok && it.next(tile, r0, r1, j)) {
                 const int m_blk = tile % args.m_tiles;
-                for (int r = r0; r < r1 && ok; ++r) {
-                    for (int h = 0; h < C::KR / C::KA; ++h) {
-                        if (!mbar_wait(&x_empty[xs], xph ^ 1)) { ok = false; break; }
-                        mbar_arrive_expect_tx(&x_full[xs], C::X_BYTES);
-                        tma_load_2d(smem + C::OFF_X + xs * C::X_BYTES, &tmap_x, r * C::KR + h * C::KA, m_blk * BX,
-                                    &x_full[xs]);
-                        ++x_issued;
-                        if (++xs == C::X_STAGES) { xs = 0; xph ^= 1; }
+                for (int r = r0; r < r1; ++r, ++b) {
+                    // stage b % X_STAGES last held block b - X_STAGES
+                    const int prev = b - C::X_STAGES;
+                    if (prev >= 0 && !mbar_wait(&blk_done[prev % C::NDONE], (uint32_t)(prev / C::NDONE) & 1u)) {
+                        ok = false;
+                        break;
                     }
+                    const int xs = b % C::X_STAGES;
+                    mbar_arrive_expect_tx(&x_full[xs], C::X_BYTES);
+                    uint8_t *dst = smem + C::OFF_X + xs * C::X_BYTES;
+                    tma_load_2d(dst, &tmap_x, r * C::KR, m_blk * BX, &x_full[xs]);
+                    tma_load_2d(dst + C::X_HALF_BYTES, &tmap_x, r * C::KR + C::KA, m_blk * BX, &x_full[xs]);
                 }
             }
             if (!ok) {
-                for (int i = 0; i < x_issued && i < C::X_STAGES; ++i) {
-                    if (--xs < 0) { xs = C::X_STAGES - 1; xph ^= 1; }
-                    (void)mbar_wait(&x_full[xs], xph);
-                }
+                // let the copies already issued land before the CTA can exit
+                for (int i = 1; i <= C::X_STAGES && b - i >= 0; ++i)
+                    (void)mbar_wait(&x_full[(b - i) % C::X_STAGES], (uint32_t)((b - i) / C::X_STAGES) & 1u);
             }
         }
-    } else if (warp == C::WARP_MMA) {
-        // ----------------------------------------------------------- MMA issuer
+    } else if (warp == C::WARP_MMA || warp >= C::WARP_ISS1) {
+        // ----------------------------------------------------------- MMA issuers
+        // Issuer i accumulates K-steps k = i, i + NISS, ... of every 64-K half into chain i.
         if (lane == 0) {
-            int as = 0, xs = 0, ab = 0;
-            uint32_t aph = 0, xph = 0, abph = 0;
+            const int iss = warp == C::WARP_MMA ? 0 : warp - C::WARP_ISS1 + 1;
+            int ab = 0;
+            uint32_t abph = 0;
+            int as0 = 0, xs = 0, ds = 0;       // A half-stage of the block's first half, x stage, blk_done slot
+            uint32_t aph = 0, xph = 0;
             bool ok = true;
             constexpr uint32_t idesc = idesc_bf16_f32(128, BX);
             while (ok && it.next(tile, r0, r1, j)) {
                 if (!mbar_wait(&acc_empty[ab], abph ^ 1)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + C::A_COLS + ab * C::ACC_COLS;
-                uint32_t fresh = (1u << C::NCHAIN) - 1u;  // chains not yet written in this run
-                for (int r = r0; r < r1 && ok; ++r) {
-                    for (int h = 0; h < C::KR / C::KA; ++h) {
-                        if (!mbar_wait(&a_full[as], aph) || !mbar_wait(&x_full[xs], xph)) { ok = false; break; }
+                const uint32_t d_tmem = tmem_base + C::A_COLS + ab * C::ACC_COLS + iss * BX;
+                uint32_t acc = 0;              // 0 for the chain's first MMA of the run
+                for (int r = r0; r < r1; ++r) {
+                    const uint32_t xaddr = sbase + C::OFF_X + xs * C::X_BYTES;
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        if (!mbar_wait(&a_full[as0 + h], aph)) { ok = false; break; }
+                        if (h == 0 && !mbar_wait(&x_full[xs], xph)) { ok = false; break; }
                         tc_fence_after();
-                        const uint32_t a_tmem = tmem_base + as * 32;
-                        const uint64_t bdesc = smem_desc_sw128(sbase + C::OFF_X + xs * C::X_BYTES);
+                        const uint32_t a_tmem = tmem_base + (as0 + h) * 32;
+                        const uint64_t bdesc = smem_desc_sw128(xaddr + h * C::X_HALF_BYTES);
 #pragma unroll
                         for (int k = 0; k < C::KA / 16; ++k) {
-                            const int ch = k % C::NCHAIN;
-                            umma_bf16_ts(d_tmem + ch * BX, a_tmem + 8 * k, bdesc + 2 * k, idesc,
-                                         ((fresh >> ch) & 1u) ? 0u : 1u);
-                            fresh &= ~(1u << ch);
+                            if (k % C::NISS != iss % C::NISS) continue;
+                            umma_bf16_ts(d_tmem, a_tmem + 8 * k, bdesc + 2 * k, idesc, acc);
+                            acc = 1;
                         }
-                        umma_commit(&a_empty[as]);
-                        umma_commit(&x_empty[xs]);
-                        if (++as == C::A_STAGES) { as = 0; aph ^= 1; }
-                        if (++xs == C::X_STAGES) { xs = 0; xph ^= 1; }
                     }
+                    if (!ok) break;
+                    umma_commit(&blk_done[ds]);
+                    as0 += 2;
+                    if (as0 == C::A_STAGES) { as0 = 0; aph ^= 1; }
+                    if (++xs == C::X_STAGES) { xs = 0; xph ^= 1; }
+                    if (++ds == C::NDONE) ds = 0;
                 }
                 if (ok) umma_commit(&acc_full[ab]);
                 if (++ab == C::NACC) { ab = 0; abph ^= 1; }
@@ -427,32 +446,39 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
             const uint32_t rph = (uint32_t)(blk / C::RAW_STAGES) & 1u;
             if (!warp_wait(&raw_full[rs], rph)) { ok = false; break; }
             const uint8_t *rawc = smem + C::OFF_RAW + rs * C::RAW_BYTES + row * (C::KR / 2);
-            uint32_t cw[16];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const uint4 v = *reinterpret_cast<const uint4 *>(rawc + ((((uint32_t)c) ^ sw64) << 4));
-                cw[4 * c] = v.x; cw[4 * c + 1] = v.y; cw[4 * c + 2] = v.z; cw[4 * c + 3] = v.w;
-            }
-            const uint4 sv = *reinterpret_cast<const uint4 *>(smem + C::OFF_RAW + rs * C::RAW_BYTES + C::RAW_CODE_BYTES +
-                                                             row * (C::KR / 8));
-            const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&raw_empty[rs]);   // the raw words are in registers now
+            const uint8_t *raws = smem + C::OFF_RAW + rs * C::RAW_BYTES + C::RAW_CODE_BYTES + row * (C::KR / 8);
 #pragma unroll
             for (int h = 0; h < C::KR / C::KA; ++h) {     // two 64-K A stages per block
                 const int sidx = blk * 2 + h;
                 const int as = sidx % C::A_STAGES;
-                const uint32_t aph = (uint32_t)(sidx / C::A_STAGES) & 1u;
+                // this half's 8 code words (two 16-byte chunks) and 2 sign words
+                uint32_t cw[8];
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    const uint4 v = *reinterpret_cast<const uint4 *>(rawc + ((((uint32_t)(2 * h + c)) ^ sw64) << 4));
+                    cw[4 * c] = v.x; cw[4 * c + 1] = v.y; cw[4 * c + 2] = v.z; cw[4 * c + 3] = v.w;
+                }
+                const uint2 sv = *reinterpret_cast<const uint2 *>(raws + 8 * h);
+                const uint32_t sw[2] = {sv.x, sv.y};
+                if (h == 1) {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&raw_empty[rs]);   // the block's raw words are in registers now
+                }
                 uint32_t o[2][16];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    const int w = 8 * h + i;
                     uint32_t t4[4];
-                    opqbits::decode8_table(cw[w], sw[w >> 2], (uint32_t)(w & 3), lw, lw2, load, t4);
+                    opqbits::decode8_table(cw[i], sw[i >> 2], (uint32_t)(i & 3), lw, lw2, load, t4);
 #pragma unroll
                     for (int e = 0; e < 4; ++e) o[i >> 2][(i & 3) * 4 + e] = t4[e];
                 }
-                if (!warp_wait(&a_empty[as], aph ^ 1)) { ok = false; break; }
+                // the block's A slot last held block blk - A_BLOCKS
+                const int prev = blk - C::A_BLOCKS;
+                if (h == 0 && prev >= 0 &&
+                    !warp_wait(&blk_done[prev % C::NDONE], (uint32_t)(prev / C::NDONE) & 1u)) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
                 tmem_st_32x32b_x16(tm_row + as * 32, o[0]);
                 tmem_st_32x32b_x16(tm_row + as * 32 + 16, o[1]);
@@ -559,26 +585,46 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
                         const int64_t jj = tile - unit_begin(c, gridDim.x, U) / args.kblocks;
                         mybase = args.ws + ((size_t)c * args.runs_max + (size_t)jj) * (size_t)(BX * C::BW);
                     }
-                    // every lane runs the loops (shuffles need all lanes); only rows < N store
-                    for (int col = 0; col < BX; ++col) {
-                        const int m = m_blk * BX + col;
-                        if (m >= args.M) break;
-                        float acc = 0.0f;
+                    // Every lane runs the loops (shuffles need all lanes); only rows < N store.
+                    // 8 columns per pass, the next part's 8 loads issued before the current
+                    // part's adds; each sum still runs over parts 0, 1, ... from 0.0f.
+                    auto part_base = [&](uint32_t p) -> const float * {
+                        if (p < 32)
+                            return reinterpret_cast<const float *>(
+                                __shfl_sync(0xFFFFFFFFu, reinterpret_cast<unsigned long long>(mybase), (int)p));
+                        const int64_t c = c_lo + p;
+                        const int64_t jj = tile - unit_begin(c, gridDim.x, U) / args.kblocks;
+                        return args.ws + ((size_t)c * args.runs_max + (size_t)jj) * (size_t)(BX * C::BW);
+                    };
+                    const int mcols = min(BX, args.M - m_blk * BX);
+                    for (int c0 = 0; c0 < mcols; c0 += 8) {
+                        float acc[8], cur[8], nxt[8];
+                        const float *b0 = part_base(0) + (size_t)c0 * C::BW + row;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            acc[i] = 0.0f;
+                            cur[i] = (c0 + i < mcols) ? __ldcg(b0 + (size_t)i * C::BW) : 0.0f;
+                        }
                         for (uint32_t p = 0; p < parts; ++p) {
-                            const float *base;
-                            if (p < 32) {
-                                base = reinterpret_cast<const float *>(
-                                    __shfl_sync(0xFFFFFFFFu, reinterpret_cast<unsigned long long>(mybase), (int)p));
-                            } else {
-                                const int64_t c = c_lo + p;
-                                const int64_t jj = tile - unit_begin(c, gridDim.x, U) / args.kblocks;
-                                base = args.ws + ((size_t)c * args.runs_max + (size_t)jj) * (size_t)(BX * C::BW);
+                            if (p + 1 < parts) {
+                                const float *bn = part_base(p + 1) + (size_t)c0 * C::BW + row;
+#pragma unroll
+                                for (int i = 0; i < 8; ++i) nxt[i] = (c0 + i < mcols) ? __ldcg(bn + (size_t)i * C::BW) : 0.0f;
                             }
-                            acc += __ldcg(base + (size_t)col * C::BW + row);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                acc[i] += cur[i];
+                                cur[i] = nxt[i];
+                            }
                         }
                         if (n < args.N) {
-                            const __nv_bfloat16 o = __float2bfloat16_rn(acc * scale);
-                            args.y[(size_t)m * args.N + n] = *reinterpret_cast<const uint16_t *>(&o);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                if (c0 + i < mcols) {
+                                    const __nv_bfloat16 o = __float2bfloat16_rn(acc[i] * scale);
+                                    args.y[(size_t)(m_blk * BX + c0 + i) * args.N + n] = *reinterpret_cast<const uint16_t *>(&o);
+                                }
+                            }
                         }
                     }
                     if (lane == 0) atomicExch(args.counters + (size_t)tile * 4 + q, 0u);   // ready for the next call
