@@ -80,7 +80,7 @@ class ClockSampler:
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", "20"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.reader = threading.Thread(target=self._read, daemon=True)
             self.reader.start()
@@ -91,7 +91,14 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self, start: bool):
+        """Bracket the timed region: only samples taken inside it are summarised."""
+        if start:
+            self.t0 = time.time()
+        else:
+            self.t1 = time.time()
 
     def __exit__(self, *exc):
         if self.proc is not None:
@@ -105,7 +112,10 @@ class ClockSampler:
     def summary(self):
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
+        t0, t1 = getattr(self, "t0", 0.0), getattr(self, "t1", float("inf"))
+        for ts, line in self.lines:
+            if not (t0 <= ts <= t1 + 0.05):
+                continue
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
                 continue
@@ -148,10 +158,19 @@ def gpu_arm(args, rank, world, local_rank):
     flush = torch.empty((4 * max(l2, 64 << 20),), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step():
+    def step(ev=None):
+        # ev: optional 4 events bracketing the three launches (timed region only)
+        if ev is not None:
+            ev[0].record(stream)
         opq.quantize(w, alpha, out=(codes, signs, scales))
+        if ev is not None:
+            ev[1].record(stream)
         opq.linear(x, codes, signs, scales, alpha, out=y, workspace=ws)
+        if ev is not None:
+            ev[2].record(stream)
         opq.dequantize(codes, signs, scales, alpha, out=wq)
+        if ev is not None:
+            ev[3].record(stream)
 
     launches_per_step = 1 + opq.plan(M, N, K)[2] + 1
 
@@ -164,20 +183,22 @@ def gpu_arm(args, rank, world, local_rank):
     torch.cuda.synchronize()
     assert opq.device_error() == 0
 
-    # ---- timed region: K steps, L2 flushed between steps (outside the event pairs)
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    # ---- timed region: K steps, L2 flushed between steps (outside the event pairs); the
+    # events bracketing each launch give the per-kernel durations of the same region
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize()
     with ClockSampler(local_rank) as clocks:
+        clocks.mark(True)
         for i in range(args.steps):
             flush.zero_()
-            starts[i].record(stream)
-            step()
-            ends[i].record(stream)
+            step(evs[i])
         torch.cuda.synchronize()
+        clocks.mark(False)
     barrier()
-    per_step = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    per_step = [e[0].elapsed_time(e[3]) for e in evs]
+    live = {name: statistics.fmean(e[a].elapsed_time(e[b]) for e in evs)
+            for name, a, b in (("quantize", 0, 1), ("linear", 1, 2), ("dequantize", 2, 3))}
     ms_step = sum(per_step) / len(per_step)
     if world > 1:
         t = torch.tensor([ms_step], device=dev)
@@ -202,9 +223,8 @@ def gpu_arm(args, rank, world, local_rank):
         return statistics.median(ts), ts
 
     peaks, peak_src = load_peaks()
-    t_q, _ = time_kernel(lambda: opq.quantize(w, alpha, out=(codes, signs, scales)))
-    t_l, _ = time_kernel(lambda: opq.linear(x, codes, signs, scales, alpha, out=y, workspace=ws))
-    t_d, _ = time_kernel(lambda: opq.dequantize(codes, signs, scales, alpha, out=wq))
+    # mean launch durations inside the timed region (each launch starts with a flushed L2)
+    t_q, t_l, t_d = live["quantize"], live["linear"], live["dequantize"]
     q_bytes = N * K * 2 + N * K // 8 * 5 + 4 * N      # read W, write codes (K/2 B) + signs (K/8 B) + scales
     d_bytes = N * K // 8 * 5 + 4 * N + N * K * 2
     l_bytes = N * K * 5 // 8 + 4 * N + 2 * M * K + 2 * M * N
@@ -274,10 +294,11 @@ def gpu_arm(args, rank, world, local_rank):
         ms_e2e = float(t.item())
     barrier()
 
-    traffic = recorded_traffic("linear_tile_kernel")
-    roof = {"bound": "tensor", "kernel": "linear_tile_kernel", "achieved": linear_tflops,
+    traffic = recorded_traffic("linear_kernel")
+    roof = {"bound": "tensor", "kernel": "linear_kernel<256>", "achieved": linear_tflops,
             "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": linear_tflops / peaks["bf16_tflops"],
-            "traffic": traffic, "algorithmic_bytes": l_bytes, "peak_source": f"bf16 burst, {peak_src}"}
+            "traffic": traffic, "algorithmic_flops": flops, "algorithmic_bytes": l_bytes,
+            "launch_ms": t_l, "peak_source": f"bf16 dense burst, {peak_src}"}
     out = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -289,6 +310,7 @@ def gpu_arm(args, rank, world, local_rank):
         "e2e": {"value": world * flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms_e2e,
                 "h2d_bytes_per_step": w.numel() * 2 + x.numel() * 2, "d2h_bytes_per_step": y.numel() * 2},
         "gpu_launches": launches_per_step * args.steps,
+        "kernels_live_ms": live,
         "clocks": clocks.summary(),
         "peaks": peaks,
     }
@@ -296,7 +318,7 @@ def gpu_arm(args, rank, world, local_rank):
 
 
 # --------------------------------------------------------------------------- CPU arms
-def cpu_oracle_sample(budget_s: float = 15.0):
+def cpu_oracle_sample(budget_s: float = 12.0):
     """Time the fp64 oracle on a bounded sample of the bench workload: quantize 256
     weight rows and the linear for 16 activation rows against those 256 weight rows."""
     import numpy as np
@@ -314,11 +336,11 @@ def cpu_oracle_sample(budget_s: float = 15.0):
         r = oracle.quantize(ws, lin.alpha)
         oracle.linear(xs, r["codes"], r["signs"], r["scales"], lin.alpha)
         reps += 1
-        if time.perf_counter() - t0 > budget_s or reps >= 1000:
+        if time.perf_counter() - t0 > budget_s:
             break
     dt = (time.perf_counter() - t0) / reps
     flops = 2.0 * xs.shape[0] * rows * lin.K
-    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    cores = oracle.num_threads()
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
             "sample": f"quantize {rows}x{lin.K} + linear {xs.shape[0]}x{lin.K} @ {rows}x{lin.K}^T "
                       f"({reps} reps, {dt:.3f} s each)",
@@ -344,7 +366,7 @@ def reference_arm(args):
     dt = sum(ts) / len(ts)
     flops = 2.0 * xs.shape[0] * ws.shape[0] * lin.K
     v = flops / dt / 1e12
-    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    cores = oracle.num_threads()
     return {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -388,7 +410,7 @@ def profile_run(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="opq", choices=["opq", "reference"])
     ap.add_argument("--no-sweep", action="store_true")

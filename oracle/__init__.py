@@ -51,6 +51,7 @@ def _bind(path: str):
     lib.oracle_double_to_bf16.argtypes = [D]
     lib.oracle_double_to_bf16.restype = ctypes.c_uint16
     lib.oracle_rounding_mode_ok.restype = ctypes.c_int
+    lib.oracle_num_threads.restype = ctypes.c_int
     return lib
 
 
@@ -167,6 +168,10 @@ class Oracle:
         self._lib.oracle_uniform_int4(_p(w), N, K, _p(out))
         return out
 
+    def num_threads(self) -> int:
+        """OpenMP threads the oracle's loops run on."""
+        return int(self._lib.oracle_num_threads())
+
     def double_to_bf16(self, v: float) -> int:
         return int(self._lib.oracle_double_to_bf16(float(v)))
 
@@ -209,6 +214,10 @@ def snr_db(*a, **k):
 
 def uniform_int4(*a, **k):
     return default().uniform_int4(*a, **k)
+
+
+def num_threads() -> int:
+    return default().num_threads()
 
 
 def double_to_bf16(*a, **k):

@@ -33,6 +33,9 @@
 #include <stdlib.h>
 #include <stdint.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 
 #define OPQ_LEVELS 15
 
@@ -81,6 +84,16 @@ static uint16_t double_to_bf16_rne(double x)
 }
 
 int oracle_rounding_mode_ok(void) { return fegetround() == FE_TONEAREST; }
+
+/* threads the OpenMP loops use (1 when built without OpenMP); reported beside timings */
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
 
 uint16_t oracle_double_to_bf16(double x) { return double_to_bf16_rne(x); }
 
