@@ -154,6 +154,7 @@ struct Plan {
     int m_tiles, n_tiles, kblocks;
     int grid;       // CTAs of the linear kernel
     int runs_max;   // mode 1
+    int tail_split; // mode 0: 2 = the tiles past the last whole wave run as two half-width runs
     size_t counter_bytes;   // mode 1: the zero-between-calls arrival counters at the workspace start
     size_t ws_bytes;
     int launches;
@@ -191,6 +192,11 @@ Plan make_plan(int64_t M, int64_t N, int64_t K) {
         const int64_t tiles = (int64_t)p.m_tiles * p.n_tiles;
         p.grid = (int)(tiles < kPlanSMs ? tiles : kPlanSMs);
         p.runs_max = 1;
+        // tiles left after the whole waves: when there are at most half as many as CTAs, each
+        // is split along its activation rows over two CTAs, so that the last wave takes half a
+        // tile's time instead of a whole one
+        const int64_t tail = tiles - (tiles / p.grid) * p.grid;
+        p.tail_split = (tail > 0 && 2 * tail <= p.grid && p.bx >= 32) ? 2 : 1;
         p.counter_bytes = 0;
         p.ws_bytes = 0;
     }
@@ -225,8 +231,9 @@ void dispatch_quant(int vpl, const uint16_t *w, int64_t N, int64_t K, int64_t ld
 }
 
 template <int BX>
-cudaError_t launch_linear(DeviceInfo *di, const Plan &plan, const CUtensorMap &xmap, const CUtensorMap &cmap,
-                          const CUtensorMap &smap, const opqk::LinearArgs &a, cudaStream_t st) {
+cudaError_t launch_linear(DeviceInfo *di, const Plan &plan, const CUtensorMap &xmap, const CUtensorMap &xhmap,
+                          const CUtensorMap &cmap, const CUtensorMap &smap, const opqk::LinearArgs &a,
+                          cudaStream_t st) {
     using C = opqk::Cfg<BX>;
     const int key = BX / 16;
     if (!di->linear_attr[key]) {
@@ -235,7 +242,7 @@ cudaError_t launch_linear(DeviceInfo *di, const Plan &plan, const CUtensorMap &x
         if (e != cudaSuccess) return e;
         di->linear_attr[key] = true;
     }
-    opqk::linear_kernel<BX><<<plan.grid, C::THREADS, C::SMEM_BYTES, st>>>(xmap, cmap, smap, a);
+    opqk::linear_kernel<BX><<<plan.grid, C::THREADS, C::SMEM_BYTES, st>>>(xmap, xhmap, cmap, smap, a);
     return cudaGetLastError();
 }
 
@@ -369,10 +376,16 @@ opq_status opq_linear(const uint16_t *x, int64_t M, int64_t K, const uint32_t *c
     a.kblocks = plan.kblocks;
     a.mode = plan.mode;
     a.runs_max = plan.runs_max;
+    a.tail_split = plan.mode == 0 ? plan.tail_split : 1;
     lut_bf16(alpha, a.lut);
 
-    CUtensorMap xmap, cmap, smap;
+    CUtensorMap xmap, xhmap, cmap, smap;
     if ((s = make_x_map(&xmap, x, M, K, (uint32_t)plan.bx)) != OPQ_OK) return s;
+    if (a.tail_split == 2) {
+        if ((s = make_x_map(&xhmap, x, M, K, (uint32_t)plan.bx / 2)) != OPQ_OK) return s;
+    } else {
+        xhmap = xmap;   // not read by the kernel
+    }
     if ((s = make_u32_map(&cmap, codes, N, K / 8, 16u, 128u, CU_TENSOR_MAP_SWIZZLE_64B)) != OPQ_OK) return s;
     // the sign plane's rows are 16-byte aligned (a TMA requirement) when K % 128 == 0; otherwise the
     // kernel copies the sign words with cp.async
@@ -384,11 +397,11 @@ opq_status opq_linear(const uint16_t *x, int64_t M, int64_t K, const uint32_t *c
     }
     cudaError_t e;
     switch (plan.bx) {
-        case 16: e = launch_linear<16>(di, plan, xmap, cmap, smap, a, st); break;
-        case 32: e = launch_linear<32>(di, plan, xmap, cmap, smap, a, st); break;
-        case 64: e = launch_linear<64>(di, plan, xmap, cmap, smap, a, st); break;
-        case 128: e = launch_linear<128>(di, plan, xmap, cmap, smap, a, st); break;
-        default: e = launch_linear<256>(di, plan, xmap, cmap, smap, a, st); break;
+        case 16: e = launch_linear<16>(di, plan, xmap, xhmap, cmap, smap, a, st); break;
+        case 32: e = launch_linear<32>(di, plan, xmap, xhmap, cmap, smap, a, st); break;
+        case 64: e = launch_linear<64>(di, plan, xmap, xhmap, cmap, smap, a, st); break;
+        case 128: e = launch_linear<128>(di, plan, xmap, xhmap, cmap, smap, a, st); break;
+        default: e = launch_linear<256>(di, plan, xmap, xhmap, cmap, smap, a, st); break;
     }
     if (e != cudaSuccess) return cuda_fail(e);
     e = cudaGetLastError();

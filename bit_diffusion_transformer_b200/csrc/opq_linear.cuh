@@ -125,6 +125,8 @@ struct LinearArgs {
     int kblocks;            // 128-K blocks per tile
     int mode;               // 0 whole tiles strided over CTAs, 1 contiguous unit ranges (stream-K)
     int runs_max;           // mode 1: most runs one CTA can have
+    int tail_split;         // mode 0: 2 = tiles past the last full wave run as two half-width
+                            // (BX/2 activation rows) runs on different CTAs; 1 = whole tiles
     uint16_t lut[16];       // bf16 (q/15)^(1/alpha)
 };
 
@@ -135,31 +137,52 @@ __host__ __device__ __forceinline__ int64_t unit_owner(int64_t u, int64_t C, int
     return ((u + 1) * C - 1) / U;
 }
 
-// The sequence of runs of one CTA; every role walks the same sequence.
+// The sequence of runs of one CTA; every role walks the same sequence. A run is one
+// weight tile, a range of its 128-K blocks and a range of its activation rows.
 struct RunIter {
-    int mode, tiles, kblocks, grid;
+    int mode, tiles, kblocks, grid, cta;
     int64_t u, u_end;   // mode 1
     int t_next;         // mode 0
+    int full_end;       // mode 0: tiles in whole waves (handed out strided)
+    int split;          // mode 0: 1 or 2 runs per tile after the whole waves
+    bool tail_done;
     int run_idx;
-    __device__ __forceinline__ void init(const LinearArgs &a, int tiles_, int grid_, int cta) {
+    __device__ __forceinline__ void init(const LinearArgs &a, int tiles_, int grid_, int cta_) {
         mode = a.mode;
         tiles = tiles_;
         kblocks = a.kblocks;
         grid = grid_;
+        cta = cta_;
         run_idx = 0;
-        t_next = cta;
+        t_next = cta_;
+        split = a.tail_split;
+        full_end = split == 2 ? (tiles_ / grid_) * grid_ : tiles_;
+        tail_done = false;
         const int64_t U = (int64_t)tiles * kblocks;
-        u = unit_begin(cta, grid_, U);
-        u_end = unit_begin(cta + 1, grid_, U);
+        u = unit_begin(cta_, grid_, U);
+        u_end = unit_begin(cta_ + 1, grid_, U);
     }
-    // next run: tile, block range [r0, r1), run index j; false at the end
-    __device__ __forceinline__ bool next(int &tile, int &r0, int &r1, int &j) {
+    // next run: tile, block range [r0, r1), run index j, activation rows [xoff, xoff + xrows)
+    // of the tile's bx; false at the end
+    __device__ __forceinline__ bool next(int &tile, int &r0, int &r1, int &j, int &xoff, int &xrows, int bx) {
+        xoff = 0;
+        xrows = bx;
         if (mode == 0) {
-            if (t_next >= tiles) return false;
-            tile = t_next;
+            if (t_next < full_end) {
+                tile = t_next;
+                t_next += grid;
+            } else if (split == 2) {
+                // tail tile t is run by CTAs 2 (t - full_end) and 2 (t - full_end) + 1, one half each
+                if (tail_done || cta >= 2 * (tiles - full_end)) return false;
+                tile = full_end + (cta >> 1);
+                xrows = bx / 2;
+                xoff = (cta & 1) * xrows;
+                tail_done = true;
+            } else {
+                return false;
+            }
             r0 = 0;
             r1 = kblocks;
-            t_next += grid;
         } else {
             if (u >= u_end) return false;
             tile = (int)(u / kblocks);
@@ -170,6 +193,10 @@ struct RunIter {
         }
         j = run_idx++;
         return true;
+    }
+    __device__ __forceinline__ bool next(int &tile, int &r0, int &r1, int &j) {
+        int xo, xr;
+        return next(tile, r0, r1, j, xo, xr, 2);
     }
 };
 
@@ -233,8 +260,9 @@ struct Cfg {
 
 template <int BX>
 __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
-    linear_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_codes,
-                  const __grid_constant__ CUtensorMap tmap_signs, const __grid_constant__ LinearArgs args) {
+    linear_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_xh,
+                  const __grid_constant__ CUtensorMap tmap_codes, const __grid_constant__ CUtensorMap tmap_signs,
+                  const __grid_constant__ LinearArgs args) {
     using C = Cfg<BX>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = smem_u32(smem_raw);
@@ -287,7 +315,10 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
         tma_prefetch_desc(&tmap_codes);
         if (signs_by_tma) tma_prefetch_desc(&tmap_signs);
     }
-    if (warp == C::WARP_XLOAD && lane == 0) tma_prefetch_desc(&tmap_x);
+    if (warp == C::WARP_XLOAD && lane == 0) {
+        tma_prefetch_desc(&tmap_x);
+        if (args.tail_split == 2) tma_prefetch_desc(&tmap_xh);
+    }
     if (warp == C::WARP_MMA) {
         tmem_alloc(tmem_slot, C::TMEM_COLS);
         tmem_relinquish();
@@ -359,8 +390,14 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
         if (lane == 0) {
             int b = 0;                 // the CTA's block index
             bool ok = true;
-            while (ok && it.next(tile, r0, r1, j)) {
+            int xoff, xrows;
+            while (ok && it.next(tile, r0, r1, j, xoff, xrows, BX)) {
                 const int m_blk = tile % args.m_tiles;
+                // a half-width run loads its BX/2 activation rows with the half-height box
+                const bool half = xrows != BX;
+                const void *xmap = half ? (const void *)&tmap_xh : (const void *)&tmap_x;
+                const uint32_t xbytes = half ? C::X_BYTES / 2 : C::X_BYTES;
+                const int xrow = m_blk * BX + xoff;
                 for (int r = r0; r < r1; ++r, ++b) {
                     // stage b % X_STAGES last held block b - X_STAGES
                     const int prev = b - C::X_STAGES;
@@ -369,10 +406,10 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
                         break;
                     }
                     const int xs = b % C::X_STAGES;
-                    mbar_arrive_expect_tx(&x_full[xs], C::X_BYTES);
+                    mbar_arrive_expect_tx(&x_full[xs], xbytes);
                     uint8_t *dst = smem + C::OFF_X + xs * C::X_BYTES;
-                    tma_load_2d(dst, &tmap_x, r * C::KR, m_blk * BX, &x_full[xs]);
-                    tma_load_2d(dst + C::X_HALF_BYTES, &tmap_x, r * C::KR + C::KA, m_blk * BX, &x_full[xs]);
+                    tma_load_2d(dst, xmap, r * C::KR, xrow, &x_full[xs]);
+                    tma_load_2d(dst + C::X_HALF_BYTES, xmap, r * C::KR + C::KA, xrow, &x_full[xs]);
                 }
             }
             if (!ok) {
@@ -391,8 +428,11 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
             int as0 = 0, xs = 0, ds = 0;       // A half-stage of the block's first half, x stage, blk_done slot
             uint32_t aph = 0, xph = 0;
             bool ok = true;
-            constexpr uint32_t idesc = idesc_bf16_f32(128, BX);
-            while (ok && it.next(tile, r0, r1, j)) {
+            constexpr uint32_t idesc_full = idesc_bf16_f32(128, BX);
+            constexpr uint32_t idesc_half = idesc_bf16_f32(128, BX / 2);
+            int xoff, xrows;
+            while (ok && it.next(tile, r0, r1, j, xoff, xrows, BX)) {
+                const uint32_t idesc = xrows == BX ? idesc_full : idesc_half;
                 if (!mbar_wait(&acc_empty[ab], abph ^ 1)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + C::A_COLS + ab * C::ACC_COLS + iss * BX;
@@ -499,7 +539,8 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
         int ab = 0;
         uint32_t abph = 0;
         int sb = 0;
-        while (it.next(tile, r0, r1, j)) {
+        int xoff, xrows;
+        while (it.next(tile, r0, r1, j, xoff, xrows, BX)) {
             const int n_blk = tile / args.m_tiles, m_blk = tile % args.m_tiles;
             const int n = n_blk * C::BW + row;
             const int n0 = n_blk * C::BW + q * 32;           // first row of this warp's quarter
@@ -511,7 +552,7 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
             float *wsp = full ? nullptr
                               : args.ws + ((size_t)blockIdx.x * args.runs_max + j) * (size_t)(BX * C::BW);
 #pragma unroll 1
-            for (int c0 = 0; c0 < BX; c0 += 16) {
+            for (int c0 = 0; c0 < xrows; c0 += 16) {
                 uint32_t v[16];
                 tmem_ld_32x32b_x16(taddr + c0, v);
                 if (C::NCHAIN > 1) {
@@ -526,7 +567,7 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
                 }
                 tmem_ld_wait();
                 if (full) {
-                    const int m0 = m_blk * BX + c0;
+                    const int m0 = m_blk * BX + xoff + c0;
                     if (vec_y && n0 + 32 <= args.N) {
                         // stage [16 m][32 n] bf16, then each lane stores 32 contiguous bytes of one m row
                         const uint32_t sbuf = stage0 + (uint32_t)sb * 1024u;

@@ -218,6 +218,15 @@ def test_linear_alpha(alpha):
     linear_parity(x, w, alpha)
 
 
+@pytest.mark.parametrize("M,N,K", [(512, 10240, 256), (300, 9728, 160)])
+def test_linear_tail_split(M, N, K):
+    # more tiles than one wave of CTAs, with the leftover tiles (at most half a wave) each
+    # run as two half-width runs on two CTAs: every output, including the ragged last m-tile
+    lin = workloads.Linear("tail", M, N, K, w_seed=M + N, x_seed=K)
+    x, w = lin.make("cpu")
+    linear_parity(x, w, 0.73)
+
+
 def test_linear_deterministic():
     for M in (16, 700):
         lin = workloads.Linear("det", M, 1024, 1024, w_seed=1, x_seed=2)
