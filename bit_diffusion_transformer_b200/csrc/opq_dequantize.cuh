@@ -1,10 +1,15 @@
 // opq_dequantize.cuh — packed planes -> bf16 W'.
 //
 // "OPQ INT4 Z-Image" model card, "inference decoding": w = sign * (q/15)^(1/alpha)
-// * max. The 16 magnitudes (q/15)^(1/alpha) arrive as fp64 (formed on the host),
-// the product with the row scale is formed in fp64 and rounded once to bf16.
-// One thread per code word (8 weights): 4 + 1 bytes in, 16 bytes out.
+// * max. The 16 magnitudes (q/15)^(1/alpha) arrive as fp64 (formed on the host);
+// per row, the 16 products with the row scale are formed in fp64 and rounded once
+// to bf16 (one per lane), and every weight of the row is then a byte-plane table
+// lookup (opq_bits.h decode8) with its sign bit ORed in — the same bits as forming
+// the product per weight, since RNE is symmetric under negation.
+// One warp per row; a lane takes 32 weights at a time (16 B of codes + one sign word
+// in, 64 B out), consecutive lanes on consecutive chunks.
 #pragma once
+#include "opq_bits.h"
 #include "opq_device.cuh"
 
 namespace opqk {
@@ -28,33 +33,56 @@ __device__ __forceinline__ uint32_t f64_to_bf16_rne(double p) {
 __global__ void __launch_bounds__(256) dequantize_kernel(const uint32_t *__restrict__ codes,
                                                          const uint32_t *__restrict__ signs,
                                                          const float *__restrict__ scales, uint32_t rows,
-                                                         uint32_t nvec, const __grid_constant__ DequantParams dp,
+                                                         uint32_t chunks, const __grid_constant__ DequantParams dp,
                                                          uint16_t *__restrict__ out) {
-    __shared__ double lut[16];
-    if (threadIdx.x < 16) lut[threadIdx.x] = dp.lut[threadIdx.x];
-    __syncthreads();
-    const uint64_t total = (uint64_t)rows * nvec;
-    for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-         i += (uint64_t)gridDim.x * blockDim.x) {
-        const uint64_t n = i / nvec;
-        const uint32_t j = (uint32_t)(i - n * nvec);
-        const uint32_t c = __ldg(codes + i);
-        const uint32_t sb = (__ldg(signs + n * (nvec / 4) + j / 4) >> (8 * (j & 3))) & 0xFFu;
-        const double sc = (double)__ldg(scales + n);
-        uint32_t o[4];
+    const uint32_t lane = threadIdx.x & 31u;
+    const uint32_t warps = gridDim.x * (blockDim.x >> 5);
+    // lane q (and q + 16) holds LUT[q] for the products
+    const double lut_q = dp.lut[lane & 15u];
+    for (uint32_t n = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); n < rows; n += warps) {
+        const uint32_t e = f64_to_bf16_rne(lut_q * (double)__ldg(scales + n));
+        opqbits::DecodeTable T;
 #pragma unroll
-        for (int p = 0; p < 4; ++p) {
-            uint32_t h[2];
+        for (int j = 0; j < 4; ++j) {
+            uint32_t l = 0, h = 0;
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int idx = 2 * p + e;
-                double v = lut[(c >> (4 * idx)) & 0xFu] * sc;
-                if ((sb >> idx) & 1u) v = -v;
-                h[e] = f64_to_bf16_rne(v);
+            for (int t = 0; t < 4; ++t) {
+                const uint32_t v = __shfl_sync(0xFFFFFFFFu, e, 4 * j + t);
+                l |= (v & 0xFFu) << (8 * t);
+                h |= ((v >> 8) & 0xFFu) << (8 * t);
             }
-            o[p] = h[0] | (h[1] << 16);
+            T.L[j] = l;
+            T.H[j] = h;
         }
-        reinterpret_cast<uint4 *>(out)[i] = make_uint4(o[0], o[1], o[2], o[3]);
+        const uint4 *crow = reinterpret_cast<const uint4 *>(codes + (size_t)n * chunks * 4u);
+        const uint32_t *srow = signs + (size_t)n * chunks;
+        uint4 *orow = reinterpret_cast<uint4 *>(out + (size_t)n * chunks * 32u);
+        // up to four chunks per lane per pass, their loads issued before any decoding
+        for (uint32_t i0 = lane; i0 < chunks; i0 += 128u) {
+            uint4 c[4];
+            uint32_t sw[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const uint32_t i = i0 + 32u * u;
+                c[u] = i < chunks ? __ldg(crow + i) : make_uint4(0u, 0u, 0u, 0u);
+                sw[u] = i < chunks ? __ldg(srow + i) : 0u;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const uint32_t i = i0 + 32u * u;
+                if (i >= chunks) break;
+                uint32_t o[16];
+                opqbits::decode8(c[u].x, sw[u] & 0xFFu, T, &o[0]);
+                opqbits::decode8(c[u].y, (sw[u] >> 8) & 0xFFu, T, &o[4]);
+                opqbits::decode8(c[u].z, (sw[u] >> 16) & 0xFFu, T, &o[8]);
+                opqbits::decode8(c[u].w, sw[u] >> 24, T, &o[12]);
+                uint4 *dst = orow + (size_t)i * 4u;
+                dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+                dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+                dst[2] = make_uint4(o[8], o[9], o[10], o[11]);
+                dst[3] = make_uint4(o[12], o[13], o[14], o[15]);
+            }
+        }
     }
 }
 
