@@ -130,6 +130,47 @@ void lut_bf16(float alpha, uint16_t (&lut)[16]) {
 
 // uint32 plane [rows, words] row-major, box {box_words, box_rows}, zero fill. With the
 // 64-byte swizzle (box rows of 64 bytes) 16-byte chunk c of row r lands at c ^ ((r >> 1) & 3).
+// uint32 plane [rows, words_per_row] viewed as 3-D {w (words within a 128-K block), rows, blocks}:
+// box {w, box_rows, box_blocks} lands as box_blocks consecutive [box_rows][w] images. Needs
+// words_per_row == w * blocks (K % 128 == 0) and 16-byte rows.
+opq_status make_u32_block_map(CUtensorMap *map, const void *p, int64_t rows, uint32_t w, int64_t blocks,
+                              uint32_t box_rows, uint32_t box_blocks, CUtensorMapSwizzle swizzle) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return OPQ_ERR_CUDA;
+    cuuint64_t dims[3] = {(cuuint64_t)w, (cuuint64_t)rows, (cuuint64_t)blocks};
+    cuuint64_t strides[2] = {(cuuint64_t)w * (cuuint64_t)blocks * 4u, (cuuint64_t)w * 4u};
+    cuuint32_t box[3] = {w, box_rows, box_blocks};
+    cuuint32_t estr[3] = {1u, 1u, 1u};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void *>(p), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        t_last_cuda_error = (int)r;
+        return OPQ_ERR_CUDA;
+    }
+    return OPQ_OK;
+}
+
+// x [rows, K] bf16 viewed as 3-D {64 (K within a 64-K chunk), rows, K / 64}, box {64, box_rows,
+// chunks}, 128-byte swizzle: the chunks land one after the other (needs K % 64 == 0).
+opq_status make_x_chunk_map(CUtensorMap *map, const void *x, int64_t rows, int64_t K, uint32_t box_rows,
+                            uint32_t chunks) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return OPQ_ERR_CUDA;
+    cuuint64_t dims[3] = {64u, (cuuint64_t)rows, (cuuint64_t)(K / 64)};
+    cuuint64_t strides[2] = {(cuuint64_t)K * 2u, 128u};
+    cuuint32_t box[3] = {64u, box_rows, chunks};
+    cuuint32_t estr[3] = {1u, 1u, 1u};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(x), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        t_last_cuda_error = (int)r;
+        return OPQ_ERR_CUDA;
+    }
+    return OPQ_OK;
+}
+
 opq_status make_u32_map(CUtensorMap *map, const void *p, int64_t rows, int64_t words, uint32_t box_words,
                         uint32_t box_rows, CUtensorMapSwizzle swizzle) {
     EncodeTiledFn fn = encode_fn();
@@ -152,6 +193,8 @@ struct Plan {
     int mode;       // 0 whole tiles, 1 stream-K with a fixed-order fix-up
     int bx;         // activation rows per tile (the MMA N)
     int m_tiles, n_tiles, kblocks;
+    int grp;        // 128-K blocks per load group of the chosen tile width
+    int ngroups;    // load groups per tile
     int grid;       // CTAs of the linear kernel
     int runs_max;   // mode 1
     int tail_split; // mode 0: 2 = the tiles past the last whole wave run as two half-width runs
@@ -174,17 +217,23 @@ Plan make_plan(int64_t M, int64_t N, int64_t K) {
     p.n_tiles = (int)((N + 127) / 128);
     if (M <= 128) {
         p.bx = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
+        // the narrow tiles fetch several 128-K blocks per copy through 3-D views of the planes,
+        // which need whole blocks (K % 128 == 0); other K take the one-block-per-copy width
+        if (K % 128 != 0) p.bx = 128;
         p.m_tiles = 1;
     } else {
         p.bx = 256;
         p.m_tiles = (int)((M + 255) / 256);
     }
+    // blocks per load group: must match the kernel's Cfg<BX>::GRP
+    p.grp = p.bx <= 16 ? 4 : (p.bx <= 64 ? 2 : 1);
+    p.ngroups = (p.kblocks + p.grp - 1) / p.grp;
     if (M <= 128 && p.n_tiles <= kCounterTiles) {
         p.mode = 1;
-        const int64_t U = (int64_t)p.n_tiles * p.kblocks;
+        const int64_t U = (int64_t)p.n_tiles * p.ngroups;
         p.grid = (int)(U < kPlanSMs ? U : kPlanSMs);
         const int64_t per = (U + p.grid - 1) / p.grid;
-        p.runs_max = (int)((per + p.kblocks - 1) / p.kblocks + 1);
+        p.runs_max = (int)((per + p.ngroups - 1) / p.ngroups + 1);
         p.counter_bytes = kCounterBytes;
         p.ws_bytes = p.counter_bytes + (size_t)p.grid * (size_t)p.runs_max * (size_t)p.bx * 128u * sizeof(float);
     } else {
@@ -374,26 +423,39 @@ opq_status opq_linear(const uint16_t *x, int64_t M, int64_t K, const uint32_t *c
     a.m_tiles = plan.m_tiles;
     a.n_tiles = plan.n_tiles;
     a.kblocks = plan.kblocks;
+    a.ngroups = plan.ngroups;
     a.mode = plan.mode;
     a.runs_max = plan.runs_max;
     a.tail_split = plan.mode == 0 ? plan.tail_split : 1;
     lut_bf16(alpha, a.lut);
 
     CUtensorMap xmap, xhmap, cmap, smap;
-    if ((s = make_x_map(&xmap, x, M, K, (uint32_t)plan.bx)) != OPQ_OK) return s;
+    // the sign plane's rows are 16-byte aligned (a TMA requirement) when K % 128 == 0; otherwise the
+    // kernel copies the sign words with cp.async
+    a.signs_tma = (K % 128 == 0) ? 1 : 0;
+    if (plan.grp > 1) {
+        // load groups of plan.grp blocks per copy (K % 128 == 0 here)
+        const int64_t kb = K / 128;
+        if ((s = make_x_chunk_map(&xmap, x, M, K, (uint32_t)plan.bx, 2u * (uint32_t)plan.grp)) != OPQ_OK) return s;
+        if ((s = make_u32_block_map(&cmap, codes, N, 16u, kb, 128u, (uint32_t)plan.grp, CU_TENSOR_MAP_SWIZZLE_64B)) !=
+            OPQ_OK)
+            return s;
+        if ((s = make_u32_block_map(&smap, signs, N, 4u, kb, 128u, (uint32_t)plan.grp, CU_TENSOR_MAP_SWIZZLE_NONE)) !=
+            OPQ_OK)
+            return s;
+    } else {
+        if ((s = make_x_map(&xmap, x, M, K, (uint32_t)plan.bx)) != OPQ_OK) return s;
+        if ((s = make_u32_map(&cmap, codes, N, K / 8, 16u, 128u, CU_TENSOR_MAP_SWIZZLE_64B)) != OPQ_OK) return s;
+        if (a.signs_tma) {
+            if ((s = make_u32_map(&smap, signs, N, K / 32, 4u, 128u, CU_TENSOR_MAP_SWIZZLE_NONE)) != OPQ_OK) return s;
+        } else {
+            smap = cmap;   // not read by the kernel
+        }
+    }
     if (a.tail_split == 2) {
         if ((s = make_x_map(&xhmap, x, M, K, (uint32_t)plan.bx / 2)) != OPQ_OK) return s;
     } else {
         xhmap = xmap;   // not read by the kernel
-    }
-    if ((s = make_u32_map(&cmap, codes, N, K / 8, 16u, 128u, CU_TENSOR_MAP_SWIZZLE_64B)) != OPQ_OK) return s;
-    // the sign plane's rows are 16-byte aligned (a TMA requirement) when K % 128 == 0; otherwise the
-    // kernel copies the sign words with cp.async
-    a.signs_tma = (K % 128 == 0) ? 1 : 0;
-    if (a.signs_tma) {
-        if ((s = make_u32_map(&smap, signs, N, K / 32, 4u, 128u, CU_TENSOR_MAP_SWIZZLE_NONE)) != OPQ_OK) return s;
-    } else {
-        smap = cmap;   // not read by the kernel
     }
     cudaError_t e;
     switch (plan.bx) {

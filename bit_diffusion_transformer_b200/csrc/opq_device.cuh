@@ -40,6 +40,11 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+// `count` arrivals at once
+__device__ __forceinline__ void mbar_arrive_count(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                  : "memory");
@@ -73,6 +78,33 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
     }
 }
 
+// ------------------------------------------------- shared-memory counters --
+// A monotonic arrival counter in shared memory, for a consumer thread that must not pay an
+// mbarrier wait per step (a wait costs an MMA-issuing thread a few hundred cycles).
+__device__ __forceinline__ void counter_add_release(uint32_t *cnt, uint32_t v) {
+    asm volatile("red.release.cta.shared::cta.add.u32 [%0], %1;" ::"r"(smem_u32(cnt)), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ uint32_t counter_load_acquire(const uint32_t *cnt) {
+    uint32_t v;
+    asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(cnt)) : "memory");
+    return v;
+}
+
+// Wait until *cnt >= target (counts are monotonic). Same time limit and error word as mbar_wait.
+__device__ __forceinline__ bool counter_wait(const uint32_t *cnt, uint32_t target) {
+    if ((int32_t)(counter_load_acquire(cnt) - target) >= 0) return true;
+    const uint64_t t0 = globaltimer();
+    while (true) {
+        for (int i = 0; i < 64; ++i)
+            if ((int32_t)(counter_load_acquire(cnt) - target) >= 0) return true;
+        if (globaltimer() - t0 > kWaitLimitNs) {
+            atomicOr(&g_error, kErrWaitTimeout);
+            return false;
+        }
+    }
+}
+
 // ----------------------------------------------------------------------- TMA --
 __device__ __forceinline__ void tma_prefetch_desc(const void *tmap) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
@@ -85,6 +117,15 @@ __device__ __forceinline__ void tma_load_2d(void *smem_dst, const void *tmap, in
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
         ::"r"(smem_u32(smem_dst)), "l"(tmap), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// 3-D tiled bulk tensor load (coordinates innermost first), completion counted on `bar`.
+__device__ __forceinline__ void tma_load_3d(void *smem_dst, const void *tmap, int32_t c0, int32_t c1, int32_t c2,
+                                            uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
+        ::"r"(smem_u32(smem_dst)), "l"(tmap), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
         : "memory");
 }
 

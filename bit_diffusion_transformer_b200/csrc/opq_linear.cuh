@@ -123,6 +123,8 @@ struct LinearArgs {
     int M, N, K;
     int m_tiles, n_tiles;
     int kblocks;            // 128-K blocks per tile
+    int ngroups;            // load groups per tile: consecutive blocks fetched by one copy per plane
+                            // (balanced sizes ceil / floor of kblocks / ngroups, never above GRP)
     int mode;               // 0 whole tiles strided over CTAs, 1 contiguous unit ranges (stream-K)
     int runs_max;           // mode 1: most runs one CTA can have
     int tail_split;         // mode 0: 2 = tiles past the last full wave run as two half-width
@@ -137,11 +139,28 @@ __host__ __device__ __forceinline__ int64_t unit_owner(int64_t u, int64_t C, int
     return ((u + 1) * C - 1) / U;
 }
 
-// The sequence of runs of one CTA; every role walks the same sequence. A run is one
-// weight tile, a range of its 128-K blocks and a range of its activation rows.
+// Load groups of a tile: ng groups of consecutive 128-K blocks, sizes as even as possible
+// (the first kb % ng groups one block longer), group g starting at block start(g).
+struct LGroups {
+    int q, rem;
+    __device__ __forceinline__ void init(int kb, int ng) {
+        q = kb / ng;
+        rem = kb - q * ng;
+    }
+    __device__ __forceinline__ int start(int g) const { return g * q + (g < rem ? g : rem); }
+};
+
+// One run of a CTA: a weight tile, a range of its load groups [g0, g1) (blocks [r0, r1)),
+// its index j among the CTA's runs, and the activation rows [xoff, xoff + xrows) of the tile.
+struct Run {
+    int tile, g0, g1, r0, r1, j, xoff, xrows;
+};
+
+// The sequence of runs of one CTA; every role walks the same sequence.
 struct RunIter {
-    int mode, tiles, kblocks, grid, cta;
-    int64_t u, u_end;   // mode 1
+    int mode, tiles, ng, grid, cta;
+    LGroups lg;
+    int64_t u, u_end;   // mode 1: units = (tile, load group)
     int t_next;         // mode 0
     int full_end;       // mode 0: tiles in whole waves (handed out strided)
     int split;          // mode 0: 1 or 2 runs per tile after the whole waves
@@ -150,7 +169,8 @@ struct RunIter {
     __device__ __forceinline__ void init(const LinearArgs &a, int tiles_, int grid_, int cta_) {
         mode = a.mode;
         tiles = tiles_;
-        kblocks = a.kblocks;
+        ng = a.ngroups;
+        lg.init(a.kblocks, a.ngroups);
         grid = grid_;
         cta = cta_;
         run_idx = 0;
@@ -158,45 +178,42 @@ struct RunIter {
         split = a.tail_split;
         full_end = split == 2 ? (tiles_ / grid_) * grid_ : tiles_;
         tail_done = false;
-        const int64_t U = (int64_t)tiles * kblocks;
+        const int64_t U = (int64_t)tiles * ng;
         u = unit_begin(cta_, grid_, U);
         u_end = unit_begin(cta_ + 1, grid_, U);
     }
-    // next run: tile, block range [r0, r1), run index j, activation rows [xoff, xoff + xrows)
-    // of the tile's bx; false at the end
-    __device__ __forceinline__ bool next(int &tile, int &r0, int &r1, int &j, int &xoff, int &xrows, int bx) {
-        xoff = 0;
-        xrows = bx;
+    // the next run for a tile of bx activation rows; false at the end
+    __device__ __forceinline__ bool next(Run &R, int bx) {
+        R.xoff = 0;
+        R.xrows = bx;
         if (mode == 0) {
             if (t_next < full_end) {
-                tile = t_next;
+                R.tile = t_next;
                 t_next += grid;
             } else if (split == 2) {
                 // tail tile t is run by CTAs 2 (t - full_end) and 2 (t - full_end) + 1, one half each
                 if (tail_done || cta >= 2 * (tiles - full_end)) return false;
-                tile = full_end + (cta >> 1);
-                xrows = bx / 2;
-                xoff = (cta & 1) * xrows;
+                R.tile = full_end + (cta >> 1);
+                R.xrows = bx / 2;
+                R.xoff = (cta & 1) * R.xrows;
                 tail_done = true;
             } else {
                 return false;
             }
-            r0 = 0;
-            r1 = kblocks;
+            R.g0 = 0;
+            R.g1 = ng;
         } else {
             if (u >= u_end) return false;
-            tile = (int)(u / kblocks);
-            r0 = (int)(u - (int64_t)tile * kblocks);
-            const int64_t end = (int64_t)r0 + (u_end - u);
-            r1 = end < (int64_t)kblocks ? (int)end : kblocks;
-            u += r1 - r0;
+            R.tile = (int)(u / ng);
+            R.g0 = (int)(u - (int64_t)R.tile * ng);
+            const int64_t end = (int64_t)R.g0 + (u_end - u);
+            R.g1 = end < (int64_t)ng ? (int)end : ng;
+            u += R.g1 - R.g0;
         }
-        j = run_idx++;
+        R.r0 = lg.start(R.g0);
+        R.r1 = lg.start(R.g1);
+        R.j = run_idx++;
         return true;
-    }
-    __device__ __forceinline__ bool next(int &tile, int &r0, int &r1, int &j) {
-        int xo, xr;
-        return next(tile, r0, r1, j, xo, xr, 2);
     }
 };
 
@@ -205,16 +222,25 @@ struct Cfg {
     static constexpr int BW = 128;                     // weight rows per tile (MMA M)
     static constexpr int KR = 128;                     // K per raw (codes/signs) stage
     static constexpr int KA = 64;                      // K per A stage (TMEM) and per x stage (smem)
-    static constexpr int RAW_STAGES = BX >= 256 ? 2 : (BX >= 128 ? 4 : 6);
+    // Blocks per load group (one TMA copy per plane and per group: under load the SM's copy
+    // engine serves a copy every few hundred ns almost whatever its size, so narrow tiles,
+    // whose per-block data is small, fetch several blocks per copy). GRP > 1 needs K % 128 == 0.
+    static constexpr int GRP = BX <= 16 ? 4 : (BX <= 64 ? 2 : 1);
+    // raw stages hold one load group each; a decoder group waiting on a stage knows only that
+    // the block three before its own was loaded, so at least three stages keep parity waits exact
+    static constexpr int RAW_STAGES = GRP > 1 ? 3 : (BX >= 256 ? 2 : (BX >= 128 ? 4 : 6));
     static constexpr int A_STAGES = 8;                 // 32 TMEM columns each (64 K of bf16 pairs)
     static constexpr int A_BLOCKS = A_STAGES / 2;      // 128-K blocks of A held in TMEM
     static constexpr int A_COLS = A_STAGES * 32;
-    // x stages hold a whole 128-K block (two 64-K swizzle atoms' worth of columns)
-    static constexpr int X_STAGES = BX >= 256 ? 2 : (BX >= 128 ? 3 : (BX >= 64 ? 4 : (BX >= 32 ? 8 : 10)));
+    // x stages hold one load group (two 64-K swizzle atoms' worth of columns per block)
+    static constexpr int X_STAGES = GRP == 4 ? 2 : (GRP == 2 ? (BX >= 64 ? 2 : 4) : (BX >= 256 ? 2 : 3));
     // One tcgen05.commit per 128-K block frees both its A slot and its x stage: a commit
     // stalls the tensor pipe for a few hundred cycles, so there is one per 8 MMAs, not per 4.
     // Slot b % NDONE of `blk_done` completes when the MMAs of the CTA's block b are done.
-    static constexpr int NDONE = X_STAGES > A_BLOCKS ? X_STAGES : A_BLOCKS;
+    // The x producer waits for the last block of the group X_STAGES groups back; with up to
+    // (X_STAGES - 1) GRP blocks in between, 1 + (X_STAGES - 1) GRP slots keep that wait exact.
+    static constexpr int NDONE_X = 1 + (X_STAGES - 1) * GRP;
+    static constexpr int NDONE = NDONE_X > A_BLOCKS ? NDONE_X : A_BLOCKS;
     // independent accumulation chains per tile: consecutive MMAs into one accumulator
     // serialize on its latency, which dominates when N (= BX) is small; K-step k of a
     // stage goes to chain k % NCHAIN and the epilogue adds the chains in a fixed order
@@ -222,19 +248,21 @@ struct Cfg {
     static constexpr int ACC_COLS = NCHAIN * BX;       // one accumulator buffer (all chains)
     static constexpr int NACC = (A_COLS + 2 * ACC_COLS <= 512) ? 2 : 1;   // accumulator buffers
     static constexpr uint32_t TMEM_COLS = 512;
-    static constexpr int RAW_CODE_BYTES = BW * KR / 2;    // 8 KiB: [128 rows][16 words], 64-byte swizzle
-    static constexpr int RAW_SIGN_BYTES = BW * KR / 8;    // 2 KiB: [128 rows][4 words]
-    static constexpr int RAW_BYTES = RAW_CODE_BYTES + RAW_SIGN_BYTES;
+    static constexpr int BLK_CODE_BYTES = BW * KR / 2;    // 8 KiB per block: [128 rows][16 words], 64-byte swizzle
+    static constexpr int BLK_SIGN_BYTES = BW * KR / 8;    // 2 KiB per block: [128 rows][4 words]
+    static constexpr int RAW_CODE_BYTES = GRP * BLK_CODE_BYTES;   // a stage: GRP blocks of codes, then of signs
+    static constexpr int RAW_BYTES = GRP * (BLK_CODE_BYTES + BLK_SIGN_BYTES);
     static constexpr int X_HALF_BYTES = BX * KA * 2;   // one 64-K half: BX rows x 128 bytes, 128-byte swizzle
-    static constexpr int X_BYTES = 2 * X_HALF_BYTES;
+    static constexpr int X_BYTES = GRP * 2 * X_HALF_BYTES;   // a stage: the group's halves in K order
     static constexpr int STAGE_EPI_BYTES = 4 * 2 * 16 * 32 * 2;   // 4 warps x 2 buffers x [16 m][32 n] bf16
     static constexpr int OFF_TABLE = 0;
     static constexpr int OFF_RAW = OFF_TABLE + (int)opqbits::kPairTableBytes;
     static constexpr int OFF_X = OFF_RAW + RAW_STAGES * RAW_BYTES;
     static constexpr int OFF_EPI = OFF_X + X_STAGES * X_BYTES;
     static constexpr int OFF_BAR = OFF_EPI + STAGE_EPI_BYTES;
-    static constexpr int NUM_BARS = 2 * RAW_STAGES + X_STAGES + A_STAGES + NDONE + 2 * NACC + 1;
-    static constexpr int OFF_TMEM = OFF_BAR + NUM_BARS * 8;
+    static constexpr int NUM_BARS = 2 * RAW_STAGES + X_STAGES + NDONE + 2 * NACC + 1;
+    static constexpr int OFF_CNT = OFF_BAR + NUM_BARS * 8;     // A-stage ready counters
+    static constexpr int OFF_TMEM = OFF_CNT + A_STAGES * 4;
     static constexpr int SMEM_BYTES = OFF_TMEM + 16 + 1024;
     // decoder groups of 4 warps: group g decodes the CTA's 128-K blocks g, g + G, ...;
     // thread r of a group owns weight row r (TMEM lane r) and decodes its whole 128-K block row
@@ -274,8 +302,10 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
     uint64_t *raw_full = bars;
     uint64_t *raw_empty = raw_full + C::RAW_STAGES;
     uint64_t *x_full = raw_empty + C::RAW_STAGES;
-    uint64_t *a_full = x_full + C::X_STAGES;
-    uint64_t *blk_done = a_full + C::A_STAGES;
+    uint64_t *blk_done = x_full + C::X_STAGES;
+    // a_ready[s]: arrivals of decoder warps on A half-stage s (4 per fill, monotonic), polled by
+    // the MMA issuers with plain acquire loads
+    uint32_t *a_ready = reinterpret_cast<uint32_t *>(smem + C::OFF_CNT);
     uint64_t *acc_full = blk_done + C::NDONE;
     uint64_t *acc_empty = acc_full + C::NACC;
     uint64_t *drain = acc_empty + C::NACC;
@@ -285,24 +315,15 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
     const int tiles = args.m_tiles * args.n_tiles;
     const bool signs_by_tma = args.signs_tma != 0;
 
-    // ---- pair table: 32 copies of value(b) then 32 copies of spread(b) per entry b
-    for (int e = threadIdx.x; e < 512; e += C::THREADS) {
-        const uint32_t b = (uint32_t)e & 255u;
-        const uint32_t v = e < 256 ? ((uint32_t)args.lut[b & 15u] | ((uint32_t)args.lut[b >> 4] << 16))
-                                   : opqbits::sign_spread(b);
-        const uint32_t dst = sbase + C::OFF_TABLE + b * 256u + (e < 256 ? 0u : 128u);
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst + 16u * k), "r"(v) : "memory");
-    }
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::RAW_STAGES; ++s) {
-            // the codes' (and signs') expect_tx arrival, plus 32 cp.async arrivals when signs are copied by threads
-            mbar_init(&raw_full[s], signs_by_tma ? 1 : 1 + 32);
-            mbar_init(&raw_empty[s], 4);          // the 4 warps of the group that decodes the block
+            // the copies' expect_tx arrival, plus 32 cp.async arrivals when signs are copied by threads
+            mbar_init(&raw_full[s], (C::GRP > 1 || signs_by_tma) ? 1 : 1 + 32);
+            // the 4 warps of the decoding group, once per block of the stage's load group
+            mbar_init(&raw_empty[s], 4 * C::GRP);
         }
         for (int s = 0; s < C::X_STAGES; ++s) mbar_init(&x_full[s], 1);
-        for (int s = 0; s < C::A_STAGES; ++s) mbar_init(&a_full[s], 4);   // the 4 warps of the decoding group
+        for (int s = 0; s < C::A_STAGES; ++s) a_ready[s] = 0u;
         for (int s = 0; s < C::NDONE; ++s) mbar_init(&blk_done[s], C::NISS);   // one commit per issuer
         for (int s = 0; s < C::NACC; ++s) {
             mbar_init(&acc_full[s], C::NISS);
@@ -330,18 +351,21 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
 
     RunIter it;
     it.init(args, tiles, gridDim.x, blockIdx.x);
-    int tile, r0, r1, j;
+    Run R;
+    const LGroups lg = it.lg;
 
     if (warp == C::WARP_LOAD) {
         // ----------------------------------------------------------- raw producer
+        // one stage per load group: GRP blocks of codes and of signs
         const int swd = args.K / 32;        // sign words per row
         int rs = 0;
         uint32_t rph = 0;
         int raw_issued = 0;
         bool ok = true;
-        while (ok && it.next(tile, r0, r1, j)) {
-            const int n_blk = tile / args.m_tiles;
-            for (int r = r0; r < r1 && ok; ++r) {
+        while (ok && it.next(R, BX)) {
+            const int n_blk = R.tile / args.m_tiles;
+            for (int g = R.g0; g < R.g1 && ok; ++g) {
+                const int r = lg.start(g), nb = lg.start(g + 1) - r;
                 // lane 0 waits for the stage; the verdict and the ordering reach the other lanes
                 int okw = 1;
                 if (lane == 0) okw = mbar_wait(&raw_empty[rs], rph ^ 1) ? 1 : 0;
@@ -350,14 +374,26 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
                 if (!okw) { ok = false; break; }
                 const uint32_t dst = sbase + C::OFF_RAW + rs * C::RAW_BYTES;
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(&raw_full[rs], signs_by_tma ? C::RAW_BYTES : C::RAW_CODE_BYTES);
-                    tma_load_2d(smem + C::OFF_RAW + rs * C::RAW_BYTES, &tmap_codes, r * (C::KR / 8), n_blk * C::BW,
-                                &raw_full[rs]);
-                    if (signs_by_tma)
-                        tma_load_2d(smem + C::OFF_RAW + rs * C::RAW_BYTES + C::RAW_CODE_BYTES, &tmap_signs,
-                                    r * (C::KR / 32), n_blk * C::BW, &raw_full[rs]);
+                    uint8_t *sd = smem + C::OFF_RAW + rs * C::RAW_BYTES;
+                    if (C::GRP > 1) {
+                        // 3-D boxes {words, 128 rows, GRP blocks}: the group's blocks one after the
+                        // other (blocks past the tile's end read as zero, blocks of the next group
+                        // are fetched and not used)
+                        mbar_arrive_expect_tx(&raw_full[rs], C::RAW_BYTES);
+                        tma_load_3d(sd, &tmap_codes, 0, n_blk * C::BW, r, &raw_full[rs]);
+                        tma_load_3d(sd + C::RAW_CODE_BYTES, &tmap_signs, 0, n_blk * C::BW, r, &raw_full[rs]);
+                        // the decoders arrive once per block and warp: supply the arrivals of the
+                        // group's missing blocks so that the stage's phase can complete
+                        if (nb < C::GRP) mbar_arrive_count(&raw_empty[rs], 4u * (uint32_t)(C::GRP - nb));
+                    } else {
+                        mbar_arrive_expect_tx(&raw_full[rs], signs_by_tma ? C::RAW_BYTES : C::RAW_CODE_BYTES);
+                        tma_load_2d(sd, &tmap_codes, r * (C::KR / 8), n_blk * C::BW, &raw_full[rs]);
+                        if (signs_by_tma)
+                            tma_load_2d(sd + C::RAW_CODE_BYTES, &tmap_signs, r * (C::KR / 32), n_blk * C::BW,
+                                        &raw_full[rs]);
+                    }
                 }
-                if (!signs_by_tma) {
+                if (C::GRP == 1 && !signs_by_tma) {
                     // sign words: 128 rows x 4 words; copy i of lane l is word 32 i + l of the stage
                     // (consecutive lanes, consecutive banks); out-of-range words read as 0
 #pragma unroll
@@ -389,33 +425,44 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
         // ----------------------------------------------------------- x producer
         if (lane == 0) {
             int b = 0;                 // the CTA's block index
+            int v = 0;                 // the CTA's load-group index
+            int last_blk[C::X_STAGES]; // last block of the group each x stage holds
             bool ok = true;
-            int xoff, xrows;
-            while (ok && it.next(tile, r0, r1, j, xoff, xrows, BX)) {
-                const int m_blk = tile % args.m_tiles;
+            while (ok && it.next(R, BX)) {
+                const int m_blk = R.tile % args.m_tiles;
                 // a half-width run loads its BX/2 activation rows with the half-height box
-                const bool half = xrows != BX;
+                const bool half = R.xrows != BX;
                 const void *xmap = half ? (const void *)&tmap_xh : (const void *)&tmap_x;
                 const uint32_t xbytes = half ? C::X_BYTES / 2 : C::X_BYTES;
-                const int xrow = m_blk * BX + xoff;
-                for (int r = r0; r < r1; ++r, ++b) {
-                    // stage b % X_STAGES last held block b - X_STAGES
-                    const int prev = b - C::X_STAGES;
-                    if (prev >= 0 && !mbar_wait(&blk_done[prev % C::NDONE], (uint32_t)(prev / C::NDONE) & 1u)) {
-                        ok = false;
-                        break;
+                const int xrow = m_blk * BX + R.xoff;
+                for (int g = R.g0; g < R.g1; ++g, ++v) {
+                    const int r = lg.start(g), nb = lg.start(g + 1) - r;
+                    const int xs = v % C::X_STAGES;
+                    // the stage last held group v - X_STAGES: wait until its last block's MMAs are done
+                    if (v >= C::X_STAGES) {
+                        const int prev = last_blk[xs];
+                        if (!mbar_wait(&blk_done[prev % C::NDONE], (uint32_t)(prev / C::NDONE) & 1u)) {
+                            ok = false;
+                            break;
+                        }
                     }
-                    const int xs = b % C::X_STAGES;
                     mbar_arrive_expect_tx(&x_full[xs], xbytes);
                     uint8_t *dst = smem + C::OFF_X + xs * C::X_BYTES;
-                    tma_load_2d(dst, xmap, r * C::KR, xrow, &x_full[xs]);
-                    tma_load_2d(dst + C::X_HALF_BYTES, xmap, r * C::KR + C::KA, xrow, &x_full[xs]);
+                    if (C::GRP > 1) {
+                        // box {64, BX, 2 GRP}: the group's 64-K halves one after the other
+                        tma_load_3d(dst, xmap, 0, xrow, 2 * r, &x_full[xs]);
+                    } else {
+                        tma_load_2d(dst, xmap, r * C::KR, xrow, &x_full[xs]);
+                        tma_load_2d(dst + C::X_HALF_BYTES, xmap, r * C::KR + C::KA, xrow, &x_full[xs]);
+                    }
+                    b += nb;
+                    last_blk[xs] = b - 1;
                 }
             }
             if (!ok) {
                 // let the copies already issued land before the CTA can exit
-                for (int i = 1; i <= C::X_STAGES && b - i >= 0; ++i)
-                    (void)mbar_wait(&x_full[(b - i) % C::X_STAGES], (uint32_t)((b - i) / C::X_STAGES) & 1u);
+                for (int i = 1; i <= C::X_STAGES && v - i >= 0; ++i)
+                    (void)mbar_wait(&x_full[(v - i) % C::X_STAGES], (uint32_t)((v - i) / C::X_STAGES) & 1u);
             }
         }
     } else if (warp == C::WARP_MMA || warp >= C::WARP_ISS1) {
@@ -426,39 +473,45 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
             int ab = 0;
             uint32_t abph = 0;
             int as0 = 0, xs = 0, ds = 0;       // A half-stage of the block's first half, x stage, blk_done slot
-            uint32_t aph = 0, xph = 0;
+            uint32_t aph_n = 0, xph = 0;       // fills of the A ring so far, x ring parity
             bool ok = true;
             constexpr uint32_t idesc_full = idesc_bf16_f32(128, BX);
             constexpr uint32_t idesc_half = idesc_bf16_f32(128, BX / 2);
-            int xoff, xrows;
-            while (ok && it.next(tile, r0, r1, j, xoff, xrows, BX)) {
-                const uint32_t idesc = xrows == BX ? idesc_full : idesc_half;
+            while (ok && it.next(R, BX)) {
+                const uint32_t idesc = R.xrows == BX ? idesc_full : idesc_half;
                 if (!mbar_wait(&acc_empty[ab], abph ^ 1)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + C::A_COLS + ab * C::ACC_COLS + iss * BX;
                 uint32_t acc = 0;              // 0 for the chain's first MMA of the run
-                for (int r = r0; r < r1; ++r) {
-                    const uint32_t xaddr = sbase + C::OFF_X + xs * C::X_BYTES;
+                for (int g = R.g0; g < R.g1 && ok; ++g) {
+                    const int nb = lg.start(g + 1) - lg.start(g);
+                    if (!mbar_wait(&x_full[xs], xph)) { ok = false; break; }
+                    const uint32_t xbase = sbase + C::OFF_X + xs * C::X_BYTES;
+                    for (int jj = 0; jj < nb; ++jj) {
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        if (!mbar_wait(&a_full[as0 + h], aph)) { ok = false; break; }
-                        if (h == 0 && !mbar_wait(&x_full[xs], xph)) { ok = false; break; }
-                        tc_fence_after();
-                        const uint32_t a_tmem = tmem_base + (as0 + h) * 32;
-                        const uint64_t bdesc = smem_desc_sw128(xaddr + h * C::X_HALF_BYTES);
+                        for (int h = 0; h < 2; ++h) {
+                            // fill number aph_n of this half-stage: 4 decoder-warp arrivals each
+                            if (!counter_wait(&a_ready[as0 + h], 4u * (aph_n + 1u))) { ok = false; break; }
+                            tc_fence_after();
+                            const uint32_t a_tmem = tmem_base + (as0 + h) * 32;
+                            const uint64_t bdesc = smem_desc_sw128(xbase + (2 * jj + h) * C::X_HALF_BYTES);
+                            // K-steps iss, iss + NISS, ...: a fixed count per issuer and no branch
+                            // between the MMAs (a branch around tcgen05.mma costs the issuing
+                            // thread far more than the MMA itself)
 #pragma unroll
-                        for (int k = 0; k < C::KA / 16; ++k) {
-                            if (k % C::NISS != iss % C::NISS) continue;
-                            umma_bf16_ts(d_tmem, a_tmem + 8 * k, bdesc + 2 * k, idesc, acc);
-                            acc = 1;
+                            for (int t = 0; t < C::KA / 16 / C::NISS; ++t) {
+                                const int k = iss + t * C::NISS;
+                                umma_bf16_ts(d_tmem, a_tmem + 8 * k, bdesc + 2 * k, idesc, acc);
+                                acc = 1;
+                            }
                         }
+                        if (!ok) break;
+                        umma_commit(&blk_done[ds]);
+                        as0 += 2;
+                        if (as0 == C::A_STAGES) { as0 = 0; ++aph_n; }
+                        if (++ds == C::NDONE) ds = 0;
                     }
-                    if (!ok) break;
-                    umma_commit(&blk_done[ds]);
-                    as0 += 2;
-                    if (as0 == C::A_STAGES) { as0 = 0; aph ^= 1; }
                     if (++xs == C::X_STAGES) { xs = 0; xph ^= 1; }
-                    if (++ds == C::NDONE) ds = 0;
                 }
                 if (ok) umma_commit(&acc_full[ab]);
                 if (++ab == C::NACC) { ab = 0; abph ^= 1; }
@@ -469,7 +522,20 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
         }
     } else if (warp < C::WARP_EPI0) {
         // ----------------------------------------------------------- decoders
-        const int g = (warp - C::WARP_DEC0) >> 2;        // decoder group
+        // The pair table (only the decoders read it) is built here, while the producers' first
+        // copies are in flight: 32 copies of value(b) then 32 copies of spread(b) per entry b.
+        for (int e = threadIdx.x - C::WARP_DEC0 * 32; e < 512; e += C::NUM_DEC_WARPS * 32) {
+            const uint32_t b = (uint32_t)e & 255u;
+            const uint32_t v = e < 256 ? ((uint32_t)args.lut[b & 15u] | ((uint32_t)args.lut[b >> 4] << 16))
+                                       : opqbits::sign_spread(b);
+            const uint32_t dst = sbase + C::OFF_TABLE + b * 256u + (e < 256 ? 0u : 128u);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst + 16u * k), "r"(v) : "memory");
+        }
+        // all decoder warps (named barrier 1) see the whole table before decoding
+        asm volatile("bar.sync 1, %0;" ::"r"(C::NUM_DEC_WARPS * 32) : "memory");
+        const int g_dec = (warp - C::WARP_DEC0) >> 2;    // decoder group
         const int q = warp & 3;                          // TMEM lane quarter this warp may access
         const int row = q * 32 + lane;                   // weight row in the tile = TMEM lane
         const uint32_t lw = 4u * lane, lw2 = 128u + 4u * lane;
@@ -478,69 +544,77 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
         // 64-byte swizzle of the codes stage: 16-byte chunk c of row r sits at chunk c ^ ((r >> 1) & 3)
         const uint32_t sw64 = (uint32_t)((row >> 1) & 3);
         const uint32_t tm_row = tmem_base + ((uint32_t)(q * 32) << 16);
-        int nblocks = 0;
-        while (it.next(tile, r0, r1, j)) nblocks += r1 - r0;
         bool ok = true;
-        for (int blk = g; blk < nblocks && ok; blk += C::GROUPS) {
-            const int rs = blk % C::RAW_STAGES;
-            const uint32_t rph = (uint32_t)(blk / C::RAW_STAGES) & 1u;
-            if (!warp_wait(&raw_full[rs], rph)) { ok = false; break; }
-            const uint8_t *rawc = smem + C::OFF_RAW + rs * C::RAW_BYTES + row * (C::KR / 2);
-            const uint8_t *raws = smem + C::OFF_RAW + rs * C::RAW_BYTES + C::RAW_CODE_BYTES + row * (C::KR / 8);
+        int blk = 0;                 // the CTA's block index
+        int u = 0;                   // the CTA's load-group index (= raw stage use)
+        // group g_dec decodes the CTA's blocks g_dec, g_dec + GROUPS, ...
+        while (ok && it.next(R, BX)) {
+            for (int g = R.g0; g < R.g1 && ok; ++g, ++u) {
+                const int nb = lg.start(g + 1) - lg.start(g);
+                const int rs = u % C::RAW_STAGES;
+                const uint32_t rph = (uint32_t)(u / C::RAW_STAGES) & 1u;
+                for (int jj = 0; jj < nb; ++jj, ++blk) {
+                    if (blk % C::GROUPS != g_dec) continue;
+                    if (!warp_wait(&raw_full[rs], rph)) { ok = false; break; }
+                    const uint8_t *rawc = smem + C::OFF_RAW + rs * C::RAW_BYTES + jj * C::BLK_CODE_BYTES + row * (C::KR / 2);
+                    uint32_t cw[16];
 #pragma unroll
-            for (int h = 0; h < C::KR / C::KA; ++h) {     // two 64-K A stages per block
-                const int sidx = blk * 2 + h;
-                const int as = sidx % C::A_STAGES;
-                // this half's 8 code words (two 16-byte chunks) and 2 sign words
-                uint32_t cw[8];
-#pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    const uint4 v = *reinterpret_cast<const uint4 *>(rawc + ((((uint32_t)(2 * h + c)) ^ sw64) << 4));
-                    cw[4 * c] = v.x; cw[4 * c + 1] = v.y; cw[4 * c + 2] = v.z; cw[4 * c + 3] = v.w;
-                }
-                const uint2 sv = *reinterpret_cast<const uint2 *>(raws + 8 * h);
-                const uint32_t sw[2] = {sv.x, sv.y};
-                if (h == 1) {
+                    for (int c = 0; c < 4; ++c) {
+                        const uint4 vv = *reinterpret_cast<const uint4 *>(rawc + ((((uint32_t)c) ^ sw64) << 4));
+                        cw[4 * c] = vv.x; cw[4 * c + 1] = vv.y; cw[4 * c + 2] = vv.z; cw[4 * c + 3] = vv.w;
+                    }
+                    const uint4 sv = *reinterpret_cast<const uint4 *>(smem + C::OFF_RAW + rs * C::RAW_BYTES +
+                                                                     C::RAW_CODE_BYTES + jj * C::BLK_SIGN_BYTES +
+                                                                     row * (C::KR / 8));
+                    const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&raw_empty[rs]);   // the block's raw words are in registers now
-                }
-                uint32_t o[2][16];
+                    if (lane == 0) mbar_arrive(&raw_empty[rs]);   // the raw words are in registers now
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    uint32_t t4[4];
-                    opqbits::decode8_table(cw[i], sw[i >> 2], (uint32_t)(i & 3), lw, lw2, load, t4);
+                    for (int h = 0; h < C::KR / C::KA; ++h) {     // two 64-K A stages per block
+                        const int sidx = blk * 2 + h;
+                        const int as = sidx % C::A_STAGES;
+                        uint32_t o[2][16];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) o[i >> 2][(i & 3) * 4 + e] = t4[e];
+                        for (int i = 0; i < 8; ++i) {
+                            const int w = 8 * h + i;
+                            uint32_t t4[4];
+                            opqbits::decode8_table(cw[w], sw[w >> 2], (uint32_t)(w & 3), lw, lw2, load, t4);
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) o[i >> 2][(i & 3) * 4 + e] = t4[e];
+                        }
+                        // the block's A slot last held block blk - A_BLOCKS
+                        const int prev = blk - C::A_BLOCKS;
+                        if (h == 0 && prev >= 0 &&
+                            !warp_wait(&blk_done[prev % C::NDONE], (uint32_t)(prev / C::NDONE) & 1u)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        tmem_st_32x32b_x16(tm_row + as * 32, o[0]);
+                        tmem_st_32x32b_x16(tm_row + as * 32 + 16, o[1]);
+                        tmem_st_wait();
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) counter_add_release(&a_ready[as], 1u);
+                    }
+                    if (!ok) break;
                 }
-                // the block's A slot last held block blk - A_BLOCKS
-                const int prev = blk - C::A_BLOCKS;
-                if (h == 0 && prev >= 0 &&
-                    !warp_wait(&blk_done[prev % C::NDONE], (uint32_t)(prev / C::NDONE) & 1u)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                tmem_st_32x32b_x16(tm_row + as * 32, o[0]);
-                tmem_st_32x32b_x16(tm_row + as * 32 + 16, o[1]);
-                tmem_st_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&a_full[as]);
+                if (!ok) break;
             }
         }
     } else {
         // ----------------------------------------------------------- epilogue
         const int q = warp & 3;
         const int row = q * 32 + lane;
-        const int64_t U = (int64_t)tiles * args.kblocks;
+        const int64_t U = (int64_t)tiles * args.ngroups;
         const bool vec_y = (args.N % 8) == 0;
         // per-warp staging for y: 2 buffers of [16 m][32 n] bf16
         const uint32_t stage0 = sbase + C::OFF_EPI + (uint32_t)(warp - C::WARP_EPI0) * 2048u;
         int ab = 0;
         uint32_t abph = 0;
         int sb = 0;
-        int xoff, xrows;
-        while (it.next(tile, r0, r1, j, xoff, xrows, BX)) {
+        while (it.next(R, BX)) {
+            const int tile = R.tile, r0 = R.r0, r1 = R.r1, j = R.j, xoff = R.xoff, xrows = R.xrows;
             const int n_blk = tile / args.m_tiles, m_blk = tile % args.m_tiles;
             const int n = n_blk * C::BW + row;
             const int n0 = n_blk * C::BW + q * 32;           // first row of this warp's quarter
@@ -609,8 +683,8 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
             if (!full) {
                 // The last of the tile's CTAs to get here (per lane quarter) adds every
                 // CTA's partial rows in CTA order, so the sum does not depend on timing.
-                const int64_t c_lo = unit_owner((int64_t)tile * args.kblocks, gridDim.x, U);
-                const int64_t c_hi = unit_owner((int64_t)(tile + 1) * args.kblocks - 1, gridDim.x, U);
+                const int64_t c_lo = unit_owner((int64_t)tile * args.ngroups, gridDim.x, U);
+                const int64_t c_hi = unit_owner((int64_t)(tile + 1) * args.ngroups - 1, gridDim.x, U);
                 const uint32_t parts = (uint32_t)(c_hi - c_lo + 1);
                 __threadfence();
                 __syncwarp();
@@ -623,7 +697,7 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
                     const float *mybase = nullptr;
                     if ((uint32_t)lane < parts) {
                         const int64_t c = c_lo + lane;
-                        const int64_t jj = tile - unit_begin(c, gridDim.x, U) / args.kblocks;
+                        const int64_t jj = tile - unit_begin(c, gridDim.x, U) / args.ngroups;
                         mybase = args.ws + ((size_t)c * args.runs_max + (size_t)jj) * (size_t)(BX * C::BW);
                     }
                     // Every lane runs the loops (shuffles need all lanes); only rows < N store.
@@ -634,7 +708,7 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
                             return reinterpret_cast<const float *>(
                                 __shfl_sync(0xFFFFFFFFu, reinterpret_cast<unsigned long long>(mybase), (int)p));
                         const int64_t c = c_lo + p;
-                        const int64_t jj = tile - unit_begin(c, gridDim.x, U) / args.kblocks;
+                        const int64_t jj = tile - unit_begin(c, gridDim.x, U) / args.ngroups;
                         return args.ws + ((size_t)c * args.runs_max + (size_t)jj) * (size_t)(BX * C::BW);
                     };
                     const int mcols = min(BX, args.M - m_blk * BX);
@@ -674,6 +748,9 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
         }
     }
 
+    // roles run on single lanes: reconverge every warp before the CTA barrier, so that the
+    // barrier (and the warp-wide TMEM release after it) waits for every lane's last operation
+    __syncwarp();
     tc_fence_before();
     __syncthreads();
     if (warp == C::WARP_MMA) {

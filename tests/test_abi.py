@@ -90,16 +90,22 @@ def test_dequantize_and_linear_argument_errors(lib):
 
 
 def test_plan_and_workspace_host_logic(lib):
-    # small M: stream-K over (128-row weight tile, 128-K block) units on at most 148 CTAs
+    # small M: stream-K over (128-row weight tile, load group) units on at most 148 CTAs; a load
+    # group is 4 (16-row tiles), 2 (32- and 64-row tiles) or 1 consecutive 128-K blocks, the
+    # tile's blocks split into ceil(blocks / group) groups; narrow tiles need K % 128 == 0
     for M, N, K in [(1, 11520, 3840), (16, 11520, 3840), (64, 11520, 3840), (128, 11520, 3840),
-                    (1, 3840, 3840), (17, 257, 96), (1, 64, 32)]:
+                    (1, 3840, 3840), (17, 257, 96), (1, 64, 32), (5, 300, 640), (40, 1000, 160)]:
         path, ctas, launches = opq.plan(M, N, K)
         assert path == 1 and launches == 1
         bx = 16 if M <= 16 else 32 if M <= 32 else 64 if M <= 64 else 128
-        units = -(-N // 128) * -(-K // 128)
+        if K % 128:
+            bx = 128
+        grp = 4 if bx <= 16 else 2 if bx <= 64 else 1
+        groups = -(-(-(-K // 128)) // grp)
+        units = -(-N // 128) * groups
         assert ctas == min(148, units)
         per = -(-units // ctas)
-        runs_max = -(-per // -(-K // 128)) + 1
+        runs_max = -(-per // groups) + 1
         counters = 4096 * 4 * 4        # fixed region: 4 arrival counters for each of up to 4096 weight tiles
         assert opq.workspace_size(M, N, K) == counters + ctas * runs_max * bx * 128 * 4
     # large M: whole 128 x 256 tiles, one persistent CTA per SM, no workspace

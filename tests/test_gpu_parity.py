@@ -218,6 +218,25 @@ def test_linear_alpha(alpha):
     linear_parity(x, w, alpha)
 
 
+@pytest.mark.parametrize("M", [1, 16, 33, 64])
+@pytest.mark.parametrize("N,K", [(300, 384), (1000, 640), (130, 128), (2000, 1152)])
+def test_linear_load_groups(M, N, K):
+    # narrow tiles fetch 2 or 4 consecutive 128-K blocks per copy; K = 128 (one block), 384
+    # (a group shorter than the copy), 640 (groups of 3 and 2) and 1152 (three groups of 3)
+    lin = workloads.Linear("groups", M, N, K, w_seed=3 * M + N, x_seed=5 * M + K)
+    x, w = lin.make("cpu")
+    linear_parity(x, w, 0.73)
+
+
+@pytest.mark.parametrize("M,N,K", [(16, 8192, 1152), (40, 9000, 640)])
+def test_linear_load_groups_split_tiles(M, N, K):
+    # more (tile, load group) units than CTAs: tiles shared by several CTAs, partial sums added
+    # in CTA order
+    lin = workloads.Linear("groups-split", M, N, K, w_seed=N, x_seed=M)
+    x, w = lin.make("cpu")
+    linear_parity(x, w, 0.73)
+
+
 @pytest.mark.parametrize("M,N,K", [(512, 10240, 256), (300, 9728, 160)])
 def test_linear_tail_split(M, N, K):
     # more tiles than one wave of CTAs, with the leftover tiles (at most half a wave) each
