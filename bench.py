@@ -30,7 +30,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_SOURCES = ["bit_diffusion_transformer_b200/csrc/opq_linear.cuh", "bit_diffusion_transformer_b200/csrc/opq_bits.h",
+KERNEL_SOURCES = ["bit_diffusion_transformer_b200/csrc/opq_linear_wide.cuh",
+                  "bit_diffusion_transformer_b200/csrc/opq_linear.cuh", "bit_diffusion_transformer_b200/csrc/opq_bits.h",
                   "bit_diffusion_transformer_b200/csrc/opq_device.cuh"]
 METRIC = "opq_linear TFLOP/s (% bf16 peak) & quantize/small-M weight GB/s (% HBM)"
 
@@ -315,8 +316,8 @@ def gpu_arm(args, rank, world, local_rank):
         ms_e2e = float(t.item())
     barrier()
 
-    traffic = recorded_traffic("linear_kernel")
-    roof = {"bound": "tensor", "kernel": "linear_kernel<256>", "achieved": linear_tflops,
+    traffic = recorded_traffic("wide_kernel")
+    roof = {"bound": "tensor", "kernel": "wide_kernel<256>", "achieved": linear_tflops,
             "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": linear_tflops / peaks["bf16_tflops"],
             "traffic": traffic, "algorithmic_flops": flops, "algorithmic_bytes": l_bytes,
             "launch_ms": t_l, "peak_source": f"bf16 dense burst, {peak_src}"}

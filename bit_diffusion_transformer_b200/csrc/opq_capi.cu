@@ -13,6 +13,7 @@
 #include "opq.h"
 #include "opq_dequantize.cuh"
 #include "opq_linear.cuh"
+#include "opq_linear_wide.cuh"
 #include "opq_quantize.cuh"
 
 namespace {
@@ -295,6 +296,38 @@ cudaError_t launch_linear(DeviceInfo *di, const Plan &plan, const CUtensorMap &x
     return cudaGetLastError();
 }
 
+// the wide-tile kernel (256 activation rows per tile, whole tiles, one block per copy)
+cudaError_t launch_linear_wide(DeviceInfo *di, const Plan &plan, const CUtensorMap &xmap, const CUtensorMap &xhmap,
+                               const CUtensorMap &cmap, const CUtensorMap &smap, const opqk::LinearArgs &n,
+                               cudaStream_t st) {
+    using C = opqk_wide::Cfg<256>;
+    opqk_wide::LinearArgs a{};
+    a.signs = n.signs;
+    a.scales = n.scales;
+    a.y = n.y;
+    a.ws = n.ws;
+    a.counters = n.counters;
+    a.signs_tma = n.signs_tma;
+    a.M = n.M;
+    a.N = n.N;
+    a.K = n.K;
+    a.m_tiles = n.m_tiles;
+    a.n_tiles = n.n_tiles;
+    a.kblocks = n.kblocks;
+    a.mode = n.mode;
+    a.runs_max = n.runs_max;
+    a.tail_split = n.tail_split;
+    for (int i = 0; i < 16; ++i) a.lut[i] = n.lut[i];
+    if (!di->linear_attr[16]) {
+        cudaError_t e = cudaFuncSetAttribute(opqk_wide::wide_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             C::SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        di->linear_attr[16] = true;
+    }
+    opqk_wide::wide_kernel<256><<<plan.grid, C::THREADS, C::SMEM_BYTES, st>>>(xmap, xhmap, cmap, smap, a);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 extern "C" {
@@ -463,7 +496,7 @@ opq_status opq_linear(const uint16_t *x, int64_t M, int64_t K, const uint32_t *c
         case 32: e = launch_linear<32>(di, plan, xmap, xhmap, cmap, smap, a, st); break;
         case 64: e = launch_linear<64>(di, plan, xmap, xhmap, cmap, smap, a, st); break;
         case 128: e = launch_linear<128>(di, plan, xmap, xhmap, cmap, smap, a, st); break;
-        default: e = launch_linear<256>(di, plan, xmap, xhmap, cmap, smap, a, st); break;
+        default: e = launch_linear_wide(di, plan, xmap, xhmap, cmap, smap, a, st); break;
     }
     if (e != cudaSuccess) return cuda_fail(e);
     e = cudaGetLastError();

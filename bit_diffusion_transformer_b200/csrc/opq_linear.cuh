@@ -1,37 +1,36 @@
-// opq_linear.cuh — y = x W'^T with W' decoded on the fly from the OPQ planes.
+// opq_linear.cuh — y = x W'^T with W' decoded on the fly from the OPQ planes,
+// for narrow activation tiles (M <= 128: the weight-streaming regime).
 //
 // "OPQ INT4 Z-Image" model card: the OPQLinear forward decodes
 // w = sign * (q/15)^(1/alpha) * max ("inference decoding") and multiplies.
 // Here the row scale max is deferred to the epilogue: the tensor cores see
 // sign * bf16((q/15)^(1/alpha)) and each fp32 sum is multiplied by scale[n] once.
 //
-// One kernel, templated on BX (activation rows per tile, 16..256):
+// One kernel, templated on BX (activation rows per tile, 16..128):
 //
 //   D^T[128 x BX] = W'_tile[128 x K] * x_tile[BX x K]^T     (tcgen05, kind::f16)
 //
 // Weights sit on the MMA's 128-row side so that each decoded weight meets BX
 // activation rows. Per CTA (one per SM, persistent):
-//   warp 0       raw producer: packed codes of 128 weight rows x 128 K by TMA
-//                (64-byte swizzle), their sign words by cp.async (the sign plane's
-//                row stride need not be 16-byte aligned)
-//   warp 1       TMEM allocation and the single-thread MMA issue; A comes from TMEM
-//   warp 2       x producer: x tiles (BX rows x 64 K, 128-byte swizzle) by TMA, on
-//                its own thread so that neither ring throttles the other
-//   warps 3..10  decoders: two threads per weight row, 32 weights each per 64-K
-//                stage, through the shared-memory pair table (opq_bits.h), written
-//                to TMEM with tcgen05.st as the MMA's A operand; the store of one
-//                stage drains while the next stage is decoded
-//   warps 11..14 epilogue: accumulator TMEM -> registers -> * scale[n] -> bf16 y,
+//   warp 0       raw producer: codes (64-byte swizzle) and signs of 128 weight rows,
+//                one load group (GRP consecutive 128-K blocks) per pair of TMA copies
+//   warp 1       TMEM allocation and MMA issue (chain 0); A comes from TMEM
+//   warp 2       x producer: the load group's x (BX rows, 128-byte swizzle), one copy
+//   warps 3..14  three decoder groups of 4 warps (= the 128 TMEM lanes): each thread owns
+//                one weight row and decodes 128 weights per block through the shared-memory
+//                pair table (opq_bits.h), written to TMEM with tcgen05.st as the A operand
+//   warps 15..18 epilogue: accumulator TMEM -> registers -> * scale[n] -> bf16 y,
 //                or fp32 partial sums for tiles split across CTAs
-// TMEM columns: [0, 256) eight 64-K A stages; [256, 256 + NACC * BX) accumulators.
+//   warps 19..   the other accumulation chains' MMA issuers (narrow tiles)
+// TMEM columns: [0, A_COLS) the A ring; then NACC accumulator buffers of NCHAIN x BX.
 //
-// Work is a list of runs (tile, range of 128-K blocks). Mode 0 gives each CTA
-// whole tiles (tile = blockIdx.x + i * gridDim.x). Mode 1 (stream-K) cuts the
-// flattened (tile, 128-K block) sequence into one contiguous range per CTA; a
-// tile covered by several CTAs leaves fp32 partial sums in the workspace, and
-// the epilogue warp that arrives last on the tile's counter (one per 32-row
-// quarter) adds all partials in CTA order (deterministic), scales, rounds, stores
-// y and resets the counter to zero.
+// Work is a list of runs (tile, range of load groups). Mode 1 (stream-K) cuts the
+// flattened (tile, load group) sequence into one contiguous range per CTA; a tile covered
+// by several CTAs leaves fp32 partial sums in the workspace, and the epilogue warp that
+// arrives last on the tile's counter (one per 32-row quarter) adds all partials in CTA
+// order (deterministic), scales, rounds, stores y and resets the counter to zero.
+// Mode 0 (whole tiles strided over CTAs) serves shapes with more tiles than counters.
+// Wide tiles (M > 128) use opq_linear_wide.cuh.
 #pragma once
 #include <cuda_bf16.h>
 
@@ -45,6 +44,13 @@ using namespace opqdev;
 __device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
     uint32_t v;
     asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+// A load from read-only shared data (the pair table): not volatile, so the compiler may batch
+// independent lookups; its address depends on data loaded after the table was published.
+__device__ __forceinline__ uint32_t lds_ro_u32(uint32_t addr) {
+    uint32_t v;
+    asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
     return v;
 }
 __device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
@@ -260,9 +266,8 @@ struct Cfg {
     static constexpr int OFF_X = OFF_RAW + RAW_STAGES * RAW_BYTES;
     static constexpr int OFF_EPI = OFF_X + X_STAGES * X_BYTES;
     static constexpr int OFF_BAR = OFF_EPI + STAGE_EPI_BYTES;
-    static constexpr int NUM_BARS = 2 * RAW_STAGES + X_STAGES + NDONE + 2 * NACC + 1;
-    static constexpr int OFF_CNT = OFF_BAR + NUM_BARS * 8;     // A-stage ready counters
-    static constexpr int OFF_TMEM = OFF_CNT + A_STAGES * 4;
+    static constexpr int NUM_BARS = 2 * RAW_STAGES + X_STAGES + A_STAGES + NDONE + 2 * NACC + 1;
+    static constexpr int OFF_TMEM = OFF_BAR + NUM_BARS * 8;
     static constexpr int SMEM_BYTES = OFF_TMEM + 16 + 1024;
     // decoder groups of 4 warps: group g decodes the CTA's 128-K blocks g, g + G, ...;
     // thread r of a group owns weight row r (TMEM lane r) and decodes its whole 128-K block row
@@ -302,10 +307,8 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
     uint64_t *raw_full = bars;
     uint64_t *raw_empty = raw_full + C::RAW_STAGES;
     uint64_t *x_full = raw_empty + C::RAW_STAGES;
-    uint64_t *blk_done = x_full + C::X_STAGES;
-    // a_ready[s]: arrivals of decoder warps on A half-stage s (4 per fill, monotonic), polled by
-    // the MMA issuers with plain acquire loads
-    uint32_t *a_ready = reinterpret_cast<uint32_t *>(smem + C::OFF_CNT);
+    uint64_t *a_full = x_full + C::X_STAGES;
+    uint64_t *blk_done = a_full + C::A_STAGES;
     uint64_t *acc_full = blk_done + C::NDONE;
     uint64_t *acc_empty = acc_full + C::NACC;
     uint64_t *drain = acc_empty + C::NACC;
@@ -323,7 +326,7 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
             mbar_init(&raw_empty[s], 4 * C::GRP);
         }
         for (int s = 0; s < C::X_STAGES; ++s) mbar_init(&x_full[s], 1);
-        for (int s = 0; s < C::A_STAGES; ++s) a_ready[s] = 0u;
+        for (int s = 0; s < C::A_STAGES; ++s) mbar_init(&a_full[s], 4);   // the 4 warps of the decoding group
         for (int s = 0; s < C::NDONE; ++s) mbar_init(&blk_done[s], C::NISS);   // one commit per issuer
         for (int s = 0; s < C::NACC; ++s) {
             mbar_init(&acc_full[s], C::NISS);
@@ -473,7 +476,7 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
             int ab = 0;
             uint32_t abph = 0;
             int as0 = 0, xs = 0, ds = 0;       // A half-stage of the block's first half, x stage, blk_done slot
-            uint32_t aph_n = 0, xph = 0;       // fills of the A ring so far, x ring parity
+            uint32_t aph = 0, xph = 0;
             bool ok = true;
             constexpr uint32_t idesc_full = idesc_bf16_f32(128, BX);
             constexpr uint32_t idesc_half = idesc_bf16_f32(128, BX / 2);
@@ -490,8 +493,7 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
                     for (int jj = 0; jj < nb; ++jj) {
 #pragma unroll
                         for (int h = 0; h < 2; ++h) {
-                            // fill number aph_n of this half-stage: 4 decoder-warp arrivals each
-                            if (!counter_wait(&a_ready[as0 + h], 4u * (aph_n + 1u))) { ok = false; break; }
+                            if (!mbar_wait(&a_full[as0 + h], aph)) { ok = false; break; }
                             tc_fence_after();
                             const uint32_t a_tmem = tmem_base + (as0 + h) * 32;
                             const uint64_t bdesc = smem_desc_sw128(xbase + (2 * jj + h) * C::X_HALF_BYTES);
@@ -508,7 +510,7 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
                         if (!ok) break;
                         umma_commit(&blk_done[ds]);
                         as0 += 2;
-                        if (as0 == C::A_STAGES) { as0 = 0; ++aph_n; }
+                        if (as0 == C::A_STAGES) { as0 = 0; aph ^= 1; }
                         if (++ds == C::NDONE) ds = 0;
                     }
                     if (++xs == C::X_STAGES) { xs = 0; xph ^= 1; }
@@ -539,8 +541,9 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
         const int q = warp & 3;                          // TMEM lane quarter this warp may access
         const int row = q * 32 + lane;                   // weight row in the tile = TMEM lane
         const uint32_t lw = 4u * lane, lw2 = 128u + 4u * lane;
-        const uint32_t *tabp = reinterpret_cast<const uint32_t *>(smem + C::OFF_TABLE);
-        auto load = [&](uint32_t off) { return tabp[off >> 2]; };
+        // table lookups by byte offset from the table's shared-memory address (one add per lookup)
+        const uint32_t tab = sbase + C::OFF_TABLE;
+        auto load = [&](uint32_t off) { return lds_ro_u32(tab + off); };
         // 64-byte swizzle of the codes stage: 16-byte chunk c of row r sits at chunk c ^ ((r >> 1) & 3)
         const uint32_t sw64 = (uint32_t)((row >> 1) & 3);
         const uint32_t tm_row = tmem_base + ((uint32_t)(q * 32) << 16);
@@ -595,7 +598,7 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
                         tmem_st_wait();
                         tc_fence_before();
                         __syncwarp();
-                        if (lane == 0) counter_add_release(&a_ready[as], 1u);
+                        if (lane == 0) mbar_arrive(&a_full[as]);
                     }
                     if (!ok) break;
                 }

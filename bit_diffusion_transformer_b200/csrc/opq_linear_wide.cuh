@@ -1,0 +1,592 @@
+// opq_linear_wide.cuh — y = x W'^T for wide activation tiles (more than 128 rows of x).
+//
+// "OPQ INT4 Z-Image" model card: the OPQLinear forward decodes
+// w = sign * (q/15)^(1/alpha) * max ("inference decoding") and multiplies. As in
+// opq_linear.cuh, the tensor cores see sign * bf16((q/15)^(1/alpha)) and each fp32 sum is
+// multiplied by scale[n] once in the epilogue.
+//
+// Tiles of 128 weight rows x 256 activation rows, one persistent CTA per SM, tensor-bound:
+//   warp 0       raw producer: codes (TMA, 64-byte swizzle) and signs of 128 rows x 128 K
+//                per stage, one 128-K block per copy
+//   warp 1       TMEM allocation and the MMA issue; A from TMEM, B = x from shared memory
+//   warp 2       x producer: 256 rows x 64 K per copy, two per block (128-byte swizzle)
+//   warps 3..10  two decoder groups (4 warps = the 128 TMEM lanes) through the pair table,
+//                A written to TMEM with tcgen05.st
+//   warps 11..14 epilogue
+// Whole tiles are strided over the CTAs; tiles past the last whole wave (at most half as
+// many as CTAs) run as two 128-row halves on two CTAs. The narrow-tile kernel
+// (opq_linear.cuh) fetches several blocks per copy and splits K over CTAs instead; at this
+// width its wait structure measured ~6% slower, so the two regimes keep separate kernels.
+#pragma once
+#include "opq_linear.cuh"
+
+namespace opqk_wide {
+
+using namespace opqk;
+
+struct LinearArgs {
+    const uint32_t *signs;  // sign plane [N, K/32]
+    const float *scales;
+    uint16_t *y;
+    float *ws;              // mode 1: fp32 partials [grid][runs_max][BX][128]
+    uint32_t *counters;     // mode 1: arrivals per (tile, TMEM lane quarter); zero between calls
+    int signs_tma;          // 1: sign plane rows are 16-byte aligned (K % 128 == 0), load it by TMA
+    int M, N, K;
+    int m_tiles, n_tiles;
+    int kblocks;            // 128-K blocks per tile
+    int mode;               // 0 whole tiles strided over CTAs, 1 contiguous unit ranges (stream-K)
+    int runs_max;           // mode 1: most runs one CTA can have
+    int tail_split;         // mode 0: 2 = tiles past the last full wave run as two half-width
+                            // (BX/2 activation rows) runs on different CTAs; 1 = whole tiles
+    uint16_t lut[16];       // bf16 (q/15)^(1/alpha)
+};
+
+// The sequence of runs of one CTA; every role walks the same sequence. A run is one
+// weight tile, a range of its 128-K blocks and a range of its activation rows.
+struct RunIter {
+    int mode, tiles, kblocks, grid, cta;
+    int64_t u, u_end;   // mode 1
+    int t_next;         // mode 0
+    int full_end;       // mode 0: tiles in whole waves (handed out strided)
+    int split;          // mode 0: 1 or 2 runs per tile after the whole waves
+    bool tail_done;
+    int run_idx;
+    __device__ __forceinline__ void init(const LinearArgs &a, int tiles_, int grid_, int cta_) {
+        mode = a.mode;
+        tiles = tiles_;
+        kblocks = a.kblocks;
+        grid = grid_;
+        cta = cta_;
+        run_idx = 0;
+        t_next = cta_;
+        split = a.tail_split;
+        full_end = split == 2 ? (tiles_ / grid_) * grid_ : tiles_;
+        tail_done = false;
+        const int64_t U = (int64_t)tiles * kblocks;
+        u = unit_begin(cta_, grid_, U);
+        u_end = unit_begin(cta_ + 1, grid_, U);
+    }
+    // next run: tile, block range [r0, r1), run index j, activation rows [xoff, xoff + xrows)
+    // of the tile's bx; false at the end
+    __device__ __forceinline__ bool next(int &tile, int &r0, int &r1, int &j, int &xoff, int &xrows, int bx) {
+        xoff = 0;
+        xrows = bx;
+        if (mode == 0) {
+            if (t_next < full_end) {
+                tile = t_next;
+                t_next += grid;
+            } else if (split == 2) {
+                // tail tile t is run by CTAs 2 (t - full_end) and 2 (t - full_end) + 1, one half each
+                if (tail_done || cta >= 2 * (tiles - full_end)) return false;
+                tile = full_end + (cta >> 1);
+                xrows = bx / 2;
+                xoff = (cta & 1) * xrows;
+                tail_done = true;
+            } else {
+                return false;
+            }
+            r0 = 0;
+            r1 = kblocks;
+        } else {
+            if (u >= u_end) return false;
+            tile = (int)(u / kblocks);
+            r0 = (int)(u - (int64_t)tile * kblocks);
+            const int64_t end = (int64_t)r0 + (u_end - u);
+            r1 = end < (int64_t)kblocks ? (int)end : kblocks;
+            u += r1 - r0;
+        }
+        j = run_idx++;
+        return true;
+    }
+    __device__ __forceinline__ bool next(int &tile, int &r0, int &r1, int &j) {
+        int xo, xr;
+        return next(tile, r0, r1, j, xo, xr, 2);
+    }
+};
+
+template <int BX>
+struct Cfg {
+    static constexpr int BW = 128;                     // weight rows per tile (MMA M)
+    static constexpr int KR = 128;                     // K per raw (codes/signs) stage
+    static constexpr int KA = 64;                      // K per A stage (TMEM) and per x stage (smem)
+    static constexpr int RAW_STAGES = BX >= 256 ? 2 : (BX >= 128 ? 4 : 6);
+    static constexpr int A_STAGES = 8;                 // 32 TMEM columns each (64 K of bf16 pairs)
+    static constexpr int A_BLOCKS = A_STAGES / 2;      // 128-K blocks of A held in TMEM
+    static constexpr int A_COLS = A_STAGES * 32;
+    // x stages hold a whole 128-K block (two 64-K swizzle atoms' worth of columns)
+    static constexpr int X_STAGES = BX >= 256 ? 2 : (BX >= 128 ? 3 : (BX >= 64 ? 4 : (BX >= 32 ? 8 : 10)));
+    // One tcgen05.commit per 128-K block frees both its A slot and its x stage: a commit
+    // stalls the tensor pipe for a few hundred cycles, so there is one per 8 MMAs, not per 4.
+    // Slot b % NDONE of `blk_done` completes when the MMAs of the CTA's block b are done.
+    static constexpr int NDONE = X_STAGES > A_BLOCKS ? X_STAGES : A_BLOCKS;
+    // independent accumulation chains per tile: consecutive MMAs into one accumulator
+    // serialize on its latency, which dominates when N (= BX) is small; K-step k of a
+    // stage goes to chain k % NCHAIN and the epilogue adds the chains in a fixed order
+    static constexpr int NCHAIN = BX <= 32 ? 4 : (BX <= 64 ? 2 : 1);
+    static constexpr int ACC_COLS = NCHAIN * BX;       // one accumulator buffer (all chains)
+    static constexpr int NACC = (A_COLS + 2 * ACC_COLS <= 512) ? 2 : 1;   // accumulator buffers
+    static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr int RAW_CODE_BYTES = BW * KR / 2;    // 8 KiB: [128 rows][16 words], 64-byte swizzle
+    static constexpr int RAW_SIGN_BYTES = BW * KR / 8;    // 2 KiB: [128 rows][4 words]
+    static constexpr int RAW_BYTES = RAW_CODE_BYTES + RAW_SIGN_BYTES;
+    static constexpr int X_HALF_BYTES = BX * KA * 2;   // one 64-K half: BX rows x 128 bytes, 128-byte swizzle
+    static constexpr int X_BYTES = 2 * X_HALF_BYTES;
+    static constexpr int STAGE_EPI_BYTES = 4 * 2 * 16 * 32 * 2;   // 4 warps x 2 buffers x [16 m][32 n] bf16
+    static constexpr int OFF_TABLE = 0;
+    static constexpr int OFF_RAW = OFF_TABLE + (int)opqbits::kPairTableBytes;
+    static constexpr int OFF_X = OFF_RAW + RAW_STAGES * RAW_BYTES;
+    static constexpr int OFF_EPI = OFF_X + X_STAGES * X_BYTES;
+    static constexpr int OFF_BAR = OFF_EPI + STAGE_EPI_BYTES;
+    static constexpr int NUM_BARS = 2 * RAW_STAGES + X_STAGES + A_STAGES + NDONE + 2 * NACC + 1;
+    static constexpr int OFF_TMEM = OFF_BAR + NUM_BARS * 8;
+    static constexpr int SMEM_BYTES = OFF_TMEM + 16 + 1024;
+    // decoder groups of 4 warps: group g decodes the CTA's 128-K blocks g, g + G, ...;
+    // thread r of a group owns weight row r (TMEM lane r) and decodes its whole 128-K block row
+    static constexpr int GROUPS = BX >= 256 ? 2 : 3;
+    // a group waits on raw stage blk % RAW_STAGES knowing only that its own previous block
+    // (blk - GROUPS) was loaded, so the stage's previous phase (block blk - RAW_STAGES) must
+    // be at least that old for the parity test to be exact
+    static_assert(RAW_STAGES >= GROUPS, "raw ring shorter than the decoder rotation");
+    static constexpr int WARP_LOAD = 0, WARP_MMA = 1, WARP_XLOAD = 2, WARP_DEC0 = 3, NUM_DEC_WARPS = 4 * GROUPS;
+    static constexpr int WARP_EPI0 = WARP_DEC0 + NUM_DEC_WARPS;
+    // One MMA-issuing thread per accumulation chain: a thread issues one tcgen05.mma every
+    // few dozen cycles, far slower than the tensor pipe runs a narrow (N <= 64) MMA, so the
+    // chains are issued from separate warps (warp 1, then warps WARP_ISS1...).
+    static constexpr int NISS = NCHAIN;
+    static constexpr int WARP_ISS1 = WARP_EPI0 + 4;
+    static constexpr int THREADS = (WARP_ISS1 + NISS - 1) * 32;
+    static_assert(SMEM_BYTES <= 232448, "shared memory");
+    static_assert(BX % 16 == 0 && BX >= 16 && BX <= 256, "MMA N");
+    static_assert(A_COLS + NACC * ACC_COLS <= 512, "TMEM columns");
+    static_assert(RAW_BYTES % 1024 == 0 && X_BYTES % 1024 == 0, "stage alignment");
+    static_assert(A_STAGES % 2 == 0, "a block is two A half-stages");
+};
+
+template <int BX>
+__global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
+    wide_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_xh,
+                  const __grid_constant__ CUtensorMap tmap_codes, const __grid_constant__ CUtensorMap tmap_signs,
+                  const __grid_constant__ LinearArgs args) {
+    using C = Cfg<BX>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_base = smem_u32(smem_raw);
+    const uint32_t pad = ((raw_base + 1023u) & ~1023u) - raw_base;
+    uint8_t *smem = smem_raw + pad;
+    const uint32_t sbase = raw_base + pad;
+
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
+    uint64_t *raw_full = bars;
+    uint64_t *raw_empty = raw_full + C::RAW_STAGES;
+    uint64_t *x_full = raw_empty + C::RAW_STAGES;
+    uint64_t *a_full = x_full + C::X_STAGES;
+    uint64_t *blk_done = a_full + C::A_STAGES;
+    uint64_t *acc_full = blk_done + C::NDONE;
+    uint64_t *acc_empty = acc_full + C::NACC;
+    uint64_t *drain = acc_empty + C::NACC;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_TMEM);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tiles = args.m_tiles * args.n_tiles;
+    const bool signs_by_tma = args.signs_tma != 0;
+
+    // ---- pair table: 32 copies of value(b) then 32 copies of spread(b) per entry b
+    for (int e = threadIdx.x; e < 512; e += C::THREADS) {
+        const uint32_t b = (uint32_t)e & 255u;
+        const uint32_t v = e < 256 ? ((uint32_t)args.lut[b & 15u] | ((uint32_t)args.lut[b >> 4] << 16))
+                                   : opqbits::sign_spread(b);
+        const uint32_t dst = sbase + C::OFF_TABLE + b * 256u + (e < 256 ? 0u : 128u);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst + 16u * k), "r"(v) : "memory");
+    }
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::RAW_STAGES; ++s) {
+            // the codes' (and signs') expect_tx arrival, plus 32 cp.async arrivals when signs are copied by threads
+            mbar_init(&raw_full[s], signs_by_tma ? 1 : 1 + 32);
+            mbar_init(&raw_empty[s], 4);          // the 4 warps of the group that decodes the block
+        }
+        for (int s = 0; s < C::X_STAGES; ++s) mbar_init(&x_full[s], 1);
+        for (int s = 0; s < C::A_STAGES; ++s) mbar_init(&a_full[s], 4);   // the 4 warps of the decoding group
+        for (int s = 0; s < C::NDONE; ++s) mbar_init(&blk_done[s], C::NISS);   // one commit per issuer
+        for (int s = 0; s < C::NACC; ++s) {
+            mbar_init(&acc_full[s], C::NISS);
+            mbar_init(&acc_empty[s], 4);
+        }
+        mbar_init(drain, C::NISS);
+        fence_mbar_init();
+    }
+    if (warp == C::WARP_LOAD && lane == 0) {
+        tma_prefetch_desc(&tmap_codes);
+        if (signs_by_tma) tma_prefetch_desc(&tmap_signs);
+    }
+    if (warp == C::WARP_XLOAD && lane == 0) {
+        tma_prefetch_desc(&tmap_x);
+        if (args.tail_split == 2) tma_prefetch_desc(&tmap_xh);
+    }
+    if (warp == C::WARP_MMA) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    RunIter it;
+    it.init(args, tiles, gridDim.x, blockIdx.x);
+    int tile, r0, r1, j;
+
+    if (warp == C::WARP_LOAD) {
+        // ----------------------------------------------------------- raw producer
+        const int swd = args.K / 32;        // sign words per row
+        int rs = 0;
+        uint32_t rph = 0;
+        int raw_issued = 0;
+        bool ok = true;
+        while (ok && it.next(tile, r0, r1, j)) {
+            const int n_blk = tile / args.m_tiles;
+            for (int r = r0; r < r1 && ok; ++r) {
+                // lane 0 waits for the stage; the verdict and the ordering reach the other lanes
+                int okw = 1;
+                if (lane == 0) okw = mbar_wait(&raw_empty[rs], rph ^ 1) ? 1 : 0;
+                okw = __shfl_sync(0xFFFFFFFFu, okw, 0);
+                __syncwarp();
+                if (!okw) { ok = false; break; }
+                const uint32_t dst = sbase + C::OFF_RAW + rs * C::RAW_BYTES;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&raw_full[rs], signs_by_tma ? C::RAW_BYTES : C::RAW_CODE_BYTES);
+                    tma_load_2d(smem + C::OFF_RAW + rs * C::RAW_BYTES, &tmap_codes, r * (C::KR / 8), n_blk * C::BW,
+                                &raw_full[rs]);
+                    if (signs_by_tma)
+                        tma_load_2d(smem + C::OFF_RAW + rs * C::RAW_BYTES + C::RAW_CODE_BYTES, &tmap_signs,
+                                    r * (C::KR / 32), n_blk * C::BW, &raw_full[rs]);
+                }
+                if (!signs_by_tma) {
+                    // sign words: 128 rows x 4 words; copy i of lane l is word 32 i + l of the stage
+                    // (consecutive lanes, consecutive banks); out-of-range words read as 0
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int e = i * 32 + lane;
+                        const int row = e >> 2, w = e & 3;
+                        const int n = n_blk * C::BW + row, kw = r * 4 + w;
+                        const bool in = n < args.N && kw < swd;
+                        const uint32_t *src = args.signs + (in ? (size_t)n * swd + kw : 0);
+                        cp_async_4(dst + C::RAW_CODE_BYTES + row * 16 + w * 4, src, in ? 4u : 0u);
+                    }
+                    cp_async_mbar_arrive(&raw_full[rs]);
+                }
+                ++raw_issued;
+                if (++rs == C::RAW_STAGES) { rs = 0; rph ^= 1; }
+            }
+        }
+        if (!ok) {
+            // let every copy already issued land before the CTA can exit
+            asm volatile("cp.async.wait_all;" ::: "memory");
+            if (lane == 0) {
+                for (int i = 0; i < raw_issued && i < C::RAW_STAGES; ++i) {
+                    if (--rs < 0) { rs = C::RAW_STAGES - 1; rph ^= 1; }
+                    (void)mbar_wait(&raw_full[rs], rph);
+                }
+            }
+        }
+    } else if (warp == C::WARP_XLOAD) {
+        // ----------------------------------------------------------- x producer
+        if (lane == 0) {
+            int b = 0;                 // the CTA's block index
+            bool ok = true;
+            int xoff, xrows;
+            while (ok && it.next(tile, r0, r1, j, xoff, xrows, BX)) {
+                const int m_blk = tile % args.m_tiles;
+                // a half-width run loads its BX/2 activation rows with the half-height box
+                const bool half = xrows != BX;
+                const void *xmap = half ? (const void *)&tmap_xh : (const void *)&tmap_x;
+                const uint32_t xbytes = half ? C::X_BYTES / 2 : C::X_BYTES;
+                const int xrow = m_blk * BX + xoff;
+                for (int r = r0; r < r1; ++r, ++b) {
+                    // stage b % X_STAGES last held block b - X_STAGES
+                    const int prev = b - C::X_STAGES;
+                    if (prev >= 0 && !mbar_wait(&blk_done[prev % C::NDONE], (uint32_t)(prev / C::NDONE) & 1u)) {
+                        ok = false;
+                        break;
+                    }
+                    const int xs = b % C::X_STAGES;
+                    mbar_arrive_expect_tx(&x_full[xs], xbytes);
+                    uint8_t *dst = smem + C::OFF_X + xs * C::X_BYTES;
+                    tma_load_2d(dst, xmap, r * C::KR, xrow, &x_full[xs]);
+                    tma_load_2d(dst + C::X_HALF_BYTES, xmap, r * C::KR + C::KA, xrow, &x_full[xs]);
+                }
+            }
+            if (!ok) {
+                // let the copies already issued land before the CTA can exit
+                for (int i = 1; i <= C::X_STAGES && b - i >= 0; ++i)
+                    (void)mbar_wait(&x_full[(b - i) % C::X_STAGES], (uint32_t)((b - i) / C::X_STAGES) & 1u);
+            }
+        }
+    } else if (warp == C::WARP_MMA || warp >= C::WARP_ISS1) {
+        // ----------------------------------------------------------- MMA issuers
+        // Issuer i accumulates K-steps k = i, i + NISS, ... of every 64-K half into chain i.
+        if (lane == 0) {
+            const int iss = warp == C::WARP_MMA ? 0 : warp - C::WARP_ISS1 + 1;
+            int ab = 0;
+            uint32_t abph = 0;
+            int as0 = 0, xs = 0, ds = 0;       // A half-stage of the block's first half, x stage, blk_done slot
+            uint32_t aph = 0, xph = 0;
+            bool ok = true;
+            constexpr uint32_t idesc_full = idesc_bf16_f32(128, BX);
+            constexpr uint32_t idesc_half = idesc_bf16_f32(128, BX / 2);
+            int xoff, xrows;
+            while (ok && it.next(tile, r0, r1, j, xoff, xrows, BX)) {
+                const uint32_t idesc = xrows == BX ? idesc_full : idesc_half;
+                if (!mbar_wait(&acc_empty[ab], abph ^ 1)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + C::A_COLS + ab * C::ACC_COLS + iss * BX;
+                uint32_t acc = 0;              // 0 for the chain's first MMA of the run
+                for (int r = r0; r < r1; ++r) {
+                    const uint32_t xaddr = sbase + C::OFF_X + xs * C::X_BYTES;
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        if (!mbar_wait(&a_full[as0 + h], aph)) { ok = false; break; }
+                        if (h == 0 && !mbar_wait(&x_full[xs], xph)) { ok = false; break; }
+                        tc_fence_after();
+                        const uint32_t a_tmem = tmem_base + (as0 + h) * 32;
+                        const uint64_t bdesc = smem_desc_sw128(xaddr + h * C::X_HALF_BYTES);
+#pragma unroll
+                        for (int k = 0; k < C::KA / 16; ++k) {
+                            if (k % C::NISS != iss % C::NISS) continue;
+                            umma_bf16_ts(d_tmem, a_tmem + 8 * k, bdesc + 2 * k, idesc, acc);
+                            acc = 1;
+                        }
+                    }
+                    if (!ok) break;
+                    umma_commit(&blk_done[ds]);
+                    as0 += 2;
+                    if (as0 == C::A_STAGES) { as0 = 0; aph ^= 1; }
+                    if (++xs == C::X_STAGES) { xs = 0; xph ^= 1; }
+                    if (++ds == C::NDONE) ds = 0;
+                }
+                if (ok) umma_commit(&acc_full[ab]);
+                if (++ab == C::NACC) { ab = 0; abph ^= 1; }
+            }
+            // every MMA issued by this thread has completed once `drain` flips
+            umma_commit(drain);
+            (void)mbar_wait(drain, 0);
+        }
+    } else if (warp < C::WARP_EPI0) {
+        // ----------------------------------------------------------- decoders
+        const int g = (warp - C::WARP_DEC0) >> 2;        // decoder group
+        const int q = warp & 3;                          // TMEM lane quarter this warp may access
+        const int row = q * 32 + lane;                   // weight row in the tile = TMEM lane
+        const uint32_t lw = 4u * lane, lw2 = 128u + 4u * lane;
+        const uint32_t *tabp = reinterpret_cast<const uint32_t *>(smem + C::OFF_TABLE);
+        auto load = [&](uint32_t off) { return tabp[off >> 2]; };
+        // 64-byte swizzle of the codes stage: 16-byte chunk c of row r sits at chunk c ^ ((r >> 1) & 3)
+        const uint32_t sw64 = (uint32_t)((row >> 1) & 3);
+        const uint32_t tm_row = tmem_base + ((uint32_t)(q * 32) << 16);
+        int nblocks = 0;
+        while (it.next(tile, r0, r1, j)) nblocks += r1 - r0;
+        bool ok = true;
+        for (int blk = g; blk < nblocks && ok; blk += C::GROUPS) {
+            const int rs = blk % C::RAW_STAGES;
+            const uint32_t rph = (uint32_t)(blk / C::RAW_STAGES) & 1u;
+            if (!warp_wait(&raw_full[rs], rph)) { ok = false; break; }
+            const uint8_t *rawc = smem + C::OFF_RAW + rs * C::RAW_BYTES + row * (C::KR / 2);
+            const uint8_t *raws = smem + C::OFF_RAW + rs * C::RAW_BYTES + C::RAW_CODE_BYTES + row * (C::KR / 8);
+#pragma unroll
+            for (int h = 0; h < C::KR / C::KA; ++h) {     // two 64-K A stages per block
+                const int sidx = blk * 2 + h;
+                const int as = sidx % C::A_STAGES;
+                // this half's 8 code words (two 16-byte chunks) and 2 sign words
+                uint32_t cw[8];
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    const uint4 v = *reinterpret_cast<const uint4 *>(rawc + ((((uint32_t)(2 * h + c)) ^ sw64) << 4));
+                    cw[4 * c] = v.x; cw[4 * c + 1] = v.y; cw[4 * c + 2] = v.z; cw[4 * c + 3] = v.w;
+                }
+                const uint2 sv = *reinterpret_cast<const uint2 *>(raws + 8 * h);
+                const uint32_t sw[2] = {sv.x, sv.y};
+                if (h == 1) {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&raw_empty[rs]);   // the block's raw words are in registers now
+                }
+                uint32_t o[2][16];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    uint32_t t4[4];
+                    opqbits::decode8_table(cw[i], sw[i >> 2], (uint32_t)(i & 3), lw, lw2, load, t4);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) o[i >> 2][(i & 3) * 4 + e] = t4[e];
+                }
+                // the block's A slot last held block blk - A_BLOCKS
+                const int prev = blk - C::A_BLOCKS;
+                if (h == 0 && prev >= 0 &&
+                    !warp_wait(&blk_done[prev % C::NDONE], (uint32_t)(prev / C::NDONE) & 1u)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                tmem_st_32x32b_x16(tm_row + as * 32, o[0]);
+                tmem_st_32x32b_x16(tm_row + as * 32 + 16, o[1]);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&a_full[as]);
+            }
+        }
+    } else {
+        // ----------------------------------------------------------- epilogue
+        const int q = warp & 3;
+        const int row = q * 32 + lane;
+        const int64_t U = (int64_t)tiles * args.kblocks;
+        const bool vec_y = (args.N % 8) == 0;
+        // per-warp staging for y: 2 buffers of [16 m][32 n] bf16
+        const uint32_t stage0 = sbase + C::OFF_EPI + (uint32_t)(warp - C::WARP_EPI0) * 2048u;
+        int ab = 0;
+        uint32_t abph = 0;
+        int sb = 0;
+        int xoff, xrows;
+        while (it.next(tile, r0, r1, j, xoff, xrows, BX)) {
+            const int n_blk = tile / args.m_tiles, m_blk = tile % args.m_tiles;
+            const int n = n_blk * C::BW + row;
+            const int n0 = n_blk * C::BW + q * 32;           // first row of this warp's quarter
+            const bool full = (r0 == 0 && r1 == args.kblocks);
+            const float scale = n < args.N ? __ldg(args.scales + n) : 0.0f;
+            if (!warp_wait(&acc_full[ab], abph)) break;
+            tc_fence_after();
+            const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + C::A_COLS + ab * C::ACC_COLS;
+            float *wsp = full ? nullptr
+                              : args.ws + ((size_t)blockIdx.x * args.runs_max + j) * (size_t)(BX * C::BW);
+#pragma unroll 1
+            for (int c0 = 0; c0 < xrows; c0 += 16) {
+                uint32_t v[16];
+                tmem_ld_32x32b_x16(taddr + c0, v);
+                if (C::NCHAIN > 1) {
+#pragma unroll
+                    for (int ch = 1; ch < C::NCHAIN; ++ch) {
+                        uint32_t u[16];
+                        tmem_ld_32x32b_x16(taddr + ch * BX + c0, u);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) + __uint_as_float(u[i]));
+                    }
+                }
+                tmem_ld_wait();
+                if (full) {
+                    const int m0 = m_blk * BX + xoff + c0;
+                    if (vec_y && n0 + 32 <= args.N) {
+                        // stage [16 m][32 n] bf16, then each lane stores 32 contiguous bytes of one m row
+                        const uint32_t sbuf = stage0 + (uint32_t)sb * 1024u;
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const __nv_bfloat16 o = __float2bfloat16_rn(__uint_as_float(v[i]) * scale);
+                            asm volatile("st.shared.u16 [%0], %1;" ::"r"(sbuf + (uint32_t)i * 64u + (uint32_t)lane * 2u),
+                                         "h"(*reinterpret_cast<const unsigned short *>(&o)) : "memory");
+                        }
+                        __syncwarp();
+                        const int mi = lane >> 1, hf = lane & 1;
+                        if (m0 + mi < args.M) {
+                            const uint4 w0 = lds_v4(sbuf + (uint32_t)mi * 64u + (uint32_t)hf * 32u);
+                            const uint4 w1 = lds_v4(sbuf + (uint32_t)mi * 64u + (uint32_t)hf * 32u + 16u);
+                            uint4 *dst = reinterpret_cast<uint4 *>(args.y + (size_t)(m0 + mi) * args.N + n0 + hf * 16);
+                            dst[0] = w0;
+                            dst[1] = w1;
+                        }
+                        sb ^= 1;
+                    } else if (n < args.N) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const int m = m0 + i;
+                            if (m < args.M) {
+                                const __nv_bfloat16 o = __float2bfloat16_rn(__uint_as_float(v[i]) * scale);
+                                args.y[(size_t)m * args.N + n] = *reinterpret_cast<const uint16_t *>(&o);
+                            }
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) wsp[(size_t)(c0 + i) * C::BW + row] = __uint_as_float(v[i]);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[ab]);
+            if (++ab == C::NACC) { ab = 0; abph ^= 1; }
+            if (!full) {
+                // The last of the tile's CTAs to get here (per lane quarter) adds every
+                // CTA's partial rows in CTA order, so the sum does not depend on timing.
+                const int64_t c_lo = unit_owner((int64_t)tile * args.kblocks, gridDim.x, U);
+                const int64_t c_hi = unit_owner((int64_t)(tile + 1) * args.kblocks - 1, gridDim.x, U);
+                const uint32_t parts = (uint32_t)(c_hi - c_lo + 1);
+                __threadfence();
+                __syncwarp();
+                uint32_t old = 0;
+                if (lane == 0) old = atomicAdd(args.counters + (size_t)tile * 4 + q, 1u);
+                old = __shfl_sync(0xFFFFFFFFu, old, 0);
+                if (old == parts - 1) {
+                    __threadfence();
+                    // lane i (< parts) resolves part i's base; bases are broadcast by shuffles
+                    const float *mybase = nullptr;
+                    if ((uint32_t)lane < parts) {
+                        const int64_t c = c_lo + lane;
+                        const int64_t jj = tile - unit_begin(c, gridDim.x, U) / args.kblocks;
+                        mybase = args.ws + ((size_t)c * args.runs_max + (size_t)jj) * (size_t)(BX * C::BW);
+                    }
+                    // Every lane runs the loops (shuffles need all lanes); only rows < N store.
+                    // 8 columns per pass, the next part's 8 loads issued before the current
+                    // part's adds; each sum still runs over parts 0, 1, ... from 0.0f.
+                    auto part_base = [&](uint32_t p) -> const float * {
+                        if (p < 32)
+                            return reinterpret_cast<const float *>(
+                                __shfl_sync(0xFFFFFFFFu, reinterpret_cast<unsigned long long>(mybase), (int)p));
+                        const int64_t c = c_lo + p;
+                        const int64_t jj = tile - unit_begin(c, gridDim.x, U) / args.kblocks;
+                        return args.ws + ((size_t)c * args.runs_max + (size_t)jj) * (size_t)(BX * C::BW);
+                    };
+                    const int mcols = min(BX, args.M - m_blk * BX);
+                    for (int c0 = 0; c0 < mcols; c0 += 8) {
+                        float acc[8], cur[8], nxt[8];
+                        const float *b0 = part_base(0) + (size_t)c0 * C::BW + row;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            acc[i] = 0.0f;
+                            cur[i] = (c0 + i < mcols) ? __ldcg(b0 + (size_t)i * C::BW) : 0.0f;
+                        }
+                        for (uint32_t p = 0; p < parts; ++p) {
+                            if (p + 1 < parts) {
+                                const float *bn = part_base(p + 1) + (size_t)c0 * C::BW + row;
+#pragma unroll
+                                for (int i = 0; i < 8; ++i) nxt[i] = (c0 + i < mcols) ? __ldcg(bn + (size_t)i * C::BW) : 0.0f;
+                            }
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                acc[i] += cur[i];
+                                cur[i] = nxt[i];
+                            }
+                        }
+                        if (n < args.N) {
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                if (c0 + i < mcols) {
+                                    const __nv_bfloat16 o = __float2bfloat16_rn(acc[i] * scale);
+                                    args.y[(size_t)(m_blk * BX + c0 + i) * args.N + n] = *reinterpret_cast<const uint16_t *>(&o);
+                                }
+                            }
+                        }
+                    }
+                    if (lane == 0) atomicExch(args.counters + (size_t)tile * 4 + q, 0u);   // ready for the next call
+                }
+            }
+        }
+    }
+
+    // roles run on single lanes: reconverge every warp before the CTA barrier, so that the
+    // barrier (and the warp-wide TMEM release after it) waits for every lane's last operation
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == C::WARP_MMA) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+}  // namespace opqk_wide
