@@ -72,6 +72,59 @@ OPQ_HD uint32_t quant_pair(uint32_t w2, const uint32_t (&P)[16]) {
     return (k3 & 0x00080008u) | (k2 & 0x00040004u) | (k1 & 0x00020002u) | (k0 & 0x00010001u);
 }
 
+// Same codes with the four comparisons done as packed bf16 compares (set.ge.u32.bf16x2:
+// 0xFFFF in each half where a >= b, exact for subnormals, false for NaN), which leaves the
+// integer pipe only the threshold selects. Here P[k] holds T[k] in both halves with +inf
+// (0x7F80) as the unreachable level instead of 0x8000; for finite non-negative halves it
+// returns exactly quant_pair's codes.
+OPQ_HD uint32_t bf16x2_ge_mask(uint32_t a, uint32_t b) {
+#if defined(__CUDA_ARCH__)
+    uint32_t r;
+    asm("set.ge.u32.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+#else
+    uint32_t r = 0;
+    for (int h = 0; h < 2; ++h) {
+        const uint32_t ua = ((a >> (16 * h)) & 0xFFFFu) << 16, ub = ((b >> (16 * h)) & 0xFFFFu) << 16;
+        float fa, fb;
+        __builtin_memcpy(&fa, &ua, 4);
+        __builtin_memcpy(&fb, &ub, 4);
+        if (fa >= fb) r |= 0xFFFFu << (16 * h);
+    }
+    return r;
+#endif
+}
+
+// 0xFFFF in each half where the bf16 value is < 0 (so -0.0 and NaN give 0).
+OPQ_HD uint32_t bf16x2_neg_mask(uint32_t a) {
+#if defined(__CUDA_ARCH__)
+    uint32_t r;
+    asm("set.lt.u32.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(0u));
+    return r;
+#else
+    uint32_t r = 0;
+    for (int h = 0; h < 2; ++h) {
+        const uint32_t ua = ((a >> (16 * h)) & 0xFFFFu) << 16;
+        float fa;
+        __builtin_memcpy(&fa, &ua, 4);
+        if (fa < 0.0f) r |= 0xFFFFu << (16 * h);
+    }
+    return r;
+#endif
+}
+
+OPQ_HD uint32_t quant_pair_f(uint32_t w2, const uint32_t (&P)[16]) {
+    const uint32_t a = w2 & 0x7FFF7FFFu;
+    const uint32_t k3 = bf16x2_ge_mask(a, P[8]);                      // q >= 8
+    const uint32_t k2 = bf16x2_ge_mask(a, sel_mask(k3, P[12], P[4]));   // q >= 4 + 8c3
+    const uint32_t t1 = sel_mask(k3, sel_mask(k2, P[14], P[10]), sel_mask(k2, P[6], P[2]));
+    const uint32_t k1 = bf16x2_ge_mask(a, t1);
+    const uint32_t b0 = sel_mask(k2, sel_mask(k1, P[7], P[5]), sel_mask(k1, P[3], P[1]));
+    const uint32_t b1 = sel_mask(k2, sel_mask(k1, P[15], P[13]), sel_mask(k1, P[11], P[9]));
+    const uint32_t k0 = bf16x2_ge_mask(a, sel_mask(k3, b1, b0));
+    return (k3 & 0x00080008u) | (k2 & 0x00040004u) | (k1 & 0x00020002u) | (k0 & 0x00010001u);
+}
+
 // 8 weights (4 bf16 pairs, elements 0..7) -> one code word, element i in nibble i.
 OPQ_HD uint32_t pack_codes(uint32_t q0, uint32_t q1, uint32_t q2, uint32_t q3) {
     // q_p holds element 2p in bits 0..3 and element 2p+1 in bits 16..19

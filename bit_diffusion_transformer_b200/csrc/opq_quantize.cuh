@@ -7,8 +7,8 @@
 // Every lane loads its 16-byte vectors of the row once (coalesced, kept in
 // registers), the group reduces max |w| in the bf16 bit domain, lanes 0..14
 // form the 15 exact per-row thresholds in fp64, and each vector of 8 weights is
-// coded by a branch-free binary search on two 16-bit halves at a time
-// (opqbits::quant_pair) — no pow on the device.
+// coded by a branch-free binary search on two bf16 halves at a time with packed
+// bf16 compares (opqbits::quant_pair_f) — no pow on the device.
 #pragma once
 #include "opq_bits.h"
 #include "opq_device.cuh"
@@ -39,7 +39,7 @@ __device__ __forceinline__ uint32_t level_threshold(float mxf, int k, const Quan
     uint32_t tb = (fb >> 16) + ((fb & 0xFFFFu) != 0u ? 1u : 0u);
     const bool exact = ((fb & 0xFFFFu) == 0u) && ((double)f == th);
     if ((k & 1) && exact) tb += 1u;
-    return tb < 0x8000u ? tb : 0x8000u;
+    return tb < 0x7F80u ? tb : 0x7F80u;   // +inf: unreachable (only for a non-finite max)
 }
 
 template <int G, int VPL>
@@ -83,7 +83,8 @@ __global__ void __launch_bounds__(256) quantize_kernel(const uint16_t *__restric
             __syncthreads();
         }
         const float mxf = __uint_as_float(mx << 16);
-        uint32_t myT = 0x8000u;
+        // +inf marks a level no finite weight reaches (all levels of an all-zero row)
+        uint32_t myT = 0x7F80u;
         if (lane < 15 && mx != 0u) myT = level_threshold(mxf, lane + 1, qp);
         uint32_t P[16];
         P[0] = 0;
@@ -97,14 +98,12 @@ __global__ void __launch_bounds__(256) quantize_kernel(const uint16_t *__restric
         for (int j = 0; j < VPL; ++j) {
             const int64_t vi = (int64_t)j * 32 * G + gl;
             const uint4 x = v[j];
-            const uint32_t code = opqbits::pack_codes(opqbits::quant_pair(x.x, P), opqbits::quant_pair(x.y, P),
-                                                      opqbits::quant_pair(x.z, P), opqbits::quant_pair(x.w, P));
-            // the sign bit counts only for a non-zero magnitude (w < 0; -0.0 stores 0)
-            const uint32_t nz_x = ((x.x & 0x7FFF7FFFu) + 0x7FFF7FFFu) | 0x7FFF7FFFu;
-            const uint32_t nz_y = ((x.y & 0x7FFF7FFFu) + 0x7FFF7FFFu) | 0x7FFF7FFFu;
-            const uint32_t nz_z = ((x.z & 0x7FFF7FFFu) + 0x7FFF7FFFu) | 0x7FFF7FFFu;
-            const uint32_t nz_w = ((x.w & 0x7FFF7FFFu) + 0x7FFF7FFFu) | 0x7FFF7FFFu;
-            const uint32_t sb = opqbits::sign_byte(x.x & nz_x, x.y & nz_y, x.z & nz_z, x.w & nz_w);
+            const uint32_t code = opqbits::pack_codes(opqbits::quant_pair_f(x.x, P), opqbits::quant_pair_f(x.y, P),
+                                                      opqbits::quant_pair_f(x.z, P), opqbits::quant_pair_f(x.w, P));
+            // sign bit = w < 0 (so -0.0 stores 0): a packed compare with zero gives 0xFFFF per
+            // negative half, whose top bit sign_byte collects
+            const uint32_t sb = opqbits::sign_byte(opqbits::bf16x2_neg_mask(x.x), opqbits::bf16x2_neg_mask(x.y),
+                                                   opqbits::bf16x2_neg_mask(x.z), opqbits::bf16x2_neg_mask(x.w));
             // four consecutive vectors (lanes gl..gl+3) form one sign word
             uint32_t sw = sb << (8 * (gl & 3));
             sw |= __shfl_xor_sync(0xFFFFFFFFu, sw, 1);

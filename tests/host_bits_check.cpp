@@ -43,8 +43,29 @@ int main() {
             for (int k = 1; k <= 15; ++k) { want_lo += (m >= T[k]); want_hi += (m2 >= T[k]); }
             CHECK((q2 & 0xFFFFu) == want_lo && (q2 >> 16) == want_hi,
                   "quant_pair trial %d m %x m2 %x got %x want %x %x", trial, m, m2, q2, want_lo, want_hi);
+            // the packed-compare form: +inf stands for the unreachable level; finite halves only
+            // (codes of non-finite weights are unspecified)
+            if (m < 0x7F80u && m2 < 0x7F80u) {
+                uint32_t PF[16];
+                for (int k = 0; k < 16; ++k) PF[k] = (T[k] == 0x8000u ? 0x7F80u : T[k]) * 0x00010001u;
+                const uint32_t qf = quant_pair_f(w2, PF);
+                CHECK(qf == q2, "quant_pair_f trial %d m %x m2 %x got %x want %x", trial, m, m2, qf, q2);
+            }
         }
     }
+    // bf16x2_neg_mask: w < 0 per half (negative zero and NaN are not negative)
+    for (uint32_t a = 0; a < 0x10000u; ++a) {
+        const bool neg = (a & 0x8000u) && (a & 0x7FFFu) != 0u && (a & 0x7FFFu) <= 0x7F80u;
+        const uint32_t r = opqbits::bf16x2_neg_mask(a | (a << 16));
+        CHECK(r == (neg ? 0xFFFFFFFFu : 0u), "bf16x2_neg_mask %x -> %x", a, r);
+    }
+    // bf16x2_ge_mask host emulation against plain float compares, subnormals and zeros included
+    for (uint32_t a = 0; a < 0x7F80u; a += 3)
+        for (uint32_t b : {0x0000u, 0x0001u, 0x007Fu, 0x0080u, 0x3F80u, 0x7F7Fu, 0x7F80u}) {
+            const uint32_t r = bf16x2_ge_mask(a | (b << 16), b | (a << 16));
+            CHECK((r & 0xFFFFu) == (a >= b ? 0xFFFFu : 0u) && (r >> 16) == (b >= a ? 0xFFFFu : 0u),
+                  "bf16x2_ge_mask %x %x -> %x", a, b, r);
+        }
     // --- pack_codes / sign_byte
     for (int trial = 0; trial < 100000; ++trial) {
         uint32_t q[8], w[4], want_code = 0, want_sb = 0;
