@@ -40,6 +40,19 @@ __global__ void __launch_bounds__(256) dequantize_kernel(const uint32_t *__restr
     // lane q (and q + 16) holds LUT[q] for the products
     const double lut_q = dp.lut[lane & 15u];
     for (uint32_t n = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); n < rows; n += warps) {
+        const uint4 *crow = reinterpret_cast<const uint4 *>(codes + (size_t)n * chunks * 4u);
+        const uint32_t *srow = signs + (size_t)n * chunks;
+        uint4 *orow = reinterpret_cast<uint4 *>(out + (size_t)n * chunks * 32u);
+        // the first pass's loads go out before the row's table is formed, so that the fp64
+        // products and shuffles overlap their latency
+        uint4 c[4];
+        uint32_t sw[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const uint32_t i = lane + 32u * u;
+            c[u] = i < chunks ? __ldg(crow + i) : make_uint4(0u, 0u, 0u, 0u);
+            sw[u] = i < chunks ? __ldg(srow + i) : 0u;
+        }
         const uint32_t e = f64_to_bf16_rne(lut_q * (double)__ldg(scales + n));
         opqbits::DecodeTable T;
 #pragma unroll
@@ -54,19 +67,8 @@ __global__ void __launch_bounds__(256) dequantize_kernel(const uint32_t *__restr
             T.L[j] = l;
             T.H[j] = h;
         }
-        const uint4 *crow = reinterpret_cast<const uint4 *>(codes + (size_t)n * chunks * 4u);
-        const uint32_t *srow = signs + (size_t)n * chunks;
-        uint4 *orow = reinterpret_cast<uint4 *>(out + (size_t)n * chunks * 32u);
-        // up to four chunks per lane per pass, their loads issued before any decoding
+        // up to four chunks per lane per pass, the next pass's loads issued before decoding
         for (uint32_t i0 = lane; i0 < chunks; i0 += 128u) {
-            uint4 c[4];
-            uint32_t sw[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const uint32_t i = i0 + 32u * u;
-                c[u] = i < chunks ? __ldg(crow + i) : make_uint4(0u, 0u, 0u, 0u);
-                sw[u] = i < chunks ? __ldg(srow + i) : 0u;
-            }
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 const uint32_t i = i0 + 32u * u;
@@ -81,6 +83,13 @@ __global__ void __launch_bounds__(256) dequantize_kernel(const uint32_t *__restr
                 dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
                 dst[2] = make_uint4(o[8], o[9], o[10], o[11]);
                 dst[3] = make_uint4(o[12], o[13], o[14], o[15]);
+            }
+            const uint32_t i1 = i0 + 128u;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const uint32_t i = i1 + 32u * u;
+                c[u] = i < chunks ? __ldg(crow + i) : make_uint4(0u, 0u, 0u, 0u);
+                sw[u] = i < chunks ? __ldg(srow + i) : 0u;
             }
         }
     }
