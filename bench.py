@@ -66,6 +66,23 @@ def recorded_traffic(kernel: str):
     return e.get("dram_bytes_per_launch")
 
 
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The slowest rank's time (all ranks take part; one rank returns its own)."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(world: int, flops_per_replica: float, ms: float) -> float:
+    """Weak-scaling replicas: every rank runs the same step; the job's rate is all ranks' work
+    over the slowest rank's time."""
+    return world * flops_per_replica / (ms * 1e-3) / 1e12
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle-reason samples while the timed region runs."""
 
@@ -200,14 +217,10 @@ def gpu_arm(args, rank, world, local_rank):
     per_step = [e[0].elapsed_time(e[3]) for e in evs]
     live = {name: statistics.fmean(e[a].elapsed_time(e[b]) for e in evs)
             for name, a, b in (("quantize", 0, 1), ("linear", 1, 2), ("dequantize", 2, 3))}
-    ms_step = sum(per_step) / len(per_step)
-    if world > 1:
-        t = torch.tensor([ms_step], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step = float(t.item())
+    ms_step = max_over_ranks(sum(per_step) / len(per_step), world, dev)
     assert opq.device_error() == 0
     flops = 2.0 * M * N * K
-    value = world * flops / (ms_step * 1e-3) / 1e12
+    value = whole_job_tflops(world, flops, ms_step)
 
     # ---- per-kernel timings (events on the launching stream, L2 flushed before each)
     def time_kernel(fn, reps=20):
@@ -309,11 +322,7 @@ def gpu_arm(args, rank, world, local_rank):
         e2e_step()
     eb.record(stream)
     eb.synchronize()
-    ms_e2e = ea.elapsed_time(eb) / args.steps
-    if world > 1:
-        t = torch.tensor([ms_e2e], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_e2e = float(t.item())
+    ms_e2e = max_over_ranks(ea.elapsed_time(eb) / args.steps, world, dev)
     barrier()
 
     traffic = recorded_traffic("wide_kernel")
@@ -329,7 +338,7 @@ def gpu_arm(args, rank, world, local_rank):
                    "step": "quantize W + linear x W'^T + dequantize W'", "parallelism": f"replicas{world}",
                    "l2": "flushed between timed steps (4x L2 buffer write outside the event pairs)"},
         "kernels": kernels, "small_m": small, "roofline": roof, "snr_db": snr,
-        "e2e": {"value": world * flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms_e2e,
+        "e2e": {"value": whole_job_tflops(world, flops, ms_e2e), "unit": "TFLOP/s", "ms_per_step": ms_e2e,
                 "h2d_bytes_per_step": w.numel() * 2 + x.numel() * 2, "d2h_bytes_per_step": y.numel() * 2},
         "gpu_launches": launches_per_step * args.steps,
         "kernels_live_ms": live,
