@@ -13,6 +13,7 @@ namespace opqdev {
 // definition lives here.
 __device__ uint32_t g_error = 0;
 constexpr uint32_t kErrWaitTimeout = 1u;
+constexpr uint32_t kErrSmemAlign = 2u;     // dynamic shared memory not on the 1 KiB boundary
 
 // A bounded wait gives up after this many nanoseconds of %globaltimer.
 constexpr uint64_t kWaitLimitNs = 4000000000ull;   // 4 s

@@ -109,7 +109,7 @@ struct Cfg {
     static constexpr int BW = 128;                     // weight rows per tile (MMA M)
     static constexpr int KR = 128;                     // K per raw (codes/signs) stage
     static constexpr int KA = 64;                      // K per A stage (TMEM) and per x stage (smem)
-    static constexpr int RAW_STAGES = BX >= 256 ? 2 : (BX >= 128 ? 4 : 6);
+    static constexpr int RAW_STAGES = BX >= 256 ? 3 : (BX >= 128 ? 4 : 6);
     static constexpr int A_STAGES = 8;                 // 32 TMEM columns each (64 K of bf16 pairs)
     static constexpr int A_BLOCKS = A_STAGES / 2;      // 128-K blocks of A held in TMEM
     static constexpr int A_COLS = A_STAGES * 32;
@@ -131,7 +131,7 @@ struct Cfg {
     static constexpr int RAW_BYTES = RAW_CODE_BYTES + RAW_SIGN_BYTES;
     static constexpr int X_HALF_BYTES = BX * KA * 2;   // one 64-K half: BX rows x 128 bytes, 128-byte swizzle
     static constexpr int X_BYTES = 2 * X_HALF_BYTES;
-    static constexpr int STAGE_EPI_BYTES = 4 * 2 * 16 * 32 * 2;   // 4 warps x 2 buffers x [16 m][32 n] bf16
+    static constexpr int STAGE_EPI_BYTES = 4 * 16 * 32 * 2;   // 4 warps x [16 m][32 n] bf16
     static constexpr int OFF_TABLE = 0;
     static constexpr int OFF_RAW = OFF_TABLE + (int)opqbits::kPairTableBytes;
     static constexpr int OFF_X = OFF_RAW + RAW_STAGES * RAW_BYTES;
@@ -139,7 +139,9 @@ struct Cfg {
     static constexpr int OFF_BAR = OFF_EPI + STAGE_EPI_BYTES;
     static constexpr int NUM_BARS = 2 * RAW_STAGES + X_STAGES + A_STAGES + NDONE + 2 * NACC + 1;
     static constexpr int OFF_TMEM = OFF_BAR + NUM_BARS * 8;
-    static constexpr int SMEM_BYTES = OFF_TMEM + 16 + 1024;
+    // no alignment slack: the third raw stage needs it, and the kernel checks on entry that the
+    // dynamic window starts on the 1 KiB boundary the swizzled stages need
+    static constexpr int SMEM_BYTES = OFF_TMEM + 16;
     // decoder groups of 4 warps: group g decodes the CTA's 128-K blocks g, g + G, ...;
     // thread r of a group owns weight row r (TMEM lane r) and decodes its whole 128-K block row
     static constexpr int GROUPS = BX >= 256 ? 2 : 3;
@@ -168,11 +170,12 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
                   const __grid_constant__ CUtensorMap tmap_codes, const __grid_constant__ CUtensorMap tmap_signs,
                   const __grid_constant__ LinearArgs args) {
     using C = Cfg<BX>;
-    extern __shared__ uint8_t smem_raw[];
-    const uint32_t raw_base = smem_u32(smem_raw);
-    const uint32_t pad = ((raw_base + 1023u) & ~1023u) - raw_base;
-    uint8_t *smem = smem_raw + pad;
-    const uint32_t sbase = raw_base + pad;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const uint32_t sbase = smem_u32(smem);
+    if ((sbase & 1023u) != 0u) {   // the same for every CTA: nothing has been started yet
+        if (threadIdx.x == 0) atomicOr(&g_error, kErrSmemAlign);
+        return;
+    }
 
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
     uint64_t *raw_full = bars;
@@ -438,11 +441,10 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
         const int row = q * 32 + lane;
         const int64_t U = (int64_t)tiles * args.kblocks;
         const bool vec_y = (args.N % 8) == 0;
-        // per-warp staging for y: 2 buffers of [16 m][32 n] bf16
-        const uint32_t stage0 = sbase + C::OFF_EPI + (uint32_t)(warp - C::WARP_EPI0) * 2048u;
+        // per-warp staging for y: [16 m][32 n] bf16
+        const uint32_t sbuf = sbase + C::OFF_EPI + (uint32_t)(warp - C::WARP_EPI0) * 1024u;
         int ab = 0;
         uint32_t abph = 0;
-        int sb = 0;
         int xoff, xrows;
         while (it.next(tile, r0, r1, j, xoff, xrows, BX)) {
             const int n_blk = tile / args.m_tiles, m_blk = tile % args.m_tiles;
@@ -474,7 +476,6 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
                     const int m0 = m_blk * BX + xoff + c0;
                     if (vec_y && n0 + 32 <= args.N) {
                         // stage [16 m][32 n] bf16, then each lane stores 32 contiguous bytes of one m row
-                        const uint32_t sbuf = stage0 + (uint32_t)sb * 1024u;
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
                             const __nv_bfloat16 o = __float2bfloat16_rn(__uint_as_float(v[i]) * scale);
@@ -490,7 +491,7 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
                             dst[0] = w0;
                             dst[1] = w1;
                         }
-                        sb ^= 1;
+                        __syncwarp();   // the buffer is rewritten by the next 16 columns
                     } else if (n < args.N) {
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {

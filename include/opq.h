@@ -154,10 +154,13 @@ opq_status opq_linear_noalloc(const uint16_t *x, int64_t M, int64_t K, const uin
 /*
  * opq_device_error — reads and clears the library's device-side error word on
  * the current device (synchronises `stream`). 0 = no error; otherwise a bitmask
- * of OPQ_DEVERR_* recorded by a kernel whose bounded wait on a barrier gave up
- * (the kernel then returned early and its output is invalid).
+ * of OPQ_DEVERR_* recorded by a kernel that returned early, leaving its output
+ * invalid: WAIT_TIMEOUT when a bounded wait on a barrier gave up, SMEM_ALIGN when
+ * the dynamic shared-memory window did not start on the 1 KiB boundary that the
+ * 128-byte-swizzled tensor-core operand stages need.
  */
 #define OPQ_DEVERR_WAIT_TIMEOUT 1u
+#define OPQ_DEVERR_SMEM_ALIGN 2u
 opq_status opq_device_error(void *stream, uint32_t *err);
 
 /* Human-readable name of a status. */
