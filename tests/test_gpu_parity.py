@@ -246,6 +246,15 @@ def test_linear_tail_split(M, N, K):
     linear_parity(x, w, 0.73)
 
 
+@pytest.mark.parametrize("M,N,K", [(260, 700, 576), (512, 10240, 192), (257, 300, 64)])
+def test_linear_wide_half_block(M, N, K):
+    # 256-row tiles whose last 128-K block holds one 64-K half (K % 128 == 64): the second half
+    # of that block reads as zeros; the middle case also splits its leftover tiles in two
+    lin = workloads.Linear("half-block", M, N, K, w_seed=M * 3 + K, x_seed=N)
+    x, w = lin.make("cpu")
+    linear_parity(x, w, 0.73)
+
+
 def test_linear_deterministic():
     for M in (16, 700):
         lin = workloads.Linear("det", M, 1024, 1024, w_seed=1, x_seed=2)
