@@ -137,7 +137,7 @@ struct Cfg {
     static constexpr int OFF_X = OFF_RAW + RAW_STAGES * RAW_BYTES;
     static constexpr int OFF_EPI = OFF_X + X_STAGES * X_BYTES;
     static constexpr int OFF_BAR = OFF_EPI + STAGE_EPI_BYTES;
-    static constexpr int NUM_BARS = 2 * RAW_STAGES + X_STAGES + A_STAGES + NDONE + 2 * NACC + 1;
+    static constexpr int NUM_BARS = 2 * RAW_STAGES + A_BLOCKS + NDONE + 2 * NACC + 1;
     static constexpr int OFF_TMEM = OFF_BAR + NUM_BARS * 8;
     // no alignment slack: the third raw stage needs it, and the kernel checks on entry that the
     // dynamic window starts on the 1 KiB boundary the swizzled stages need
@@ -162,6 +162,10 @@ struct Cfg {
     static_assert(A_COLS + NACC * ACC_COLS <= 512, "TMEM columns");
     static_assert(RAW_BYTES % 1024 == 0 && X_BYTES % 1024 == 0, "stage alignment");
     static_assert(A_STAGES % 2 == 0, "a block is two A half-stages");
+    // `ready` slot b % A_BLOCKS takes block b's x copy and its A tile: the x producer re-arms it
+    // for block b only after blk_done of block b - X_STAGES, which must come after the MMAs
+    // that waited on the slot's previous phase (block b - A_BLOCKS)
+    static_assert(A_BLOCKS >= X_STAGES, "ready ring shorter than the x ring");
 };
 
 template <int BX>
@@ -180,9 +184,11 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
     uint64_t *raw_full = bars;
     uint64_t *raw_empty = raw_full + C::RAW_STAGES;
-    uint64_t *x_full = raw_empty + C::RAW_STAGES;
-    uint64_t *a_full = x_full + C::X_STAGES;
-    uint64_t *blk_done = a_full + C::A_STAGES;
+    // ready[b % A_BLOCKS]: block b's x copy has landed (the x producer's expect_tx arrival and
+    // the copy's bytes) and its A tile is in TMEM (one arrival per decoder warp) -- the MMA
+    // issuer waits once per block
+    uint64_t *ready = raw_empty + C::RAW_STAGES;
+    uint64_t *blk_done = ready + C::A_BLOCKS;
     uint64_t *acc_full = blk_done + C::NDONE;
     uint64_t *acc_empty = acc_full + C::NACC;
     uint64_t *drain = acc_empty + C::NACC;
@@ -192,6 +198,71 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
     const int tiles = args.m_tiles * args.n_tiles;
     const bool signs_by_tma = args.signs_tma != 0;
 
+    RunIter it;
+    it.init(args, tiles, gridDim.x, blockIdx.x);
+    int tile, r0, r1, j;
+
+    // one 128-K block of codes and signs (signs by TMA) into raw stage rs
+    auto issue_raw = [&](int rs, int r, int n_blk) {
+        mbar_arrive_expect_tx(&raw_full[rs], C::RAW_BYTES);
+        tma_load_2d(smem + C::OFF_RAW + rs * C::RAW_BYTES, &tmap_codes, r * (C::KR / 8), n_blk * C::BW, &raw_full[rs]);
+        tma_load_2d(smem + C::OFF_RAW + rs * C::RAW_BYTES + C::RAW_CODE_BYTES, &tmap_signs, r * (C::KR / 32),
+                    n_blk * C::BW, &raw_full[rs]);
+    };
+    // the CTA's block b (block r of its tile): x (BX rows, or BX/2 for a half-width run) into
+    // x stage b % X_STAGES, completing on ready[b % A_BLOCKS]
+    auto issue_x = [&](int b, int r, int tile_, int xoff, int xrows) {
+        const bool half = xrows != BX;
+        const void *xmap = half ? (const void *)&tmap_xh : (const void *)&tmap_x;
+        const int xrow = (tile_ % args.m_tiles) * BX + xoff;
+        uint64_t *bar = &ready[b % C::A_BLOCKS];
+        mbar_arrive_expect_tx(bar, half ? C::X_BYTES / 2 : C::X_BYTES);
+        uint8_t *dst = smem + C::OFF_X + (b % C::X_STAGES) * C::X_BYTES;
+        tma_load_2d(dst, xmap, r * C::KR, xrow, bar);
+        tma_load_2d(dst + C::X_HALF_BYTES, xmap, r * C::KR + C::KA, xrow, bar);
+    };
+
+    // The first copies go out before anything else: a cold copy takes microseconds to land,
+    // and building the pair table and allocating TMEM hide most of that. Thread 0 (the raw
+    // producer's lane) initialises every barrier but `ready` and fills the raw ring; the x
+    // producer's lane initialises `ready` and fills the x ring. Nobody else touches a barrier
+    // before the CTA-wide barrier below.
+    int pre_raw = 0, pre_x = 0;   // blocks already issued by the two producers
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::RAW_STAGES; ++s) {
+            // the codes' (and signs') expect_tx arrival, plus 32 cp.async arrivals when signs are copied by threads
+            mbar_init(&raw_full[s], signs_by_tma ? 1 : 1 + 32);
+            mbar_init(&raw_empty[s], 4);          // the 4 warps of the group that decodes the block
+        }
+        for (int s = 0; s < C::NDONE; ++s) mbar_init(&blk_done[s], C::NISS);   // one commit per issuer
+        for (int s = 0; s < C::NACC; ++s) {
+            mbar_init(&acc_full[s], C::NISS);
+            mbar_init(&acc_empty[s], 4);
+        }
+        mbar_init(drain, C::NISS);
+        fence_mbar_init();
+        tma_prefetch_desc(&tmap_codes);
+        if (signs_by_tma) {
+            tma_prefetch_desc(&tmap_signs);
+            RunIter pit = it;
+            while (pre_raw < C::RAW_STAGES && pit.next(tile, r0, r1, j)) {
+                const int n_blk = tile / args.m_tiles;
+                for (int r = r0; r < r1 && pre_raw < C::RAW_STAGES; ++r, ++pre_raw) issue_raw(pre_raw, r, n_blk);
+            }
+        }
+    }
+    if (warp == C::WARP_XLOAD && lane == 0) {
+        // the x producer's expect_tx arrival and the 4 warps of the decoding group
+        for (int s = 0; s < C::A_BLOCKS; ++s) mbar_init(&ready[s], 1 + 4);
+        fence_mbar_init();
+        tma_prefetch_desc(&tmap_x);
+        if (args.tail_split == 2) tma_prefetch_desc(&tmap_xh);
+        RunIter pit = it;
+        int xoff, xrows;
+        while (pre_x < C::X_STAGES && pit.next(tile, r0, r1, j, xoff, xrows, BX)) {
+            for (int r = r0; r < r1 && pre_x < C::X_STAGES; ++r, ++pre_x) issue_x(pre_x, r, tile, xoff, xrows);
+        }
+    }
     // ---- pair table: 32 copies of value(b) then 32 copies of spread(b) per entry b
     for (int e = threadIdx.x; e < 512; e += C::THREADS) {
         const uint32_t b = (uint32_t)e & 255u;
@@ -202,30 +273,6 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
         for (int k = 0; k < 8; ++k)
             asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst + 16u * k), "r"(v) : "memory");
     }
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < C::RAW_STAGES; ++s) {
-            // the codes' (and signs') expect_tx arrival, plus 32 cp.async arrivals when signs are copied by threads
-            mbar_init(&raw_full[s], signs_by_tma ? 1 : 1 + 32);
-            mbar_init(&raw_empty[s], 4);          // the 4 warps of the group that decodes the block
-        }
-        for (int s = 0; s < C::X_STAGES; ++s) mbar_init(&x_full[s], 1);
-        for (int s = 0; s < C::A_STAGES; ++s) mbar_init(&a_full[s], 4);   // the 4 warps of the decoding group
-        for (int s = 0; s < C::NDONE; ++s) mbar_init(&blk_done[s], C::NISS);   // one commit per issuer
-        for (int s = 0; s < C::NACC; ++s) {
-            mbar_init(&acc_full[s], C::NISS);
-            mbar_init(&acc_empty[s], 4);
-        }
-        mbar_init(drain, C::NISS);
-        fence_mbar_init();
-    }
-    if (warp == C::WARP_LOAD && lane == 0) {
-        tma_prefetch_desc(&tmap_codes);
-        if (signs_by_tma) tma_prefetch_desc(&tmap_signs);
-    }
-    if (warp == C::WARP_XLOAD && lane == 0) {
-        tma_prefetch_desc(&tmap_x);
-        if (args.tail_split == 2) tma_prefetch_desc(&tmap_xh);
-    }
     if (warp == C::WARP_MMA) {
         tmem_alloc(tmem_slot, C::TMEM_COLS);
         tmem_relinquish();
@@ -235,10 +282,6 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    RunIter it;
-    it.init(args, tiles, gridDim.x, blockIdx.x);
-    int tile, r0, r1, j;
-
     if (warp == C::WARP_LOAD) {
         // ----------------------------------------------------------- raw producer
         const int swd = args.K / 32;        // sign words per row
@@ -246,9 +289,15 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
         uint32_t rph = 0;
         int raw_issued = 0;
         bool ok = true;
+        pre_raw = __shfl_sync(0xFFFFFFFFu, pre_raw, 0);
         while (ok && it.next(tile, r0, r1, j)) {
             const int n_blk = tile / args.m_tiles;
             for (int r = r0; r < r1 && ok; ++r) {
+                if (raw_issued < pre_raw) {   // issued before the CTA-wide barrier
+                    ++raw_issued;
+                    if (++rs == C::RAW_STAGES) { rs = 0; rph ^= 1; }
+                    continue;
+                }
                 // lane 0 waits for the stage; the verdict and the ordering reach the other lanes
                 int okw = 1;
                 if (lane == 0) okw = mbar_wait(&raw_empty[rs], rph ^ 1) ? 1 : 0;
@@ -257,12 +306,13 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
                 if (!okw) { ok = false; break; }
                 const uint32_t dst = sbase + C::OFF_RAW + rs * C::RAW_BYTES;
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(&raw_full[rs], signs_by_tma ? C::RAW_BYTES : C::RAW_CODE_BYTES);
-                    tma_load_2d(smem + C::OFF_RAW + rs * C::RAW_BYTES, &tmap_codes, r * (C::KR / 8), n_blk * C::BW,
-                                &raw_full[rs]);
-                    if (signs_by_tma)
-                        tma_load_2d(smem + C::OFF_RAW + rs * C::RAW_BYTES + C::RAW_CODE_BYTES, &tmap_signs,
-                                    r * (C::KR / 32), n_blk * C::BW, &raw_full[rs]);
+                    if (signs_by_tma) {
+                        issue_raw(rs, r, n_blk);
+                    } else {
+                        mbar_arrive_expect_tx(&raw_full[rs], C::RAW_CODE_BYTES);
+                        tma_load_2d(smem + C::OFF_RAW + rs * C::RAW_BYTES, &tmap_codes, r * (C::KR / 8),
+                                    n_blk * C::BW, &raw_full[rs]);
+                    }
                 }
                 if (!signs_by_tma) {
                     // sign words: 128 rows x 4 words; copy i of lane l is word 32 i + l of the stage
@@ -299,30 +349,23 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
             bool ok = true;
             int xoff, xrows;
             while (ok && it.next(tile, r0, r1, j, xoff, xrows, BX)) {
-                const int m_blk = tile % args.m_tiles;
-                // a half-width run loads its BX/2 activation rows with the half-height box
-                const bool half = xrows != BX;
-                const void *xmap = half ? (const void *)&tmap_xh : (const void *)&tmap_x;
-                const uint32_t xbytes = half ? C::X_BYTES / 2 : C::X_BYTES;
-                const int xrow = m_blk * BX + xoff;
                 for (int r = r0; r < r1; ++r, ++b) {
+                    if (b < pre_x) continue;   // issued before the CTA-wide barrier
                     // stage b % X_STAGES last held block b - X_STAGES
                     const int prev = b - C::X_STAGES;
                     if (prev >= 0 && !mbar_wait(&blk_done[prev % C::NDONE], (uint32_t)(prev / C::NDONE) & 1u)) {
                         ok = false;
                         break;
                     }
-                    const int xs = b % C::X_STAGES;
-                    mbar_arrive_expect_tx(&x_full[xs], xbytes);
-                    uint8_t *dst = smem + C::OFF_X + xs * C::X_BYTES;
-                    tma_load_2d(dst, xmap, r * C::KR, xrow, &x_full[xs]);
-                    tma_load_2d(dst + C::X_HALF_BYTES, xmap, r * C::KR + C::KA, xrow, &x_full[xs]);
+                    // a half-width run loads its BX/2 activation rows with the half-height box
+                    issue_x(b, r, tile, xoff, xrows);
                 }
             }
             if (!ok) {
-                // let the copies already issued land before the CTA can exit
+                // let the copies already issued land before the CTA can exit (a slot whose decoder
+                // arrivals never come ends this wait by its time limit)
                 for (int i = 1; i <= C::X_STAGES && b - i >= 0; ++i)
-                    (void)mbar_wait(&x_full[(b - i) % C::X_STAGES], (uint32_t)((b - i) / C::X_STAGES) & 1u);
+                    (void)mbar_wait(&ready[(b - i) % C::A_BLOCKS], (uint32_t)((b - i) / C::A_BLOCKS) & 1u);
             }
         }
     } else if (warp == C::WARP_MMA || warp >= C::WARP_ISS1) {
@@ -333,7 +376,7 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
             int ab = 0;
             uint32_t abph = 0;
             int as0 = 0, xs = 0, ds = 0;       // A half-stage of the block's first half, x stage, blk_done slot
-            uint32_t aph = 0, xph = 0;
+            uint32_t rph = 0;                  // parity of ready[as0 / 2]
             bool ok = true;
             constexpr uint32_t idesc_full = idesc_bf16_f32(128, BX);
             constexpr uint32_t idesc_half = idesc_bf16_f32(128, BX / 2);
@@ -346,11 +389,10 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
                 uint32_t acc = 0;              // 0 for the chain's first MMA of the run
                 for (int r = r0; r < r1; ++r) {
                     const uint32_t xaddr = sbase + C::OFF_X + xs * C::X_BYTES;
+                    if (!mbar_wait(&ready[as0 >> 1], rph)) { ok = false; break; }
+                    tc_fence_after();
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
-                        if (!mbar_wait(&a_full[as0 + h], aph)) { ok = false; break; }
-                        if (h == 0 && !mbar_wait(&x_full[xs], xph)) { ok = false; break; }
-                        tc_fence_after();
                         const uint32_t a_tmem = tmem_base + (as0 + h) * 32;
                         const uint64_t bdesc = smem_desc_sw128(xaddr + h * C::X_HALF_BYTES);
 #pragma unroll
@@ -360,11 +402,10 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
                             acc = 1;
                         }
                     }
-                    if (!ok) break;
                     umma_commit(&blk_done[ds]);
                     as0 += 2;
-                    if (as0 == C::A_STAGES) { as0 = 0; aph ^= 1; }
-                    if (++xs == C::X_STAGES) { xs = 0; xph ^= 1; }
+                    if (as0 == C::A_STAGES) { as0 = 0; rph ^= 1; }
+                    if (++xs == C::X_STAGES) xs = 0;
                     if (++ds == C::NDONE) ds = 0;
                 }
                 if (ok) umma_commit(&acc_full[ab]);
@@ -429,10 +470,12 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
                 tc_fence_after();
                 tmem_st_32x32b_x16(tm_row + as * 32, o[0]);
                 tmem_st_32x32b_x16(tm_row + as * 32 + 16, o[1]);
-                tmem_st_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&a_full[as]);
+                if (h == 1) {   // both halves stored: the block's A tile is complete
+                    tmem_st_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&ready[blk % C::A_BLOCKS]);
+                }
             }
         }
     } else {
