@@ -206,11 +206,14 @@ struct Plan {
 
 // The schedule depends on the shape alone (a fixed 148-CTA budget), so the
 // workspace size and the result bits are the same on every B200.
-// Stream-K arrival counters occupy a fixed region at the start of every
-// workspace (4 per weight tile, at most kCounterTiles tiles), so that no shape's
-// partial sums ever land on counters another shape relies on being zero.
+// Arrival counters occupy a fixed region at the start of every workspace (stream-K: 4 per
+// weight tile, at most kCounterTiles tiles; the half-K tail of the wide schedule: 8 per tail
+// tile, at most 74 tail tiles), so that no shape's partial sums ever land on counters another
+// shape relies on being zero.
 constexpr int kCounterTiles = 4096;
 constexpr size_t kCounterBytes = (size_t)kCounterTiles * 4u * sizeof(uint32_t);   // 64 KiB
+// the half-K tail needs this many 128-K blocks to beat splitting the activation rows
+constexpr int kKSplitMinBlocks = 8;
 
 Plan make_plan(int64_t M, int64_t N, int64_t K) {
     Plan p{};
@@ -243,12 +246,23 @@ Plan make_plan(int64_t M, int64_t N, int64_t K) {
         p.grid = (int)(tiles < kPlanSMs ? tiles : kPlanSMs);
         p.runs_max = 1;
         // tiles left after the whole waves: when there are at most half as many as CTAs, each
-        // is split along its activation rows over two CTAs, so that the last wave takes half a
-        // tile's time instead of a whole one
+        // is split over two CTAs, so that the last wave takes about half a tile's time instead
+        // of a whole one. 256-row tiles with at least 8 blocks split K (each CTA decodes half
+        // the tile's weights; the two fp32 partial sums meet in the workspace); otherwise the
+        // activation rows are split (each CTA decodes all of them for half the rows)
         const int64_t tail = tiles - (tiles / p.grid) * p.grid;
-        p.tail_split = (tail > 0 && 2 * tail <= p.grid && p.bx >= 32) ? 2 : 1;
+        p.tail_split = 1;
         p.counter_bytes = 0;
         p.ws_bytes = 0;
+        if (tail > 0 && 2 * tail <= p.grid) {
+            if (p.bx == 256 && p.kblocks >= kKSplitMinBlocks) {
+                p.tail_split = 3;
+                p.counter_bytes = kCounterBytes;
+                p.ws_bytes = p.counter_bytes + (size_t)tail * 256u * 128u * sizeof(float);
+            } else if (p.bx >= 32) {
+                p.tail_split = 2;
+            }
+        }
     }
     p.launches = 1;
     return p;
@@ -301,6 +315,7 @@ cudaError_t launch_linear_wide(DeviceInfo *di, const Plan &plan, const CUtensorM
                                const CUtensorMap &cmap, const CUtensorMap &smap, const opqk::LinearArgs &n,
                                cudaStream_t st) {
     using C = opqk_wide::Cfg<256>;
+    if (plan.mode != 0) return cudaErrorInvalidValue;   // the wide kernel runs whole-tile schedules only
     opqk_wide::LinearArgs a{};
     a.signs = n.signs;
     a.scales = n.scales;

@@ -28,16 +28,18 @@ struct LinearArgs {
     const uint32_t *signs;  // sign plane [N, K/32]
     const float *scales;
     uint16_t *y;
-    float *ws;              // mode 1: fp32 partials [grid][runs_max][BX][128]
-    uint32_t *counters;     // mode 1: arrivals per (tile, TMEM lane quarter); zero between calls
+    float *ws;              // tail_split 3: fp32 partial sums [tail tile][lane quarter][BX m][32 n]
+    uint32_t *counters;     // tail_split 3: per (tail tile, TMEM lane quarter) an arrival count and a
+                            // published flag, 8 words per tail tile; zero between calls
     int signs_tma;          // 1: sign plane rows are 16-byte aligned (K % 128 == 0), load it by TMA
     int M, N, K;
     int m_tiles, n_tiles;
     int kblocks;            // 128-K blocks per tile
-    int mode;               // 0 whole tiles strided over CTAs, 1 contiguous unit ranges (stream-K)
+    int mode;               // 0 whole tiles strided over CTAs (the only mode this kernel is launched with)
     int runs_max;           // mode 1: most runs one CTA can have
-    int tail_split;         // mode 0: 2 = tiles past the last full wave run as two half-width
-                            // (BX/2 activation rows) runs on different CTAs; 1 = whole tiles
+    int tail_split;         // mode 0, tiles past the last whole wave: 2 = each runs as two half-width
+                            // (BX/2 activation rows) runs on two CTAs; 3 = each runs as two
+                            // half-K runs on two CTAs whose partial sums meet in `ws`; 1 = whole
     uint16_t lut[16];       // bf16 (q/15)^(1/alpha)
 };
 
@@ -48,7 +50,7 @@ struct RunIter {
     int64_t u, u_end;   // mode 1
     int t_next;         // mode 0
     int full_end;       // mode 0: tiles in whole waves (handed out strided)
-    int split;          // mode 0: 1 or 2 runs per tile after the whole waves
+    int split;          // mode 0: tail_split
     bool tail_done;
     int run_idx;
     __device__ __forceinline__ void init(const LinearArgs &a, int tiles_, int grid_, int cta_) {
@@ -60,7 +62,7 @@ struct RunIter {
         run_idx = 0;
         t_next = cta_;
         split = a.tail_split;
-        full_end = split == 2 ? (tiles_ / grid_) * grid_ : tiles_;
+        full_end = split >= 2 ? (tiles_ / grid_) * grid_ : tiles_;
         tail_done = false;
         const int64_t U = (int64_t)tiles * kblocks;
         u = unit_begin(cta_, grid_, U);
@@ -75,13 +77,25 @@ struct RunIter {
             if (t_next < full_end) {
                 tile = t_next;
                 t_next += grid;
-            } else if (split == 2) {
-                // tail tile t is run by CTAs 2 (t - full_end) and 2 (t - full_end) + 1, one half each
+            } else if (split >= 2) {
+                // tail tile t is run by CTAs 2 (t - full_end) and 2 (t - full_end) + 1, one half
+                // of its activation rows (split 2) or of its 128-K blocks (split 3) each
                 if (tail_done || cta >= 2 * (tiles - full_end)) return false;
                 tile = full_end + (cta >> 1);
-                xrows = bx / 2;
-                xoff = (cta & 1) * xrows;
                 tail_done = true;
+                r0 = 0;
+                r1 = kblocks;
+                if (split == 2) {
+                    xrows = bx / 2;
+                    xoff = (cta & 1) * xrows;
+                } else {
+                    // the even CTA takes the smaller share of K, so that it has usually published
+                    // its partial sums by the time the odd CTA, which then adds them, is done
+                    const int k0 = kblocks * 7 / 16;
+                    if (cta & 1) r0 = k0; else r1 = k0;
+                }
+                j = run_idx++;
+                return true;
             } else {
                 return false;
             }
@@ -131,13 +145,11 @@ struct Cfg {
     static constexpr int RAW_BYTES = RAW_CODE_BYTES + RAW_SIGN_BYTES;
     static constexpr int X_HALF_BYTES = BX * KA * 2;   // one 64-K half: BX rows x 128 bytes, 128-byte swizzle
     static constexpr int X_BYTES = 2 * X_HALF_BYTES;
-    static constexpr int STAGE_EPI_BYTES = 4 * 16 * 32 * 2;   // 4 warps x [16 m][32 n] bf16
     static constexpr int OFF_TABLE = 0;
     static constexpr int OFF_RAW = OFF_TABLE + (int)opqbits::kPairTableBytes;
     static constexpr int OFF_X = OFF_RAW + RAW_STAGES * RAW_BYTES;
-    static constexpr int OFF_EPI = OFF_X + X_STAGES * X_BYTES;
-    static constexpr int OFF_BAR = OFF_EPI + STAGE_EPI_BYTES;
-    static constexpr int NUM_BARS = 2 * RAW_STAGES + A_BLOCKS + NDONE + 2 * NACC + 1;
+    static constexpr int OFF_BAR = OFF_X + X_STAGES * X_BYTES;
+    static constexpr int NUM_BARS = 2 * RAW_STAGES + A_BLOCKS + NDONE + 2 * NACC + 1 + 4;
     static constexpr int OFF_TMEM = OFF_BAR + NUM_BARS * 8;
     // no alignment slack: the third raw stage needs it, and the kernel checks on entry that the
     // dynamic window starts on the 1 KiB boundary the swizzled stages need
@@ -192,6 +204,7 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
     uint64_t *acc_full = blk_done + C::NDONE;
     uint64_t *acc_empty = acc_full + C::NACC;
     uint64_t *drain = acc_empty + C::NACC;
+    uint64_t *fixb = drain + 1;   // per TMEM lane quarter: the partner's partial sums have landed
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_TMEM);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -240,6 +253,7 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
             mbar_init(&acc_empty[s], 4);
         }
         mbar_init(drain, C::NISS);
+        for (int s = 0; s < 4; ++s) mbar_init(&fixb[s], 1);
         fence_mbar_init();
         tma_prefetch_desc(&tmap_codes);
         if (signs_by_tma) {
@@ -482,13 +496,39 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
         // ----------------------------------------------------------- epilogue
         const int q = warp & 3;
         const int row = q * 32 + lane;
-        const int64_t U = (int64_t)tiles * args.kblocks;
         const bool vec_y = (args.N % 8) == 0;
-        // per-warp staging for y: [16 m][32 n] bf16
-        const uint32_t sbuf = sbase + C::OFF_EPI + (uint32_t)(warp - C::WARP_EPI0) * 1024u;
         int ab = 0;
         uint32_t abph = 0;
         int xoff, xrows;
+        // y[m0 .. m0 + 15][n] = bf16(v[i] * scale) for this lane's weight row n
+        auto store16 = [&](const uint32_t (&v)[16], int m0, int n, int n0, float scale) {
+            if (vec_y && n0 + 32 <= args.N) {
+                // rows m0 + 2i and m0 + 2i + 1 packed as bf16 pairs; lanes n and n ^ 1 swap halves
+                // so that the even lane holds row m0 + 2i and the odd lane row m0 + 2i + 1, each
+                // for weight rows n & ~1 and (n & ~1) + 1: one 4-byte store per lane per row pair
+                const uint32_t odd = (uint32_t)lane & 1u;
+                const uint32_t sel = odd ? 0x3276u : 0x5410u;
+                uint32_t *yw = reinterpret_cast<uint32_t *>(args.y + (size_t)(m0 + (int)odd) * args.N + n0 +
+                                                            (lane & ~1));
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const uint32_t pk = pack_bf16x2_rn(__uint_as_float(v[2 * i]) * scale,
+                                                                __uint_as_float(v[2 * i + 1]) * scale);
+                    const uint32_t other = __shfl_xor_sync(0xFFFFFFFFu, pk, 1);
+                    const uint32_t word = __byte_perm(pk, other, sel);
+                    if (m0 + 2 * i + (int)odd < args.M) yw[(size_t)i * (size_t)args.N] = word;
+                }
+            } else if (n < args.N) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int m = m0 + i;
+                    if (m < args.M) {
+                        const __nv_bfloat16 o = __float2bfloat16_rn(__uint_as_float(v[i]) * scale);
+                        args.y[(size_t)m * args.N + n] = *reinterpret_cast<const uint16_t *>(&o);
+                    }
+                }
+            }
+        };
         while (it.next(tile, r0, r1, j, xoff, xrows, BX)) {
             const int n_blk = tile / args.m_tiles, m_blk = tile % args.m_tiles;
             const int n = n_blk * C::BW + row;
@@ -498,127 +538,79 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
             if (!warp_wait(&acc_full[ab], abph)) break;
             tc_fence_after();
             const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + C::A_COLS + ab * C::ACC_COLS;
-            float *wsp = full ? nullptr
-                              : args.ws + ((size_t)blockIdx.x * args.runs_max + j) * (size_t)(BX * C::BW);
+            if (full) {
 #pragma unroll 1
-            for (int c0 = 0; c0 < xrows; c0 += 16) {
-                uint32_t v[16];
-                tmem_ld_32x32b_x16(taddr + c0, v);
-                if (C::NCHAIN > 1) {
-#pragma unroll
-                    for (int ch = 1; ch < C::NCHAIN; ++ch) {
-                        uint32_t u[16];
-                        tmem_ld_32x32b_x16(taddr + ch * BX + c0, u);
+                for (int c0 = 0; c0 < xrows; c0 += 16) {
+                    uint32_t v[16];
+                    tmem_ld_32x32b_x16(taddr + c0, v);
+                    tmem_ld_wait();
+                    store16(v, m_blk * BX + xoff + c0, n, n0, scale);
+                }
+            } else {
+                // Half-K tail run (the CTA's last): the tile's other half of K ran on the partner
+                // CTA. Per lane quarter, the first of the two to get here publishes its fp32
+                // partial sums to the workspace and raises a flag; the second waits for the flag
+                // (the first is running and waits on nothing), copies the partner's sums in and
+                // writes y from the total. p0 + p1 is the same in either order, so y does not
+                // depend on which CTA arrives first.
+                const int tt = tile - it.full_end;
+                uint32_t *arrivals = args.counters + (size_t)tt * 8 + 2 * q;
+                uint32_t *published = arrivals + 1;
+                float *part = args.ws + ((size_t)tt * 4 + q) * (size_t)(BX * 32);   // [BX m][32 n] fp32
+                uint32_t old = 0;
+                if (lane == 0) old = atomicAdd(arrivals, 1u);
+                old = __shfl_sync(0xFFFFFFFFu, old, 0);
+                if (old == 0) {
+#pragma unroll 1
+                    for (int c0 = 0; c0 < BX; c0 += 16) {
+                        uint32_t v[16];
+                        tmem_ld_32x32b_x16(taddr + c0, v);
                         tmem_ld_wait();
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) + __uint_as_float(u[i]));
+                        for (int i = 0; i < 16; ++i) part[(size_t)(c0 + i) * 32 + lane] = __uint_as_float(v[i]);
                     }
-                }
-                tmem_ld_wait();
-                if (full) {
-                    const int m0 = m_blk * BX + xoff + c0;
-                    if (vec_y && n0 + 32 <= args.N) {
-                        // stage [16 m][32 n] bf16, then each lane stores 32 contiguous bytes of one m row
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const __nv_bfloat16 o = __float2bfloat16_rn(__uint_as_float(v[i]) * scale);
-                            asm volatile("st.shared.u16 [%0], %1;" ::"r"(sbuf + (uint32_t)i * 64u + (uint32_t)lane * 2u),
-                                         "h"(*reinterpret_cast<const unsigned short *>(&o)) : "memory");
-                        }
-                        __syncwarp();
-                        const int mi = lane >> 1, hf = lane & 1;
-                        if (m0 + mi < args.M) {
-                            const uint4 w0 = lds_v4(sbuf + (uint32_t)mi * 64u + (uint32_t)hf * 32u);
-                            const uint4 w1 = lds_v4(sbuf + (uint32_t)mi * 64u + (uint32_t)hf * 32u + 16u);
-                            uint4 *dst = reinterpret_cast<uint4 *>(args.y + (size_t)(m0 + mi) * args.N + n0 + hf * 16);
-                            dst[0] = w0;
-                            dst[1] = w1;
-                        }
-                        __syncwarp();   // the buffer is rewritten by the next 16 columns
-                    } else if (n < args.N) {
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const int m = m0 + i;
-                            if (m < args.M) {
-                                const __nv_bfloat16 o = __float2bfloat16_rn(__uint_as_float(v[i]) * scale);
-                                args.y[(size_t)m * args.N + n] = *reinterpret_cast<const uint16_t *>(&o);
-                            }
-                        }
-                    }
+                    __threadfence();
+                    __syncwarp();
+                    if (lane == 0) flag_store_release(published, 1u);
                 } else {
+                    int okw = 1;
+                    if (lane == 0) okw = flag_wait(published, 1u) ? 1 : 0;
+                    okw = __shfl_sync(0xFFFFFFFFu, okw, 0);
+                    // this is the CTA's last run and its MMAs are complete, so the x ring is idle:
+                    // quarter q's partner sums land in its 32 KiB there
+                    const uint32_t pbuf = sbase + C::OFF_X + (uint32_t)q * (uint32_t)(BX * 32 * 4);
+                    if (okw && lane == 0) {
+                        fence_proxy_async_all();
+                        mbar_arrive_expect_tx(&fixb[q], BX * 32 * 4);
+                        bulk_load(smem + C::OFF_X + q * (BX * 32 * 4), part, BX * 32 * 4, &fixb[q]);
+                    }
+                    if (okw && warp_wait(&fixb[q], 0)) {
+#pragma unroll 1
+                        for (int c0 = 0; c0 < BX; c0 += 16) {
+                            uint32_t v[16];
+                            tmem_ld_32x32b_x16(taddr + c0, v);
+                            tmem_ld_wait();
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) wsp[(size_t)(c0 + i) * C::BW + row] = __uint_as_float(v[i]);
+                            for (int i = 0; i < 16; ++i) {
+                                float o;
+                                asm volatile("ld.shared.f32 %0, [%1];"
+                                             : "=f"(o) : "r"(pbuf + (uint32_t)((c0 + i) * 32 + lane) * 4u));
+                                v[i] = __float_as_uint(__uint_as_float(v[i]) + o);
+                            }
+                            store16(v, m_blk * BX + c0, n, n0, scale);
+                        }
+                    }
+                    // ready for the next call (after a timeout the workspace must be zeroed again)
+                    if (lane == 0) {
+                        arrivals[0] = 0u;
+                        published[0] = 0u;
+                    }
                 }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[ab]);
             if (++ab == C::NACC) { ab = 0; abph ^= 1; }
-            if (!full) {
-                // The last of the tile's CTAs to get here (per lane quarter) adds every
-                // CTA's partial rows in CTA order, so the sum does not depend on timing.
-                const int64_t c_lo = unit_owner((int64_t)tile * args.kblocks, gridDim.x, U);
-                const int64_t c_hi = unit_owner((int64_t)(tile + 1) * args.kblocks - 1, gridDim.x, U);
-                const uint32_t parts = (uint32_t)(c_hi - c_lo + 1);
-                __threadfence();
-                __syncwarp();
-                uint32_t old = 0;
-                if (lane == 0) old = atomicAdd(args.counters + (size_t)tile * 4 + q, 1u);
-                old = __shfl_sync(0xFFFFFFFFu, old, 0);
-                if (old == parts - 1) {
-                    __threadfence();
-                    // lane i (< parts) resolves part i's base; bases are broadcast by shuffles
-                    const float *mybase = nullptr;
-                    if ((uint32_t)lane < parts) {
-                        const int64_t c = c_lo + lane;
-                        const int64_t jj = tile - unit_begin(c, gridDim.x, U) / args.kblocks;
-                        mybase = args.ws + ((size_t)c * args.runs_max + (size_t)jj) * (size_t)(BX * C::BW);
-                    }
-                    // Every lane runs the loops (shuffles need all lanes); only rows < N store.
-                    // 8 columns per pass, the next part's 8 loads issued before the current
-                    // part's adds; each sum still runs over parts 0, 1, ... from 0.0f.
-                    auto part_base = [&](uint32_t p) -> const float * {
-                        if (p < 32)
-                            return reinterpret_cast<const float *>(
-                                __shfl_sync(0xFFFFFFFFu, reinterpret_cast<unsigned long long>(mybase), (int)p));
-                        const int64_t c = c_lo + p;
-                        const int64_t jj = tile - unit_begin(c, gridDim.x, U) / args.kblocks;
-                        return args.ws + ((size_t)c * args.runs_max + (size_t)jj) * (size_t)(BX * C::BW);
-                    };
-                    const int mcols = min(BX, args.M - m_blk * BX);
-                    for (int c0 = 0; c0 < mcols; c0 += 8) {
-                        float acc[8], cur[8], nxt[8];
-                        const float *b0 = part_base(0) + (size_t)c0 * C::BW + row;
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            acc[i] = 0.0f;
-                            cur[i] = (c0 + i < mcols) ? __ldcg(b0 + (size_t)i * C::BW) : 0.0f;
-                        }
-                        for (uint32_t p = 0; p < parts; ++p) {
-                            if (p + 1 < parts) {
-                                const float *bn = part_base(p + 1) + (size_t)c0 * C::BW + row;
-#pragma unroll
-                                for (int i = 0; i < 8; ++i) nxt[i] = (c0 + i < mcols) ? __ldcg(bn + (size_t)i * C::BW) : 0.0f;
-                            }
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) {
-                                acc[i] += cur[i];
-                                cur[i] = nxt[i];
-                            }
-                        }
-                        if (n < args.N) {
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) {
-                                if (c0 + i < mcols) {
-                                    const __nv_bfloat16 o = __float2bfloat16_rn(acc[i] * scale);
-                                    args.y[(size_t)(m_blk * BX + c0 + i) * args.N + n] = *reinterpret_cast<const uint16_t *>(&o);
-                                }
-                            }
-                        }
-                    }
-                    if (lane == 0) atomicExch(args.counters + (size_t)tile * 4 + q, 0u);   // ready for the next call
-                }
-            }
         }
     }
 

@@ -108,12 +108,23 @@ def test_plan_and_workspace_host_logic(lib):
         runs_max = -(-per // groups) + 1
         counters = 4096 * 4 * 4        # fixed region: 4 arrival counters for each of up to 4096 weight tiles
         assert opq.workspace_size(M, N, K) == counters + ctas * runs_max * bx * 128 * 4
-    # large M: whole 128 x 256 tiles, one persistent CTA per SM, no workspace
-    for M, N, K in [(129, 100, 32), (3072, 3840, 3840), (4096, 10240, 3840), (8, 4097 * 128, 64)]:
+    # large M: whole 128 x 256 tiles, one persistent CTA per SM. Tiles past the last whole wave,
+    # when at most half as many as CTAs, run on two CTAs each; 256-row tiles of at least 8
+    # 128-K blocks split K, and their fp32 partial sums (128 x 256 per tail tile) meet in the
+    # workspace after the counter region; everything else needs no workspace
+    for M, N, K in [(129, 100, 32), (3072, 3840, 3840), (4096, 10240, 3840), (8, 4097 * 128, 64),
+                    (512, 10240, 256), (512, 10240, 1024), (300, 9728, 160)]:
         path, ctas, launches = opq.plan(M, N, K)
         assert path == 0 and launches == 1
-        assert ctas == min(148, -(-M // 256) * -(-N // 128))
-        assert opq.workspace_size(M, N, K) == 0
+        bx = 256 if M > 128 else 128
+        tiles = -(-M // bx) * -(-N // 128)
+        assert ctas == min(148, tiles)
+        tail = tiles - (tiles // ctas) * ctas
+        ksplit = bx == 256 and 0 < tail and 2 * tail <= ctas and -(-K // 128) >= 8
+        want = 4096 * 4 * 4 + tail * 256 * 128 * 4 if ksplit else 0
+        assert opq.workspace_size(M, N, K) == want
+    assert opq.workspace_size(3072, 3840, 3840) == 65536 + 64 * 131072     # 360 tiles: 64 past 2 waves
+    assert opq.workspace_size(512, 10240, 1024) == 65536 + 12 * 131072     # 160 tiles: 12 past 1 wave
     sz = ctypes.c_size_t(0)
     assert lib.opq_linear_workspace_size(0, 4, 32, ctypes.byref(sz)) == 1
     assert lib.opq_linear_workspace_size(4, 4, 40, ctypes.byref(sz)) == 2

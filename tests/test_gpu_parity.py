@@ -255,9 +255,39 @@ def test_linear_wide_half_block(M, N, K):
     linear_parity(x, w, 0.73)
 
 
+@pytest.mark.parametrize("M,N,K", [(512, 10240, 1024), (300, 9728, 1152)])
+def test_linear_tail_ksplit(M, N, K):
+    # the tiles past the last whole wave each run as two half-K runs on two CTAs whose fp32
+    # partial sums meet in the workspace (3 + 5 and 3 + 6 blocks; the second has a ragged m-tile)
+    lin = workloads.Linear("tail-k", M, N, K, w_seed=M + K, x_seed=N)
+    x, w = lin.make("cpu")
+    linear_parity(x, w, 0.73)
+
+
+def test_linear_ksplit_workspace_reuse():
+    # one zero-filled workspace serves repeated calls: y is bitwise the same each time and the
+    # arrival counters at the workspace start are back at zero after every call
+    M, N, K = 512, 10240, 1024
+    need = opq.workspace_size(M, N, K)
+    assert need > 65536
+    lin = workloads.Linear("ws-reuse", M, N, K, w_seed=3, x_seed=4)
+    x, w = lin.make(DEV)
+    planes = opq.quantize(w)
+    ws = torch.zeros(need, dtype=torch.uint8, device=DEV)
+    ys = []
+    for _ in range(3):
+        ys.append(opq.linear(x, *planes, workspace=ws))
+        torch.cuda.synchronize()
+        assert int(ws[:65536].count_nonzero()) == 0
+        no_device_error()
+    assert torch.equal(ys[0], ys[1]) and torch.equal(ys[0], ys[2])
+    assert torch.equal(ys[0], opq.linear_noalloc(x, *planes))
+
+
 def test_linear_deterministic():
-    for M in (16, 700):
-        lin = workloads.Linear("det", M, 1024, 1024, w_seed=1, x_seed=2)
+    for M in (16, 700, 512):
+        N = 10240 if M == 512 else 1024   # 512 x 10240: a half-K tail
+        lin = workloads.Linear("det", M, N, 1024, w_seed=1, x_seed=2)
         x, w = lin.make(DEV)
         planes = opq.quantize(w)
         y1 = opq.linear(x, *planes)
