@@ -266,7 +266,7 @@ struct Cfg {
     static constexpr int OFF_X = OFF_RAW + RAW_STAGES * RAW_BYTES;
     static constexpr int OFF_EPI = OFF_X + X_STAGES * X_BYTES;
     static constexpr int OFF_BAR = OFF_EPI + STAGE_EPI_BYTES;
-    static constexpr int NUM_BARS = 2 * RAW_STAGES + X_STAGES + A_STAGES + NDONE + 2 * NACC + 1;
+    static constexpr int NUM_BARS = 2 * RAW_STAGES + X_STAGES + A_BLOCKS + NDONE + 2 * NACC + 1;
     static constexpr int OFF_TMEM = OFF_BAR + NUM_BARS * 8;
     static constexpr int SMEM_BYTES = OFF_TMEM + 16 + 1024;
     // decoder groups of 4 warps: group g decodes the CTA's 128-K blocks g, g + G, ...;
@@ -307,8 +307,8 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
     uint64_t *raw_full = bars;
     uint64_t *raw_empty = raw_full + C::RAW_STAGES;
     uint64_t *x_full = raw_empty + C::RAW_STAGES;
-    uint64_t *a_full = x_full + C::X_STAGES;
-    uint64_t *blk_done = a_full + C::A_STAGES;
+    uint64_t *a_full = x_full + C::X_STAGES;    // per A slot (128-K block): its A tile is in TMEM
+    uint64_t *blk_done = a_full + C::A_BLOCKS;
     uint64_t *acc_full = blk_done + C::NDONE;
     uint64_t *acc_empty = acc_full + C::NACC;
     uint64_t *drain = acc_empty + C::NACC;
@@ -326,7 +326,7 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
             mbar_init(&raw_empty[s], 4 * C::GRP);
         }
         for (int s = 0; s < C::X_STAGES; ++s) mbar_init(&x_full[s], 1);
-        for (int s = 0; s < C::A_STAGES; ++s) mbar_init(&a_full[s], 4);   // the 4 warps of the decoding group
+        for (int s = 0; s < C::A_BLOCKS; ++s) mbar_init(&a_full[s], 4);   // the 4 warps of the decoding group
         for (int s = 0; s < C::NDONE; ++s) mbar_init(&blk_done[s], C::NISS);   // one commit per issuer
         for (int s = 0; s < C::NACC; ++s) {
             mbar_init(&acc_full[s], C::NISS);
@@ -491,10 +491,12 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
                     if (!mbar_wait(&x_full[xs], xph)) { ok = false; break; }
                     const uint32_t xbase = sbase + C::OFF_X + xs * C::X_BYTES;
                     for (int jj = 0; jj < nb; ++jj) {
+                        // one wait per block: a wait right before an MMA costs the issuing thread
+                        // about as much as the MMAs of a narrow block
+                        if (!mbar_wait(&a_full[as0 >> 1], aph)) { ok = false; break; }
+                        tc_fence_after();
 #pragma unroll
                         for (int h = 0; h < 2; ++h) {
-                            if (!mbar_wait(&a_full[as0 + h], aph)) { ok = false; break; }
-                            tc_fence_after();
                             const uint32_t a_tmem = tmem_base + (as0 + h) * 32;
                             const uint64_t bdesc = smem_desc_sw128(xbase + (2 * jj + h) * C::X_HALF_BYTES);
                             // K-steps iss, iss + NISS, ...: a fixed count per issuer and no branch
@@ -595,10 +597,12 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
                         tc_fence_after();
                         tmem_st_32x32b_x16(tm_row + as * 32, o[0]);
                         tmem_st_32x32b_x16(tm_row + as * 32 + 16, o[1]);
-                        tmem_st_wait();
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&a_full[as]);
+                        if (h == 1) {   // both halves stored: the block's A tile is complete
+                            tmem_st_wait();
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(&a_full[blk % C::A_BLOCKS]);
+                        }
                     }
                     if (!ok) break;
                 }
