@@ -528,14 +528,14 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
         // ----------------------------------------------------------- decoders
         // The pair table (only the decoders read it) is built here, while the producers' first
         // copies are in flight: 32 copies of value(b) then 32 copies of spread(b) per entry b.
-        for (int e = threadIdx.x - C::WARP_DEC0 * 32; e < 512; e += C::NUM_DEC_WARPS * 32) {
+        // A warp writes whole entries (lane l the l-th copy), so the LUT entries it reads are the
+        // same in every lane: one broadcast load each instead of up to 16 serialised ones.
+        for (int e = warp - C::WARP_DEC0; e < 512; e += C::NUM_DEC_WARPS) {
             const uint32_t b = (uint32_t)e & 255u;
             const uint32_t v = e < 256 ? ((uint32_t)args.lut[b & 15u] | ((uint32_t)args.lut[b >> 4] << 16))
                                        : opqbits::sign_spread(b);
-            const uint32_t dst = sbase + C::OFF_TABLE + b * 256u + (e < 256 ? 0u : 128u);
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-                asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst + 16u * k), "r"(v) : "memory");
+            const uint32_t dst = sbase + C::OFF_TABLE + b * 256u + (e < 256 ? 0u : 128u) + 4u * (uint32_t)lane;
+            asm volatile("st.shared.u32 [%0], %1;" ::"r"(dst), "r"(v) : "memory");
         }
         // all decoder warps (named barrier 1) see the whole table before decoding
         asm volatile("bar.sync 1, %0;" ::"r"(C::NUM_DEC_WARPS * 32) : "memory");
