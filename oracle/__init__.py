@@ -50,6 +50,16 @@ def _bind(path: str):
     lib.oracle_uniform_int4.argtypes = [P, I, I, P]
     lib.oracle_double_to_bf16.argtypes = [D]
     lib.oracle_double_to_bf16.restype = ctypes.c_uint16
+    lib.oracle_quantize_grouped.argtypes = [P, I, I, I, I, D, P, P, P, P, P]
+    lib.oracle_quantize_grouped.restype = None
+    lib.oracle_dequantize_grouped_f64.argtypes = [P, P, P, I, I, I, D, P]
+    lib.oracle_dequantize_grouped_bf16.argtypes = [P, P, P, I, I, I, D, P]
+    lib.oracle_linear_grouped.argtypes = [P, I, I, P, P, P, I, I, D, P, P]
+    lib.oracle_linear_grouped_pairs.argtypes = [P, I, I, P, P, P, I, I, D, I, P, P, P, P]
+    lib.oracle_fp16_value.argtypes = [ctypes.c_uint16]
+    lib.oracle_fp16_value.restype = D
+    lib.oracle_fp16_from_nonneg.argtypes = [D]
+    lib.oracle_fp16_from_nonneg.restype = ctypes.c_uint16
     lib.oracle_rounding_mode_ok.restype = ctypes.c_int
     lib.oracle_num_threads.restype = ctypes.c_int
     return lib
@@ -155,6 +165,83 @@ class Oracle:
                                     ms.size, _p(ms), _p(ns), _p(y), _p(b))
         return y, b
 
+    # ---- group-wise variant: one float16 max per GS consecutive weights of a row ----
+    def quantize_grouped(self, w, gs: int, alpha: float, want_ties: bool = False, want_v15: bool = False):
+        """OPQ-quantize bf16 W[N, K] group by group (GS weights per group along K).
+
+        Returns dict(codes uint32[N, K/8], signs uint32[N, K/32], gmax uint16[N, K/GS] (float16
+        bits), near_tie uint8[N, K] | None, v15 float64[N, K] | None).
+        """
+        w = _u16(w)
+        N, K = w.shape
+        assert K % 32 == 0 and K % gs == 0
+        lib = self._lib
+        assert lib.oracle_rounding_mode_ok() == 1
+        codes = np.zeros((N, K // 8), np.uint32)
+        signs = np.zeros((N, K // 32), np.uint32)
+        gmax = np.zeros((N, K // gs), np.uint16)
+        ties = np.zeros((N, K), np.uint8) if want_ties else None
+        v15 = np.zeros((N, K), np.float64) if want_v15 else None
+        lib.oracle_quantize_grouped(_p(w), N, K, K, int(gs), float(alpha), _p(codes), _p(signs), _p(gmax),
+                                    _p(ties) if ties is not None else None,
+                                    _p(v15) if v15 is not None else None)
+        return dict(codes=codes, signs=signs, gmax=gmax, near_tie=ties, v15=v15)
+
+    def _grouped_planes(self, codes, signs, gmax):
+        codes = np.ascontiguousarray(codes, np.uint32)
+        signs = np.ascontiguousarray(signs, np.uint32)
+        gmax = np.ascontiguousarray(gmax, np.uint16)
+        N, cw = codes.shape
+        K = cw * 8
+        assert gmax.shape[0] == N and K % gmax.shape[1] == 0
+        return codes, signs, gmax, N, K, K // gmax.shape[1]
+
+    def dequantize_grouped_f64(self, codes, signs, gmax, alpha: float) -> np.ndarray:
+        codes, signs, gmax, N, K, gs = self._grouped_planes(codes, signs, gmax)
+        out = np.zeros((N, K), np.float64)
+        self._lib.oracle_dequantize_grouped_f64(_p(codes), _p(signs), _p(gmax), N, K, gs, float(alpha), _p(out))
+        return out
+
+    def dequantize_grouped_bf16(self, codes, signs, gmax, alpha: float) -> np.ndarray:
+        """Returns uint16 bf16 bit patterns [N, K]."""
+        codes, signs, gmax, N, K, gs = self._grouped_planes(codes, signs, gmax)
+        out = np.zeros((N, K), np.uint16)
+        self._lib.oracle_dequantize_grouped_bf16(_p(codes), _p(signs), _p(gmax), N, K, gs, float(alpha), _p(out))
+        return out
+
+    def linear_grouped(self, x, codes, signs, gmax, alpha: float):
+        """y = x @ W'^T in fp64 with its error bound B = |x| @ |W'|^T. Returns (y, B)."""
+        x = _u16(x)
+        M, K = x.shape
+        codes, signs, gmax, N, Kc, gs = self._grouped_planes(codes, signs, gmax)
+        assert Kc == K
+        y = np.zeros((M, N), np.float64)
+        b = np.zeros((M, N), np.float64)
+        self._lib.oracle_linear_grouped(_p(x), M, K, _p(codes), _p(signs), _p(gmax), N, gs, float(alpha),
+                                        _p(y), _p(b))
+        return y, b
+
+    def linear_grouped_pairs(self, x, codes, signs, gmax, alpha: float, ms, ns):
+        x = _u16(x)
+        M, K = x.shape
+        codes, signs, gmax, N, Kc, gs = self._grouped_planes(codes, signs, gmax)
+        assert Kc == K
+        ms = np.ascontiguousarray(ms, np.int64)
+        ns = np.ascontiguousarray(ns, np.int64)
+        assert ms.shape == ns.shape
+        assert (ms >= 0).all() and (ms < M).all() and (ns >= 0).all() and (ns < N).all()
+        y = np.zeros(ms.shape, np.float64)
+        b = np.zeros(ms.shape, np.float64)
+        self._lib.oracle_linear_grouped_pairs(_p(x), M, K, _p(codes), _p(signs), _p(gmax), N, gs, float(alpha),
+                                              ms.size, _p(ms), _p(ns), _p(y), _p(b))
+        return y, b
+
+    def fp16_value(self, bits: int) -> float:
+        return float(self._lib.oracle_fp16_value(int(bits)))
+
+    def fp16_from_nonneg(self, v: float) -> int:
+        return int(self._lib.oracle_fp16_from_nonneg(float(v)))
+
     def snr_db(self, w, w_rec: np.ndarray) -> float:
         w = _u16(w)
         w_rec = np.ascontiguousarray(w_rec, np.float64)
@@ -210,6 +297,34 @@ def linear_pairs(*a, **k):
 
 def snr_db(*a, **k):
     return default().snr_db(*a, **k)
+
+
+def quantize_grouped(*a, **k):
+    return default().quantize_grouped(*a, **k)
+
+
+def dequantize_grouped_f64(*a, **k):
+    return default().dequantize_grouped_f64(*a, **k)
+
+
+def dequantize_grouped_bf16(*a, **k):
+    return default().dequantize_grouped_bf16(*a, **k)
+
+
+def linear_grouped(*a, **k):
+    return default().linear_grouped(*a, **k)
+
+
+def linear_grouped_pairs(*a, **k):
+    return default().linear_grouped_pairs(*a, **k)
+
+
+def fp16_value(*a, **k):
+    return default().fp16_value(*a, **k)
+
+
+def fp16_from_nonneg(*a, **k):
+    return default().fp16_from_nonneg(*a, **k)
 
 
 def uniform_int4(*a, **k):

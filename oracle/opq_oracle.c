@@ -13,8 +13,9 @@
  * decoding" (w = sign * (q/15)^(1/alpha) * max).
  *
  * Readings where the page is silent or is overridden by the task contract:
- *   - max|w| is taken per output row (row n of W[N,K]) and stored as fp32;
- *     the page uses a per-128 group max in fp16.
+ *   - max|w| is taken per output row (row n of W[N,K]) and stored as fp32
+ *     (the per-row format); the page's own per-group float16 max is the
+ *     group-wise variant further down, with its readings there.
  *   - round() is round-half-to-even on the exact real value, here evaluated
  *     with nearbyint() under the default rounding mode.
  *   - for alpha == 1 the power is the identity and v*15 is evaluated as
@@ -102,6 +103,46 @@ uint16_t oracle_double_to_bf16(double x) { return double_to_bf16_rne(x); }
 /* near_tie (optional, may be NULL): one byte per element, 1 = |v15 - (floor + .5)| <= 1e-6 */
 /* v15_out (optional): the oracle's 15 * u^alpha per element                  */
 /* ------------------------------------------------------------------------ */
+/* max |w| over row[k0 .. k1) */
+static double max_abs(const uint16_t *row, int64_t k0, int64_t k1)
+{
+    double mx = 0.0;
+    for (int64_t k = k0; k < k1; ++k) {
+        double a = fabs(bf16_value(row[k]));
+        if (a > mx)
+            mx = a;
+    }
+    return mx;
+}
+
+/* steps 2-4 for element k of row n against the max mx: code and sign into the packed planes
+ * (cw code words and sw sign words per row, both zeroed beforehand), the near-tie flag and
+ * 15 u^alpha */
+static void quantize_element(double wk, double mx, double alpha, int64_t n, int64_t k, int64_t K,
+                             int64_t cw, int64_t sw, uint32_t *codes, uint32_t *signs,
+                             uint8_t *near_tie, double *v15_out)
+{
+    double a = fabs(wk);
+    double v15;
+    if (mx == 0.0)
+        v15 = 0.0;
+    else if (alpha == 1.0)
+        v15 = (15.0 * a) / mx;                 /* u^1 = u */
+    else
+        v15 = 15.0 * pow(a / mx, alpha);       /* 15 * u^alpha */
+    double qd = nearbyint(v15);                /* ties to even */
+    if (qd < 0.0) qd = 0.0;
+    if (qd > OPQ_LEVELS) qd = OPQ_LEVELS;
+    uint32_t q = (uint32_t)qd;
+    uint32_t s = (wk < 0.0) ? 1u : 0u;
+    codes[n * cw + k / 8] |= q << (4 * (k % 8));
+    signs[n * sw + k / 32] |= s << (k % 32);
+    if (near_tie)
+        near_tie[n * K + k] = (fabs(v15 - (floor(v15) + 0.5)) <= 1e-6) ? 1 : 0;
+    if (v15_out)
+        v15_out[n * K + k] = v15;
+}
+
 void oracle_quantize(const uint16_t *w, int64_t N, int64_t K, int64_t ldw, double alpha,
                      uint32_t *codes, uint32_t *signs, float *scales,
                      uint8_t *near_tie, double *v15_out)
@@ -111,39 +152,14 @@ void oracle_quantize(const uint16_t *w, int64_t N, int64_t K, int64_t ldw, doubl
     for (int64_t n = 0; n < N; ++n) {
         const uint16_t *row = w + n * ldw;
         /* step 1: max |w| over the row */
-        double mx = 0.0;
-        for (int64_t k = 0; k < K; ++k) {
-            double a = fabs(bf16_value(row[k]));
-            if (a > mx)
-                mx = a;
-        }
+        double mx = max_abs(row, 0, K);
         scales[n] = (float)mx;  /* exact: mx is a bf16 value */
         for (int64_t j = 0; j < cw; ++j)
             codes[n * cw + j] = 0;
         for (int64_t j = 0; j < sw; ++j)
             signs[n * sw + j] = 0;
-        for (int64_t k = 0; k < K; ++k) {
-            double wk = bf16_value(row[k]);
-            double a = fabs(wk);
-            double v15;
-            if (mx == 0.0)
-                v15 = 0.0;
-            else if (alpha == 1.0)
-                v15 = (15.0 * a) / mx;                 /* u^1 = u */
-            else
-                v15 = 15.0 * pow(a / mx, alpha);       /* 15 * u^alpha */
-            double qd = nearbyint(v15);                /* ties to even */
-            if (qd < 0.0) qd = 0.0;
-            if (qd > OPQ_LEVELS) qd = OPQ_LEVELS;
-            uint32_t q = (uint32_t)qd;
-            uint32_t s = (wk < 0.0) ? 1u : 0u;
-            codes[n * cw + k / 8] |= q << (4 * (k % 8));
-            signs[n * sw + k / 32] |= s << (k % 32);
-            if (near_tie)
-                near_tie[n * K + k] = (fabs(v15 - (floor(v15) + 0.5)) <= 1e-6) ? 1 : 0;
-            if (v15_out)
-                v15_out[n * K + k] = v15;
-        }
+        for (int64_t k = 0; k < K; ++k)
+            quantize_element(bf16_value(row[k]), mx, alpha, n, k, K, cw, sw, codes, signs, near_tie, v15_out);
     }
 }
 
@@ -192,9 +208,25 @@ void oracle_dequantize_bf16(const uint32_t *codes, const uint32_t *signs, const 
 /* linear: y[m, n] = sum_k x[m, k] * w'[n, k] (fp64, unrounded w'),          */
 /* bound[m, n] = sum_k |x[m, k]| * |w'[n, k]|                                */
 /* ------------------------------------------------------------------------ */
-void oracle_linear(const uint16_t *x, int64_t M, int64_t K,
-                   const uint32_t *codes, const uint32_t *signs, const float *scales,
-                   int64_t N, double alpha, double *y, double *bound)
+/* where w'[n, k] comes from: one scale per row, or one float16 max per group */
+typedef struct {
+    const uint32_t *codes, *signs;
+    const float *scales;     /* per row, or NULL */
+    const uint16_t *gmax;    /* per group (float16 bits), or NULL */
+    int64_t K, GS;
+    double alpha;
+} planes_t;
+
+static double group_max_at(const uint16_t *gmax, int64_t K, int64_t GS, int64_t n, int64_t k);
+
+static double wprime(const planes_t *p, int64_t n, int64_t k)
+{
+    double mx = p->scales ? (double)p->scales[n] : group_max_at(p->gmax, p->K, p->GS, n, k);
+    return dequant_value(code_at(p->codes, p->K, n, k), sign_at(p->signs, p->K, n, k), p->alpha, mx);
+}
+
+static void linear_rows(const uint16_t *x, int64_t M, int64_t K, const planes_t *p, int64_t N,
+                        double *y, double *bound)
 {
 #pragma omp parallel
     {
@@ -203,8 +235,7 @@ void oracle_linear(const uint16_t *x, int64_t M, int64_t K,
 #pragma omp for schedule(dynamic, 1)
         for (int64_t n = 0; n < N; ++n) {
             for (int64_t k = 0; k < K; ++k)
-                wrow[k] = dequant_value(code_at(codes, K, n, k), sign_at(signs, K, n, k),
-                                        alpha, (double)scales[n]);
+                wrow[k] = wprime(p, n, k);
             for (int64_t m = 0; m < M; ++m) {
                 double acc = 0.0, b = 0.0;
                 for (int64_t k = 0; k < K; ++k) {
@@ -222,20 +253,15 @@ void oracle_linear(const uint16_t *x, int64_t M, int64_t K,
 }
 
 /* the same sum for an explicit list of (m, n) output positions */
-void oracle_linear_pairs(const uint16_t *x, int64_t M, int64_t K,
-                         const uint32_t *codes, const uint32_t *signs, const float *scales,
-                         int64_t N, double alpha, int64_t count, const int64_t *ms,
-                         const int64_t *ns, double *y, double *bound)
+static void linear_list(const uint16_t *x, int64_t K, const planes_t *p, int64_t count,
+                        const int64_t *ms, const int64_t *ns, double *y, double *bound)
 {
-    (void)M;
-    (void)N;
 #pragma omp parallel for schedule(dynamic, 16)
     for (int64_t i = 0; i < count; ++i) {
         int64_t m = ms[i], n = ns[i];
         double acc = 0.0, b = 0.0;
         for (int64_t k = 0; k < K; ++k) {
-            double wv = dequant_value(code_at(codes, K, n, k), sign_at(signs, K, n, k),
-                                      alpha, (double)scales[n]);
+            double wv = wprime(p, n, k);
             double xv = bf16_value(x[m * K + k]);
             acc += xv * wv;
             b += fabs(xv) * fabs(wv);
@@ -244,6 +270,150 @@ void oracle_linear_pairs(const uint16_t *x, int64_t M, int64_t K,
         if (bound)
             bound[i] = b;
     }
+}
+
+void oracle_linear(const uint16_t *x, int64_t M, int64_t K,
+                   const uint32_t *codes, const uint32_t *signs, const float *scales,
+                   int64_t N, double alpha, double *y, double *bound)
+{
+    planes_t p = {codes, signs, scales, NULL, K, K, alpha};
+    linear_rows(x, M, K, &p, N, y, bound);
+}
+
+void oracle_linear_pairs(const uint16_t *x, int64_t M, int64_t K,
+                         const uint32_t *codes, const uint32_t *signs, const float *scales,
+                         int64_t N, double alpha, int64_t count, const int64_t *ms,
+                         const int64_t *ns, double *y, double *bound)
+{
+    (void)M;
+    (void)N;
+    planes_t p = {codes, signs, scales, NULL, K, K, alpha};
+    linear_list(x, K, &p, count, ms, ns, y, bound);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Group-wise variant: the model card's own storage format ("Technical        */
+/* details / storage format": one float16 group max shared by every 128       */
+/* weights; its "OPQ configuration" lists group sizes 32, 64, 128 and 256).   */
+/* A group is GS consecutive weights of one row (K % GS == 0). Readings:      */
+/*   - the group max is max|w| over the group, stored as IEEE binary16,       */
+/*     rounded to nearest even; a max beyond the largest finite float16       */
+/*     (65504) saturates to it instead of becoming infinity;                  */
+/*   - quantization and decoding both use the stored float16 max, so that     */
+/*     they agree (for a max in float16's normal range the conversion is      */
+/*     exact: a bf16 value has 8 significant bits, float16 has 11);           */
+/*   - |w| above a max that rounded down (float16's subnormal range) gives    */
+/*     u > 1 and a code clamped to 15; a group whose stored max is 0          */
+/*     quantizes to all-zero codes; the rest as for the per-row format.       */
+/* ------------------------------------------------------------------------ */
+
+/* float16 bit pattern -> exact double, from the binary16 definition */
+static double fp16_value(uint16_t bits)
+{
+    int s = (bits >> 15) & 1, e = (bits >> 10) & 0x1F, m = bits & 0x3FF;
+    double v;
+    if (e == 0)
+        v = ldexp((double)m, -24);                    /* subnormal: m * 2^-24 */
+    else if (e == 0x1F)
+        v = m ? NAN : INFINITY;
+    else
+        v = ldexp((double)(1024 + m), e - 25);         /* (1 + m/1024) * 2^(e-15) */
+    return s ? -v : v;
+}
+
+/* non-negative double -> float16 bit pattern: 11 significant bits at the value's binade
+ * (binade floored at the subnormal quantum 2^-24), round to nearest even, saturating at
+ * 65504 */
+static uint16_t nonneg_to_fp16_rne_sat(double a)
+{
+    if (!(a > 0.0))
+        return 0;
+    int e;
+    (void)frexp(a, &e);                 /* a = m * 2^e, m in [0.5, 1) */
+    int qexp = e - 11;
+    if (qexp < -24)
+        qexp = -24;
+    double v = ldexp(nearbyint(ldexp(a, -qexp)), qexp);
+    if (v > 65504.0)
+        v = 65504.0;
+    if (v < ldexp(1.0, -14))            /* subnormal (or zero): v / 2^-24 quanta */
+        return (uint16_t)ldexp(v, 24);
+    (void)frexp(v, &e);                 /* v = m * 2^e, m in [0.5, 1) */
+    int field = e - 1 + 15;
+    uint16_t mant = (uint16_t)(ldexp(v, 11 - e) - 1024.0);   /* exact: v has <= 11 bits */
+    return (uint16_t)((field << 10) | mant);
+}
+
+double oracle_fp16_value(uint16_t bits) { return fp16_value(bits); }
+uint16_t oracle_fp16_from_nonneg(double a) { return nonneg_to_fp16_rne_sat(a); }
+
+/* gmax: uint16 float16 bits [N, K / GS] */
+void oracle_quantize_grouped(const uint16_t *w, int64_t N, int64_t K, int64_t ldw, int64_t GS,
+                             double alpha, uint32_t *codes, uint32_t *signs, uint16_t *gmax,
+                             uint8_t *near_tie, double *v15_out)
+{
+    const int64_t cw = K / 8, sw = K / 32, ng = K / GS;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n) {
+        const uint16_t *row = w + n * ldw;
+        for (int64_t j = 0; j < cw; ++j)
+            codes[n * cw + j] = 0;
+        for (int64_t j = 0; j < sw; ++j)
+            signs[n * sw + j] = 0;
+        for (int64_t g = 0; g < ng; ++g) {
+            /* step 1: max |w| over the group, kept as float16 */
+            uint16_t gb = nonneg_to_fp16_rne_sat(max_abs(row, g * GS, (g + 1) * GS));
+            gmax[n * ng + g] = gb;
+            /* steps 2-4 per weight, against the stored max */
+            for (int64_t k = g * GS; k < (g + 1) * GS; ++k)
+                quantize_element(bf16_value(row[k]), fp16_value(gb), alpha, n, k, K, cw, sw, codes, signs,
+                                 near_tie, v15_out);
+        }
+    }
+}
+
+static double group_max_at(const uint16_t *gmax, int64_t K, int64_t GS, int64_t n, int64_t k)
+{
+    return fp16_value(gmax[n * (K / GS) + k / GS]);
+}
+
+void oracle_dequantize_grouped_f64(const uint32_t *codes, const uint32_t *signs, const uint16_t *gmax,
+                                   int64_t N, int64_t K, int64_t GS, double alpha, double *out)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k)
+            out[n * K + k] = dequant_value(code_at(codes, K, n, k), sign_at(signs, K, n, k), alpha,
+                                           group_max_at(gmax, K, GS, n, k));
+}
+
+void oracle_dequantize_grouped_bf16(const uint32_t *codes, const uint32_t *signs, const uint16_t *gmax,
+                                    int64_t N, int64_t K, int64_t GS, double alpha, uint16_t *out)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k)
+            out[n * K + k] = double_to_bf16_rne(dequant_value(code_at(codes, K, n, k), sign_at(signs, K, n, k),
+                                                              alpha, group_max_at(gmax, K, GS, n, k)));
+}
+
+void oracle_linear_grouped(const uint16_t *x, int64_t M, int64_t K, const uint32_t *codes,
+                           const uint32_t *signs, const uint16_t *gmax, int64_t N, int64_t GS,
+                           double alpha, double *y, double *bound)
+{
+    planes_t p = {codes, signs, NULL, gmax, K, GS, alpha};
+    linear_rows(x, M, K, &p, N, y, bound);
+}
+
+void oracle_linear_grouped_pairs(const uint16_t *x, int64_t M, int64_t K, const uint32_t *codes,
+                                 const uint32_t *signs, const uint16_t *gmax, int64_t N, int64_t GS,
+                                 double alpha, int64_t count, const int64_t *ms, const int64_t *ns,
+                                 double *y, double *bound)
+{
+    (void)M;
+    (void)N;
+    planes_t p = {codes, signs, NULL, gmax, K, GS, alpha};
+    linear_list(x, K, &p, count, ms, ns, y, bound);
 }
 
 /* ------------------------------------------------------------------------ */

@@ -292,3 +292,121 @@ def pin_snr_ordering(orc):
 PINS = [pin_golden_fixtures, pin_alpha1_exact_rational, pin_max_zero_monotone,
         pin_bruteforce_nearest_level, pin_threshold_identity, pin_lut_decimal,
         pin_roundtrip_idempotent, pin_linear, pin_bf16_rounding, pin_snr_ordering]
+
+
+# ------------------------------------------------- group-wise variant pins --
+def pin_fp16_conversion(orc):
+    """float16 decode and encode against numpy's binary16 (an independent implementation)."""
+    bits = np.arange(0x7C00, dtype=np.uint16)                  # every non-negative finite pattern
+    want = bits.view(np.float16).astype(np.float64)
+    got = np.array([orc.fp16_value(int(b)) for b in bits[::7]])
+    assert np.array_equal(got, want[::7])
+    assert orc.fp16_value(0x8001) == -(2.0 ** -24)
+    # encode every positive finite bf16 value (RNE; beyond 65504 the reading saturates)
+    pos = np.arange(1, 0x7F80, 3, dtype=np.uint16)
+    vals = bits_to_f64(pos)
+    enc = np.array([orc.fp16_from_nonneg(float(v)) for v in vals], dtype=np.uint16)
+    inrange = vals <= 65504.0
+    ref = vals[inrange].astype(np.float16).view(np.uint16)
+    assert np.array_equal(enc[inrange], ref)
+    assert (enc[~inrange] == 0x7BFF).all()
+    # hand-derived: 1.0, 65504, 0.10009765625 = bf16 0x3DCD, 2^-24, 2^-20 + 2^-27 (rounds down)
+    assert orc.fp16_from_nonneg(1.0) == 0x3C00
+    assert orc.fp16_from_nonneg(65504.0) == 0x7BFF
+    assert orc.fp16_from_nonneg(0.10009765625) == 0x2E68
+    assert orc.fp16_from_nonneg(2.0 ** -24) == 0x0001
+    assert orc.fp16_from_nonneg(2.0 ** -20 + 2.0 ** -27) == 0x0010
+    assert orc.fp16_from_nonneg(0.0) == 0
+    # 11 significant bits survive; ties go to even (1 + 2^-11 -> 1.0, 1 + 3 * 2^-11 -> 1 + 2^-9)
+    assert orc.fp16_from_nonneg(1.0 + 2.0 ** -10) == 0x3C01
+    assert orc.fp16_from_nonneg(1.0 + 2.0 ** -11) == 0x3C00
+    assert orc.fp16_from_nonneg(1.0 + 3 * 2.0 ** -11) == 0x3C02
+    # arbitrary doubles across float16's range against numpy's conversion
+    rng = np.random.default_rng(3)
+    v = np.exp(rng.uniform(np.log(2.0 ** -26), np.log(60000.0), 4000))
+    got = np.array([orc.fp16_from_nonneg(float(a)) for a in v], dtype=np.uint16)
+    assert np.array_equal(got, v.astype(np.float16).view(np.uint16))
+
+
+def _grouped_weights(N, K, seed):
+    g = torch.Generator().manual_seed(seed)
+    w = torch.randn(N, K, generator=g, dtype=torch.float64) * 0.02
+    w[:, ::17] *= 6.0                                          # a few larger weights per group
+    return w.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16).copy()
+
+
+def pin_grouped_is_rowwise_per_group(orc):
+    """Group-wise quantization of W[N, K] with group size GS is the per-row quantization of W
+    reshaped to [N K / GS, GS] (each group a row), with the row max stored as float16."""
+    N, K = 6, 1024
+    w = _grouped_weights(N, K, 11)
+    for gs in (32, 64, 128, 256):
+        for alpha in (0.45, 0.73, 1.0):
+            rg = orc.quantize_grouped(w, gs, alpha, want_ties=True)
+            rr = orc.quantize(w.reshape(N * K // gs, gs), alpha, want_ties=True)
+            assert np.array_equal(rg["codes"].reshape(-1), rr["codes"].reshape(-1))
+            assert np.array_equal(rg["signs"].reshape(-1), rr["signs"].reshape(-1))
+            assert np.array_equal(rg["near_tie"].reshape(-1), rr["near_tie"].reshape(-1))
+            want_g = rr["scales"].astype(np.float16).view(np.uint16)   # exact: maxima in float16's normal range
+            assert np.array_equal(rg["gmax"].reshape(-1), want_g)
+            dg = orc.dequantize_grouped_f64(rg["codes"], rg["signs"], rg["gmax"], alpha)
+            dr = orc.dequantize_f64(rr["codes"], rr["signs"], rr["scales"], alpha)
+            assert np.array_equal(dg.reshape(-1), dr.reshape(-1))
+            bg = orc.dequantize_grouped_bf16(rg["codes"], rg["signs"], rg["gmax"], alpha)
+            br = orc.dequantize_bf16(rr["codes"], rr["signs"], rr["scales"], alpha)
+            assert np.array_equal(bg.reshape(-1), br.reshape(-1))
+
+
+def pin_grouped_worked_example(orc):
+    """One 32-weight group by hand: max 0.5 (float16 0x3800), u = 1, 1/2, 1/4, 1/8, 0 at
+    alpha 0.73 -> 15 u^alpha = 15, 9.04, 5.45, 3.29, 0 -> codes 15, 9, 5, 3, 0; a second group
+    of the same row holds only zeros (max 0: all codes 0, sign of -0.0 is 0)."""
+    row = [0.5, -0.25, 0.125, 0.0625, 0.0] + [0.0] * 27 + [0.0, -0.0] + [0.0] * 30
+    w = bf16_bits(row).reshape(1, 64)
+    r = orc.quantize_grouped(w, 32, 0.73)
+    q = unpack_codes(r["codes"])[0]
+    s = unpack_signs(r["signs"])[0]
+    assert list(q[:5]) == [15, 9, 5, 3, 0] and not q[5:].any()
+    assert list(s[:5]) == [0, 1, 0, 0, 0] and not s[5:].any()
+    assert list(r["gmax"][0]) == [0x3800, 0]
+    d = orc.dequantize_grouped_f64(r["codes"], r["signs"], r["gmax"], 0.73)[0]
+    assert d[0] == 0.5 and d[1] == -((9 / 15) ** (1 / 0.73)) * 0.5 and not d[32:].any()
+
+
+def pin_grouped_range_edges(orc):
+    """A max beyond float16 saturates to 65504 (codes of larger weights clamp at 15); a max in
+    float16's subnormal range rounds (2^-20 + 2^-27 -> 2^-20) and the max itself codes to 15."""
+    big = [1e5 if i == 3 else 0.0 for i in range(32)]
+    tiny_max = 2.0 ** -20 + 2.0 ** -27
+    tiny = [tiny_max if i == 5 else (2.0 ** -22 if i == 6 else 0.0) for i in range(32)]
+    big_b = bf16_bits([float(torch.tensor(v).to(torch.bfloat16)) for v in big])
+    w = np.concatenate([big_b, bf16_bits(tiny)]).reshape(1, 64)
+    r = orc.quantize_grouped(w, 32, 0.73)
+    q = unpack_codes(r["codes"])[0]
+    assert list(r["gmax"][0]) == [0x7BFF, 0x0010]
+    assert q[3] == 15 and q[32 + 5] == 15
+    # 2^-22 / 2^-20 = 1/4 -> 15 * 0.25^0.73 = 5.45 -> 5
+    assert q[32 + 6] == 5
+
+
+def pin_grouped_linear(orc):
+    """The group-wise linear is x @ W'^T with W' the group-wise dequantization (numpy fp64
+    matmul as the independent sum), and the pair list agrees with the full product."""
+    N, K, M = 40, 512, 7
+    w = _grouped_weights(N, K, 5)
+    g = torch.Generator().manual_seed(6)
+    x = torch.randn(M, K, generator=g).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16).copy()
+    for gs in (64, 128):
+        r = orc.quantize_grouped(w, gs, 0.73)
+        wd = orc.dequantize_grouped_f64(r["codes"], r["signs"], r["gmax"], 0.73)
+        y, b = orc.linear_grouped(x, r["codes"], r["signs"], r["gmax"], 0.73)
+        xf = bits_to_f64(x)
+        assert np.allclose(y, xf @ wd.T, rtol=1e-12, atol=1e-12)
+        assert np.allclose(b, np.abs(xf) @ np.abs(wd).T, rtol=1e-12, atol=1e-12)
+        ms = np.array([0, 6, 3, 2]); ns = np.array([0, 39, 17, 5])
+        yp, bp = orc.linear_grouped_pairs(x, r["codes"], r["signs"], r["gmax"], 0.73, ms, ns)
+        assert np.array_equal(yp, y[ms, ns]) and np.array_equal(bp, b[ms, ns])
+
+
+PINS += [pin_fp16_conversion, pin_grouped_is_rowwise_per_group, pin_grouped_worked_example,
+         pin_grouped_range_edges, pin_grouped_linear]

@@ -32,11 +32,20 @@ MUTANTS = [
      "double xv = bf16_value(x[k * M + m]);\n                    acc += xv * wrow[k];"),
     ("pairs_n_for_m", "int64_t m = ms[i], n = ns[i];", "int64_t m = ms[i], n = ms[i];"),
     ("bound_signed", "b += fabs(xv) * fabs(wrow[k]);", "b += xv * wrow[k];"),
-    ("max_signed", "double a = fabs(bf16_value(row[k]));\n            if (a > mx)",
-     "double a = bf16_value(row[k]);\n            if (a > mx)"),
+    ("max_signed", "double a = fabs(bf16_value(row[k]));\n        if (a > mx)",
+     "double a = bf16_value(row[k]);\n        if (a > mx)"),
     ("bf16_round_half_up", "double r = nearbyint(ldexp(a, -qexp));", "double r = floor(ldexp(a, -qexp) + 0.5);"),
     ("bf16_truncate", "double r = nearbyint(ldexp(a, -qexp));", "double r = floor(ldexp(a, -qexp));"),
     ("near_tie_band_wide", "<= 1e-6) ? 1 : 0;", "<= 1e-3) ? 1 : 0;"),
+    # group-wise variant
+    ("group_index_wrapped", "return fp16_value(gmax[n * (K / GS) + k / GS]);",
+     "return fp16_value(gmax[n * (K / GS) + k % (K / GS)]);"),
+    ("group_max_cumulative", "max_abs(row, g * GS, (g + 1) * GS)", "max_abs(row, 0, (g + 1) * GS)"),
+    ("fp16_truncate", "double v = ldexp(nearbyint(ldexp(a, -qexp)), qexp);",
+     "double v = ldexp(floor(ldexp(a, -qexp)), qexp);"),
+    ("fp16_ten_bits", "int qexp = e - 11;", "int qexp = e - 10;"),
+    ("fp16_no_saturation", "if (v > 65504.0)\n        v = 65504.0;", "if (v > 1e30)\n        v = 65504.0;"),
+    ("fp16_subnormal_floor", "if (qexp < -24)\n        qexp = -24;", "if (qexp < -25)\n        qexp = -25;"),
 ]
 
 
