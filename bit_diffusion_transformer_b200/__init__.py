@@ -28,7 +28,7 @@ _STATUS = {0: "OPQ_OK", 1: "OPQ_ERR_INVALID_ARG", 2: "OPQ_ERR_UNSUPPORTED_SHAPE"
 
 EXPORTS = ["opq_quantize", "opq_dequantize", "opq_linear_workspace_size", "opq_linear", "opq_linear_plan",
            "opq_linear_noalloc", "opq_device_error", "opq_status_string", "opq_last_cuda_error",
-           "opq_abi_version"]
+           "opq_abi_version", "opq_quantize_grouped", "opq_dequantize_grouped"]
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 
@@ -59,10 +59,12 @@ def load(path: str = LIB_PATH):
                                     ctypes.POINTER(ctypes.c_int)]
     lib.opq_linear_noalloc.argtypes = [P, I, I, P, P, P, I, F, P, P]
     lib.opq_device_error.argtypes = [P, ctypes.POINTER(ctypes.c_uint32)]
+    lib.opq_quantize_grouped.argtypes = [P, I, I, I, I, F, P, P, P, P]
+    lib.opq_dequantize_grouped.argtypes = [P, P, P, I, I, I, F, P, P]
     lib.opq_status_string.argtypes = [ctypes.c_int]
     lib.opq_status_string.restype = ctypes.c_char_p
     for f in ("opq_quantize", "opq_dequantize", "opq_linear_workspace_size", "opq_linear", "opq_linear_plan",
-              "opq_linear_noalloc", "opq_device_error"):
+              "opq_linear_noalloc", "opq_device_error", "opq_quantize_grouped", "opq_dequantize_grouped"):
         getattr(lib, f).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -113,6 +115,35 @@ def dequantize(codes: torch.Tensor, signs: torch.Tensor, scales: torch.Tensor, a
     w = out if out is not None else torch.empty((N, K), dtype=torch.bfloat16, device=codes.device)
     _check(load().opq_dequantize(_ptr(codes), _ptr(signs), _ptr(scales), N, K, float(alpha), _ptr(w),
                                  _stream(codes.device)), "opq_dequantize")
+    return w
+
+
+def quantize_grouped(w: torch.Tensor, group_size: int = 128, alpha: float = ALPHA, out=None):
+    """Group-wise OPQ of bf16 W[N, K] -> (codes, signs, gmax float16 [N, K/group_size])."""
+    assert w.dtype == torch.bfloat16 and w.dim() == 2
+    _need_cuda(w)
+    N, K = w.shape
+    if out is None:
+        codes = torch.empty((N, K // 8), dtype=torch.int32, device=w.device)
+        signs = torch.empty((N, K // 32), dtype=torch.int32, device=w.device)
+        gmax = torch.empty((N, K // group_size), dtype=torch.float16, device=w.device)
+    else:
+        codes, signs, gmax = out
+    _check(load().opq_quantize_grouped(_ptr(w), N, K, K, int(group_size), float(alpha), _ptr(codes), _ptr(signs),
+                                       _ptr(gmax), _stream(w.device)), "opq_quantize_grouped")
+    return codes, signs, gmax
+
+
+def dequantize_grouped(codes: torch.Tensor, signs: torch.Tensor, gmax: torch.Tensor, alpha: float = ALPHA,
+                       out=None):
+    """Group-wise packed planes -> bf16 W'[N, K] (the group size is K / gmax.shape[1])."""
+    _need_cuda(codes, signs, gmax)
+    N, cw = codes.shape
+    K = cw * 8
+    gs = K // gmax.shape[1]
+    w = out if out is not None else torch.empty((N, K), dtype=torch.bfloat16, device=codes.device)
+    _check(load().opq_dequantize_grouped(_ptr(codes), _ptr(signs), _ptr(gmax), N, K, gs, float(alpha), _ptr(w),
+                                         _stream(codes.device)), "opq_dequantize_grouped")
     return w
 
 

@@ -12,6 +12,7 @@
 
 #include "opq.h"
 #include "opq_dequantize.cuh"
+#include "opq_grouped.cuh"
 #include "opq_linear.cuh"
 #include "opq_linear_wide.cuh"
 #include "opq_quantize.cuh"
@@ -391,6 +392,70 @@ opq_status opq_quantize(const uint16_t *w, int64_t N, int64_t K, int64_t ldw, fl
         const int64_t blocks = N;
         const int grid = (int)(blocks < (int64_t)di->sms * 8 ? blocks : (int64_t)di->sms * 8);
         dispatch_quant<8>(vpl, w, N, K, ldw, qp, codes, signs, scales, grid, st);
+    }
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? OPQ_OK : cuda_fail(e);
+}
+
+// group-wise format: group size 32, 64, 128 or 256 dividing K
+static opq_status check_group(int64_t K, int64_t gs) {
+    if (gs != 32 && gs != 64 && gs != 128 && gs != 256) return OPQ_ERR_INVALID_ARG;
+    if (K % gs != 0) return OPQ_ERR_UNSUPPORTED_SHAPE;
+    return OPQ_OK;
+}
+
+opq_status opq_quantize_grouped(const uint16_t *w, int64_t N, int64_t K, int64_t ldw, int64_t group_size,
+                                float alpha, uint32_t *codes, uint32_t *signs, uint16_t *gmax, void *stream) {
+    opq_status s = check_sizes(N, K);
+    if (s != OPQ_OK) return s;
+    if ((s = check_group(K, group_size)) != OPQ_OK) return s;
+    if (ldw < K || ldw % 8 != 0) return OPQ_ERR_INVALID_ARG;
+    if (!alpha_ok(alpha)) return OPQ_ERR_INVALID_ARG;
+    if ((s = check_ptrs({w, codes, signs, gmax})) != OPQ_OK) return s;
+    opqk::QuantParams qp{};
+    const double inv = 1.0 / (double)alpha;
+    qp.t[0] = 0.0;
+    for (int k = 1; k < 16; ++k) qp.t[k] = std::pow(((double)k - 0.5) / 15.0, inv);
+    qp.alpha_is_one = (alpha == 1.0f) ? 1 : 0;
+    DeviceInfo *di = nullptr;
+    if ((s = device_info(&di)) != OPQ_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    // one warp per row, 8 rows per block
+    const int64_t blocks = (N + 7) / 8;
+    const int grid = (int)(blocks < (int64_t)di->sms * 8 ? blocks : (int64_t)di->sms * 8);
+    switch (group_size) {
+        case 32: opqk::quantize_grouped_kernel<32><<<grid, 256, 0, st>>>(w, N, K, ldw, qp, codes, signs, gmax); break;
+        case 64: opqk::quantize_grouped_kernel<64><<<grid, 256, 0, st>>>(w, N, K, ldw, qp, codes, signs, gmax); break;
+        case 128: opqk::quantize_grouped_kernel<128><<<grid, 256, 0, st>>>(w, N, K, ldw, qp, codes, signs, gmax); break;
+        default: opqk::quantize_grouped_kernel<256><<<grid, 256, 0, st>>>(w, N, K, ldw, qp, codes, signs, gmax); break;
+    }
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? OPQ_OK : cuda_fail(e);
+}
+
+opq_status opq_dequantize_grouped(const uint32_t *codes, const uint32_t *signs, const uint16_t *gmax, int64_t N,
+                                  int64_t K, int64_t group_size, float alpha, uint16_t *w_out, void *stream) {
+    opq_status s = check_sizes(N, K);
+    if (s != OPQ_OK) return s;
+    if ((s = check_group(K, group_size)) != OPQ_OK) return s;
+    if (!alpha_ok(alpha)) return OPQ_ERR_INVALID_ARG;
+    if ((uint64_t)N * (uint64_t)(K / 8) >= (1ull << 40)) return OPQ_ERR_UNSUPPORTED_SHAPE;
+    if ((s = check_ptrs({codes, signs, gmax, w_out})) != OPQ_OK) return s;
+    opqk::DequantParams dp{};
+    const double inv = 1.0 / (double)alpha;
+    for (int q = 0; q < 16; ++q) dp.lut[q] = std::pow((double)q / 15.0, inv);
+    DeviceInfo *di = nullptr;
+    if ((s = device_info(&di)) != OPQ_OK) return s;
+    uint64_t blocks = ((uint64_t)N + 7) / 8;
+    const uint64_t cap = (uint64_t)di->sms * 16;
+    if (blocks > cap) blocks = cap;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const uint32_t rows = (uint32_t)N, chunks = (uint32_t)(K / 32);
+    switch (group_size) {
+        case 32: opqk::dequantize_grouped_kernel<32><<<(int)blocks, 256, 0, st>>>(codes, signs, gmax, rows, chunks, dp, w_out); break;
+        case 64: opqk::dequantize_grouped_kernel<64><<<(int)blocks, 256, 0, st>>>(codes, signs, gmax, rows, chunks, dp, w_out); break;
+        case 128: opqk::dequantize_grouped_kernel<128><<<(int)blocks, 256, 0, st>>>(codes, signs, gmax, rows, chunks, dp, w_out); break;
+        default: opqk::dequantize_grouped_kernel<256><<<(int)blocks, 256, 0, st>>>(codes, signs, gmax, rows, chunks, dp, w_out); break;
     }
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? OPQ_OK : cuda_fail(e);

@@ -83,6 +83,35 @@ opq_status opq_dequantize(const uint32_t *codes, const uint32_t *signs, const fl
                           int64_t N, int64_t K, float alpha, uint16_t *w_out, void *stream);
 
 /*
+ * Group-wise format — the card's own storage ("Technical details / storage
+ * format": one float16 max shared by every 128 weights; its configuration also
+ * lists group sizes 32, 64 and 256). Row n's weights k = g*GS .. g*GS + GS - 1
+ * form group g; u = |w| / gmax[n, g] with gmax the group's max |w| stored as
+ * IEEE float16 (round to nearest even, saturating at 65504), the stored value
+ * being the one both quantization and decoding use. Codes and signs are packed
+ * exactly as in the per-row format:
+ *   codes  uint32   [N, K/8]
+ *   signs  uint32   [N, K/32]
+ *   gmax   float16  [N, K/GS] (passed as 16-bit patterns)
+ * group_size must be 32, 64, 128 or 256 (OPQ_ERR_INVALID_ARG otherwise) and
+ * divide K (OPQ_ERR_UNSUPPORTED_SHAPE otherwise). A group whose stored max is
+ * 0 has all-zero codes; weights above a max that rounded down in float16's
+ * subnormal range code to 15.
+ *
+ * opq_quantize_grouped — as opq_quantize, one max per group; any K (no
+ * register-resident row).
+ */
+opq_status opq_quantize_grouped(const uint16_t *w, int64_t N, int64_t K, int64_t ldw, int64_t group_size,
+                                float alpha, uint32_t *codes, uint32_t *signs, uint16_t *gmax, void *stream);
+
+/*
+ * opq_dequantize_grouped — w'[n, k] = bf16(sign * (q/15)^(1/alpha) * gmax[n, k / GS]),
+ * the product formed in fp64 and rounded once (round to nearest even).
+ */
+opq_status opq_dequantize_grouped(const uint32_t *codes, const uint32_t *signs, const uint16_t *gmax, int64_t N,
+                                  int64_t K, int64_t group_size, float alpha, uint16_t *w_out, void *stream);
+
+/*
  * opq_linear_workspace_size — device scratch bytes opq_linear needs for an
  * M x K by (N x K)^T product (0 when the chosen kernel needs none).
  */
