@@ -28,7 +28,8 @@ _STATUS = {0: "OPQ_OK", 1: "OPQ_ERR_INVALID_ARG", 2: "OPQ_ERR_UNSUPPORTED_SHAPE"
 
 EXPORTS = ["opq_quantize", "opq_dequantize", "opq_linear_workspace_size", "opq_linear", "opq_linear_plan",
            "opq_linear_noalloc", "opq_device_error", "opq_status_string", "opq_last_cuda_error",
-           "opq_abi_version", "opq_quantize_grouped", "opq_dequantize_grouped"]
+           "opq_abi_version", "opq_quantize_grouped", "opq_dequantize_grouped",
+           "opq_linear_grouped", "opq_linear_grouped_workspace_size"]
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 
@@ -61,10 +62,13 @@ def load(path: str = LIB_PATH):
     lib.opq_device_error.argtypes = [P, ctypes.POINTER(ctypes.c_uint32)]
     lib.opq_quantize_grouped.argtypes = [P, I, I, I, I, F, P, P, P, P]
     lib.opq_dequantize_grouped.argtypes = [P, P, P, I, I, I, F, P, P]
+    lib.opq_linear_grouped.argtypes = [P, I, I, P, P, P, I, I, F, P, P, S, P]
+    lib.opq_linear_grouped_workspace_size.argtypes = [I, I, I, I, ctypes.POINTER(S)]
     lib.opq_status_string.argtypes = [ctypes.c_int]
     lib.opq_status_string.restype = ctypes.c_char_p
     for f in ("opq_quantize", "opq_dequantize", "opq_linear_workspace_size", "opq_linear", "opq_linear_plan",
-              "opq_linear_noalloc", "opq_device_error", "opq_quantize_grouped", "opq_dequantize_grouped"):
+              "opq_linear_noalloc", "opq_device_error", "opq_quantize_grouped", "opq_dequantize_grouped", "opq_linear_grouped",
+              "opq_linear_grouped_workspace_size"):
         getattr(lib, f).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -145,6 +149,32 @@ def dequantize_grouped(codes: torch.Tensor, signs: torch.Tensor, gmax: torch.Ten
     _check(load().opq_dequantize_grouped(_ptr(codes), _ptr(signs), _ptr(gmax), N, K, gs, float(alpha), _ptr(w),
                                          _stream(codes.device)), "opq_dequantize_grouped")
     return w
+
+
+def grouped_workspace_size(M: int, N: int, K: int, group_size: int) -> int:
+    b = ctypes.c_size_t(0)
+    _check(load().opq_linear_grouped_workspace_size(M, N, K, int(group_size), ctypes.byref(b)),
+           "opq_linear_grouped_workspace_size")
+    return int(b.value)
+
+
+def linear_grouped(x: torch.Tensor, codes: torch.Tensor, signs: torch.Tensor, gmax: torch.Tensor,
+                   alpha: float = ALPHA, out=None, workspace=None):
+    """y = x @ W'^T for bf16 x[M, K] and a group-wise packed W[N, K] -> bf16 y[M, N]."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2
+    _need_cuda(x, codes, signs, gmax)
+    M, K = x.shape
+    N = codes.shape[0]
+    gs = K // gmax.shape[1]
+    y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    need = grouped_workspace_size(M, N, K, gs)
+    if need and workspace is None:
+        workspace = torch.zeros((need,), dtype=torch.uint8, device=x.device)   # must start zeroed
+    ws_ptr = _ptr(workspace) if workspace is not None else ctypes.c_void_p(0)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(load().opq_linear_grouped(_ptr(x), M, K, _ptr(codes), _ptr(signs), _ptr(gmax), N, gs, float(alpha),
+                                     _ptr(y), ws_ptr, ws_bytes, _stream(x.device)), "opq_linear_grouped")
+    return y
 
 
 def workspace_size(M: int, N: int, K: int) -> int:

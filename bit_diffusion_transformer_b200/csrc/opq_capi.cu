@@ -66,7 +66,7 @@ uint16_t host_bf16(double v) {
 
 struct DeviceInfo {
     int sms = 0;
-    bool linear_attr[17] = {false};
+    bool linear_attr[21] = {false};   // narrow BX / 16, 16 = wide, 17 .. 20 = wide group-wise (GS 32 .. 256)
 };
 std::mutex g_mu;
 DeviceInfo g_dev[64];
@@ -216,11 +216,12 @@ constexpr size_t kCounterBytes = (size_t)kCounterTiles * 4u * sizeof(uint32_t); 
 // the half-K tail needs this many 128-K blocks to beat splitting the activation rows
 constexpr int kKSplitMinBlocks = 8;
 
-Plan make_plan(int64_t M, int64_t N, int64_t K) {
+// `wide`: 256-row tiles for every M (the group-wise format has only the wide kernel)
+Plan make_plan(int64_t M, int64_t N, int64_t K, bool wide = false) {
     Plan p{};
     p.kblocks = (int)((K + 127) / 128);
     p.n_tiles = (int)((N + 127) / 128);
-    if (M <= 128) {
+    if (M <= 128 && !wide) {
         p.bx = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
         // the narrow tiles fetch several 128-K blocks per copy through 3-D views of the planes,
         // which need whole blocks (K % 128 == 0); other K take the one-block-per-copy width
@@ -233,7 +234,7 @@ Plan make_plan(int64_t M, int64_t N, int64_t K) {
     // blocks per load group: must match the kernel's Cfg<BX>::GRP
     p.grp = p.bx <= 16 ? 4 : (p.bx <= 64 ? 2 : 1);
     p.ngroups = (p.kblocks + p.grp - 1) / p.grp;
-    if (M <= 128 && p.n_tiles <= kCounterTiles) {
+    if (M <= 128 && !wide && p.n_tiles <= kCounterTiles) {
         p.mode = 1;
         const int64_t U = (int64_t)p.n_tiles * p.ngroups;
         p.grid = (int)(U < kPlanSMs ? U : kPlanSMs);
@@ -312,9 +313,10 @@ cudaError_t launch_linear(DeviceInfo *di, const Plan &plan, const CUtensorMap &x
 }
 
 // the wide-tile kernel (256 activation rows per tile, whole tiles, one block per copy)
+template <int GS>
 cudaError_t launch_linear_wide(DeviceInfo *di, const Plan &plan, const CUtensorMap &xmap, const CUtensorMap &xhmap,
                                const CUtensorMap &cmap, const CUtensorMap &smap, const opqk::LinearArgs &n,
-                               cudaStream_t st) {
+                               const uint16_t *gmax, float alpha, cudaStream_t st) {
     using C = opqk_wide::Cfg<256>;
     if (plan.mode != 0) return cudaErrorInvalidValue;   // the wide kernel runs whole-tile schedules only
     opqk_wide::LinearArgs a{};
@@ -334,13 +336,18 @@ cudaError_t launch_linear_wide(DeviceInfo *di, const Plan &plan, const CUtensorM
     a.runs_max = n.runs_max;
     a.tail_split = n.tail_split;
     for (int i = 0; i < 16; ++i) a.lut[i] = n.lut[i];
-    if (!di->linear_attr[16]) {
-        cudaError_t e = cudaFuncSetAttribute(opqk_wide::wide_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    a.gmax = gmax;
+    a.ngk = GS > 0 ? n.K / GS : 0;
+    const double inv = 1.0 / (double)alpha;
+    for (int q = 0; q < 16; ++q) a.lutf[q] = (float)std::pow((double)q / 15.0, inv);
+    const int key = GS == 0 ? 16 : (GS == 32 ? 17 : GS == 64 ? 18 : GS == 128 ? 19 : 20);
+    if (!di->linear_attr[key]) {
+        cudaError_t e = cudaFuncSetAttribute(opqk_wide::wide_kernel<256, GS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              C::SMEM_BYTES);
         if (e != cudaSuccess) return e;
-        di->linear_attr[16] = true;
+        di->linear_attr[key] = true;
     }
-    opqk_wide::wide_kernel<256><<<plan.grid, C::THREADS, C::SMEM_BYTES, st>>>(xmap, xhmap, cmap, smap, a);
+    opqk_wide::wide_kernel<256, GS><<<plan.grid, C::THREADS, C::SMEM_BYTES, st>>>(xmap, xhmap, cmap, smap, a);
     return cudaGetLastError();
 }
 
@@ -505,16 +512,19 @@ opq_status opq_linear_plan(int64_t M, int64_t N, int64_t K, int *path, int *ctas
     return OPQ_OK;
 }
 
-opq_status opq_linear(const uint16_t *x, int64_t M, int64_t K, const uint32_t *codes, const uint32_t *signs,
-                      const float *scales, int64_t N, float alpha, uint16_t *y, void *workspace,
-                      size_t workspace_bytes, void *stream) {
+// the per-row format (scales, gs = 0) or the group-wise one (gmax, gs = 32 .. 256)
+static opq_status linear_impl(const uint16_t *x, int64_t M, int64_t K, const uint32_t *codes, const uint32_t *signs,
+                              const float *scales, const uint16_t *gmax, int64_t gs, int64_t N, float alpha,
+                              uint16_t *y, void *workspace, size_t workspace_bytes, void *stream) {
     if (M < 1) return OPQ_ERR_INVALID_ARG;
     opq_status s = check_sizes(N, K);
     if (s != OPQ_OK) return s;
+    if (gs > 0 && (s = check_group(K, gs)) != OPQ_OK) return s;
     if (M > INT32_MAX) return OPQ_ERR_UNSUPPORTED_SHAPE;
     if (!alpha_ok(alpha)) return OPQ_ERR_INVALID_ARG;
-    if ((s = check_ptrs({x, codes, signs, scales, y})) != OPQ_OK) return s;
-    const Plan plan = make_plan(M, N, K);
+    if ((s = check_ptrs({x, codes, signs, gs > 0 ? (const void *)gmax : (const void *)scales, y})) != OPQ_OK)
+        return s;
+    const Plan plan = make_plan(M, N, K, gs > 0);
     if (plan.ws_bytes > 0) {
         if (workspace == nullptr || workspace_bytes < plan.ws_bytes) return OPQ_ERR_WORKSPACE;
         if ((s = check_ptrs({workspace})) != OPQ_OK) return s;
@@ -576,11 +586,44 @@ opq_status opq_linear(const uint16_t *x, int64_t M, int64_t K, const uint32_t *c
         case 32: e = launch_linear<32>(di, plan, xmap, xhmap, cmap, smap, a, st); break;
         case 64: e = launch_linear<64>(di, plan, xmap, xhmap, cmap, smap, a, st); break;
         case 128: e = launch_linear<128>(di, plan, xmap, xhmap, cmap, smap, a, st); break;
-        default: e = launch_linear_wide(di, plan, xmap, xhmap, cmap, smap, a, st); break;
+        default:
+            switch (gs) {
+                case 0: e = launch_linear_wide<0>(di, plan, xmap, xhmap, cmap, smap, a, nullptr, alpha, st); break;
+                case 32: e = launch_linear_wide<32>(di, plan, xmap, xhmap, cmap, smap, a, gmax, alpha, st); break;
+                case 64: e = launch_linear_wide<64>(di, plan, xmap, xhmap, cmap, smap, a, gmax, alpha, st); break;
+                case 128: e = launch_linear_wide<128>(di, plan, xmap, xhmap, cmap, smap, a, gmax, alpha, st); break;
+                default: e = launch_linear_wide<256>(di, plan, xmap, xhmap, cmap, smap, a, gmax, alpha, st); break;
+            }
+            break;
     }
     if (e != cudaSuccess) return cuda_fail(e);
     e = cudaGetLastError();
     return e == cudaSuccess ? OPQ_OK : cuda_fail(e);
+}
+
+opq_status opq_linear(const uint16_t *x, int64_t M, int64_t K, const uint32_t *codes, const uint32_t *signs,
+                      const float *scales, int64_t N, float alpha, uint16_t *y, void *workspace,
+                      size_t workspace_bytes, void *stream) {
+    return linear_impl(x, M, K, codes, signs, scales, nullptr, 0, N, alpha, y, workspace, workspace_bytes, stream);
+}
+
+opq_status opq_linear_grouped(const uint16_t *x, int64_t M, int64_t K, const uint32_t *codes, const uint32_t *signs,
+                              const uint16_t *gmax, int64_t N, int64_t group_size, float alpha, uint16_t *y,
+                              void *workspace, size_t workspace_bytes, void *stream) {
+    if (group_size == 0) return OPQ_ERR_INVALID_ARG;
+    return linear_impl(x, M, K, codes, signs, nullptr, gmax, group_size, N, alpha, y, workspace, workspace_bytes,
+                       stream);
+}
+
+opq_status opq_linear_grouped_workspace_size(int64_t M, int64_t N, int64_t K, int64_t group_size, size_t *bytes) {
+    if (!bytes) return OPQ_ERR_INVALID_ARG;
+    if (M < 1) return OPQ_ERR_INVALID_ARG;
+    opq_status s = check_sizes(N, K);
+    if (s != OPQ_OK) return s;
+    if ((s = check_group(K, group_size)) != OPQ_OK) return s;
+    if (M > INT32_MAX) return OPQ_ERR_UNSUPPORTED_SHAPE;
+    *bytes = make_plan(M, N, K, true).ws_bytes;
+    return OPQ_OK;
 }
 
 opq_status opq_device_error(void *stream, uint32_t *err) {

@@ -18,6 +18,8 @@
 // (opq_linear.cuh) fetches several blocks per copy and splits K over CTAs instead; at this
 // width its wait structure measured ~6% slower, so the two regimes keep separate kernels.
 #pragma once
+#include <cuda_fp16.h>
+
 #include "opq_linear.cuh"
 
 namespace opqk_wide {
@@ -41,7 +43,23 @@ struct LinearArgs {
                             // (BX/2 activation rows) runs on two CTAs; 3 = each runs as two
                             // half-K runs on two CTAs whose partial sums meet in `ws`; 1 = whole
     uint16_t lut[16];       // bf16 (q/15)^(1/alpha)
+    // group-wise format (GS > 0)
+    const uint16_t *gmax;   // float16 [N, K / GS]
+    int ngk;                // groups per row (K / GS)
+    float lutf[16];         // (q/15)^(1/alpha) in fp32
 };
+
+// a group's 16 decoded magnitudes bf16(lutf[q] * gm) as byte planes (opq_bits.h DecodeTable)
+__device__ __forceinline__ void make_group_table(opqbits::DecodeTable &T, const float (&lutf)[16], float gm) {
+    uint32_t wd[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) wd[j] = pack_bf16x2_rn(lutf[2 * j] * gm, lutf[2 * j + 1] * gm);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        T.L[i] = __byte_perm(wd[2 * i], wd[2 * i + 1], 0x6420u);   // low bytes of entries 4i .. 4i + 3
+        T.H[i] = __byte_perm(wd[2 * i], wd[2 * i + 1], 0x7531u);   // their high bytes
+    }
+}
 
 // The sequence of runs of one CTA; every role walks the same sequence. A run is one
 // weight tile, a range of its 128-K blocks and a range of its activation rows.
@@ -180,7 +198,11 @@ struct Cfg {
     static_assert(A_BLOCKS >= X_STAGES, "ready ring shorter than the x ring");
 };
 
-template <int BX>
+// GS = 0: one fp32 scale per weight row, applied to the accumulated sums in the epilogue.
+// GS = 32 .. 256: one float16 max per GS weights of a row (the group-wise format); the
+// decoders form each group's 16 magnitudes bf16(LUT[q] * max) in registers and decode by
+// byte-plane lookups, and the epilogue applies no scale.
+template <int BX, int GS = 0>
 __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
     wide_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_xh,
                   const __grid_constant__ CUtensorMap tmap_codes, const __grid_constant__ CUtensorMap tmap_signs,
@@ -440,13 +462,19 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
         // 64-byte swizzle of the codes stage: 16-byte chunk c of row r sits at chunk c ^ ((r >> 1) & 3)
         const uint32_t sw64 = (uint32_t)((row >> 1) & 3);
         const uint32_t tm_row = tmem_base + ((uint32_t)(q * 32) << 16);
-        int nblocks = 0;
-        while (it.next(tile, r0, r1, j)) nblocks += r1 - r0;
-        bool ok = true;
-        for (int blk = g; blk < nblocks && ok; blk += C::GROUPS) {
+        // one 128-K block of this group: raw words in, A tile (both 64-K halves) out to TMEM;
+        // block r of a tile whose weight rows start at n_base (r, n_base used by the group-wise format)
+        auto run_block = [&](int blk, int r, int n_base) -> bool {
+            const int n_row = n_base + row;
+            auto gmax_at = [&](int gi) -> float {
+                return n_row < args.N ? __half2float(__ushort_as_half(__ldg(args.gmax + (size_t)n_row * args.ngk + gi)))
+                                      : 0.0f;
+            };
+            (void)gmax_at;
+            (void)r;
             const int rs = blk % C::RAW_STAGES;
             const uint32_t rph = (uint32_t)(blk / C::RAW_STAGES) & 1u;
-            if (!warp_wait(&raw_full[rs], rph)) { ok = false; break; }
+            if (!warp_wait(&raw_full[rs], rph)) return false;
             const uint8_t *rawc = smem + C::OFF_RAW + rs * C::RAW_BYTES + row * (C::KR / 2);
             const uint8_t *raws = smem + C::OFF_RAW + rs * C::RAW_BYTES + C::RAW_CODE_BYTES + row * (C::KR / 8);
 #pragma unroll
@@ -467,20 +495,34 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
                     if (lane == 0) mbar_arrive(&raw_empty[rs]);   // the block's raw words are in registers now
                 }
                 uint32_t o[2][16];
+                if constexpr (GS == 0) {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    uint32_t t4[4];
-                    opqbits::decode8_table(cw[i], sw[i >> 2], (uint32_t)(i & 3), lw, lw2, load, t4);
+                    for (int i = 0; i < 8; ++i) {
+                        uint32_t t4[4];
+                        opqbits::decode8_table(cw[i], sw[i >> 2], (uint32_t)(i & 3), lw, lw2, load, t4);
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) o[i >> 2][(i & 3) * 4 + e] = t4[e];
+                        for (int e = 0; e < 4; ++e) o[i >> 2][(i & 3) * 4 + e] = t4[e];
+                    }
+                } else {
+                    // the half's group (two groups of 32 weights when GS = 32)
+                    const int gi = (r * C::KR + h * C::KA) / GS;
+                    opqbits::DecodeTable Ta, Tb;
+                    make_group_table(Ta, args.lutf, gmax_at(gi));
+                    if constexpr (GS == 32) make_group_table(Tb, args.lutf, gmax_at(gi + 1));
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        uint32_t t4[4];
+                        opqbits::decode8(cw[i], (sw[i >> 2] >> (8 * (i & 3))) & 0xFFu,
+                                         (GS == 32 && i >= 4) ? Tb : Ta, t4);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) o[i >> 2][(i & 3) * 4 + e] = t4[e];
+                    }
                 }
                 // the block's A slot last held block blk - A_BLOCKS
                 const int prev = blk - C::A_BLOCKS;
                 if (h == 0 && prev >= 0 &&
-                    !warp_wait(&blk_done[prev % C::NDONE], (uint32_t)(prev / C::NDONE) & 1u)) {
-                    ok = false;
-                    break;
-                }
+                    !warp_wait(&blk_done[prev % C::NDONE], (uint32_t)(prev / C::NDONE) & 1u))
+                    return false;
                 tc_fence_after();
                 tmem_st_32x32b_x16(tm_row + as * 32, o[0]);
                 tmem_st_32x32b_x16(tm_row + as * 32 + 16, o[1]);
@@ -490,6 +532,20 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&ready[blk % C::A_BLOCKS]);
                 }
+            }
+            return true;
+        };
+        bool ok = true;
+        if constexpr (GS == 0) {
+            int nblocks = 0;
+            while (it.next(tile, r0, r1, j)) nblocks += r1 - r0;
+            for (int blk = g; blk < nblocks && ok; blk += C::GROUPS) ok = run_block(blk, 0, 0);
+        } else {
+            int blk = 0;
+            while (ok && it.next(tile, r0, r1, j)) {
+                const int n_base = (tile / args.m_tiles) * C::BW;
+                for (int r = r0; r < r1 && ok; ++r, ++blk)
+                    if (blk % C::GROUPS == g) ok = run_block(blk, r, n_base);
             }
         }
     } else {
@@ -534,7 +590,7 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
             const int n = n_blk * C::BW + row;
             const int n0 = n_blk * C::BW + q * 32;           // first row of this warp's quarter
             const bool full = (r0 == 0 && r1 == args.kblocks);
-            const float scale = n < args.N ? __ldg(args.scales + n) : 0.0f;
+            const float scale = GS > 0 ? 1.0f : (n < args.N ? __ldg(args.scales + n) : 0.0f);
             if (!warp_wait(&acc_full[ab], abph)) break;
             tc_fence_after();
             const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + C::A_COLS + ab * C::ACC_COLS;

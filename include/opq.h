@@ -112,6 +112,20 @@ opq_status opq_dequantize_grouped(const uint32_t *codes, const uint32_t *signs, 
                                   int64_t K, int64_t group_size, float alpha, uint16_t *w_out, void *stream);
 
 /*
+ * opq_linear_grouped — y = x W'^T with W' in the group-wise format: each decoded
+ * weight is bf16(sign * (q/15)^(1/alpha) * gmax) (the product formed in fp32 from
+ * fp32 magnitudes, then rounded to bf16) and enters the bf16 tensor-core product
+ * with fp32 accumulation; y is the sum rounded once to bf16. Arguments as for
+ * opq_linear, with gmax and group_size in place of scales. Every M runs on the
+ * 256-activation-row tile schedule; the workspace is sized by
+ * opq_linear_grouped_workspace_size and follows opq_linear's workspace rules.
+ */
+opq_status opq_linear_grouped(const uint16_t *x, int64_t M, int64_t K, const uint32_t *codes,
+                              const uint32_t *signs, const uint16_t *gmax, int64_t N, int64_t group_size,
+                              float alpha, uint16_t *y, void *workspace, size_t workspace_bytes, void *stream);
+opq_status opq_linear_grouped_workspace_size(int64_t M, int64_t N, int64_t K, int64_t group_size, size_t *bytes);
+
+/*
  * opq_linear_workspace_size — device scratch bytes opq_linear needs for an
  * M x K by (N x K)^T product (0 when the chosen kernel needs none).
  */

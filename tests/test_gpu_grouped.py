@@ -131,3 +131,77 @@ def test_grouped_argument_errors():
     assert lib.opq_dequantize_grouped(P(c), P(s), P(g), 4, 96, 128, 0.73, P(w), st) == 2
     torch.cuda.synchronize()
     no_device_error()
+
+
+# -------------------------------------------------------------------- linear --
+def grouped_linear_parity(x_cpu, w_cpu, gs, alpha, pairs=None, seed=0):
+    ref = oracle.quantize_grouped(w_cpu, gs, alpha)
+    M, K = x_cpu.shape
+    N = w_cpu.shape[0]
+    codes, signs = to_dev_u32(ref["codes"]), to_dev_u32(ref["signs"])
+    gmax = torch.from_numpy(ref["gmax"].view(np.float16)).to(DEV)
+    yb, y, pad = guarded((M, N), torch.bfloat16, 0x6B)
+    opq.linear_grouped(x_cpu.to(DEV), codes, signs, gmax, alpha, out=y)
+    torch.cuda.synchronize()
+    check_guards(yb, pad, 0x6B)
+    no_device_error()
+    yg = (u16(y).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    if pairs is None:
+        yref, bound = oracle.linear_grouped(x_cpu, ref["codes"], ref["signs"], ref["gmax"], alpha)
+        got = yg
+    else:
+        rng = np.random.default_rng(seed)
+        ms = np.concatenate([rng.integers(0, M, pairs), [0, M - 1, 0, M - 1]])
+        ns = np.concatenate([rng.integers(0, N, pairs), [0, N - 1, N - 1, 0]])
+        yref, bound = oracle.linear_grouped_pairs(x_cpu, ref["codes"], ref["signs"], ref["gmax"], alpha, ms, ns)
+        got = yg[ms, ns]
+    err = np.abs(got - yref)
+    tol = 1e-2 * bound + 1e-3
+    assert not (err > tol).any(), f"{int((err > tol).sum())} outputs out of tolerance"
+    assert np.isfinite(got).all()
+    return y
+
+
+@pytest.mark.parametrize("gs", GROUP_SIZES)
+@pytest.mark.parametrize("M,N,K", [(1, 300, 512), (17, 257, 1024), (129, 600, 768), (300, 130, 1280)])
+def test_linear_grouped_shapes(gs, M, N, K):
+    if K % gs:
+        pytest.skip("group size does not divide K")
+    lin = workloads.Linear("grouped-lin", M, N, K, w_seed=M + N + gs, x_seed=K + gs)
+    x, w = lin.make("cpu")
+    grouped_linear_parity(x, w, gs, 0.73)
+
+
+@pytest.mark.parametrize("alpha", [0.45, 1.0])
+def test_linear_grouped_alpha(alpha):
+    lin = workloads.Linear("grouped-alpha", 64, 384, 640, alpha=alpha, w_seed=5, x_seed=6)
+    x, w = lin.make("cpu")
+    grouped_linear_parity(x, w, 128, alpha)
+
+
+@pytest.mark.parametrize("M,N,K,gs", [(512, 10240, 1024, 128), (300, 9728, 256, 64), (512, 10240, 1152, 32)])
+def test_linear_grouped_tails(M, N, K, gs):
+    # past the last whole wave: half-K runs whose partial sums meet in the workspace (K >= 1024),
+    # or half-row runs (K = 256)
+    lin = workloads.Linear("grouped-tail", M, N, K, w_seed=N, x_seed=M)
+    x, w = lin.make("cpu")
+    grouped_linear_parity(x, w, gs, 0.73)
+
+
+def test_linear_grouped_full_size_sampled():
+    lin = workloads.dit_attn_proj()
+    x, w = lin.make("cpu")
+    grouped_linear_parity(x, w, 128, lin.alpha, pairs=3000, seed=1)
+
+
+def test_linear_grouped_deterministic_and_planes_from_gpu():
+    lin = workloads.Linear("grouped-det", 700, 3840, 1024, w_seed=1, x_seed=2)
+    x, w = lin.make(DEV)
+    planes = opq.quantize_grouped(w, 128, lin.alpha)
+    ws = torch.zeros(max(opq.grouped_workspace_size(700, 3840, 1024, 128), 16), dtype=torch.uint8, device=DEV)
+    y1 = opq.linear_grouped(x, *planes, lin.alpha, workspace=ws)
+    y2 = opq.linear_grouped(x, *planes, lin.alpha, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+    assert int(ws[:65536].count_nonzero()) == 0
+    no_device_error()
