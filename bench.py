@@ -276,6 +276,38 @@ def gpu_arm(args, rank, world, local_rank):
         del wqkv, pq
         assert opq.device_error() == 0
 
+    # ---- the group-wise format (the model card's own storage: one float16 max per GS weights)
+    # on the same weight and activations: quantize, linear, dequantize at GS = 128 and 32
+    grouped = {}
+    if not args.no_sweep:
+        wq_g = torch.empty_like(w)
+        y_g = torch.empty_like(y)
+        for gs in (128, 32):
+            cg, sg, gg = opq.quantize_grouped(w, gs, alpha)
+            ws_g = torch.zeros((max(opq.grouped_workspace_size(M, N, K, gs), 16),), dtype=torch.uint8, device=dev)
+            fq = lambda: opq.quantize_grouped(w, gs, alpha, out=(cg, sg, gg))
+            fl_ = lambda: opq.linear_grouped(x, cg, sg, gg, alpha, out=y_g, workspace=ws_g)
+            fd = lambda: opq.dequantize_grouped(cg, sg, gg, alpha, out=wq_g)
+            for f_ in (fq, fl_, fd):
+                for _ in range(3):
+                    f_()
+            tq_, _ = time_kernel(fq)
+            tl_, _ = time_kernel(fl_)
+            td_, _ = time_kernel(fd)
+            gq_bytes = N * K * 2 + N * K // 8 * 5 + 2 * N * (K // gs)
+            gd_bytes = N * K // 8 * 5 + 2 * N * (K // gs) + N * K * 2
+            g_tflops = flops / (tl_ * 1e-3) / 1e12
+            grouped[str(gs)] = {
+                "quantize": {"ms": tq_, "gbs": gq_bytes / (tq_ * 1e-3) / 1e9,
+                             "frac_hbm": gq_bytes / (tq_ * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+                "linear": {"ms": tl_, "tflops": g_tflops, "frac_bf16": g_tflops / peaks["bf16_tflops"]},
+                "dequantize": {"ms": td_, "gbs": gd_bytes / (td_ * 1e-3) / 1e9,
+                               "frac_hbm": gd_bytes / (td_ * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+            }
+            del ws_g
+        del wq_g, y_g
+        assert opq.device_error() == 0
+
     # ---- SNR context (the model card's "+7.2 dB" claim is on Z-Image weights; these are the
     # synthetic Student-t weights of the bench workload): OPQ through the library at alpha 0.73
     # and 1.0 (same 4-bit + sign + row max format), and per-row symmetric INT4 round(w/(max/7))
@@ -292,6 +324,9 @@ def gpu_arm(args, rank, world, local_rank):
     wf = w.float()
     step7 = wf.abs().amax(dim=1, keepdim=True).clamp_min(1e-30) / 7.0
     snr["int4_symmetric_row"] = snr_db(w, (torch.round(wf / step7).clamp(-7, 7) * step7).to(torch.bfloat16))
+    p_ = opq.quantize_grouped(w, 128, alpha)
+    opq.dequantize_grouped(*p_, alpha, out=w_rec)
+    snr[f"opq_alpha_{alpha:g}_group128"] = snr_db(w, w_rec)
     snr["gain_vs_int4_db"] = snr[f"opq_alpha_{alpha:g}"] - snr["int4_symmetric_row"]
     snr["gain_vs_alpha1_db"] = snr[f"opq_alpha_{alpha:g}"] - snr["opq_alpha_1"]
     snr["model_card_claim_db"] = 7.2
@@ -337,7 +372,7 @@ def gpu_arm(args, rank, world, local_rank):
         "config": {"workload": lin.name, "M": M, "N": N, "K": K, "alpha": alpha,
                    "step": "quantize W + linear x W'^T + dequantize W'", "parallelism": f"replicas{world}",
                    "l2": "flushed between timed steps (4x L2 buffer write outside the event pairs)"},
-        "kernels": kernels, "small_m": small, "roofline": roof, "snr_db": snr,
+        "kernels": kernels, "small_m": small, "grouped": grouped, "roofline": roof, "snr_db": snr,
         "e2e": {"value": whole_job_tflops(world, flops, ms_e2e), "unit": "TFLOP/s", "ms_per_step": ms_e2e,
                 "h2d_bytes_per_step": w.numel() * 2 + x.numel() * 2, "d2h_bytes_per_step": y.numel() * 2},
         "gpu_launches": launches_per_step * args.steps,
