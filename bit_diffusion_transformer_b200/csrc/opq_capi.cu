@@ -66,7 +66,9 @@ uint16_t host_bf16(double v) {
 
 struct DeviceInfo {
     int sms = 0;
-    bool linear_attr[21] = {false};   // narrow BX / 16, 16 = wide, 17 .. 20 = wide group-wise (GS 32 .. 256)
+    // dynamic shared memory raised, per [group size index: 0 per-row, 1..4 GS 32..256][kernel: BX 16, 32,
+    // 64, 128, wide]
+    bool linear_attr[5][5] = {};
 };
 std::mutex g_mu;
 DeviceInfo g_dev[64];
@@ -296,19 +298,21 @@ void dispatch_quant(int vpl, const uint16_t *w, int64_t N, int64_t K, int64_t ld
     }
 }
 
-template <int BX>
+constexpr int gs_index(int gs) { return gs == 0 ? 0 : gs == 32 ? 1 : gs == 64 ? 2 : gs == 128 ? 3 : 4; }
+
+template <int BX, int GS>
 cudaError_t launch_linear(DeviceInfo *di, const Plan &plan, const CUtensorMap &xmap, const CUtensorMap &xhmap,
                           const CUtensorMap &cmap, const CUtensorMap &smap, const opqk::LinearArgs &a,
                           cudaStream_t st) {
     using C = opqk::Cfg<BX>;
-    const int key = BX / 16;
-    if (!di->linear_attr[key]) {
-        cudaError_t e = cudaFuncSetAttribute(opqk::linear_kernel<BX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    const int key = BX == 16 ? 0 : BX == 32 ? 1 : BX == 64 ? 2 : 3;
+    if (!di->linear_attr[gs_index(GS)][key]) {
+        cudaError_t e = cudaFuncSetAttribute(opqk::linear_kernel<BX, GS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              C::SMEM_BYTES);
         if (e != cudaSuccess) return e;
-        di->linear_attr[key] = true;
+        di->linear_attr[gs_index(GS)][key] = true;
     }
-    opqk::linear_kernel<BX><<<plan.grid, C::THREADS, C::SMEM_BYTES, st>>>(xmap, xhmap, cmap, smap, a);
+    opqk::linear_kernel<BX, GS><<<plan.grid, C::THREADS, C::SMEM_BYTES, st>>>(xmap, xhmap, cmap, smap, a);
     return cudaGetLastError();
 }
 
@@ -316,7 +320,7 @@ cudaError_t launch_linear(DeviceInfo *di, const Plan &plan, const CUtensorMap &x
 template <int GS>
 cudaError_t launch_linear_wide(DeviceInfo *di, const Plan &plan, const CUtensorMap &xmap, const CUtensorMap &xhmap,
                                const CUtensorMap &cmap, const CUtensorMap &smap, const opqk::LinearArgs &n,
-                               const uint16_t *gmax, float alpha, cudaStream_t st) {
+                               cudaStream_t st) {
     using C = opqk_wide::Cfg<256>;
     if (plan.mode != 0) return cudaErrorInvalidValue;   // the wide kernel runs whole-tile schedules only
     opqk_wide::LinearArgs a{};
@@ -336,16 +340,14 @@ cudaError_t launch_linear_wide(DeviceInfo *di, const Plan &plan, const CUtensorM
     a.runs_max = n.runs_max;
     a.tail_split = n.tail_split;
     for (int i = 0; i < 16; ++i) a.lut[i] = n.lut[i];
-    a.gmax = gmax;
-    a.ngk = GS > 0 ? n.K / GS : 0;
-    const double inv = 1.0 / (double)alpha;
-    for (int q = 0; q < 16; ++q) a.lutf[q] = (float)std::pow((double)q / 15.0, inv);
-    const int key = GS == 0 ? 16 : (GS == 32 ? 17 : GS == 64 ? 18 : GS == 128 ? 19 : 20);
-    if (!di->linear_attr[key]) {
+    a.gmax = n.gmax;
+    a.ngk = n.ngk;
+    for (int q = 0; q < 16; ++q) a.lutf[q] = n.lutf[q];
+    if (!di->linear_attr[gs_index(GS)][4]) {
         cudaError_t e = cudaFuncSetAttribute(opqk_wide::wide_kernel<256, GS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              C::SMEM_BYTES);
         if (e != cudaSuccess) return e;
-        di->linear_attr[key] = true;
+        di->linear_attr[gs_index(GS)][4] = true;
     }
     opqk_wide::wide_kernel<256, GS><<<plan.grid, C::THREADS, C::SMEM_BYTES, st>>>(xmap, xhmap, cmap, smap, a);
     return cudaGetLastError();
@@ -512,6 +514,22 @@ opq_status opq_linear_plan(int64_t M, int64_t N, int64_t K, int *path, int *ctas
     return OPQ_OK;
 }
 
+// the kernel the plan picked, for group size GS (0 = per-row scales)
+extern "C++" {
+template <int GS>
+static cudaError_t launch_any(DeviceInfo *di, const Plan &plan, const CUtensorMap &xmap, const CUtensorMap &xhmap,
+                              const CUtensorMap &cmap, const CUtensorMap &smap, const opqk::LinearArgs &a,
+                              cudaStream_t st) {
+    switch (plan.bx) {
+        case 16: return launch_linear<16, GS>(di, plan, xmap, xhmap, cmap, smap, a, st);
+        case 32: return launch_linear<32, GS>(di, plan, xmap, xhmap, cmap, smap, a, st);
+        case 64: return launch_linear<64, GS>(di, plan, xmap, xhmap, cmap, smap, a, st);
+        case 128: return launch_linear<128, GS>(di, plan, xmap, xhmap, cmap, smap, a, st);
+        default: return launch_linear_wide<GS>(di, plan, xmap, xhmap, cmap, smap, a, st);
+    }
+}
+}  // extern "C++"
+
 // the per-row format (scales, gs = 0) or the group-wise one (gmax, gs = 32 .. 256)
 static opq_status linear_impl(const uint16_t *x, int64_t M, int64_t K, const uint32_t *codes, const uint32_t *signs,
                               const float *scales, const uint16_t *gmax, int64_t gs, int64_t N, float alpha,
@@ -524,7 +542,7 @@ static opq_status linear_impl(const uint16_t *x, int64_t M, int64_t K, const uin
     if (!alpha_ok(alpha)) return OPQ_ERR_INVALID_ARG;
     if ((s = check_ptrs({x, codes, signs, gs > 0 ? (const void *)gmax : (const void *)scales, y})) != OPQ_OK)
         return s;
-    const Plan plan = make_plan(M, N, K, gs > 0);
+    const Plan plan = make_plan(M, N, K);
     if (plan.ws_bytes > 0) {
         if (workspace == nullptr || workspace_bytes < plan.ws_bytes) return OPQ_ERR_WORKSPACE;
         if ((s = check_ptrs({workspace})) != OPQ_OK) return s;
@@ -551,6 +569,12 @@ static opq_status linear_impl(const uint16_t *x, int64_t M, int64_t K, const uin
     a.runs_max = plan.runs_max;
     a.tail_split = plan.mode == 0 ? plan.tail_split : 1;
     lut_bf16(alpha, a.lut);
+    a.gmax = gmax;
+    a.ngk = gs > 0 ? (int)(K / gs) : 0;
+    {
+        const double inv = 1.0 / (double)alpha;
+        for (int q = 0; q < 16; ++q) a.lutf[q] = (float)std::pow((double)q / 15.0, inv);
+    }
 
     CUtensorMap xmap, xhmap, cmap, smap;
     // the sign plane's rows are 16-byte aligned (a TMA requirement) when K % 128 == 0; otherwise the
@@ -581,20 +605,12 @@ static opq_status linear_impl(const uint16_t *x, int64_t M, int64_t K, const uin
         xhmap = xmap;   // not read by the kernel
     }
     cudaError_t e;
-    switch (plan.bx) {
-        case 16: e = launch_linear<16>(di, plan, xmap, xhmap, cmap, smap, a, st); break;
-        case 32: e = launch_linear<32>(di, plan, xmap, xhmap, cmap, smap, a, st); break;
-        case 64: e = launch_linear<64>(di, plan, xmap, xhmap, cmap, smap, a, st); break;
-        case 128: e = launch_linear<128>(di, plan, xmap, xhmap, cmap, smap, a, st); break;
-        default:
-            switch (gs) {
-                case 0: e = launch_linear_wide<0>(di, plan, xmap, xhmap, cmap, smap, a, nullptr, alpha, st); break;
-                case 32: e = launch_linear_wide<32>(di, plan, xmap, xhmap, cmap, smap, a, gmax, alpha, st); break;
-                case 64: e = launch_linear_wide<64>(di, plan, xmap, xhmap, cmap, smap, a, gmax, alpha, st); break;
-                case 128: e = launch_linear_wide<128>(di, plan, xmap, xhmap, cmap, smap, a, gmax, alpha, st); break;
-                default: e = launch_linear_wide<256>(di, plan, xmap, xhmap, cmap, smap, a, gmax, alpha, st); break;
-            }
-            break;
+    switch (gs) {
+        case 0: e = launch_any<0>(di, plan, xmap, xhmap, cmap, smap, a, st); break;
+        case 32: e = launch_any<32>(di, plan, xmap, xhmap, cmap, smap, a, st); break;
+        case 64: e = launch_any<64>(di, plan, xmap, xhmap, cmap, smap, a, st); break;
+        case 128: e = launch_any<128>(di, plan, xmap, xhmap, cmap, smap, a, st); break;
+        default: e = launch_any<256>(di, plan, xmap, xhmap, cmap, smap, a, st); break;
     }
     if (e != cudaSuccess) return cuda_fail(e);
     e = cudaGetLastError();
@@ -622,7 +638,7 @@ opq_status opq_linear_grouped_workspace_size(int64_t M, int64_t N, int64_t K, in
     if (s != OPQ_OK) return s;
     if ((s = check_group(K, group_size)) != OPQ_OK) return s;
     if (M > INT32_MAX) return OPQ_ERR_UNSUPPORTED_SHAPE;
-    *bytes = make_plan(M, N, K, true).ws_bytes;
+    *bytes = make_plan(M, N, K).ws_bytes;
     return OPQ_OK;
 }
 

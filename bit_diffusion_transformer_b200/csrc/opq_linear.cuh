@@ -32,6 +32,7 @@
 // Mode 0 (whole tiles strided over CTAs) serves shapes with more tiles than counters.
 // Wide tiles (M > 128) use opq_linear_wide.cuh.
 #pragma once
+#include <cuda_fp16.h>
 #include <cuda_bf16.h>
 
 #include "opq_bits.h"
@@ -136,7 +137,23 @@ struct LinearArgs {
     int tail_split;         // mode 0: 2 = tiles past the last full wave run as two half-width
                             // (BX/2 activation rows) runs on different CTAs; 1 = whole tiles
     uint16_t lut[16];       // bf16 (q/15)^(1/alpha)
+    // group-wise format (GS > 0)
+    const uint16_t *gmax;   // float16 [N, K / GS]
+    int ngk;                // groups per row (K / GS)
+    float lutf[16];         // (q/15)^(1/alpha) in fp32
 };
+
+// a group's 16 decoded magnitudes bf16(lutf[q] * gm) as byte planes (opq_bits.h DecodeTable)
+__device__ __forceinline__ void make_group_table(opqbits::DecodeTable &T, const float (&lutf)[16], float gm) {
+    uint32_t wd[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) wd[j] = pack_bf16x2_rn(lutf[2 * j] * gm, lutf[2 * j + 1] * gm);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        T.L[i] = __byte_perm(wd[2 * i], wd[2 * i + 1], 0x6420u);   // low bytes of entries 4i .. 4i + 3
+        T.H[i] = __byte_perm(wd[2 * i], wd[2 * i + 1], 0x7531u);   // their high bytes
+    }
+}
 
 // Units (tile, 128-K block) of CTA c out of C in stream-K mode: [begin(c), begin(c + 1)).
 __host__ __device__ __forceinline__ int64_t unit_begin(int64_t c, int64_t C, int64_t U) { return (c * U) / C; }
@@ -291,7 +308,9 @@ struct Cfg {
     static_assert(A_STAGES % 2 == 0, "a block is two A half-stages");
 };
 
-template <int BX>
+// GS = 0: one fp32 scale per weight row, applied in the epilogue; GS = 32 .. 256: one float16
+// max per GS weights of a row (the group-wise format), applied in the decode, no epilogue scale
+template <int BX, int GS = 0>
 __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
     linear_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_xh,
                   const __grid_constant__ CUtensorMap tmap_codes, const __grid_constant__ CUtensorMap tmap_signs,
@@ -579,13 +598,36 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
                         const int sidx = blk * 2 + h;
                         const int as = sidx % C::A_STAGES;
                         uint32_t o[2][16];
+                        if constexpr (GS == 0) {
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const int w = 8 * h + i;
-                            uint32_t t4[4];
-                            opqbits::decode8_table(cw[w], sw[w >> 2], (uint32_t)(w & 3), lw, lw2, load, t4);
+                            for (int i = 0; i < 8; ++i) {
+                                const int w = 8 * h + i;
+                                uint32_t t4[4];
+                                opqbits::decode8_table(cw[w], sw[w >> 2], (uint32_t)(w & 3), lw, lw2, load, t4);
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) o[i >> 2][(i & 3) * 4 + e] = t4[e];
+                                for (int e = 0; e < 4; ++e) o[i >> 2][(i & 3) * 4 + e] = t4[e];
+                            }
+                        } else {
+                            // the half's group (two groups of 32 weights when GS = 32), of weight row n
+                            const int n = (R.tile / args.m_tiles) * C::BW + row;
+                            const int gi = ((lg.start(g) + jj) * C::KR + h * C::KA) / GS;
+                            auto gmax_at = [&](int gx) -> float {
+                                return n < args.N
+                                           ? __half2float(__ushort_as_half(__ldg(args.gmax + (size_t)n * args.ngk + gx)))
+                                           : 0.0f;
+                            };
+                            opqbits::DecodeTable Ta, Tb;
+                            make_group_table(Ta, args.lutf, gmax_at(gi));
+                            if constexpr (GS == 32) make_group_table(Tb, args.lutf, gmax_at(gi + 1));
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                const int w = 8 * h + i;
+                                uint32_t t4[4];
+                                opqbits::decode8(cw[w], (sw[w >> 2] >> (8 * (w & 3))) & 0xFFu,
+                                                 (GS == 32 && i >= 4) ? Tb : Ta, t4);
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) o[i >> 2][(i & 3) * 4 + e] = t4[e];
+                            }
                         }
                         // the block's A slot last held block blk - A_BLOCKS
                         const int prev = blk - C::A_BLOCKS;
@@ -626,7 +668,7 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
             const int n = n_blk * C::BW + row;
             const int n0 = n_blk * C::BW + q * 32;           // first row of this warp's quarter
             const bool full = (r0 == 0 && r1 == args.kblocks);
-            const float scale = n < args.N ? __ldg(args.scales + n) : 0.0f;
+            const float scale = GS > 0 ? 1.0f : (n < args.N ? __ldg(args.scales + n) : 0.0f);
             if (!warp_wait(&acc_full[ab], abph)) break;
             tc_fence_after();
             const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + C::A_COLS + ab * C::ACC_COLS;

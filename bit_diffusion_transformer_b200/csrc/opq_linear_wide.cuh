@@ -49,17 +49,6 @@ struct LinearArgs {
     float lutf[16];         // (q/15)^(1/alpha) in fp32
 };
 
-// a group's 16 decoded magnitudes bf16(lutf[q] * gm) as byte planes (opq_bits.h DecodeTable)
-__device__ __forceinline__ void make_group_table(opqbits::DecodeTable &T, const float (&lutf)[16], float gm) {
-    uint32_t wd[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) wd[j] = pack_bf16x2_rn(lutf[2 * j] * gm, lutf[2 * j + 1] * gm);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        T.L[i] = __byte_perm(wd[2 * i], wd[2 * i + 1], 0x6420u);   // low bytes of entries 4i .. 4i + 3
-        T.H[i] = __byte_perm(wd[2 * i], wd[2 * i + 1], 0x7531u);   // their high bytes
-    }
-}
 
 // The sequence of runs of one CTA; every role walks the same sequence. A run is one
 // weight tile, a range of its 128-K blocks and a range of its activation rows.

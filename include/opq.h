@@ -116,8 +116,8 @@ opq_status opq_dequantize_grouped(const uint32_t *codes, const uint32_t *signs, 
  * weight is bf16(sign * (q/15)^(1/alpha) * gmax) (the product formed in fp32 from
  * fp32 magnitudes, then rounded to bf16) and enters the bf16 tensor-core product
  * with fp32 accumulation; y is the sum rounded once to bf16. Arguments as for
- * opq_linear, with gmax and group_size in place of scales. Every M runs on the
- * 256-activation-row tile schedule; the workspace is sized by
+ * opq_linear, with gmax and group_size in place of scales, and the same
+ * schedule as opq_linear for the shape; the workspace is sized by
  * opq_linear_grouped_workspace_size and follows opq_linear's workspace rules.
  */
 opq_status opq_linear_grouped(const uint16_t *x, int64_t M, int64_t K, const uint32_t *codes,
