@@ -29,7 +29,9 @@ _STATUS = {0: "OPQ_OK", 1: "OPQ_ERR_INVALID_ARG", 2: "OPQ_ERR_UNSUPPORTED_SHAPE"
 EXPORTS = ["opq_quantize", "opq_dequantize", "opq_linear_workspace_size", "opq_linear", "opq_linear_plan",
            "opq_linear_noalloc", "opq_device_error", "opq_status_string", "opq_last_cuda_error",
            "opq_abi_version", "opq_quantize_grouped", "opq_dequantize_grouped",
-           "opq_linear_grouped", "opq_linear_grouped_workspace_size"]
+           "opq_linear_grouped", "opq_linear_grouped_workspace_size", "opq_linear_fused",
+           "opq_linear_grouped_fused"]
+ACTIVATIONS = {"none": 0, "silu": 1, "gelu_tanh": 2}
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 
@@ -64,11 +66,13 @@ def load(path: str = LIB_PATH):
     lib.opq_dequantize_grouped.argtypes = [P, P, P, I, I, I, F, P, P]
     lib.opq_linear_grouped.argtypes = [P, I, I, P, P, P, I, I, F, P, P, S, P]
     lib.opq_linear_grouped_workspace_size.argtypes = [I, I, I, I, ctypes.POINTER(S)]
+    lib.opq_linear_fused.argtypes = [P, I, I, P, P, P, I, F, P, ctypes.c_int, P, P, S, P]
+    lib.opq_linear_grouped_fused.argtypes = [P, I, I, P, P, P, I, I, F, P, ctypes.c_int, P, P, S, P]
     lib.opq_status_string.argtypes = [ctypes.c_int]
     lib.opq_status_string.restype = ctypes.c_char_p
     for f in ("opq_quantize", "opq_dequantize", "opq_linear_workspace_size", "opq_linear", "opq_linear_plan",
               "opq_linear_noalloc", "opq_device_error", "opq_quantize_grouped", "opq_dequantize_grouped", "opq_linear_grouped",
-              "opq_linear_grouped_workspace_size"):
+              "opq_linear_grouped_workspace_size", "opq_linear_fused", "opq_linear_grouped_fused"):
         getattr(lib, f).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -174,6 +178,54 @@ def linear_grouped(x: torch.Tensor, codes: torch.Tensor, signs: torch.Tensor, gm
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check(load().opq_linear_grouped(_ptr(x), M, K, _ptr(codes), _ptr(signs), _ptr(gmax), N, gs, float(alpha),
                                      _ptr(y), ws_ptr, ws_bytes, _stream(x.device)), "opq_linear_grouped")
+    return y
+
+
+def _workspace(need: int, workspace, device):
+    if need and workspace is None:
+        workspace = torch.zeros((need,), dtype=torch.uint8, device=device)   # must start zeroed
+    ptr = _ptr(workspace) if workspace is not None else ctypes.c_void_p(0)
+    nbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    return workspace, ptr, nbytes
+
+
+def linear_fused(x: torch.Tensor, codes: torch.Tensor, signs: torch.Tensor, scales: torch.Tensor,
+                 alpha: float = ALPHA, bias: torch.Tensor | None = None, act: str = "none", out=None,
+                 workspace=None):
+    """y = act(x @ W'^T + bias) (the nn.Linear a OPQLinear replaces, with the activation that follows)."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2
+    _need_cuda(x, codes, signs, scales)
+    if bias is not None:
+        assert bias.dtype == torch.bfloat16
+        _need_cuda(bias)
+    M, K = x.shape
+    N = codes.shape[0]
+    y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    workspace, ws_ptr, ws_bytes = _workspace(workspace_size(M, N, K), workspace, x.device)
+    _check(load().opq_linear_fused(_ptr(x), M, K, _ptr(codes), _ptr(signs), _ptr(scales), N, float(alpha),
+                                   _ptr(bias) if bias is not None else ctypes.c_void_p(0), ACTIVATIONS[act],
+                                   _ptr(y), ws_ptr, ws_bytes, _stream(x.device)), "opq_linear_fused")
+    return y
+
+
+def linear_grouped_fused(x: torch.Tensor, codes: torch.Tensor, signs: torch.Tensor, gmax: torch.Tensor,
+                         alpha: float = ALPHA, bias: torch.Tensor | None = None, act: str = "none", out=None,
+                         workspace=None):
+    """y = act(x @ W'^T + bias) for a group-wise packed W."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2
+    _need_cuda(x, codes, signs, gmax)
+    if bias is not None:
+        assert bias.dtype == torch.bfloat16
+        _need_cuda(bias)
+    M, K = x.shape
+    N = codes.shape[0]
+    gs = K // gmax.shape[1]
+    y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    workspace, ws_ptr, ws_bytes = _workspace(grouped_workspace_size(M, N, K, gs), workspace, x.device)
+    _check(load().opq_linear_grouped_fused(_ptr(x), M, K, _ptr(codes), _ptr(signs), _ptr(gmax), N, gs,
+                                           float(alpha), _ptr(bias) if bias is not None else ctypes.c_void_p(0),
+                                           ACTIVATIONS[act], _ptr(y), ws_ptr, ws_bytes, _stream(x.device)),
+           "opq_linear_grouped_fused")
     return y
 
 

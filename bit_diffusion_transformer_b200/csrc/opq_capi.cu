@@ -342,6 +342,8 @@ cudaError_t launch_linear_wide(DeviceInfo *di, const Plan &plan, const CUtensorM
     for (int i = 0; i < 16; ++i) a.lut[i] = n.lut[i];
     a.gmax = n.gmax;
     a.ngk = n.ngk;
+    a.bias = n.bias;
+    a.act = n.act;
     for (int q = 0; q < 16; ++q) a.lutf[q] = n.lutf[q];
     if (!di->linear_attr[gs_index(GS)][4]) {
         cudaError_t e = cudaFuncSetAttribute(opqk_wide::wide_kernel<256, GS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -533,7 +535,8 @@ static cudaError_t launch_any(DeviceInfo *di, const Plan &plan, const CUtensorMa
 // the per-row format (scales, gs = 0) or the group-wise one (gmax, gs = 32 .. 256)
 static opq_status linear_impl(const uint16_t *x, int64_t M, int64_t K, const uint32_t *codes, const uint32_t *signs,
                               const float *scales, const uint16_t *gmax, int64_t gs, int64_t N, float alpha,
-                              uint16_t *y, void *workspace, size_t workspace_bytes, void *stream) {
+                              const uint16_t *bias, int activation, uint16_t *y, void *workspace,
+                              size_t workspace_bytes, void *stream) {
     if (M < 1) return OPQ_ERR_INVALID_ARG;
     opq_status s = check_sizes(N, K);
     if (s != OPQ_OK) return s;
@@ -542,6 +545,9 @@ static opq_status linear_impl(const uint16_t *x, int64_t M, int64_t K, const uin
     if (!alpha_ok(alpha)) return OPQ_ERR_INVALID_ARG;
     if ((s = check_ptrs({x, codes, signs, gs > 0 ? (const void *)gmax : (const void *)scales, y})) != OPQ_OK)
         return s;
+    if (activation != OPQ_ACT_NONE && activation != OPQ_ACT_SILU && activation != OPQ_ACT_GELU_TANH)
+        return OPQ_ERR_INVALID_ARG;
+    if (bias && (s = check_ptrs({bias})) != OPQ_OK) return s;
     const Plan plan = make_plan(M, N, K);
     if (plan.ws_bytes > 0) {
         if (workspace == nullptr || workspace_bytes < plan.ws_bytes) return OPQ_ERR_WORKSPACE;
@@ -571,6 +577,8 @@ static opq_status linear_impl(const uint16_t *x, int64_t M, int64_t K, const uin
     lut_bf16(alpha, a.lut);
     a.gmax = gmax;
     a.ngk = gs > 0 ? (int)(K / gs) : 0;
+    a.bias = bias;
+    a.act = activation;
     {
         const double inv = 1.0 / (double)alpha;
         for (int q = 0; q < 16; ++q) a.lutf[q] = (float)std::pow((double)q / 15.0, inv);
@@ -620,15 +628,32 @@ static opq_status linear_impl(const uint16_t *x, int64_t M, int64_t K, const uin
 opq_status opq_linear(const uint16_t *x, int64_t M, int64_t K, const uint32_t *codes, const uint32_t *signs,
                       const float *scales, int64_t N, float alpha, uint16_t *y, void *workspace,
                       size_t workspace_bytes, void *stream) {
-    return linear_impl(x, M, K, codes, signs, scales, nullptr, 0, N, alpha, y, workspace, workspace_bytes, stream);
+    return linear_impl(x, M, K, codes, signs, scales, nullptr, 0, N, alpha, nullptr, OPQ_ACT_NONE, y, workspace,
+                       workspace_bytes, stream);
+}
+
+opq_status opq_linear_fused(const uint16_t *x, int64_t M, int64_t K, const uint32_t *codes, const uint32_t *signs,
+                            const float *scales, int64_t N, float alpha, const uint16_t *bias, int activation,
+                            uint16_t *y, void *workspace, size_t workspace_bytes, void *stream) {
+    return linear_impl(x, M, K, codes, signs, scales, nullptr, 0, N, alpha, bias, activation, y, workspace,
+                       workspace_bytes, stream);
 }
 
 opq_status opq_linear_grouped(const uint16_t *x, int64_t M, int64_t K, const uint32_t *codes, const uint32_t *signs,
                               const uint16_t *gmax, int64_t N, int64_t group_size, float alpha, uint16_t *y,
                               void *workspace, size_t workspace_bytes, void *stream) {
     if (group_size == 0) return OPQ_ERR_INVALID_ARG;
-    return linear_impl(x, M, K, codes, signs, nullptr, gmax, group_size, N, alpha, y, workspace, workspace_bytes,
-                       stream);
+    return linear_impl(x, M, K, codes, signs, nullptr, gmax, group_size, N, alpha, nullptr, OPQ_ACT_NONE, y,
+                       workspace, workspace_bytes, stream);
+}
+
+opq_status opq_linear_grouped_fused(const uint16_t *x, int64_t M, int64_t K, const uint32_t *codes,
+                                    const uint32_t *signs, const uint16_t *gmax, int64_t N, int64_t group_size,
+                                    float alpha, const uint16_t *bias, int activation, uint16_t *y, void *workspace,
+                                    size_t workspace_bytes, void *stream) {
+    if (group_size == 0) return OPQ_ERR_INVALID_ARG;
+    return linear_impl(x, M, K, codes, signs, nullptr, gmax, group_size, N, alpha, bias, activation, y, workspace,
+                       workspace_bytes, stream);
 }
 
 opq_status opq_linear_grouped_workspace_size(int64_t M, int64_t N, int64_t K, int64_t group_size, size_t *bytes) {

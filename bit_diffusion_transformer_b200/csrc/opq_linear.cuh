@@ -141,7 +141,30 @@ struct LinearArgs {
     const uint16_t *gmax;   // float16 [N, K / GS]
     int ngk;                // groups per row (K / GS)
     float lutf[16];         // (q/15)^(1/alpha) in fp32
+    // fused epilogue
+    const uint16_t *bias;   // bf16 [N] added to every output row, or null
+    int act;                // EPI_NONE, EPI_SILU, EPI_GELU_TANH
 };
+
+enum { EPI_NONE = 0, EPI_SILU = 1, EPI_GELU_TANH = 2 };
+
+// One output before its bf16 rounding: the fp32 sum times the row scale, plus the bias, through
+// the activation (SiLU v / (1 + e^-v); GELU's tanh form 0.5 v (1 + tanh(sqrt(2/pi) (v + 0.044715
+// v^3)))). With no bias and no activation this is the plain product acc * scale.
+__device__ __forceinline__ float epi_value(float acc, float scale, float bias, int act) {
+    float v = acc * scale;
+    if (bias != 0.0f) v += bias;
+    if (act == EPI_SILU) {
+        v = v / (1.0f + expf(-v));
+    } else if (act == EPI_GELU_TANH) {
+        v = 0.5f * v * (1.0f + tanhf(0.7978845608028654f * (v + 0.044715f * v * v * v)));
+    }
+    return v;
+}
+
+__device__ __forceinline__ float bias_at(const uint16_t *bias, int n, int N) {
+    return (bias != nullptr && n < N) ? __uint_as_float((uint32_t)__ldg(bias + n) << 16) : 0.0f;
+}
 
 // a group's 16 decoded magnitudes bf16(lutf[q] * gm) as byte planes (opq_bits.h DecodeTable)
 __device__ __forceinline__ void make_group_table(opqbits::DecodeTable &T, const float (&lutf)[16], float gm) {
@@ -669,6 +692,12 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
             const int n0 = n_blk * C::BW + q * 32;           // first row of this warp's quarter
             const bool full = (r0 == 0 && r1 == args.kblocks);
             const float scale = GS > 0 ? 1.0f : (n < args.N ? __ldg(args.scales + n) : 0.0f);
+            const float bias = bias_at(args.bias, n, args.N);
+            // the plain product, or the fused epilogue (bias, activation): chosen per tile, so the
+            // plain path carries none of the fused code
+            const bool plain = args.bias == nullptr && args.act == EPI_NONE;
+            auto fv_plain = [scale](float a) { return a * scale; };
+            auto fv_fused = [scale, bias, &args](float a) { return epi_value(a, scale, bias, args.act); };
             if (!warp_wait(&acc_full[ab], abph)) break;
             tc_fence_after();
             const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + C::A_COLS + ab * C::ACC_COLS;
@@ -690,36 +719,40 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
                 }
                 tmem_ld_wait();
                 if (full) {
-                    const int m0 = m_blk * BX + xoff + c0;
-                    if (vec_y && n0 + 32 <= args.N) {
-                        // stage [16 m][32 n] bf16, then each lane stores 32 contiguous bytes of one m row
-                        const uint32_t sbuf = stage0 + (uint32_t)sb * 1024u;
+                    auto store_full = [&](auto &&fv) {
+                        const int m0 = m_blk * BX + xoff + c0;
+                        if (vec_y && n0 + 32 <= args.N) {
+                            // stage [16 m][32 n] bf16, then each lane stores 32 contiguous bytes of one m row
+                            const uint32_t sbuf = stage0 + (uint32_t)sb * 1024u;
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const __nv_bfloat16 o = __float2bfloat16_rn(__uint_as_float(v[i]) * scale);
-                            asm volatile("st.shared.u16 [%0], %1;" ::"r"(sbuf + (uint32_t)i * 64u + (uint32_t)lane * 2u),
-                                         "h"(*reinterpret_cast<const unsigned short *>(&o)) : "memory");
-                        }
-                        __syncwarp();
-                        const int mi = lane >> 1, hf = lane & 1;
-                        if (m0 + mi < args.M) {
-                            const uint4 w0 = lds_v4(sbuf + (uint32_t)mi * 64u + (uint32_t)hf * 32u);
-                            const uint4 w1 = lds_v4(sbuf + (uint32_t)mi * 64u + (uint32_t)hf * 32u + 16u);
-                            uint4 *dst = reinterpret_cast<uint4 *>(args.y + (size_t)(m0 + mi) * args.N + n0 + hf * 16);
-                            dst[0] = w0;
-                            dst[1] = w1;
-                        }
-                        sb ^= 1;
-                    } else if (n < args.N) {
+                            for (int i = 0; i < 16; ++i) {
+                                const __nv_bfloat16 o = __float2bfloat16_rn(fv(__uint_as_float(v[i])));
+                                asm volatile("st.shared.u16 [%0], %1;" ::"r"(sbuf + (uint32_t)i * 64u + (uint32_t)lane * 2u),
+                                             "h"(*reinterpret_cast<const unsigned short *>(&o)) : "memory");
+                            }
+                            __syncwarp();
+                            const int mi = lane >> 1, hf = lane & 1;
+                            if (m0 + mi < args.M) {
+                                const uint4 w0 = lds_v4(sbuf + (uint32_t)mi * 64u + (uint32_t)hf * 32u);
+                                const uint4 w1 = lds_v4(sbuf + (uint32_t)mi * 64u + (uint32_t)hf * 32u + 16u);
+                                uint4 *dst = reinterpret_cast<uint4 *>(args.y + (size_t)(m0 + mi) * args.N + n0 + hf * 16);
+                                dst[0] = w0;
+                                dst[1] = w1;
+                            }
+                            sb ^= 1;
+                        } else if (n < args.N) {
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const int m = m0 + i;
-                            if (m < args.M) {
-                                const __nv_bfloat16 o = __float2bfloat16_rn(__uint_as_float(v[i]) * scale);
-                                args.y[(size_t)m * args.N + n] = *reinterpret_cast<const uint16_t *>(&o);
+                            for (int i = 0; i < 16; ++i) {
+                                const int m = m0 + i;
+                                if (m < args.M) {
+                                    const __nv_bfloat16 o = __float2bfloat16_rn(fv(__uint_as_float(v[i])));
+                                    args.y[(size_t)m * args.N + n] = *reinterpret_cast<const uint16_t *>(&o);
+                                }
                             }
                         }
-                    }
+                    };
+                    if (plain) store_full(fv_plain);
+                    else store_full(fv_fused);
                 } else {
 #pragma unroll
                     for (int i = 0; i < 16; ++i) wsp[(size_t)(c0 + i) * C::BW + row] = __uint_as_float(v[i]);
@@ -781,14 +814,18 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
                                 cur[i] = nxt[i];
                             }
                         }
-                        if (n < args.N) {
+                        auto store8 = [&](auto &&fv) {
 #pragma unroll
                             for (int i = 0; i < 8; ++i) {
                                 if (c0 + i < mcols) {
-                                    const __nv_bfloat16 o = __float2bfloat16_rn(acc[i] * scale);
+                                    const __nv_bfloat16 o = __float2bfloat16_rn(fv(acc[i]));
                                     args.y[(size_t)(m_blk * BX + c0 + i) * args.N + n] = *reinterpret_cast<const uint16_t *>(&o);
                                 }
                             }
+                        };
+                        if (n < args.N) {
+                            if (plain) store8(fv_plain);
+                            else store8(fv_fused);
                         }
                     }
                     if (lane == 0) atomicExch(args.counters + (size_t)tile * 4 + q, 0u);   // ready for the next call

@@ -47,6 +47,9 @@ struct LinearArgs {
     const uint16_t *gmax;   // float16 [N, K / GS]
     int ngk;                // groups per row (K / GS)
     float lutf[16];         // (q/15)^(1/alpha) in fp32
+    // fused epilogue
+    const uint16_t *bias;   // bf16 [N] added to every output row, or null
+    int act;                // EPI_NONE, EPI_SILU, EPI_GELU_TANH
 };
 
 
@@ -546,7 +549,7 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
         uint32_t abph = 0;
         int xoff, xrows;
         // y[m0 .. m0 + 15][n] = bf16(v[i] * scale) for this lane's weight row n
-        auto store16 = [&](const uint32_t (&v)[16], int m0, int n, int n0, float scale) {
+        auto store16 = [&](const uint32_t (&v)[16], int m0, int n, int n0, auto &&fv) {
             if (vec_y && n0 + 32 <= args.N) {
                 // rows m0 + 2i and m0 + 2i + 1 packed as bf16 pairs; lanes n and n ^ 1 swap halves
                 // so that the even lane holds row m0 + 2i and the odd lane row m0 + 2i + 1, each
@@ -557,8 +560,7 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
                                                             (lane & ~1));
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    const uint32_t pk = pack_bf16x2_rn(__uint_as_float(v[2 * i]) * scale,
-                                                                __uint_as_float(v[2 * i + 1]) * scale);
+                    const uint32_t pk = pack_bf16x2_rn(fv(__uint_as_float(v[2 * i])), fv(__uint_as_float(v[2 * i + 1])));
                     const uint32_t other = __shfl_xor_sync(0xFFFFFFFFu, pk, 1);
                     const uint32_t word = __byte_perm(pk, other, sel);
                     if (m0 + 2 * i + (int)odd < args.M) yw[(size_t)i * (size_t)args.N] = word;
@@ -568,7 +570,7 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
                 for (int i = 0; i < 16; ++i) {
                     const int m = m0 + i;
                     if (m < args.M) {
-                        const __nv_bfloat16 o = __float2bfloat16_rn(__uint_as_float(v[i]) * scale);
+                        const __nv_bfloat16 o = __float2bfloat16_rn(fv(__uint_as_float(v[i])));
                         args.y[(size_t)m * args.N + n] = *reinterpret_cast<const uint16_t *>(&o);
                     }
                 }
@@ -580,6 +582,16 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
             const int n0 = n_blk * C::BW + q * 32;           // first row of this warp's quarter
             const bool full = (r0 == 0 && r1 == args.kblocks);
             const float scale = GS > 0 ? 1.0f : (n < args.N ? __ldg(args.scales + n) : 0.0f);
+            const float bias = bias_at(args.bias, n, args.N);
+            // the plain product, or the fused epilogue (bias, activation): chosen per tile, so the
+            // plain path carries none of the fused code
+            const bool plain = args.bias == nullptr && args.act == EPI_NONE;
+            auto fv_plain = [scale](float a) { return a * scale; };
+            auto fv_fused = [scale, bias, &args](float a) { return epi_value(a, scale, bias, args.act); };
+            auto store = [&](const uint32_t (&v)[16], int m0) {
+                if (plain) store16(v, m0, n, n0, fv_plain);
+                else store16(v, m0, n, n0, fv_fused);
+            };
             if (!warp_wait(&acc_full[ab], abph)) break;
             tc_fence_after();
             const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + C::A_COLS + ab * C::ACC_COLS;
@@ -589,7 +601,7 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
                     uint32_t v[16];
                     tmem_ld_32x32b_x16(taddr + c0, v);
                     tmem_ld_wait();
-                    store16(v, m_blk * BX + xoff + c0, n, n0, scale);
+                    store(v, m_blk * BX + xoff + c0);
                 }
             } else {
                 // Half-K tail run (the CTA's last): the tile's other half of K ran on the partner
@@ -642,7 +654,7 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
                                              : "=f"(o) : "r"(pbuf + (uint32_t)((c0 + i) * 32 + lane) * 4u));
                                 v[i] = __float_as_uint(__uint_as_float(v[i]) + o);
                             }
-                            store16(v, m_blk * BX + c0, n, n0, scale);
+                            store(v, m_blk * BX + c0);
                         }
                     }
                     // ready for the next call (after a timeout the workspace must be zeroed again)

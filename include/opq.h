@@ -126,6 +126,29 @@ opq_status opq_linear_grouped(const uint16_t *x, int64_t M, int64_t K, const uin
 opq_status opq_linear_grouped_workspace_size(int64_t M, int64_t N, int64_t K, int64_t group_size, size_t *bytes);
 
 /*
+ * Fused epilogue — the OPQLinear layers replace nn.Linear modules, which carry a
+ * bias, and in the transformer's feed-forward blocks an activation follows.
+ * opq_linear_fused / opq_linear_grouped_fused are opq_linear / opq_linear_grouped
+ * with, per output, v = sum * scale (per-row format; the group-wise sum carries its
+ * scales already) + bias[n], then the activation, in fp32, rounded once to bf16:
+ *   bias        bf16 [N] device (16-byte aligned), or NULL for none
+ *   activation  OPQ_ACT_NONE, OPQ_ACT_SILU (v / (1 + e^-v)) or OPQ_ACT_GELU_TANH
+ *               (0.5 v (1 + tanh(sqrt(2/pi) (v + 0.044715 v^3)))); anything else is
+ *               OPQ_ERR_INVALID_ARG
+ * Workspace and schedule as for the unfused calls.
+ */
+#define OPQ_ACT_NONE 0
+#define OPQ_ACT_SILU 1
+#define OPQ_ACT_GELU_TANH 2
+opq_status opq_linear_fused(const uint16_t *x, int64_t M, int64_t K, const uint32_t *codes, const uint32_t *signs,
+                            const float *scales, int64_t N, float alpha, const uint16_t *bias, int activation,
+                            uint16_t *y, void *workspace, size_t workspace_bytes, void *stream);
+opq_status opq_linear_grouped_fused(const uint16_t *x, int64_t M, int64_t K, const uint32_t *codes,
+                                    const uint32_t *signs, const uint16_t *gmax, int64_t N, int64_t group_size,
+                                    float alpha, const uint16_t *bias, int activation, uint16_t *y, void *workspace,
+                                    size_t workspace_bytes, void *stream);
+
+/*
  * opq_linear_workspace_size — device scratch bytes opq_linear needs for an
  * M x K by (N x K)^T product (0 when the chosen kernel needs none).
  */

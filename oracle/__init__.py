@@ -60,6 +60,8 @@ def _bind(path: str):
     lib.oracle_fp16_value.restype = D
     lib.oracle_fp16_from_nonneg.argtypes = [D]
     lib.oracle_fp16_from_nonneg.restype = ctypes.c_uint16
+    lib.oracle_apply_epilogue.argtypes = [P, I, I, P, ctypes.c_int]
+    lib.oracle_apply_epilogue.restype = None
     lib.oracle_rounding_mode_ok.restype = ctypes.c_int
     lib.oracle_num_threads.restype = ctypes.c_int
     return lib
@@ -236,6 +238,16 @@ class Oracle:
                                               ms.size, _p(ms), _p(ns), _p(y), _p(b))
         return y, b
 
+    def apply_epilogue(self, y: np.ndarray, bias=None, act: int = 0) -> np.ndarray:
+        """act(y + bias[n]) on a copy of y[M, N] (fp64); bias as bf16 bits [N] or None;
+        act 0 none, 1 SiLU, 2 GELU (tanh form)."""
+        y = np.array(y, dtype=np.float64, order="C", copy=True)
+        M, N = y.shape
+        b = None if bias is None else _u16(bias)
+        assert b is None or b.shape == (N,)
+        self._lib.oracle_apply_epilogue(_p(y), M, N, _p(b) if b is not None else None, int(act))
+        return y
+
     def fp16_value(self, bits: int) -> float:
         return float(self._lib.oracle_fp16_value(int(bits)))
 
@@ -321,6 +333,10 @@ def linear_grouped_pairs(*a, **k):
 
 def fp16_value(*a, **k):
     return default().fp16_value(*a, **k)
+
+
+def apply_epilogue(*a, **k):
+    return default().apply_epilogue(*a, **k)
 
 
 def fp16_from_nonneg(*a, **k):

@@ -29,6 +29,7 @@
  *
  * Build: plain C99, -O2, no fast-math (IEEE semantics are relied on).
  */
+#define _DEFAULT_SOURCE
 #include <fenv.h>
 #include <math.h>
 #include <stdlib.h>
@@ -414,6 +415,27 @@ void oracle_linear_grouped_pairs(const uint16_t *x, int64_t M, int64_t K, const 
     (void)N;
     planes_t p = {codes, signs, NULL, gmax, K, GS, alpha};
     linear_list(x, K, &p, count, ms, ns, y, bound);
+}
+
+/* ------------------------------------------------------------------------ */
+/* fused epilogue of the linear: the OPQLinear layers replace nn.Linear       */
+/* modules (y = x W^T + b); in the feed-forward blocks an activation follows. */
+/* In place on y[M, N]: y = act(y + bias[n]), fp64. act 0 none, 1 SiLU        */
+/* v / (1 + e^-v), 2 GELU's tanh form 0.5 v (1 + tanh(sqrt(2/pi) (v +        */
+/* 0.044715 v^3))). bias: bf16 bits [N] or NULL.                              */
+/* ------------------------------------------------------------------------ */
+void oracle_apply_epilogue(double *y, int64_t M, int64_t N, const uint16_t *bias, int act)
+{
+    const double c = sqrt(2.0 / M_PI);
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            double v = y[m * N + n] + (bias ? bf16_value(bias[n]) : 0.0);
+            if (act == 1)
+                v = v / (1.0 + exp(-v));
+            else if (act == 2)
+                v = 0.5 * v * (1.0 + tanh(c * (v + 0.044715 * v * v * v)));
+            y[m * N + n] = v;
+        }
 }
 
 /* ------------------------------------------------------------------------ */

@@ -410,3 +410,30 @@ def pin_grouped_linear(orc):
 
 PINS += [pin_fp16_conversion, pin_grouped_is_rowwise_per_group, pin_grouped_worked_example,
          pin_grouped_range_edges, pin_grouped_linear]
+
+
+# ------------------------------------------------------- fused epilogue pins --
+def pin_epilogue(orc):
+    """act(y + b): SiLU and GELU's tanh form against torch's fp64 implementations, closed forms
+    at 0 and 1 (silu(1) = 1 / (1 + e^-1), gelu_tanh(1) = (1 + tanh(sqrt(2/pi) 1.044715)) / 2),
+    and the bias added per output column."""
+    rng = np.random.default_rng(9)
+    y = rng.normal(0.0, 3.0, (5, 40))
+    t = torch.from_numpy(y)
+    assert np.allclose(orc.apply_epilogue(y, None, 1), torch.nn.functional.silu(t).numpy(), rtol=1e-14, atol=1e-15)
+    assert np.allclose(orc.apply_epilogue(y, None, 2),
+                       torch.nn.functional.gelu(t, approximate="tanh").numpy(), rtol=1e-14, atol=1e-15)
+    assert np.array_equal(orc.apply_epilogue(y, None, 0), y)
+    e = orc.apply_epilogue(np.array([[0.0, 1.0]]), None, 1)[0]
+    assert e[0] == 0.0 and abs(e[1] - 0.7310585786300049) < 1e-15
+    g = orc.apply_epilogue(np.array([[0.0, 1.0]]), None, 2)[0]
+    assert g[0] == 0.0 and abs(g[1] - 0.8411919906082768) < 1e-15
+    b = bf16_bits([0.5 * (i % 7) - 1.5 for i in range(40)])
+    got = orc.apply_epilogue(y, b, 0)
+    assert np.array_equal(got, y + bits_to_f64(b)[None, :])
+    assert np.allclose(orc.apply_epilogue(y, b, 1),
+                       torch.nn.functional.silu(t + torch.from_numpy(bits_to_f64(b))[None, :]).numpy(),
+                       rtol=1e-14, atol=1e-15)
+
+
+PINS += [pin_epilogue]

@@ -45,6 +45,10 @@ MUTANTS = [
      "double v = ldexp(floor(ldexp(a, -qexp)), qexp);"),
     ("fp16_ten_bits", "int qexp = e - 11;", "int qexp = e - 10;"),
     ("fp16_no_saturation", "if (v > 65504.0)\n        v = 65504.0;", "if (v > 1e30)\n        v = 65504.0;"),
+    # fused epilogue
+    ("silu_exp_sign", "v = v / (1.0 + exp(-v));", "v = v / (1.0 + exp(v));"),
+    ("gelu_square", "0.044715 * v * v * v", "0.044715 * v * v"),
+    ("bias_dropped", "double v = y[m * N + n] + (bias ? bf16_value(bias[n]) : 0.0);", "double v = y[m * N + n];"),
     ("fp16_subnormal_floor", "if (qexp < -24)\n        qexp = -24;", "if (qexp < -25)\n        qexp = -25;"),
 ]
 
