@@ -327,6 +327,12 @@ def gpu_arm(args, rank, world, local_rank):
     p_ = opq.quantize_grouped(w, 128, alpha)
     opq.dequantize_grouped(*p_, alpha, out=w_rec)
     snr[f"opq_alpha_{alpha:g}_group128"] = snr_db(w, w_rec)
+    if not args.no_sweep:
+        # the alpha search over 0.30 .. 1.00 (the card's configuration range) on this weight
+        for gs_ in (0, 128):
+            best_a, snrs = opq.alpha_search(w, opq.ALPHA_GRID, gs_)
+            snr[f"alpha_search_{'row' if gs_ == 0 else 'group128'}"] = {
+                "best_alpha": best_a, "snr_db": dict(zip([f"{a_:.2f}" for a_ in opq.ALPHA_GRID], snrs))}
     snr["gain_vs_int4_db"] = snr[f"opq_alpha_{alpha:g}"] - snr["int4_symmetric_row"]
     snr["gain_vs_alpha1_db"] = snr[f"opq_alpha_{alpha:g}"] - snr["opq_alpha_1"]
     snr["model_card_claim_db"] = 7.2

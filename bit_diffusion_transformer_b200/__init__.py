@@ -30,7 +30,7 @@ EXPORTS = ["opq_quantize", "opq_dequantize", "opq_linear_workspace_size", "opq_l
            "opq_linear_noalloc", "opq_device_error", "opq_status_string", "opq_last_cuda_error",
            "opq_abi_version", "opq_quantize_grouped", "opq_dequantize_grouped",
            "opq_linear_grouped", "opq_linear_grouped_workspace_size", "opq_linear_fused",
-           "opq_linear_grouped_fused"]
+           "opq_linear_grouped_fused", "opq_alpha_search", "opq_alpha_search_workspace_size"]
 ACTIVATIONS = {"none": 0, "silu": 1, "gelu_tanh": 2}
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
@@ -66,13 +66,16 @@ def load(path: str = LIB_PATH):
     lib.opq_dequantize_grouped.argtypes = [P, P, P, I, I, I, F, P, P]
     lib.opq_linear_grouped.argtypes = [P, I, I, P, P, P, I, I, F, P, P, S, P]
     lib.opq_linear_grouped_workspace_size.argtypes = [I, I, I, I, ctypes.POINTER(S)]
+    lib.opq_alpha_search_workspace_size.argtypes = [I, ctypes.POINTER(S)]
+    lib.opq_alpha_search.argtypes = [P, I, I, I, I, P, ctypes.c_int32, P, P, P, S, P]
     lib.opq_linear_fused.argtypes = [P, I, I, P, P, P, I, F, P, ctypes.c_int, P, P, S, P]
     lib.opq_linear_grouped_fused.argtypes = [P, I, I, P, P, P, I, I, F, P, ctypes.c_int, P, P, S, P]
     lib.opq_status_string.argtypes = [ctypes.c_int]
     lib.opq_status_string.restype = ctypes.c_char_p
     for f in ("opq_quantize", "opq_dequantize", "opq_linear_workspace_size", "opq_linear", "opq_linear_plan",
               "opq_linear_noalloc", "opq_device_error", "opq_quantize_grouped", "opq_dequantize_grouped", "opq_linear_grouped",
-              "opq_linear_grouped_workspace_size", "opq_linear_fused", "opq_linear_grouped_fused"):
+              "opq_linear_grouped_workspace_size", "opq_linear_fused", "opq_linear_grouped_fused",
+              "opq_alpha_search", "opq_alpha_search_workspace_size"):
         getattr(lib, f).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -227,6 +230,30 @@ def linear_grouped_fused(x: torch.Tensor, codes: torch.Tensor, signs: torch.Tens
                                            ACTIVATIONS[act], _ptr(y), ws_ptr, ws_bytes, _stream(x.device)),
            "opq_linear_grouped_fused")
     return y
+
+
+ALPHA_GRID = tuple(round(0.30 + 0.05 * i, 2) for i in range(15))   # 0.30 .. 1.00
+
+
+def alpha_search(w: torch.Tensor, alphas=ALPHA_GRID, group_size: int = 0):
+    """SNR (dB) of OPQ at each alpha for bf16 W[N, K] (per-row format, or group-wise when
+    group_size > 0) -> (best alpha, [snr_db per alpha])."""
+    import numpy as np
+    assert w.dtype == torch.bfloat16 and w.dim() == 2
+    _need_cuda(w)
+    N, K = w.shape
+    b = ctypes.c_size_t(0)
+    _check(load().opq_alpha_search_workspace_size(N, ctypes.byref(b)), "opq_alpha_search_workspace_size")
+    ws = torch.empty((b.value,), dtype=torch.uint8, device=w.device)
+    a = np.ascontiguousarray(alphas, dtype=np.float32)
+    snr = np.zeros(a.shape, dtype=np.float64)
+    best = ctypes.c_float(0.0)
+    _check(load().opq_alpha_search(_ptr(w), N, K, K, int(group_size), a.ctypes.data_as(ctypes.c_void_p), a.size,
+                                   snr.ctypes.data_as(ctypes.c_void_p), ctypes.byref(best), _ptr(ws), b.value,
+                                   _stream(w.device)), "opq_alpha_search")
+    i = int(np.argmax(snr))            # the first largest, as the library picks it
+    assert float(np.float32(alphas[i])) == best.value
+    return alphas[i], snr.tolist()
 
 
 def workspace_size(M: int, N: int, K: int) -> int:

@@ -9,6 +9,7 @@
 #include <cstring>
 #include <initializer_list>
 #include <mutex>
+#include <vector>
 
 #include "opq.h"
 #include "opq_dequantize.cuh"
@@ -470,6 +471,67 @@ opq_status opq_dequantize_grouped(const uint32_t *codes, const uint32_t *signs, 
     }
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? OPQ_OK : cuda_fail(e);
+}
+
+opq_status opq_alpha_search_workspace_size(int64_t N, size_t *bytes) {
+    if (!bytes || N < 1 || N > INT32_MAX) return OPQ_ERR_INVALID_ARG;
+    *bytes = (size_t)N * 2u * sizeof(double);
+    return OPQ_OK;
+}
+
+opq_status opq_alpha_search(const uint16_t *w, int64_t N, int64_t K, int64_t ldw, int64_t group_size,
+                            const float *alphas, int32_t count, double *snr_db, float *best_alpha, void *workspace,
+                            size_t workspace_bytes, void *stream) {
+    opq_status s = check_sizes(N, K);
+    if (s != OPQ_OK) return s;
+    if (group_size != 0 && (s = check_group(K, group_size)) != OPQ_OK) return s;
+    if (ldw < K || ldw % 8 != 0) return OPQ_ERR_INVALID_ARG;
+    if (!alphas || !snr_db || !best_alpha || count < 1) return OPQ_ERR_INVALID_ARG;
+    for (int32_t i = 0; i < count; ++i)
+        if (!alpha_ok(alphas[i])) return OPQ_ERR_INVALID_ARG;
+    if ((s = check_ptrs({w})) != OPQ_OK) return s;
+    if (!workspace || workspace_bytes < (size_t)N * 2u * sizeof(double)) return OPQ_ERR_WORKSPACE;
+    if ((s = check_ptrs({workspace})) != OPQ_OK) return s;
+    DeviceInfo *di = nullptr;
+    if ((s = device_info(&di)) != OPQ_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    double *err = reinterpret_cast<double *>(workspace);
+    double *sig = err + N;
+    std::vector<double> h((size_t)N * 2u);
+    const int64_t blocks = (N + 7) / 8;
+    const int grid = (int)(blocks < (int64_t)di->sms * 8 ? blocks : (int64_t)di->sms * 8);
+    int best = 0;
+    for (int32_t i = 0; i < count; ++i) {
+        const float alpha = alphas[i];
+        opqk::ErrorParams ep{};
+        const double inv = 1.0 / (double)alpha;
+        ep.qp.t[0] = 0.0;
+        for (int k = 1; k < 16; ++k) ep.qp.t[k] = std::pow(((double)k - 0.5) / 15.0, inv);
+        ep.qp.alpha_is_one = (alpha == 1.0f) ? 1 : 0;
+        for (int q = 0; q < 16; ++q) ep.lutf[q] = (float)std::pow((double)q / 15.0, inv);
+        switch (group_size) {
+            case 0: opqk::quant_error_kernel<0><<<grid, 256, 0, st>>>(w, N, K, ldw, ep, err, sig); break;
+            case 32: opqk::quant_error_kernel<32><<<grid, 256, 0, st>>>(w, N, K, ldw, ep, err, sig); break;
+            case 64: opqk::quant_error_kernel<64><<<grid, 256, 0, st>>>(w, N, K, ldw, ep, err, sig); break;
+            case 128: opqk::quant_error_kernel<128><<<grid, 256, 0, st>>>(w, N, K, ldw, ep, err, sig); break;
+            default: opqk::quant_error_kernel<256><<<grid, 256, 0, st>>>(w, N, K, ldw, ep, err, sig); break;
+        }
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e);
+        e = cudaMemcpyAsync(h.data(), err, (size_t)N * 2u * sizeof(double), cudaMemcpyDeviceToHost, st);
+        if (e != cudaSuccess) return cuda_fail(e);
+        e = cudaStreamSynchronize(st);
+        if (e != cudaSuccess) return cuda_fail(e);
+        double es = 0.0, ss = 0.0;
+        for (int64_t n = 0; n < N; ++n) {
+            es += h[(size_t)n];
+            ss += h[(size_t)(N + n)];
+        }
+        snr_db[i] = es == 0.0 ? HUGE_VAL : 10.0 * std::log10(ss / es);
+        if (snr_db[i] > snr_db[best]) best = i;
+    }
+    *best_alpha = alphas[best];
+    return OPQ_OK;
 }
 
 opq_status opq_dequantize(const uint32_t *codes, const uint32_t *signs, const float *scales, int64_t N, int64_t K,

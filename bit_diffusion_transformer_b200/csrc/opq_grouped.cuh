@@ -139,3 +139,105 @@ __global__ void __launch_bounds__(256) dequantize_grouped_kernel(const uint32_t 
 }
 
 }  // namespace opqk
+
+namespace opqk {
+
+// Quantization error of one alpha, for the alpha search: per row n, the squared error of the
+// decoded weights (sign equal, so (w - w')^2 = (|w| - LUT[q] max)^2 with LUT[q] max in fp32)
+// and the weights' squared sum, both accumulated in fp64 in a fixed order. GS = 0: the per-row
+// format (the row max first, then the row again); GS > 0: the group-wise format, rounds of 256
+// weights as in quantize_grouped_kernel. Codes come from the same exact threshold search.
+struct ErrorParams {
+    QuantParams qp;
+    float lutf[16];   // (q/15)^(1/alpha)
+};
+
+template <int GS>
+__global__ void __launch_bounds__(256) quant_error_kernel(const uint16_t *__restrict__ w, int64_t N, int64_t K,
+                                                          int64_t ldw, const __grid_constant__ ErrorParams ep,
+                                                          double *__restrict__ err, double *__restrict__ sig) {
+    constexpr int VPG = GS > 0 ? GS / 8 : 32;     // lanes sharing one max in a round (the warp for GS = 0)
+    constexpr int TPL = (15 + VPG - 1) / VPG;
+    __shared__ float lut_s[16];
+    if (threadIdx.x < 16) lut_s[threadIdx.x] = ep.lutf[threadIdx.x];
+    __syncthreads();
+    const int lane = threadIdx.x & 31;
+    const int seg = lane & ~(VPG - 1);
+    const int gl = lane - seg;
+    const int64_t nvec = K / 8, rounds = (nvec + 31) / 32;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t n = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); n < N; n += warps) {
+        const uint16_t *rp = w + n * ldw;
+        uint32_t rowmx = 0;
+        if (GS == 0) {
+            for (int64_t vi = lane; vi < nvec; vi += 32) {
+                const uint4 x = ld_stream_v4(rp + vi * 8);
+                const uint32_t m2 = __vmaxu2(__vmaxu2(x.x & 0x7FFF7FFFu, x.y & 0x7FFF7FFFu),
+                                             __vmaxu2(x.z & 0x7FFF7FFFu, x.w & 0x7FFF7FFFu));
+                rowmx = max(rowmx, max(m2 & 0xFFFFu, m2 >> 16));
+            }
+            rowmx = __reduce_max_sync(0xFFFFFFFFu, rowmx);
+        }
+        double e_acc = 0.0, s_acc = 0.0;
+        uint32_t P[16];
+        P[0] = 0;
+        float mxf = __uint_as_float(rowmx << 16);
+        if (GS == 0) {
+            uint32_t myT = 0x7F80u;
+            if (lane < 15 && rowmx != 0u) myT = level_threshold(mxf, lane + 1, ep.qp);
+#pragma unroll
+            for (int k = 1; k < 16; ++k) P[k] = __shfl_sync(0xFFFFFFFFu, myT, k - 1) * 0x00010001u;
+        }
+        for (int64_t r = 0; r < rounds; ++r) {
+            const int64_t vi = r * 32 + lane;
+            const bool valid = vi < nvec;
+            const uint4 x = valid ? ld_stream_v4(rp + vi * 8) : make_uint4(0, 0, 0, 0);
+            if (GS > 0) {
+                const uint32_t m2 = __vmaxu2(__vmaxu2(x.x & 0x7FFF7FFFu, x.y & 0x7FFF7FFFu),
+                                             __vmaxu2(x.z & 0x7FFF7FFFu, x.w & 0x7FFF7FFFu));
+                uint32_t mx = max(m2 & 0xFFFFu, m2 >> 16);
+#pragma unroll
+                for (int o = 1; o < VPG; o <<= 1) mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+                const uint16_t gb = fp16_bits_sat(__uint_as_float(mx << 16));
+                mxf = __half2float(__ushort_as_half(gb));
+                uint32_t myT[TPL];
+#pragma unroll
+                for (int t = 0; t < TPL; ++t) {
+                    const int k = gl + 1 + t * VPG;
+                    myT[t] = (k <= 15 && mxf != 0.0f) ? level_threshold(mxf, k, ep.qp) : 0x7F80u;
+                }
+#pragma unroll
+                for (int k = 1; k < 16; ++k)
+                    P[k] = __shfl_sync(0xFFFFFFFFu, myT[(k - 1) / VPG], seg + (k - 1) % VPG) * 0x00010001u;
+            }
+            const uint32_t words[4] = {x.x, x.y, x.z, x.w};
+            float e_r = 0.0f, s_r = 0.0f;
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                const uint32_t q2 = opqbits::quant_pair_f(words[p], P);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const float a = __uint_as_float(((words[p] >> (16 * h)) & 0x7FFFu) << 16);
+                    const float d = a - lut_s[(q2 >> (16 * h)) & 0xFu] * mxf;
+                    e_r = fmaf(d, d, e_r);
+                    s_r = fmaf(a, a, s_r);
+                }
+            }
+            if (valid) {
+                e_acc += (double)e_r;
+                s_acc += (double)s_r;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            e_acc += __shfl_xor_sync(0xFFFFFFFFu, e_acc, o);
+            s_acc += __shfl_xor_sync(0xFFFFFFFFu, s_acc, o);
+        }
+        if (lane == 0) {
+            err[n] = e_acc;
+            sig[n] = s_acc;
+        }
+    }
+}
+
+}  // namespace opqk

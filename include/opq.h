@@ -149,6 +149,24 @@ opq_status opq_linear_grouped_fused(const uint16_t *x, int64_t M, int64_t K, con
                                     size_t workspace_bytes, void *stream);
 
 /*
+ * opq_alpha_search — the card's alpha is a per-model choice in 0.3 .. 1.0 (its
+ * "OPQ configuration"; "why alpha = 0.73": a flat optimum on Z-Image weights). For
+ * each candidate alpha this quantizes W (per-row format when group_size is 0,
+ * else group-wise with that group size) and measures the SNR of the decoded
+ * weights against W, 10 log10(sum w^2 / sum (w - w')^2) with w' = sign *
+ * (q/15)^(1/alpha) * max in fp32, summed in fp64 in a fixed order. Nothing is
+ * written but the results; the call synchronises `stream`.
+ *   alphas       HOST float [count], each finite and > 0; count >= 1
+ *   snr_db       HOST double [count], written (+HUGE_VAL for an exact reconstruction)
+ *   best_alpha   HOST float, written: the first alpha with the largest SNR
+ *   workspace    device scratch of opq_alpha_search_workspace_size(N) bytes
+ */
+opq_status opq_alpha_search_workspace_size(int64_t N, size_t *bytes);
+opq_status opq_alpha_search(const uint16_t *w, int64_t N, int64_t K, int64_t ldw, int64_t group_size,
+                            const float *alphas, int32_t count, double *snr_db, float *best_alpha, void *workspace,
+                            size_t workspace_bytes, void *stream);
+
+/*
  * opq_linear_workspace_size — device scratch bytes opq_linear needs for an
  * M x K by (N x K)^T product (0 when the chosen kernel needs none).
  */

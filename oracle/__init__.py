@@ -335,6 +335,23 @@ def fp16_value(*a, **k):
     return default().fp16_value(*a, **k)
 
 
+def alpha_search(w, alphas, group_size: int = 0):
+    """SNR (dB) of the oracle's OPQ at each alpha: quantize, decode (unrounded fp64), SNR against
+    the bf16 weights -> (first alpha with the largest SNR, [snr per alpha])."""
+    o = default()
+    snr = []
+    for a in alphas:
+        if group_size:
+            r = o.quantize_grouped(w, group_size, float(a))
+            rec = o.dequantize_grouped_f64(r["codes"], r["signs"], r["gmax"], float(a))
+        else:
+            r = o.quantize(w, float(a))
+            rec = o.dequantize_f64(r["codes"], r["signs"], r["scales"], float(a))
+        snr.append(o.snr_db(w, rec))
+    best = max(range(len(snr)), key=lambda i: (snr[i], -i))
+    return float(alphas[best]), snr
+
+
 def apply_epilogue(*a, **k):
     return default().apply_epilogue(*a, **k)
 
