@@ -465,8 +465,12 @@ def profile_run(args):
     y = torch.empty((lin.M, lin.N), dtype=torch.bfloat16, device=dev)
     wq = torch.empty_like(w)
     ws = torch.zeros((max(opq.workspace_size(lin.M, lin.N, lin.K), 16),), dtype=torch.uint8, device=dev)
+    gplanes = opq.quantize_grouped(w, 128, lin.alpha)
+    gws = torch.zeros((max(opq.grouped_workspace_size(lin.M, lin.N, lin.K, 128), 16),), dtype=torch.uint8, device=dev)
     fns = {"quantize": lambda: opq.quantize(w, lin.alpha, out=planes),
-           "dequantize": lambda: opq.dequantize(*planes, lin.alpha, out=wq)}
+           "dequantize": lambda: opq.dequantize(*planes, lin.alpha, out=wq),
+           "grouped_quantize": lambda: opq.quantize_grouped(w, 128, lin.alpha, out=gplanes),
+           "grouped_linear": lambda: opq.linear_grouped(x, *gplanes, lin.alpha, out=y, workspace=gws)}
     fn = fns.get(args.profile, lambda: opq.linear(x, *planes, lin.alpha, out=y, workspace=ws))
     for _ in range(args.warmup):
         fn()
@@ -489,7 +493,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", default=None,
                     help="profiling run: warm up, then launch only this kernel --steps times "
-                         "(quantize | linear | dequantize | small<M>) on the bench workload")
+                         "(quantize | linear | dequantize | grouped_quantize | grouped_linear | small<M>) "
+                         "on the bench workload")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
