@@ -338,7 +338,6 @@ cudaError_t launch_linear_wide(DeviceInfo *di, const Plan &plan, const CUtensorM
     a.n_tiles = n.n_tiles;
     a.kblocks = n.kblocks;
     a.mode = n.mode;
-    a.runs_max = n.runs_max;
     a.tail_split = n.tail_split;
     for (int i = 0; i < 16; ++i) a.lut[i] = n.lut[i];
     a.gmax = n.gmax;

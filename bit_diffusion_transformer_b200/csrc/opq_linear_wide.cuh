@@ -37,8 +37,7 @@ struct LinearArgs {
     int M, N, K;
     int m_tiles, n_tiles;
     int kblocks;            // 128-K blocks per tile
-    int mode;               // 0 whole tiles strided over CTAs (the only mode this kernel is launched with)
-    int runs_max;           // mode 1: most runs one CTA can have
+    int mode;               // 0: whole tiles strided over CTAs (the only schedule this kernel runs)
     int tail_split;         // mode 0, tiles past the last whole wave: 2 = each runs as two half-width
                             // (BX/2 activation rows) runs on two CTAs; 3 = each runs as two
                             // half-K runs on two CTAs whose partial sums meet in `ws`; 1 = whole
@@ -54,17 +53,17 @@ struct LinearArgs {
 
 
 // The sequence of runs of one CTA; every role walks the same sequence. A run is one
-// weight tile, a range of its 128-K blocks and a range of its activation rows.
+// weight tile, a range of its 128-K blocks and a range of its activation rows. Whole tiles
+// are handed out strided over the CTAs; the tiles past the last whole wave are split over
+// two CTAs each (tail_split 2: activation rows, 3: K) or run whole (1).
 struct RunIter {
-    int mode, tiles, kblocks, grid, cta;
-    int64_t u, u_end;   // mode 1
-    int t_next;         // mode 0
-    int full_end;       // mode 0: tiles in whole waves (handed out strided)
-    int split;          // mode 0: tail_split
+    int tiles, kblocks, grid, cta;
+    int t_next;
+    int full_end;       // tiles in whole waves
+    int split;          // tail_split
     bool tail_done;
     int run_idx;
     __device__ __forceinline__ void init(const LinearArgs &a, int tiles_, int grid_, int cta_) {
-        mode = a.mode;
         tiles = tiles_;
         kblocks = a.kblocks;
         grid = grid_;
@@ -74,50 +73,34 @@ struct RunIter {
         split = a.tail_split;
         full_end = split >= 2 ? (tiles_ / grid_) * grid_ : tiles_;
         tail_done = false;
-        const int64_t U = (int64_t)tiles * kblocks;
-        u = unit_begin(cta_, grid_, U);
-        u_end = unit_begin(cta_ + 1, grid_, U);
     }
     // next run: tile, block range [r0, r1), run index j, activation rows [xoff, xoff + xrows)
     // of the tile's bx; false at the end
     __device__ __forceinline__ bool next(int &tile, int &r0, int &r1, int &j, int &xoff, int &xrows, int bx) {
         xoff = 0;
         xrows = bx;
-        if (mode == 0) {
-            if (t_next < full_end) {
-                tile = t_next;
-                t_next += grid;
-            } else if (split >= 2) {
-                // tail tile t is run by CTAs 2 (t - full_end) and 2 (t - full_end) + 1, one half
-                // of its activation rows (split 2) or of its 128-K blocks (split 3) each
-                if (tail_done || cta >= 2 * (tiles - full_end)) return false;
-                tile = full_end + (cta >> 1);
-                tail_done = true;
-                r0 = 0;
-                r1 = kblocks;
-                if (split == 2) {
-                    xrows = bx / 2;
-                    xoff = (cta & 1) * xrows;
-                } else {
-                    // the even CTA takes the smaller share of K, so that it has usually published
-                    // its partial sums by the time the odd CTA, which then adds them, is done
-                    const int k0 = kblocks * 7 / 16;
-                    if (cta & 1) r0 = k0; else r1 = k0;
-                }
-                j = run_idx++;
-                return true;
+        r0 = 0;
+        r1 = kblocks;
+        if (t_next < full_end) {
+            tile = t_next;
+            t_next += grid;
+        } else if (split >= 2) {
+            // tail tile t is run by CTAs 2 (t - full_end) and 2 (t - full_end) + 1, one half
+            // of its activation rows (split 2) or of its 128-K blocks (split 3) each
+            if (tail_done || cta >= 2 * (tiles - full_end)) return false;
+            tile = full_end + (cta >> 1);
+            tail_done = true;
+            if (split == 2) {
+                xrows = bx / 2;
+                xoff = (cta & 1) * xrows;
             } else {
-                return false;
+                // the even CTA takes the smaller share of K, so that it has usually published
+                // its partial sums by the time the odd CTA, which then adds them, is done
+                const int k0 = kblocks * 7 / 16;
+                if (cta & 1) r0 = k0; else r1 = k0;
             }
-            r0 = 0;
-            r1 = kblocks;
         } else {
-            if (u >= u_end) return false;
-            tile = (int)(u / kblocks);
-            r0 = (int)(u - (int64_t)tile * kblocks);
-            const int64_t end = (int64_t)r0 + (u_end - u);
-            r1 = end < (int64_t)kblocks ? (int)end : kblocks;
-            u += r1 - r0;
+            return false;
         }
         j = run_idx++;
         return true;
