@@ -60,6 +60,10 @@ def _bind(path: str):
     lib.oracle_fp16_value.restype = D
     lib.oracle_fp16_from_nonneg.argtypes = [D]
     lib.oracle_fp16_from_nonneg.restype = ctypes.c_uint16
+    lib.oracle_quantize_bits.argtypes = [P, I, I, I, ctypes.c_int, D, P, P, P, P, P]
+    lib.oracle_quantize_bits.restype = None
+    lib.oracle_dequantize_bits_f64.argtypes = [P, P, P, I, I, ctypes.c_int, D, P]
+    lib.oracle_dequantize_bits_bf16.argtypes = [P, P, P, I, I, ctypes.c_int, D, P]
     lib.oracle_apply_epilogue.argtypes = [P, I, I, P, ctypes.c_int]
     lib.oracle_apply_epilogue.restype = None
     lib.oracle_rounding_mode_ok.restype = ctypes.c_int
@@ -238,6 +242,44 @@ class Oracle:
                                               ms.size, _p(ms), _p(ns), _p(y), _p(b))
         return y, b
 
+    # ---- other bit widths: 2^bits - 1 levels, codes as one little-endian bit stream per row ----
+    def quantize_bits(self, w, bits: int, alpha: float, want_ties: bool = False, want_v: bool = False):
+        """Per-row OPQ with `bits`-bit magnitudes. Returns dict(codes uint32[N, K bits/32], signs,
+        scales, near_tie, v) as quantize does (v = L u^alpha)."""
+        w = _u16(w)
+        N, K = w.shape
+        assert K % 32 == 0 and bits in (3, 4, 5, 6)
+        lib = self._lib
+        assert lib.oracle_rounding_mode_ok() == 1
+        codes = np.zeros((N, K * bits // 32), np.uint32)
+        signs = np.zeros((N, K // 32), np.uint32)
+        scales = np.zeros((N,), np.float32)
+        ties = np.zeros((N, K), np.uint8) if want_ties else None
+        v = np.zeros((N, K), np.float64) if want_v else None
+        lib.oracle_quantize_bits(_p(w), N, K, K, int(bits), float(alpha), _p(codes), _p(signs), _p(scales),
+                                 _p(ties) if ties is not None else None, _p(v) if v is not None else None)
+        return dict(codes=codes, signs=signs, scales=scales, near_tie=ties, v=v)
+
+    def _bits_planes(self, codes, signs, scales, bits):
+        codes = np.ascontiguousarray(codes, np.uint32)
+        signs = np.ascontiguousarray(signs, np.uint32)
+        scales = np.ascontiguousarray(scales, np.float32)
+        N = codes.shape[0]
+        K = codes.shape[1] * 32 // bits
+        return codes, signs, scales, N, K
+
+    def dequantize_bits_f64(self, codes, signs, scales, bits: int, alpha: float) -> np.ndarray:
+        codes, signs, scales, N, K = self._bits_planes(codes, signs, scales, bits)
+        out = np.zeros((N, K), np.float64)
+        self._lib.oracle_dequantize_bits_f64(_p(codes), _p(signs), _p(scales), N, K, int(bits), float(alpha), _p(out))
+        return out
+
+    def dequantize_bits_bf16(self, codes, signs, scales, bits: int, alpha: float) -> np.ndarray:
+        codes, signs, scales, N, K = self._bits_planes(codes, signs, scales, bits)
+        out = np.zeros((N, K), np.uint16)
+        self._lib.oracle_dequantize_bits_bf16(_p(codes), _p(signs), _p(scales), N, K, int(bits), float(alpha), _p(out))
+        return out
+
     def apply_epilogue(self, y: np.ndarray, bias=None, act: int = 0) -> np.ndarray:
         """act(y + bias[n]) on a copy of y[M, N] (fp64); bias as bf16 bits [N] or None;
         act 0 none, 1 SiLU, 2 GELU (tanh form)."""
@@ -354,6 +396,18 @@ def alpha_search(w, alphas, group_size: int = 0):
 
 def apply_epilogue(*a, **k):
     return default().apply_epilogue(*a, **k)
+
+
+def quantize_bits(*a, **k):
+    return default().quantize_bits(*a, **k)
+
+
+def dequantize_bits_f64(*a, **k):
+    return default().dequantize_bits_f64(*a, **k)
+
+
+def dequantize_bits_bf16(*a, **k):
+    return default().dequantize_bits_bf16(*a, **k)
 
 
 def fp16_from_nonneg(*a, **k):

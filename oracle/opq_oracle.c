@@ -119,24 +119,30 @@ static double max_abs(const uint16_t *row, int64_t k0, int64_t k1)
 /* steps 2-4 for element k of row n against the max mx: code and sign into the packed planes
  * (cw code words and sw sign words per row, both zeroed beforehand), the near-tie flag and
  * 15 u^alpha */
-static void quantize_element(double wk, double mx, double alpha, int64_t n, int64_t k, int64_t K,
+static void quantize_element(double wk, double mx, double alpha, int bits, int64_t n, int64_t k, int64_t K,
                              int64_t cw, int64_t sw, uint32_t *codes, uint32_t *signs,
                              uint8_t *near_tie, double *v15_out)
 {
+    const double levels = (double)((1 << bits) - 1);   /* 15 for the card's 4 bits */
     double a = fabs(wk);
     double v15;
     if (mx == 0.0)
         v15 = 0.0;
     else if (alpha == 1.0)
-        v15 = (15.0 * a) / mx;                 /* u^1 = u */
+        v15 = (levels * a) / mx;                 /* u^1 = u */
     else
-        v15 = 15.0 * pow(a / mx, alpha);       /* 15 * u^alpha */
-    double qd = nearbyint(v15);                /* ties to even */
+        v15 = levels * pow(a / mx, alpha);       /* L * u^alpha */
+    double qd = nearbyint(v15);                  /* ties to even */
     if (qd < 0.0) qd = 0.0;
-    if (qd > OPQ_LEVELS) qd = OPQ_LEVELS;
+    if (qd > levels) qd = levels;
     uint32_t q = (uint32_t)qd;
     uint32_t s = (wk < 0.0) ? 1u : 0u;
-    codes[n * cw + k / 8] |= q << (4 * (k % 8));
+    /* the codes of a row as one little-endian bit stream: element k at bits k*bits .. of the
+     * row's words (for 4 bits: nibble k % 8 of word k / 8) */
+    const int64_t bit = k * bits;
+    codes[n * cw + bit / 32] |= q << (bit % 32);
+    if (bit % 32 + bits > 32)
+        codes[n * cw + bit / 32 + 1] |= q >> (32 - bit % 32);
     signs[n * sw + k / 32] |= s << (k % 32);
     if (near_tie)
         near_tie[n * K + k] = (fabs(v15 - (floor(v15) + 0.5)) <= 1e-6) ? 1 : 0;
@@ -160,7 +166,28 @@ void oracle_quantize(const uint16_t *w, int64_t N, int64_t K, int64_t ldw, doubl
         for (int64_t j = 0; j < sw; ++j)
             signs[n * sw + j] = 0;
         for (int64_t k = 0; k < K; ++k)
-            quantize_element(bf16_value(row[k]), mx, alpha, n, k, K, cw, sw, codes, signs, near_tie, v15_out);
+            quantize_element(bf16_value(row[k]), mx, alpha, 4, n, k, K, cw, sw, codes, signs, near_tie, v15_out);
+    }
+}
+
+/* the same per-row quantization with `bits` bits per magnitude (3, 4, 5 or 6; the card's
+ * "OPQ configuration" lists them, its storage section describes 4): 2^bits - 1 levels, the
+ * codes of a row packed as one little-endian bit stream of K * bits / 32 words */
+void oracle_quantize_bits(const uint16_t *w, int64_t N, int64_t K, int64_t ldw, int bits, double alpha,
+                          uint32_t *codes, uint32_t *signs, float *scales, uint8_t *near_tie, double *vl_out)
+{
+    const int64_t cw = K * bits / 32, sw = K / 32;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n) {
+        const uint16_t *row = w + n * ldw;
+        double mx = max_abs(row, 0, K);
+        scales[n] = (float)mx;
+        for (int64_t j = 0; j < cw; ++j)
+            codes[n * cw + j] = 0;
+        for (int64_t j = 0; j < sw; ++j)
+            signs[n * sw + j] = 0;
+        for (int64_t k = 0; k < K; ++k)
+            quantize_element(bf16_value(row[k]), mx, alpha, bits, n, k, K, cw, sw, codes, signs, near_tie, vl_out);
     }
 }
 
@@ -176,10 +203,25 @@ static uint32_t sign_at(const uint32_t *signs, int64_t K, int64_t n, int64_t k)
 }
 
 /* w' = sign * (q/15)^(1/alpha) * max, unrounded fp64 */
+static double dequant_value_levels(uint32_t q, uint32_t s, double alpha, double mx, double levels)
+{
+    double mag = pow((double)q / levels, 1.0 / alpha) * mx;
+    return s ? -mag : mag;
+}
+
 static double dequant_value(uint32_t q, uint32_t s, double alpha, double mx)
 {
-    double mag = pow((double)q / 15.0, 1.0 / alpha) * mx;
-    return s ? -mag : mag;
+    return dequant_value_levels(q, s, alpha, mx, 15.0);
+}
+
+/* code of element (n, k) of a `bits`-bit stream plane */
+static uint32_t code_at_bits(const uint32_t *codes, int64_t K, int bits, int64_t n, int64_t k)
+{
+    const int64_t cw = K * bits / 32, bit = k * bits;
+    uint64_t two = codes[n * cw + bit / 32];
+    if (bit % 32 + bits > 32)
+        two |= (uint64_t)codes[n * cw + bit / 32 + 1] << 32;
+    return (uint32_t)(two >> (bit % 32)) & ((1u << bits) - 1u);
 }
 
 /* dequantize to fp64 (unrounded) */
@@ -203,6 +245,29 @@ void oracle_dequantize_bf16(const uint32_t *codes, const uint32_t *signs, const 
             out[n * K + k] = double_to_bf16_rne(dequant_value(code_at(codes, K, n, k),
                                                               sign_at(signs, K, n, k),
                                                               alpha, (double)scales[n]));
+}
+
+void oracle_dequantize_bits_f64(const uint32_t *codes, const uint32_t *signs, const float *scales, int64_t N,
+                                int64_t K, int bits, double alpha, double *out)
+{
+    const double levels = (double)((1 << bits) - 1);
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k)
+            out[n * K + k] = dequant_value_levels(code_at_bits(codes, K, bits, n, k), sign_at(signs, K, n, k), alpha,
+                                                  (double)scales[n], levels);
+}
+
+void oracle_dequantize_bits_bf16(const uint32_t *codes, const uint32_t *signs, const float *scales, int64_t N,
+                                 int64_t K, int bits, double alpha, uint16_t *out)
+{
+    const double levels = (double)((1 << bits) - 1);
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k)
+            out[n * K + k] = double_to_bf16_rne(dequant_value_levels(code_at_bits(codes, K, bits, n, k),
+                                                                     sign_at(signs, K, n, k), alpha,
+                                                                     (double)scales[n], levels));
 }
 
 /* ------------------------------------------------------------------------ */
@@ -367,7 +432,7 @@ void oracle_quantize_grouped(const uint16_t *w, int64_t N, int64_t K, int64_t ld
             gmax[n * ng + g] = gb;
             /* steps 2-4 per weight, against the stored max */
             for (int64_t k = g * GS; k < (g + 1) * GS; ++k)
-                quantize_element(bf16_value(row[k]), fp16_value(gb), alpha, n, k, K, cw, sw, codes, signs,
+                quantize_element(bf16_value(row[k]), fp16_value(gb), alpha, 4, n, k, K, cw, sw, codes, signs,
                                  near_tie, v15_out);
         }
     }

@@ -437,3 +437,64 @@ def pin_epilogue(orc):
 
 
 PINS += [pin_epilogue]
+
+
+# ------------------------------------------------------ other bit widths pins --
+def pin_bits_four_is_default(orc):
+    """4-bit codes through the bit-width path equal the card's nibble format."""
+    w = tiny_weights()
+    for alpha in (0.45, 0.73, 1.0):
+        a = orc.quantize_bits(w, 4, alpha, want_ties=True)
+        b = orc.quantize(w, alpha, want_ties=True)
+        for k in ("codes", "signs", "scales", "near_tie"):
+            assert np.array_equal(a[k], b[k]), k
+
+
+def _stream_codes(codes: np.ndarray, K: int, bits: int) -> np.ndarray:
+    """Unpack a little-endian bit stream with Python integers (independent of the oracle)."""
+    out = np.zeros((codes.shape[0], K), np.int64)
+    for n in range(codes.shape[0]):
+        big = 0
+        for j, word in enumerate(codes[n].tolist()):
+            big |= int(word) << (32 * j)
+        for k in range(K):
+            out[n, k] = (big >> (k * bits)) & ((1 << bits) - 1)
+    return out
+
+
+def pin_bits_bruteforce(orc):
+    """3, 5 and 6 bits: every code is the nearest level of L u^alpha (L = 2^bits - 1, ties to
+    even) in long double, unpacked from the stream with Python integers."""
+    w = tiny_weights()[:24]
+    x = bits_to_f64(w).astype(np.longdouble)
+    mx = np.abs(x).max(axis=1, keepdims=True)
+    for bits in (3, 5, 6):
+        L = (1 << bits) - 1
+        for alpha in (0.45, 0.73):
+            r = orc.quantize_bits(w, bits, alpha, want_ties=True)
+            got = _stream_codes(r["codes"], w.shape[1], bits)
+            v = L * (np.abs(x) / mx) ** np.longdouble(alpha)
+            want = np.clip(np.rint(v), 0, L).astype(np.int64)
+            mism = (got != want) & ~r["near_tie"].astype(bool)
+            assert not mism.any(), (bits, alpha, int(mism.sum()))
+            assert np.array_equal(unpack_signs(r["signs"]), (x < 0).astype(np.uint8))
+
+
+def pin_bits_worked_stream(orc):
+    """3 bits at alpha = 1, by hand: row q/4 for q = 7, 0, 1, ..., 6 (max 1.75, so 7 |w| / max
+    = q exactly) -> codes q_k at bits 3k of a 96-bit stream, and the decode gives the row back."""
+    qs = [7, 0, 1, 2, 3, 4, 5, 6] * 4
+    row = [q / 4 for q in qs]
+    w = bf16_bits(row).reshape(1, 32)
+    r = orc.quantize_bits(w, 3, 1.0)
+    big = sum(q << (3 * k) for k, q in enumerate(qs))
+    want = [(big >> (32 * j)) & 0xFFFFFFFF for j in range(3)]
+    assert [int(v) for v in r["codes"][0]] == want
+    assert r["scales"][0] == 1.75
+    d = orc.dequantize_bits_f64(r["codes"], r["signs"], r["scales"], 3, 1.0)
+    assert np.array_equal(d[0], np.array(row))
+    db = orc.dequantize_bits_bf16(r["codes"], r["signs"], r["scales"], 3, 1.0)
+    assert np.array_equal(db[0], w[0])
+
+
+PINS += [pin_bits_four_is_default, pin_bits_bruteforce, pin_bits_worked_stream]

@@ -14,17 +14,17 @@ SRC = os.path.join(os.path.dirname(oracle.__file__), "opq_oracle.c")
 # (id, text in the oracle source, replacement): each must occur exactly once
 MUTANTS = [
     ("round_half_up", "double qd = nearbyint(v15);", "double qd = floor(v15 + 0.5);"),
-    ("nibble_order_reversed", "codes[n * cw + k / 8] |= q << (4 * (k % 8));",
-     "codes[n * cw + k / 8] |= q << (4 * (7 - k % 8));"),
+    ("nibble_order_reversed", "codes[n * cw + bit / 32] |= q << (bit % 32);",
+     "codes[n * cw + bit / 32] |= q << (28 - bit % 32);"),
     ("sign_bit_order_reversed", "signs[n * sw + k / 32] |= s << (k % 32);",
      "signs[n * sw + k / 32] |= s << (31 - k % 32);"),
-    ("forward_exponent_inverted", "v15 = 15.0 * pow(a / mx, alpha);",
-     "v15 = 15.0 * pow(a / mx, 1.0 / alpha);"),
-    ("inverse_exponent_not_inverted", "double mag = pow((double)q / 15.0, 1.0 / alpha) * mx;",
-     "double mag = pow((double)q / 15.0, alpha) * mx;"),
-    ("fourteen_levels", "v15 = 15.0 * pow(a / mx, alpha);", "v15 = 14.0 * pow(a / mx, alpha);"),
-    ("scale_dropped_in_dequant", "double mag = pow((double)q / 15.0, 1.0 / alpha) * mx;",
-     "double mag = pow((double)q / 15.0, 1.0 / alpha);"),
+    ("forward_exponent_inverted", "v15 = levels * pow(a / mx, alpha);",
+     "v15 = levels * pow(a / mx, 1.0 / alpha);"),
+    ("inverse_exponent_not_inverted", "double mag = pow((double)q / levels, 1.0 / alpha) * mx;",
+     "double mag = pow((double)q / levels, alpha) * mx;"),
+    ("fourteen_levels", "v15 = levels * pow(a / mx, alpha);", "v15 = (levels - 1.0) * pow(a / mx, alpha);"),
+    ("scale_dropped_in_dequant", "double mag = pow((double)q / levels, 1.0 / alpha) * mx;",
+     "double mag = pow((double)q / levels, 1.0 / alpha);"),
     ("sign_test_flipped", "uint32_t s = (wk < 0.0) ? 1u : 0u;", "uint32_t s = (wk > 0.0) ? 1u : 0u;"),
     ("negative_zero_negative", "uint32_t s = (wk < 0.0) ? 1u : 0u;", "uint32_t s = signbit(wk) ? 1u : 0u;"),
     ("sign_dropped_in_dequant", "return s ? -mag : mag;", "return mag;"),
@@ -45,6 +45,9 @@ MUTANTS = [
      "double v = ldexp(floor(ldexp(a, -qexp)), qexp);"),
     ("fp16_ten_bits", "int qexp = e - 11;", "int qexp = e - 10;"),
     ("fp16_no_saturation", "if (v > 65504.0)\n        v = 65504.0;", "if (v > 1e30)\n        v = 65504.0;"),
+    # bit widths other than 4
+    ("stream_carry_dropped", "two |= (uint64_t)codes[n * cw + bit / 32 + 1] << 32;", "two |= 0;"),
+    ("stream_carry_write_dropped", "codes[n * cw + bit / 32 + 1] |= q >> (32 - bit % 32);", "(void)0;"),
     # fused epilogue
     ("silu_exp_sign", "v = v / (1.0 + exp(-v));", "v = v / (1.0 + exp(v));"),
     ("gelu_square", "0.044715 * v * v * v", "0.044715 * v * v"),
