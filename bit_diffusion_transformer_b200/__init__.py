@@ -30,7 +30,8 @@ EXPORTS = ["opq_quantize", "opq_dequantize", "opq_linear_workspace_size", "opq_l
            "opq_linear_noalloc", "opq_device_error", "opq_status_string", "opq_last_cuda_error",
            "opq_abi_version", "opq_quantize_grouped", "opq_dequantize_grouped",
            "opq_linear_grouped", "opq_linear_grouped_workspace_size", "opq_linear_fused",
-           "opq_linear_grouped_fused", "opq_alpha_search", "opq_alpha_search_workspace_size"]
+           "opq_linear_grouped_fused", "opq_alpha_search", "opq_alpha_search_workspace_size",
+           "opq_quantize_bits", "opq_dequantize_bits"]
 ACTIVATIONS = {"none": 0, "silu": 1, "gelu_tanh": 2}
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
@@ -67,6 +68,8 @@ def load(path: str = LIB_PATH):
     lib.opq_linear_grouped.argtypes = [P, I, I, P, P, P, I, I, F, P, P, S, P]
     lib.opq_linear_grouped_workspace_size.argtypes = [I, I, I, I, ctypes.POINTER(S)]
     lib.opq_alpha_search_workspace_size.argtypes = [I, ctypes.POINTER(S)]
+    lib.opq_quantize_bits.argtypes = [P, I, I, I, ctypes.c_int32, F, P, P, P, P]
+    lib.opq_dequantize_bits.argtypes = [P, P, P, I, I, ctypes.c_int32, F, P, P]
     lib.opq_alpha_search.argtypes = [P, I, I, I, I, P, ctypes.c_int32, P, P, P, S, P]
     lib.opq_linear_fused.argtypes = [P, I, I, P, P, P, I, F, P, ctypes.c_int, P, P, S, P]
     lib.opq_linear_grouped_fused.argtypes = [P, I, I, P, P, P, I, I, F, P, ctypes.c_int, P, P, S, P]
@@ -75,7 +78,7 @@ def load(path: str = LIB_PATH):
     for f in ("opq_quantize", "opq_dequantize", "opq_linear_workspace_size", "opq_linear", "opq_linear_plan",
               "opq_linear_noalloc", "opq_device_error", "opq_quantize_grouped", "opq_dequantize_grouped", "opq_linear_grouped",
               "opq_linear_grouped_workspace_size", "opq_linear_fused", "opq_linear_grouped_fused",
-              "opq_alpha_search", "opq_alpha_search_workspace_size"):
+              "opq_alpha_search", "opq_alpha_search_workspace_size", "opq_quantize_bits", "opq_dequantize_bits"):
         getattr(lib, f).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -230,6 +233,34 @@ def linear_grouped_fused(x: torch.Tensor, codes: torch.Tensor, signs: torch.Tens
                                            ACTIVATIONS[act], _ptr(y), ws_ptr, ws_bytes, _stream(x.device)),
            "opq_linear_grouped_fused")
     return y
+
+
+def quantize_bits(w: torch.Tensor, bits: int, alpha: float = ALPHA, out=None):
+    """Per-row OPQ with `bits`-bit magnitudes (3..6) -> (codes int32 [N, K*bits/32], signs, scales)."""
+    assert w.dtype == torch.bfloat16 and w.dim() == 2
+    _need_cuda(w)
+    N, K = w.shape
+    if out is None:
+        codes = torch.empty((N, K * bits // 32), dtype=torch.int32, device=w.device)
+        signs = torch.empty((N, K // 32), dtype=torch.int32, device=w.device)
+        scales = torch.empty((N,), dtype=torch.float32, device=w.device)
+    else:
+        codes, signs, scales = out
+    _check(load().opq_quantize_bits(_ptr(w), N, K, K, int(bits), float(alpha), _ptr(codes), _ptr(signs), _ptr(scales),
+                                    _stream(w.device)), "opq_quantize_bits")
+    return codes, signs, scales
+
+
+def dequantize_bits(codes: torch.Tensor, signs: torch.Tensor, scales: torch.Tensor, bits: int, alpha: float = ALPHA,
+                    out=None):
+    """`bits`-bit packed planes -> bf16 W'[N, K]."""
+    _need_cuda(codes, signs, scales)
+    N = codes.shape[0]
+    K = codes.shape[1] * 32 // bits
+    w = out if out is not None else torch.empty((N, K), dtype=torch.bfloat16, device=codes.device)
+    _check(load().opq_dequantize_bits(_ptr(codes), _ptr(signs), _ptr(scales), N, K, int(bits), float(alpha), _ptr(w),
+                                      _stream(codes.device)), "opq_dequantize_bits")
+    return w
 
 
 ALPHA_GRID = tuple(round(0.30 + 0.05 * i, 2) for i in range(15))   # 0.30 .. 1.00

@@ -472,6 +472,63 @@ opq_status opq_dequantize_grouped(const uint32_t *codes, const uint32_t *signs, 
     return e == cudaSuccess ? OPQ_OK : cuda_fail(e);
 }
 
+opq_status opq_quantize_bits(const uint16_t *w, int64_t N, int64_t K, int64_t ldw, int32_t bits, float alpha,
+                             uint32_t *codes, uint32_t *signs, float *scales, void *stream) {
+    opq_status s = check_sizes(N, K);
+    if (s != OPQ_OK) return s;
+    if (bits < 3 || bits > 6) return OPQ_ERR_INVALID_ARG;
+    if (ldw < K || ldw % 8 != 0) return OPQ_ERR_INVALID_ARG;
+    if (!alpha_ok(alpha)) return OPQ_ERR_INVALID_ARG;
+    if ((s = check_ptrs({w, codes, signs, scales})) != OPQ_OK) return s;
+    const int L = (1 << bits) - 1;
+    opqk::BitsQuantParams bp{};
+    const double inv = 1.0 / (double)alpha;
+    for (int k = 1; k <= L; ++k) bp.t[k] = std::pow(((double)k - 0.5) / (double)L, inv);
+    bp.alpha_is_one = (alpha == 1.0f) ? 1 : 0;
+    DeviceInfo *di = nullptr;
+    if ((s = device_info(&di)) != OPQ_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t blocks = (N + 7) / 8;
+    const int grid = (int)(blocks < (int64_t)di->sms * 8 ? blocks : (int64_t)di->sms * 8);
+    switch (bits) {
+        case 3: opqk::quantize_bits_kernel<3><<<grid, 256, 0, st>>>(w, N, K, ldw, bp, codes, signs, scales); break;
+        case 4: opqk::quantize_bits_kernel<4><<<grid, 256, 0, st>>>(w, N, K, ldw, bp, codes, signs, scales); break;
+        case 5: opqk::quantize_bits_kernel<5><<<grid, 256, 0, st>>>(w, N, K, ldw, bp, codes, signs, scales); break;
+        default: opqk::quantize_bits_kernel<6><<<grid, 256, 0, st>>>(w, N, K, ldw, bp, codes, signs, scales); break;
+    }
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? OPQ_OK : cuda_fail(e);
+}
+
+opq_status opq_dequantize_bits(const uint32_t *codes, const uint32_t *signs, const float *scales, int64_t N, int64_t K,
+                               int32_t bits, float alpha, uint16_t *w_out, void *stream) {
+    opq_status s = check_sizes(N, K);
+    if (s != OPQ_OK) return s;
+    if (bits < 3 || bits > 6) return OPQ_ERR_INVALID_ARG;
+    if (!alpha_ok(alpha)) return OPQ_ERR_INVALID_ARG;
+    if ((uint64_t)N * (uint64_t)(K / 8) >= (1ull << 40)) return OPQ_ERR_UNSUPPORTED_SHAPE;
+    if ((s = check_ptrs({codes, signs, scales, w_out})) != OPQ_OK) return s;
+    const int L = (1 << bits) - 1;
+    opqk::BitsDequantParams dp{};
+    const double inv = 1.0 / (double)alpha;
+    for (int q = 0; q <= L; ++q) dp.lut[q] = std::pow((double)q / (double)L, inv);
+    DeviceInfo *di = nullptr;
+    if ((s = device_info(&di)) != OPQ_OK) return s;
+    uint64_t blocks = ((uint64_t)N + 7) / 8;
+    const uint64_t cap = (uint64_t)di->sms * 16;
+    if (blocks > cap) blocks = cap;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const uint32_t rows = (uint32_t)N, chunks = (uint32_t)(K / 32);
+    switch (bits) {
+        case 3: opqk::dequantize_bits_kernel<3><<<(int)blocks, 256, 0, st>>>(codes, signs, scales, rows, chunks, dp, w_out); break;
+        case 4: opqk::dequantize_bits_kernel<4><<<(int)blocks, 256, 0, st>>>(codes, signs, scales, rows, chunks, dp, w_out); break;
+        case 5: opqk::dequantize_bits_kernel<5><<<(int)blocks, 256, 0, st>>>(codes, signs, scales, rows, chunks, dp, w_out); break;
+        default: opqk::dequantize_bits_kernel<6><<<(int)blocks, 256, 0, st>>>(codes, signs, scales, rows, chunks, dp, w_out); break;
+    }
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? OPQ_OK : cuda_fail(e);
+}
+
 opq_status opq_alpha_search_workspace_size(int64_t N, size_t *bytes) {
     if (!bytes || N < 1 || N > INT32_MAX) return OPQ_ERR_INVALID_ARG;
     *bytes = (size_t)N * 2u * sizeof(double);

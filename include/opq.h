@@ -149,6 +149,22 @@ opq_status opq_linear_grouped_fused(const uint16_t *x, int64_t M, int64_t K, con
                                     size_t workspace_bytes, void *stream);
 
 /*
+ * Other bit widths — the card's configuration lists 3, 4, 5 and 6 bits per
+ * magnitude; its storage section describes 4. With `bits` bits there are
+ * L = 2^bits - 1 levels, q = round(L u^alpha) (ties to even) and
+ * w' = sign * (q/L)^(1/alpha) * max, one fp32 max per row. The codes of a row
+ * form one little-endian bit stream: element k at bits k*bits .. k*bits+bits-1
+ * of the row's K*bits/32 uint32 words (for 4 bits: nibble k % 8 of word k / 8,
+ * the per-row format above). Signs and scales as in the per-row format. These
+ * widths have quantize and dequantize; opq_linear takes 4-bit codes only.
+ *   codes  uint32 [N, K*bits/32];  bits 3..6 (OPQ_ERR_INVALID_ARG otherwise)
+ */
+opq_status opq_quantize_bits(const uint16_t *w, int64_t N, int64_t K, int64_t ldw, int32_t bits, float alpha,
+                             uint32_t *codes, uint32_t *signs, float *scales, void *stream);
+opq_status opq_dequantize_bits(const uint32_t *codes, const uint32_t *signs, const float *scales, int64_t N, int64_t K,
+                               int32_t bits, float alpha, uint16_t *w_out, void *stream);
+
+/*
  * opq_alpha_search — the card's alpha is a per-model choice in 0.3 .. 1.0 (its
  * "OPQ configuration"; "why alpha = 0.73": a flat optimum on Z-Image weights). For
  * each candidate alpha this quantizes W (per-row format when group_size is 0,

@@ -14,7 +14,7 @@ import bit_diffusion_transformer_b200 as opq
 import oracle
 import workloads
 from oracle_pins import unpack_codes
-from test_gpu_parity import (DEV, TIE_FRACTION_LIMIT, check_guards, guarded, no_device_error, to_dev_u32, u16,
+from test_gpu_parity import (DEV, TIE_FRACTION_LIMIT, alpha32, check_guards, guarded, no_device_error, to_dev_u32, u16,
                              u32)
 
 pytestmark = pytest.mark.gpu
@@ -92,7 +92,7 @@ def test_dequantize_grouped_bit_exact(gs, alpha):
     lin = workloads.Linear("grouped-dq", 1, 257, 1024, w_seed=gs)
     w = lin.make_weights("cpu")
     ref = oracle.quantize_grouped(w, gs, alpha)
-    want = oracle.dequantize_grouped_bf16(ref["codes"], ref["signs"], ref["gmax"], alpha)
+    want = oracle.dequantize_grouped_bf16(ref["codes"], ref["signs"], ref["gmax"], alpha32(alpha))
     N, K = w.shape
     ob, out, pad = guarded((N, K), torch.bfloat16, 0x77)
     gmax = torch.from_numpy(ref["gmax"].view(np.float16)).to(DEV)
@@ -111,7 +111,7 @@ def test_grouped_full_size_roundtrip():
     ref = grouped_quant_parity(w, 128, lin.alpha)
     codes, signs, gmax = opq.quantize_grouped(w, 128, lin.alpha)
     got = opq.dequantize_grouped(codes, signs, gmax, lin.alpha)
-    want = oracle.dequantize_grouped_bf16(u32(codes), u32(signs), u16(gmax), lin.alpha)
+    want = oracle.dequantize_grouped_bf16(u32(codes), u32(signs), u16(gmax), alpha32(lin.alpha))
     assert np.array_equal(u16(got), want)
     assert ref["gmax"].shape == (3840, 30)
     no_device_error()

@@ -26,6 +26,12 @@ DEV = "cuda"
 TIE_FRACTION_LIMIT = 1e-6
 
 
+def alpha32(alpha: float) -> float:
+    """The alpha a call receives: the C ABI passes it as float32, so bit-exact comparisons
+    evaluate the oracle at that value."""
+    return float(np.float32(alpha))
+
+
 def u16(t: torch.Tensor) -> np.ndarray:
     return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
 
@@ -140,7 +146,7 @@ def test_quantize_deterministic():
 def test_dequantize_bit_exact(alpha):
     w = workloads.tiny().make_weights("cpu")
     ref = oracle.quantize(w, alpha)
-    want = oracle.dequantize_bf16(ref["codes"], ref["signs"], ref["scales"], alpha)
+    want = oracle.dequantize_bf16(ref["codes"], ref["signs"], ref["scales"], alpha32(alpha))
     codes, signs = to_dev_u32(ref["codes"]), to_dev_u32(ref["signs"])
     scales = torch.from_numpy(ref["scales"]).to(DEV)
     N, K = w.shape
@@ -156,7 +162,7 @@ def test_dequantize_full_size_bit_exact():
     lin = workloads.small_m(1)
     w = lin.make_weights("cpu")
     ref = oracle.quantize(w, lin.alpha)
-    want = oracle.dequantize_bf16(ref["codes"], ref["signs"], ref["scales"], lin.alpha)
+    want = oracle.dequantize_bf16(ref["codes"], ref["signs"], ref["scales"], alpha32(lin.alpha))
     got = opq.dequantize(to_dev_u32(ref["codes"]), to_dev_u32(ref["signs"]),
                          torch.from_numpy(ref["scales"]).to(DEV), lin.alpha)
     assert np.array_equal(u16(got), want)
