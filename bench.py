@@ -128,11 +128,20 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
+        t0, t1 = getattr(self, "t0", 0.0), getattr(self, "t1", float("inf"))
+        out = self._summarise(t0, t1 + 0.05)
+        if out["sm_mhz"] is None:
+            # a timed region shorter than the sampling interval: the samples next to it
+            out = self._summarise(t0 - 0.15, t1 + 0.15)
+            if out["sm_mhz"] is not None:
+                out["window"] = "adjacent samples (timed region shorter than the 20 ms sampling interval)"
+        return out
+
+    def _summarise(self, lo, hi):
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        t0, t1 = getattr(self, "t0", 0.0), getattr(self, "t1", float("inf"))
         for ts, line in self.lines:
-            if not (t0 <= ts <= t1 + 0.05):
+            if not (lo <= ts <= hi):
                 continue
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:

@@ -602,11 +602,11 @@ opq_status opq_dequantize(const uint32_t *codes, const uint32_t *signs, const fl
     for (int q = 0; q < 16; ++q) dp.lut[q] = std::pow((double)q / 15.0, inv);
     DeviceInfo *di = nullptr;
     if ((s = device_info(&di)) != OPQ_OK) return s;
-    // one warp per row, 8 rows per block
-    uint64_t blocks = ((uint64_t)N + 7) / 8;
-    const uint64_t cap = (uint64_t)di->sms * 16;
+    // one warp per row, 4 rows per block
+    uint64_t blocks = ((uint64_t)N + 3) / 4;
+    const uint64_t cap = (uint64_t)di->sms * 32;
     if (blocks > cap) blocks = cap;
-    opqk::dequantize_kernel<<<(int)blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+    opqk::dequantize_kernel<<<(int)blocks, 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
         codes, signs, scales, (uint32_t)N, (uint32_t)(K / 32), dp, w_out);
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? OPQ_OK : cuda_fail(e);

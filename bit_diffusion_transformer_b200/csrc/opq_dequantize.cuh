@@ -6,8 +6,8 @@
 // to bf16 (one per lane), and every weight of the row is then a byte-plane table
 // lookup (opq_bits.h decode8) with its sign bit ORed in — the same bits as forming
 // the product per weight, since RNE is symmetric under negation.
-// One warp per row; a lane takes 32 weights at a time (16 B of codes + one sign word
-// in, 64 B out), consecutive lanes on consecutive chunks.
+// One warp per row, four rows per block; a lane takes one code word (8 weights) at a
+// time, consecutive lanes on consecutive words.
 #pragma once
 #include "opq_bits.h"
 #include "opq_device.cuh"
@@ -30,28 +30,32 @@ __device__ __forceinline__ uint32_t f64_to_bf16_rne(double p) {
     return (fb + 0x7FFFu + ((fb >> 16) & 1u)) >> 16;
 }
 
-__global__ void __launch_bounds__(256) dequantize_kernel(const uint32_t *__restrict__ codes,
+// Lane l of a row's warp takes the code words l, l + 32, ... (8 weights each): per word a
+// 4-byte code load, its sign byte, and a 16-byte bf16 store, so that each warp-wide store
+// covers 512 contiguous bytes. The first batch of loads goes out before the row's table
+// is formed, so the fp64 products and shuffles overlap their latency.
+constexpr int DQ_BATCH = 16;   // code words per lane in flight
+
+__global__ void __launch_bounds__(128) dequantize_kernel(const uint32_t *__restrict__ codes,
                                                          const uint32_t *__restrict__ signs,
                                                          const float *__restrict__ scales, uint32_t rows,
                                                          uint32_t chunks, const __grid_constant__ DequantParams dp,
                                                          uint16_t *__restrict__ out) {
     const uint32_t lane = threadIdx.x & 31u;
     const uint32_t warps = gridDim.x * (blockDim.x >> 5);
+    const uint32_t nwords = chunks * 4u;   // code words per row
     // lane q (and q + 16) holds LUT[q] for the products
     const double lut_q = dp.lut[lane & 15u];
     for (uint32_t n = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); n < rows; n += warps) {
-        const uint4 *crow = reinterpret_cast<const uint4 *>(codes + (size_t)n * chunks * 4u);
-        const uint32_t *srow = signs + (size_t)n * chunks;
+        const uint32_t *crow = codes + (size_t)n * nwords;
+        const uint8_t *sbytes = reinterpret_cast<const uint8_t *>(signs + (size_t)n * chunks);
         uint4 *orow = reinterpret_cast<uint4 *>(out + (size_t)n * chunks * 32u);
-        // the first pass's loads go out before the row's table is formed, so that the fp64
-        // products and shuffles overlap their latency
-        uint4 c[4];
-        uint32_t sw[4];
+        uint32_t c[DQ_BATCH], sb[DQ_BATCH];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const uint32_t i = lane + 32u * u;
-            c[u] = i < chunks ? __ldg(crow + i) : make_uint4(0u, 0u, 0u, 0u);
-            sw[u] = i < chunks ? __ldg(srow + i) : 0u;
+        for (int u = 0; u < DQ_BATCH; ++u) {
+            const uint32_t j = lane + 32u * u;
+            c[u] = j < nwords ? __ldg(crow + j) : 0u;
+            sb[u] = j < nwords ? (uint32_t)__ldg(sbytes + j) : 0u;
         }
         const uint32_t e = f64_to_bf16_rne(lut_q * (double)__ldg(scales + n));
         opqbits::DecodeTable T;
@@ -67,29 +71,23 @@ __global__ void __launch_bounds__(256) dequantize_kernel(const uint32_t *__restr
             T.L[j] = l;
             T.H[j] = h;
         }
-        // up to four chunks per lane per pass, the next pass's loads issued before decoding
-        for (uint32_t i0 = lane; i0 < chunks; i0 += 128u) {
+        for (uint32_t j0 = lane;; j0 += 32u * DQ_BATCH) {
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const uint32_t i = i0 + 32u * u;
-                if (i >= chunks) break;
-                uint32_t o[16];
-                opqbits::decode8(c[u].x, sw[u] & 0xFFu, T, &o[0]);
-                opqbits::decode8(c[u].y, (sw[u] >> 8) & 0xFFu, T, &o[4]);
-                opqbits::decode8(c[u].z, (sw[u] >> 16) & 0xFFu, T, &o[8]);
-                opqbits::decode8(c[u].w, sw[u] >> 24, T, &o[12]);
-                uint4 *dst = orow + (size_t)i * 4u;
-                dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
-                dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
-                dst[2] = make_uint4(o[8], o[9], o[10], o[11]);
-                dst[3] = make_uint4(o[12], o[13], o[14], o[15]);
+            for (int u = 0; u < DQ_BATCH; ++u) {
+                const uint32_t j = j0 + 32u * u;
+                if (j < nwords) {
+                    uint32_t o[4];
+                    opqbits::decode8(c[u], sb[u], T, o);
+                    orow[j] = make_uint4(o[0], o[1], o[2], o[3]);
+                }
             }
-            const uint32_t i1 = i0 + 128u;
+            const uint32_t j1 = j0 + 32u * DQ_BATCH;
+            if (j1 - lane >= nwords) break;   // warp-uniform: no word of the next batch exists
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const uint32_t i = i1 + 32u * u;
-                c[u] = i < chunks ? __ldg(crow + i) : make_uint4(0u, 0u, 0u, 0u);
-                sw[u] = i < chunks ? __ldg(srow + i) : 0u;
+            for (int u = 0; u < DQ_BATCH; ++u) {
+                const uint32_t j = j1 + 32u * u;
+                c[u] = j < nwords ? __ldg(crow + j) : 0u;
+                sb[u] = j < nwords ? (uint32_t)__ldg(sbytes + j) : 0u;
             }
         }
     }

@@ -5,10 +5,17 @@
 //
 // One row is handled by a group of G warps (G = 1 for K <= 4096, 8 above).
 // Every lane loads its 16-byte vectors of the row once (coalesced, kept in
-// registers), the group reduces max |w| in the bf16 bit domain, lanes 0..14
-// form the 15 exact per-row thresholds in fp64, and each vector of 8 weights is
-// coded by a branch-free binary search on two bf16 halves at a time with packed
-// bf16 compares (opqbits::quant_pair_f) — no pow on the device.
+// registers), the group reduces max |w| in the bf16 bit domain, and lanes 0..14
+// form the 15 exact per-row thresholds T_k in fp64 — no pow on the device.
+//
+// Coding by table. For a non-negative bf16 value the bit pattern is monotone in
+// the value, so q(|w|) = #{k : T_k <= |w|} is a non-increasing step function of
+// d = bits(max) - bits(|w|), and q = 0 from d_z = bits(max) - T_1 + 1 on. The group
+// writes the row's table q(d), d = 0..d_z, one byte per entry, into shared memory
+// (each thread walks a contiguous run of entries down the thresholds), and every
+// weight is then one packed subtract, one clamp and one byte lookup. Rows whose
+// table would not fit (d_z >= TAB_ENTRIES: alpha below about 0.16) or whose max is
+// NaN take the branch-free binary search on bf16 pairs (opqbits::quant_pair_f).
 #pragma once
 #include "opq_bits.h"
 #include "opq_device.cuh"
@@ -42,8 +49,19 @@ __device__ __forceinline__ uint32_t level_threshold(float mxf, int k, const Quan
     return tb < 0x7F80u ? tb : 0x7F80u;   // +inf: unreachable (only for a non-finite max)
 }
 
+constexpr uint32_t TAB_ENTRIES = 4096;   // bytes of a row's code table
+
+// codes of two bf16 weights (a pair) by table: d = min(bits(max) - bits(|w|), d_z) per half,
+// both halves offset by the row's table offset in the block's tables (mmb = (max + base) per
+// half, dzb = (d_z + base) per half: base <= 7 * TAB_ENTRIES = 28672 and max <= 0x7F80, so no
+// half passes 16 bits, and max >= |w| per half, so nothing borrows across halves)
+__device__ __forceinline__ uint32_t table_pair(const uint8_t *tb, uint32_t x, uint32_t mmb, uint32_t dzb) {
+    const uint32_t d = __vminu2(mmb - (x & 0x7FFF7FFFu), dzb);
+    return (uint32_t)tb[d & 0xFFFFu] | ((uint32_t)tb[d >> 16] << 16);
+}
+
 template <int G, int VPL>
-__global__ void __launch_bounds__(256) quantize_kernel(const uint16_t *__restrict__ w, int64_t N, int64_t K,
+__global__ void __launch_bounds__(256, 2) quantize_kernel(const uint16_t *__restrict__ w, int64_t N, int64_t K,
                                                        int64_t ldw, const __grid_constant__ QuantParams qp,
                                                        uint32_t *__restrict__ codes, uint32_t *__restrict__ signs,
                                                        float *__restrict__ scales) {
@@ -53,6 +71,8 @@ __global__ void __launch_bounds__(256) quantize_kernel(const uint16_t *__restric
     const int gl = (warp % G) * 32 + lane;  // lane index inside the row group
     const int64_t nvec = K / 8;
     __shared__ uint32_t red[8];
+    __shared__ __align__(16) uint32_t tab[ROWS][TAB_ENTRIES / 4];
+    __shared__ uint16_t thr[ROWS][16];
 
     for (int64_t row0 = (int64_t)blockIdx.x * ROWS; row0 < N; row0 += (int64_t)gridDim.x * ROWS) {
         const int64_t n = row0 + slot;
@@ -86,20 +106,72 @@ __global__ void __launch_bounds__(256) quantize_kernel(const uint16_t *__restric
         // +inf marks a level no finite weight reaches (all levels of an all-zero row)
         uint32_t myT = 0x7F80u;
         if (lane < 15 && mx != 0u) myT = level_threshold(mxf, lane + 1, qp);
-        uint32_t P[16];
-        P[0] = 0;
-#pragma unroll
-        for (int k = 1; k < 16; ++k) P[k] = __shfl_sync(0xFFFFFFFFu, myT, k - 1) * 0x00010001u;
+        const uint32_t T1 = __shfl_sync(0xFFFFFFFFu, myT, 0);
+        const uint32_t dz = T1 <= mx ? mx - T1 + 1u : 0u;
+        // group-uniform: mx is the group's max
+        const bool by_table = mx <= 0x7F80u && dz < TAB_ENTRIES;
 
         if (valid && gl == 0) scales[n] = mxf;
         uint32_t *crow = codes + (valid ? n : 0) * nvec;
         uint32_t *srow = signs + (valid ? n : 0) * (nvec / 4);
+        uint32_t cw[VPL];
+        if (by_table) {
+            if (gl < 15) thr[slot][gl + 1] = (uint16_t)myT;
+            if (G == 1) __syncwarp(); else __syncthreads();
+            // entries 0..dz as words of 4; a thread takes a contiguous run, starting from
+            // q(e0) = #{k : T_k <= max - e0} and lowering q as max - e drops below T_q
+            const uint32_t words = (dz + 4u) >> 2, per = (words + 32u * G - 1u) / (32u * G);
+            const uint32_t w0 = (uint32_t)gl * per, w1 = min(w0 + per, words);
+            if (w0 < w1) {
+                const int b0 = (int)mx - (int)(4u * w0);
+                uint32_t q = 0;
+#pragma unroll
+                for (int k = 1; k < 16; ++k) q += (int)thr[slot][k] <= b0 ? 1u : 0u;
+                int tq = q ? (int)thr[slot][q] : 0;
+                for (uint32_t wd = w0; wd < w1; ++wd) {
+                    uint32_t word = 0;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int b = (int)mx - (int)(4u * wd + j);
+                        while (q > 0u && b < tq) {
+                            --q;
+                            tq = q ? (int)thr[slot][q] : 0;
+                        }
+                        word |= q << (8 * j);
+                    }
+                    tab[slot][wd] = word;
+                }
+            }
+            if (G == 1) __syncwarp(); else __syncthreads();
+            const uint8_t *tb = reinterpret_cast<const uint8_t *>(&tab[0][0]);
+            const uint32_t base = (uint32_t)slot * TAB_ENTRIES;
+            const uint32_t mmb = (mx + base) * 0x00010001u, dzb = (dz + base) * 0x00010001u;
+#pragma unroll
+            for (int j = 0; j < VPL; ++j) {
+                const uint4 x = v[j];
+                // q_p holds element 2p in bits 0..3 and element 2p+1 in bits 16..19
+                cw[j] = opqbits::pack_codes(table_pair(tb, x.x, mmb, dzb), table_pair(tb, x.y, mmb, dzb),
+                                            table_pair(tb, x.z, mmb, dzb), table_pair(tb, x.w, mmb, dzb));
+            }
+            // the table and thresholds are rewritten for the next row only after every
+            // thread of the group has finished its lookups
+            if (G == 1) __syncwarp(); else __syncthreads();
+        } else {
+            uint32_t P[16];
+            P[0] = 0;
+#pragma unroll
+            for (int k = 1; k < 16; ++k) P[k] = __shfl_sync(0xFFFFFFFFu, myT, k - 1) * 0x00010001u;
+#pragma unroll
+            for (int j = 0; j < VPL; ++j) {
+                const uint4 x = v[j];
+                cw[j] = opqbits::pack_codes(opqbits::quant_pair_f(x.x, P), opqbits::quant_pair_f(x.y, P),
+                                            opqbits::quant_pair_f(x.z, P), opqbits::quant_pair_f(x.w, P));
+            }
+        }
 #pragma unroll
         for (int j = 0; j < VPL; ++j) {
             const int64_t vi = (int64_t)j * 32 * G + gl;
             const uint4 x = v[j];
-            const uint32_t code = opqbits::pack_codes(opqbits::quant_pair_f(x.x, P), opqbits::quant_pair_f(x.y, P),
-                                                      opqbits::quant_pair_f(x.z, P), opqbits::quant_pair_f(x.w, P));
             // sign bit = w < 0 (so -0.0 stores 0): a packed compare with zero gives 0xFFFF per
             // negative half, whose top bit sign_byte collects
             const uint32_t sb = opqbits::sign_byte(opqbits::bf16x2_neg_mask(x.x), opqbits::bf16x2_neg_mask(x.y),
@@ -109,7 +181,7 @@ __global__ void __launch_bounds__(256) quantize_kernel(const uint16_t *__restric
             sw |= __shfl_xor_sync(0xFFFFFFFFu, sw, 1);
             sw |= __shfl_xor_sync(0xFFFFFFFFu, sw, 2);
             if (valid && vi < nvec) {
-                crow[vi] = code;
+                crow[vi] = cw[j];
                 if ((gl & 3) == 0) srow[vi / 4] = sw;
             }
         }

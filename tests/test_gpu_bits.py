@@ -23,7 +23,7 @@ def bits_parity(w, bits, alpha):
     for b, p, f in ((cb, cpad, 0xA5), (sb, spad, 0x5A), (fb, fpad, 0x3C)):
         check_guards(b, p, f)
     no_device_error()
-    ref = oracle.quantize_bits(w, bits, alpha, want_ties=True)
+    ref = oracle.quantize_bits(w, bits, alpha32(alpha), want_ties=True)
     assert np.array_equal(u32(scales.view(torch.int32)), ref["scales"].view(np.uint32))
     assert np.array_equal(u32(signs), ref["signs"])
     if np.array_equal(u32(codes), ref["codes"]):

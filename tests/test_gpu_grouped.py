@@ -33,7 +33,7 @@ def grouped_quant_parity(w: torch.Tensor, gs: int, alpha: float):
     check_guards(sb, spad, 0x5A)
     check_guards(gb, gpad, 0x3C)
     no_device_error()
-    ref = oracle.quantize_grouped(w, gs, alpha, want_ties=True)
+    ref = oracle.quantize_grouped(w, gs, alpha32(alpha), want_ties=True)
     assert np.array_equal(u16(gmax), ref["gmax"]), "group maxima differ"
     assert np.array_equal(u32(signs), ref["signs"]), "signs differ"
     qg, qo = unpack_codes(u32(codes)), unpack_codes(ref["codes"])

@@ -80,7 +80,7 @@ def quant_parity(w: torch.Tensor, alpha: float, rows=None):
     check_guards(fb, fpad, 0x3C)
     no_device_error()
     wc = w if rows is None else w[torch.as_tensor(rows, device=w.device)]
-    ref = oracle.quantize(wc, alpha, want_ties=True)
+    ref = oracle.quantize(wc, alpha32(alpha), want_ties=True)
     sel = slice(None) if rows is None else np.asarray(rows)
     g_scales = u32(scales.view(torch.int32))[sel]
     assert np.array_equal(g_scales, ref["scales"].view(np.uint32)), "scales differ"
@@ -109,6 +109,16 @@ def test_quantize_shapes(N, K):
     quant_parity(lin.make_weights(DEV), 0.73)
 
 
+@pytest.mark.parametrize("alpha", [0.1, 0.2, 0.3, 3.0])
+@pytest.mark.parametrize("N,K", [(40, 3840), (3, 10240)])
+def test_quantize_alpha_range(alpha, N, K):
+    # a row's code table covers bits(max) - bits(|w|) up to 4095: alpha 0.2 and 0.3 fill
+    # most of it, alpha 0.1 needs more (those rows take the threshold search instead),
+    # alpha 3 crowds the levels near the max; one warp per row (K = 3840) and eight (10240)
+    lin = workloads.Linear("alpha-range", 1, N, K, w_seed=N + K)
+    quant_parity(lin.make_weights(DEV), alpha)
+
+
 def test_quantize_ldw_and_special_rows():
     N, K, ldw = 8, 96, 136
     g = torch.Generator(device=DEV).manual_seed(3)
@@ -126,7 +136,7 @@ def test_quantize_ldw_and_special_rows():
         st = opq.load().opq_quantize(opq._ptr(big), N, K, ldw, alpha, opq._ptr(codes), opq._ptr(signs),
                                      opq._ptr(scales), opq._stream(big.device))
         assert st == 0
-        ref = oracle.quantize(big[:, :K].contiguous(), alpha, want_ties=True)
+        ref = oracle.quantize(big[:, :K].contiguous(), alpha32(alpha), want_ties=True)
         assert np.array_equal(u32(codes), ref["codes"])
         assert np.array_equal(u32(signs), ref["signs"])
         assert np.array_equal(u32(scales.view(torch.int32)), ref["scales"].view(np.uint32))
