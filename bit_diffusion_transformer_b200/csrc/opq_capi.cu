@@ -394,10 +394,10 @@ opq_status opq_quantize(const uint16_t *w, int64_t N, int64_t K, int64_t ldw, fl
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const int64_t nvec = K / 8;
     if (K <= 4096) {
-        const int vpl = (int)((nvec + 31) / 32);
-        const int64_t blocks = (N + 7) / 8;
-        const int grid = (int)(blocks < (int64_t)di->sms * 8 ? blocks : (int64_t)di->sms * 8);
-        dispatch_quant<1>(vpl, w, N, K, ldw, qp, codes, signs, scales, grid, st);
+        // one warp per row, two rows per block
+        const int64_t blocks = (N + opqk::QR_ROWS - 1) / opqk::QR_ROWS;
+        const int grid = (int)(blocks < (int64_t)di->sms * 32 ? blocks : (int64_t)di->sms * 32);
+        opqk::quantize_rows_kernel<<<grid, 64, 0, st>>>(w, N, K, ldw, qp, codes, signs, scales);
     } else {
         const int vpl = (int)((nvec + 255) / 256);
         const int64_t blocks = N;

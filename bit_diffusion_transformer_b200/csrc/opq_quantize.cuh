@@ -3,7 +3,7 @@
 // "OPQ INT4 Z-Image" model card, "OPQ principle": u = |w|/max, v = u^alpha,
 // q = round(15 v); "storage format": 8 magnitudes and 32 signs per uint32.
 //
-// One row is handled by a group of G warps (G = 1 for K <= 4096, 8 above).
+// quantize_kernel (K > 4096): one row is handled by a group of G = 8 warps.
 // Every lane loads its 16-byte vectors of the row once (coalesced, kept in
 // registers), the group reduces max |w| in the bf16 bit domain, and lanes 0..14
 // form the 15 exact per-row thresholds T_k in fp64 — no pow on the device.
@@ -184,6 +184,145 @@ __global__ void __launch_bounds__(256, 2) quantize_kernel(const uint16_t *__rest
                 crow[vi] = cw[j];
                 if ((gl & 3) == 0) srow[vi / 4] = sw;
             }
+        }
+    }
+}
+
+// ------------------------------------------------------------------------------------------
+// K <= 4096: one warp per row, two rows per 64-thread block, and the row read twice — a first
+// pass for max |w| (8 vectors per lane in flight), a second for the codes (the row is then in
+// L2). Holding no row in registers keeps a thread near 60 registers, so every row of a
+// projection-sized matrix is in flight at once (about 26 rows per SM) instead of 16 rows per
+// SM in two uneven waves. Coding as in quantize_kernel: the row's table where it fits, the
+// packed binary search otherwise.
+// ------------------------------------------------------------------------------------------
+constexpr int QR_ROWS = 2;
+
+struct TableCoder {
+    const uint8_t *tb;
+    uint32_t mmb, dzb;
+    __device__ __forceinline__ uint32_t operator()(const uint4 &x) const {
+        return opqbits::pack_codes(table_pair(tb, x.x, mmb, dzb), table_pair(tb, x.y, mmb, dzb),
+                                   table_pair(tb, x.z, mmb, dzb), table_pair(tb, x.w, mmb, dzb));
+    }
+};
+
+struct SearchCoder {
+    uint32_t P[16];
+    __device__ __forceinline__ uint32_t operator()(const uint4 &x) const {
+        return opqbits::pack_codes(opqbits::quant_pair_f(x.x, P), opqbits::quant_pair_f(x.y, P),
+                                   opqbits::quant_pair_f(x.z, P), opqbits::quant_pair_f(x.w, P));
+    }
+};
+
+// the coding pass of one row by one warp: vectors lane, lane + 32, ... in batches of B per lane
+template <int B, class Coder>
+__device__ __forceinline__ void code_row(const Coder &cd, const uint16_t *rp, int64_t nvec, int lane,
+                                         uint32_t *crow, uint32_t *srow) {
+    for (int64_t v0 = 0; v0 < nvec; v0 += 32 * B) {
+        uint4 x[B];
+#pragma unroll
+        for (int u = 0; u < B; ++u) {
+            const int64_t vi = v0 + 32 * u + lane;
+            x[u] = vi < nvec ? ld_stream_v4(rp + vi * 8) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < B; ++u) {
+            const int64_t vi = v0 + 32 * u + lane;
+            const uint32_t code = cd(x[u]);
+            const uint32_t sb = opqbits::sign_byte(opqbits::bf16x2_neg_mask(x[u].x), opqbits::bf16x2_neg_mask(x[u].y),
+                                                   opqbits::bf16x2_neg_mask(x[u].z), opqbits::bf16x2_neg_mask(x[u].w));
+            // four consecutive vectors (lanes 4m .. 4m+3 of one batch slot) form one sign word
+            uint32_t sw = sb << (8 * (lane & 3));
+            sw |= __shfl_xor_sync(0xFFFFFFFFu, sw, 1);
+            sw |= __shfl_xor_sync(0xFFFFFFFFu, sw, 2);
+            if (vi < nvec) {
+                crow[vi] = code;
+                if ((lane & 3) == 0) srow[vi / 4] = sw;
+            }
+        }
+    }
+}
+
+__global__ void __launch_bounds__(64) quantize_rows_kernel(const uint16_t *__restrict__ w, int64_t N, int64_t K,
+                                                           int64_t ldw, const __grid_constant__ QuantParams qp,
+                                                           uint32_t *__restrict__ codes,
+                                                           uint32_t *__restrict__ signs,
+                                                           float *__restrict__ scales) {
+    constexpr int B = 8;
+    const int lane = threadIdx.x & 31, slot = threadIdx.x >> 5;
+    const int64_t nvec = K / 8;
+    __shared__ __align__(16) uint32_t tab[QR_ROWS][TAB_ENTRIES / 4];
+    __shared__ uint16_t thr[QR_ROWS][16];
+
+    // warps never wait on one another (only __syncwarp below), so a warp without a row leaves
+    for (int64_t n = (int64_t)blockIdx.x * QR_ROWS + slot; n < N; n += (int64_t)gridDim.x * QR_ROWS) {
+        const uint16_t *rp = w + n * ldw;
+        uint32_t mx2 = 0;
+        for (int64_t v0 = 0; v0 < nvec; v0 += 32 * B) {
+            uint4 x[B];
+#pragma unroll
+            for (int u = 0; u < B; ++u) {
+                const int64_t vi = v0 + 32 * u + lane;
+                x[u] = vi < nvec ? ld_stream_v4(rp + vi * 8) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int u = 0; u < B; ++u) {
+                mx2 = __vmaxu2(mx2, x[u].x & 0x7FFF7FFFu);
+                mx2 = __vmaxu2(mx2, x[u].y & 0x7FFF7FFFu);
+                mx2 = __vmaxu2(mx2, x[u].z & 0x7FFF7FFFu);
+                mx2 = __vmaxu2(mx2, x[u].w & 0x7FFF7FFFu);
+            }
+        }
+        uint32_t mx = max(mx2 & 0xFFFFu, mx2 >> 16);
+        mx = __reduce_max_sync(0xFFFFFFFFu, mx);
+        const float mxf = __uint_as_float(mx << 16);
+        uint32_t myT = 0x7F80u;
+        if (lane < 15 && mx != 0u) myT = level_threshold(mxf, lane + 1, qp);
+        const uint32_t T1 = __shfl_sync(0xFFFFFFFFu, myT, 0);
+        const uint32_t dz = T1 <= mx ? mx - T1 + 1u : 0u;
+        if (lane == 0) scales[n] = mxf;
+        uint32_t *crow = codes + n * nvec;
+        uint32_t *srow = signs + n * (nvec / 4);
+        if (mx <= 0x7F80u && dz < TAB_ENTRIES) {
+            if (lane < 15) thr[slot][lane + 1] = (uint16_t)myT;
+            __syncwarp();
+            const uint32_t words = (dz + 4u) >> 2, per = (words + 31u) >> 5;
+            const uint32_t w0 = (uint32_t)lane * per, w1 = min(w0 + per, words);
+            if (w0 < w1) {
+                const int b0 = (int)mx - (int)(4u * w0);
+                uint32_t q = 0;
+#pragma unroll
+                for (int k = 1; k < 16; ++k) q += (int)thr[slot][k] <= b0 ? 1u : 0u;
+                int tq = q ? (int)thr[slot][q] : 0;
+                for (uint32_t wd = w0; wd < w1; ++wd) {
+                    uint32_t word = 0;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int b = (int)mx - (int)(4u * wd + j);
+                        while (q > 0u && b < tq) {
+                            --q;
+                            tq = q ? (int)thr[slot][q] : 0;
+                        }
+                        word |= q << (8 * j);
+                    }
+                    tab[slot][wd] = word;
+                }
+            }
+            __syncwarp();
+            const uint32_t base = (uint32_t)slot * TAB_ENTRIES;
+            const TableCoder cd{reinterpret_cast<const uint8_t *>(&tab[0][0]), (mx + base) * 0x00010001u,
+                                (dz + base) * 0x00010001u};
+            code_row<B>(cd, rp, nvec, lane, crow, srow);
+            // the row's table and thresholds are rewritten for the next row only after every
+            // lane has finished its lookups
+            __syncwarp();
+        } else {
+            SearchCoder cd;
+            cd.P[0] = 0;
+#pragma unroll
+            for (int k = 1; k < 16; ++k) cd.P[k] = __shfl_sync(0xFFFFFFFFu, myT, k - 1) * 0x00010001u;
+            code_row<4>(cd, rp, nvec, lane, crow, srow);
         }
     }
 }
