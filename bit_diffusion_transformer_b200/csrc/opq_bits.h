@@ -133,6 +133,57 @@ OPQ_HD uint32_t pack_codes(uint32_t q0, uint32_t q1, uint32_t q2, uint32_t q3) {
     return prmt(prmt(t0, t1, 0x0040u), prmt(t2, t3, 0x0040u), 0x5410u);
 }
 
+// ---------------------------------------------------------------------------
+// Coding by table. For non-negative bf16 values the bit pattern is monotone in
+// the value, so with a row's nondecreasing thresholds T_1..T_15 (bf16 bits) the
+// code q(a) = #{k : T_k <= a} of a magnitude a <= mx depends only on d = mx - a,
+// and is 0 from d_z = mx - T_1 + 1 on.
+// ---------------------------------------------------------------------------
+// Entries e in [4 w0, 4 w1) of the table q(mx - e), as words of four bytes (byte j
+// of word wd is entry 4 wd + j): q at the first entry by counting, then lowered
+// while walking down the thresholds. T[1..15] must be nondecreasing; entries past
+// mx (e > mx) are 0.
+OPQ_HD void code_table_run(const uint16_t *T, uint32_t mx, uint32_t w0, uint32_t w1, uint32_t *tab) {
+    if (w0 >= w1) return;
+    const int b0 = (int)mx - (int)(4u * w0);
+    uint32_t q = 0;
+    for (int k = 1; k < 16; ++k) q += (int)T[k] <= b0 ? 1u : 0u;
+    int tq = q ? (int)T[q] : 0;
+    for (uint32_t wd = w0; wd < w1; ++wd) {
+        uint32_t word = 0;
+        for (int j = 0; j < 4; ++j) {
+            const int b = (int)mx - (int)(4u * wd + j);
+            while (q > 0u && b < tq) {
+                --q;
+                tq = q ? (int)T[q] : 0;
+            }
+            word |= q << (8 * j);
+        }
+        tab[wd] = word;
+    }
+}
+
+// per-half unsigned 16-bit minimum
+OPQ_HD uint32_t vminu2(uint32_t a, uint32_t b) {
+#if defined(__CUDA_ARCH__)
+    return __vminu2(a, b);
+#else
+    const uint32_t lo = (a & 0xFFFFu) < (b & 0xFFFFu) ? (a & 0xFFFFu) : (b & 0xFFFFu);
+    const uint32_t hi = (a >> 16) < (b >> 16) ? (a >> 16) : (b >> 16);
+    return lo | (hi << 16);
+#endif
+}
+
+// Codes of a bf16 pair x (q in bits 0..3 and 16..19) from a row's table stored at
+// byte offset `base` of tb: per half d = min(mx - |w|, d_z), read at base + d.
+// mmb = (mx + base) and dzb = (d_z + base) in both halves; the caller keeps
+// mx + base below 2^16 and |w| <= mx per half, so nothing carries or borrows
+// across the halves.
+OPQ_HD uint32_t table_pair(const uint8_t *tb, uint32_t x, uint32_t mmb, uint32_t dzb) {
+    const uint32_t d = vminu2(mmb - (x & 0x7FFF7FFFu), dzb);
+    return (uint32_t)tb[d & 0xFFFFu] | ((uint32_t)tb[d >> 16] << 16);
+}
+
 // Sign bits (bf16 sign bit set) of 8 weights held as 4 bf16 pairs -> bits 0..7.
 OPQ_HD uint32_t sign_byte(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3) {
     // gather the high byte of every bf16 (its top bit is the sign), then move the

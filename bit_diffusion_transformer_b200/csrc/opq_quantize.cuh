@@ -51,14 +51,8 @@ __device__ __forceinline__ uint32_t level_threshold(float mxf, int k, const Quan
 
 constexpr uint32_t TAB_ENTRIES = 4096;   // bytes of a row's code table
 
-// codes of two bf16 weights (a pair) by table: d = min(bits(max) - bits(|w|), d_z) per half,
-// both halves offset by the row's table offset in the block's tables (mmb = (max + base) per
-// half, dzb = (d_z + base) per half: base <= 7 * TAB_ENTRIES = 28672 and max <= 0x7F80, so no
-// half passes 16 bits, and max >= |w| per half, so nothing borrows across halves)
-__device__ __forceinline__ uint32_t table_pair(const uint8_t *tb, uint32_t x, uint32_t mmb, uint32_t dzb) {
-    const uint32_t d = __vminu2(mmb - (x & 0x7FFF7FFFu), dzb);
-    return (uint32_t)tb[d & 0xFFFFu] | ((uint32_t)tb[d >> 16] << 16);
-}
+// Table lookups (opqbits::table_pair) index a block's tables with the row's table offset
+// base <= 7 * TAB_ENTRIES = 28672 folded in; with max <= 0x7F80 no half passes 16 bits.
 
 template <int G, int VPL>
 __global__ void __launch_bounds__(256, 2) quantize_kernel(const uint16_t *__restrict__ w, int64_t N, int64_t K,
@@ -122,26 +116,7 @@ __global__ void __launch_bounds__(256, 2) quantize_kernel(const uint16_t *__rest
             // q(e0) = #{k : T_k <= max - e0} and lowering q as max - e drops below T_q
             const uint32_t words = (dz + 4u) >> 2, per = (words + 32u * G - 1u) / (32u * G);
             const uint32_t w0 = (uint32_t)gl * per, w1 = min(w0 + per, words);
-            if (w0 < w1) {
-                const int b0 = (int)mx - (int)(4u * w0);
-                uint32_t q = 0;
-#pragma unroll
-                for (int k = 1; k < 16; ++k) q += (int)thr[slot][k] <= b0 ? 1u : 0u;
-                int tq = q ? (int)thr[slot][q] : 0;
-                for (uint32_t wd = w0; wd < w1; ++wd) {
-                    uint32_t word = 0;
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int b = (int)mx - (int)(4u * wd + j);
-                        while (q > 0u && b < tq) {
-                            --q;
-                            tq = q ? (int)thr[slot][q] : 0;
-                        }
-                        word |= q << (8 * j);
-                    }
-                    tab[slot][wd] = word;
-                }
-            }
+            opqbits::code_table_run(&thr[slot][0], mx, w0, w1, &tab[slot][0]);
             if (G == 1) __syncwarp(); else __syncthreads();
             const uint8_t *tb = reinterpret_cast<const uint8_t *>(&tab[0][0]);
             const uint32_t base = (uint32_t)slot * TAB_ENTRIES;
@@ -150,8 +125,8 @@ __global__ void __launch_bounds__(256, 2) quantize_kernel(const uint16_t *__rest
             for (int j = 0; j < VPL; ++j) {
                 const uint4 x = v[j];
                 // q_p holds element 2p in bits 0..3 and element 2p+1 in bits 16..19
-                cw[j] = opqbits::pack_codes(table_pair(tb, x.x, mmb, dzb), table_pair(tb, x.y, mmb, dzb),
-                                            table_pair(tb, x.z, mmb, dzb), table_pair(tb, x.w, mmb, dzb));
+                cw[j] = opqbits::pack_codes(opqbits::table_pair(tb, x.x, mmb, dzb), opqbits::table_pair(tb, x.y, mmb, dzb),
+                                            opqbits::table_pair(tb, x.z, mmb, dzb), opqbits::table_pair(tb, x.w, mmb, dzb));
             }
             // the table and thresholds are rewritten for the next row only after every
             // thread of the group has finished its lookups
@@ -202,8 +177,8 @@ struct TableCoder {
     const uint8_t *tb;
     uint32_t mmb, dzb;
     __device__ __forceinline__ uint32_t operator()(const uint4 &x) const {
-        return opqbits::pack_codes(table_pair(tb, x.x, mmb, dzb), table_pair(tb, x.y, mmb, dzb),
-                                   table_pair(tb, x.z, mmb, dzb), table_pair(tb, x.w, mmb, dzb));
+        return opqbits::pack_codes(opqbits::table_pair(tb, x.x, mmb, dzb), opqbits::table_pair(tb, x.y, mmb, dzb),
+                                   opqbits::table_pair(tb, x.z, mmb, dzb), opqbits::table_pair(tb, x.w, mmb, dzb));
     }
 };
 
@@ -289,26 +264,7 @@ __global__ void __launch_bounds__(64) quantize_rows_kernel(const uint16_t *__res
             __syncwarp();
             const uint32_t words = (dz + 4u) >> 2, per = (words + 31u) >> 5;
             const uint32_t w0 = (uint32_t)lane * per, w1 = min(w0 + per, words);
-            if (w0 < w1) {
-                const int b0 = (int)mx - (int)(4u * w0);
-                uint32_t q = 0;
-#pragma unroll
-                for (int k = 1; k < 16; ++k) q += (int)thr[slot][k] <= b0 ? 1u : 0u;
-                int tq = q ? (int)thr[slot][q] : 0;
-                for (uint32_t wd = w0; wd < w1; ++wd) {
-                    uint32_t word = 0;
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int b = (int)mx - (int)(4u * wd + j);
-                        while (q > 0u && b < tq) {
-                            --q;
-                            tq = q ? (int)thr[slot][q] : 0;
-                        }
-                        word |= q << (8 * j);
-                    }
-                    tab[slot][wd] = word;
-                }
-            }
+            opqbits::code_table_run(&thr[slot][0], mx, w0, w1, &tab[slot][0]);
             __syncwarp();
             const uint32_t base = (uint32_t)slot * TAB_ENTRIES;
             const TableCoder cd{reinterpret_cast<const uint8_t *>(&tab[0][0]), (mx + base) * 0x00010001u,

@@ -136,6 +136,61 @@ int main() {
             }
         }
     }
+    // --- code_table_run / table_pair: the quantize kernels' per-row code table. Thresholds
+    // nondecreasing (crowded, repeated, unreachable), every thread partition the kernels use;
+    // each entry against q(b) = #{k : T_k <= b}, each lookup against q(|w|) for every |w| <= mx
+    {
+        auto count_le = [](const uint16_t *T, int b) {
+            uint32_t q = 0;
+            for (int k = 1; k < 16; ++k) q += (int)T[k] <= b ? 1u : 0u;
+            return q;
+        };
+        const uint32_t TAB = 4096;
+        std::vector<uint32_t> tabw(8 * TAB / 4);
+        for (int trial = 0; trial < 600; ++trial) {
+            uint32_t mx = (uint32_t)(rng() % 0x7F81u);
+            if (trial % 9 == 0) mx = 0x7F80u;            // +inf max
+            if (trial % 13 == 0) mx = (uint32_t)(rng() % 64u);   // subnormal-range max
+            uint16_t T[16] = {0};
+            if (mx == 0u || trial % 17 == 0) {
+                for (int k = 1; k < 16; ++k) T[k] = 0x7F80u;   // an all-zero row: no level reachable
+            } else {
+                // T_15 <= mx; spread below it over up to 16 binades, or crowded near it
+                std::vector<uint32_t> v(15);
+                const uint32_t span = (trial % 5 == 0) ? 40u : 2048u + (uint32_t)(rng() % 2048u);
+                for (auto &x : v) x = mx > span ? mx - (uint32_t)(rng() % span) : 1u + (uint32_t)(rng() % mx);
+                if (trial % 7 == 0) v[3] = v[4] = v[5];        // repeated thresholds
+                std::sort(v.begin(), v.end());
+                for (int k = 1; k < 16; ++k) T[k] = (uint16_t)std::max<uint32_t>(1u, v[k - 1]);
+            }
+            const uint32_t T1 = T[1];
+            const uint32_t dz = T1 <= mx ? mx - T1 + 1u : 0u;
+            if (dz >= TAB) continue;                           // such rows take the search
+            const uint32_t words = (dz + 4u) >> 2;
+            for (uint32_t P : {1u, 32u, 256u}) {
+                const uint32_t slot = (uint32_t)(rng() % 8u), base = slot * TAB;
+                std::fill(tabw.begin(), tabw.end(), 0xEEEEEEEEu);
+                const uint32_t per = (words + P - 1u) / P;
+                for (uint32_t g = 0; g < P; ++g) {
+                    const uint32_t w0 = g * per, w1 = std::min(w0 + per, words);
+                    code_table_run(T, mx, w0, w1, &tabw[base / 4]);
+                }
+                const uint8_t *tb = reinterpret_cast<const uint8_t *>(tabw.data());
+                for (uint32_t e = 0; e < 4u * words; ++e)
+                    CHECK(tb[base + e] == count_le(T, (int)mx - (int)e), "code_table_run trial %d P %u e %u got %u want %u",
+                          trial, P, e, tb[base + e], count_le(T, (int)mx - (int)e));
+                const uint32_t mmb = (mx + base) * 0x00010001u, dzb = (dz + base) * 0x00010001u;
+                const uint32_t step = mx > 20000u ? 7u : 1u;
+                for (uint32_t a = 0; a <= mx; a += step) {
+                    const uint32_t a2 = (uint32_t)(rng() % (mx + 1u));
+                    const uint32_t x = a | (a2 << 16) | ((uint32_t)(rng() & 1u) << 15) | ((uint32_t)(rng() & 1u) << 31);
+                    const uint32_t q = table_pair(tb, x, mmb, dzb);
+                    const uint32_t want = count_le(T, (int)a) | (count_le(T, (int)a2) << 16);
+                    CHECK(q == want, "table_pair trial %d a %x a2 %x got %x want %x", trial, a, a2, q, want);
+                }
+            }
+        }
+    }
     std::printf("%s fails=%d\n", fails ? "FAIL" : "OK", fails);
     return fails ? 1 : 0;
 }
