@@ -151,3 +151,9 @@ def test_shard_range_covers_rows():
             assert max(sizes) - min(sizes) <= 1 and max(sizes) == sharded.shard_width(n, world)
     with pytest.raises(ValueError):
         sharded.shard_range(8, 2, 2)
+    # more ranks than rows: the rank without a row is refused before it quantizes anything
+    calls = []
+    with pytest.raises(ValueError):
+        sharded.quantize_shard(torch.zeros((1, 32), dtype=torch.bfloat16), 1, 2, 0.73,
+                               quantize_fn=lambda w, a: calls.append(w.shape))
+    assert calls == []
