@@ -111,7 +111,7 @@ __device__ __forceinline__ void fence_proxy_async_all() {
 }
 
 // Untiled bulk copy of `bytes` (a multiple of 16; both addresses 16-byte aligned) from global
-// memory into this CTA's shared memory, completing on the mbarrier (no multicast).
+// memory into this CTA's shared memory, completing on the mbarrier (this CTA only).
 __device__ __forceinline__ void bulk_load(void *smem_dst, const void *gsrc, uint32_t bytes, uint64_t *bar) {
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
                  ::"r"(smem_u32(smem_dst)), "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
