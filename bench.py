@@ -317,6 +317,49 @@ def gpu_arm(args, rank, world, local_rank):
         del wq_g, y_g
         assert opq.device_error() == 0
 
+    # ---- the other bit widths of the card's configuration (3, 5, 6: 2^bits - 1 levels, codes as
+    # one bit stream per row) on the same weight: quantize, dequantize, and the SNR of each width
+    bits_out = {}
+    fused = {}
+    if not args.no_sweep:
+        wq_b = torch.empty_like(w)
+        for b_ in (3, 5, 6):
+            cb, sb, fb = opq.quantize_bits(w, b_, alpha)
+            fq = lambda: opq.quantize_bits(w, b_, alpha, out=(cb, sb, fb))
+            fd = lambda: opq.dequantize_bits(cb, sb, fb, b_, alpha, out=wq_b)
+            for f_ in (fq, fd):
+                for _ in range(3):
+                    f_()
+            tq_, _ = time_kernel(fq)
+            td_, _ = time_kernel(fd)
+            packed = N * K * b_ // 8 + N * K // 8 + 4 * N
+            bq_bytes = N * K * 2 + packed
+            bd_bytes = packed + N * K * 2
+            bits_out[str(b_)] = {
+                "quantize": {"ms": tq_, "gbs": bq_bytes / (tq_ * 1e-3) / 1e9,
+                             "frac_hbm": bq_bytes / (tq_ * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+                "dequantize": {"ms": td_, "gbs": bd_bytes / (td_ * 1e-3) / 1e9,
+                               "frac_hbm": bd_bytes / (td_ * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+                "snr_db": None}
+            opq.dequantize_bits(cb, sb, fb, b_, alpha, out=wq_b)
+            r_ = w.double()
+            bits_out[str(b_)]["snr_db"] = float(10.0 * torch.log10((r_ * r_).sum() / ((r_ - wq_b.double()) ** 2).sum()))
+            del cb, sb, fb
+        del wq_b
+        # the linear with its epilogue fused (bias + SiLU), as the layer an nn.Linear + activation
+        # becomes: same weight, activations and schedule as the step's linear
+        bias = (torch.arange(N, device=dev, dtype=torch.float32) * 1e-3 - 1.0).to(torch.bfloat16)
+        y_f = torch.empty_like(y)
+        for act in ("silu", "gelu_tanh"):
+            ff = lambda: opq.linear_fused(x, codes, signs, scales, alpha, bias=bias, act=act, out=y_f, workspace=ws)
+            for _ in range(3):
+                ff()
+            tf_, _ = time_kernel(ff)
+            f_tflops = flops / (tf_ * 1e-3) / 1e12
+            fused[act] = {"ms": tf_, "tflops": f_tflops, "frac_bf16": f_tflops / peaks["bf16_tflops"]}
+        del y_f
+        assert opq.device_error() == 0
+
     # ---- SNR context (the model card's "+7.2 dB" claim is on Z-Image weights; these are the
     # synthetic Student-t weights of the bench workload): OPQ through the library at alpha 0.73
     # and 1.0 (same 4-bit + sign + row max format), and per-row symmetric INT4 round(w/(max/7))
@@ -387,7 +430,8 @@ def gpu_arm(args, rank, world, local_rank):
         "config": {"workload": lin.name, "M": M, "N": N, "K": K, "alpha": alpha,
                    "step": "quantize W + linear x W'^T + dequantize W'", "parallelism": f"replicas{world}",
                    "l2": "flushed between timed steps (4x L2 buffer write outside the event pairs)"},
-        "kernels": kernels, "small_m": small, "grouped": grouped, "roofline": roof, "snr_db": snr,
+        "kernels": kernels, "small_m": small, "grouped": grouped, "bits": bits_out, "fused": fused,
+        "roofline": roof, "snr_db": snr,
         "e2e": {"value": whole_job_tflops(world, flops, ms_e2e), "unit": "TFLOP/s", "ms_per_step": ms_e2e,
                 "h2d_bytes_per_step": w.numel() * 2 + x.numel() * 2, "d2h_bytes_per_step": y.numel() * 2},
         "gpu_launches": launches_per_step * args.steps,
