@@ -661,10 +661,10 @@ static opq_status linear_impl(const uint16_t *x, int64_t M, int64_t K, const uin
     if (gs > 0 && (s = check_group(K, gs)) != OPQ_OK) return s;
     if (M > INT32_MAX) return OPQ_ERR_UNSUPPORTED_SHAPE;
     if (!alpha_ok(alpha)) return OPQ_ERR_INVALID_ARG;
-    if ((s = check_ptrs({x, codes, signs, gs > 0 ? (const void *)gmax : (const void *)scales, y})) != OPQ_OK)
-        return s;
     if (activation != OPQ_ACT_NONE && activation != OPQ_ACT_SILU && activation != OPQ_ACT_GELU_TANH)
         return OPQ_ERR_INVALID_ARG;
+    if ((s = check_ptrs({x, codes, signs, gs > 0 ? (const void *)gmax : (const void *)scales, y})) != OPQ_OK)
+        return s;
     if (bias && (s = check_ptrs({bias})) != OPQ_OK) return s;
     const Plan plan = make_plan(M, N, K);
     if (plan.ws_bytes > 0) {

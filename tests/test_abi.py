@@ -89,6 +89,47 @@ def test_dequantize_and_linear_argument_errors(lib):
     assert L(x, 2, 32, c, s, sc, 4, 0.73, y, None, 0, None) == 6
 
 
+def test_grouped_fused_bits_alpha_argument_errors(lib):
+    keep = []
+    def b(n, off=0):
+        a, p = _buf(n, off)
+        keep.append(a)
+        return p
+    w, c, s, g, sc, out = b(256 * 2), b(64), b(16), b(64), b(16), b(512)
+    # group-wise: listed sizes only, dividing K
+    assert lib.opq_quantize_grouped(w, 4, 96, 96, 48, 0.73, c, s, g, None) == 1
+    assert lib.opq_quantize_grouped(w, 4, 96, 96, 64, 0.73, c, s, g, None) == 2
+    assert lib.opq_quantize_grouped(w, 4, 96, 96, 32, 0.73, c, s, g, None) == 6     # host memory
+    assert lib.opq_dequantize_grouped(c, s, g, 4, 96, 128, 0.73, out, None) == 2
+    sz = ctypes.c_size_t(0)
+    assert lib.opq_linear_grouped_workspace_size(4, 4, 96, 48, ctypes.byref(sz)) == 1
+    # fused epilogue: activation codes 0..2 only, checked before the pointers
+    x, y = b(4096), b(4096)
+    assert lib.opq_linear_fused(x, 2, 32, c, s, sc, 4, 0.73, None, 3, y, None, 0, None) == 1
+    assert lib.opq_linear_fused(x, 2, 32, c, s, sc, 4, 0.73, None, -1, y, None, 0, None) == 1
+    assert lib.opq_linear_fused(x, 2, 32, c, s, sc, 4, 0.73, None, 1, y, None, 0, None) == 6
+    assert lib.opq_linear_grouped_fused(x, 2, 32, c, s, g, 4, 48, 0.73, None, 1, y, None, 0, None) == 1
+    # bit widths 3..6
+    for bits in (0, 2, 7, 8):
+        assert lib.opq_quantize_bits(w, 4, 32, 32, bits, 0.73, c, s, sc, None) == 1
+        assert lib.opq_dequantize_bits(c, s, sc, 4, 32, bits, 0.73, out, None) == 1
+    assert lib.opq_quantize_bits(w, 4, 48, 48, 3, 0.73, c, s, sc, None) == 2
+    assert lib.opq_quantize_bits(w, 4, 32, 36, 3, 0.73, c, s, sc, None) == 1       # ldw % 8 != 0
+    assert lib.opq_quantize_bits(w, 4, 32, 32, 5, 0.73, c, s, sc, None) == 6
+    assert lib.opq_dequantize_bits(c, s, sc, 4, 32, 6, float("nan"), out, None) == 1
+    assert lib.opq_dequantize_bits(c, s, sc, 4, 32, 6, 0.73, out, None) == 6
+    # alpha search: at least one candidate, every candidate finite and > 0
+    alphas = (ctypes.c_float * 2)(0.5, 0.73)
+    snr = (ctypes.c_double * 2)()
+    best = ctypes.c_float()
+    ab = lib.opq_alpha_search
+    assert ab(w, 4, 32, 32, 0, alphas, 0, snr, ctypes.byref(best), None, 0, None) == 1
+    assert ab(w, 4, 32, 32, 0, (ctypes.c_float * 1)(-1.0), 1, snr, ctypes.byref(best), None, 0, None) == 1
+    assert ab(w, 4, 32, 32, 48, alphas, 2, snr, ctypes.byref(best), None, 0, None) == 1
+    assert ab(w, 4, 32, 32, 0, alphas, 2, None, ctypes.byref(best), None, 0, None) == 1
+    assert ab(w, 4, 32, 32, 0, alphas, 2, snr, ctypes.byref(best), None, 0, None) == 6
+
+
 def test_plan_and_workspace_host_logic(lib):
     # small M: stream-K over (128-row weight tile, load group) units on at most 148 CTAs; a load
     # group is 4 (16-row tiles), 2 (32- and 64-row tiles) or 1 consecutive 128-K blocks, the
