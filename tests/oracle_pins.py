@@ -289,9 +289,47 @@ def pin_snr_ordering(orc):
     assert snr[1.0] > snr["int4"] + 2.0, snr
 
 
+def pin_snr_closed_form(orc):
+    """SNR = 10 log10(sum w^2 / sum (w - w')^2) on hand-worked pairs (the model card's
+    "+7.2 dB" is a ratio of signal to quantization-error power in decibels):
+    w = [1, 1], w' = [1, 0.5]: 10 log10(2 / 0.25) = 10 log10 8;
+    w = [2, -1], w' = [1.5, -1]: 10 log10(5 / 0.25) = 10 log10 20 (the values differ from
+    their absolute values and squares, so an unsquared term changes the result);
+    an exact reconstruction has no error power: +inf."""
+    w = bf16_bits([1.0, 1.0])
+    got = orc.snr_db(w, np.array([1.0, 0.5]))
+    assert abs(got - 10.0 * np.log10(8.0)) < 1e-12, got
+    assert abs(got - 9.030899869919435) < 1e-12, got
+    w = bf16_bits([2.0, -1.0])
+    got = orc.snr_db(w, np.array([1.5, -1.0]))
+    assert abs(got - 13.010299956639813) < 1e-12, got
+    got = orc.snr_db(bf16_bits([0.25, -3.0, 0.0]), np.array([0.25, -3.0, 0.0]))
+    assert got == float("inf"), got
+
+
+def pin_uniform_int4_worked(orc):
+    """The symmetric INT4 baseline clip(RNE(w / (max/7)), -7, 7) * max/7 on hand-worked rows.
+    Row 0 has max 0.4375 = 7/16, so the step is exactly 1/16 and w/step is exact:
+    0.03125 -> 0.5 -> 0 and 0.15625 -> 2.5 -> 2 (ties to even), 0.09375 -> 1.5 -> 2,
+    -0.09375 -> -2, 0.1875 -> 3, the max -> 7 (reconstructs to itself).
+    Row 1 has its max on a negative weight: -0.4375 -> -7. Row 2 is all zero."""
+    K = 8
+    rows = [[0.03125, 0.15625, 0.09375, -0.09375, 0.1875, 0.4375, 0.0, -0.03125],
+            [-0.4375, 0.25, 0.3125, -0.21875, 0.0, 0.0625, -0.0625, 0.125],
+            [0.0] * K]
+    w = np.stack([bf16_bits(r) for r in rows])
+    want_q = np.array([[0, 2, 2, -2, 3, 7, 0, 0],
+                       [-7, 4, 5, -4, 0, 1, -1, 2],   # 0.21875 -> 3.5 -> 4 (even)
+                       [0] * K], np.float64)
+    want = want_q * np.array([[0.0625], [0.0625], [0.0]])
+    got = orc.uniform_int4(w)
+    assert np.array_equal(got, want), (got, want)
+
+
 PINS = [pin_golden_fixtures, pin_alpha1_exact_rational, pin_max_zero_monotone,
         pin_bruteforce_nearest_level, pin_threshold_identity, pin_lut_decimal,
-        pin_roundtrip_idempotent, pin_linear, pin_bf16_rounding, pin_snr_ordering]
+        pin_roundtrip_idempotent, pin_linear, pin_bf16_rounding, pin_snr_ordering,
+        pin_snr_closed_form, pin_uniform_int4_worked]
 
 
 # ------------------------------------------------- group-wise variant pins --

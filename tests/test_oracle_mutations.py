@@ -53,6 +53,14 @@ MUTANTS = [
     ("gelu_square", "0.044715 * v * v * v", "0.044715 * v * v"),
     ("bias_dropped", "double v = y[m * N + n] + (bias ? bf16_value(bias[n]) : 0.0);", "double v = y[m * N + n];"),
     ("fp16_subnormal_floor", "if (qexp < -24)\n        qexp = -24;", "if (qexp < -25)\n        qexp = -25;"),
+    # SNR and the symmetric INT4 baseline (quality context)
+    ("snr_amplitude_decibels", "return 10.0 * log10(sig / err);", "return 20.0 * log10(sig / err);"),
+    ("snr_ratio_inverted", "return 10.0 * log10(sig / err);", "return 10.0 * log10(err / sig);"),
+    ("snr_error_unsquared", "err += d * d;", "err += fabs(d);"),
+    ("snr_signal_unsquared", "sig += a * a;", "sig += fabs(a);"),
+    ("int4_step_over_eight", "nearbyint(v / (mx / 7.0));", "nearbyint(v / (mx / 8.0));"),
+    ("int4_round_half_up", "nearbyint(v / (mx / 7.0));", "floor(v / (mx / 7.0) + 0.5);"),
+    ("int4_reconstruction_unscaled", "w_rec[n * K + k] = q * mx / 7.0;", "w_rec[n * K + k] = q / 7.0;"),
 ]
 
 
