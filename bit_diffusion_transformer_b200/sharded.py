@@ -29,6 +29,14 @@ def shard_range(n_rows: int, rank: int, world: int):
     return lo, lo + base + (1 if rank < rem else 0)
 
 
+def shard_layers(n_layers: int, rank: int, world: int):
+    """Layers of ``rank`` in a whole-model quantize pass: round-robin, so that every rank gets
+    the same mix of matrix shapes (layers are independent under OPQ)."""
+    if world < 1 or not 0 <= rank < world:
+        raise ValueError(f"rank {rank} out of range for world {world}")
+    return list(range(rank, n_layers, world))
+
+
 def shard_width(n_rows: int, world: int) -> int:
     """Width of the gathered blocks: the largest shard."""
     return -(-n_rows // world)

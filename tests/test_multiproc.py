@@ -28,7 +28,7 @@ def _rank_main(rank, world, port, out_dir):
     import sys
     sys.path.insert(0, ROOT)
     import bench
-    import workloads
+    from bit_diffusion_transformer_b200 import sharded
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
@@ -36,8 +36,8 @@ def _rank_main(rank, world, port, out_dir):
         ms = bench.max_over_ranks(1.5 + rank, world, "cpu")
         value = bench.whole_job_tflops(world, 90.6e9, ms)
         # sharding: every row / layer exactly once over the ranks
-        rows = workloads.shard_rows(11520, rank, world)
-        layers = workloads.shard_layers(210, rank, world)
+        rows = sharded.shard_range(11520, rank, world)
+        layers = sharded.shard_layers(210, rank, world)
         gathered = [None] * world
         dist.all_gather_object(gathered, (rows, layers))
         dist.barrier()

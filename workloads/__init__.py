@@ -171,16 +171,3 @@ class WholeModel:
     @property
     def weights(self) -> int:
         return sum(l.N * l.K for l in self.layers)
-
-
-def shard_rows(n_rows: int, rank: int, world: int):
-    """Contiguous row range [lo, hi) of rank ``rank`` out of ``world`` (rows are independent)."""
-    base, rem = divmod(n_rows, world)
-    lo = rank * base + min(rank, rem)
-    hi = lo + base + (1 if rank < rem else 0)
-    return lo, hi
-
-
-def shard_layers(n_layers: int, rank: int, world: int):
-    """Round-robin layer assignment for the whole-model pass."""
-    return list(range(rank, n_layers, world))
