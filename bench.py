@@ -1,11 +1,16 @@
 """Benchmark of the OPQ hot path on B200: quantize -> linear -> dequantize.
 
-One step = opq_quantize(W) + opq_linear(x, W') + opq_dequantize(W') on the DiT
-attention-projection workload (x 3072x3840 N(0,1), W 3840x3840 Student-t(4),
-std 0.02, 0.1% outlier rows, alpha = 0.73), inputs resident in HBM. The line's
-value is the step's linear TFLOP/s (2 M N K per step over the step time,
-summed over ranks); per-kernel figures, the small-M weight-streaming sweep
-and the roofline of the dominant kernel are reported beside it.
+Headline workload: the whole-model pass of a synthetic diffusion transformer,
+30 blocks x (4 attention matrices 3840x3840, two FFN up-projections 10240x3840,
+one down-projection 3840x10240) = 210 matrices, 5.31 G weights (10.62 GB bf16,
+Student-t(4), std 0.02, alpha = 0.73), activations 3072 x K N(0,1). One step =
+quantize all 210 matrices, opq_linear at M = 3072 on every layer, dequantize
+all 210; inputs resident in HBM and 84x larger than L2. The line's value is the
+step's linear TFLOP/s (2 M N K summed over the layers, over the step time,
+summed over ranks); quantize-all GB/s, linear TFLOP/s per shape class and the
+roofline of the dominant kernel are reported beside it, with the FFN pair at
+three alphas, the attention projection, the small-M weight-streaming sweep
+and the library's other formats as extras.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl opq|reference]
 
@@ -19,6 +24,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -160,6 +166,104 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+
+
+# --------------------------------------------------------------------------- byte / flop counts
+def quant_bytes(N, K):
+    """quantize: read W (2 B), write codes (K/2 B) + signs (K/8 B) per row, and the fp32 scales."""
+    return N * K * 2 + N * K // 8 * 5 + 4 * N
+
+
+def dequant_bytes(N, K):
+    return N * K // 8 * 5 + 4 * N + N * K * 2
+
+
+def linear_bytes(M, N, K):
+    return N * K * 5 // 8 + 4 * N + 2 * M * K + 2 * M * N
+
+
+# shape classes of the whole-model pass: (name, N, K)
+WM_CLASSES = (("attn_3840x3840", 3840, 3840), ("ffn_up_10240x3840", 10240, 3840),
+              ("ffn_down_3840x10240", 3840, 10240))
+
+
+def wm_class(N, K):
+    for name, n, k in WM_CLASSES:
+        if (n, k) == (N, K):
+            return name
+    raise ValueError((N, K))
+
+
+class WholeModelState:
+    """Device buffers of the whole-model pass: every layer's W, packed planes and W' are
+    views into one allocation per tensor kind; one activation tensor per K and one output
+    per N (every layer runs at M = 3072)."""
+
+    def __init__(self, dev, opq, workloads, torch):
+        self.model = workloads.WholeModel()
+        self.M, self.alpha = self.model.M, self.model.alpha
+        total = self.model.weights
+        rows = sum(l.N for l in self.model.layers)
+        bf16 = torch.bfloat16
+        self.W = torch.empty((total,), dtype=bf16, device=dev)
+        self.Wq = torch.empty((total,), dtype=bf16, device=dev)
+        self.codes = torch.empty((total // 8,), dtype=torch.int32, device=dev)
+        self.signs = torch.empty((total // 32,), dtype=torch.int32, device=dev)
+        self.scales = torch.empty((rows,), dtype=torch.float32, device=dev)
+        self.layers = []
+        off = roff = 0
+        for l in self.model.layers:
+            n, k = l.N, l.K
+            L = {"name": l.name, "N": n, "K": k, "cls": wm_class(n, k), "off": off,
+                 "w": self.W[off:off + n * k].view(n, k), "wq": self.Wq[off:off + n * k].view(n, k),
+                 "c": self.codes[off // 8:(off + n * k) // 8].view(n, k // 8),
+                 "s": self.signs[off // 32:(off + n * k) // 32].view(n, k // 32),
+                 "sc": self.scales[roff:roff + n]}
+            # each layer's draw comes from its own seeded generator on the device
+            L["w"].copy_(l.make_weights(dev))
+            self.layers.append(L)
+            off += n * k
+            roff += n
+        first = {}
+        for l in self.model.layers:
+            first.setdefault(l.K, l)
+        self.x = {k: l.make_x(dev) for k, l in first.items()}
+        self.y = {n: torch.empty((self.M, n), dtype=bf16, device=dev) for n in {l.N for l in self.model.layers}}
+        need = max(opq.workspace_size(self.M, l.N, l.K) for l in self.model.layers)
+        self.ws = torch.zeros((max(need, 16),), dtype=torch.uint8, device=dev)
+        self.by_class = {c[0]: [L for L in self.layers if L["cls"] == c[0]] for c in WM_CLASSES}
+
+    def phase(self, opq, what, cls):
+        a, M = self.alpha, self.M
+        for L in self.by_class[cls]:
+            if what == "quantize":
+                opq.quantize(L["w"], a, out=(L["c"], L["s"], L["sc"]))
+            elif what == "linear":
+                opq.linear(self.x[L["K"]], L["c"], L["s"], L["sc"], a, out=self.y[L["N"]], workspace=self.ws)
+            else:
+                opq.dequantize(L["c"], L["s"], L["sc"], a, out=L["wq"])
+
+    def counts(self, cls):
+        Ls = self.by_class[cls]
+        return {"matrices": len(Ls),
+                "quantize_bytes": sum(quant_bytes(L["N"], L["K"]) for L in Ls),
+                "dequantize_bytes": sum(dequant_bytes(L["N"], L["K"]) for L in Ls),
+                "linear_flops": sum(2.0 * self.M * L["N"] * L["K"] for L in Ls),
+                "linear_bytes": sum(linear_bytes(self.M, L["N"], L["K"]) for L in Ls)}
+
+
+PHASES = ("quantize", "linear", "dequantize")
+
+
+def capture_graph(torch, fn):
+    """One CUDA graph of the launches `fn` enqueues (the library's calls are plain kernel
+    launches on the current stream; nothing is allocated inside)."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, capture_error_mode="relaxed"):
+        fn()
+    return g
+
+
 # --------------------------------------------------------------------------- GPU arm
 def gpu_arm(args, rank, world, local_rank):
     import torch
@@ -171,71 +275,21 @@ def gpu_arm(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     opq.load()
-    lin = workloads.dit_attn_proj()
-    M, N, K, alpha = lin.M, lin.N, lin.K, lin.alpha
-    x, w = lin.make(dev)
-    codes = torch.empty((N, K // 8), dtype=torch.int32, device=dev)
-    signs = torch.empty((N, K // 32), dtype=torch.int32, device=dev)
-    scales = torch.empty((N,), dtype=torch.float32, device=dev)
-    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-    wq = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
-    ws_bytes = opq.workspace_size(M, N, K)
-    ws = torch.zeros((max(ws_bytes, 16),), dtype=torch.uint8, device=dev)
+    peaks, peak_src = load_peaks()
+    stream = torch.cuda.current_stream(dev)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush = torch.empty((4 * max(l2, 64 << 20),), dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream(dev)
-
-    def step(ev=None):
-        # ev: optional 4 events bracketing the three launches (timed region only)
-        if ev is not None:
-            ev[0].record(stream)
-        opq.quantize(w, alpha, out=(codes, signs, scales))
-        if ev is not None:
-            ev[1].record(stream)
-        opq.linear(x, codes, signs, scales, alpha, out=y, workspace=ws)
-        if ev is not None:
-            ev[2].record(stream)
-        opq.dequantize(codes, signs, scales, alpha, out=wq)
-        if ev is not None:
-            ev[3].record(stream)
-
-    launches_per_step = 1 + opq.plan(M, N, K)[2] + 1
 
     def barrier():
         if world > 1:
             dist.barrier()
 
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    assert opq.device_error() == 0
-
-    # ---- timed region: K steps, L2 flushed between steps (outside the event pairs); the
-    # events bracketing each launch give the per-kernel durations of the same region
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(local_rank) as clocks:
-        clocks.mark(True)
-        for i in range(args.steps):
-            flush.zero_()
-            step(evs[i])
-        torch.cuda.synchronize()
-        clocks.mark(False)
-    barrier()
-    per_step = [e[0].elapsed_time(e[3]) for e in evs]
-    live = {name: statistics.fmean(e[a].elapsed_time(e[b]) for e in evs)
-            for name, a, b in (("quantize", 0, 1), ("linear", 1, 2), ("dequantize", 2, 3))}
-    ms_step = max_over_ranks(sum(per_step) / len(per_step), world, dev)
-    assert opq.device_error() == 0
-    flops = 2.0 * M * N * K
-    value = whole_job_tflops(world, flops, ms_step)
-
-    # ---- per-kernel timings (events on the launching stream, L2 flushed before each)
-    def time_kernel(fn, reps=20):
+    def time_kernel(fn, reps=20, flush_l2=True):
+        """Median duration of one call, events on the launching stream, L2 flushed before each."""
         ts = []
         for _ in range(reps):
-            flush.zero_()
+            if flush_l2:
+                flush.zero_()
             a = torch.cuda.Event(enable_timing=True)
             b = torch.cuda.Event(enable_timing=True)
             a.record(stream)
@@ -243,129 +297,352 @@ def gpu_arm(args, rank, world, local_rank):
             b.record(stream)
             b.synchronize()
             ts.append(a.elapsed_time(b))
-        return statistics.median(ts), ts
+        return statistics.median(ts)
 
-    peaks, peak_src = load_peaks()
-    # mean launch durations inside the timed region (each launch starts with a flushed L2)
-    t_q, t_l, t_d = live["quantize"], live["linear"], live["dequantize"]
-    q_bytes = N * K * 2 + N * K // 8 * 5 + 4 * N      # read W, write codes (K/2 B) + signs (K/8 B) + scales
-    d_bytes = N * K // 8 * 5 + 4 * N + N * K * 2
-    l_bytes = N * K * 5 // 8 + 4 * N + 2 * M * K + 2 * M * N
-    linear_tflops = flops / (t_l * 1e-3) / 1e12
-    kernels = {
-        "quantize": {"ms": t_q, "gbs": q_bytes / (t_q * 1e-3) / 1e9,
-                     "frac_hbm": q_bytes / (t_q * 1e-3) / 1e9 / peaks["hbm_gbs"]},
-        "linear": {"ms": t_l, "tflops": linear_tflops, "frac_bf16": linear_tflops / peaks["bf16_tflops"],
-                   "path": opq.plan(M, N, K)[0]},
-        "dequantize": {"ms": t_d, "gbs": d_bytes / (t_d * 1e-3) / 1e9,
-                       "frac_hbm": d_bytes / (t_d * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+    # ---------------------------------------------------------------- the whole-model step
+    S = WholeModelState(dev, opq, workloads, torch)
+    M, alpha = S.M, S.alpha
+    cls_names = [c[0] for c in WM_CLASSES]
+    for what in PHASES:                      # eager pass: kernel attributes, TMA encoder lookup
+        for c in cls_names:
+            S.phase(opq, what, c)
+    torch.cuda.synchronize()
+    assert opq.device_error() == 0
+    graphs = {(what, c): capture_graph(torch, lambda w_=what, c_=c: S.phase(opq, w_, c_))
+              for what in PHASES for c in cls_names}
+    order = [(what, c) for what in PHASES for c in cls_names]
+
+    def step(ev=None):
+        for i, key in enumerate(order):
+            if ev is not None:
+                ev[i].record(stream)
+            graphs[key].replay()
+        if ev is not None:
+            ev[len(order)].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert opq.device_error() == 0
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(order) + 1)] for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clocks:
+        clocks.mark(True)
+        for i in range(args.steps):
+            step(evs[i])
+        torch.cuda.synchronize()
+        clocks.mark(False)
+    barrier()
+    assert opq.device_error() == 0
+    per_step = [e[0].elapsed_time(e[-1]) for e in evs]
+    seg = {key: statistics.fmean(e[i].elapsed_time(e[i + 1]) for e in evs) for i, key in enumerate(order)}
+    ms_step = max_over_ranks(statistics.fmean(per_step), world, dev)
+    cnt = {c: S.counts(c) for c in cls_names}
+    flops = sum(cnt[c]["linear_flops"] for c in cls_names)
+    value = whole_job_tflops(world, flops, ms_step)
+    hbm, bf16 = peaks["hbm_gbs"], peaks["bf16_tflops"]
+    bf16_sus = peaks.get("bf16_tflops_sustained", bf16)
+
+    def gbs_entry(ms, nbytes, extra=None):
+        g = nbytes / (ms * 1e-3) / 1e9
+        d = {"ms": ms, "gbs": g, "frac_hbm": g / hbm, "bytes": nbytes}
+        d.update(extra or {})
+        return d
+
+    def tf_entry(ms, fl, extra=None):
+        t = fl / (ms * 1e-3) / 1e12
+        d = {"ms": ms, "tflops": t, "frac_bf16": t / bf16, "frac_bf16_sustained": t / bf16_sus}
+        d.update(extra or {})
+        return d
+
+    kernels = {}
+    for what, key_b in (("quantize", "quantize_bytes"), ("dequantize", "dequantize_bytes")):
+        ms = sum(seg[(what, c)] for c in cls_names)
+        kernels[f"{what}_all"] = gbs_entry(ms, sum(cnt[c][key_b] for c in cls_names), {
+            "matrices": len(S.layers),
+            "by_class": {c: gbs_entry(seg[(what, c)], cnt[c][key_b], {"matrices": cnt[c]["matrices"]})
+                         for c in cls_names}})
+    ms_lin = sum(seg[("linear", c)] for c in cls_names)
+    kernels["linear_all"] = tf_entry(ms_lin, flops, {
+        "layers": len(S.layers), "M": M,
+        "by_class": {c: tf_entry(seg[("linear", c)], cnt[c]["linear_flops"],
+                                 {"layers": cnt[c]["matrices"], "plan": list(opq.plan(M, *[(n, k) for nm, n, k in WM_CLASSES if nm == c][0]))})
+                     for c in cls_names}})
+    launches_per_step = 3 * len(S.layers)
+    linear_tflops = kernels["linear_all"]["tflops"]
+
+    # ---------------------------------------------------------------- e2e: host buffers
+    # Every step copies all 210 weights and both activation tensors from host memory, runs
+    # the three phases through the public calls and copies every layer's y back to the host.
+    e2e = None
+    if not args.no_e2e:
+        total_bytes = S.W.numel() * 2
+        w_host = torch.empty((S.W.numel(),), dtype=torch.bfloat16)
+        w_host.copy_(S.W)
+        cudart = torch.cuda.cudart()
+        reg = cudart.cudaHostRegister(w_host.data_ptr(), total_bytes, 0)
+        registered = int(reg) == 0
+        x_host = {k: v.cpu().pin_memory() for k, v in S.x.items()}
+        y_host = {n: torch.empty(v.shape, dtype=v.dtype).pin_memory() for n, v in S.y.items()}
+
+        def e2e_step():
+            for k in S.x:
+                S.x[k].copy_(x_host[k], non_blocking=True)
+            for L in S.layers:
+                n, k = L["N"], L["K"]
+                L["w"].copy_(w_host[L["off"]:L["off"] + n * k].view(n, k), non_blocking=True)
+            for L in S.layers:
+                opq.quantize(L["w"], alpha, out=(L["c"], L["s"], L["sc"]))
+            for L in S.layers:
+                y = S.y[L["N"]]
+                opq.linear(S.x[L["K"]], L["c"], L["s"], L["sc"], alpha, out=y, workspace=S.ws)
+                y_host[L["N"]].copy_(y, non_blocking=True)
+            for L in S.layers:
+                opq.dequantize(L["c"], L["s"], L["sc"], alpha, out=L["wq"])
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e_steps = max(1, min(args.steps, 3))
+        ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ea.record(stream)
+        for _ in range(e_steps):
+            e2e_step()
+        eb.record(stream)
+        eb.synchronize()
+        ms_e2e = max_over_ranks(ea.elapsed_time(eb) / e_steps, world, dev)
+        barrier()
+        assert opq.device_error() == 0
+        h2d = total_bytes + sum(v.numel() * 2 for v in S.x.values())
+        d2h = sum(M * L["N"] * 2 for L in S.layers)
+        e2e = {"value": whole_job_tflops(world, flops, ms_e2e), "unit": "TFLOP/s", "ms_per_step": ms_e2e,
+               "steps": e_steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "host_weights": "registered (page-locked) host memory" if registered else "pageable host memory",
+               "copies": "210 weight H2D + 2 activation H2D + 210 y D2H per step"}
+        if registered:
+            cudart.cudaHostUnregister(w_host.data_ptr())
+        del w_host
+    traffic = recorded_traffic("wide_kernel_whole_model")
+    roof = {"bound": "tensor", "kernel": "opqk_wide::wide_kernel<256, 0>", "achieved": linear_tflops,
+            "peak": bf16, "unit": "TFLOP/s", "frac": linear_tflops / bf16,
+            "frac_of_sustained_peak": linear_tflops / bf16_sus, "traffic": traffic,
+            "algorithmic_flops_per_launch": flops / len(S.layers),
+            "algorithmic_bytes_per_launch": sum(cnt[c]["linear_bytes"] for c in cls_names) / len(S.layers),
+            "launch_ms": ms_lin / len(S.layers), "launches": len(S.layers),
+            "peak_source": f"bf16 dense burst, {peak_src} (frac_of_sustained_peak: the power-capped loop)",
+            "note": "achieved = the 210 layers' 2 M N K over their summed launch durations (the mean "
+                    "launch of the mix); traffic = ncu DRAM bytes per launch averaged over the mix"}
+    # free the whole-model buffers before the extras
+    whole = {"ms_per_step": ms_step, "per_step_ms": {f"{w}:{c}": seg[(w, c)] for (w, c) in order}}
+    del graphs, S
+    torch.cuda.empty_cache()
+
+    extras = {}
+    if not args.no_sweep:
+        extras = gpu_extras(args, opq, workloads, torch, dev, peaks, time_kernel, flush)
+
+    out = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded Student-t(4) weights std 0.02 drawn per layer on the device, N(0,1) activations)",
+        "config": {"workload": "dit_whole_model_30blocks_210layers_m3072", "blocks": 30, "layers": 210,
+                   "weights": 5308416000, "M": M, "alpha": alpha,
+                   "step": "quantize all 210 W + linear x W'^T on every layer (M 3072) + dequantize all 210",
+                   "parallelism": f"replicas{world}",
+                   "l2": "inputs larger than L2 (10.62 GB of weights per step against a 126 MB L2); no flush",
+                   "launch": "each phase and shape class is one CUDA graph of the library's launches"},
+        "kernels": kernels, "whole_model": whole, "roofline": roof,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks.summary(),
+        "peaks": peaks,
     }
+    if e2e is not None:
+        out["e2e"] = e2e
+    out.update(extras)
+    return out
 
-    # ---- weight-streaming sweep (fused-QKV 11520x3840, M in {1, 16, 64, 256})
+
+def gpu_extras(args, opq, workloads, torch, dev, peaks, time_kernel, flush):
+    """The FFN pair at three alphas, the attention projection step, the small-M weight
+    stream, the group-wise format, other bit widths, the fused epilogue, SNR context."""
+    hbm, bf16 = peaks["hbm_gbs"], peaks["bf16_tflops"]
+    stream = torch.cuda.current_stream(dev)
+    out = {}
+
+    # ---- the DiT FFN pair: x 4096x3840 through W1 10240x3840, x' 4096x10240 through W2
+    # 3840x10240, at alpha 0.45, 0.73 and 1.0 (the draws do not depend on alpha)
+    up0, down0 = workloads.dit_ffn_pair(workloads.ALPHA)
+    xu, wu = up0.make(dev)
+    xd, wd = down0.make(dev)
+    yu = torch.empty((up0.M, up0.N), dtype=torch.bfloat16, device=dev)
+    yd = torch.empty((down0.M, down0.N), dtype=torch.bfloat16, device=dev)
+    wsu = torch.zeros((max(opq.workspace_size(up0.M, up0.N, up0.K), 16),), dtype=torch.uint8, device=dev)
+    wsd = torch.zeros((max(opq.workspace_size(down0.M, down0.N, down0.K), 16),), dtype=torch.uint8, device=dev)
+    ffn = {}
+    for a in (0.45, 0.73, 1.0):
+        pu = opq.quantize(wu, a)
+        pd = opq.quantize(wd, a)
+        fu = lambda: opq.linear(xu, *pu, a, out=yu, workspace=wsu)
+        fd = lambda: opq.linear(xd, *pd, a, out=yd, workspace=wsd)
+        fq = lambda: opq.quantize(wu, a, out=pu)
+        for f_ in (fu, fd, fq):
+            for _ in range(3):
+                f_()
+        tu, td, tq = time_kernel(fu, 10), time_kernel(fd, 10), time_kernel(fq, 10)
+        flu, fld = 2.0 * up0.M * up0.N * up0.K, 2.0 * down0.M * down0.N * down0.K
+        qb = quant_bytes(up0.N, up0.K)
+        ffn[f"{a:g}"] = {
+            "up": {"ms": tu, "tflops": flu / tu / 1e9, "frac_bf16": flu / tu / 1e9 / bf16,
+                   "plan": list(opq.plan(up0.M, up0.N, up0.K))},
+            "down": {"ms": td, "tflops": fld / td / 1e9, "frac_bf16": fld / td / 1e9 / bf16,
+                     "plan": list(opq.plan(down0.M, down0.N, down0.K))},
+            "pair": {"ms": tu + td, "tflops": (flu + fld) / (tu + td) / 1e9,
+                     "frac_bf16": (flu + fld) / (tu + td) / 1e9 / bf16},
+            "quantize_w1": {"ms": tq, "gbs": qb / tq / 1e6, "frac_hbm": qb / tq / 1e6 / hbm}}
+        del pu, pd
+    assert opq.device_error() == 0
+    out["ffn_pair"] = {"workload": "dit_ffn_pair x 4096x3840 @ W1 10240x3840, x' 4096x10240 @ W2 3840x10240",
+                       "l2": "flushed before each launch", "by_alpha": ffn}
+    del xu, wu, xd, wd, yu, yd, wsu, wsd
+
+    # ---- the attention projection step (x 3072x3840, W 3840x3840 with outlier rows)
+    lin = workloads.dit_attn_proj()
+    M, N, K, alpha = lin.M, lin.N, lin.K, lin.alpha
+    x, w = lin.make(dev)
+    codes, signs, scales = opq.quantize(w, alpha)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    wq = torch.empty_like(w)
+    ws = torch.zeros((max(opq.workspace_size(M, N, K), 16),), dtype=torch.uint8, device=dev)
+    fq = lambda: opq.quantize(w, alpha, out=(codes, signs, scales))
+    fl = lambda: opq.linear(x, codes, signs, scales, alpha, out=y, workspace=ws)
+    fdq = lambda: opq.dequantize(codes, signs, scales, alpha, out=wq)
+    for f_ in (fq, fl, fdq):
+        for _ in range(3):
+            f_()
+    t_q, t_l, t_d = time_kernel(fq, 50), time_kernel(fl, 50), time_kernel(fdq, 50)
+    flops = 2.0 * M * N * K
+    out["attn_proj"] = {
+        "workload": lin.name, "l2": "flushed before each launch",
+        "quantize": {"ms": t_q, "gbs": quant_bytes(N, K) / t_q / 1e6, "frac_hbm": quant_bytes(N, K) / t_q / 1e6 / hbm},
+        "linear": {"ms": t_l, "tflops": flops / t_l / 1e9, "frac_bf16": flops / t_l / 1e9 / bf16,
+                   "plan": list(opq.plan(M, N, K))},
+        "dequantize": {"ms": t_d, "gbs": dequant_bytes(N, K) / t_d / 1e6,
+                       "frac_hbm": dequant_bytes(N, K) / t_d / 1e6 / hbm}}
+
+    # ---- weight-streaming sweep: fused-QKV W 11520x3840, M in {1, 16, 64, 256}. The launches
+    # run back to back (one CUDA graph) over rotating copies of the packed weight that together
+    # hold more than 4x L2, so every launch streams its weight from HBM and the per-launch
+    # time carries no launch or event overhead; a single flushed launch is reported beside it.
+    qkv = workloads.small_m(1)
+    wqkv = qkv.make_weights(dev)
+    pq = opq.quantize(wqkv, alpha)
+    wbytes = qkv.N * qkv.K * 5 // 8 + 4 * qkv.N
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    ncopy = int(math.ceil(4 * l2 / wbytes)) + 1
+    copies = [tuple(t.clone() for t in pq) for _ in range(ncopy)]
     small = {}
-    if not args.no_sweep:
-        qkv = workloads.small_m(1)
-        wqkv = qkv.make_weights(dev)
-        pq = opq.quantize(wqkv, alpha)
-        for m in workloads.SMALL_M_SWEEP:
-            xm = workloads.small_m(m).make_x(dev)
-            ym = torch.empty((m, qkv.N), dtype=torch.bfloat16, device=dev)
-            wsm = torch.zeros((max(opq.workspace_size(m, qkv.N, qkv.K), 16),), dtype=torch.uint8, device=dev)
-            fn = lambda: opq.linear(xm, *pq, alpha, out=ym, workspace=wsm)
-            for _ in range(3):
-                fn()
-            tm, _ = time_kernel(fn, reps=30)
-            wbytes = qkv.N * qkv.K * 5 // 8 + 4 * qkv.N
-            abytes = wbytes + 2 * m * qkv.K + 2 * m * qkv.N
-            fl = 2.0 * m * qkv.N * qkv.K
-            small[str(m)] = {"us": tm * 1e3, "weight_gbs": wbytes / (tm * 1e-3) / 1e9,
-                             "bytes_gbs": abytes / (tm * 1e-3) / 1e9,
-                             "frac_hbm": abytes / (tm * 1e-3) / 1e9 / peaks["hbm_gbs"],
-                             "tflops": fl / (tm * 1e-3) / 1e12, "plan": list(opq.plan(m, qkv.N, qkv.K))}
-        del wqkv, pq
-        assert opq.device_error() == 0
+    for m in workloads.SMALL_M_SWEEP:
+        xm = workloads.small_m(m).make_x(dev)
+        ym = torch.empty((m, qkv.N), dtype=torch.bfloat16, device=dev)
+        wsm = torch.zeros((max(opq.workspace_size(m, qkv.N, qkv.K), 16),), dtype=torch.uint8, device=dev)
+        reps = 2 * ncopy
 
-    # ---- the group-wise format (the model card's own storage: one float16 max per GS weights)
-    # on the same weight and activations: quantize, linear, dequantize at GS = 128 and 32
+        def run_all(xm=xm, ym=ym, wsm=wsm):
+            for r in range(reps):
+                opq.linear(xm, *copies[r % ncopy], alpha, out=ym, workspace=wsm)
+
+        run_all()
+        torch.cuda.synchronize()
+        g = capture_graph(torch, run_all)
+        for _ in range(2):
+            g.replay()
+        tg = time_kernel(g.replay, 10, flush_l2=False) / reps
+        single = time_kernel(lambda: opq.linear(xm, *pq, alpha, out=ym, workspace=wsm), 20)
+        abytes = wbytes + 2 * m * qkv.K + 2 * m * qkv.N
+        fl_ = 2.0 * m * qkv.N * qkv.K
+        small[str(m)] = {"us": tg * 1e3, "weight_gbs": wbytes / tg / 1e6, "bytes_gbs": abytes / tg / 1e6,
+                         "frac_hbm": abytes / tg / 1e6 / hbm, "tflops": fl_ / tg / 1e9,
+                         "frac_bf16": fl_ / tg / 1e9 / bf16, "single_launch_us": single * 1e3,
+                         "plan": list(opq.plan(m, qkv.N, qkv.K))}
+        del g
+    out["small_m"] = {"workload": "qkv 11520x3840, M in {1, 16, 64, 256}",
+                      "method": f"{2 * ncopy} back-to-back launches in one CUDA graph over {ncopy} copies of "
+                                f"the packed weight ({ncopy * wbytes / 1e6:.0f} MB > 4x L2); per-launch time = "
+                                f"graph time / launches", "by_m": small}
+    del copies, wqkv, pq
+    assert opq.device_error() == 0
+
+    # ---- the group-wise format (one float16 max per GS weights) on the projection
     grouped = {}
-    if not args.no_sweep:
-        wq_g = torch.empty_like(w)
-        y_g = torch.empty_like(y)
-        for gs in (128, 32):
-            cg, sg, gg = opq.quantize_grouped(w, gs, alpha)
-            ws_g = torch.zeros((max(opq.grouped_workspace_size(M, N, K, gs), 16),), dtype=torch.uint8, device=dev)
-            fq = lambda: opq.quantize_grouped(w, gs, alpha, out=(cg, sg, gg))
-            fl_ = lambda: opq.linear_grouped(x, cg, sg, gg, alpha, out=y_g, workspace=ws_g)
-            fd = lambda: opq.dequantize_grouped(cg, sg, gg, alpha, out=wq_g)
-            for f_ in (fq, fl_, fd):
-                for _ in range(3):
-                    f_()
-            tq_, _ = time_kernel(fq)
-            tl_, _ = time_kernel(fl_)
-            td_, _ = time_kernel(fd)
-            gq_bytes = N * K * 2 + N * K // 8 * 5 + 2 * N * (K // gs)
-            gd_bytes = N * K // 8 * 5 + 2 * N * (K // gs) + N * K * 2
-            g_tflops = flops / (tl_ * 1e-3) / 1e12
-            grouped[str(gs)] = {
-                "quantize": {"ms": tq_, "gbs": gq_bytes / (tq_ * 1e-3) / 1e9,
-                             "frac_hbm": gq_bytes / (tq_ * 1e-3) / 1e9 / peaks["hbm_gbs"]},
-                "linear": {"ms": tl_, "tflops": g_tflops, "frac_bf16": g_tflops / peaks["bf16_tflops"]},
-                "dequantize": {"ms": td_, "gbs": gd_bytes / (td_ * 1e-3) / 1e9,
-                               "frac_hbm": gd_bytes / (td_ * 1e-3) / 1e9 / peaks["hbm_gbs"]},
-            }
-            del ws_g
-        del wq_g, y_g
-        assert opq.device_error() == 0
-
-    # ---- the other bit widths of the card's configuration (3, 5, 6: 2^bits - 1 levels, codes as
-    # one bit stream per row) on the same weight: quantize, dequantize, and the SNR of each width
-    bits_out = {}
-    fused = {}
-    if not args.no_sweep:
-        wq_b = torch.empty_like(w)
-        for b_ in (3, 5, 6):
-            cb, sb, fb = opq.quantize_bits(w, b_, alpha)
-            fq = lambda: opq.quantize_bits(w, b_, alpha, out=(cb, sb, fb))
-            fd = lambda: opq.dequantize_bits(cb, sb, fb, b_, alpha, out=wq_b)
-            for f_ in (fq, fd):
-                for _ in range(3):
-                    f_()
-            tq_, _ = time_kernel(fq)
-            td_, _ = time_kernel(fd)
-            packed = N * K * b_ // 8 + N * K // 8 + 4 * N
-            bq_bytes = N * K * 2 + packed
-            bd_bytes = packed + N * K * 2
-            bits_out[str(b_)] = {
-                "quantize": {"ms": tq_, "gbs": bq_bytes / (tq_ * 1e-3) / 1e9,
-                             "frac_hbm": bq_bytes / (tq_ * 1e-3) / 1e9 / peaks["hbm_gbs"]},
-                "dequantize": {"ms": td_, "gbs": bd_bytes / (td_ * 1e-3) / 1e9,
-                               "frac_hbm": bd_bytes / (td_ * 1e-3) / 1e9 / peaks["hbm_gbs"]},
-                "snr_db": None}
-            opq.dequantize_bits(cb, sb, fb, b_, alpha, out=wq_b)
-            r_ = w.double()
-            bits_out[str(b_)]["snr_db"] = float(10.0 * torch.log10((r_ * r_).sum() / ((r_ - wq_b.double()) ** 2).sum()))
-            del cb, sb, fb
-        del wq_b
-        # the linear with its epilogue fused (bias + SiLU), as the layer an nn.Linear + activation
-        # becomes: same weight, activations and schedule as the step's linear
-        bias = (torch.arange(N, device=dev, dtype=torch.float32) * 1e-3 - 1.0).to(torch.bfloat16)
-        y_f = torch.empty_like(y)
-        for act in ("silu", "gelu_tanh"):
-            ff = lambda: opq.linear_fused(x, codes, signs, scales, alpha, bias=bias, act=act, out=y_f, workspace=ws)
+    wq_g = torch.empty_like(w)
+    y_g = torch.empty_like(y)
+    for gs in (128, 32):
+        cg, sg, gg = opq.quantize_grouped(w, gs, alpha)
+        ws_g = torch.zeros((max(opq.grouped_workspace_size(M, N, K, gs), 16),), dtype=torch.uint8, device=dev)
+        fq_ = lambda: opq.quantize_grouped(w, gs, alpha, out=(cg, sg, gg))
+        fl_ = lambda: opq.linear_grouped(x, cg, sg, gg, alpha, out=y_g, workspace=ws_g)
+        fd_ = lambda: opq.dequantize_grouped(cg, sg, gg, alpha, out=wq_g)
+        for f_ in (fq_, fl_, fd_):
             for _ in range(3):
-                ff()
-            tf_, _ = time_kernel(ff)
-            f_tflops = flops / (tf_ * 1e-3) / 1e12
-            fused[act] = {"ms": tf_, "tflops": f_tflops, "frac_bf16": f_tflops / peaks["bf16_tflops"]}
-        del y_f
-        assert opq.device_error() == 0
+                f_()
+        tq_, tl_, td_ = time_kernel(fq_), time_kernel(fl_), time_kernel(fd_)
+        gq_bytes = N * K * 2 + N * K // 8 * 5 + 2 * N * (K // gs)
+        gd_bytes = N * K // 8 * 5 + 2 * N * (K // gs) + N * K * 2
+        grouped[str(gs)] = {
+            "quantize": {"ms": tq_, "gbs": gq_bytes / tq_ / 1e6, "frac_hbm": gq_bytes / tq_ / 1e6 / hbm},
+            "linear": {"ms": tl_, "tflops": flops / tl_ / 1e9, "frac_bf16": flops / tl_ / 1e9 / bf16},
+            "dequantize": {"ms": td_, "gbs": gd_bytes / td_ / 1e6, "frac_hbm": gd_bytes / td_ / 1e6 / hbm}}
+        del ws_g
+    out["grouped"] = grouped
+    del wq_g, y_g
 
-    # ---- SNR context (the model card's "+7.2 dB" claim is on Z-Image weights; these are the
-    # synthetic Student-t weights of the bench workload): OPQ through the library at alpha 0.73
-    # and 1.0 (same 4-bit + sign + row max format), and per-row symmetric INT4 round(w/(max/7))
+    # ---- the other bit widths (3, 5, 6): quantize, dequantize and SNR on the projection weight
+    bits_out = {}
+    wq_b = torch.empty_like(w)
+    r_ = w.double()
+    for b_ in (3, 5, 6):
+        cb, sb, fb = opq.quantize_bits(w, b_, alpha)
+        fq_ = lambda: opq.quantize_bits(w, b_, alpha, out=(cb, sb, fb))
+        fd_ = lambda: opq.dequantize_bits(cb, sb, fb, b_, alpha, out=wq_b)
+        for f_ in (fq_, fd_):
+            for _ in range(3):
+                f_()
+        tq_, td_ = time_kernel(fq_), time_kernel(fd_)
+        packed = N * K * b_ // 8 + N * K // 8 + 4 * N
+        opq.dequantize_bits(cb, sb, fb, b_, alpha, out=wq_b)
+        bits_out[str(b_)] = {
+            "quantize": {"ms": tq_, "gbs": (N * K * 2 + packed) / tq_ / 1e6,
+                         "frac_hbm": (N * K * 2 + packed) / tq_ / 1e6 / hbm},
+            "dequantize": {"ms": td_, "gbs": (packed + N * K * 2) / td_ / 1e6,
+                           "frac_hbm": (packed + N * K * 2) / td_ / 1e6 / hbm},
+            "snr_db": float(10.0 * torch.log10((r_ * r_).sum() / ((r_ - wq_b.double()) ** 2).sum()))}
+        del cb, sb, fb
+    out["bits"] = bits_out
+    del wq_b, r_
+
+    # ---- the linear with bias + activation fused into its epilogue, same shape as the step
+    bias = (torch.arange(N, device=dev, dtype=torch.float32) * 1e-3 - 1.0).to(torch.bfloat16)
+    y_f = torch.empty_like(y)
+    fused = {"plain_ms": t_l}
+    for act in ("silu", "gelu_tanh"):
+        ff = lambda: opq.linear_fused(x, codes, signs, scales, alpha, bias=bias, act=act, out=y_f, workspace=ws)
+        for _ in range(3):
+            ff()
+        tf_ = time_kernel(ff)
+        fused[act] = {"ms": tf_, "tflops": flops / tf_ / 1e9, "frac_bf16": flops / tf_ / 1e9 / bf16,
+                      "vs_plain": tf_ / t_l}
+    out["fused"] = fused
+    del y_f
+    assert opq.device_error() == 0
+
+    # ---- SNR context (the card's "+7.2 dB" is on Z-Image weights; these are the synthetic
+    # Student-t weights): OPQ at alpha 0.73 and 1.0, per-row symmetric INT4, group-wise
     def snr_db(ref, rec):
-        r = ref.double()
-        return float(10.0 * torch.log10((r * r).sum() / ((r - rec.double()) ** 2).sum()))
+        rr = ref.double()
+        return float(10.0 * torch.log10((rr * rr).sum() / ((rr - rec.double()) ** 2).sum()))
 
     w_rec = torch.empty_like(w)
     snr = {}
@@ -379,126 +656,89 @@ def gpu_arm(args, rank, world, local_rank):
     p_ = opq.quantize_grouped(w, 128, alpha)
     opq.dequantize_grouped(*p_, alpha, out=w_rec)
     snr[f"opq_alpha_{alpha:g}_group128"] = snr_db(w, w_rec)
-    if not args.no_sweep:
-        # the alpha search over 0.30 .. 1.00 (the card's configuration range) on this weight
-        for gs_ in (0, 128):
-            best_a, snrs = opq.alpha_search(w, opq.ALPHA_GRID, gs_)
-            snr[f"alpha_search_{'row' if gs_ == 0 else 'group128'}"] = {
-                "best_alpha": best_a, "snr_db": dict(zip([f"{a_:.2f}" for a_ in opq.ALPHA_GRID], snrs))}
+    for gs_ in (0, 128):
+        best_a, snrs = opq.alpha_search(w, opq.ALPHA_GRID, gs_)
+        snr[f"alpha_search_{'row' if gs_ == 0 else 'group128'}"] = {
+            "best_alpha": best_a, "snr_db": dict(zip([f"{a_:.2f}" for a_ in opq.ALPHA_GRID], snrs))}
     snr["gain_vs_int4_db"] = snr[f"opq_alpha_{alpha:g}"] - snr["int4_symmetric_row"]
     snr["gain_vs_alpha1_db"] = snr[f"opq_alpha_{alpha:g}"] - snr["opq_alpha_1"]
     snr["model_card_claim_db"] = 7.2
-    del w_rec
-
-    # ---- end to end through the public API with host buffers
-    w_host = w.cpu().pin_memory()
-    x_host = x.cpu().pin_memory()
-    y_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
-    w_dev = torch.empty_like(w)
-    x_dev = torch.empty_like(x)
-
-    def e2e_step():
-        w_dev.copy_(w_host, non_blocking=True)
-        x_dev.copy_(x_host, non_blocking=True)
-        opq.quantize(w_dev, alpha, out=(codes, signs, scales))
-        opq.linear(x_dev, codes, signs, scales, alpha, out=y, workspace=ws)
-        opq.dequantize(codes, signs, scales, alpha, out=wq)
-        y_host.copy_(y, non_blocking=True)
-
-    for _ in range(2):
-        e2e_step()
-    torch.cuda.synchronize()
-    barrier()
-    ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    ea.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    eb.record(stream)
-    eb.synchronize()
-    ms_e2e = max_over_ranks(ea.elapsed_time(eb) / args.steps, world, dev)
-    barrier()
-
-    traffic = recorded_traffic("wide_kernel")
-    roof = {"bound": "tensor", "kernel": "wide_kernel<256>", "achieved": linear_tflops,
-            "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": linear_tflops / peaks["bf16_tflops"],
-            "traffic": traffic, "algorithmic_flops": flops, "algorithmic_bytes": l_bytes,
-            "launch_ms": t_l, "peak_source": f"bf16 dense burst, {peak_src}"}
-    out = {
-        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded Student-t(4) weights, N(0,1) activations)",
-        "config": {"workload": lin.name, "M": M, "N": N, "K": K, "alpha": alpha,
-                   "step": "quantize W + linear x W'^T + dequantize W'", "parallelism": f"replicas{world}",
-                   "l2": "flushed between timed steps (4x L2 buffer write outside the event pairs)"},
-        "kernels": kernels, "small_m": small, "grouped": grouped, "bits": bits_out, "fused": fused,
-        "roofline": roof, "snr_db": snr,
-        "e2e": {"value": whole_job_tflops(world, flops, ms_e2e), "unit": "TFLOP/s", "ms_per_step": ms_e2e,
-                "h2d_bytes_per_step": w.numel() * 2 + x.numel() * 2, "d2h_bytes_per_step": y.numel() * 2},
-        "gpu_launches": launches_per_step * args.steps,
-        "kernels_live_ms": live,
-        "clocks": clocks.summary(),
-        "peaks": peaks,
-    }
+    out["snr_db"] = snr
     return out
 
 
 # --------------------------------------------------------------------------- CPU arms
-def cpu_oracle_sample(budget_s: float = 12.0):
-    """Time the fp64 oracle on a bounded sample of the bench workload: quantize 256
-    weight rows and the linear for 16 activation rows against those 256 weight rows."""
-    import numpy as np
-    import oracle
+def oracle_sample():
+    """A bounded sample of the whole-model pass for the fp64 oracle: 256 weight rows of an
+    attention matrix and of the FFN down-projection (block 0), quantized, and the linear of
+    16 activation rows against those rows."""
     import workloads
+    model = workloads.WholeModel(blocks=1)
+    out = []
+    for l in (model.layers[0], model.layers[6]):
+        x = l.make_x("cpu")[:16].contiguous()
+        w = l.make_weights("cpu")[:256].contiguous()
+        out.append((x, w, l.alpha))
+    return out
 
-    lin = workloads.dit_attn_proj()
-    x, w = lin.make("cpu")
-    rows = 256
-    xs, ws = x[:16].contiguous(), w[:rows].contiguous()
+
+def oracle_step(oracle, sample):
+    for x, w, a in sample:
+        r = oracle.quantize(w, a)
+        oracle.linear(x, r["codes"], r["signs"], r["scales"], a)
+
+
+def sample_counts(sample):
+    flops = sum(2.0 * x.shape[0] * w.shape[0] * w.shape[1] for x, w, _ in sample)
+    qbytes = sum(quant_bytes(w.shape[0], w.shape[1]) for _, w, _ in sample)
+    return flops, qbytes
+
+
+SAMPLE_TEXT = ("quantize 256 rows of W 3840x3840 and of W2 3840x10240 (block 0) + linear 16 x-rows against "
+               "those 256 rows of each")
+
+
+def cpu_oracle_sample(budget_s: float = 12.0):
+    """Time the fp64 oracle on the bounded sample of the whole-model workload."""
+    import oracle
     oracle.build()
+    sample = oracle_sample()
     t0 = time.perf_counter()
     reps = 0
     while True:
-        r = oracle.quantize(ws, lin.alpha)
-        oracle.linear(xs, r["codes"], r["signs"], r["scales"], lin.alpha)
+        oracle_step(oracle, sample)
         reps += 1
         if time.perf_counter() - t0 > budget_s:
             break
     dt = (time.perf_counter() - t0) / reps
-    flops = 2.0 * xs.shape[0] * rows * lin.K
-    cores = oracle.num_threads()
-    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-            "sample": f"quantize {rows}x{lin.K} + linear {xs.shape[0]}x{lin.K} @ {rows}x{lin.K}^T "
-                      f"({reps} reps, {dt:.3f} s each)",
-            "seconds_per_sample": dt}
+    flops, qbytes = sample_counts(sample)
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{SAMPLE_TEXT} ({reps} reps, {dt:.3f} s each)", "seconds_per_sample": dt,
+            "quantize_gbs_in_sample": qbytes / dt / 1e9}
 
 
 def reference_arm(args):
     import oracle
-    import workloads
-    lin = workloads.dit_attn_proj()
-    x, w = lin.make("cpu")
-    xs, ws = x[:16].contiguous(), w[:256].contiguous()
     oracle.build()
+    sample = oracle_sample()
     for _ in range(args.warmup):
-        r = oracle.quantize(ws, lin.alpha)
-        oracle.linear(xs, r["codes"], r["signs"], r["scales"], lin.alpha)
+        oracle_step(oracle, sample)
     ts = []
     for _ in range(args.steps):
         t0 = time.perf_counter()
-        r = oracle.quantize(ws, lin.alpha)
-        oracle.linear(xs, r["codes"], r["signs"], r["scales"], lin.alpha)
+        oracle_step(oracle, sample)
         ts.append(time.perf_counter() - t0)
     dt = sum(ts) / len(ts)
-    flops = 2.0 * xs.shape[0] * ws.shape[0] * lin.K
+    flops, _ = sample_counts(sample)
     v = flops / dt / 1e12
     cores = oracle.num_threads()
     return {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": lin.name, "sample": "quantize 256 weight rows + linear 16 x 256 outputs",
+            "config": {"workload": "dit_whole_model_30blocks_210layers_m3072", "sample": SAMPLE_TEXT,
                        "parallelism": "cpu"},
             "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                             "sample": "quantize 256x3840 + linear 16x3840 @ 256x3840^T per step"},
+                             "sample": SAMPLE_TEXT + " per step"},
             "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
@@ -509,22 +749,31 @@ def profile_run(args):
     import workloads
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    if args.profile.startswith("small"):
-        lin = workloads.small_m(int(args.profile[5:]))
+    shapes = {"attn": workloads.dit_attn_proj(),
+              # the whole-model pass's three shape classes at M = 3072 (block 0's seeds)
+              "wm_attn": workloads.WholeModel(blocks=1).layers[0],
+              "wm_up": workloads.WholeModel(blocks=1).layers[4],
+              "wm_down": workloads.WholeModel(blocks=1).layers[6],
+              "ffn_up": workloads.dit_ffn_pair()[0], "ffn_down": workloads.dit_ffn_pair()[1]}
+    if args.shape.startswith("small"):
+        lin = workloads.small_m(int(args.shape[5:]))
     else:
-        lin = workloads.dit_attn_proj()
+        lin = shapes[args.shape]
     x, w = lin.make(dev)
     planes = opq.quantize(w, lin.alpha)
     y = torch.empty((lin.M, lin.N), dtype=torch.bfloat16, device=dev)
     wq = torch.empty_like(w)
     ws = torch.zeros((max(opq.workspace_size(lin.M, lin.N, lin.K), 16),), dtype=torch.uint8, device=dev)
-    gplanes = opq.quantize_grouped(w, 128, lin.alpha)
-    gws = torch.zeros((max(opq.grouped_workspace_size(lin.M, lin.N, lin.K, 128), 16),), dtype=torch.uint8, device=dev)
     fns = {"quantize": lambda: opq.quantize(w, lin.alpha, out=planes),
            "dequantize": lambda: opq.dequantize(*planes, lin.alpha, out=wq),
-           "grouped_quantize": lambda: opq.quantize_grouped(w, 128, lin.alpha, out=gplanes),
-           "grouped_linear": lambda: opq.linear_grouped(x, *gplanes, lin.alpha, out=y, workspace=gws)}
-    fn = fns.get(args.profile, lambda: opq.linear(x, *planes, lin.alpha, out=y, workspace=ws))
+           "linear": lambda: opq.linear(x, *planes, lin.alpha, out=y, workspace=ws)}
+    if args.profile.startswith("grouped"):
+        gplanes = opq.quantize_grouped(w, 128, lin.alpha)
+        gws = torch.zeros((max(opq.grouped_workspace_size(lin.M, lin.N, lin.K, 128), 16),), dtype=torch.uint8,
+                          device=dev)
+        fns["grouped_quantize"] = lambda: opq.quantize_grouped(w, 128, lin.alpha, out=gplanes)
+        fns["grouped_linear"] = lambda: opq.linear_grouped(x, *gplanes, lin.alpha, out=y, workspace=gws)
+    fn = fns[args.profile]
     for _ in range(args.warmup):
         fn()
     torch.cuda.synchronize()
@@ -539,15 +788,17 @@ def profile_run(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=400)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="opq", choices=["opq", "reference"])
-    ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the extras (FFN pair, projection, small M, ...)")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", default=None,
                     help="profiling run: warm up, then launch only this kernel --steps times "
-                         "(quantize | linear | dequantize | grouped_quantize | grouped_linear | small<M>) "
-                         "on the bench workload")
+                         "(quantize | linear | dequantize | grouped_quantize | grouped_linear) on --shape")
+    ap.add_argument("--shape", default="attn",
+                    help="profiling shape: attn | wm_attn | wm_up | wm_down | ffn_up | ffn_down | small<M>")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -31,7 +31,7 @@ EXPORTS = ["opq_quantize", "opq_dequantize", "opq_linear_workspace_size", "opq_l
            "opq_abi_version", "opq_quantize_grouped", "opq_dequantize_grouped",
            "opq_linear_grouped", "opq_linear_grouped_workspace_size", "opq_linear_fused",
            "opq_linear_grouped_fused", "opq_alpha_search", "opq_alpha_search_workspace_size",
-           "opq_quantize_bits", "opq_dequantize_bits"]
+           "opq_quantize_bits", "opq_dequantize_bits", "opq_set_wait_limit_ns"]
 ACTIVATIONS = {"none": 0, "silu": 1, "gelu_tanh": 2}
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
@@ -73,12 +73,14 @@ def load(path: str = LIB_PATH):
     lib.opq_alpha_search.argtypes = [P, I, I, I, I, P, ctypes.c_int32, P, P, P, S, P]
     lib.opq_linear_fused.argtypes = [P, I, I, P, P, P, I, F, P, ctypes.c_int, P, P, S, P]
     lib.opq_linear_grouped_fused.argtypes = [P, I, I, P, P, P, I, I, F, P, ctypes.c_int, P, P, S, P]
+    lib.opq_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
     lib.opq_status_string.argtypes = [ctypes.c_int]
     lib.opq_status_string.restype = ctypes.c_char_p
     for f in ("opq_quantize", "opq_dequantize", "opq_linear_workspace_size", "opq_linear", "opq_linear_plan",
               "opq_linear_noalloc", "opq_device_error", "opq_quantize_grouped", "opq_dequantize_grouped", "opq_linear_grouped",
               "opq_linear_grouped_workspace_size", "opq_linear_fused", "opq_linear_grouped_fused",
-              "opq_alpha_search", "opq_alpha_search_workspace_size", "opq_quantize_bits", "opq_dequantize_bits"):
+              "opq_alpha_search", "opq_alpha_search_workspace_size", "opq_quantize_bits", "opq_dequantize_bits",
+              "opq_set_wait_limit_ns"):
         getattr(lib, f).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -336,8 +338,17 @@ def linear_noalloc(x: torch.Tensor, codes: torch.Tensor, signs: torch.Tensor, sc
     return y
 
 
+DEVERR_WAIT_TIMEOUT = 1
+DEVERR_SMEM_ALIGN = 2
+
+
 def device_error(device=None) -> int:
     """Read and clear the library's device-side error word (synchronises the current stream)."""
     v = ctypes.c_uint32(0)
     _check(load().opq_device_error(_stream(device), ctypes.byref(v)), "opq_device_error")
     return int(v.value)
+
+
+def set_wait_limit_ns(ns: int = 0):
+    """Time after which the kernels' bounded waits give up on the current device (0: the 4 s default)."""
+    _check(load().opq_set_wait_limit_ns(int(ns)), "opq_set_wait_limit_ns")

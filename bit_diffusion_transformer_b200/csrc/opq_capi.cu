@@ -785,19 +785,6 @@ opq_status opq_linear_grouped_workspace_size(int64_t M, int64_t N, int64_t K, in
     return OPQ_OK;
 }
 
-opq_status opq_device_error(void *stream, uint32_t *err) {
-    if (!err) return OPQ_ERR_INVALID_ARG;
-    cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
-    if (e != cudaSuccess) return cuda_fail(e);
-    uint32_t v = 0, zero = 0;
-    e = cudaMemcpyFromSymbol(&v, opqdev::g_error, sizeof v);
-    if (e != cudaSuccess) return cuda_fail(e);
-    e = cudaMemcpyToSymbol(opqdev::g_error, &zero, sizeof zero);
-    if (e != cudaSuccess) return cuda_fail(e);
-    *err = v;
-    return OPQ_OK;
-}
-
 // ---------------------------------------------------------------------------
 // Allocation-free linear: the split-K scratch lives in a static device array.
 // ---------------------------------------------------------------------------
@@ -828,6 +815,45 @@ opq_status noalloc_scratch(void **out) {
     return OPQ_OK;
 }
 }  // namespace
+
+extern "C" opq_status opq_device_error(void *stream, uint32_t *err) {
+    if (!err) return OPQ_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e);
+    uint32_t v = 0, zero = 0;
+    e = cudaMemcpyFromSymbol(&v, opqdev::g_error, sizeof v);
+    if (e != cudaSuccess) return cuda_fail(e);
+    e = cudaMemcpyToSymbol(opqdev::g_error, &zero, sizeof zero);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (v & opqdev::kErrWaitTimeout) {
+        // A call that gave up waiting can leave arrival counters or published flags set. In a
+        // caller's workspace the caller zeroes them; the allocation-free linear's counters sit
+        // in the library's static array, so they are cleared here (a memset, no allocation).
+        int dev = 0;
+        e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return cuda_fail(e);
+        void *p = nullptr;
+        if (dev >= 0 && dev < 64) {
+            std::lock_guard<std::mutex> lk(g_noalloc_mu);
+            p = g_noalloc_ptr[dev];
+        }
+        if (p != nullptr) {
+            e = cudaMemsetAsync(p, 0, kCounterBytes, st);
+            if (e != cudaSuccess) return cuda_fail(e);
+            e = cudaStreamSynchronize(st);
+            if (e != cudaSuccess) return cuda_fail(e);
+        }
+    }
+    *err = v;
+    return OPQ_OK;
+}
+
+extern "C" opq_status opq_set_wait_limit_ns(uint64_t ns) {
+    const uint64_t v = ns == 0 ? opqdev::kWaitLimitNs : ns;
+    cudaError_t e = cudaMemcpyToSymbol(opqdev::g_wait_limit_ns, &v, sizeof v);
+    return e == cudaSuccess ? OPQ_OK : cuda_fail(e);
+}
 
 extern "C" opq_status opq_linear_noalloc(const uint16_t *x, int64_t M, int64_t K, const uint32_t *codes,
                                          const uint32_t *signs, const float *scales, int64_t N, float alpha,

@@ -15,8 +15,15 @@ __device__ uint32_t g_error = 0;
 constexpr uint32_t kErrWaitTimeout = 1u;
 constexpr uint32_t kErrSmemAlign = 2u;     // dynamic shared memory not on the 1 KiB boundary
 
-// A bounded wait gives up after this many nanoseconds of %globaltimer.
+// A bounded wait gives up after g_wait_limit_ns nanoseconds of %globaltimer: 4 s unless the
+// host changed it (opq_set_wait_limit_ns, for diagnostics and tests). It is read only once a
+// wait did not succeed at its first try.
 constexpr uint64_t kWaitLimitNs = 4000000000ull;   // 4 s
+__device__ uint64_t g_wait_limit_ns = kWaitLimitNs;
+
+__device__ __forceinline__ uint64_t wait_limit_ns() {
+    return *reinterpret_cast<volatile const uint64_t *>(&g_wait_limit_ns);
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -64,15 +71,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete. Returns false (and
-// records kErrWaitTimeout) if it has not completed within kWaitLimitNs.
+// records kErrWaitTimeout) if it has not completed within the wait limit.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
     const uint32_t a = smem_u32(bar);
     if (mbar_try_wait(a, parity)) return true;
-    const uint64_t t0 = globaltimer();
+    const uint64_t t0 = globaltimer(), limit = wait_limit_ns();
     while (true) {
         for (int i = 0; i < 64; ++i)
             if (mbar_try_wait(a, parity)) return true;
-        if (globaltimer() - t0 > kWaitLimitNs) {
+        if (globaltimer() - t0 > limit) {
             atomicOr(&g_error, kErrWaitTimeout);
             return false;
         }
@@ -140,11 +147,11 @@ __device__ __forceinline__ uint32_t flag_load_acquire(const uint32_t *p) {
 // on anything itself. Same time limit and error word as mbar_wait.
 __device__ __forceinline__ bool flag_wait(const uint32_t *p, uint32_t want) {
     if (flag_load_acquire(p) == want) return true;
-    const uint64_t t0 = globaltimer();
+    const uint64_t t0 = globaltimer(), limit = wait_limit_ns();
     while (true) {
         for (int i = 0; i < 64; ++i)
             if (flag_load_acquire(p) == want) return true;
-        if (globaltimer() - t0 > kWaitLimitNs) {
+        if (globaltimer() - t0 > limit) {
             atomicOr(&g_error, kErrWaitTimeout);
             return false;
         }

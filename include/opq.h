@@ -242,6 +242,9 @@ opq_status opq_linear_plan(int64_t M, int64_t N, int64_t K, int *path, int *ctas
  *   - All calls share the one array and it keeps the last call's contents. Its
  *     leading arrival counters must be zero when a call starts: the array is zero
  *     when the library loads and every completed call leaves them at zero again.
+ *     A call whose bounded wait gave up (opq_device_error reports
+ *     OPQ_DEVERR_WAIT_TIMEOUT) can leave them set; opq_device_error clears them
+ *     when it reports that error, so read it before the next call of this kind.
  *     Calls that overlap on the GPU (different streams, or different host threads
  *     without ordering) race on the array and give wrong results.
  *   - No device memory is allocated or freed by this call.
@@ -258,10 +261,27 @@ opq_status opq_linear_noalloc(const uint16_t *x, int64_t M, int64_t K, const uin
  * invalid: WAIT_TIMEOUT when a bounded wait on a barrier gave up, SMEM_ALIGN when
  * the dynamic shared-memory window did not start on the 1 KiB boundary that the
  * 128-byte-swizzled tensor-core operand stages need.
+ * After a WAIT_TIMEOUT a caller-provided linear workspace must be zero-filled
+ * again before its next use; the arrival counters of opq_linear_noalloc's static
+ * array are zeroed by this call itself (a memset on `stream`, synchronised; no
+ * opq_linear_noalloc call may be in flight on another stream meanwhile).
  */
 #define OPQ_DEVERR_WAIT_TIMEOUT 1u
 #define OPQ_DEVERR_SMEM_ALIGN 2u
 opq_status opq_device_error(void *stream, uint32_t *err);
+
+/*
+ * opq_set_wait_limit_ns — the time after which a kernel's bounded wait on a
+ * barrier or a flag gives up (records OPQ_DEVERR_WAIT_TIMEOUT, lets its own copies
+ * in flight land, frees its tensor memory and returns) on the current device;
+ * ns = 0 restores the default of 4 s. Every wait in a healthy call ends within
+ * that call's own run time, so the limit only bounds how long a broken
+ * protocol (for example a workspace that was not zeroed) can hold the GPU; tests
+ * shorten it to see a time-out quickly. The value is written with a
+ * synchronous copy to device memory and is read by kernels launched after the
+ * call returns; do not change it while library kernels run on other streams.
+ */
+opq_status opq_set_wait_limit_ns(uint64_t ns);
 
 /* Human-readable name of a status. */
 const char *opq_status_string(opq_status s);
