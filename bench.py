@@ -232,13 +232,19 @@ class WholeModelState:
         need = max(opq.workspace_size(self.M, l.N, l.K) for l in self.model.layers)
         self.ws = torch.zeros((max(need, 16),), dtype=torch.uint8, device=dev)
         self.by_class = {c[0]: [L for L in self.layers if L["cls"] == c[0]] for c in WM_CLASSES}
+        # one opq_quantize_batched call per shape class quantizes all its matrices in one stream
+        self.jobs = {c: (opq.quantize_jobs([L["w"] for L in Ls], [(L["c"], L["s"], L["sc"]) for L in Ls],
+                                           self.alpha), [L["w"] for L in Ls],
+                         [(L["c"], L["s"], L["sc"]) for L in Ls]) for c, Ls in self.by_class.items()}
 
     def phase(self, opq, what, cls):
         a, M = self.alpha, self.M
+        if what == "quantize":
+            jobs, ws, outs = self.jobs[cls]
+            opq.quantize_batched(ws, a, outs=outs, jobs=jobs)
+            return
         for L in self.by_class[cls]:
-            if what == "quantize":
-                opq.quantize(L["w"], a, out=(L["c"], L["s"], L["sc"]))
-            elif what == "linear":
+            if what == "linear":
                 opq.linear(self.x[L["K"]], L["c"], L["s"], L["sc"], a, out=self.y[L["N"]], workspace=self.ws)
             else:
                 opq.dequantize(L["c"], L["s"], L["sc"], a, out=L["wq"])
@@ -370,7 +376,9 @@ def gpu_arm(args, rank, world, local_rank):
         "by_class": {c: tf_entry(seg[("linear", c)], cnt[c]["linear_flops"],
                                  {"layers": cnt[c]["matrices"], "plan": list(opq.plan(M, *[(n, k) for nm, n, k in WM_CLASSES if nm == c][0]))})
                      for c in cls_names}})
-    launches_per_step = 3 * len(S.layers)
+    # library kernels per step: the batched quantize (one launch per 128 matrices of a class), one
+    # linear and one dequantize per layer
+    launches_per_step = sum(-(-cnt[c]["matrices"] // 128) for c in cls_names) + 2 * len(S.layers)
     linear_tflops = kernels["linear_all"]["tflops"]
 
     # ---------------------------------------------------------------- e2e: host buffers
@@ -393,8 +401,9 @@ def gpu_arm(args, rank, world, local_rank):
             for L in S.layers:
                 n, k = L["N"], L["K"]
                 L["w"].copy_(w_host[L["off"]:L["off"] + n * k].view(n, k), non_blocking=True)
-            for L in S.layers:
-                opq.quantize(L["w"], alpha, out=(L["c"], L["s"], L["sc"]))
+            for c in cls_names:
+                jobs, ws_, outs_ = S.jobs[c]
+                opq.quantize_batched(ws_, alpha, outs=outs_, jobs=jobs)
             for L in S.layers:
                 y = S.y[L["N"]]
                 opq.linear(S.x[L["K"]], L["c"], L["s"], L["sc"], alpha, out=y, workspace=S.ws)
@@ -450,7 +459,8 @@ def gpu_arm(args, rank, world, local_rank):
         "data": "synthetic (seeded Student-t(4) weights std 0.02 drawn per layer on the device, N(0,1) activations)",
         "config": {"workload": "dit_whole_model_30blocks_210layers_m3072", "blocks": 30, "layers": 210,
                    "weights": 5308416000, "M": M, "alpha": alpha,
-                   "step": "quantize all 210 W + linear x W'^T on every layer (M 3072) + dequantize all 210",
+                   "step": "quantize all 210 W (one batched call per shape class) + linear x W'^T on every "
+                           "layer (M 3072) + dequantize all 210",
                    "parallelism": f"replicas{world}",
                    "l2": "inputs larger than L2 (10.62 GB of weights per step against a 126 MB L2); no flush",
                    "launch": "each phase and shape class is one CUDA graph of the library's launches"},
@@ -764,7 +774,9 @@ def profile_run(args):
     y = torch.empty((lin.M, lin.N), dtype=torch.bfloat16, device=dev)
     wq = torch.empty_like(w)
     ws = torch.zeros((max(opq.workspace_size(lin.M, lin.N, lin.K), 16),), dtype=torch.uint8, device=dev)
+    jobs = opq.quantize_jobs([w], [planes], lin.alpha)
     fns = {"quantize": lambda: opq.quantize(w, lin.alpha, out=planes),
+           "quantize_batched": lambda: opq.quantize_batched([w], lin.alpha, outs=[planes], jobs=jobs),
            "dequantize": lambda: opq.dequantize(*planes, lin.alpha, out=wq),
            "linear": lambda: opq.linear(x, *planes, lin.alpha, out=y, workspace=ws)}
     if args.profile.startswith("grouped"):
@@ -796,7 +808,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", default=None,
                     help="profiling run: warm up, then launch only this kernel --steps times "
-                         "(quantize | linear | dequantize | grouped_quantize | grouped_linear) on --shape")
+                         "(quantize | quantize_batched | linear | dequantize | grouped_quantize | grouped_linear) "
+                         "on --shape")
     ap.add_argument("--shape", default="attn",
                     help="profiling shape: attn | wm_attn | wm_up | wm_down | ffn_up | ffn_down | small<M>")
     args = ap.parse_args()

@@ -31,7 +31,8 @@ EXPORTS = ["opq_quantize", "opq_dequantize", "opq_linear_workspace_size", "opq_l
            "opq_abi_version", "opq_quantize_grouped", "opq_dequantize_grouped",
            "opq_linear_grouped", "opq_linear_grouped_workspace_size", "opq_linear_fused",
            "opq_linear_grouped_fused", "opq_alpha_search", "opq_alpha_search_workspace_size",
-           "opq_quantize_bits", "opq_dequantize_bits", "opq_set_wait_limit_ns"]
+           "opq_quantize_bits", "opq_dequantize_bits", "opq_set_wait_limit_ns",
+           "opq_quantize_batched"]
 ACTIVATIONS = {"none": 0, "silu": 1, "gelu_tanh": 2}
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
@@ -74,13 +75,14 @@ def load(path: str = LIB_PATH):
     lib.opq_linear_fused.argtypes = [P, I, I, P, P, P, I, F, P, ctypes.c_int, P, P, S, P]
     lib.opq_linear_grouped_fused.argtypes = [P, I, I, P, P, P, I, I, F, P, ctypes.c_int, P, P, S, P]
     lib.opq_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+    lib.opq_quantize_batched.argtypes = [P, I, F, P]
     lib.opq_status_string.argtypes = [ctypes.c_int]
     lib.opq_status_string.restype = ctypes.c_char_p
     for f in ("opq_quantize", "opq_dequantize", "opq_linear_workspace_size", "opq_linear", "opq_linear_plan",
               "opq_linear_noalloc", "opq_device_error", "opq_quantize_grouped", "opq_dequantize_grouped", "opq_linear_grouped",
               "opq_linear_grouped_workspace_size", "opq_linear_fused", "opq_linear_grouped_fused",
               "opq_alpha_search", "opq_alpha_search_workspace_size", "opq_quantize_bits", "opq_dequantize_bits",
-              "opq_set_wait_limit_ns"):
+              "opq_set_wait_limit_ns", "opq_quantize_batched"):
         getattr(lib, f).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -121,6 +123,39 @@ def quantize(w: torch.Tensor, alpha: float = ALPHA, out=None):
     _check(load().opq_quantize(_ptr(w), N, K, K, float(alpha), _ptr(codes), _ptr(signs), _ptr(scales),
                                _stream(w.device)), "opq_quantize")
     return codes, signs, scales
+
+
+class QuantJob(ctypes.Structure):
+    """One matrix of opq_quantize_batched (the C struct opq_quant_job)."""
+    _fields_ = [("w", ctypes.c_void_p), ("N", ctypes.c_int64), ("K", ctypes.c_int64), ("ldw", ctypes.c_int64),
+                ("codes", ctypes.c_void_p), ("signs", ctypes.c_void_p), ("scales", ctypes.c_void_p)]
+
+
+def quantize_jobs(ws, outs, alpha: float = ALPHA):
+    """The descriptor array of opq_quantize_batched for bf16 weights ``ws`` and their
+    output planes ``outs`` [(codes, signs, scales), ...] (built once, reusable)."""
+    assert len(ws) == len(outs) and len(ws) > 0
+    arr = (QuantJob * len(ws))()
+    for i, (w, (c, s, f)) in enumerate(zip(ws, outs)):
+        assert w.dtype == torch.bfloat16 and w.dim() == 2
+        _need_cuda(w, c, s, f)
+        N, K = w.shape
+        arr[i] = QuantJob(w.data_ptr(), N, K, K, c.data_ptr(), s.data_ptr(), f.data_ptr())
+    return arr
+
+
+def quantize_batched(ws, alpha: float = ALPHA, outs=None, jobs=None):
+    """OPQ-quantize a list of bf16 matrices in one pass -> [(codes, signs, scales), ...].
+    ``jobs`` (from quantize_jobs) skips rebuilding the descriptors for the same buffers."""
+    if outs is None:
+        outs = [(torch.empty((w.shape[0], w.shape[1] // 8), dtype=torch.int32, device=w.device),
+                 torch.empty((w.shape[0], w.shape[1] // 32), dtype=torch.int32, device=w.device),
+                 torch.empty((w.shape[0],), dtype=torch.float32, device=w.device)) for w in ws]
+    if jobs is None:
+        jobs = quantize_jobs(ws, outs, alpha)
+    _check(load().opq_quantize_batched(ctypes.cast(jobs, ctypes.c_void_p), len(jobs), float(alpha),
+                                       _stream(ws[0].device)), "opq_quantize_batched")
+    return outs
 
 
 def dequantize(codes: torch.Tensor, signs: torch.Tensor, scales: torch.Tensor, alpha: float = ALPHA, out=None):

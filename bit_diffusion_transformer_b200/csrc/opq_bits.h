@@ -137,51 +137,69 @@ OPQ_HD uint32_t pack_codes(uint32_t q0, uint32_t q1, uint32_t q2, uint32_t q3) {
 // Coding by table. For non-negative bf16 values the bit pattern is monotone in
 // the value, so with a row's nondecreasing thresholds T_1..T_15 (bf16 bits) the
 // code q(a) = #{k : T_k <= a} of a magnitude a <= mx depends only on d = mx - a,
-// and is 0 from d_z = mx - T_1 + 1 on.
+// and is 0 from d_z = mx - T_1 + 1 on. A row's table holds q(mx - e) for the
+// entries e = 0 .. d_z, one byte each, with q in both nibbles (q * 17).
 // ---------------------------------------------------------------------------
-// Entries e in [4 w0, 4 w1) of the table q(mx - e), as words of four bytes (byte j
-// of word wd is entry 4 wd + j): q at the first entry by counting, then lowered
-// while walking down the thresholds. T[1..15] must be nondecreasing; entries past
-// mx (e > mx) are 0.
-OPQ_HD void code_table_run(const uint16_t *T, uint32_t mx, uint32_t w0, uint32_t w1, uint32_t *tab) {
-    if (w0 >= w1) return;
-    const int b0 = (int)mx - (int)(4u * w0);
-    uint32_t q = 0;
-    for (int k = 1; k < 16; ++k) q += (int)T[k] <= b0 ? 1u : 0u;
-    int tq = q ? (int)T[q] : 0;
-    for (uint32_t wd = w0; wd < w1; ++wd) {
-        uint32_t word = 0;
-        for (int j = 0; j < 4; ++j) {
-            const int b = (int)mx - (int)(4u * wd + j);
-            while (q > 0u && b < tq) {
-                --q;
-                tq = q ? (int)T[q] : 0;
-            }
-            word |= q << (8 * j);
-        }
-        tab[wd] = word;
+// One table word from the level boundaries. With B_k = bits(max) - T_k + 1 (0 when level k is
+// out of reach), q(e) = #{k : B_k > e}. For word w (entries 4w .. 4w + 3) inside a stretch of
+// entries (lo, hi] of the table: c_full = #{k : B_k > hi} levels hold for every entry of the
+// stretch, and each boundary B inside the stretch (lo < B <= hi) adds 1 to the entries e < B
+// of the word, i.e. to its first clamp(B - 4w, 0, 4) bytes. `inside` lists those boundaries.
+OPQ_HD uint32_t table_word_from_bounds(uint32_t c_full, const int *inside, int n_inside, uint32_t w) {
+    uint32_t word = c_full * 0x01010101u;
+    for (int i = 0; i < n_inside; ++i) {
+        int c = inside[i] - (int)(4u * w);
+        c = c < 0 ? 0 : (c > 4 ? 4 : c);
+        word += c == 0 ? 0u : (0x01010101u >> (8 * (4 - c)));
     }
+    return word;
 }
 
-// per-half unsigned 16-bit minimum
-OPQ_HD uint32_t vminu2(uint32_t a, uint32_t b) {
+// Per-half maximum of two bf16 pairs (max.bf16x2): for non-negative finite halves it is the
+// larger bit pattern, so it serves as a packed unsigned 16-bit max on magnitudes; a NaN half
+// gives the canonical NaN 0x7FFF.
+OPQ_HD uint32_t bf16x2_max(uint32_t a, uint32_t b) {
 #if defined(__CUDA_ARCH__)
-    return __vminu2(a, b);
+    uint32_t r;
+    asm("max.NaN.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
 #else
-    const uint32_t lo = (a & 0xFFFFu) < (b & 0xFFFFu) ? (a & 0xFFFFu) : (b & 0xFFFFu);
-    const uint32_t hi = (a >> 16) < (b >> 16) ? (a >> 16) : (b >> 16);
-    return lo | (hi << 16);
+    uint32_t r = 0;
+    for (int h = 0; h < 2; ++h) {
+        const uint32_t ua = ((a >> (16 * h)) & 0xFFFFu) << 16, ub = ((b >> (16 * h)) & 0xFFFFu) << 16;
+        float fa, fb;
+        __builtin_memcpy(&fa, &ua, 4);
+        __builtin_memcpy(&fb, &ub, 4);
+        uint32_t m;
+        if (fa != fa || fb != fb) m = 0x7FFFu;
+        else m = (fa >= fb ? ua : ub) >> 16;
+        r |= m << (16 * h);
+    }
+    return r;
 #endif
 }
 
-// Codes of a bf16 pair x (q in bits 0..3 and 16..19) from a row's table stored at
-// byte offset `base` of tb: per half d = min(mx - |w|, d_z), read at base + d.
-// mmb = (mx + base) and dzb = (d_z + base) in both halves; the caller keeps
-// mx + base below 2^16 and |w| <= mx per half, so nothing carries or borrows
-// across the halves.
-OPQ_HD uint32_t table_pair(const uint8_t *tb, uint32_t x, uint32_t mmb, uint32_t dzb) {
-    const uint32_t d = vminu2(mmb - (x & 0x7FFF7FFFu), dzb);
-    return (uint32_t)tb[d & 0xFFFFu] | ((uint32_t)tb[d >> 16] << 16);
+// The code byte of a magnitude pair a (sign bits cleared; element 2p in the low nibble, 2p + 1
+// in the high nibble) from a row table at byte offset `base` of tb whose entries hold q in both
+// nibbles: the low half's entry gives the low nibble, the high half's the high nibble. The clamp is
+// done on the magnitudes: d = mmb - max(a, lo2) stays within [base, base + d_z] per half
+// (lo2 = bits(max) - d_z and mmb = bits(max) + base in both halves; the caller keeps
+// bits(max) + base below 2^16 and a <= bits(max) per half, so no half borrows from the other);
+// the index of the high half comes from a multiply-high so that it issues on the FMA pipe.
+OPQ_HD uint32_t table_byte_clamped(const uint8_t *tb, uint32_t a, uint32_t lo2, uint32_t mmb) {
+    const uint32_t d = mmb - bf16x2_max(a, lo2);
+#if defined(__CUDA_ARCH__)
+    uint32_t hi;
+    asm("mul.hi.u32 %0, %1, 65536;" : "=r"(hi) : "r"(d));
+#else
+    const uint32_t hi = d >> 16;
+#endif
+    return ((uint32_t)tb[d & 0xFFFFu] & 0x0Fu) | ((uint32_t)tb[hi] & 0xF0u);
+}
+
+// Four code bytes (each in the low byte of its word) -> one code word, byte p = b_p.
+OPQ_HD uint32_t codes_word(uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3) {
+    return prmt(prmt(b0, b1, 0x0040u), prmt(b2, b3, 0x0040u), 0x5410u);
 }
 
 // Sign bits (bf16 sign bit set) of 8 weights held as 4 bf16 pairs -> bits 0..7.

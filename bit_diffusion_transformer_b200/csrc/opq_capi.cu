@@ -17,6 +17,7 @@
 #include "opq_linear.cuh"
 #include "opq_linear_wide.cuh"
 #include "opq_quantize.cuh"
+#include "opq_quantize_stream.cuh"
 
 namespace {
 
@@ -67,6 +68,7 @@ uint16_t host_bf16(double v) {
 
 struct DeviceInfo {
     int sms = 0;
+    bool stream_quant_attr[3] = {};   // dynamic shared memory raised for quantize_stream_kernel<1, 4, 8>
     // dynamic shared memory raised, per [group size index: 0 per-row, 1..4 GS 32..256][kernel: BX 16, 32,
     // 64, 128, wide]
     bool linear_attr[5][5] = {};
@@ -280,25 +282,6 @@ opq_status check_sizes(int64_t N, int64_t K) {
     return OPQ_OK;
 }
 
-template <int G, int V>
-void launch_quant(const uint16_t *w, int64_t N, int64_t K, int64_t ldw, const opqk::QuantParams &qp,
-                  uint32_t *codes, uint32_t *signs, float *scales, int grid, cudaStream_t st) {
-    opqk::quantize_kernel<G, V><<<grid, 256, 0, st>>>(w, N, K, ldw, qp, codes, signs, scales);
-}
-
-template <int G>
-void dispatch_quant(int vpl, const uint16_t *w, int64_t N, int64_t K, int64_t ldw, const opqk::QuantParams &qp,
-                    uint32_t *codes, uint32_t *signs, float *scales, int grid, cudaStream_t st) {
-    switch (vpl) {
-#define OPQ_Q(V) \
-    case V: launch_quant<G, V>(w, N, K, ldw, qp, codes, signs, scales, grid, st); break;
-        OPQ_Q(1) OPQ_Q(2) OPQ_Q(3) OPQ_Q(4) OPQ_Q(5) OPQ_Q(6) OPQ_Q(7) OPQ_Q(8)
-        OPQ_Q(9) OPQ_Q(10) OPQ_Q(11) OPQ_Q(12) OPQ_Q(13) OPQ_Q(14) OPQ_Q(15) OPQ_Q(16)
-#undef OPQ_Q
-        default: break;
-    }
-}
-
 constexpr int gs_index(int gs) { return gs == 0 ? 0 : gs == 32 ? 1 : gs == 64 ? 2 : gs == 128 ? 3 : 4; }
 
 template <int BX, int GS>
@@ -376,36 +359,93 @@ const char *opq_status_string(opq_status s) {
     return "OPQ_ERR_UNKNOWN";
 }
 
-opq_status opq_quantize(const uint16_t *w, int64_t N, int64_t K, int64_t ldw, float alpha, uint32_t *codes,
-                        uint32_t *signs, float *scales, void *stream) {
-    opq_status s = check_sizes(N, K);
-    if (s != OPQ_OK) return s;
-    if (K > 32768) return OPQ_ERR_UNSUPPORTED_SHAPE;
-    if (ldw < K || ldw % 8 != 0) return OPQ_ERR_INVALID_ARG;
+// The row-streaming quantize over a list of matrices: validation, then one launch per row-width
+// class (one, four or eight warps per row) and per QS_MAX_JOBS matrices of the class.
+extern "C++" {
+template <int G>
+static opq_status launch_quant_stream(DeviceInfo *di, const opq_quant_job *jobs, const std::vector<int64_t> &idx,
+                                      const opqk::QuantParams &qp, cudaStream_t st) {
+    using C = opqk::QsCfg<G>;
+    int64_t kmax = 0;
+    for (int64_t i : idx) kmax = jobs[i].K > kmax ? jobs[i].K : kmax;
+    // one slot holds one row of the widest matrix of the class
+    const int slot_bytes = (int)((2 * kmax + 127) / 128 * 128);
+    int nslots = C::RING_MAX / slot_bytes;
+    if (nslots > opqk::QS_MAX_SLOTS) nslots = opqk::QS_MAX_SLOTS;
+    if (nslots < 2) return OPQ_ERR_UNSUPPORTED_SHAPE;
+    const int smem = opqk::QS_OFF_RING + nslots * slot_bytes;
+    const int gi = G == 1 ? 0 : (G == 4 ? 1 : 2);
+    if (!di->stream_quant_attr[gi]) {
+        cudaError_t e = cudaFuncSetAttribute(opqk::quantize_stream_kernel<G>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             opqk::QS_OFF_RING + C::RING_MAX);
+        if (e != cudaSuccess) return cuda_fail(e);
+        di->stream_quant_attr[gi] = true;
+    }
+    static thread_local opqk::QsParams P;   // ~7 KB: kept off the stack
+    for (size_t c0 = 0; c0 < idx.size(); c0 += opqk::QS_MAX_JOBS) {
+        std::memset(&P, 0, sizeof P);
+        P.qp = qp;
+        P.nslots = nslots;
+        P.slot_bytes = slot_bytes;
+        const size_t n = idx.size() - c0 < (size_t)opqk::QS_MAX_JOBS ? idx.size() - c0 : (size_t)opqk::QS_MAX_JOBS;
+        int64_t rows = 0;
+        for (size_t i = 0; i < n; ++i) {
+            const opq_quant_job &J = jobs[idx[c0 + i]];
+            opqk::QsJob &q = P.job[i];
+            q.w = J.w;
+            q.codes = J.codes;
+            q.signs = J.signs;
+            q.scales = J.scales;
+            q.ldw = J.ldw;
+            q.N = (int32_t)J.N;
+            q.K = (int32_t)J.K;
+            q.row_begin = rows;
+            rows += J.N;
+        }
+        P.njobs = (int32_t)n;
+        P.rows = rows;
+        const int64_t groups = rows < (int64_t)di->sms * C::NG ? rows : (int64_t)di->sms * C::NG;
+        const int grid = (int)((groups + C::NG - 1) / C::NG);
+        opqk::quantize_stream_kernel<G><<<grid, opqk::QS_THREADS, smem, st>>>(P);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    return OPQ_OK;
+}
+}  // extern "C++"
+
+static opq_status quantize_jobs(const opq_quant_job *jobs, int64_t count, float alpha, void *stream) {
+    if (jobs == nullptr || count < 1) return OPQ_ERR_INVALID_ARG;
     if (!alpha_ok(alpha)) return OPQ_ERR_INVALID_ARG;
-    if ((s = check_ptrs({w, codes, signs, scales})) != OPQ_OK) return s;
+    for (int64_t i = 0; i < count; ++i) {
+        const opq_quant_job &J = jobs[i];
+        opq_status s = check_sizes(J.N, J.K);
+        if (s != OPQ_OK) return s;
+        if (J.K > 32768) return OPQ_ERR_UNSUPPORTED_SHAPE;
+        if (J.ldw < J.K || J.ldw % 8 != 0) return OPQ_ERR_INVALID_ARG;
+    }
+    for (int64_t i = 0; i < count; ++i) {
+        opq_status s = check_ptrs({jobs[i].w, jobs[i].codes, jobs[i].signs, jobs[i].scales});
+        if (s != OPQ_OK) return s;
+    }
+    DeviceInfo *di = nullptr;
+    opq_status s = device_info(&di);
+    if (s != OPQ_OK) return s;
     opqk::QuantParams qp{};
     const double inv = 1.0 / (double)alpha;
-    qp.t[0] = 0.0;
     for (int k = 1; k < 16; ++k) qp.t[k] = std::pow(((double)k - 0.5) / 15.0, inv);
     qp.alpha_is_one = (alpha == 1.0f) ? 1 : 0;
-    DeviceInfo *di = nullptr;
-    if ((s = device_info(&di)) != OPQ_OK) return s;
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    const int64_t nvec = K / 8;
-    if (K <= 4096) {
-        // one warp per row, two rows per block
-        const int64_t blocks = (N + opqk::QR_ROWS - 1) / opqk::QR_ROWS;
-        const int grid = (int)(blocks < (int64_t)di->sms * 32 ? blocks : (int64_t)di->sms * 32);
-        opqk::quantize_rows_kernel<<<grid, 64, 0, st>>>(w, N, K, ldw, qp, codes, signs, scales);
-    } else {
-        const int vpl = (int)((nvec + 255) / 256);
-        const int64_t blocks = N;
-        const int grid = (int)(blocks < (int64_t)di->sms * 8 ? blocks : (int64_t)di->sms * 8);
-        dispatch_quant<8>(vpl, w, N, K, ldw, qp, codes, signs, scales, grid, st);
+    std::vector<int64_t> cls[3];
+    for (int64_t i = 0; i < count; ++i) {
+        const int g = opqk::qs_group_warps(jobs[i].K);
+        cls[g == 1 ? 0 : (g == 4 ? 1 : 2)].push_back(i);
     }
-    cudaError_t e = cudaGetLastError();
-    return e == cudaSuccess ? OPQ_OK : cuda_fail(e);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (!cls[0].empty() && (s = launch_quant_stream<1>(di, jobs, cls[0], qp, st)) != OPQ_OK) return s;
+    if (!cls[1].empty() && (s = launch_quant_stream<4>(di, jobs, cls[1], qp, st)) != OPQ_OK) return s;
+    if (!cls[2].empty() && (s = launch_quant_stream<8>(di, jobs, cls[2], qp, st)) != OPQ_OK) return s;
+    return OPQ_OK;
 }
 
 // group-wise format: group size 32, 64, 128 or 256 dividing K
@@ -413,6 +453,16 @@ static opq_status check_group(int64_t K, int64_t gs) {
     if (gs != 32 && gs != 64 && gs != 128 && gs != 256) return OPQ_ERR_INVALID_ARG;
     if (K % gs != 0) return OPQ_ERR_UNSUPPORTED_SHAPE;
     return OPQ_OK;
+}
+
+opq_status opq_quantize_batched(const opq_quant_job *jobs, int64_t count, float alpha, void *stream) {
+    return quantize_jobs(jobs, count, alpha, stream);
+}
+
+opq_status opq_quantize(const uint16_t *w, int64_t N, int64_t K, int64_t ldw, float alpha, uint32_t *codes,
+                        uint32_t *signs, float *scales, void *stream) {
+    const opq_quant_job job = {w, N, K, ldw, codes, signs, scales};
+    return quantize_jobs(&job, 1, alpha, stream);
 }
 
 opq_status opq_quantize_grouped(const uint16_t *w, int64_t N, int64_t K, int64_t ldw, int64_t group_size,

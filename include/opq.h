@@ -71,6 +71,29 @@ opq_status opq_quantize(const uint16_t *w, int64_t N, int64_t K, int64_t ldw, fl
                         uint32_t *codes, uint32_t *signs, float *scales, void *stream);
 
 /*
+ * opq_quantize_batched — opq_quantize over a list of matrices in one pass: the card's
+ * whole-model quantization ("Quantize and save": every linear layer of the
+ * transformer) as one stream through HBM instead of one launch per matrix.
+ *   jobs    HOST array of `count` descriptors (count >= 1), read before the call
+ *           returns; each names a bf16 weight and its output planes, all device
+ *           memory, with the meaning, layout and limits of opq_quantize's arguments
+ *           (K % 32 == 0, K <= 32768, ldw >= K, ldw % 8 == 0, 16-byte aligned)
+ *   alpha   the power, shared by every matrix of the call
+ * Outputs are bit-identical to opq_quantize on each matrix. The work is dealt to
+ * one CTA per SM by rows (matrices of up to 128 per launch); a job's output planes
+ * must not overlap another job's. An invalid descriptor fails the whole call before
+ * anything is launched.
+ */
+typedef struct opq_quant_job {
+    const uint16_t *w;   /* bf16 [N, ldw] */
+    int64_t N, K, ldw;
+    uint32_t *codes;     /* [N, K/8] */
+    uint32_t *signs;     /* [N, K/32] */
+    float *scales;       /* [N] */
+} opq_quant_job;
+opq_status opq_quantize_batched(const opq_quant_job *jobs, int64_t count, float alpha, void *stream);
+
+/*
  * opq_dequantize — the card's "inference decoding": w' = sign * (q/15)^(1/alpha) * max.
  *   codes, signs, scales  packed weight as produced by opq_quantize (device)
  *   N, K                  as for opq_quantize

@@ -136,9 +136,10 @@ int main() {
             }
         }
     }
-    // --- code_table_run / table_pair: the quantize kernels' per-row code table. Thresholds
-    // nondecreasing (crowded, repeated, unreachable), every thread partition the kernels use;
-    // each entry against q(b) = #{k : T_k <= b}, each lookup against q(|w|) for every |w| <= mx
+    // --- the quantize kernel's per-row code table: built word by word from the level boundaries
+    // in stretches of 32 words (one per lane, as the kernel's ballots do), every entry against
+    // q(b) = #{k : T_k <= b}; and the lookup of every magnitude up to the max at several table
+    // offsets. Thresholds nondecreasing: spread, crowded, repeated, unreachable.
     {
         auto count_le = [](const uint16_t *T, int b) {
             uint32_t q = 0;
@@ -146,7 +147,7 @@ int main() {
             return q;
         };
         const uint32_t TAB = 4096;
-        std::vector<uint32_t> tabw(8 * TAB / 4);
+        std::vector<uint32_t> tabw(16 * TAB / 4);
         for (int trial = 0; trial < 600; ++trial) {
             uint32_t mx = (uint32_t)(rng() % 0x7F81u);
             if (trial % 9 == 0) mx = 0x7F80u;            // +inf max
@@ -167,29 +168,51 @@ int main() {
             const uint32_t dz = T1 <= mx ? mx - T1 + 1u : 0u;
             if (dz >= TAB) continue;                           // such rows take the search
             const uint32_t words = (dz + 4u) >> 2;
-            for (uint32_t P : {1u, 32u, 256u}) {
-                const uint32_t slot = (uint32_t)(rng() % 8u), base = slot * TAB;
+            int B[16];
+            for (int k = 1; k < 16; ++k) B[k] = (int)T[k] <= (int)mx ? (int)mx - (int)T[k] + 1 : 0;
+            CHECK((uint32_t)B[1] == dz, "B_1 != dz trial %d", trial);
+            for (uint32_t slot : {0u, 7u, 15u}) {
+                const uint32_t base = slot * TAB;
+                if (base + 0x7F80u >= 0x10000u) continue;      // the kernels keep max + base below 2^16
                 std::fill(tabw.begin(), tabw.end(), 0xEEEEEEEEu);
-                const uint32_t per = (words + P - 1u) / P;
-                for (uint32_t g = 0; g < P; ++g) {
-                    const uint32_t w0 = g * per, w1 = std::min(w0 + per, words);
-                    code_table_run(T, mx, w0, w1, &tabw[base / 4]);
-                }
                 const uint8_t *tb = reinterpret_cast<const uint8_t *>(tabw.data());
+                for (uint32_t i0 = 0; i0 < words; i0 += 32u) {
+                    const int lo = (int)(4u * i0), hi = lo + 127;
+                    uint32_t c_full = 0;
+                    int inside[16], n_in = 0;
+                    for (int k = 1; k < 16; ++k) {
+                        if (B[k] > hi) ++c_full;
+                        else if (B[k] > lo) inside[n_in++] = B[k];
+                    }
+                    for (uint32_t w = i0; w < std::min(i0 + 32u, words); ++w)
+                        tabw[base / 4 + w] = table_word_from_bounds(c_full, inside, n_in, w) * 0x11u;
+                }
                 for (uint32_t e = 0; e < 4u * words; ++e)
-                    CHECK(tb[base + e] == count_le(T, (int)mx - (int)e), "code_table_run trial %d P %u e %u got %u want %u",
-                          trial, P, e, tb[base + e], count_le(T, (int)mx - (int)e));
-                const uint32_t mmb = (mx + base) * 0x00010001u, dzb = (dz + base) * 0x00010001u;
+                    CHECK(tb[base + e] == 17u * count_le(T, (int)mx - (int)e), "table trial %d base %u e %u got %u want %u",
+                          trial, base, e, tb[base + e], 17u * count_le(T, (int)mx - (int)e));
+                const uint32_t mmb = (mx + base) * 0x00010001u, lo2 = (mx - dz) * 0x00010001u;
                 const uint32_t step = mx > 20000u ? 7u : 1u;
                 for (uint32_t a = 0; a <= mx; a += step) {
                     const uint32_t a2 = (uint32_t)(rng() % (mx + 1u));
-                    const uint32_t x = a | (a2 << 16) | ((uint32_t)(rng() & 1u) << 15) | ((uint32_t)(rng() & 1u) << 31);
-                    const uint32_t q = table_pair(tb, x, mmb, dzb);
-                    const uint32_t want = count_le(T, (int)a) | (count_le(T, (int)a2) << 16);
-                    CHECK(q == want, "table_pair trial %d a %x a2 %x got %x want %x", trial, a, a2, q, want);
+                    const uint32_t b = table_byte_clamped(tb, a | (a2 << 16), lo2, mmb);
+                    CHECK(b == (count_le(T, (int)a) | (count_le(T, (int)a2) << 4)), "table_byte_clamped %x %x mx %x",
+                          a, a2, mx);
                 }
             }
         }
+    }
+    // bf16x2_max on non-negative finite halves: the larger bit pattern
+    for (int t = 0; t < 200000; ++t) {
+        const uint32_t a = (uint32_t)(rng() % 0x7F81u), b = (uint32_t)(rng() % 0x7F81u);
+        const uint32_t c = (uint32_t)(rng() % 0x7F81u), d = (uint32_t)(rng() % 0x7F81u);
+        const uint32_t r = bf16x2_max(a | (c << 16), b | (d << 16));
+        CHECK(r == (std::max(a, b) | (std::max(c, d) << 16)), "bf16x2_max %x %x %x %x -> %x", a, b, c, d, r);
+    }
+    // codes_word: byte p of the word is the low byte of b_p
+    for (int t = 0; t < 1000; ++t) {
+        const uint32_t b[4] = {(uint32_t)rng(), (uint32_t)rng(), (uint32_t)rng(), (uint32_t)rng()};
+        const uint32_t want = (b[0] & 0xFFu) | ((b[1] & 0xFFu) << 8) | ((b[2] & 0xFFu) << 16) | ((b[3] & 0xFFu) << 24);
+        CHECK(codes_word(b[0], b[1], b[2], b[3]) == want, "codes_word %x %x %x %x", b[0], b[1], b[2], b[3]);
     }
     std::printf("%s fails=%d\n", fails ? "FAIL" : "OK", fails);
     return fails ? 1 : 0;
