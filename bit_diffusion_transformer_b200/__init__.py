@@ -32,7 +32,7 @@ EXPORTS = ["opq_quantize", "opq_dequantize", "opq_linear_workspace_size", "opq_l
            "opq_linear_grouped", "opq_linear_grouped_workspace_size", "opq_linear_fused",
            "opq_linear_grouped_fused", "opq_alpha_search", "opq_alpha_search_workspace_size",
            "opq_quantize_bits", "opq_dequantize_bits", "opq_set_wait_limit_ns",
-           "opq_quantize_batched"]
+           "opq_quantize_batched", "opq_linear_bits", "opq_linear_bits_workspace_size"]
 ACTIVATIONS = {"none": 0, "silu": 1, "gelu_tanh": 2}
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
@@ -76,13 +76,15 @@ def load(path: str = LIB_PATH):
     lib.opq_linear_grouped_fused.argtypes = [P, I, I, P, P, P, I, I, F, P, ctypes.c_int, P, P, S, P]
     lib.opq_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
     lib.opq_quantize_batched.argtypes = [P, I, F, P]
+    lib.opq_linear_bits.argtypes = [P, I, I, P, P, P, I, ctypes.c_int32, F, P, P, S, P]
+    lib.opq_linear_bits_workspace_size.argtypes = [I, I, I, ctypes.c_int32, ctypes.POINTER(S)]
     lib.opq_status_string.argtypes = [ctypes.c_int]
     lib.opq_status_string.restype = ctypes.c_char_p
     for f in ("opq_quantize", "opq_dequantize", "opq_linear_workspace_size", "opq_linear", "opq_linear_plan",
               "opq_linear_noalloc", "opq_device_error", "opq_quantize_grouped", "opq_dequantize_grouped", "opq_linear_grouped",
               "opq_linear_grouped_workspace_size", "opq_linear_fused", "opq_linear_grouped_fused",
               "opq_alpha_search", "opq_alpha_search_workspace_size", "opq_quantize_bits", "opq_dequantize_bits",
-              "opq_set_wait_limit_ns", "opq_quantize_batched"):
+              "opq_set_wait_limit_ns", "opq_quantize_batched", "opq_linear_bits", "opq_linear_bits_workspace_size"):
         getattr(lib, f).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -298,6 +300,30 @@ def dequantize_bits(codes: torch.Tensor, signs: torch.Tensor, scales: torch.Tens
     _check(load().opq_dequantize_bits(_ptr(codes), _ptr(signs), _ptr(scales), N, K, int(bits), float(alpha), _ptr(w),
                                       _stream(codes.device)), "opq_dequantize_bits")
     return w
+
+
+def bits_workspace_size(M: int, N: int, K: int, bits: int) -> int:
+    b = ctypes.c_size_t(0)
+    _check(load().opq_linear_bits_workspace_size(M, N, K, int(bits), ctypes.byref(b)), "opq_linear_bits_workspace_size")
+    return int(b.value)
+
+
+def linear_bits(x: torch.Tensor, codes: torch.Tensor, signs: torch.Tensor, scales: torch.Tensor, bits: int,
+                alpha: float = ALPHA, out=None, workspace=None):
+    """y = x @ W'^T for a W[N, K] packed with `bits`-bit magnitudes (3..6, codes int32 [N, K*bits/32])."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2
+    _need_cuda(x, codes, signs, scales)
+    M, K = x.shape
+    N = codes.shape[0]
+    y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    need = bits_workspace_size(M, N, K, bits)
+    if need and workspace is None:
+        workspace = torch.zeros((need,), dtype=torch.uint8, device=x.device)   # must start zeroed
+    ws_ptr = _ptr(workspace) if workspace is not None else ctypes.c_void_p(0)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(load().opq_linear_bits(_ptr(x), M, K, _ptr(codes), _ptr(signs), _ptr(scales), N, int(bits), float(alpha),
+                                  _ptr(y), ws_ptr, ws_bytes, _stream(x.device)), "opq_linear_bits")
+    return y
 
 
 ALPHA_GRID = tuple(round(0.30 + 0.05 * i, 2) for i in range(15))   # 0.30 .. 1.00

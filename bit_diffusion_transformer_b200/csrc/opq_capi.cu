@@ -72,6 +72,7 @@ struct DeviceInfo {
     // dynamic shared memory raised, per [group size index: 0 per-row, 1..4 GS 32..256][kernel: BX 16, 32,
     // 64, 128, wide]
     bool linear_attr[5][5] = {};
+    bool bits_attr[3] = {};           // the wide kernel at 3, 5 and 6 bits
 };
 std::mutex g_mu;
 DeviceInfo g_dev[64];
@@ -284,6 +285,24 @@ opq_status check_sizes(int64_t N, int64_t K) {
 
 constexpr int gs_index(int gs) { return gs == 0 ? 0 : gs == 32 ? 1 : gs == 64 ? 2 : gs == 128 ? 3 : 4; }
 
+// A linear kernel launch that lets the next programmatically launched kernel of the stream start
+// its global-memory-free set-up while this one finishes (the kernels wait for their predecessor
+// before touching global memory: opq_device.cuh, pdl_wait).
+template <class Kern, class... Args>
+cudaError_t launch_programmatic(Kern kernel, int grid, int threads, int smem, cudaStream_t st, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3((unsigned)threads);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 template <int BX, int GS>
 cudaError_t launch_linear(DeviceInfo *di, const Plan &plan, const CUtensorMap &xmap, const CUtensorMap &xhmap,
                           const CUtensorMap &cmap, const CUtensorMap &smap, const opqk::LinearArgs &a,
@@ -296,16 +315,17 @@ cudaError_t launch_linear(DeviceInfo *di, const Plan &plan, const CUtensorMap &x
         if (e != cudaSuccess) return e;
         di->linear_attr[gs_index(GS)][key] = true;
     }
-    opqk::linear_kernel<BX, GS><<<plan.grid, C::THREADS, C::SMEM_BYTES, st>>>(xmap, xhmap, cmap, smap, a);
-    return cudaGetLastError();
+    cudaError_t e = launch_programmatic(opqk::linear_kernel<BX, GS>, plan.grid, C::THREADS, C::SMEM_BYTES, st, xmap,
+                                        xhmap, cmap, smap, a);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 // the wide-tile kernel (256 activation rows per tile, whole tiles, one block per copy)
-template <int GS>
+template <int GS, int BITS = 4>
 cudaError_t launch_linear_wide(DeviceInfo *di, const Plan &plan, const CUtensorMap &xmap, const CUtensorMap &xhmap,
                                const CUtensorMap &cmap, const CUtensorMap &smap, const opqk::LinearArgs &n,
                                cudaStream_t st) {
-    using C = opqk_wide::Cfg<256>;
+    using C = opqk_wide::Cfg<256, BITS>;
     if (plan.mode != 0) return cudaErrorInvalidValue;   // the wide kernel runs whole-tile schedules only
     opqk_wide::LinearArgs a{};
     a.signs = n.signs;
@@ -328,14 +348,17 @@ cudaError_t launch_linear_wide(DeviceInfo *di, const Plan &plan, const CUtensorM
     a.bias = n.bias;
     a.act = n.act;
     for (int q = 0; q < 16; ++q) a.lutf[q] = n.lutf[q];
-    if (!di->linear_attr[gs_index(GS)][4]) {
-        cudaError_t e = cudaFuncSetAttribute(opqk_wide::wide_kernel<256, GS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             C::SMEM_BYTES);
+    for (int q = 0; q < 64; ++q) a.lutb[q] = n.lutb[q];
+    bool &attr = BITS == 4 ? di->linear_attr[gs_index(GS)][4] : di->bits_attr[BITS == 3 ? 0 : BITS - 4];
+    if (!attr) {
+        cudaError_t e = cudaFuncSetAttribute(opqk_wide::wide_kernel<256, GS, BITS>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
         if (e != cudaSuccess) return e;
-        di->linear_attr[gs_index(GS)][4] = true;
+        attr = true;
     }
-    opqk_wide::wide_kernel<256, GS><<<plan.grid, C::THREADS, C::SMEM_BYTES, st>>>(xmap, xhmap, cmap, smap, a);
-    return cudaGetLastError();
+    cudaError_t e = launch_programmatic(opqk_wide::wide_kernel<256, GS, BITS>, plan.grid, C::THREADS, C::SMEM_BYTES, st,
+                                        xmap, xhmap, cmap, smap, a);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace
@@ -822,6 +845,87 @@ opq_status opq_linear_grouped_fused(const uint16_t *x, int64_t M, int64_t K, con
     if (group_size == 0) return OPQ_ERR_INVALID_ARG;
     return linear_impl(x, M, K, codes, signs, nullptr, gmax, group_size, N, alpha, bias, activation, y, workspace,
                        workspace_bytes, stream);
+}
+
+static opq_status check_bits_linear(int64_t M, int64_t N, int64_t K, int32_t bits) {
+    if (M < 1) return OPQ_ERR_INVALID_ARG;
+    opq_status s = check_sizes(N, K);
+    if (s != OPQ_OK) return s;
+    if (bits < 3 || bits > 6) return OPQ_ERR_INVALID_ARG;
+    if (M > INT32_MAX) return OPQ_ERR_UNSUPPORTED_SHAPE;
+    // a 128-K block of a row is 4 bits words, copied whole by the tensor copies
+    if (bits != 4 && K % 128 != 0) return OPQ_ERR_UNSUPPORTED_SHAPE;
+    return OPQ_OK;
+}
+
+opq_status opq_linear_bits_workspace_size(int64_t M, int64_t N, int64_t K, int32_t bits, size_t *bytes) {
+    if (!bytes) return OPQ_ERR_INVALID_ARG;
+    opq_status s = check_bits_linear(M, N, K, bits);
+    if (s != OPQ_OK) return s;
+    *bytes = bits == 4 ? make_plan(M, N, K).ws_bytes : make_plan(M, N, K, true).ws_bytes;
+    return OPQ_OK;
+}
+
+opq_status opq_linear_bits(const uint16_t *x, int64_t M, int64_t K, const uint32_t *codes, const uint32_t *signs,
+                           const float *scales, int64_t N, int32_t bits, float alpha, uint16_t *y, void *workspace,
+                           size_t workspace_bytes, void *stream) {
+    opq_status s = check_bits_linear(M, N, K, bits);
+    if (s != OPQ_OK) return s;
+    if (bits == 4) return opq_linear(x, M, K, codes, signs, scales, N, alpha, y, workspace, workspace_bytes, stream);
+    if (!alpha_ok(alpha)) return OPQ_ERR_INVALID_ARG;
+    if ((s = check_ptrs({x, codes, signs, scales, y})) != OPQ_OK) return s;
+    const Plan plan = make_plan(M, N, K, true);
+    if (plan.ws_bytes > 0) {
+        if (workspace == nullptr || workspace_bytes < plan.ws_bytes) return OPQ_ERR_WORKSPACE;
+        if ((s = check_ptrs({workspace})) != OPQ_OK) return s;
+    }
+    DeviceInfo *di = nullptr;
+    if ((s = device_info(&di)) != OPQ_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    opqk::LinearArgs a{};
+    a.signs = signs;
+    a.scales = scales;
+    a.y = y;
+    a.counters = reinterpret_cast<uint32_t *>(workspace);
+    a.ws = plan.ws_bytes ? reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(workspace) + plan.counter_bytes)
+                         : nullptr;
+    a.M = (int)M;
+    a.N = (int)N;
+    a.K = (int)K;
+    a.m_tiles = plan.m_tiles;
+    a.n_tiles = plan.n_tiles;
+    a.kblocks = plan.kblocks;
+    a.ngroups = plan.ngroups;
+    a.mode = plan.mode;
+    a.runs_max = plan.runs_max;
+    a.tail_split = plan.tail_split;
+    a.signs_tma = 1;
+    a.act = OPQ_ACT_NONE;
+    {
+        const int L = (1 << bits) - 1;
+        const double inv = 1.0 / (double)alpha;
+        for (int q = 0; q <= L; ++q) a.lutb[q] = host_bf16(std::pow((double)q / (double)L, inv));
+    }
+    CUtensorMap xmap, xhmap, cmap, smap;
+    if ((s = make_x_map(&xmap, x, M, K, (uint32_t)plan.bx)) != OPQ_OK) return s;
+    if ((s = make_u32_map(&cmap, codes, N, K * bits / 32, 4u * (uint32_t)bits, 128u, CU_TENSOR_MAP_SWIZZLE_NONE)) !=
+        OPQ_OK)
+        return s;
+    if ((s = make_u32_map(&smap, signs, N, K / 32, 4u, 128u, CU_TENSOR_MAP_SWIZZLE_NONE)) != OPQ_OK) return s;
+    if (a.tail_split == 2) {
+        if ((s = make_x_map(&xhmap, x, M, K, (uint32_t)plan.bx / 2)) != OPQ_OK) return s;
+    } else {
+        xhmap = xmap;   // not read by the kernel
+    }
+    cudaError_t e;
+    switch (bits) {
+        case 3: e = launch_linear_wide<0, 3>(di, plan, xmap, xhmap, cmap, smap, a, st); break;
+        case 5: e = launch_linear_wide<0, 5>(di, plan, xmap, xhmap, cmap, smap, a, st); break;
+        default: e = launch_linear_wide<0, 6>(di, plan, xmap, xhmap, cmap, smap, a, st); break;
+    }
+    if (e != cudaSuccess) return cuda_fail(e);
+    e = cudaGetLastError();
+    return e == cudaSuccess ? OPQ_OK : cuda_fail(e);
 }
 
 opq_status opq_linear_grouped_workspace_size(int64_t M, int64_t N, int64_t K, int64_t group_size, size_t *bytes) {

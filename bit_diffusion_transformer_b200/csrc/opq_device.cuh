@@ -86,6 +86,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
     }
 }
 
+// ------------------------------------------- programmatic dependent launch --
+// The linear kernels are launched so that the next kernel of the stream that was launched the
+// same way may start while they finish: every CTA signals it at entry, and every thread waits for
+// the previous kernel of the stream (its completion and the visibility of its writes) before its
+// first access to global memory. Work before the wait (barrier set-up, tensor-memory allocation,
+// the decode table) touches no global memory, so it may overlap the previous kernel's last CTAs.
+// Both are no-ops for a kernel launched without the programmatic attribute.
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ----------------------------------------------------------------------- TMA --
 __device__ __forceinline__ void tma_prefetch_desc(const void *tmap) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");

@@ -14,14 +14,13 @@
 // activation rows. Per CTA (one per SM, persistent):
 //   warp 0       raw producer: codes (64-byte swizzle) and signs of 128 weight rows,
 //                one load group (GRP consecutive 128-K blocks) per pair of TMA copies
-//   warp 1       TMEM allocation and MMA issue (chain 0); A comes from TMEM
+//   warp 1       TMEM allocation and MMA issue (every accumulation chain); A comes from TMEM
 //   warp 2       x producer: the load group's x (BX rows, 128-byte swizzle), one copy
 //   warps 3..14  three decoder groups of 4 warps (= the 128 TMEM lanes): each thread owns
 //                one weight row and decodes 128 weights per block through the shared-memory
 //                pair table (opq_bits.h), written to TMEM with tcgen05.st as the A operand
 //   warps 15..18 epilogue: accumulator TMEM -> registers -> * scale[n] -> bf16 y,
 //                or fp32 partial sums for tiles split across CTAs
-//   warps 19..   the other accumulation chains' MMA issuers (narrow tiles)
 // TMEM columns: [0, A_COLS) the A ring; then NACC accumulator buffers of NCHAIN x BX.
 //
 // Work is a list of runs (tile, range of load groups). Mode 1 (stream-K) cuts the
@@ -137,6 +136,7 @@ struct LinearArgs {
     int tail_split;         // mode 0: 2 = tiles past the last full wave run as two half-width
                             // (BX/2 activation rows) runs on different CTAs; 1 = whole tiles
     uint16_t lut[16];       // bf16 (q/15)^(1/alpha)
+    uint16_t lutb[64];      // other bit widths (wide kernel): bf16 (q/L)^(1/alpha), q = 0..L, L = 2^bits - 1
     // group-wise format (GS > 0)
     const uint16_t *gmax;   // float16 [N, K / GS]
     int ngk;                // groups per row (K / GS)
@@ -148,16 +148,26 @@ struct LinearArgs {
 
 enum { EPI_NONE = 0, EPI_SILU = 1, EPI_GELU_TANH = 2 };
 
+// tanh by the hardware approximation (tanh.approx.f32, absolute error about 5e-4), one MUFU op
+__device__ __forceinline__ float tanh_hw(float x) {
+    float y;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // One output before its bf16 rounding: the fp32 sum times the row scale, plus the bias, through
-// the activation (SiLU v / (1 + e^-v); GELU's tanh form 0.5 v (1 + tanh(sqrt(2/pi) (v + 0.044715
-// v^3)))). With no bias and no activation this is the plain product acc * scale.
+// the activation. SiLU v / (1 + e^-v) = v (1/2 + tanh(v/2) / 2); GELU's tanh form
+// 0.5 v (1 + tanh(sqrt(2/pi) (v + 0.044715 v^3))). Both take one hardware tanh, so the epilogue
+// that the next tile's MMAs wait for stays short; the approximation's error (at most about
+// 2.5e-4 |v| in the output) is far inside the linear's tolerance. With no bias and no
+// activation this is the plain product acc * scale.
 __device__ __forceinline__ float epi_value(float acc, float scale, float bias, int act) {
-    float v = acc * scale;
-    if (bias != 0.0f) v += bias;
+    float v = fmaf(acc, scale, bias);
     if (act == EPI_SILU) {
-        v = v / (1.0f + expf(-v));
+        v = v * fmaf(0.5f, tanh_hw(0.5f * v), 0.5f);
     } else if (act == EPI_GELU_TANH) {
-        v = 0.5f * v * (1.0f + tanhf(0.7978845608028654f * (v + 0.044715f * v * v * v)));
+        const float u = 0.7978845608028654f * fmaf(0.044715f * v, v * v, v);
+        v = 0.5f * v * (1.0f + tanh_hw(u));
     }
     return v;
 }
@@ -316,12 +326,17 @@ struct Cfg {
     // (blk - GROUPS) was loaded, so the stage's previous phase (block blk - RAW_STAGES) must
     // be at least that old for the parity test to be exact
     static_assert(RAW_STAGES >= GROUPS, "raw ring shorter than the decoder rotation");
+    // a decoder waits for block b - A_BLOCKS on blk_done knowing only that its own previous wait
+    // (block b - GROUPS - A_BLOCKS) succeeded; the parity test is exact only if that implies block
+    // b - A_BLOCKS - NDONE has completed, i.e. NDONE >= GROUPS (completions come in block order)
+    static_assert(NDONE >= GROUPS, "done ring shorter than the decoder rotation");
     static constexpr int WARP_LOAD = 0, WARP_MMA = 1, WARP_XLOAD = 2, WARP_DEC0 = 3, NUM_DEC_WARPS = 4 * GROUPS;
     static constexpr int WARP_EPI0 = WARP_DEC0 + NUM_DEC_WARPS;
-    // One MMA-issuing thread per accumulation chain: a thread issues one tcgen05.mma every
-    // few dozen cycles, far slower than the tensor pipe runs a narrow (N <= 64) MMA, so the
-    // chains are issued from separate warps (warp 1, then warps WARP_ISS1...).
-    static constexpr int NISS = NCHAIN;
+    // One MMA-issuing thread for all the chains: consecutive K-steps go to different chains, so
+    // no MMA waits for its predecessor's result, and one tcgen05.commit per block covers them all
+    // (a commit stalls the tensor pipe for a few hundred cycles; per-chain issuer threads needed
+    // one commit each, and measured ~0.65 us per 128-K block at BX = 16 against ~0.3 us of decode)
+    static constexpr int NISS = 1;
     static constexpr int WARP_ISS1 = WARP_EPI0 + 4;
     static constexpr int THREADS = (WARP_ISS1 + NISS - 1) * 32;
     static_assert(SMEM_BYTES <= 232448, "shared memory");
@@ -360,6 +375,7 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
     const int tiles = args.m_tiles * args.n_tiles;
     const bool signs_by_tma = args.signs_tma != 0;
 
+    if (threadIdx.x == 0) pdl_launch_dependents();
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::RAW_STAGES; ++s) {
             // the copies' expect_tx arrival, plus 32 cp.async arrivals when signs are copied by threads
@@ -402,6 +418,7 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
     if (warp == C::WARP_LOAD) {
         // ----------------------------------------------------------- raw producer
         // one stage per load group: GRP blocks of codes and of signs
+        pdl_wait();
         const int swd = args.K / 32;        // sign words per row
         int rs = 0;
         uint32_t rph = 0;
@@ -468,6 +485,7 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
         }
     } else if (warp == C::WARP_XLOAD) {
         // ----------------------------------------------------------- x producer
+        pdl_wait();
         if (lane == 0) {
             int b = 0;                 // the CTA's block index
             int v = 0;                 // the CTA's load-group index
@@ -511,10 +529,10 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
             }
         }
     } else if (warp == C::WARP_MMA || warp >= C::WARP_ISS1) {
-        // ----------------------------------------------------------- MMA issuers
-        // Issuer i accumulates K-steps k = i, i + NISS, ... of every 64-K half into chain i.
+        // ----------------------------------------------------------- MMA issuer
+        // The run's i-th MMA (K-step k of a 64-K half) accumulates into chain i % NCHAIN (= k % NCHAIN,
+        // NCHAIN divides the 4 K-steps of a half); a chain's first MMA of the run starts it afresh.
         if (lane == 0) {
-            const int iss = warp == C::WARP_MMA ? 0 : warp - C::WARP_ISS1 + 1;
             int ab = 0;
             uint32_t abph = 0;
             int as0 = 0, xs = 0, ds = 0;       // A half-stage of the block's first half, x stage, blk_done slot
@@ -526,8 +544,8 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
                 const uint32_t idesc = R.xrows == BX ? idesc_full : idesc_half;
                 if (!mbar_wait(&acc_empty[ab], abph ^ 1)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + C::A_COLS + ab * C::ACC_COLS + iss * BX;
-                uint32_t acc = 0;              // 0 for the chain's first MMA of the run
+                const uint32_t d_base = tmem_base + C::A_COLS + ab * C::ACC_COLS;
+                uint32_t started = 0;          // MMAs of this run issued so far
                 for (int g = R.g0; g < R.g1 && ok; ++g) {
                     const int nb = lg.start(g + 1) - lg.start(g);
                     if (!mbar_wait(&x_full[xs], xph)) { ok = false; break; }
@@ -541,14 +559,13 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
                         for (int h = 0; h < 2; ++h) {
                             const uint32_t a_tmem = tmem_base + (as0 + h) * 32;
                             const uint64_t bdesc = smem_desc_sw128(xbase + (2 * jj + h) * C::X_HALF_BYTES);
-                            // K-steps iss, iss + NISS, ...: a fixed count per issuer and no branch
-                            // between the MMAs (a branch around tcgen05.mma costs the issuing
-                            // thread far more than the MMA itself)
+                            // a fixed count of MMAs and no branch between them (a branch around
+                            // tcgen05.mma costs the issuing thread far more than the MMA itself)
 #pragma unroll
-                            for (int t = 0; t < C::KA / 16 / C::NISS; ++t) {
-                                const int k = iss + t * C::NISS;
-                                umma_bf16_ts(d_tmem, a_tmem + 8 * k, bdesc + 2 * k, idesc, acc);
-                                acc = 1;
+                            for (int k = 0; k < C::KA / 16; ++k) {
+                                umma_bf16_ts(d_base + (uint32_t)((k % C::NCHAIN) * BX), a_tmem + 8 * k, bdesc + 2 * k,
+                                             idesc, started >= (uint32_t)C::NCHAIN ? 1u : 0u);
+                                ++started;
                             }
                         }
                         if (!ok) break;
@@ -581,6 +598,7 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
         }
         // all decoder warps (named barrier 1) see the whole table before decoding
         asm volatile("bar.sync 1, %0;" ::"r"(C::NUM_DEC_WARPS * 32) : "memory");
+        pdl_wait();   // the group-wise scales are read from global memory
         const int g_dec = (warp - C::WARP_DEC0) >> 2;    // decoder group
         const int q = warp & 3;                          // TMEM lane quarter this warp may access
         const int row = q * 32 + lane;                   // weight row in the tile = TMEM lane
@@ -676,6 +694,7 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
         }
     } else {
         // ----------------------------------------------------------- epilogue
+        pdl_wait();
         const int q = warp & 3;
         const int row = q * 32 + lane;
         const int64_t U = (int64_t)tiles * args.ngroups;

@@ -42,6 +42,7 @@ struct LinearArgs {
                             // (BX/2 activation rows) runs on two CTAs; 3 = each runs as two
                             // half-K runs on two CTAs whose partial sums meet in `ws`; 1 = whole
     uint16_t lut[16];       // bf16 (q/15)^(1/alpha)
+    uint16_t lutb[64];      // other bit widths: bf16 (q/L)^(1/alpha), q = 0..L, L = 2^BITS - 1
     // group-wise format (GS > 0)
     const uint16_t *gmax;   // float16 [N, K / GS]
     int ngk;                // groups per row (K / GS)
@@ -111,12 +112,16 @@ struct RunIter {
     }
 };
 
-template <int BX>
+// BITS: bits per magnitude code. 4 is the nibble format, decoded two weights per lookup of the
+// pair table; 3, 5 and 6 are per-row bit streams (element k at bits k*BITS .. k*BITS + BITS - 1
+// of the row's words), decoded one code at a time.
+template <int BX, int BITS = 4>
 struct Cfg {
     static constexpr int BW = 128;                     // weight rows per tile (MMA M)
     static constexpr int KR = 128;                     // K per raw (codes/signs) stage
     static constexpr int KA = 64;                      // K per A stage (TMEM) and per x stage (smem)
-    static constexpr int RAW_STAGES = BX >= 256 ? 3 : (BX >= 128 ? 4 : 6);
+    // the 5- and 6-bit stages are larger: two of them keep the shared memory within bounds
+    static constexpr int RAW_STAGES = BITS >= 5 ? 2 : (BX >= 256 ? 3 : (BX >= 128 ? 4 : 6));
     static constexpr int A_STAGES = 8;                 // 32 TMEM columns each (64 K of bf16 pairs)
     static constexpr int A_BLOCKS = A_STAGES / 2;      // 128-K blocks of A held in TMEM
     static constexpr int A_COLS = A_STAGES * 32;
@@ -133,7 +138,8 @@ struct Cfg {
     static constexpr int ACC_COLS = NCHAIN * BX;       // one accumulator buffer (all chains)
     static constexpr int NACC = (A_COLS + 2 * ACC_COLS <= 512) ? 2 : 1;   // accumulator buffers
     static constexpr uint32_t TMEM_COLS = 512;
-    static constexpr int RAW_CODE_BYTES = BW * KR / 2;    // 8 KiB: [128 rows][16 words], 64-byte swizzle
+    static constexpr int RAW_CODE_BYTES = BW * KR * BITS / 8;   // [128 rows][4 BITS words] (4 bits: 64-byte swizzle)
+    static constexpr int CODE_WORDS = KR * BITS / 32;           // code words per row and block
     static constexpr int RAW_SIGN_BYTES = BW * KR / 8;    // 2 KiB: [128 rows][4 words]
     static constexpr int RAW_BYTES = RAW_CODE_BYTES + RAW_SIGN_BYTES;
     static constexpr int X_HALF_BYTES = BX * KA * 2;   // one 64-K half: BX rows x 128 bytes, 128-byte swizzle
@@ -154,6 +160,10 @@ struct Cfg {
     // (blk - GROUPS) was loaded, so the stage's previous phase (block blk - RAW_STAGES) must
     // be at least that old for the parity test to be exact
     static_assert(RAW_STAGES >= GROUPS, "raw ring shorter than the decoder rotation");
+    // a decoder waits for block b - A_BLOCKS on blk_done knowing only that its own previous wait
+    // (block b - GROUPS - A_BLOCKS) succeeded; the parity test is exact only if that implies block
+    // b - A_BLOCKS - NDONE has completed, i.e. NDONE >= GROUPS (completions come in block order)
+    static_assert(NDONE >= GROUPS, "done ring shorter than the decoder rotation");
     static constexpr int WARP_LOAD = 0, WARP_MMA = 1, WARP_XLOAD = 2, WARP_DEC0 = 3, NUM_DEC_WARPS = 4 * GROUPS;
     static constexpr int WARP_EPI0 = WARP_DEC0 + NUM_DEC_WARPS;
     // One MMA-issuing thread per accumulation chain: a thread issues one tcgen05.mma every
@@ -177,12 +187,39 @@ struct Cfg {
 // GS = 32 .. 256: one float16 max per GS weights of a row (the group-wise format); the
 // decoders form each group's 16 magnitudes bf16(LUT[q] * max) in registers and decode by
 // byte-plane lookups, and the epilogue applies no scale.
-template <int BX, int GS = 0>
-__global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
+// One 64-K half of a weight row in a BITS-bit stream (its 2 BITS code words in cw, its two sign
+// words in sw) -> the 64 weights sign * bf16 LUT[q] as 32 bf16 pairs, pair P (weights 2P, 2P + 1)
+// in o[P / 16][P % 16]. The table entry of code q holds LUT[q] in both halves (one copy per lane
+// at byte 256 q + 4 lane); the sign spreads are the pair table's (opq_bits.h).
+template <int BITS, class Load>
+__device__ __forceinline__ void decode_half_bits(const uint32_t (&cw)[2 * BITS], const uint32_t (&sw)[2], uint32_t lw,
+                                                 uint32_t lw2, Load load, uint32_t (&o)[2][16]) {
+    constexpr uint32_t MASK = (1u << BITS) - 1u;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {          // sign byte j: weights 8j .. 8j + 7
+        const uint32_t x = load(opqbits::prmt(sw[j >> 2], lw2, 0x5504u | ((uint32_t)(j & 3) << 4)));
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {      // pair 4j + e
+            uint32_t m[2];
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                const int bit = (8 * j + 2 * e + t) * BITS, wi = bit >> 5, sh = bit & 31;
+                const uint32_t q = (sh + BITS <= 32) ? ((cw[wi] >> sh) & MASK)
+                                                     : (__funnelshift_r(cw[wi], cw[(wi + 1) % (2 * BITS)], sh) & MASK);
+                m[t] = load((q << 8) | lw);
+            }
+            o[j >> 2][(j & 3) * 4 + e] = __byte_perm(m[0], m[1], 0x7610u) ^ ((x << e) & 0x80008000u);
+        }
+    }
+}
+
+template <int BX, int GS = 0, int BITS = 4>
+__global__ void __launch_bounds__(Cfg<BX, BITS>::THREADS, 1)
     wide_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_xh,
                   const __grid_constant__ CUtensorMap tmap_codes, const __grid_constant__ CUtensorMap tmap_signs,
                   const __grid_constant__ LinearArgs args) {
-    using C = Cfg<BX>;
+    using C = Cfg<BX, BITS>;
+    static_assert(BITS == 4 || GS == 0, "the other bit widths take per-row scales");
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t sbase = smem_u32(smem);
     if ((sbase & 1023u) != 0u) {   // the same for every CTA: nothing has been started yet
@@ -215,7 +252,7 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
     // one 128-K block of codes and signs (signs by TMA) into raw stage rs
     auto issue_raw = [&](int rs, int r, int n_blk) {
         mbar_arrive_expect_tx(&raw_full[rs], C::RAW_BYTES);
-        tma_load_2d(smem + C::OFF_RAW + rs * C::RAW_BYTES, &tmap_codes, r * (C::KR / 8), n_blk * C::BW, &raw_full[rs]);
+        tma_load_2d(smem + C::OFF_RAW + rs * C::RAW_BYTES, &tmap_codes, r * C::CODE_WORDS, n_blk * C::BW, &raw_full[rs]);
         tma_load_2d(smem + C::OFF_RAW + rs * C::RAW_BYTES + C::RAW_CODE_BYTES, &tmap_signs, r * (C::KR / 32),
                     n_blk * C::BW, &raw_full[rs]);
     };
@@ -238,6 +275,7 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
     // producer's lane initialises `ready` and fills the x ring. Nobody else touches a barrier
     // before the CTA-wide barrier below.
     int pre_raw = 0, pre_x = 0;   // blocks already issued by the two producers
+    if (threadIdx.x == 0) pdl_launch_dependents();
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::RAW_STAGES; ++s) {
             // the codes' (and signs') expect_tx arrival, plus 32 cp.async arrivals when signs are copied by threads
@@ -255,6 +293,7 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
         tma_prefetch_desc(&tmap_codes);
         if (signs_by_tma) {
             tma_prefetch_desc(&tmap_signs);
+            pdl_wait();
             RunIter pit = it;
             while (pre_raw < C::RAW_STAGES && pit.next(tile, r0, r1, j)) {
                 const int n_blk = tile / args.m_tiles;
@@ -268,6 +307,7 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
         fence_mbar_init();
         tma_prefetch_desc(&tmap_x);
         if (args.tail_split == 2) tma_prefetch_desc(&tmap_xh);
+        pdl_wait();
         RunIter pit = it;
         int xoff, xrows;
         while (pre_x < C::X_STAGES && pit.next(tile, r0, r1, j, xoff, xrows, BX)) {
@@ -277,8 +317,11 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
     // ---- pair table: 32 copies of value(b) then 32 copies of spread(b) per entry b
     for (int e = threadIdx.x; e < 512; e += C::THREADS) {
         const uint32_t b = (uint32_t)e & 255u;
-        const uint32_t v = e < 256 ? ((uint32_t)args.lut[b & 15u] | ((uint32_t)args.lut[b >> 4] << 16))
-                                   : opqbits::sign_spread(b);
+        // 4 bits: entry b holds the pair of magnitudes of code byte b; other widths: entry q < 2^BITS
+        // holds the magnitude of code q in both halves
+        const uint32_t v = e >= 256 ? opqbits::sign_spread(b)
+                           : BITS == 4 ? ((uint32_t)args.lut[b & 15u] | ((uint32_t)args.lut[b >> 4] << 16))
+                                       : (b < (1u << BITS) ? (uint32_t)args.lutb[b] * 0x00010001u : 0u);
         const uint32_t dst = sbase + C::OFF_TABLE + b * 256u + (e < 256 ? 0u : 128u);
 #pragma unroll
         for (int k = 0; k < 8; ++k)
@@ -295,6 +338,7 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
 
     if (warp == C::WARP_LOAD) {
         // ----------------------------------------------------------- raw producer
+        pdl_wait();
         const int swd = args.K / 32;        // sign words per row
         int rs = 0;
         uint32_t rph = 0;
@@ -321,7 +365,7 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
                         issue_raw(rs, r, n_blk);
                     } else {
                         mbar_arrive_expect_tx(&raw_full[rs], C::RAW_CODE_BYTES);
-                        tma_load_2d(smem + C::OFF_RAW + rs * C::RAW_BYTES, &tmap_codes, r * (C::KR / 8),
+                        tma_load_2d(smem + C::OFF_RAW + rs * C::RAW_BYTES, &tmap_codes, r * C::CODE_WORDS,
                                     n_blk * C::BW, &raw_full[rs]);
                     }
                 }
@@ -428,6 +472,7 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
         }
     } else if (warp < C::WARP_EPI0) {
         // ----------------------------------------------------------- decoders
+        pdl_wait();   // the group-wise scales are read from global memory
         const int g = (warp - C::WARP_DEC0) >> 2;        // decoder group
         const int q = warp & 3;                          // TMEM lane quarter this warp may access
         const int row = q * 32 + lane;                   // weight row in the tile = TMEM lane
@@ -450,18 +495,27 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
             const int rs = blk % C::RAW_STAGES;
             const uint32_t rph = (uint32_t)(blk / C::RAW_STAGES) & 1u;
             if (!warp_wait(&raw_full[rs], rph)) return false;
-            const uint8_t *rawc = smem + C::OFF_RAW + rs * C::RAW_BYTES + row * (C::KR / 2);
+            const uint8_t *rawc = smem + C::OFF_RAW + rs * C::RAW_BYTES + row * (C::CODE_WORDS * 4);
             const uint8_t *raws = smem + C::OFF_RAW + rs * C::RAW_BYTES + C::RAW_CODE_BYTES + row * (C::KR / 8);
 #pragma unroll
             for (int h = 0; h < C::KR / C::KA; ++h) {     // two 64-K A stages per block
                 const int sidx = blk * 2 + h;
                 const int as = sidx % C::A_STAGES;
-                // this half's 8 code words (two 16-byte chunks) and 2 sign words
-                uint32_t cw[8];
+                // this half's 2 BITS code words (4 bits: two 16-byte chunks, 64-byte swizzle) and 2 sign words
+                uint32_t cw[2 * BITS];
+                if constexpr (BITS == 4) {
 #pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    const uint4 v = *reinterpret_cast<const uint4 *>(rawc + ((((uint32_t)(2 * h + c)) ^ sw64) << 4));
-                    cw[4 * c] = v.x; cw[4 * c + 1] = v.y; cw[4 * c + 2] = v.z; cw[4 * c + 3] = v.w;
+                    for (int c = 0; c < 2; ++c) {
+                        const uint4 v = *reinterpret_cast<const uint4 *>(rawc + ((((uint32_t)(2 * h + c)) ^ sw64) << 4));
+                        cw[4 * c] = v.x; cw[4 * c + 1] = v.y; cw[4 * c + 2] = v.z; cw[4 * c + 3] = v.w;
+                    }
+                } else {
+                    // unswizzled rows of 16 BITS bytes; the half starts at word 2 BITS h (8-byte aligned)
+#pragma unroll
+                    for (int c = 0; c < BITS; ++c) {
+                        const uint2 v = *reinterpret_cast<const uint2 *>(rawc + 8 * (BITS * h + c));
+                        cw[2 * c] = v.x; cw[2 * c + 1] = v.y;
+                    }
                 }
                 const uint2 sv = *reinterpret_cast<const uint2 *>(raws + 8 * h);
                 const uint32_t sw[2] = {sv.x, sv.y};
@@ -470,7 +524,9 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
                     if (lane == 0) mbar_arrive(&raw_empty[rs]);   // the block's raw words are in registers now
                 }
                 uint32_t o[2][16];
-                if constexpr (GS == 0) {
+                if constexpr (BITS != 4) {
+                    decode_half_bits<BITS>(cw, sw, lw, lw2, load, o);
+                } else if constexpr (GS == 0) {
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
                         uint32_t t4[4];
@@ -525,6 +581,7 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
         }
     } else {
         // ----------------------------------------------------------- epilogue
+        pdl_wait();
         const int q = warp & 3;
         const int row = q * 32 + lane;
         const bool vec_y = (args.N % 8) == 0;

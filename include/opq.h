@@ -158,6 +158,8 @@ opq_status opq_linear_grouped_workspace_size(int64_t M, int64_t N, int64_t K, in
  *   activation  OPQ_ACT_NONE, OPQ_ACT_SILU (v / (1 + e^-v)) or OPQ_ACT_GELU_TANH
  *               (0.5 v (1 + tanh(sqrt(2/pi) (v + 0.044715 v^3)))); anything else is
  *               OPQ_ERR_INVALID_ARG
+ * Both activations are evaluated with the GPU's hardware tanh approximation (SiLU as
+ * v (1/2 + tanh(v/2)/2)): the output's extra error is at most about 2.5e-4 |v|.
  * Workspace and schedule as for the unfused calls.
  */
 #define OPQ_ACT_NONE 0
@@ -178,14 +180,30 @@ opq_status opq_linear_grouped_fused(const uint16_t *x, int64_t M, int64_t K, con
  * w' = sign * (q/L)^(1/alpha) * max, one fp32 max per row. The codes of a row
  * form one little-endian bit stream: element k at bits k*bits .. k*bits+bits-1
  * of the row's K*bits/32 uint32 words (for 4 bits: nibble k % 8 of word k / 8,
- * the per-row format above). Signs and scales as in the per-row format. These
- * widths have quantize and dequantize; opq_linear takes 4-bit codes only.
+ * the per-row format above). Signs and scales as in the per-row format.
  *   codes  uint32 [N, K*bits/32];  bits 3..6 (OPQ_ERR_INVALID_ARG otherwise)
  */
 opq_status opq_quantize_bits(const uint16_t *w, int64_t N, int64_t K, int64_t ldw, int32_t bits, float alpha,
                              uint32_t *codes, uint32_t *signs, float *scales, void *stream);
 opq_status opq_dequantize_bits(const uint32_t *codes, const uint32_t *signs, const float *scales, int64_t N, int64_t K,
                                int32_t bits, float alpha, uint16_t *w_out, void *stream);
+
+/*
+ * opq_linear_bits — the OPQLinear forward at any of the card's widths (its
+ * configuration lists OPQ_BITS 3, 4, 5, 6): y = x W'^T with each decoded weight
+ * sign * bf16((q/L)^(1/alpha)), L = 2^bits - 1, in a bf16 tensor-core product with
+ * fp32 accumulation; y = bf16(sum * scale[n]), as opq_linear.
+ *   x, M, K, y, workspace, workspace_bytes, stream   as for opq_linear
+ *   codes, signs, scales, N   the planes of opq_quantize_bits at `bits`
+ *   bits        3..6 (OPQ_ERR_INVALID_ARG otherwise); 4 runs opq_linear
+ * Widths 3, 5 and 6 need K % 128 == 0 (OPQ_ERR_UNSUPPORTED_SHAPE otherwise) and run
+ * 256-activation-row tiles for every M; the workspace is sized by
+ * opq_linear_bits_workspace_size and follows opq_linear's rules.
+ */
+opq_status opq_linear_bits_workspace_size(int64_t M, int64_t N, int64_t K, int32_t bits, size_t *bytes);
+opq_status opq_linear_bits(const uint16_t *x, int64_t M, int64_t K, const uint32_t *codes, const uint32_t *signs,
+                           const float *scales, int64_t N, int32_t bits, float alpha, uint16_t *y, void *workspace,
+                           size_t workspace_bytes, void *stream);
 
 /*
  * opq_alpha_search — the card's alpha is a per-model choice in 0.3 .. 1.0 (its

@@ -7,7 +7,7 @@ import torch
 import bit_diffusion_transformer_b200 as opq
 import oracle
 import workloads
-from oracle_pins import _stream_codes
+from oracle_pins import _stream_codes, bits_to_f64
 from test_gpu_parity import DEV, TIE_FRACTION_LIMIT, alpha32, check_guards, guarded, no_device_error, to_dev_u32, u16, u32
 
 pytestmark = pytest.mark.gpu
@@ -95,3 +95,76 @@ def test_bits_argument_errors():
         opq.quantize_bits(w, 7)
     with pytest.raises(opq.OPQError):
         opq.quantize_bits(w, 2)
+
+
+# ---------------------------------------------------------------- linear --
+def linear_bits_parity(x_cpu, w_cpu, bits, alpha, rows=None):
+    """GPU linear on the oracle's `bits`-bit planes against x W'^T with the oracle's fp64 W':
+    |y - y_ref| <= 1e-2 (|x| |W'|^T) + 1e-3 on every output (or the activation rows `rows`)."""
+    ref = oracle.quantize_bits(w_cpu, bits, alpha)
+    wq = oracle.dequantize_bits_f64(ref["codes"], ref["signs"], ref["scales"], bits, alpha32(alpha))
+    M, K = x_cpu.shape
+    N = w_cpu.shape[0]
+    yb, y, pad = guarded((M, N), torch.bfloat16, 0x6B)
+    opq.linear_bits(x_cpu.to(DEV), to_dev_u32(ref["codes"]), to_dev_u32(ref["signs"]),
+                    torch.from_numpy(ref["scales"]).to(DEV), bits, alpha, out=y)
+    torch.cuda.synchronize()
+    check_guards(yb, pad, 0x6B)
+    no_device_error()
+    sel = np.arange(M) if rows is None else np.asarray(rows)
+    xs = bits_to_f64(x_cpu.view(torch.int16).numpy().view(np.uint16))[sel]
+    yref = xs @ wq.T
+    bound = np.abs(xs) @ np.abs(wq).T
+    got = bits_to_f64(u16(y))[sel]
+    err = np.abs(got - yref)
+    tol = 1e-2 * bound + 1e-3
+    assert not (err > tol).any(), f"{int((err > tol).sum())} outputs out of tolerance (worst {float((err / tol).max()):.3f})"
+
+
+@pytest.mark.parametrize("bits", [3, 5, 6])
+@pytest.mark.parametrize("M,N,K", [(1, 256, 512), (16, 384, 1024), (300, 131, 640), (700, 256, 384)])
+def test_linear_bits(bits, M, N, K):
+    # ragged activation and weight rows, several 128-K blocks; every M runs the 256-row tiles
+    lin = workloads.Linear("bits-lin", M, N, K, w_seed=M + N + K + bits, x_seed=7 * bits + M)
+    x, w = lin.make("cpu")
+    linear_bits_parity(x, w, bits, 0.73)
+
+
+@pytest.mark.parametrize("bits", [3, 6])
+@pytest.mark.parametrize("alpha", [0.45, 1.0])
+def test_linear_bits_alpha(bits, alpha):
+    lin = workloads.Linear("bits-lin-a", 64, 256, 1024, w_seed=bits, x_seed=3)
+    x, w = lin.make("cpu")
+    linear_bits_parity(x, w, bits, alpha)
+
+
+@pytest.mark.parametrize("bits", [3, 5, 6])
+def test_linear_bits_full_size_sampled(bits):
+    """The attention projection (x 3072 x 3840, W 3840 x 3840): whole waves of tiles and the
+    split tail; every output of 40 activation rows spread over the tiles."""
+    lin = workloads.dit_attn_proj()
+    x, w = lin.make("cpu")
+    rows = sorted(set(list(range(0, lin.M, 79)) + [lin.M - 1, 2047, 2048, 2303]))
+    linear_bits_parity(x, w, bits, lin.alpha, rows=rows)
+
+
+def test_linear_bits_four_is_the_nibble_linear():
+    lin = workloads.Linear("bits4", 64, 256, 512, w_seed=5, x_seed=6)
+    x, w = lin.make(DEV)
+    planes = opq.quantize(w)
+    assert torch.equal(opq.linear_bits(x, *planes, 4), opq.linear(x, *planes))
+
+
+def test_linear_bits_argument_errors():
+    x = torch.zeros((4, 96), dtype=torch.bfloat16, device=DEV)
+    w = torch.zeros((8, 96), dtype=torch.bfloat16, device=DEV)
+    c, s, f = opq.quantize_bits(w, 3)
+    y = torch.empty((4, 8), dtype=torch.bfloat16, device=DEV)
+    lib, st = opq.load(), opq._stream(x.device)
+    # K % 128 != 0 at 3 bits
+    assert lib.opq_linear_bits(opq._ptr(x), 4, 96, opq._ptr(c), opq._ptr(s), opq._ptr(f), 8, 3, 0.73, opq._ptr(y),
+                               None, 0, st) == 2
+    for b in (2, 7):
+        assert lib.opq_linear_bits(opq._ptr(x), 4, 96, opq._ptr(c), opq._ptr(s), opq._ptr(f), 8, b, 0.73,
+                                   opq._ptr(y), None, 0, st) == 1
+    no_device_error()
