@@ -617,10 +617,12 @@ def gpu_extras(args, opq, workloads, torch, dev, peaks, time_kernel, flush):
         cb, sb, fb = opq.quantize_bits(w, b_, alpha)
         fq_ = lambda: opq.quantize_bits(w, b_, alpha, out=(cb, sb, fb))
         fd_ = lambda: opq.dequantize_bits(cb, sb, fb, b_, alpha, out=wq_b)
-        for f_ in (fq_, fd_):
+        ws_b = torch.zeros((max(opq.bits_workspace_size(M, N, K, b_), 16),), dtype=torch.uint8, device=dev)
+        fl_b = lambda: opq.linear_bits(x, cb, sb, fb, b_, alpha, out=y, workspace=ws_b)
+        for f_ in (fq_, fd_, fl_b):
             for _ in range(3):
                 f_()
-        tq_, td_ = time_kernel(fq_), time_kernel(fd_)
+        tq_, td_, tl_ = time_kernel(fq_), time_kernel(fd_), time_kernel(fl_b)
         packed = N * K * b_ // 8 + N * K // 8 + 4 * N
         opq.dequantize_bits(cb, sb, fb, b_, alpha, out=wq_b)
         bits_out[str(b_)] = {
@@ -628,7 +630,9 @@ def gpu_extras(args, opq, workloads, torch, dev, peaks, time_kernel, flush):
                          "frac_hbm": (N * K * 2 + packed) / tq_ / 1e6 / hbm},
             "dequantize": {"ms": td_, "gbs": (packed + N * K * 2) / td_ / 1e6,
                            "frac_hbm": (packed + N * K * 2) / td_ / 1e6 / hbm},
+            "linear": {"ms": tl_, "tflops": flops / tl_ / 1e9, "frac_bf16": flops / tl_ / 1e9 / bf16},
             "snr_db": float(10.0 * torch.log10((r_ * r_).sum() / ((r_ - wq_b.double()) ** 2).sum()))}
+        del ws_b
         del cb, sb, fb
     out["bits"] = bits_out
     del wq_b, r_
