@@ -11,7 +11,8 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 SO = os.path.join(HERE, "libopq.so")
 SOURCES = ["opq_capi.cu"]
-HEADERS = ["opq_bits.h", "opq_device.cuh", "opq_quantize.cuh", "opq_dequantize.cuh", "opq_linear.cuh", "opq_linear_wide.cuh", "opq_grouped.cuh"]
+HEADERS = ["opq_bits.h", "opq_device.cuh", "opq_quantize.cuh", "opq_quantize_stream.cuh", "opq_dequantize.cuh",
+           "opq_linear.cuh", "opq_linear_wide.cuh", "opq_grouped.cuh"]
 
 
 def _nvcc() -> str:

@@ -14,14 +14,15 @@
 // activation rows. Per CTA (one per SM, persistent):
 //   warp 0       raw producer: codes (64-byte swizzle) and signs of 128 weight rows,
 //                one load group (GRP consecutive 128-K blocks) per pair of TMA copies
-//   warp 1       TMEM allocation and MMA issue (every accumulation chain); A comes from TMEM
+//   warp 1       TMEM allocation and MMA issue; A comes from TMEM. For BX <= 32 warps 19, 20
+//                issue too: one issuer per decoder group, each with its own accumulator
 //   warp 2       x producer: the load group's x (BX rows, 128-byte swizzle), one copy
 //   warps 3..14  three decoder groups of 4 warps (= the 128 TMEM lanes): each thread owns
 //                one weight row and decodes 128 weights per block through the shared-memory
 //                pair table (opq_bits.h), written to TMEM with tcgen05.st as the A operand
 //   warps 15..18 epilogue: accumulator TMEM -> registers -> * scale[n] -> bf16 y,
 //                or fp32 partial sums for tiles split across CTAs
-// TMEM columns: [0, A_COLS) the A ring; then NACC accumulator buffers of NCHAIN x BX.
+// TMEM columns: [0, A_COLS) the A ring; then NACC accumulator buffers of NCH_ALL chains x BX.
 //
 // Work is a list of runs (tile, range of load groups). Mode 1 (stream-K) cuts the
 // flattened (tile, load group) sequence into one contiguous range per CTA; a tile covered
@@ -285,23 +286,49 @@ struct Cfg {
     // raw stages hold one load group each; a decoder group waiting on a stage knows only that
     // the block three before its own was loaded, so at least three stages keep parity waits exact
     static constexpr int RAW_STAGES = GRP > 1 ? 3 : (BX >= 256 ? 2 : (BX >= 128 ? 4 : 6));
-    static constexpr int A_STAGES = 8;                 // 32 TMEM columns each (64 K of bf16 pairs)
-    static constexpr int A_BLOCKS = A_STAGES / 2;      // 128-K blocks of A held in TMEM
+    // decoder groups of 4 warps: group g decodes the CTA's 128-K blocks g, g + G, ...;
+    // thread r of a group owns weight row r (TMEM lane r) and decodes its whole 128-K block row
+    static constexpr int GROUPS = BX >= 256 ? 2 : 3;
+    // MMA issuers. A narrow block's 8 MMAs take one issuing thread longer than a decoder group
+    // takes to decode the block, so narrow tiles (BX <= 32) give every decoder group an issuer
+    // of its own (issuer i issues the blocks group i decodes, into its own accumulator) and
+    // the tensor pipe takes MMAs from three threads at once; wider tiles keep one issuer.
+    static constexpr int NISS = BX <= 32 ? GROUPS : 1;
+    // A ring in TMEM, in 128-K blocks (two 64-K half-stages of 32 columns each). With one
+    // issuer per group, block b uses slot b % A_BLOCKS and A_BLOCKS = 2 GROUPS, so every slot
+    // is used by one decoder group and one issuer only (two slots per group).
+    static constexpr int A_BLOCKS = NISS > 1 ? 2 * GROUPS : 4;
+    static constexpr int A_STAGES = 2 * A_BLOCKS;      // 32 TMEM columns each (64 K of bf16 pairs)
     static constexpr int A_COLS = A_STAGES * 32;
     // x stages hold one load group (two 64-K swizzle atoms' worth of columns per block)
     static constexpr int X_STAGES = GRP == 4 ? 2 : (GRP == 2 ? (BX >= 64 ? 2 : 4) : (BX >= 256 ? 2 : 3));
     // One tcgen05.commit per 128-K block frees both its A slot and its x stage: a commit
     // stalls the tensor pipe for a few hundred cycles, so there is one per 8 MMAs, not per 4.
-    // Slot b % NDONE of `blk_done` completes when the MMAs of the CTA's block b are done.
-    // The x producer waits for the last block of the group X_STAGES groups back; with up to
-    // (X_STAGES - 1) GRP blocks in between, 1 + (X_STAGES - 1) GRP slots keep that wait exact.
+    // `blk_done` is one ring of NDONE slots per issuer; issuer i's t-th block (CTA block
+    // b = t NISS + i) completes slot i NDONE + t % NDONE. An issuer's blocks complete in its
+    // issue order, so the parity of each wait is exact when:
+    //  - one issuer: the x producer waits for the last block of the group X_STAGES groups back,
+    //    with up to (X_STAGES - 1) GRP blocks in between (NDONE >= 1 + (X_STAGES - 1) GRP); a
+    //    decoder waits for block b - A_BLOCKS knowing only that its own previous wait (block
+    //    b - GROUPS - A_BLOCKS) succeeded, which implies block b - A_BLOCKS - NDONE completed
+    //    if NDONE >= GROUPS;
+    //  - an issuer per group: a decoder's previous wait was on the same issuer's ring, one of
+    //    its blocks earlier, and block b - A_BLOCKS + NISS NDONE cannot complete before block
+    //    b is decoded if NDONE > A_BLOCKS / NISS; the x producer waits for the last NISS blocks
+    //    up to the group X_STAGES back (each issuer's latest), advancing at most
+    //    ceil(GRP / NISS) <= NDONE of an issuer's blocks per group, and the newest block that
+    //    could alias a slot, last - (NISS - 1) + NISS NDONE, lies in a group not yet loaded if
+    //    NISS (NDONE - 1) >= (X_STAGES - 1) GRP.
     static constexpr int NDONE_X = 1 + (X_STAGES - 1) * GRP;
-    static constexpr int NDONE = NDONE_X > A_BLOCKS ? NDONE_X : A_BLOCKS;
+    static constexpr int NDONE = NISS > 1 ? A_BLOCKS / NISS + 1 : (NDONE_X > A_BLOCKS ? NDONE_X : A_BLOCKS);
+    static constexpr int NDONE_ALL = NISS * NDONE;
     // independent accumulation chains per tile: consecutive MMAs into one accumulator
-    // serialize on its latency, which dominates when N (= BX) is small; K-step k of a
-    // stage goes to chain k % NCHAIN and the epilogue adds the chains in a fixed order
-    static constexpr int NCHAIN = BX <= 32 ? 4 : (BX <= 64 ? 2 : 1);
-    static constexpr int ACC_COLS = NCHAIN * BX;       // one accumulator buffer (all chains)
+    // serialize on its latency, which dominates when N (= BX) is small; with one issuer, K-step
+    // k of a stage goes to chain k % NCHAIN; with an issuer per group, each issuer's blocks form
+    // one chain. The epilogue adds the chains in a fixed order.
+    static constexpr int NCHAIN = NISS > 1 ? 1 : (BX <= 32 ? 4 : (BX <= 64 ? 2 : 1));
+    static constexpr int NCH_ALL = NISS * NCHAIN;         // chains per accumulator buffer
+    static constexpr int ACC_COLS = NCH_ALL * BX;         // one accumulator buffer (all chains)
     static constexpr int NACC = (A_COLS + 2 * ACC_COLS <= 512) ? 2 : 1;   // accumulator buffers
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr int BLK_CODE_BYTES = BW * KR / 2;    // 8 KiB per block: [128 rows][16 words], 64-byte swizzle
@@ -316,29 +343,26 @@ struct Cfg {
     static constexpr int OFF_X = OFF_RAW + RAW_STAGES * RAW_BYTES;
     static constexpr int OFF_EPI = OFF_X + X_STAGES * X_BYTES;
     static constexpr int OFF_BAR = OFF_EPI + STAGE_EPI_BYTES;
-    static constexpr int NUM_BARS = 2 * RAW_STAGES + X_STAGES + A_BLOCKS + NDONE + 2 * NACC + 1;
+    static constexpr int NUM_BARS = 2 * RAW_STAGES + X_STAGES + A_BLOCKS + NDONE_ALL + 2 * NACC + 1;
     static constexpr int OFF_TMEM = OFF_BAR + NUM_BARS * 8;
     static constexpr int SMEM_BYTES = OFF_TMEM + 16 + 1024;
-    // decoder groups of 4 warps: group g decodes the CTA's 128-K blocks g, g + G, ...;
-    // thread r of a group owns weight row r (TMEM lane r) and decodes its whole 128-K block row
-    static constexpr int GROUPS = BX >= 256 ? 2 : 3;
     // a group waits on raw stage blk % RAW_STAGES knowing only that its own previous block
     // (blk - GROUPS) was loaded, so the stage's previous phase (block blk - RAW_STAGES) must
     // be at least that old for the parity test to be exact
     static_assert(RAW_STAGES >= GROUPS, "raw ring shorter than the decoder rotation");
-    // a decoder waits for block b - A_BLOCKS on blk_done knowing only that its own previous wait
-    // (block b - GROUPS - A_BLOCKS) succeeded; the parity test is exact only if that implies block
-    // b - A_BLOCKS - NDONE has completed, i.e. NDONE >= GROUPS (completions come in block order)
-    static_assert(NDONE >= GROUPS, "done ring shorter than the decoder rotation");
+    static_assert(NISS > 1 || NDONE >= GROUPS, "done ring shorter than the decoder rotation");
+    static_assert(NISS > 1 || NDONE >= NDONE_X, "done ring shorter than the x ring's reach");
+    static_assert(NISS == 1 || (NISS == GROUPS && A_BLOCKS % NISS == 0 && NDONE > A_BLOCKS / NISS &&
+                                NISS * (NDONE - 1) >= (X_STAGES - 1) * GRP && (GRP + NISS - 1) / NISS <= NDONE),
+                  "issuer rings too short for exact parity waits");
     static constexpr int WARP_LOAD = 0, WARP_MMA = 1, WARP_XLOAD = 2, WARP_DEC0 = 3, NUM_DEC_WARPS = 4 * GROUPS;
     static constexpr int WARP_EPI0 = WARP_DEC0 + NUM_DEC_WARPS;
-    // One MMA-issuing thread for all the chains: consecutive K-steps go to different chains, so
-    // no MMA waits for its predecessor's result, and one tcgen05.commit per block covers them all
-    // (a commit stalls the tensor pipe for a few hundred cycles; per-chain issuer threads needed
-    // one commit each, and measured ~0.65 us per 128-K block at BX = 16 against ~0.3 us of decode)
-    static constexpr int NISS = 1;
+    // issuer 0 is warp WARP_MMA (which also owns the TMEM allocation), issuer i > 0 warp WARP_ISS1 + i - 1
     static constexpr int WARP_ISS1 = WARP_EPI0 + 4;
     static constexpr int THREADS = (WARP_ISS1 + NISS - 1) * 32;
+    // the blk_done slot and parity of the CTA's block b
+    __device__ __forceinline__ static int done_slot(int b) { return (b % NISS) * NDONE + (b / NISS) % NDONE; }
+    __device__ __forceinline__ static uint32_t done_parity(int b) { return (uint32_t)((b / NISS) / NDONE) & 1u; }
     static_assert(SMEM_BYTES <= 232448, "shared memory");
     static_assert(BX % 16 == 0 && BX >= 16 && BX <= 256, "MMA N");
     static_assert(A_COLS + NACC * ACC_COLS <= 512, "TMEM columns");
@@ -366,7 +390,7 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
     uint64_t *x_full = raw_empty + C::RAW_STAGES;
     uint64_t *a_full = x_full + C::X_STAGES;    // per A slot (128-K block): its A tile is in TMEM
     uint64_t *blk_done = a_full + C::A_BLOCKS;
-    uint64_t *acc_full = blk_done + C::NDONE;
+    uint64_t *acc_full = blk_done + C::NDONE_ALL;
     uint64_t *acc_empty = acc_full + C::NACC;
     uint64_t *drain = acc_empty + C::NACC;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_TMEM);
@@ -385,7 +409,7 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
         }
         for (int s = 0; s < C::X_STAGES; ++s) mbar_init(&x_full[s], 1);
         for (int s = 0; s < C::A_BLOCKS; ++s) mbar_init(&a_full[s], 4);   // the 4 warps of the decoding group
-        for (int s = 0; s < C::NDONE; ++s) mbar_init(&blk_done[s], C::NISS);   // one commit per issuer
+        for (int s = 0; s < C::NDONE_ALL; ++s) mbar_init(&blk_done[s], 1);   // one commit (the block's issuer)
         for (int s = 0; s < C::NACC; ++s) {
             mbar_init(&acc_full[s], C::NISS);
             mbar_init(&acc_empty[s], 4);
@@ -501,13 +525,14 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
                 for (int g = R.g0; g < R.g1; ++g, ++v) {
                     const int r = lg.start(g), nb = lg.start(g + 1) - r;
                     const int xs = v % C::X_STAGES;
-                    // the stage last held group v - X_STAGES: wait until its last block's MMAs are done
+                    // the stage last held group v - X_STAGES: wait until its blocks' MMAs are done
+                    // (each issuer's latest block up to the group's last: an issuer's blocks
+                    // complete in order)
                     if (v >= C::X_STAGES) {
-                        const int prev = last_blk[xs];
-                        if (!mbar_wait(&blk_done[prev % C::NDONE], (uint32_t)(prev / C::NDONE) & 1u)) {
-                            ok = false;
-                            break;
-                        }
+                        const int last = last_blk[xs];
+                        for (int i = 0; i < C::NISS && last - i >= 0 && ok; ++i)
+                            ok = mbar_wait(&blk_done[C::done_slot(last - i)], C::done_parity(last - i));
+                        if (!ok) break;
                     }
                     mbar_arrive_expect_tx(&x_full[xs], xbytes);
                     uint8_t *dst = smem + C::OFF_X + xs * C::X_BYTES;
@@ -529,14 +554,20 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
             }
         }
     } else if (warp == C::WARP_MMA || warp >= C::WARP_ISS1) {
-        // ----------------------------------------------------------- MMA issuer
-        // The run's i-th MMA (K-step k of a 64-K half) accumulates into chain i % NCHAIN (= k % NCHAIN,
-        // NCHAIN divides the 4 K-steps of a half); a chain's first MMA of the run starts it afresh.
+        // ----------------------------------------------------------- MMA issuers
+        // One issuer: every block, the run's i-th MMA (K-step k of a 64-K half) accumulating into
+        // chain i % NCHAIN (= k % NCHAIN, NCHAIN divides the 4 K-steps of a half). An issuer per
+        // decoder group: issuer `iss` takes the CTA's blocks b with b % NISS == iss (the blocks
+        // its group decodes, in their A slots b % A_BLOCKS), all into its own chain. A chain's
+        // first MMA of the run starts it afresh. Every issuer waits for every x stage in order,
+        // so that each of its parity waits is exact.
+        const int iss = warp == C::WARP_MMA ? 0 : warp - C::WARP_ISS1 + 1;
         if (lane == 0) {
             int ab = 0;
             uint32_t abph = 0;
-            int as0 = 0, xs = 0, ds = 0;       // A half-stage of the block's first half, x stage, blk_done slot
-            uint32_t aph = 0, xph = 0;
+            int xs = 0;
+            uint32_t xph = 0;
+            int b = 0;                         // the CTA's block index
             bool ok = true;
             constexpr uint32_t idesc_full = idesc_bf16_f32(128, BX);
             constexpr uint32_t idesc_half = idesc_bf16_f32(128, BX / 2);
@@ -544,20 +575,22 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
                 const uint32_t idesc = R.xrows == BX ? idesc_full : idesc_half;
                 if (!mbar_wait(&acc_empty[ab], abph ^ 1)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t d_base = tmem_base + C::A_COLS + ab * C::ACC_COLS;
-                uint32_t started = 0;          // MMAs of this run issued so far
+                const uint32_t d_base = tmem_base + C::A_COLS + ab * C::ACC_COLS + (uint32_t)(iss * C::NCHAIN * BX);
+                uint32_t started = 0;          // MMAs of this run issued so far by this thread
                 for (int g = R.g0; g < R.g1 && ok; ++g) {
                     const int nb = lg.start(g + 1) - lg.start(g);
                     if (!mbar_wait(&x_full[xs], xph)) { ok = false; break; }
                     const uint32_t xbase = sbase + C::OFF_X + xs * C::X_BYTES;
-                    for (int jj = 0; jj < nb; ++jj) {
+                    for (int jj = 0; jj < nb; ++jj, ++b) {
+                        if (C::NISS > 1 && b % C::NISS != iss) continue;
+                        const int slot = b % C::A_BLOCKS;
                         // one wait per block: a wait right before an MMA costs the issuing thread
                         // about as much as the MMAs of a narrow block
-                        if (!mbar_wait(&a_full[as0 >> 1], aph)) { ok = false; break; }
+                        if (!mbar_wait(&a_full[slot], (uint32_t)(b / C::A_BLOCKS) & 1u)) { ok = false; break; }
                         tc_fence_after();
 #pragma unroll
                         for (int h = 0; h < 2; ++h) {
-                            const uint32_t a_tmem = tmem_base + (as0 + h) * 32;
+                            const uint32_t a_tmem = tmem_base + (uint32_t)((2 * slot + h) * 32);
                             const uint64_t bdesc = smem_desc_sw128(xbase + (2 * jj + h) * C::X_HALF_BYTES);
                             // a fixed count of MMAs and no branch between them (a branch around
                             // tcgen05.mma costs the issuing thread far more than the MMA itself)
@@ -568,11 +601,7 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
                                 ++started;
                             }
                         }
-                        if (!ok) break;
-                        umma_commit(&blk_done[ds]);
-                        as0 += 2;
-                        if (as0 == C::A_STAGES) { as0 = 0; aph ^= 1; }
-                        if (++ds == C::NDONE) ds = 0;
+                        umma_commit(&blk_done[C::done_slot(b)]);
                     }
                     if (++xs == C::X_STAGES) { xs = 0; xph ^= 1; }
                 }
@@ -672,8 +701,7 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
                         }
                         // the block's A slot last held block blk - A_BLOCKS
                         const int prev = blk - C::A_BLOCKS;
-                        if (h == 0 && prev >= 0 &&
-                            !warp_wait(&blk_done[prev % C::NDONE], (uint32_t)(prev / C::NDONE) & 1u)) {
+                        if (h == 0 && prev >= 0 && !warp_wait(&blk_done[C::done_slot(prev)], C::done_parity(prev))) {
                             ok = false;
                             break;
                         }
@@ -704,31 +732,49 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
         int ab = 0;
         uint32_t abph = 0;
         int sb = 0;
+        int bstart = 0;              // the CTA's block index at the run's start
         while (it.next(R, BX)) {
             const int tile = R.tile, r0 = R.r0, r1 = R.r1, j = R.j, xoff = R.xoff, xrows = R.xrows;
+            // the accumulator chains that hold this run's sums: all of them with one issuer; with
+            // an issuer per decoder group, issuer i's only if the run has one of its blocks
+            uint32_t cmask = (1u << C::NCH_ALL) - 1u;
+            if (C::NISS > 1) {
+                cmask = 0u;
+                for (int i = 0; i < C::NISS; ++i)
+                    if ((i - bstart % C::NISS + C::NISS) % C::NISS < r1 - r0) cmask |= 1u << i;
+            }
+            bstart += r1 - r0;
+            const int ch0 = __ffs((int)cmask) - 1;
             const int n_blk = tile / args.m_tiles, m_blk = tile % args.m_tiles;
             const int n = n_blk * C::BW + row;
             const int n0 = n_blk * C::BW + q * 32;           // first row of this warp's quarter
             const bool full = (r0 == 0 && r1 == args.kblocks);
             const float scale = GS > 0 ? 1.0f : (n < args.N ? __ldg(args.scales + n) : 0.0f);
             const float bias = bias_at(args.bias, n, args.N);
-            // the plain product, or the fused epilogue (bias, activation): chosen per tile, so the
-            // plain path carries none of the fused code
-            const bool plain = args.bias == nullptr && args.act == EPI_NONE;
+            // the plain product, or the fused epilogue (bias, activation): chosen per tile, one
+            // specialised store loop per kind, so no loop carries another kind's code. The kind is
+            // read from the parameters once: inside the loops, every y store could alias them.
+            const int act = args.act;
+            const bool plain = args.bias == nullptr && act == EPI_NONE;
             auto fv_plain = [scale](float a) { return a * scale; };
-            auto fv_fused = [scale, bias, &args](float a) { return epi_value(a, scale, bias, args.act); };
+            auto fv_bias = [scale, bias](float a) { return epi_value(a, scale, bias, EPI_NONE); };
+            auto fv_silu = [scale, bias](float a) { return epi_value(a, scale, bias, EPI_SILU); };
+            auto fv_gelu = [scale, bias](float a) { return epi_value(a, scale, bias, EPI_GELU_TANH); };
             if (!warp_wait(&acc_full[ab], abph)) break;
             tc_fence_after();
             const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + C::A_COLS + ab * C::ACC_COLS;
             float *wsp = full ? nullptr
                               : args.ws + ((size_t)blockIdx.x * args.runs_max + j) * (size_t)(BX * C::BW);
+            const int pcols = min(BX, args.M - m_blk * BX);   // partial sums: columns a run stores
 #pragma unroll 1
             for (int c0 = 0; c0 < xrows; c0 += 16) {
                 uint32_t v[16];
-                tmem_ld_32x32b_x16(taddr + c0, v);
-                if (C::NCHAIN > 1) {
+                tmem_ld_32x32b_x16(taddr + ch0 * BX + c0, v);
+                if (C::NCH_ALL > 1) {
+                    // the chains in a fixed order (warp-uniform skips)
 #pragma unroll
-                    for (int ch = 1; ch < C::NCHAIN; ++ch) {
+                    for (int ch = 1; ch < C::NCH_ALL; ++ch) {
+                        if (ch <= ch0 || ((cmask >> ch) & 1u) == 0u) continue;
                         uint32_t u[16];
                         tmem_ld_32x32b_x16(taddr + ch * BX + c0, u);
                         tmem_ld_wait();
@@ -771,10 +817,13 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
                         }
                     };
                     if (plain) store_full(fv_plain);
-                    else store_full(fv_fused);
+                    else if (act == EPI_SILU) store_full(fv_silu);
+                    else if (act == EPI_GELU_TANH) store_full(fv_gelu);
+                    else store_full(fv_bias);
                 } else {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) wsp[(size_t)(c0 + i) * C::BW + row] = __uint_as_float(v[i]);
+                    for (int i = 0; i < 16; ++i)   // the activation rows the fix-up reads (< M)
+                        if (c0 + i < pcols) wsp[(size_t)(c0 + i) * C::BW + row] = __uint_as_float(v[i]);
                 }
             }
             tc_fence_before();
@@ -844,7 +893,9 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
                         };
                         if (n < args.N) {
                             if (plain) store8(fv_plain);
-                            else store8(fv_fused);
+                            else if (act == EPI_SILU) store8(fv_silu);
+                            else if (act == EPI_GELU_TANH) store8(fv_gelu);
+                            else store8(fv_bias);
                         }
                     }
                     if (lane == 0) atomicExch(args.counters + (size_t)tile * 4 + q, 0u);   // ready for the next call

@@ -623,14 +623,20 @@ __global__ void __launch_bounds__(Cfg<BX, BITS>::THREADS, 1)
             const bool full = (r0 == 0 && r1 == args.kblocks);
             const float scale = GS > 0 ? 1.0f : (n < args.N ? __ldg(args.scales + n) : 0.0f);
             const float bias = bias_at(args.bias, n, args.N);
-            // the plain product, or the fused epilogue (bias, activation): chosen per tile, so the
-            // plain path carries none of the fused code
-            const bool plain = args.bias == nullptr && args.act == EPI_NONE;
+            // the plain product, or the fused epilogue (bias, activation): chosen per tile, one
+            // specialised store loop per kind, so no loop carries another kind's code. The kind is
+            // read from the parameters once: inside the loop, every y store could alias them.
+            const int act = args.act;
+            const bool plain = args.bias == nullptr && act == EPI_NONE;
             auto fv_plain = [scale](float a) { return a * scale; };
-            auto fv_fused = [scale, bias, &args](float a) { return epi_value(a, scale, bias, args.act); };
+            auto fv_bias = [scale, bias](float a) { return epi_value(a, scale, bias, EPI_NONE); };
+            auto fv_silu = [scale, bias](float a) { return epi_value(a, scale, bias, EPI_SILU); };
+            auto fv_gelu = [scale, bias](float a) { return epi_value(a, scale, bias, EPI_GELU_TANH); };
             auto store = [&](const uint32_t (&v)[16], int m0) {
                 if (plain) store16(v, m0, n, n0, fv_plain);
-                else store16(v, m0, n, n0, fv_fused);
+                else if (act == EPI_SILU) store16(v, m0, n, n0, fv_silu);
+                else if (act == EPI_GELU_TANH) store16(v, m0, n, n0, fv_gelu);
+                else store16(v, m0, n, n0, fv_bias);
             };
             if (!warp_wait(&acc_full[ab], abph)) break;
             tc_fence_after();
