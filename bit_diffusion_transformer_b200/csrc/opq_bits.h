@@ -202,6 +202,58 @@ OPQ_HD uint32_t codes_word(uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3) {
     return prmt(prmt(b0, b1, 0x0040u), prmt(b2, b3, 0x0040u), 0x5410u);
 }
 
+// Other bit widths: the two codes of a magnitude pair a from a row table whose entries hold q
+// itself (one byte each); clamping and offsets as table_byte_clamped.
+OPQ_HD void table_pair_bytes(const uint8_t *tb, uint32_t a, uint32_t lo2, uint32_t mmb, uint32_t &q0, uint32_t &q1) {
+    const uint32_t d = mmb - bf16x2_max(a, lo2);
+#if defined(__CUDA_ARCH__)
+    uint32_t hi;
+    asm("mul.hi.u32 %0, %1, 65536;" : "=r"(hi) : "r"(d));
+#else
+    const uint32_t hi = d >> 16;
+#endif
+    q0 = tb[d & 0xFFFFu];
+    q1 = tb[hi];
+}
+
+// The 8 BITS-bit codes q[0..7] of one vector as the vector's 8 BITS-bit piece of the row's
+// little-endian bit stream: element e at bits e BITS .. e BITS + BITS - 1 of (hi:lo).
+template <int BITS>
+OPQ_HD void pack_chunk(const uint32_t (&q)[8], uint32_t &lo, uint32_t &hi) {
+    lo = 0u;
+    hi = 0u;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        const int pos = e * BITS;
+        if (pos + BITS <= 32) {
+            lo |= q[e] << pos;
+        } else if (pos >= 32) {
+            hi |= q[e] << (pos - 32);
+        } else {
+            lo |= q[e] << pos;
+            hi |= q[e] >> (32 - pos);
+        }
+    }
+}
+
+// Four consecutive vectors (32 elements) make BITS words of the stream. Lane i of a quad holds
+// the piece of vector i (bits 8 BITS i .. 8 BITS (i + 1) - 1 of the quad's stream) and, from its
+// neighbour, the piece of vector i + 1; it writes the words that start inside its own piece,
+// at most two. quad_word gives the t-th of them (t = 0, 1): false if there is none, else its
+// word index in the quad and its value.
+template <int BITS>
+OPQ_HD bool quad_word(uint32_t lo, uint32_t hi, uint32_t nlo, uint32_t nhi, uint32_t i, uint32_t t, uint32_t &w,
+                      uint32_t &word) {
+    const uint32_t piece = 8u * BITS;
+    const uint32_t b0 = piece * i;
+    w = (b0 + 31u) / 32u + t;
+    if (32u * w >= b0 + piece) return false;   // starts in the next lane's piece (or past the quad)
+    const uint32_t off = 32u * w - b0;         // 0 .. piece - 1
+    const uint64_t c = ((uint64_t)hi << 32) | lo, cn = ((uint64_t)nhi << 32) | nlo;
+    word = (uint32_t)((c >> off) | (cn << (piece - off)));
+    return true;
+}
+
 // Sign bits (bf16 sign bit set) of 8 weights held as 4 bf16 pairs -> bits 0..7.
 OPQ_HD uint32_t sign_byte(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3) {
     // gather the high byte of every bf16 (its top bit is the sign), then move the

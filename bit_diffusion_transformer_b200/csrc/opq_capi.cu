@@ -68,7 +68,7 @@ uint16_t host_bf16(double v) {
 
 struct DeviceInfo {
     int sms = 0;
-    bool stream_quant_attr[3] = {};   // dynamic shared memory raised for quantize_stream_kernel<1, 4, 8>
+    bool stream_quant_attr[3][4] = {};   // dynamic shared memory raised for quantize_stream_kernel<G, BITS>
     // dynamic shared memory raised, per [group size index: 0 per-row, 1..4 GS 32..256][kernel: BX 16, 32,
     // 64, 128, wide]
     bool linear_attr[5][5] = {};
@@ -385,9 +385,9 @@ const char *opq_status_string(opq_status s) {
 // The row-streaming quantize over a list of matrices: validation, then one launch per row-width
 // class (one, four or eight warps per row) and per QS_MAX_JOBS matrices of the class.
 extern "C++" {
-template <int G>
+template <int G, int BITS>
 static opq_status launch_quant_stream(DeviceInfo *di, const opq_quant_job *jobs, const std::vector<int64_t> &idx,
-                                      const opqk::QuantParams &qp, cudaStream_t st) {
+                                      const opqk::QuantParams &qp, const double *tl, cudaStream_t st) {
     using C = opqk::QsCfg<G>;
     int64_t kmax = 0;
     for (int64_t i : idx) kmax = jobs[i].K > kmax ? jobs[i].K : kmax;
@@ -398,17 +398,18 @@ static opq_status launch_quant_stream(DeviceInfo *di, const opq_quant_job *jobs,
     if (nslots < 2) return OPQ_ERR_UNSUPPORTED_SHAPE;
     const int smem = opqk::QS_OFF_RING + nslots * slot_bytes;
     const int gi = G == 1 ? 0 : (G == 4 ? 1 : 2);
-    if (!di->stream_quant_attr[gi]) {
-        cudaError_t e = cudaFuncSetAttribute(opqk::quantize_stream_kernel<G>,
+    if (!di->stream_quant_attr[gi][BITS - 3]) {
+        cudaError_t e = cudaFuncSetAttribute(opqk::quantize_stream_kernel<G, BITS>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              opqk::QS_OFF_RING + C::RING_MAX);
         if (e != cudaSuccess) return cuda_fail(e);
-        di->stream_quant_attr[gi] = true;
+        di->stream_quant_attr[gi][BITS - 3] = true;
     }
     static thread_local opqk::QsParams P;   // ~7 KB: kept off the stack
     for (size_t c0 = 0; c0 < idx.size(); c0 += opqk::QS_MAX_JOBS) {
         std::memset(&P, 0, sizeof P);
         P.qp = qp;
+        for (int k = 0; k < 64; ++k) P.tl[k] = tl[k];
         P.nslots = nslots;
         P.slot_bytes = slot_bytes;
         const size_t n = idx.size() - c0 < (size_t)opqk::QS_MAX_JOBS ? idx.size() - c0 : (size_t)opqk::QS_MAX_JOBS;
@@ -430,15 +431,26 @@ static opq_status launch_quant_stream(DeviceInfo *di, const opq_quant_job *jobs,
         P.rows = rows;
         const int64_t groups = rows < (int64_t)di->sms * C::NG ? rows : (int64_t)di->sms * C::NG;
         const int grid = (int)((groups + C::NG - 1) / C::NG);
-        opqk::quantize_stream_kernel<G><<<grid, opqk::QS_THREADS, smem, st>>>(P);
+        opqk::quantize_stream_kernel<G, BITS><<<grid, opqk::QS_THREADS, smem, st>>>(P);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail(e);
     }
     return OPQ_OK;
 }
+
+template <int BITS>
+static opq_status launch_quant_classes(DeviceInfo *di, const opq_quant_job *jobs, const std::vector<int64_t> (&cls)[3],
+                                       const opqk::QuantParams &qp, const double *tl, cudaStream_t st) {
+    opq_status s = OPQ_OK;
+    if (!cls[0].empty() && (s = launch_quant_stream<1, BITS>(di, jobs, cls[0], qp, tl, st)) != OPQ_OK) return s;
+    if (!cls[1].empty() && (s = launch_quant_stream<4, BITS>(di, jobs, cls[1], qp, tl, st)) != OPQ_OK) return s;
+    if (!cls[2].empty() && (s = launch_quant_stream<8, BITS>(di, jobs, cls[2], qp, tl, st)) != OPQ_OK) return s;
+    return OPQ_OK;
+}
 }  // extern "C++"
 
-static opq_status quantize_jobs(const opq_quant_job *jobs, int64_t count, float alpha, void *stream) {
+// `bits` bits per magnitude code (4: the card's nibble format; 3, 5, 6: per-row bit streams)
+static opq_status quantize_jobs(const opq_quant_job *jobs, int64_t count, float alpha, void *stream, int bits = 4) {
     if (jobs == nullptr || count < 1) return OPQ_ERR_INVALID_ARG;
     if (!alpha_ok(alpha)) return OPQ_ERR_INVALID_ARG;
     for (int64_t i = 0; i < count; ++i) {
@@ -459,16 +471,21 @@ static opq_status quantize_jobs(const opq_quant_job *jobs, int64_t count, float 
     const double inv = 1.0 / (double)alpha;
     for (int k = 1; k < 16; ++k) qp.t[k] = std::pow(((double)k - 0.5) / 15.0, inv);
     qp.alpha_is_one = (alpha == 1.0f) ? 1 : 0;
+    double tl[64] = {};
+    const int L = (1 << bits) - 1;
+    for (int k = 1; k <= L; ++k) tl[k] = std::pow(((double)k - 0.5) / (double)L, inv);
     std::vector<int64_t> cls[3];
     for (int64_t i = 0; i < count; ++i) {
         const int g = opqk::qs_group_warps(jobs[i].K);
         cls[g == 1 ? 0 : (g == 4 ? 1 : 2)].push_back(i);
     }
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (!cls[0].empty() && (s = launch_quant_stream<1>(di, jobs, cls[0], qp, st)) != OPQ_OK) return s;
-    if (!cls[1].empty() && (s = launch_quant_stream<4>(di, jobs, cls[1], qp, st)) != OPQ_OK) return s;
-    if (!cls[2].empty() && (s = launch_quant_stream<8>(di, jobs, cls[2], qp, st)) != OPQ_OK) return s;
-    return OPQ_OK;
+    switch (bits) {
+        case 3: return launch_quant_classes<3>(di, jobs, cls, qp, tl, st);
+        case 5: return launch_quant_classes<5>(di, jobs, cls, qp, tl, st);
+        case 6: return launch_quant_classes<6>(di, jobs, cls, qp, tl, st);
+        default: return launch_quant_classes<4>(di, jobs, cls, qp, tl, st);
+    }
 }
 
 // group-wise format: group size 32, 64, 128 or 256 dividing K
@@ -547,30 +564,9 @@ opq_status opq_dequantize_grouped(const uint32_t *codes, const uint32_t *signs, 
 
 opq_status opq_quantize_bits(const uint16_t *w, int64_t N, int64_t K, int64_t ldw, int32_t bits, float alpha,
                              uint32_t *codes, uint32_t *signs, float *scales, void *stream) {
-    opq_status s = check_sizes(N, K);
-    if (s != OPQ_OK) return s;
     if (bits < 3 || bits > 6) return OPQ_ERR_INVALID_ARG;
-    if (ldw < K || ldw % 8 != 0) return OPQ_ERR_INVALID_ARG;
-    if (!alpha_ok(alpha)) return OPQ_ERR_INVALID_ARG;
-    if ((s = check_ptrs({w, codes, signs, scales})) != OPQ_OK) return s;
-    const int L = (1 << bits) - 1;
-    opqk::BitsQuantParams bp{};
-    const double inv = 1.0 / (double)alpha;
-    for (int k = 1; k <= L; ++k) bp.t[k] = std::pow(((double)k - 0.5) / (double)L, inv);
-    bp.alpha_is_one = (alpha == 1.0f) ? 1 : 0;
-    DeviceInfo *di = nullptr;
-    if ((s = device_info(&di)) != OPQ_OK) return s;
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    const int64_t blocks = (N + 7) / 8;
-    const int grid = (int)(blocks < (int64_t)di->sms * 8 ? blocks : (int64_t)di->sms * 8);
-    switch (bits) {
-        case 3: opqk::quantize_bits_kernel<3><<<grid, 256, 0, st>>>(w, N, K, ldw, bp, codes, signs, scales); break;
-        case 4: opqk::quantize_bits_kernel<4><<<grid, 256, 0, st>>>(w, N, K, ldw, bp, codes, signs, scales); break;
-        case 5: opqk::quantize_bits_kernel<5><<<grid, 256, 0, st>>>(w, N, K, ldw, bp, codes, signs, scales); break;
-        default: opqk::quantize_bits_kernel<6><<<grid, 256, 0, st>>>(w, N, K, ldw, bp, codes, signs, scales); break;
-    }
-    cudaError_t e = cudaGetLastError();
-    return e == cudaSuccess ? OPQ_OK : cuda_fail(e);
+    const opq_quant_job job = {w, N, K, ldw, codes, signs, scales};
+    return quantize_jobs(&job, 1, alpha, stream, bits);
 }
 
 opq_status opq_dequantize_bits(const uint32_t *codes, const uint32_t *signs, const float *scales, int64_t N, int64_t K,

@@ -246,89 +246,9 @@ namespace opqk {
 
 // ------------------------------------------------------------------------------------------
 // Other bit widths (3, 5, 6; 4 is the card's format): 2^BITS - 1 levels per row, the codes of
-// a row as one little-endian bit stream (element k at bits k * BITS of the row's words).
+// a row as one little-endian bit stream (element k at bits k * BITS of the row's words). Their
+// quantize is the row-streaming kernel (opq_quantize_stream.cuh) at BITS.
 // ------------------------------------------------------------------------------------------
-struct BitsQuantParams {
-    double t[64];      // t[k] = ((k - 1/2) / L)^(1/alpha), k = 1..L
-    int alpha_is_one;  // thresholds formed as max * (2k - 1) / (2L) (exact quotient)
-};
-
-// smallest bf16 magnitude (bits) that codes to >= k out of L levels (as level_threshold)
-__device__ __forceinline__ uint32_t level_threshold_L(float mxf, int k, int L, const BitsQuantParams &bp) {
-    const double th = bp.alpha_is_one ? ((double)mxf * (double)(2 * k - 1)) / (double)(2 * L) : (double)mxf * bp.t[k];
-    const float f = __double2float_ru(th);
-    const uint32_t fb = __float_as_uint(f);
-    uint32_t tb = (fb >> 16) + ((fb & 0xFFFFu) != 0u ? 1u : 0u);
-    const bool exact = ((fb & 0xFFFFu) == 0u) && ((double)f == th);
-    if ((k & 1) && exact) tb += 1u;
-    return tb < 0x7F80u ? tb : 0x7F80u;
-}
-
-// One warp per row: the row max (a first pass over the row), the row's L thresholds in shared
-// memory, then rounds of 256 weights: a binary search per weight over the thresholds, the
-// round's 8 BITS code words assembled in shared memory and stored together.
-template <int BITS>
-__global__ void __launch_bounds__(256) quantize_bits_kernel(const uint16_t *__restrict__ w, int64_t N, int64_t K,
-                                                            int64_t ldw, const __grid_constant__ BitsQuantParams bp,
-                                                            uint32_t *__restrict__ codes,
-                                                            uint32_t *__restrict__ signs,
-                                                            float *__restrict__ scales) {
-    constexpr int L = (1 << BITS) - 1;
-    constexpr int WPR = 8 * BITS;             // code words per round of 256 weights
-    __shared__ uint16_t thr[8][64];
-    __shared__ uint32_t pk[8][WPR];
-    const int lane = threadIdx.x & 31, wi = threadIdx.x >> 5;
-    const int64_t nvec = K / 8, rounds = (nvec + 31) / 32, cw = K * BITS / 32;
-    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
-    for (int64_t n = (int64_t)blockIdx.x * (blockDim.x >> 5) + wi; n < N; n += warps) {
-        const uint16_t *rp = w + n * ldw;
-        uint32_t mx = 0;
-        for (int64_t vi = lane; vi < nvec; vi += 32) {
-            const uint4 x = ld_stream_v4(rp + vi * 8);
-            const uint32_t m2 = __vmaxu2(__vmaxu2(x.x & 0x7FFF7FFFu, x.y & 0x7FFF7FFFu),
-                                         __vmaxu2(x.z & 0x7FFF7FFFu, x.w & 0x7FFF7FFFu));
-            mx = max(mx, max(m2 & 0xFFFFu, m2 >> 16));
-        }
-        mx = __reduce_max_sync(0xFFFFFFFFu, mx);
-        const float mxf = __uint_as_float(mx << 16);
-        if (lane == 0) scales[n] = mxf;
-        for (int k = lane + 1; k <= L; k += 32)
-            thr[wi][k] = (uint16_t)(mx != 0u ? level_threshold_L(mxf, k, L, bp) : 0x7F80u);
-        __syncwarp();
-        for (int64_t r = 0; r < rounds; ++r) {
-            const int64_t vi = r * 32 + lane;
-            const bool valid = vi < nvec;
-            const uint4 x = valid ? ld_stream_v4(rp + vi * 8) : make_uint4(0, 0, 0, 0);
-            for (int j = lane; j < WPR; j += 32) pk[wi][j] = 0u;
-            __syncwarp();
-            const uint32_t words[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const uint32_t a = (words[e >> 1] >> (16 * (e & 1))) & 0x7FFFu;
-                uint32_t q = 0;
-#pragma unroll
-                for (int step = (L + 1) / 2; step > 0; step >>= 1)
-                    if (a >= thr[wi][q + step]) q += step;
-                const int bit = (lane * 8 + e) * BITS;
-                atomicOr(&pk[wi][bit >> 5], q << (bit & 31));
-                if ((bit & 31) + BITS > 32) atomicOr(&pk[wi][(bit >> 5) + 1], q >> (32 - (bit & 31)));
-            }
-            const uint32_t sb = opqbits::sign_byte(opqbits::bf16x2_neg_mask(x.x), opqbits::bf16x2_neg_mask(x.y),
-                                                   opqbits::bf16x2_neg_mask(x.z), opqbits::bf16x2_neg_mask(x.w));
-            uint32_t sw = sb << (8 * (lane & 3));
-            sw |= __shfl_xor_sync(0xFFFFFFFFu, sw, 1);
-            sw |= __shfl_xor_sync(0xFFFFFFFFu, sw, 2);
-            if (valid && (lane & 3) == 0) signs[n * (nvec / 4) + vi / 4] = sw;
-            __syncwarp();
-            // valid vectors of the round come in fours (K % 32 == 0): BITS words per four
-            const int64_t nv = min((int64_t)32, nvec - r * 32);
-            const int nw = (int)(nv * BITS / 4);
-            for (int j = lane; j < nw; j += 32) codes[n * cw + r * WPR + j] = pk[wi][j];
-            __syncwarp();
-        }
-    }
-}
-
 struct BitsDequantParams {
     double lut[64];    // (q/L)^(1/alpha), q = 0..L
 };

@@ -1,5 +1,5 @@
 // opq_quantize.cuh — the per-row arithmetic shared by the quantize kernels: the exact
-// thresholds of the 15 levels.
+// thresholds of the 15 levels (and of the 2^bits - 1 levels of the other bit widths).
 //
 // "OPQ INT4 Z-Image" model card, "OPQ principle": u = |w|/max, v = u^alpha, q = round(15 v).
 // No pow is evaluated on the device: the host forms t_k = ((k - 1/2)/15)^(1/alpha) in fp64,
@@ -38,6 +38,18 @@ __device__ __forceinline__ uint32_t level_threshold(float mxf, int k, const Quan
     const bool exact = ((fb & 0xFFFFu) == 0u) && ((double)f == th);
     if ((k & 1) && exact) tb += 1u;
     return tb < 0x7F80u ? tb : 0x7F80u;   // +inf: unreachable (only for a non-finite max)
+}
+
+// The same for a row coded on L levels (other bit widths): t_k = ((k - 1/2) / L)^(1/alpha), or
+// with alpha = 1 the exact quotient max (2k - 1) / (2L).
+__device__ __forceinline__ uint32_t level_threshold_levels(float mxf, int k, int L, double tk, int alpha_is_one) {
+    const double th = alpha_is_one ? ((double)mxf * (double)(2 * k - 1)) / (double)(2 * L) : (double)mxf * tk;
+    const float f = __double2float_ru(th);
+    const uint32_t fb = __float_as_uint(f);
+    uint32_t tb = (fb >> 16) + ((fb & 0xFFFFu) != 0u ? 1u : 0u);
+    const bool exact = ((fb & 0xFFFFu) == 0u) && ((double)f == th);
+    if ((k & 1) && exact) tb += 1u;
+    return tb < 0x7F80u ? tb : 0x7F80u;
 }
 
 }  // namespace opqk

@@ -21,6 +21,10 @@
 //                  weight, a pair's code byte is one merge.
 // Every weight is read from HBM once. The ring holds the copies of many rows in flight, the
 // registers hold the rows being coded, so the stream does not pause between rows.
+// The card's configuration also lists 3, 5 and 6 bits per magnitude: the same kernel at BITS
+// codes 2^BITS - 1 levels (thresholds in lanes 0..L-1, and 32..62 a second time for 6 bits),
+// table entries q itself, and writes each row's codes as one bit stream: the four lanes that
+// hold 32 consecutive weights assemble their BITS words with funnel shifts.
 #pragma once
 #include "opq_quantize.cuh"
 
@@ -59,7 +63,7 @@ struct QsCfg {
 
 struct QsJob {
     const uint16_t *w;     // bf16 [N, ldw]
-    uint32_t *codes;       // [N, K/8]
+    uint32_t *codes;       // [N, K bits / 32]: the row's codes (for 4 bits, 8 nibbles per word)
     uint32_t *signs;       // [N, K/32]
     float *scales;         // [N]
     int64_t ldw;
@@ -68,7 +72,8 @@ struct QsJob {
 };
 
 struct QsParams {
-    QuantParams qp;
+    QuantParams qp;        // the 15 levels of the 4-bit format (and alpha_is_one for every width)
+    double tl[64];         // other widths: t_k = ((k - 1/2) / L)^(1/alpha), k = 1..L
     int64_t rows;          // all rows of the launch
     int32_t njobs;
     int32_t nslots;        // ring slots S
@@ -101,9 +106,27 @@ __device__ __forceinline__ int qs_job_of(const QsParams &p, int64_t u, int j) {
     return j;
 }
 
-template <int G>
+// The 8 codes q[] of vector v (BITS bits each) into the row's bit stream crow: every lane calls
+// this (it shuffles within the lane's quad of consecutive vectors); `valid` lanes store.
+template <int BITS>
+__device__ __forceinline__ void qs_store_codes(uint32_t *crow, int v, const uint32_t (&q)[8], int lane, bool valid) {
+    uint32_t lo, hi;
+    opqbits::pack_chunk<BITS>(q, lo, hi);
+    const uint32_t nlo = __shfl_down_sync(0xFFFFFFFFu, lo, 1), nhi = __shfl_down_sync(0xFFFFFFFFu, hi, 1);
+    uint32_t *quad = crow + (size_t)(v >> 2) * BITS;
+#pragma unroll
+    for (uint32_t t = 0; t < 2; ++t) {
+        uint32_t w, word;
+        if (opqbits::quad_word<BITS>(lo, hi, nlo, nhi, (uint32_t)lane & 3u, t, w, word) && valid) quad[w] = word;
+    }
+}
+
+// BITS = 4: the card's nibble format; 3, 5, 6: 2^BITS - 1 levels, each row's codes one
+// little-endian bit stream (element k at bits k BITS .. k BITS + BITS - 1 of the row's words).
+template <int G, int BITS = 4>
 __global__ void __launch_bounds__(QS_THREADS, 1) quantize_stream_kernel(const __grid_constant__ QsParams p) {
     using C = QsCfg<G>;
+    constexpr int L = (1 << BITS) - 1;
     constexpr int NG = C::NG, GT = 32 * G;
     extern __shared__ __align__(128) uint8_t qs_smem[];
     __shared__ __align__(16) uint32_t qs_tab[NG * C::TAB / 4];
@@ -213,45 +236,100 @@ __global__ void __launch_bounds__(QS_THREADS, 1) quantize_stream_kernel(const __
                 break;
             }
             const float mxf = __uint_as_float(mx << 16);
-            uint32_t myT = 0x7F80u;   // +inf: a level no finite weight reaches (every level of a zero row)
-            if (lane < 15 && mx != 0u) myT = level_threshold(mxf, lane + 1, p.qp);
+            // the thresholds of levels lane + 1 and (6 bits) lane + 33; +inf: a level no finite
+            // weight reaches (every level of a zero row)
+            uint32_t myT = 0x7F80u, myT2 = 0x7F80u;
+            if (mx != 0u) {
+                if (BITS == 4) {
+                    if (lane < 15) myT = level_threshold(mxf, lane + 1, p.qp);
+                } else {
+                    if (lane < L) myT = level_threshold_levels(mxf, lane + 1, L, p.tl[lane + 1], p.qp.alpha_is_one);
+                    if (L > 32 && lane + 32 < L)
+                        myT2 = level_threshold_levels(mxf, lane + 33, L, p.tl[lane + 33], p.qp.alpha_is_one);
+                }
+            }
             const uint32_t T1 = __shfl_sync(0xFFFFFFFFu, myT, 0);
             const uint32_t dz = T1 <= mx ? mx - T1 + 1u : 0u;
             if (tg == 0) J.scales[n] = mxf;
-            uint32_t *crow = J.codes + n * (int64_t)nvec;
+            uint32_t *crow = J.codes + n * ((int64_t)nvec * BITS / 4);
             // group-uniform: mx is the group's max
             if (mx <= 0x7F80u && dz < (uint32_t)C::TAB) {
                 // the table q(e) = #{k : B_k > e}, e = 0 .. d_z, from the level boundaries
                 // B_k = bits(max) - T_k + 1 held by lanes 0..14: per stretch of GT words (one per
                 // thread of the group) one ballot counts the levels that hold over the whole stretch
                 // and the few boundaries inside it correct each word (no per-entry walk)
-                const int Bk = (lane < 15 && myT <= mx) ? (int)mx - (int)myT + 1 : 0;
+                const int Bk = (lane < L && myT <= mx) ? (int)mx - (int)myT + 1 : 0;
+                const int Bk2 = (L > 32 && lane + 32 < L && myT2 <= mx) ? (int)mx - (int)myT2 + 1 : 0;
                 const uint32_t words = (dz + 4u) >> 2;
                 for (uint32_t i0 = 0; i0 < words; i0 += GT) {
                     const int lo_e = (int)(4u * i0), hi_e = lo_e + 4 * GT - 1;
                     const uint32_t w = i0 + (uint32_t)tg;
-                    uint32_t word = __popc(__ballot_sync(0xFFFFFFFFu, Bk > hi_e)) * 0x01010101u;
-                    uint32_t in_m = __ballot_sync(0xFFFFFFFFu, Bk > lo_e && Bk <= hi_e);
-                    while (in_m) {
-                        const int k = __ffs(in_m) - 1;
-                        in_m &= in_m - 1u;
-                        const int B = __shfl_sync(0xFFFFFFFFu, Bk, k);
-                        const int c = min(max(B - (int)(4u * w), 0), 4);
-                        word += __funnelshift_rc(0x01010101u, 0u, 8 * (4 - c));
-                    }
-                    if (w < words) qs_tab[base / 4 + w] = word * 0x11u;
+                    uint32_t cnt = __popc(__ballot_sync(0xFFFFFFFFu, Bk > hi_e));
+                    if (L > 32) cnt += __popc(__ballot_sync(0xFFFFFFFFu, Bk2 > hi_e));
+                    uint32_t word = cnt * 0x01010101u;
+                    auto inside = [&](int Bl) {
+                        uint32_t in_m = __ballot_sync(0xFFFFFFFFu, Bl > lo_e && Bl <= hi_e);
+                        while (in_m) {
+                            const int k = __ffs(in_m) - 1;
+                            in_m &= in_m - 1u;
+                            const int B = __shfl_sync(0xFFFFFFFFu, Bl, k);
+                            const int c = min(max(B - (int)(4u * w), 0), 4);
+                            word += __funnelshift_rc(0x01010101u, 0u, 8 * (4 - c));
+                        }
+                    };
+                    inside(Bk);
+                    if (L > 32) inside(Bk2);
+                    // 4 bits: q in both nibbles (a pair's code byte is one merge); else q itself
+                    if (w < words) qs_tab[base / 4 + w] = BITS == 4 ? word * 0x11u : word;
                 }
                 if (G > 1) group_sync(bar_id, GT); else __syncwarp();
                 const uint32_t mmb = (mx + base) * 0x00010001u, lo2 = (mx - dz) * 0x00010001u;
 #pragma unroll
                 for (int k = 0; k < QS_VMAX; ++k) {
                     const int v = k * GT + tg;
-                    if (v < nvec) {
+                    if constexpr (BITS == 4) {
+                        if (v < nvec) {
+                            const uint4 x = a[k];
+                            crow[v] = opqbits::codes_word(opqbits::table_byte_clamped(tb, x.x, lo2, mmb),
+                                                          opqbits::table_byte_clamped(tb, x.y, lo2, mmb),
+                                                          opqbits::table_byte_clamped(tb, x.z, lo2, mmb),
+                                                          opqbits::table_byte_clamped(tb, x.w, lo2, mmb));
+                        }
+                    } else if (k * GT < nvec) {   // the batch is in the row for some lane: shuffles need them all
                         const uint4 x = a[k];
-                        crow[v] = opqbits::codes_word(opqbits::table_byte_clamped(tb, x.x, lo2, mmb),
-                                                      opqbits::table_byte_clamped(tb, x.y, lo2, mmb),
-                                                      opqbits::table_byte_clamped(tb, x.z, lo2, mmb),
-                                                      opqbits::table_byte_clamped(tb, x.w, lo2, mmb));
+                        uint32_t q[8];
+                        opqbits::table_pair_bytes(tb, x.x, lo2, mmb, q[0], q[1]);
+                        opqbits::table_pair_bytes(tb, x.y, lo2, mmb, q[2], q[3]);
+                        opqbits::table_pair_bytes(tb, x.z, lo2, mmb, q[4], q[5]);
+                        opqbits::table_pair_bytes(tb, x.w, lo2, mmb, q[6], q[7]);
+                        qs_store_codes<BITS>(crow, v, q, lane, v < nvec);
+                    }
+                }
+            } else if (BITS != 4) {
+                // rows whose table would not fit (small alpha) or whose max is not finite: a binary
+                // search per weight over the L thresholds, held in the group's table area
+                uint16_t *thr = reinterpret_cast<uint16_t *>(qs_tab) + base / 2;   // thr[k], k = 1..L
+                if (wg == 0) {
+                    if (lane < L) thr[lane + 1] = (uint16_t)myT;
+                    if (L > 32 && lane + 32 < L) thr[lane + 33] = (uint16_t)myT2;
+                }
+                if (G > 1) group_sync(bar_id, GT); else __syncwarp();
+#pragma unroll
+                for (int k = 0; k < QS_VMAX; ++k) {   // unrolled: the row stays in registers
+                    const int v = k * GT + tg;
+                    if (k * GT < nvec) {
+                        const uint32_t m[4] = {a[k].x, a[k].y, a[k].z, a[k].w};
+                        uint32_t q[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const uint32_t mag = (m[e >> 1] >> (16 * (e & 1))) & 0x7FFFu;
+                            uint32_t qq = 0;
+#pragma unroll
+                            for (int step = (L + 1) / 2; step > 0; step >>= 1)
+                                if (mag >= thr[qq + step]) qq += step;
+                            q[e] = qq;
+                        }
+                        qs_store_codes<BITS>(crow, v, q, lane, v < nvec);
                     }
                 }
             } else {

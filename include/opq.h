@@ -182,6 +182,9 @@ opq_status opq_linear_grouped_fused(const uint16_t *x, int64_t M, int64_t K, con
  * of the row's K*bits/32 uint32 words (for 4 bits: nibble k % 8 of word k / 8,
  * the per-row format above). Signs and scales as in the per-row format.
  *   codes  uint32 [N, K*bits/32];  bits 3..6 (OPQ_ERR_INVALID_ARG otherwise)
+ * opq_quantize_bits takes the arguments and limits of opq_quantize (K % 32 == 0,
+ * K <= 32768, ldw >= K, ldw % 8 == 0, w 16-byte aligned) and runs the same
+ * row-streaming kernel at the given width.
  */
 opq_status opq_quantize_bits(const uint16_t *w, int64_t N, int64_t K, int64_t ldw, int32_t bits, float alpha,
                              uint32_t *codes, uint32_t *signs, float *scales, void *stream);

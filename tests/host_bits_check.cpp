@@ -6,6 +6,7 @@
 #include <random>
 #include <algorithm>
 #include <vector>
+#include <type_traits>
 #include "opq_bits.h"
 
 using namespace opqbits;
@@ -213,6 +214,58 @@ int main() {
         const uint32_t b[4] = {(uint32_t)rng(), (uint32_t)rng(), (uint32_t)rng(), (uint32_t)rng()};
         const uint32_t want = (b[0] & 0xFFu) | ((b[1] & 0xFFu) << 8) | ((b[2] & 0xFFu) << 16) | ((b[3] & 0xFFu) << 24);
         CHECK(codes_word(b[0], b[1], b[2], b[3]) == want, "codes_word %x %x %x %x", b[0], b[1], b[2], b[3]);
+    }
+    // other bit widths: 32 random codes of a quad as pieces (pack_chunk) and the quad's words
+    // (quad_word over its four lanes) against the bit stream written one bit at a time
+    auto check_stream = [&](auto bits_tag) {
+        constexpr int B = decltype(bits_tag)::value;
+        for (int t = 0; t < 2000; ++t) {
+            uint32_t q[32];
+            for (int e = 0; e < 32; ++e) q[e] = (uint32_t)(rng() & ((1u << B) - 1u));
+            if (t == 0) for (int e = 0; e < 32; ++e) q[e] = (1u << B) - 1u;   // all ones
+            uint32_t want[B] = {};
+            for (int e = 0; e < 32; ++e)
+                for (int b = 0; b < B; ++b)
+                    if ((q[e] >> b) & 1u) want[(e * B + b) / 32] |= 1u << ((e * B + b) % 32);
+            uint32_t lo[5], hi[5];
+            for (int i = 0; i < 4; ++i) {
+                uint32_t qq[8];
+                for (int e = 0; e < 8; ++e) qq[e] = q[8 * i + e];
+                pack_chunk<B>(qq, lo[i], hi[i]);
+            }
+            lo[4] = (uint32_t)rng();   // the next quad's lane 0: must not matter
+            hi[4] = (uint32_t)rng();
+            int seen[B] = {};
+            for (uint32_t i = 0; i < 4; ++i)
+                for (uint32_t tt = 0; tt < 2; ++tt) {
+                    uint32_t w = 0, word = 0;
+                    if (!quad_word<B>(lo[i], hi[i], lo[i + 1], hi[i + 1], i, tt, w, word)) continue;
+                    CHECK(w < (uint32_t)B, "quad_word<%d> word index %u", B, w);
+                    if (w >= (uint32_t)B) continue;
+                    ++seen[w];
+                    CHECK(word == want[w], "quad_word<%d> t %d lane %u word %u got %x want %x", B, t, i, w, word, want[w]);
+                }
+            for (int w = 0; w < B; ++w) CHECK(seen[w] == 1, "quad_word<%d> word %d written %d times", B, w, seen[w]);
+        }
+    };
+    check_stream(std::integral_constant<int, 3>{});
+    check_stream(std::integral_constant<int, 4>{});
+    check_stream(std::integral_constant<int, 5>{});
+    check_stream(std::integral_constant<int, 6>{});
+    // table_pair_bytes: both codes of a magnitude pair from a table of plain q bytes
+    {
+        std::vector<uint8_t> tb(0x10000);
+        for (auto &b : tb) b = (uint8_t)(rng() & 63u);
+        for (int t = 0; t < 20000; ++t) {
+            const uint32_t mx = 0x3000u + (uint32_t)(rng() % 0x4000u), dz = 1u + (uint32_t)(rng() % 1500u);
+            const uint32_t base = 4096u * (uint32_t)(rng() % 8u);
+            if (mx + base >= 0x10000u || dz > mx) continue;
+            const uint32_t a0 = (uint32_t)(rng() % (mx + 1u)), a1 = (uint32_t)(rng() % (mx + 1u));
+            uint32_t q0 = 0, q1 = 0;
+            table_pair_bytes(tb.data(), a0 | (a1 << 16), (mx - dz) * 0x00010001u, (mx + base) * 0x00010001u, q0, q1);
+            const uint32_t e0 = mx - std::max(a0, mx - dz), e1 = mx - std::max(a1, mx - dz);
+            CHECK(q0 == tb[base + e0] && q1 == tb[base + e1], "table_pair_bytes %x %x mx %x dz %u", a0, a1, mx, dz);
+        }
     }
     std::printf("%s fails=%d\n", fails ? "FAIL" : "OK", fails);
     return fails ? 1 : 0;
