@@ -384,6 +384,10 @@ def gpu_arm(args, rank, world, local_rank):
     # ---------------------------------------------------------------- e2e: host buffers
     # Every step copies all 210 weights and both activation tensors from host memory, runs
     # the three phases through the public calls and copies every layer's y back to the host.
+    # The step is pipelined by transformer block (7 layers): the block's weights go up on a
+    # copy stream, its quantize (one batched call), linears and dequantizes run on the compute
+    # stream once they have landed, and each layer's y goes down on a second copy stream as
+    # soon as its linear is done (both copy directions run at once). Steps do not overlap.
     e2e = None
     if not args.no_e2e:
         total_bytes = S.W.numel() * 2
@@ -393,23 +397,45 @@ def gpu_arm(args, rank, world, local_rank):
         reg = cudart.cudaHostRegister(w_host.data_ptr(), total_bytes, 0)
         registered = int(reg) == 0
         x_host = {k: v.cpu().pin_memory() for k, v in S.x.items()}
-        y_host = {n: torch.empty(v.shape, dtype=v.dtype).pin_memory() for n, v in S.y.items()}
+        blocks = [S.layers[i:i + 7] for i in range(0, len(S.layers), 7)]
+        bjobs = [(opq.quantize_jobs([L["w"] for L in B], [(L["c"], L["s"], L["sc"]) for L in B], alpha),
+                  [L["w"] for L in B], [(L["c"], L["s"], L["sc"]) for L in B]) for B in blocks]
+        y_dev = [torch.empty((M, L["N"]), dtype=torch.bfloat16, device=dev) for L in S.layers]
+        y_host = [torch.empty((M, L["N"]), dtype=torch.bfloat16).pin_memory() for L in S.layers]
+        s_up, s_down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
 
         def e2e_step():
-            for k in S.x:
-                S.x[k].copy_(x_host[k], non_blocking=True)
-            for L in S.layers:
-                n, k = L["N"], L["K"]
-                L["w"].copy_(w_host[L["off"]:L["off"] + n * k].view(n, k), non_blocking=True)
-            for c in cls_names:
-                jobs, ws_, outs_ = S.jobs[c]
+            s_up.wait_stream(stream)
+            s_down.wait_stream(stream)
+            landed = []
+            with torch.cuda.stream(s_up):
+                for k in S.x:
+                    S.x[k].copy_(x_host[k], non_blocking=True)
+                for B in blocks:
+                    for L in B:
+                        n, k = L["N"], L["K"]
+                        L["w"].copy_(w_host[L["off"]:L["off"] + n * k].view(n, k), non_blocking=True)
+                    e = torch.cuda.Event()
+                    e.record(s_up)
+                    landed.append(e)
+            done = []
+            i = 0
+            for B, (jobs, ws_, outs_), e in zip(blocks, bjobs, landed):
+                stream.wait_event(e)
                 opq.quantize_batched(ws_, alpha, outs=outs_, jobs=jobs)
-            for L in S.layers:
-                y = S.y[L["N"]]
-                opq.linear(S.x[L["K"]], L["c"], L["s"], L["sc"], alpha, out=y, workspace=S.ws)
-                y_host[L["N"]].copy_(y, non_blocking=True)
-            for L in S.layers:
-                opq.dequantize(L["c"], L["s"], L["sc"], alpha, out=L["wq"])
+                for L in B:
+                    opq.linear(S.x[L["K"]], L["c"], L["s"], L["sc"], alpha, out=y_dev[i], workspace=S.ws)
+                    ev = torch.cuda.Event()
+                    ev.record(stream)
+                    done.append(ev)
+                    opq.dequantize(L["c"], L["s"], L["sc"], alpha, out=L["wq"])
+                    i += 1
+            with torch.cuda.stream(s_down):
+                for i, ev in enumerate(done):
+                    s_down.wait_event(ev)
+                    y_host[i].copy_(y_dev[i], non_blocking=True)
+            stream.wait_stream(s_up)
+            stream.wait_stream(s_down)
 
         e2e_step()
         torch.cuda.synchronize()
@@ -429,10 +455,12 @@ def gpu_arm(args, rank, world, local_rank):
         e2e = {"value": whole_job_tflops(world, flops, ms_e2e), "unit": "TFLOP/s", "ms_per_step": ms_e2e,
                "steps": e_steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "host_weights": "registered (page-locked) host memory" if registered else "pageable host memory",
-               "copies": "210 weight H2D + 2 activation H2D + 210 y D2H per step"}
+               "copies": "210 weight H2D + 2 activation H2D + 210 y D2H per step",
+               "pipeline": "per transformer block: weights up on one copy stream, quantize + linear + "
+                           "dequantize on the compute stream, each y down on another copy stream"}
         if registered:
             cudart.cudaHostUnregister(w_host.data_ptr())
-        del w_host
+        del w_host, y_dev, y_host
     traffic = recorded_traffic("wide_kernel_whole_model")
     roof = {"bound": "tensor", "kernel": "opqk_wide::wide_kernel<256, 0>", "achieved": linear_tflops,
             "peak": bf16, "unit": "TFLOP/s", "frac": linear_tflops / bf16,
