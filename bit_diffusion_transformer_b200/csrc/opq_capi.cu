@@ -354,6 +354,13 @@ cudaError_t launch_linear_wide(DeviceInfo *di, const Plan &plan, const CUtensorM
         cudaError_t e = cudaFuncSetAttribute(opqk_wide::wide_kernel<256, GS, BITS>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
         if (e != cudaSuccess) return e;
+        if (C::REG_SPLIT) {
+            // the kernel's warpgroups trade registers (setmaxnreg) on the assumption that each
+            // thread was launched with REG_LAUNCH of them; any other count is refused, not run
+            cudaFuncAttributes fa{};
+            if ((e = cudaFuncGetAttributes(&fa, opqk_wide::wide_kernel<256, GS, BITS>)) != cudaSuccess) return e;
+            if (fa.numRegs != C::REG_LAUNCH) return cudaErrorInvalidConfiguration;
+        }
         attr = true;
     }
     cudaError_t e = launch_programmatic(opqk_wide::wide_kernel<256, GS, BITS>, plan.grid, C::THREADS, C::SMEM_BYTES, st,

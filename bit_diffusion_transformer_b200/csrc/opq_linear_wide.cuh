@@ -10,9 +10,11 @@
 //                per stage, one 128-K block per copy
 //   warp 1       TMEM allocation and the MMA issue; A from TMEM, B = x from shared memory
 //   warp 2       x producer: 256 rows x 64 K per copy, two per block (128-byte swizzle)
-//   warps 3..10  two decoder groups (4 warps = the 128 TMEM lanes) through the pair table,
+//   warps 4..11  two decoder groups (4 warps = the 128 TMEM lanes) through the pair table,
 //                A written to TMEM with tcgen05.st
-//   warps 11..14 epilogue
+//   warps 12..15 epilogue: the tile's sums into registers as bf16 pairs, the accumulator
+//                released, then y stored while the next tile's MMAs run (the producers'
+//                warpgroup hands registers to the epilogue's with setmaxnreg)
 // Whole tiles are strided over the CTAs; tiles past the last whole wave (at most half as
 // many as CTAs) run as two 128-row halves on two CTAs. The narrow-tile kernel
 // (opq_linear.cuh) fetches several blocks per copy and splits K over CTAs instead; at this
@@ -164,7 +166,9 @@ struct Cfg {
     // (block b - GROUPS - A_BLOCKS) succeeded; the parity test is exact only if that implies block
     // b - A_BLOCKS - NDONE has completed, i.e. NDONE >= GROUPS (completions come in block order)
     static_assert(NDONE >= GROUPS, "done ring shorter than the decoder rotation");
-    static constexpr int WARP_LOAD = 0, WARP_MMA = 1, WARP_XLOAD = 2, WARP_DEC0 = 3, NUM_DEC_WARPS = 4 * GROUPS;
+    // Warpgroup-aligned roles (the register split below goes by warpgroup): warps 0..3 the
+    // producers and the MMA issuer (warp 3 idle), then the decoder groups, then the epilogue.
+    static constexpr int WARP_LOAD = 0, WARP_MMA = 1, WARP_XLOAD = 2, WARP_DEC0 = 4, NUM_DEC_WARPS = 4 * GROUPS;
     static constexpr int WARP_EPI0 = WARP_DEC0 + NUM_DEC_WARPS;
     // One MMA-issuing thread per accumulation chain: a thread issues one tcgen05.mma every
     // few dozen cycles, far slower than the tensor pipe runs a narrow (N <= 64) MMA, so the
@@ -172,6 +176,17 @@ struct Cfg {
     static constexpr int NISS = NCHAIN;
     static constexpr int WARP_ISS1 = WARP_EPI0 + 4;
     static constexpr int THREADS = (WARP_ISS1 + NISS - 1) * 32;
+    // Register split (BX = 256: four warpgroups). The epilogue holds the whole tile's sums as
+    // bf16 pairs (BX / 2 registers) so that it can release the single accumulator before it
+    // stores y; the producers' warpgroup gives up what the epilogue takes. The host checks that
+    // the kernel was built for exactly REG_LAUNCH registers per thread before launching it.
+    static constexpr bool REG_SPLIT = THREADS == 512 && GROUPS == 2 && NISS == 1;
+    static constexpr int REG_LAUNCH = 128;
+    static constexpr int REG_PROD = 80, REG_DEC = 120, REG_EPI = 4 * REG_LAUNCH - REG_PROD - 2 * REG_DEC;
+    static_assert(!REG_SPLIT || (REG_PROD + 2 * REG_DEC + REG_EPI == 4 * REG_LAUNCH && REG_EPI <= 256 &&
+                                 REG_PROD % 8 == 0 && REG_DEC % 8 == 0 && REG_EPI % 8 == 0 &&
+                                 THREADS * REG_LAUNCH == 65536),
+                  "register split must add up to the launch's registers");
     static_assert(SMEM_BYTES <= 232448, "shared memory");
     static_assert(BX % 16 == 0 && BX >= 16 && BX <= 256, "MMA N");
     static_assert(A_COLS + NACC * ACC_COLS <= 512, "TMEM columns");
@@ -220,6 +235,7 @@ __global__ void __launch_bounds__(Cfg<BX, BITS>::THREADS, 1)
                   const __grid_constant__ LinearArgs args) {
     using C = Cfg<BX, BITS>;
     static_assert(BITS == 4 || GS == 0, "the other bit widths take per-row scales");
+    static_assert(C::NISS == 1, "one MMA issuer (warp 1)");
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t sbase = smem_u32(smem);
     if ((sbase & 1023u) != 0u) {   // the same for every CTA: nothing has been started yet
@@ -336,141 +352,146 @@ __global__ void __launch_bounds__(Cfg<BX, BITS>::THREADS, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    if (warp == C::WARP_LOAD) {
-        // ----------------------------------------------------------- raw producer
-        pdl_wait();
-        const int swd = args.K / 32;        // sign words per row
-        int rs = 0;
-        uint32_t rph = 0;
-        int raw_issued = 0;
-        bool ok = true;
-        pre_raw = __shfl_sync(0xFFFFFFFFu, pre_raw, 0);
-        while (ok && it.next(tile, r0, r1, j)) {
-            const int n_blk = tile / args.m_tiles;
-            for (int r = r0; r < r1 && ok; ++r) {
-                if (raw_issued < pre_raw) {   // issued before the CTA-wide barrier
+    if (warp < C::WARP_DEC0) {
+        // the producers' warpgroup (warp 3 idle) gives registers to the epilogue's
+        if constexpr (C::REG_SPLIT) setmaxnreg_dec<C::REG_PROD>();
+        if (warp == C::WARP_LOAD) {
+            // ----------------------------------------------------------- raw producer
+            pdl_wait();
+            const int swd = args.K / 32;        // sign words per row
+            int rs = 0;
+            uint32_t rph = 0;
+            int raw_issued = 0;
+            bool ok = true;
+            pre_raw = __shfl_sync(0xFFFFFFFFu, pre_raw, 0);
+            while (ok && it.next(tile, r0, r1, j)) {
+                const int n_blk = tile / args.m_tiles;
+                for (int r = r0; r < r1 && ok; ++r) {
+                    if (raw_issued < pre_raw) {   // issued before the CTA-wide barrier
+                        ++raw_issued;
+                        if (++rs == C::RAW_STAGES) { rs = 0; rph ^= 1; }
+                        continue;
+                    }
+                    // lane 0 waits for the stage; the verdict and the ordering reach the other lanes
+                    int okw = 1;
+                    if (lane == 0) okw = mbar_wait(&raw_empty[rs], rph ^ 1) ? 1 : 0;
+                    okw = __shfl_sync(0xFFFFFFFFu, okw, 0);
+                    __syncwarp();
+                    if (!okw) { ok = false; break; }
+                    const uint32_t dst = sbase + C::OFF_RAW + rs * C::RAW_BYTES;
+                    if (lane == 0) {
+                        if (signs_by_tma) {
+                            issue_raw(rs, r, n_blk);
+                        } else {
+                            mbar_arrive_expect_tx(&raw_full[rs], C::RAW_CODE_BYTES);
+                            tma_load_2d(smem + C::OFF_RAW + rs * C::RAW_BYTES, &tmap_codes, r * C::CODE_WORDS,
+                                        n_blk * C::BW, &raw_full[rs]);
+                        }
+                    }
+                    if (!signs_by_tma) {
+                        // sign words: 128 rows x 4 words; copy i of lane l is word 32 i + l of the stage
+                        // (consecutive lanes, consecutive banks); out-of-range words read as 0
+    #pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const int e = i * 32 + lane;
+                            const int row = e >> 2, w = e & 3;
+                            const int n = n_blk * C::BW + row, kw = r * 4 + w;
+                            const bool in = n < args.N && kw < swd;
+                            const uint32_t *src = args.signs + (in ? (size_t)n * swd + kw : 0);
+                            cp_async_4(dst + C::RAW_CODE_BYTES + row * 16 + w * 4, src, in ? 4u : 0u);
+                        }
+                        cp_async_mbar_arrive(&raw_full[rs]);
+                    }
                     ++raw_issued;
                     if (++rs == C::RAW_STAGES) { rs = 0; rph ^= 1; }
-                    continue;
-                }
-                // lane 0 waits for the stage; the verdict and the ordering reach the other lanes
-                int okw = 1;
-                if (lane == 0) okw = mbar_wait(&raw_empty[rs], rph ^ 1) ? 1 : 0;
-                okw = __shfl_sync(0xFFFFFFFFu, okw, 0);
-                __syncwarp();
-                if (!okw) { ok = false; break; }
-                const uint32_t dst = sbase + C::OFF_RAW + rs * C::RAW_BYTES;
-                if (lane == 0) {
-                    if (signs_by_tma) {
-                        issue_raw(rs, r, n_blk);
-                    } else {
-                        mbar_arrive_expect_tx(&raw_full[rs], C::RAW_CODE_BYTES);
-                        tma_load_2d(smem + C::OFF_RAW + rs * C::RAW_BYTES, &tmap_codes, r * C::CODE_WORDS,
-                                    n_blk * C::BW, &raw_full[rs]);
-                    }
-                }
-                if (!signs_by_tma) {
-                    // sign words: 128 rows x 4 words; copy i of lane l is word 32 i + l of the stage
-                    // (consecutive lanes, consecutive banks); out-of-range words read as 0
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int e = i * 32 + lane;
-                        const int row = e >> 2, w = e & 3;
-                        const int n = n_blk * C::BW + row, kw = r * 4 + w;
-                        const bool in = n < args.N && kw < swd;
-                        const uint32_t *src = args.signs + (in ? (size_t)n * swd + kw : 0);
-                        cp_async_4(dst + C::RAW_CODE_BYTES + row * 16 + w * 4, src, in ? 4u : 0u);
-                    }
-                    cp_async_mbar_arrive(&raw_full[rs]);
-                }
-                ++raw_issued;
-                if (++rs == C::RAW_STAGES) { rs = 0; rph ^= 1; }
-            }
-        }
-        if (!ok) {
-            // let every copy already issued land before the CTA can exit
-            asm volatile("cp.async.wait_all;" ::: "memory");
-            if (lane == 0) {
-                for (int i = 0; i < raw_issued && i < C::RAW_STAGES; ++i) {
-                    if (--rs < 0) { rs = C::RAW_STAGES - 1; rph ^= 1; }
-                    (void)mbar_wait(&raw_full[rs], rph);
-                }
-            }
-        }
-    } else if (warp == C::WARP_XLOAD) {
-        // ----------------------------------------------------------- x producer
-        if (lane == 0) {
-            int b = 0;                 // the CTA's block index
-            bool ok = true;
-            int xoff, xrows;
-            while (ok && it.next(tile, r0, r1, j, xoff, xrows, BX)) {
-                for (int r = r0; r < r1; ++r, ++b) {
-                    if (b < pre_x) continue;   // issued before the CTA-wide barrier
-                    // stage b % X_STAGES last held block b - X_STAGES
-                    const int prev = b - C::X_STAGES;
-                    if (prev >= 0 && !mbar_wait(&blk_done[prev % C::NDONE], (uint32_t)(prev / C::NDONE) & 1u)) {
-                        ok = false;
-                        break;
-                    }
-                    // a half-width run loads its BX/2 activation rows with the half-height box
-                    issue_x(b, r, tile, xoff, xrows);
                 }
             }
             if (!ok) {
-                // let the copies already issued land before the CTA can exit (a slot whose decoder
-                // arrivals never come ends this wait by its time limit)
-                for (int i = 1; i <= C::X_STAGES && b - i >= 0; ++i)
-                    (void)mbar_wait(&ready[(b - i) % C::A_BLOCKS], (uint32_t)((b - i) / C::A_BLOCKS) & 1u);
-            }
-        }
-    } else if (warp == C::WARP_MMA || warp >= C::WARP_ISS1) {
-        // ----------------------------------------------------------- MMA issuers
-        // Issuer i accumulates K-steps k = i, i + NISS, ... of every 64-K half into chain i.
-        if (lane == 0) {
-            const int iss = warp == C::WARP_MMA ? 0 : warp - C::WARP_ISS1 + 1;
-            int ab = 0;
-            uint32_t abph = 0;
-            int as0 = 0, xs = 0, ds = 0;       // A half-stage of the block's first half, x stage, blk_done slot
-            uint32_t rph = 0;                  // parity of ready[as0 / 2]
-            bool ok = true;
-            constexpr uint32_t idesc_full = idesc_bf16_f32(128, BX);
-            constexpr uint32_t idesc_half = idesc_bf16_f32(128, BX / 2);
-            int xoff, xrows;
-            while (ok && it.next(tile, r0, r1, j, xoff, xrows, BX)) {
-                const uint32_t idesc = xrows == BX ? idesc_full : idesc_half;
-                if (!mbar_wait(&acc_empty[ab], abph ^ 1)) { ok = false; break; }
-                tc_fence_after();
-                const uint32_t d_tmem = tmem_base + C::A_COLS + ab * C::ACC_COLS + iss * BX;
-                uint32_t acc = 0;              // 0 for the chain's first MMA of the run
-                for (int r = r0; r < r1; ++r) {
-                    const uint32_t xaddr = sbase + C::OFF_X + xs * C::X_BYTES;
-                    if (!mbar_wait(&ready[as0 >> 1], rph)) { ok = false; break; }
-                    tc_fence_after();
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const uint32_t a_tmem = tmem_base + (as0 + h) * 32;
-                        const uint64_t bdesc = smem_desc_sw128(xaddr + h * C::X_HALF_BYTES);
-#pragma unroll
-                        for (int k = 0; k < C::KA / 16; ++k) {
-                            if (k % C::NISS != iss % C::NISS) continue;
-                            umma_bf16_ts(d_tmem, a_tmem + 8 * k, bdesc + 2 * k, idesc, acc);
-                            acc = 1;
-                        }
+                // let every copy already issued land before the CTA can exit
+                asm volatile("cp.async.wait_all;" ::: "memory");
+                if (lane == 0) {
+                    for (int i = 0; i < raw_issued && i < C::RAW_STAGES; ++i) {
+                        if (--rs < 0) { rs = C::RAW_STAGES - 1; rph ^= 1; }
+                        (void)mbar_wait(&raw_full[rs], rph);
                     }
-                    umma_commit(&blk_done[ds]);
-                    as0 += 2;
-                    if (as0 == C::A_STAGES) { as0 = 0; rph ^= 1; }
-                    if (++xs == C::X_STAGES) xs = 0;
-                    if (++ds == C::NDONE) ds = 0;
                 }
-                if (ok) umma_commit(&acc_full[ab]);
-                if (++ab == C::NACC) { ab = 0; abph ^= 1; }
             }
-            // every MMA issued by this thread has completed once `drain` flips
-            umma_commit(drain);
-            (void)mbar_wait(drain, 0);
+        } else if (warp == C::WARP_XLOAD) {
+            // ----------------------------------------------------------- x producer
+            if (lane == 0) {
+                int b = 0;                 // the CTA's block index
+                bool ok = true;
+                int xoff, xrows;
+                while (ok && it.next(tile, r0, r1, j, xoff, xrows, BX)) {
+                    for (int r = r0; r < r1; ++r, ++b) {
+                        if (b < pre_x) continue;   // issued before the CTA-wide barrier
+                        // stage b % X_STAGES last held block b - X_STAGES
+                        const int prev = b - C::X_STAGES;
+                        if (prev >= 0 && !mbar_wait(&blk_done[prev % C::NDONE], (uint32_t)(prev / C::NDONE) & 1u)) {
+                            ok = false;
+                            break;
+                        }
+                        // a half-width run loads its BX/2 activation rows with the half-height box
+                        issue_x(b, r, tile, xoff, xrows);
+                    }
+                }
+                if (!ok) {
+                    // let the copies already issued land before the CTA can exit (a slot whose decoder
+                    // arrivals never come ends this wait by its time limit)
+                    for (int i = 1; i <= C::X_STAGES && b - i >= 0; ++i)
+                        (void)mbar_wait(&ready[(b - i) % C::A_BLOCKS], (uint32_t)((b - i) / C::A_BLOCKS) & 1u);
+                }
+            }
+        } else if (warp == C::WARP_MMA) {
+            // ----------------------------------------------------------- MMA issuers
+            // Issuer i accumulates K-steps k = i, i + NISS, ... of every 64-K half into chain i.
+            if (lane == 0) {
+                const int iss = warp == C::WARP_MMA ? 0 : warp - C::WARP_ISS1 + 1;
+                int ab = 0;
+                uint32_t abph = 0;
+                int as0 = 0, xs = 0, ds = 0;       // A half-stage of the block's first half, x stage, blk_done slot
+                uint32_t rph = 0;                  // parity of ready[as0 / 2]
+                bool ok = true;
+                constexpr uint32_t idesc_full = idesc_bf16_f32(128, BX);
+                constexpr uint32_t idesc_half = idesc_bf16_f32(128, BX / 2);
+                int xoff, xrows;
+                while (ok && it.next(tile, r0, r1, j, xoff, xrows, BX)) {
+                    const uint32_t idesc = xrows == BX ? idesc_full : idesc_half;
+                    if (!mbar_wait(&acc_empty[ab], abph ^ 1)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t d_tmem = tmem_base + C::A_COLS + ab * C::ACC_COLS + iss * BX;
+                    uint32_t acc = 0;              // 0 for the chain's first MMA of the run
+                    for (int r = r0; r < r1; ++r) {
+                        const uint32_t xaddr = sbase + C::OFF_X + xs * C::X_BYTES;
+                        if (!mbar_wait(&ready[as0 >> 1], rph)) { ok = false; break; }
+                        tc_fence_after();
+    #pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const uint32_t a_tmem = tmem_base + (as0 + h) * 32;
+                            const uint64_t bdesc = smem_desc_sw128(xaddr + h * C::X_HALF_BYTES);
+    #pragma unroll
+                            for (int k = 0; k < C::KA / 16; ++k) {
+                                if (k % C::NISS != iss % C::NISS) continue;
+                                umma_bf16_ts(d_tmem, a_tmem + 8 * k, bdesc + 2 * k, idesc, acc);
+                                acc = 1;
+                            }
+                        }
+                        umma_commit(&blk_done[ds]);
+                        as0 += 2;
+                        if (as0 == C::A_STAGES) { as0 = 0; rph ^= 1; }
+                        if (++xs == C::X_STAGES) xs = 0;
+                        if (++ds == C::NDONE) ds = 0;
+                    }
+                    if (ok) umma_commit(&acc_full[ab]);
+                    if (++ab == C::NACC) { ab = 0; abph ^= 1; }
+                }
+                // every MMA issued by this thread has completed once `drain` flips
+                umma_commit(drain);
+                (void)mbar_wait(drain, 0);
+            }
         }
     } else if (warp < C::WARP_EPI0) {
+        if constexpr (C::REG_SPLIT && C::REG_DEC != C::REG_LAUNCH) setmaxnreg_dec<C::REG_DEC>();
         // ----------------------------------------------------------- decoders
         pdl_wait();   // the group-wise scales are read from global memory
         const int g = (warp - C::WARP_DEC0) >> 2;        // decoder group
@@ -580,6 +601,7 @@ __global__ void __launch_bounds__(Cfg<BX, BITS>::THREADS, 1)
             }
         }
     } else {
+        if constexpr (C::REG_SPLIT) setmaxnreg_inc<C::REG_EPI>();
         // ----------------------------------------------------------- epilogue
         pdl_wait();
         const int q = warp & 3;
@@ -588,33 +610,37 @@ __global__ void __launch_bounds__(Cfg<BX, BITS>::THREADS, 1)
         int ab = 0;
         uint32_t abph = 0;
         int xoff, xrows;
-        // y[m0 .. m0 + 15][n] = bf16(v[i] * scale) for this lane's weight row n
-        auto store16 = [&](const uint32_t (&v)[16], int m0, int n, int n0, auto &&fv) {
+        // y[m0 .. m0 + 15][n] for this lane's weight row n from the 8 bf16 pairs pk[i] =
+        // (row m0 + 2i, row m0 + 2i + 1)
+        auto store_pairs = [&](const uint32_t (&pk)[8], int m0, int n, int n0) {
             if (vec_y && n0 + 32 <= args.N) {
-                // rows m0 + 2i and m0 + 2i + 1 packed as bf16 pairs; lanes n and n ^ 1 swap halves
-                // so that the even lane holds row m0 + 2i and the odd lane row m0 + 2i + 1, each
-                // for weight rows n & ~1 and (n & ~1) + 1: one 4-byte store per lane per row pair
+                // lanes n and n ^ 1 swap halves so that the even lane holds row m0 + 2i and the odd
+                // lane row m0 + 2i + 1, each for weight rows n & ~1 and (n & ~1) + 1: one 4-byte
+                // store per lane per row pair
                 const uint32_t odd = (uint32_t)lane & 1u;
                 const uint32_t sel = odd ? 0x3276u : 0x5410u;
                 uint32_t *yw = reinterpret_cast<uint32_t *>(args.y + (size_t)(m0 + (int)odd) * args.N + n0 +
                                                             (lane & ~1));
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    const uint32_t pk = pack_bf16x2_rn(fv(__uint_as_float(v[2 * i])), fv(__uint_as_float(v[2 * i + 1])));
-                    const uint32_t other = __shfl_xor_sync(0xFFFFFFFFu, pk, 1);
-                    const uint32_t word = __byte_perm(pk, other, sel);
+                    const uint32_t other = __shfl_xor_sync(0xFFFFFFFFu, pk[i], 1);
+                    const uint32_t word = __byte_perm(pk[i], other, sel);
                     if (m0 + 2 * i + (int)odd < args.M) yw[(size_t)i * (size_t)args.N] = word;
                 }
             } else if (n < args.N) {
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const int m = m0 + i;
-                    if (m < args.M) {
-                        const __nv_bfloat16 o = __float2bfloat16_rn(fv(__uint_as_float(v[i])));
-                        args.y[(size_t)m * args.N + n] = *reinterpret_cast<const uint16_t *>(&o);
-                    }
+                    if (m < args.M) args.y[(size_t)m * args.N + n] = (uint16_t)(pk[i >> 1] >> (16 * (i & 1)));
                 }
             }
+        };
+        // y[m0 .. m0 + 15][n] = bf16(fv(v[i])) (rounded to nearest even)
+        auto store16 = [&](const uint32_t (&v)[16], int m0, int n, int n0, auto &&fv) {
+            uint32_t pk[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) pk[i] = pack_bf16x2_rn(fv(__uint_as_float(v[2 * i])), fv(__uint_as_float(v[2 * i + 1])));
+            store_pairs(pk, m0, n, n0);
         };
         while (it.next(tile, r0, r1, j, xoff, xrows, BX)) {
             const int n_blk = tile / args.m_tiles, m_blk = tile % args.m_tiles;
@@ -641,7 +667,43 @@ __global__ void __launch_bounds__(Cfg<BX, BITS>::THREADS, 1)
             if (!warp_wait(&acc_full[ab], abph)) break;
             tc_fence_after();
             const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + C::A_COLS + ab * C::ACC_COLS;
-            if (full) {
+            bool released = false;
+            if (full && act != EPI_SILU && act != EPI_GELU_TANH) {
+                // The whole tile's outputs into registers as bf16 pairs (column pair (2i, 2i + 1)
+                // in pk[i]), then the accumulator goes back to the MMA issuer at once and y is
+                // stored from registers while the next tile's MMAs run. (An activation's math
+                // would hold too many registers here: those tiles take the streaming loop below.)
+                uint32_t pk[BX / 2];
+                auto gather = [&](auto &&fv) {
+#pragma unroll
+                    for (int c0 = 0; c0 < BX; c0 += 16) {
+                        if (c0 < xrows) {
+                            uint32_t v[16];
+                            tmem_ld_32x32b_x16(taddr + c0, v);
+                            tmem_ld_wait();
+#pragma unroll
+                            for (int i = 0; i < 8; ++i)
+                                pk[c0 / 2 + i] = pack_bf16x2_rn(fv(__uint_as_float(v[2 * i])), fv(__uint_as_float(v[2 * i + 1])));
+                        }
+                    }
+                };
+                if (plain) gather(fv_plain);
+                else gather(fv_bias);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acc_empty[ab]);
+                released = true;
+#pragma unroll
+                for (int c0 = 0; c0 < BX; c0 += 16) {
+                    if (c0 < xrows) {
+                        uint32_t p8[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) p8[i] = pk[c0 / 2 + i];
+                        store_pairs(p8, m_blk * BX + xoff + c0, n, n0);
+                    }
+                }
+            } else if (full) {
+                // with an activation: 16 columns at a time, loaded, computed and stored
 #pragma unroll 1
                 for (int c0 = 0; c0 < xrows; c0 += 16) {
                     uint32_t v[16];
@@ -710,9 +772,11 @@ __global__ void __launch_bounds__(Cfg<BX, BITS>::THREADS, 1)
                     }
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[ab]);
+            if (!released) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acc_empty[ab]);
+            }
             if (++ab == C::NACC) { ab = 0; abph ^= 1; }
         }
     }
