@@ -836,13 +836,19 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
                 const int64_t c_lo = unit_owner((int64_t)tile * args.ngroups, gridDim.x, U);
                 const int64_t c_hi = unit_owner((int64_t)(tile + 1) * args.ngroups - 1, gridDim.x, U);
                 const uint32_t parts = (uint32_t)(c_hi - c_lo + 1);
-                __threadfence();
-                __syncwarp();
+                // Publication without full fences: the warp's partial stores are ordered before lane
+                // 0's release-acquire add by a 32-thread named barrier (ids 2..5, one per warp), and
+                // the last arriver's acquire is ordered before every lane's loads by the same barrier.
+                asm volatile("bar.sync %0, 32;" ::"r"(2 + q) : "memory");
                 uint32_t old = 0;
-                if (lane == 0) old = atomicAdd(args.counters + (size_t)tile * 4 + q, 1u);
+                if (lane == 0)
+                    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
+                                 : "=r"(old)
+                                 : "l"(args.counters + (size_t)tile * 4 + q)
+                                 : "memory");
                 old = __shfl_sync(0xFFFFFFFFu, old, 0);
                 if (old == parts - 1) {
-                    __threadfence();
+                    asm volatile("bar.sync %0, 32;" ::"r"(2 + q) : "memory");
                     // lane i (< parts) resolves part i's base; bases are broadcast by shuffles
                     const float *mybase = nullptr;
                     if ((uint32_t)lane < parts) {
