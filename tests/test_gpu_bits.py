@@ -49,6 +49,31 @@ def test_quantize_bits_shapes(bits, N, K):
     bits_parity(lin.make_weights(DEV), bits, 0.73)
 
 
+@pytest.mark.parametrize("bits", [3, 5, 6])
+@pytest.mark.parametrize("alpha", [0.2, 0.35])
+@pytest.mark.parametrize("N,K", [(37, 96), (300, 3840), (3, 10240)])
+def test_quantize_bits_small_alpha(bits, alpha, N, K):
+    # small alpha stretches the levels over many binades: rows whose code table would not fit
+    # (alpha below ~0.24 at 3 bits, ~0.44 at 6 bits for K <= 4096) take the threshold search
+    lin = workloads.Linear("bits_alpha", 1, N, K, w_seed=7 * N + K + bits)
+    bits_parity(lin.make_weights(DEV), bits, alpha)
+
+
+@pytest.mark.parametrize("bits", [3, 5, 6])
+def test_quantize_bits_special_rows(bits):
+    N, K = 6, 96
+    g = torch.Generator(device=DEV).manual_seed(11)
+    w = (torch.randn((N, K), generator=g, device=DEV) * 0.02).to(torch.bfloat16)
+    w[0] = 0                                  # all-zero row
+    w[1] = -0.0                               # negative zeros only
+    w[2, 5] = -w[2].abs().max() * 2           # negative maximum ...
+    w[2, 9] = w[2].abs().max()                # ... duplicated with the other sign
+    w[3] = torch.tensor([2.0 ** -130] * 48 + [-(2.0 ** -133)] * 48, dtype=torch.bfloat16, device=DEV)  # subnormal max
+    w[4, :] = w[4, 0]                         # a constant row
+    for alpha in (0.45, 1.0):
+        bits_parity(w, bits, alpha)
+
+
 def test_quantize_bits_four_equals_nibble_format():
     w = workloads.dit_attn_proj().make_weights(DEV)
     a = opq.quantize_bits(w, 4)
