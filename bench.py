@@ -236,6 +236,10 @@ class WholeModelState:
         self.jobs = {c: (opq.quantize_jobs([L["w"] for L in Ls], [(L["c"], L["s"], L["sc"]) for L in Ls],
                                            self.alpha), [L["w"] for L in Ls],
                          [(L["c"], L["s"], L["sc"]) for L in Ls]) for c, Ls in self.by_class.items()}
+        # and one opq_dequantize_batched call per shape class decodes them back
+        self.djobs = {c: (opq.dequantize_jobs([(L["c"], L["s"], L["sc"]) for L in Ls], [L["wq"] for L in Ls]),
+                          [(L["c"], L["s"], L["sc"]) for L in Ls], [L["wq"] for L in Ls])
+                      for c, Ls in self.by_class.items()}
 
     def phase(self, opq, what, cls):
         a, M = self.alpha, self.M
@@ -243,11 +247,12 @@ class WholeModelState:
             jobs, ws, outs = self.jobs[cls]
             opq.quantize_batched(ws, a, outs=outs, jobs=jobs)
             return
+        if what == "dequantize":
+            jobs, planes, outs = self.djobs[cls]
+            opq.dequantize_batched(planes, a, outs=outs, jobs=jobs)
+            return
         for L in self.by_class[cls]:
-            if what == "linear":
-                opq.linear(self.x[L["K"]], L["c"], L["s"], L["sc"], a, out=self.y[L["N"]], workspace=self.ws)
-            else:
-                opq.dequantize(L["c"], L["s"], L["sc"], a, out=L["wq"])
+            opq.linear(self.x[L["K"]], L["c"], L["s"], L["sc"], a, out=self.y[L["N"]], workspace=self.ws)
 
     def counts(self, cls):
         Ls = self.by_class[cls]
@@ -376,9 +381,9 @@ def gpu_arm(args, rank, world, local_rank):
         "by_class": {c: tf_entry(seg[("linear", c)], cnt[c]["linear_flops"],
                                  {"layers": cnt[c]["matrices"], "plan": list(opq.plan(M, *[(n, k) for nm, n, k in WM_CLASSES if nm == c][0]))})
                      for c in cls_names}})
-    # library kernels per step: the batched quantize (one launch per 128 matrices of a class), one
-    # linear and one dequantize per layer
-    launches_per_step = sum(-(-cnt[c]["matrices"] // 128) for c in cls_names) + 2 * len(S.layers)
+    # library kernels per step: the batched quantize and dequantize (one launch per 128 matrices of
+    # a class each) and one linear per layer
+    launches_per_step = 2 * sum(-(-cnt[c]["matrices"] // 128) for c in cls_names) + len(S.layers)
     linear_tflops = kernels["linear_all"]["tflops"]
 
     # ---------------------------------------------------------------- e2e: host buffers
@@ -400,6 +405,8 @@ def gpu_arm(args, rank, world, local_rank):
         blocks = [S.layers[i:i + 7] for i in range(0, len(S.layers), 7)]
         bjobs = [(opq.quantize_jobs([L["w"] for L in B], [(L["c"], L["s"], L["sc"]) for L in B], alpha),
                   [L["w"] for L in B], [(L["c"], L["s"], L["sc"]) for L in B]) for B in blocks]
+        bdjobs = [(opq.dequantize_jobs([(L["c"], L["s"], L["sc"]) for L in B], [L["wq"] for L in B]),
+                   [(L["c"], L["s"], L["sc"]) for L in B], [L["wq"] for L in B]) for B in blocks]
         y_dev = [torch.empty((M, L["N"]), dtype=torch.bfloat16, device=dev) for L in S.layers]
         y_host = [torch.empty((M, L["N"]), dtype=torch.bfloat16).pin_memory() for L in S.layers]
         s_up, s_down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
@@ -420,7 +427,7 @@ def gpu_arm(args, rank, world, local_rank):
                     landed.append(e)
             done = []
             i = 0
-            for B, (jobs, ws_, outs_), e in zip(blocks, bjobs, landed):
+            for B, (jobs, ws_, outs_), (djobs, dplanes, douts), e in zip(blocks, bjobs, bdjobs, landed):
                 stream.wait_event(e)
                 opq.quantize_batched(ws_, alpha, outs=outs_, jobs=jobs)
                 for L in B:
@@ -428,8 +435,8 @@ def gpu_arm(args, rank, world, local_rank):
                     ev = torch.cuda.Event()
                     ev.record(stream)
                     done.append(ev)
-                    opq.dequantize(L["c"], L["s"], L["sc"], alpha, out=L["wq"])
                     i += 1
+                opq.dequantize_batched(dplanes, alpha, outs=douts, jobs=djobs)
             with torch.cuda.stream(s_down):
                 for i, ev in enumerate(done):
                     s_down.wait_event(ev)
@@ -456,8 +463,9 @@ def gpu_arm(args, rank, world, local_rank):
                "steps": e_steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "host_weights": "registered (page-locked) host memory" if registered else "pageable host memory",
                "copies": "210 weight H2D + 2 activation H2D + 210 y D2H per step",
-               "pipeline": "per transformer block: weights up on one copy stream, quantize + linear + "
-                           "dequantize on the compute stream, each y down on another copy stream"}
+               "pipeline": "per transformer block: weights up on one copy stream, quantize (one batched call) + "
+                           "linears + dequantize (one batched call) on the compute stream, each y down on another "
+                           "copy stream"}
         if registered:
             cudart.cudaHostUnregister(w_host.data_ptr())
         del w_host, y_dev, y_host
@@ -488,7 +496,7 @@ def gpu_arm(args, rank, world, local_rank):
         "config": {"workload": "dit_whole_model_30blocks_210layers_m3072", "blocks": 30, "layers": 210,
                    "weights": 5308416000, "M": M, "alpha": alpha,
                    "step": "quantize all 210 W (one batched call per shape class) + linear x W'^T on every "
-                           "layer (M 3072) + dequantize all 210",
+                           "layer (M 3072) + dequantize all 210 (one batched call per shape class)",
                    "parallelism": f"replicas{world}",
                    "l2": "inputs larger than L2 (10.62 GB of weights per step against a 126 MB L2); no flush",
                    "launch": "each phase and shape class is one CUDA graph of the library's launches"},

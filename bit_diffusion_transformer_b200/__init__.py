@@ -32,7 +32,7 @@ EXPORTS = ["opq_quantize", "opq_dequantize", "opq_linear_workspace_size", "opq_l
            "opq_linear_grouped", "opq_linear_grouped_workspace_size", "opq_linear_fused",
            "opq_linear_grouped_fused", "opq_alpha_search", "opq_alpha_search_workspace_size",
            "opq_quantize_bits", "opq_dequantize_bits", "opq_set_wait_limit_ns",
-           "opq_quantize_batched", "opq_linear_bits", "opq_linear_bits_workspace_size"]
+           "opq_quantize_batched", "opq_linear_bits", "opq_linear_bits_workspace_size", "opq_dequantize_batched"]
 ACTIVATIONS = {"none": 0, "silu": 1, "gelu_tanh": 2}
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
@@ -76,6 +76,7 @@ def load(path: str = LIB_PATH):
     lib.opq_linear_grouped_fused.argtypes = [P, I, I, P, P, P, I, I, F, P, ctypes.c_int, P, P, S, P]
     lib.opq_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
     lib.opq_quantize_batched.argtypes = [P, I, F, P]
+    lib.opq_dequantize_batched.argtypes = [P, I, F, P]
     lib.opq_linear_bits.argtypes = [P, I, I, P, P, P, I, ctypes.c_int32, F, P, P, S, P]
     lib.opq_linear_bits_workspace_size.argtypes = [I, I, I, ctypes.c_int32, ctypes.POINTER(S)]
     lib.opq_status_string.argtypes = [ctypes.c_int]
@@ -84,7 +85,8 @@ def load(path: str = LIB_PATH):
               "opq_linear_noalloc", "opq_device_error", "opq_quantize_grouped", "opq_dequantize_grouped", "opq_linear_grouped",
               "opq_linear_grouped_workspace_size", "opq_linear_fused", "opq_linear_grouped_fused",
               "opq_alpha_search", "opq_alpha_search_workspace_size", "opq_quantize_bits", "opq_dequantize_bits",
-              "opq_set_wait_limit_ns", "opq_quantize_batched", "opq_linear_bits", "opq_linear_bits_workspace_size"):
+              "opq_set_wait_limit_ns", "opq_quantize_batched", "opq_linear_bits", "opq_linear_bits_workspace_size",
+              "opq_dequantize_batched"):
         getattr(lib, f).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -169,6 +171,37 @@ def dequantize(codes: torch.Tensor, signs: torch.Tensor, scales: torch.Tensor, a
     _check(load().opq_dequantize(_ptr(codes), _ptr(signs), _ptr(scales), N, K, float(alpha), _ptr(w),
                                  _stream(codes.device)), "opq_dequantize")
     return w
+
+
+class DequantJob(ctypes.Structure):
+    """One matrix of opq_dequantize_batched (the C struct opq_dequant_job)."""
+    _fields_ = [("codes", ctypes.c_void_p), ("signs", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("N", ctypes.c_int64), ("K", ctypes.c_int64), ("w_out", ctypes.c_void_p)]
+
+
+def dequantize_jobs(planes, outs):
+    """The descriptor array of opq_dequantize_batched for packed weights ``planes``
+    [(codes, signs, scales), ...] and their bf16 outputs ``outs`` (built once, reusable)."""
+    assert len(planes) == len(outs) and len(planes) > 0
+    arr = (DequantJob * len(planes))()
+    for i, ((c, s, f), w) in enumerate(zip(planes, outs)):
+        _need_cuda(c, s, f, w)
+        N, cw = c.shape
+        assert w.dtype == torch.bfloat16 and tuple(w.shape) == (N, cw * 8)
+        arr[i] = DequantJob(c.data_ptr(), s.data_ptr(), f.data_ptr(), N, cw * 8, w.data_ptr())
+    return arr
+
+
+def dequantize_batched(planes, alpha: float = ALPHA, outs=None, jobs=None):
+    """Decode a list of packed weights in one pass -> [bf16 W', ...]. ``jobs`` (from
+    dequantize_jobs) skips rebuilding the descriptors for the same buffers."""
+    if outs is None:
+        outs = [torch.empty((c.shape[0], c.shape[1] * 8), dtype=torch.bfloat16, device=c.device) for c, _, _ in planes]
+    if jobs is None:
+        jobs = dequantize_jobs(planes, outs)
+    _check(load().opq_dequantize_batched(ctypes.cast(jobs, ctypes.c_void_p), len(jobs), float(alpha),
+                                         _stream(planes[0][0].device)), "opq_dequantize_batched")
+    return outs
 
 
 def quantize_grouped(w: torch.Tensor, group_size: int = 128, alpha: float = ALPHA, out=None):

@@ -666,26 +666,64 @@ opq_status opq_alpha_search(const uint16_t *w, int64_t N, int64_t K, int64_t ldw
     return OPQ_OK;
 }
 
+// The dequantize over a list of matrices: validation of every descriptor first, then one launch
+// per DQ_MAX_JOBS matrices (one warp per row, four rows per block, at most 32 blocks per SM).
+static opq_status dequantize_jobs(const opq_dequant_job *jobs, int64_t count, float alpha, void *stream) {
+    if (jobs == nullptr || count < 1) return OPQ_ERR_INVALID_ARG;
+    if (!alpha_ok(alpha)) return OPQ_ERR_INVALID_ARG;
+    for (int64_t i = 0; i < count; ++i) {
+        const opq_dequant_job &J = jobs[i];
+        opq_status s = check_sizes(J.N, J.K);
+        if (s != OPQ_OK) return s;
+        if ((uint64_t)J.N * (uint64_t)(J.K / 8) >= (1ull << 40) || J.N > UINT32_MAX) return OPQ_ERR_UNSUPPORTED_SHAPE;
+    }
+    for (int64_t i = 0; i < count; ++i) {
+        opq_status s = check_ptrs({jobs[i].codes, jobs[i].signs, jobs[i].scales, jobs[i].w_out});
+        if (s != OPQ_OK) return s;
+    }
+    DeviceInfo *di = nullptr;
+    opq_status s = device_info(&di);
+    if (s != OPQ_OK) return s;
+    static thread_local opqk::DqParams P;   // ~6 KB: kept off the stack
+    const double inv = 1.0 / (double)alpha;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    for (int64_t c0 = 0; c0 < count; c0 += opqk::DQ_MAX_JOBS) {
+        std::memset(&P, 0, sizeof P);
+        for (int q = 0; q < 16; ++q) P.dp.lut[q] = std::pow((double)q / 15.0, inv);
+        const int64_t n = count - c0 < opqk::DQ_MAX_JOBS ? count - c0 : opqk::DQ_MAX_JOBS;
+        int64_t rows = 0;
+        for (int64_t i = 0; i < n; ++i) {
+            const opq_dequant_job &J = jobs[c0 + i];
+            opqk::DqJob &q = P.job[i];
+            q.codes = J.codes;
+            q.signs = J.signs;
+            q.scales = J.scales;
+            q.out = J.w_out;
+            q.row_begin = rows;
+            q.N = (uint32_t)J.N;
+            q.chunks = (uint32_t)(J.K / 32);
+            rows += J.N;
+        }
+        P.njobs = (int32_t)n;
+        P.rows = rows;
+        uint64_t blocks = ((uint64_t)rows + 3) / 4;
+        const uint64_t cap = (uint64_t)di->sms * 32;
+        if (blocks > cap) blocks = cap;
+        opqk::dequantize_kernel<<<(int)blocks, 128, 0, st>>>(P);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    return OPQ_OK;
+}
+
 opq_status opq_dequantize(const uint32_t *codes, const uint32_t *signs, const float *scales, int64_t N, int64_t K,
                           float alpha, uint16_t *w_out, void *stream) {
-    opq_status s = check_sizes(N, K);
-    if (s != OPQ_OK) return s;
-    if (!alpha_ok(alpha)) return OPQ_ERR_INVALID_ARG;
-    if ((uint64_t)N * (uint64_t)(K / 8) >= (1ull << 40)) return OPQ_ERR_UNSUPPORTED_SHAPE;
-    if ((s = check_ptrs({codes, signs, scales, w_out})) != OPQ_OK) return s;
-    opqk::DequantParams dp{};
-    const double inv = 1.0 / (double)alpha;
-    for (int q = 0; q < 16; ++q) dp.lut[q] = std::pow((double)q / 15.0, inv);
-    DeviceInfo *di = nullptr;
-    if ((s = device_info(&di)) != OPQ_OK) return s;
-    // one warp per row, 4 rows per block
-    uint64_t blocks = ((uint64_t)N + 3) / 4;
-    const uint64_t cap = (uint64_t)di->sms * 32;
-    if (blocks > cap) blocks = cap;
-    opqk::dequantize_kernel<<<(int)blocks, 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-        codes, signs, scales, (uint32_t)N, (uint32_t)(K / 32), dp, w_out);
-    cudaError_t e = cudaGetLastError();
-    return e == cudaSuccess ? OPQ_OK : cuda_fail(e);
+    const opq_dequant_job job = {codes, signs, scales, N, K, w_out};
+    return dequantize_jobs(&job, 1, alpha, stream);
+}
+
+opq_status opq_dequantize_batched(const opq_dequant_job *jobs, int64_t count, float alpha, void *stream) {
+    return dequantize_jobs(jobs, count, alpha, stream);
 }
 
 opq_status opq_linear_workspace_size(int64_t M, int64_t N, int64_t K, size_t *bytes) {

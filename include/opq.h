@@ -106,6 +106,28 @@ opq_status opq_dequantize(const uint32_t *codes, const uint32_t *signs, const fl
                           int64_t N, int64_t K, float alpha, uint16_t *w_out, void *stream);
 
 /*
+ * opq_dequantize_batched — opq_dequantize over a list of matrices in one pass (the
+ * inverse of opq_quantize_batched: every linear layer of a model decoded in one stream).
+ *   jobs    HOST array of `count` descriptors (count >= 1), read before the call
+ *           returns; each names a packed weight (device codes, signs, scales as
+ *           produced by opq_quantize, N, K with opq_dequantize's limits) and its bf16
+ *           output w_out [N, K] (device, 16-byte aligned)
+ *   alpha   the power used to quantize, shared by every matrix of the call
+ * Outputs are bit-identical to opq_dequantize on each matrix. The rows of up to 128
+ * matrices per launch form one sequence dealt to the warps; a job's output must not
+ * overlap another job's. An invalid descriptor fails the whole call before anything is
+ * launched.
+ */
+typedef struct opq_dequant_job {
+    const uint32_t *codes;   /* [N, K/8] */
+    const uint32_t *signs;   /* [N, K/32] */
+    const float *scales;     /* [N] */
+    int64_t N, K;
+    uint16_t *w_out;         /* bf16 [N, K] */
+} opq_dequant_job;
+opq_status opq_dequantize_batched(const opq_dequant_job *jobs, int64_t count, float alpha, void *stream);
+
+/*
  * Group-wise format — the card's own storage ("Technical details / storage
  * format": one float16 max shared by every 128 weights; its configuration also
  * lists group sizes 32, 64 and 256). Row n's weights k = g*GS .. g*GS + GS - 1

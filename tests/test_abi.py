@@ -79,6 +79,21 @@ def test_dequantize_and_linear_argument_errors(lib):
     assert lib.opq_dequantize(c, s, sc, 4, 32, 0.0, out, None) == 1
     assert lib.opq_dequantize(c, None, sc, 4, 32, 0.73, out, None) == 1
     assert lib.opq_dequantize(c, s, sc, 4, 32, 0.73, out, None) == 6
+    # the batched form: the list, then every descriptor, is checked before anything runs
+    J = (opq.DequantJob * 2)()
+    J[0] = opq.DequantJob(c, s, sc, 4, 32, out)
+    J[1] = opq.DequantJob(c, s, sc, 4, 32, out)
+    jp = ctypes.cast(J, ctypes.c_void_p)
+    assert lib.opq_dequantize_batched(None, 1, 0.73, None) == 1          # no list
+    assert lib.opq_dequantize_batched(jp, 0, 0.73, None) == 1            # empty list
+    assert lib.opq_dequantize_batched(jp, 2, float("nan"), None) == 1    # bad alpha
+    J[1] = opq.DequantJob(c, s, sc, 4, 40, out)
+    assert lib.opq_dequantize_batched(jp, 2, 0.73, None) == 2            # K % 32 != 0 in the second job
+    J[1] = opq.DequantJob(c, s, sc, 4, 32, out)
+    J[0] = opq.DequantJob(c, None, sc, 4, 32, out)
+    assert lib.opq_dequantize_batched(jp, 2, 0.73, None) == 1            # null pointer
+    J[0] = opq.DequantJob(c, s, sc, 4, 32, out)
+    assert lib.opq_dequantize_batched(jp, 2, 0.73, None) == 6            # host memory
     x, y = b(4096), b(4096)
     L = lib.opq_linear
     assert L(x, 0, 32, c, s, sc, 4, 0.73, y, None, 0, None) == 1
