@@ -69,6 +69,7 @@ uint16_t host_bf16(double v) {
 struct DeviceInfo {
     int sms = 0;
     bool stream_quant_attr[3][4] = {};   // dynamic shared memory raised for quantize_stream_kernel<G, BITS>
+    bool stream_quant_stab_attr = false; // and for its shared-mantissa-table variant
     // dynamic shared memory raised, per [group size index: 0 per-row, 1..4 GS 32..256][kernel: BX 16, 32,
     // 64, 128, wide]
     bool linear_attr[5][5] = {};
@@ -390,27 +391,29 @@ const char *opq_status_string(opq_status s) {
 }
 
 // The row-streaming quantize over a list of matrices: validation, then one launch per row-width
-// class (one, four or eight warps per row) and per QS_MAX_JOBS matrices of the class.
+// class (one, four or eight warps per row) and per QS_MAX_JOBS matrices of the class. One-warp
+// rows at 4 bits use the shared mantissa tables (STAB) when the 128 tables fit in shared memory
+// beside a ring of at least 8 rows: each table holds at most dz + 1 <= 128 log2(1/t_1) + 131
+// entries (t_1 = (1/30)^(1/alpha); the 128 accounts for the max's mantissa), which caps it
+// for alpha >= ~0.7; the kernel itself checks every table against its stride.
 extern "C++" {
-template <int G, int BITS>
-static opq_status launch_quant_stream(DeviceInfo *di, const opq_quant_job *jobs, const std::vector<int64_t> &idx,
-                                      const opqk::QuantParams &qp, const double *tl, cudaStream_t st) {
-    using C = opqk::QsCfg<G>;
-    int64_t kmax = 0;
-    for (int64_t i : idx) kmax = jobs[i].K > kmax ? jobs[i].K : kmax;
-    // one slot holds one row of the widest matrix of the class
-    const int slot_bytes = (int)((2 * kmax + 127) / 128 * 128);
-    int nslots = C::RING_MAX / slot_bytes;
+template <int G, int BITS, bool STAB>
+static opq_status launch_quant_stream_v(DeviceInfo *di, const opq_quant_job *jobs, const std::vector<int64_t> &idx,
+                                        const opqk::QuantParams &qp, const double *tl, int slot_bytes, int stab_bytes,
+                                        int stab_stride, cudaStream_t st) {
+    using C = opqk::QsCfg<G, STAB>;
+    int nslots = (C::RING_MAX - stab_bytes) / slot_bytes;
     if (nslots > opqk::QS_MAX_SLOTS) nslots = opqk::QS_MAX_SLOTS;
     if (nslots < 2) return OPQ_ERR_UNSUPPORTED_SHAPE;
-    const int smem = opqk::QS_OFF_RING + nslots * slot_bytes;
+    const int smem = opqk::QS_OFF_RING + stab_bytes + nslots * slot_bytes;
     const int gi = G == 1 ? 0 : (G == 4 ? 1 : 2);
-    if (!di->stream_quant_attr[gi][BITS - 3]) {
-        cudaError_t e = cudaFuncSetAttribute(opqk::quantize_stream_kernel<G, BITS>,
+    bool &attr = STAB ? di->stream_quant_stab_attr : di->stream_quant_attr[gi][BITS - 3];
+    if (!attr) {
+        cudaError_t e = cudaFuncSetAttribute(opqk::quantize_stream_kernel<G, BITS, STAB>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              opqk::QS_OFF_RING + C::RING_MAX);
         if (e != cudaSuccess) return cuda_fail(e);
-        di->stream_quant_attr[gi][BITS - 3] = true;
+        attr = true;
     }
     static thread_local opqk::QsParams P;   // ~7 KB: kept off the stack
     for (size_t c0 = 0; c0 < idx.size(); c0 += opqk::QS_MAX_JOBS) {
@@ -419,6 +422,8 @@ static opq_status launch_quant_stream(DeviceInfo *di, const opq_quant_job *jobs,
         for (int k = 0; k < 64; ++k) P.tl[k] = tl[k];
         P.nslots = nslots;
         P.slot_bytes = slot_bytes;
+        P.stab_bytes = stab_bytes;
+        P.stab_stride = stab_stride;
         const size_t n = idx.size() - c0 < (size_t)opqk::QS_MAX_JOBS ? idx.size() - c0 : (size_t)opqk::QS_MAX_JOBS;
         int64_t rows = 0;
         for (size_t i = 0; i < n; ++i) {
@@ -438,11 +443,30 @@ static opq_status launch_quant_stream(DeviceInfo *di, const opq_quant_job *jobs,
         P.rows = rows;
         const int64_t groups = rows < (int64_t)di->sms * C::NG ? rows : (int64_t)di->sms * C::NG;
         const int grid = (int)((groups + C::NG - 1) / C::NG);
-        opqk::quantize_stream_kernel<G, BITS><<<grid, opqk::QS_THREADS, smem, st>>>(P);
+        opqk::quantize_stream_kernel<G, BITS, STAB><<<grid, opqk::QS_THREADS, smem, st>>>(P);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail(e);
     }
     return OPQ_OK;
+}
+
+template <int G, int BITS>
+static opq_status launch_quant_stream(DeviceInfo *di, const opq_quant_job *jobs, const std::vector<int64_t> &idx,
+                                      const opqk::QuantParams &qp, const double *tl, cudaStream_t st) {
+    int64_t kmax = 0;
+    for (int64_t i : idx) kmax = jobs[i].K > kmax ? jobs[i].K : kmax;
+    // one slot holds one row of the widest matrix of the class
+    const int slot_bytes = (int)((2 * kmax + 127) / 128 * 128);
+    if constexpr (G == 1 && BITS == 4) {
+        const double t1 = qp.alpha_is_one ? 1.0 / 30.0 : qp.t[1];
+        const double dz_bound = std::ceil(-128.0 * std::log2(t1)) + 131.0;
+        const int stride = (int)((dz_bound + 4.0) / 16.0 + 1.0) * 16;   // >= 4 ((dz + 4) / 4) for dz <= dz_bound
+        const int stab_bytes = (256 + 128 * stride + 127) / 128 * 128;
+        using CS = opqk::QsCfg<1, true>;
+        if (stab_bytes <= 136 * 1024 && (CS::RING_MAX - stab_bytes) / slot_bytes >= 8)
+            return launch_quant_stream_v<1, 4, true>(di, jobs, idx, qp, tl, slot_bytes, stab_bytes, stride, st);
+    }
+    return launch_quant_stream_v<G, BITS, false>(di, jobs, idx, qp, tl, slot_bytes, 0, 0, st);
 }
 
 template <int BITS>

@@ -51,11 +51,12 @@ constexpr int QS_OFF_RING = 2 * QS_MAX_SLOTS * 8;
 __host__ __device__ constexpr int qs_group_warps(int64_t K) { return K <= 4096 ? 1 : (K <= 16384 ? 4 : 8); }
 
 // code-table entries per group: 16 groups of one warp share 32 KiB (a group's table offset plus
-// max |w| must stay below 2^16 in the packed lookups); larger groups get 4096 entries
-template <int G>
+// max |w| must stay below 2^16 in the packed lookups); larger groups get 4096 entries. With the
+// shared mantissa tables (STAB) the per-group tables only serve rows whose max is zero or tiny.
+template <int G, bool STAB = false>
 struct QsCfg {
     static constexpr int NG = QS_CONS_WARPS / G;           // groups
-    static constexpr int TAB = G == 1 ? 2048 : 4096;        // table entries (bytes) per group
+    static constexpr int TAB = STAB ? 4 : (G == 1 ? 2048 : 4096);   // table entries (bytes) per group
     static constexpr int STATIC_BYTES = NG * TAB + NG * G * 4;
     static constexpr int RING_MAX = QS_SMEM_LIMIT - QS_OFF_RING - STATIC_BYTES - 1024;
     static_assert((NG - 1) * TAB + 0x7F80 < 0x10000, "table offset + max must fit a 16-bit half");
@@ -78,9 +79,41 @@ struct QsParams {
     int32_t njobs;
     int32_t nslots;        // ring slots S
     int32_t slot_bytes;    // a multiple of 128, at least 2 K of every matrix
+    int32_t stab_bytes;    // STAB: bytes of the shared mantissa tables before the ring (else 0)
+    int32_t stab_stride;   // STAB: bytes per mantissa table (a multiple of 16)
     int32_t pad;
     QsJob job[QS_MAX_JOBS];
 };
+
+// The code table q(e) = #{k : B_k > e}, e = 0 .. dz, as dz / 4 + 1 words from the level boundaries
+// B_k = bits(max) - T_k + 1 held by lanes (Bk: levels lane + 1, Bk2: 6 bits, lane + 33): per
+// stretch of GT words (one per thread tg of the group) one ballot counts the levels that hold over
+// the whole stretch and the few boundaries inside it correct each word (no per-entry walk).
+// Word w goes to dst[w] times mult (4 bits: 0x11, q in both nibbles; else 1).
+template <int GT, int L>
+__device__ __forceinline__ void qs_build_table(uint32_t *dst, int Bk, int Bk2, uint32_t dz, int tg, uint32_t mult) {
+    const uint32_t words = (dz + 4u) >> 2;
+    for (uint32_t i0 = 0; i0 < words; i0 += GT) {
+        const int lo_e = (int)(4u * i0), hi_e = lo_e + 4 * GT - 1;
+        const uint32_t w = i0 + (uint32_t)tg;
+        uint32_t cnt = __popc(__ballot_sync(0xFFFFFFFFu, Bk > hi_e));
+        if (L > 32) cnt += __popc(__ballot_sync(0xFFFFFFFFu, Bk2 > hi_e));
+        uint32_t word = cnt * 0x01010101u;
+        auto inside = [&](int Bl) {
+            uint32_t in_m = __ballot_sync(0xFFFFFFFFu, Bl > lo_e && Bl <= hi_e);
+            while (in_m) {
+                const int k = __ffs(in_m) - 1;
+                in_m &= in_m - 1u;
+                const int B = __shfl_sync(0xFFFFFFFFu, Bl, k);
+                const int c = min(max(B - (int)(4u * w), 0), 4);
+                word += __funnelshift_rc(0x01010101u, 0u, 8 * (4 - c));
+            }
+        };
+        inside(Bk);
+        if (L > 32) inside(Bk2);
+        if (w < words) dst[w] = word * mult;
+    }
+}
 
 __device__ __forceinline__ void group_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
@@ -123,9 +156,16 @@ __device__ __forceinline__ void qs_store_codes(uint32_t *crow, int v, const uint
 
 // BITS = 4: the card's nibble format; 3, 5, 6: 2^BITS - 1 levels, each row's codes one
 // little-endian bit stream (element k at bits k BITS .. k BITS + BITS - 1 of the row's words).
-template <int G, int BITS = 4>
+// STAB (G = 1, BITS = 4): the thresholds of a row scale exactly with its max's power of two (the
+// fp64 product, the rounding up to fp32 and to bf16 and the tie test are all exact under such a
+// scaling while the thresholds stay normal), so B_k and the code table depend only on the 7
+// mantissa bits of the max. Each CTA builds the 128 tables once (from a max of each mantissa with
+// exponent 0) into shared memory in front of the ring, and a row whose smallest threshold is a
+// normal bf16 reads its mantissa's table instead of building its own.
+template <int G, int BITS = 4, bool STAB = false>
 __global__ void __launch_bounds__(QS_THREADS, 1) quantize_stream_kernel(const __grid_constant__ QsParams p) {
-    using C = QsCfg<G>;
+    using C = QsCfg<G, STAB>;
+    static_assert(!STAB || (G == 1 && BITS == 4), "shared mantissa tables: one-warp rows at 4 bits");
     constexpr int L = (1 << BITS) - 1;
     constexpr int NG = C::NG, GT = 32 * G;
     extern __shared__ __align__(128) uint8_t qs_smem[];
@@ -134,7 +174,10 @@ __global__ void __launch_bounds__(QS_THREADS, 1) quantize_stream_kernel(const __
 
     uint64_t *full = reinterpret_cast<uint64_t *>(qs_smem + QS_OFF_BAR);
     uint64_t *empty = full + QS_MAX_SLOTS;
-    const uint32_t ring = smem_u32(qs_smem + QS_OFF_RING);
+    const int ring_off = QS_OFF_RING + (STAB ? p.stab_bytes : 0);
+    const uint32_t ring = smem_u32(qs_smem + ring_off);
+    uint16_t *stab_dz = reinterpret_cast<uint16_t *>(qs_smem + QS_OFF_RING);           // STAB: dz per mantissa
+    uint32_t *stab_w = reinterpret_cast<uint32_t *>(qs_smem + QS_OFF_RING + 256);     // STAB: the tables
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int S = p.nslots;
     const int64_t grid = gridDim.x, cta = blockIdx.x;
@@ -161,7 +204,7 @@ __global__ void __launch_bounds__(QS_THREADS, 1) quantize_stream_kernel(const __
                 if (issued >= S && !mbar_wait(&empty[s], ph ^ 1u)) break;
                 const uint32_t rb = (uint32_t)J.K * 2u;
                 mbar_arrive_expect_tx(&full[s], rb);
-                bulk_load(qs_smem + QS_OFF_RING + (size_t)s * p.slot_bytes, J.w + (u - J.row_begin) * J.ldw, rb,
+                bulk_load(qs_smem + ring_off + (size_t)s * p.slot_bytes, J.w + (u - J.row_begin) * J.ldw, rb,
                           &full[s]);
                 ++issued;
                 if (++s == S) { s = 0; ph ^= 1u; }
@@ -180,6 +223,22 @@ __global__ void __launch_bounds__(QS_THREADS, 1) quantize_stream_kernel(const __
         const int bar_id = 1 + g;
         const uint8_t *tb = reinterpret_cast<const uint8_t *>(qs_tab);
         const uint32_t base = (uint32_t)g * C::TAB;
+        if constexpr (STAB) {
+            // the 128 mantissa tables: warp w builds those of mantissas w, w + 16, ...; a table that
+            // would not fit its stride is marked unusable (its rows build their own)
+            for (int m = warp; m < 128; m += QS_CONS_WARPS) {
+                const uint32_t mxr = (127u << 7) | (uint32_t)m;
+                const uint32_t myT = lane < 15 ? level_threshold(__uint_as_float(mxr << 16), lane + 1, p.qp) : 0x7F80u;
+                const uint32_t dz = mxr - __shfl_sync(0xFFFFFFFFu, myT, 0) + 1u;
+                const bool fits = 4u * ((dz + 4u) >> 2) <= (uint32_t)p.stab_stride;
+                if (lane == 0) stab_dz[m] = fits ? (uint16_t)dz : (uint16_t)0xFFFFu;
+                if (fits) {
+                    const int Bk = (lane < 15 && myT <= mxr) ? (int)mxr - (int)myT + 1 : 0;
+                    qs_build_table<32, 15>(stab_w + (uint32_t)m * (uint32_t)p.stab_stride / 4u, Bk, 0, dz, lane, 0x11u);
+                }
+            }
+            asm volatile("bar.sync 1, %0;" ::"r"(QS_CONS_WARPS * 32) : "memory");   // the consumers only
+        }
         int j = 0, s = g;
         uint32_t ph = 0;
         while (s >= S) { s -= S; ph ^= 1u; }
@@ -236,6 +295,29 @@ __global__ void __launch_bounds__(QS_THREADS, 1) quantize_stream_kernel(const __
                 break;
             }
             const float mxf = __uint_as_float(mx << 16);
+            uint32_t *crow = J.codes + n * ((int64_t)nvec * BITS / 4);
+            if constexpr (STAB) {
+                // the row's mantissa table, if its smallest threshold mx - dz + 1 is a normal bf16
+                const uint32_t dzm = (mx != 0u && mx <= 0x7F7Fu) ? (uint32_t)stab_dz[mx & 0x7Fu] : 0xFFFFu;
+                if (dzm != 0xFFFFu && mx + 1u >= dzm + 0x80u) {
+                    if (tg == 0) J.scales[n] = mxf;
+                    const uint8_t *tbm = reinterpret_cast<const uint8_t *>(stab_w) + (mx & 0x7Fu) * (uint32_t)p.stab_stride;
+                    const uint32_t mm = mx * 0x00010001u, lo2 = (mx - dzm) * 0x00010001u;
+#pragma unroll
+                    for (int k = 0; k < QS_VMAX; ++k) {
+                        const int v = k * GT + tg;
+                        if (v < nvec) {
+                            const uint4 x = a[k];
+                            crow[v] = opqbits::codes_word(opqbits::table_byte_clamped(tbm, x.x, lo2, mm),
+                                                          opqbits::table_byte_clamped(tbm, x.y, lo2, mm),
+                                                          opqbits::table_byte_clamped(tbm, x.z, lo2, mm),
+                                                          opqbits::table_byte_clamped(tbm, x.w, lo2, mm));
+                        }
+                    }
+                    __syncwarp();
+                    continue;
+                }
+            }
             // the thresholds of levels lane + 1 and (6 bits) lane + 33; +inf: a level no finite
             // weight reaches (every level of a zero row)
             uint32_t myT = 0x7F80u, myT2 = 0x7F80u;
@@ -251,37 +333,12 @@ __global__ void __launch_bounds__(QS_THREADS, 1) quantize_stream_kernel(const __
             const uint32_t T1 = __shfl_sync(0xFFFFFFFFu, myT, 0);
             const uint32_t dz = T1 <= mx ? mx - T1 + 1u : 0u;
             if (tg == 0) J.scales[n] = mxf;
-            uint32_t *crow = J.codes + n * ((int64_t)nvec * BITS / 4);
             // group-uniform: mx is the group's max
             if (mx <= 0x7F80u && dz < (uint32_t)C::TAB) {
-                // the table q(e) = #{k : B_k > e}, e = 0 .. d_z, from the level boundaries
-                // B_k = bits(max) - T_k + 1 held by lanes 0..14: per stretch of GT words (one per
-                // thread of the group) one ballot counts the levels that hold over the whole stretch
-                // and the few boundaries inside it correct each word (no per-entry walk)
                 const int Bk = (lane < L && myT <= mx) ? (int)mx - (int)myT + 1 : 0;
                 const int Bk2 = (L > 32 && lane + 32 < L && myT2 <= mx) ? (int)mx - (int)myT2 + 1 : 0;
-                const uint32_t words = (dz + 4u) >> 2;
-                for (uint32_t i0 = 0; i0 < words; i0 += GT) {
-                    const int lo_e = (int)(4u * i0), hi_e = lo_e + 4 * GT - 1;
-                    const uint32_t w = i0 + (uint32_t)tg;
-                    uint32_t cnt = __popc(__ballot_sync(0xFFFFFFFFu, Bk > hi_e));
-                    if (L > 32) cnt += __popc(__ballot_sync(0xFFFFFFFFu, Bk2 > hi_e));
-                    uint32_t word = cnt * 0x01010101u;
-                    auto inside = [&](int Bl) {
-                        uint32_t in_m = __ballot_sync(0xFFFFFFFFu, Bl > lo_e && Bl <= hi_e);
-                        while (in_m) {
-                            const int k = __ffs(in_m) - 1;
-                            in_m &= in_m - 1u;
-                            const int B = __shfl_sync(0xFFFFFFFFu, Bl, k);
-                            const int c = min(max(B - (int)(4u * w), 0), 4);
-                            word += __funnelshift_rc(0x01010101u, 0u, 8 * (4 - c));
-                        }
-                    };
-                    inside(Bk);
-                    if (L > 32) inside(Bk2);
-                    // 4 bits: q in both nibbles (a pair's code byte is one merge); else q itself
-                    if (w < words) qs_tab[base / 4 + w] = BITS == 4 ? word * 0x11u : word;
-                }
+                // 4 bits: q in both nibbles (a pair's code byte is one merge); else q itself
+                qs_build_table<GT, L>(qs_tab + base / 4, Bk, Bk2, dz, tg, BITS == 4 ? 0x11u : 1u);
                 if (G > 1) group_sync(bar_id, GT); else __syncwarp();
                 const uint32_t mmb = (mx + base) * 0x00010001u, lo2 = (mx - dz) * 0x00010001u;
 #pragma unroll
