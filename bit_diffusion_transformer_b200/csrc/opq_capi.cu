@@ -392,8 +392,8 @@ const char *opq_status_string(opq_status s) {
 
 // The row-streaming quantize over a list of matrices: validation, then one launch per row-width
 // class (one, four or eight warps per row) and per QS_MAX_JOBS matrices of the class. One-warp
-// rows at 4 bits use the shared mantissa tables (STAB) when the 128 tables fit in shared memory
-// beside a ring of at least 8 rows: each table holds at most dz + 1 <= 128 log2(1/t_1) + 131
+// rows at 4 bits use the shared mantissa tables (STAB) when the launch gives each CTA hundreds of
+// rows and the 128 tables fit in shared memory beside a ring of at least 8 rows: each table holds at most dz + 1 <= 128 log2(1/t_1) + 131
 // entries (t_1 = (1/30)^(1/alpha); the 128 accounts for the max's mantissa), which caps it
 // for alpha >= ~0.7; the kernel itself checks every table against its stride.
 extern "C++" {
@@ -457,7 +457,11 @@ static opq_status launch_quant_stream(DeviceInfo *di, const opq_quant_job *jobs,
     for (int64_t i : idx) kmax = jobs[i].K > kmax ? jobs[i].K : kmax;
     // one slot holds one row of the widest matrix of the class
     const int slot_bytes = (int)((2 * kmax + 127) / 128 * 128);
-    if constexpr (G == 1 && BITS == 4) {
+    int64_t rows = 0;
+    for (int64_t i : idx) rows += jobs[i].N;
+    // building the 128 tables costs a CTA about as much as building its own for 128 rows, so the
+    // shared tables serve launches that give every CTA many more rows than that (a whole model)
+    if constexpr (G == 1 && BITS == 4) if (rows >= 512 * (int64_t)di->sms) {
         const double t1 = qp.alpha_is_one ? 1.0 / 30.0 : qp.t[1];
         const double dz_bound = std::ceil(-128.0 * std::log2(t1)) + 131.0;
         const int stride = (int)((dz_bound + 4.0) / 16.0 + 1.0) * 16;   // >= 4 ((dz + 4) / 4) for dz <= dz_bound

@@ -149,3 +149,58 @@ def test_batched_argument_errors():
     arr[0] = opq.QuantJob(host.data_ptr(), 256, 512, 512, c.data_ptr(), s.data_ptr(), f.data_ptr())
     assert lib.opq_quantize_batched(ptr, 1, 0.73, st) == 6                   # host memory
     no_device_error()
+
+
+# a launch gives each CTA hundreds of one-warp rows from about 512 x 148 rows on: then the rows read
+# the shared mantissa tables (built once per CTA) instead of building their own
+STAB_ROWS = 80000
+
+
+@pytest.mark.parametrize("alpha", [0.73, 1.0])
+def test_power_of_two_scaled_rows(alpha):
+    """A row scaled by powers of two from 2^-126 to 2^126, repeated over a matrix large enough for
+    the shared mantissa tables (the rows share their max's mantissa: the tables serve them while
+    their thresholds stay normal, the smallest scales fall back to the per-row path), with random
+    rows between. Every row must match the oracle, and the scaled rows' codes must equal the
+    unscaled row's while they stay normal."""
+    K = 256
+    g = torch.Generator(device=DEV).manual_seed(5)
+    base = (torch.randn((1, K), generator=g, device=DEV) * 0.02).to(torch.bfloat16).float()
+    exps = list(range(-126, 127, 2))
+    scaled = torch.cat([base * (2.0 ** e) for e in exps]).to(torch.bfloat16)
+    rand = (torch.randn((STAB_ROWS - len(exps), K), generator=g, device=DEV) * 0.02).to(torch.bfloat16)
+    w = torch.cat([scaled, rand])
+    assert torch.isfinite(w.float()).all()
+    codes, signs, scales = opq.quantize(w, alpha)
+    no_device_error()
+    ref = oracle.quantize(w, alpha32(alpha), want_ties=True)
+    assert np.array_equal(u32(scales.view(torch.int32)), ref["scales"].view(np.uint32))
+    assert np.array_equal(u32(signs), ref["signs"])
+    qg, qo = unpack_codes(u32(codes)), unpack_codes(ref["codes"])
+    mism = qg != qo
+    near = ref["near_tie"].astype(bool)
+    assert int((mism & ~near).sum()) == 0
+    assert int((mism & near).sum()) <= TIE_FRACTION_LIMIT * qo.size
+    i0 = exps.index(0)
+    for i, e in enumerate(exps):
+        if -96 <= e <= 126:
+            assert torch.equal(codes[i], codes[i0]), f"exponent {e}"
+
+
+def test_batched_large_launch_sampled():
+    """21 projection-sized matrices in one call (80640 one-warp rows: the shared mantissa tables),
+    sampled rows of each against the oracle and one whole matrix against the one-matrix call,
+    which (3840 rows) builds per-row tables."""
+    ws = [workloads.Linear("big", 1, 3840, 3840, w_seed=100 + i).make_weights(DEV) for i in range(21)]
+    outs = opq.quantize_batched(ws, 0.73)
+    no_device_error()
+    rows = list(range(0, 3840, 173)) + [3839]
+    for w, (c, s_, f) in zip(ws, outs):
+        ref = oracle.quantize(w[rows].cpu(), alpha32(0.73), want_ties=True)
+        assert np.array_equal(u32(f[rows].view(torch.int32)), ref["scales"].view(np.uint32))
+        assert np.array_equal(u32(s_[rows]), ref["signs"])
+        qg, qo = unpack_codes(u32(c[rows])), unpack_codes(ref["codes"])
+        assert int(((qg != qo) & ~ref["near_tie"].astype(bool)).sum()) == 0
+    one = opq.quantize(ws[7], 0.73)
+    for a, b in zip(outs[7], one):
+        assert torch.equal(a, b)
