@@ -14,7 +14,7 @@
 // activation rows. Per CTA (one per SM, persistent):
 //   warp 0       raw producer: codes (64-byte swizzle) and signs of 128 weight rows,
 //                one load group (GRP consecutive 128-K blocks) per pair of TMA copies
-//   warp 1       TMEM allocation and MMA issue; A comes from TMEM. For BX <= 32 warps 19, 20
+//   warp 1       TMEM allocation and MMA issue; A comes from TMEM. For BX <= 64 warps 19, 20
 //                issue too: one issuer per decoder group, each with its own accumulator
 //   warp 2       x producer: the load group's x (BX rows, 128-byte swizzle), one copy
 //   warps 3..14  three decoder groups of 4 warps (= the 128 TMEM lanes): each thread owns
@@ -290,14 +290,15 @@ struct Cfg {
     // thread r of a group owns weight row r (TMEM lane r) and decodes its whole 128-K block row
     static constexpr int GROUPS = BX >= 256 ? 2 : 3;
     // MMA issuers. A narrow block's 8 MMAs take one issuing thread longer than a decoder group
-    // takes to decode the block, so narrow tiles (BX <= 32) give every decoder group an issuer
+    // takes to decode the block, so narrow tiles (BX <= 64) give every decoder group an issuer
     // of its own (issuer i issues the blocks group i decodes, into its own accumulator) and
     // the tensor pipe takes MMAs from three threads at once; wider tiles keep one issuer.
-    static constexpr int NISS = BX <= 32 ? GROUPS : 1;
+    static constexpr int NISS = BX <= 64 ? GROUPS : 1;
     // A ring in TMEM, in 128-K blocks (two 64-K half-stages of 32 columns each). With one
-    // issuer per group, block b uses slot b % A_BLOCKS and A_BLOCKS = 2 GROUPS, so every slot
-    // is used by one decoder group and one issuer only (two slots per group).
-    static constexpr int A_BLOCKS = NISS > 1 ? 2 * GROUPS : 4;
+    // issuer per group, block b uses slot b % A_BLOCKS and A_BLOCKS is a multiple of GROUPS,
+    // so every slot is used by one decoder group and one issuer only: two slots per group for
+    // BX <= 32, one for BX = 64 (whose three accumulators take 192 columns).
+    static constexpr int A_BLOCKS = NISS > 1 ? (BX <= 32 ? 2 : 1) * GROUPS : 4;
     static constexpr int A_STAGES = 2 * A_BLOCKS;      // 32 TMEM columns each (64 K of bf16 pairs)
     static constexpr int A_COLS = A_STAGES * 32;
     // x stages hold one load group (two 64-K swizzle atoms' worth of columns per block)
