@@ -344,4 +344,35 @@ OPQ_HD void decode8_table(uint32_t c, uint32_t sw, uint32_t j, uint32_t lw, uint
     out[3] = load(pair_offset(c, lw, 3)) ^ ((x << 3) & 0x80008000u);
 }
 
+#if defined(__CUDACC__)
+// Builds the pair table at shared-memory address `tab` with `nwarps` warps, this one warp `w` of
+// them. Warp store i (of 128) covers entries 2i and 2i + 1: lane l writes copies 4 (l & 7) ..
+// 4 (l & 7) + 3 of part (l >> 3) & 1 (0 value, 1 spread) of entry 2i + (l >> 4) in one 16-byte
+// store, so a warp store fills 512 contiguous bytes (no bank conflicts) and the loop loads nothing.
+// The magnitudes come by shuffles: for 4 bits, m0 = bf16 bits of LUT[lane & 15] and entry b is the
+// pair value(b); for other widths, m0 = LUT[lane], m1 = LUT[32 + lane] (codes 0 .. 2^BITS - 1)
+// and entry q < 2^BITS holds the magnitude of code q in both halves (0 above).
+template <int BITS = 4>
+__device__ __forceinline__ void build_pair_table(uint32_t tab, int w, int nwarps, int lane, uint32_t m0,
+                                                 uint32_t m1 = 0u) {
+    for (int i = w; i < 128; i += nwarps) {
+        const uint32_t b = 2u * (uint32_t)i + ((uint32_t)lane >> 4);
+        uint32_t v;
+        if (BITS == 4) {
+            const uint32_t lo = __shfl_sync(0xFFFFFFFFu, m0, (int)(b & 15u));
+            const uint32_t hi = __shfl_sync(0xFFFFFFFFu, m0, (int)(b >> 4));
+            v = lo | (hi << 16);
+        } else {
+            const uint32_t a0 = __shfl_sync(0xFFFFFFFFu, m0, (int)(b & 31u));
+            const uint32_t a1 = __shfl_sync(0xFFFFFFFFu, m1, (int)(b & 31u));
+            v = b < (1u << BITS) ? (b < 32u ? a0 : a1) * 0x00010001u : 0u;
+        }
+        if ((lane >> 3) & 1) v = sign_spread(b);
+        asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(tab + 512u * (uint32_t)i + 16u * (uint32_t)lane),
+                     "r"(v)
+                     : "memory");
+    }
+}
+#endif
+
 }  // namespace opqbits

@@ -241,7 +241,9 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, bool wide = false) {
     // blocks per load group: must match the kernel's Cfg<BX>::GRP
     p.grp = p.bx <= 16 ? 4 : (p.bx <= 64 ? 2 : 1);
     p.ngroups = (p.kblocks + p.grp - 1) / p.grp;
-    if (M <= 128 && !wide && p.n_tiles <= kCounterTiles) {
+    // stream-K (the kernel deals units in 32-bit arithmetic: units x CTAs below 2^31)
+    if (M <= 128 && !wide && p.n_tiles <= kCounterTiles &&
+        (int64_t)p.n_tiles * p.ngroups * kPlanSMs < ((int64_t)1 << 31)) {
         p.mode = 1;
         const int64_t U = (int64_t)p.n_tiles * p.ngroups;
         p.grid = (int)(U < kPlanSMs ? U : kPlanSMs);

@@ -189,10 +189,12 @@ __device__ __forceinline__ void make_group_table(opqbits::DecodeTable &T, const 
     }
 }
 
-// Units (tile, 128-K block) of CTA c out of C in stream-K mode: [begin(c), begin(c + 1)).
-__host__ __device__ __forceinline__ int64_t unit_begin(int64_t c, int64_t C, int64_t U) { return (c * U) / C; }
+// Units (tile, load group) of CTA c out of C in stream-K mode: [begin(c), begin(c + 1)).
+// 32-bit arithmetic (a 64-bit division is a long software routine on the critical path of every
+// role's start and of the fix-up): the host plans stream-K only when U * C < 2^31.
+__host__ __device__ __forceinline__ uint32_t unit_begin(uint32_t c, uint32_t C, uint32_t U) { return (c * U) / C; }
 // The CTA whose range holds unit u.
-__host__ __device__ __forceinline__ int64_t unit_owner(int64_t u, int64_t C, int64_t U) {
+__host__ __device__ __forceinline__ uint32_t unit_owner(uint32_t u, uint32_t C, uint32_t U) {
     return ((u + 1) * C - 1) / U;
 }
 
@@ -217,7 +219,8 @@ struct Run {
 struct RunIter {
     int mode, tiles, ng, grid, cta;
     LGroups lg;
-    int64_t u, u_end;   // mode 1: units = (tile, load group)
+    int t_cur, g_cur;   // mode 1: the next unit (tile, load group)
+    int left;           // mode 1: units left
     int t_next;         // mode 0
     int full_end;       // mode 0: tiles in whole waves (handed out strided)
     int split;          // mode 0: 1 or 2 runs per tile after the whole waves
@@ -235,9 +238,11 @@ struct RunIter {
         split = a.tail_split;
         full_end = split == 2 ? (tiles_ / grid_) * grid_ : tiles_;
         tail_done = false;
-        const int64_t U = (int64_t)tiles * ng;
-        u = unit_begin(cta_, grid_, U);
-        u_end = unit_begin(cta_ + 1, grid_, U);
+        const uint32_t U = (uint32_t)tiles * (uint32_t)ng;
+        const uint32_t u = unit_begin((uint32_t)cta_, (uint32_t)grid_, U);
+        left = (int)(unit_begin((uint32_t)cta_ + 1u, (uint32_t)grid_, U) - u);
+        t_cur = (int)(u / (uint32_t)ng);
+        g_cur = (int)(u - (uint32_t)t_cur * (uint32_t)ng);
     }
     // the next run for a tile of bx activation rows; false at the end
     __device__ __forceinline__ bool next(Run &R, int bx) {
@@ -260,12 +265,13 @@ struct RunIter {
             R.g0 = 0;
             R.g1 = ng;
         } else {
-            if (u >= u_end) return false;
-            R.tile = (int)(u / ng);
-            R.g0 = (int)(u - (int64_t)R.tile * ng);
-            const int64_t end = (int64_t)R.g0 + (u_end - u);
-            R.g1 = end < (int64_t)ng ? (int)end : ng;
-            u += R.g1 - R.g0;
+            if (left <= 0) return false;
+            R.tile = t_cur;
+            R.g0 = g_cur;
+            R.g1 = g_cur + left < ng ? g_cur + left : ng;
+            left -= R.g1 - R.g0;
+            ++t_cur;
+            g_cur = 0;
         }
         R.r0 = lg.start(R.g0);
         R.r1 = lg.start(R.g1);
@@ -442,14 +448,16 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
 
     if (warp == C::WARP_LOAD) {
         // ----------------------------------------------------------- raw producer
-        // one stage per load group: GRP blocks of codes and of signs
+        // one stage per load group: GRP blocks of codes and of signs. The first run is planned
+        // before the wait for the previous kernel (planning reads no global memory).
+        bool more = it.next(R, BX);
         pdl_wait();
         const int swd = args.K / 32;        // sign words per row
         int rs = 0;
         uint32_t rph = 0;
         int raw_issued = 0;
         bool ok = true;
-        while (ok && it.next(R, BX)) {
+        for (; ok && more; more = it.next(R, BX)) {
             const int n_blk = R.tile / args.m_tiles;
             for (int g = R.g0; g < R.g1 && ok; ++g) {
                 const int r = lg.start(g), nb = lg.start(g + 1) - r;
@@ -510,13 +518,14 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
         }
     } else if (warp == C::WARP_XLOAD) {
         // ----------------------------------------------------------- x producer
+        bool more = it.next(R, BX);
         pdl_wait();
         if (lane == 0) {
             int b = 0;                 // the CTA's block index
             int v = 0;                 // the CTA's load-group index
             int last_blk[C::X_STAGES]; // last block of the group each x stage holds
             bool ok = true;
-            while (ok && it.next(R, BX)) {
+            for (; ok && more; more = it.next(R, BX)) {
                 const int m_blk = R.tile % args.m_tiles;
                 // a half-width run loads its BX/2 activation rows with the half-height box
                 const bool half = R.xrows != BX;
@@ -617,15 +626,8 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
         // ----------------------------------------------------------- decoders
         // The pair table (only the decoders read it) is built here, while the producers' first
         // copies are in flight: 32 copies of value(b) then 32 copies of spread(b) per entry b.
-        // A warp writes whole entries (lane l the l-th copy), so the LUT entries it reads are the
-        // same in every lane: one broadcast load each instead of up to 16 serialised ones.
-        for (int e = warp - C::WARP_DEC0; e < 512; e += C::NUM_DEC_WARPS) {
-            const uint32_t b = (uint32_t)e & 255u;
-            const uint32_t v = e < 256 ? ((uint32_t)args.lut[b & 15u] | ((uint32_t)args.lut[b >> 4] << 16))
-                                       : opqbits::sign_spread(b);
-            const uint32_t dst = sbase + C::OFF_TABLE + b * 256u + (e < 256 ? 0u : 128u) + 4u * (uint32_t)lane;
-            asm volatile("st.shared.u32 [%0], %1;" ::"r"(dst), "r"(v) : "memory");
-        }
+        opqbits::build_pair_table(sbase + C::OFF_TABLE, warp - C::WARP_DEC0, C::NUM_DEC_WARPS, lane,
+                                  (uint32_t)args.lut[lane & 15]);
         // all decoder warps (named barrier 1) see the whole table before decoding
         asm volatile("bar.sync 1, %0;" ::"r"(C::NUM_DEC_WARPS * 32) : "memory");
         pdl_wait();   // the group-wise scales are read from global memory
@@ -726,7 +728,7 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
         pdl_wait();
         const int q = warp & 3;
         const int row = q * 32 + lane;
-        const int64_t U = (int64_t)tiles * args.ngroups;
+        const uint32_t U = (uint32_t)tiles * (uint32_t)args.ngroups;
         const bool vec_y = (args.N % 8) == 0;
         // per-warp staging for y: 2 buffers of [16 m][32 n] bf16
         const uint32_t stage0 = sbase + C::OFF_EPI + (uint32_t)(warp - C::WARP_EPI0) * 2048u;
@@ -834,8 +836,8 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
             if (!full) {
                 // The last of the tile's CTAs to get here (per lane quarter) adds every
                 // CTA's partial rows in CTA order, so the sum does not depend on timing.
-                const int64_t c_lo = unit_owner((int64_t)tile * args.ngroups, gridDim.x, U);
-                const int64_t c_hi = unit_owner((int64_t)(tile + 1) * args.ngroups - 1, gridDim.x, U);
+                const uint32_t c_lo = unit_owner((uint32_t)tile * (uint32_t)args.ngroups, gridDim.x, U);
+                const uint32_t c_hi = unit_owner((uint32_t)(tile + 1) * (uint32_t)args.ngroups - 1u, gridDim.x, U);
                 const uint32_t parts = (uint32_t)(c_hi - c_lo + 1);
                 // Publication without full fences: the warp's partial stores are ordered before lane
                 // 0's release-acquire add by a 32-thread named barrier (ids 2..5, one per warp), and
@@ -853,8 +855,8 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
                     // lane i (< parts) resolves part i's base; bases are broadcast by shuffles
                     const float *mybase = nullptr;
                     if ((uint32_t)lane < parts) {
-                        const int64_t c = c_lo + lane;
-                        const int64_t jj = tile - unit_begin(c, gridDim.x, U) / args.ngroups;
+                        const uint32_t c = c_lo + (uint32_t)lane;
+                        const uint32_t jj = (uint32_t)tile - unit_begin(c, gridDim.x, U) / (uint32_t)args.ngroups;
                         mybase = args.ws + ((size_t)c * args.runs_max + (size_t)jj) * (size_t)(BX * C::BW);
                     }
                     // Every lane runs the loops (shuffles need all lanes); only rows < N store.
@@ -864,8 +866,8 @@ __global__ void __launch_bounds__(Cfg<BX>::THREADS, 1)
                         if (p < 32)
                             return reinterpret_cast<const float *>(
                                 __shfl_sync(0xFFFFFFFFu, reinterpret_cast<unsigned long long>(mybase), (int)p));
-                        const int64_t c = c_lo + p;
-                        const int64_t jj = tile - unit_begin(c, gridDim.x, U) / args.ngroups;
+                        const uint32_t c = c_lo + p;
+                        const uint32_t jj = (uint32_t)tile - unit_begin(c, gridDim.x, U) / (uint32_t)args.ngroups;
                         return args.ws + ((size_t)c * args.runs_max + (size_t)jj) * (size_t)(BX * C::BW);
                     };
                     const int mcols = min(BX, args.M - m_blk * BX);

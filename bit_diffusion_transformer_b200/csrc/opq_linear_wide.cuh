@@ -331,18 +331,13 @@ __global__ void __launch_bounds__(Cfg<BX, BITS>::THREADS, 1)
         }
     }
     // ---- pair table: 32 copies of value(b) then 32 copies of spread(b) per entry b
-    for (int e = threadIdx.x; e < 512; e += C::THREADS) {
-        const uint32_t b = (uint32_t)e & 255u;
-        // 4 bits: entry b holds the pair of magnitudes of code byte b; other widths: entry q < 2^BITS
-        // holds the magnitude of code q in both halves
-        const uint32_t v = e >= 256 ? opqbits::sign_spread(b)
-                           : BITS == 4 ? ((uint32_t)args.lut[b & 15u] | ((uint32_t)args.lut[b >> 4] << 16))
-                                       : (b < (1u << BITS) ? (uint32_t)args.lutb[b] * 0x00010001u : 0u);
-        const uint32_t dst = sbase + C::OFF_TABLE + b * 256u + (e < 256 ? 0u : 128u);
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst + 16u * k), "r"(v) : "memory");
-    }
+    // (4 bits: entry b holds the pair of magnitudes of code byte b; other widths: entry q < 2^BITS
+    // holds the magnitude of code q in both halves)
+    if (BITS == 4)
+        opqbits::build_pair_table<4>(sbase + C::OFF_TABLE, warp, C::THREADS / 32, lane, (uint32_t)args.lut[lane & 15]);
+    else
+        opqbits::build_pair_table<BITS>(sbase + C::OFF_TABLE, warp, C::THREADS / 32, lane, (uint32_t)args.lutb[lane],
+                                        (uint32_t)args.lutb[32 + lane]);
     if (warp == C::WARP_MMA) {
         tmem_alloc(tmem_slot, C::TMEM_COLS);
         tmem_relinquish();
