@@ -164,6 +164,14 @@ def test_plan_and_workspace_host_logic(lib):
         runs_max = -(-per // groups) + 1
         counters = 4096 * 4 * 4        # fixed region: 4 arrival counters for each of up to 4096 weight tiles
         assert opq.workspace_size(M, N, K) == counters + ctas * runs_max * bx * 128 * 4
+    # stream-K deals its units in 32-bit arithmetic: it is planned only while units x 148 CTAs
+    # stays below 2^31 (4096 weight tiles x 3542 load groups of 4 blocks is the last such shape)
+    for groups in (3541, 3542, 3543, 4000):
+        K = 128 * 4 * groups
+        units = 4096 * groups
+        path, ctas, _ = opq.plan(1, 4096 * 128, K)
+        assert path == (1 if units * 148 < 2 ** 31 else 0) and ctas == 148
+        assert (opq.workspace_size(1, 4096 * 128, K) > 0) == (path == 1)
     # large M: whole 128 x 256 tiles, one persistent CTA per SM. Tiles past the last whole wave,
     # when at most half as many as CTAs, run on two CTAs each; 256-row tiles of at least 8
     # 128-K blocks split K, and their fp32 partial sums (128 x 256 per tail tile) meet in the
