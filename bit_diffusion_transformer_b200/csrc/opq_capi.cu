@@ -270,7 +270,9 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, bool wide = false) {
                 p.tail_split = 3;
                 p.counter_bytes = kCounterBytes;
                 p.ws_bytes = p.counter_bytes + (size_t)tail * 256u * 128u * sizeof(float);
-            } else if (p.bx >= 32) {
+            } else if (p.bx >= 32 && p.grp == 1) {
+                // half-width runs load their activation rows with a 2-D half-height box, so
+                // only tiles that fetch one block per copy take them
                 p.tail_split = 2;
             }
         }
@@ -311,6 +313,9 @@ cudaError_t launch_linear(DeviceInfo *di, const Plan &plan, const CUtensorMap &x
                           const CUtensorMap &cmap, const CUtensorMap &smap, const opqk::LinearArgs &a,
                           cudaStream_t st) {
     using C = opqk::Cfg<BX>;
+    // half-width runs exist only for one block per copy (2-D x boxes); the plan never asks for
+    // them otherwise, and a launch that did is refused here
+    if (a.tail_split == 2 && C::GRP != 1) return cudaErrorInvalidConfiguration;
     const int key = BX == 16 ? 0 : BX == 32 ? 1 : BX == 64 ? 2 : 3;
     if (!di->linear_attr[gs_index(GS)][key]) {
         cudaError_t e = cudaFuncSetAttribute(opqk::linear_kernel<BX, GS>, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -346,6 +346,53 @@ def test_full_whole_model_sampled_layers():
         linear_parity(x, w, lin.alpha, pairs=800)
 
 
+def linear_parity_planes(M, N, K, seed, pairs, extra_rows):
+    """GPU linear vs the fp64 oracle on random packed planes (no quantize: the largest shapes),
+    at sampled output positions plus every activation row of `extra_rows` weight rows."""
+    codes, signs, scales = workloads.random_planes(N, K, seed)
+    x_cpu = workloads.Linear("planes", M, N, K, x_seed=seed + 1).make_x("cpu")
+    yb, y, pad = guarded((M, N), torch.bfloat16, 0x6B)
+    opq.linear(x_cpu.to(DEV), to_dev_u32(codes), to_dev_u32(signs), torch.from_numpy(scales).to(DEV), 0.73, out=y)
+    torch.cuda.synchronize()
+    check_guards(yb, pad, 0x6B)
+    no_device_error()
+    rng = np.random.default_rng(seed)
+    ms = np.concatenate([rng.integers(0, M, pairs), np.repeat(np.arange(M), len(extra_rows))])
+    ns = np.concatenate([rng.integers(0, N, pairs), np.tile(np.asarray(extra_rows), M)])
+    yref, bound = oracle.linear_pairs(x_cpu, codes, signs, scales, 0.73, ms, ns)
+    got = bits_to_f64(u16(y))[ms, ns]
+    err = np.abs(got - yref)
+    tol = 1e-2 * bound + 1e-3
+    bad = err > tol
+    assert not bad.any(), f"{int(bad.sum())} outputs out of tolerance; worst excess {float((err - tol).max())}"
+    assert np.isfinite(got).all()
+
+
+@pytest.mark.parametrize("M", [1, 16])
+def test_linear_stream_k_most_tiles(M):
+    # the largest stream-K shape by weight tiles (4096: the arrival counters' whole region),
+    # K = 1024 (two load groups per tile, so CTA boundaries split tiles all along N)
+    N, K = 4096 * 128, 1024
+    path, ctas, _ = opq.plan(M, N, K)
+    assert path == 1 and ctas == 148
+    rows = [0, 1, 127, 128, N // 2, N - 129, N - 128, N - 2, N - 1]
+    linear_parity_planes(M, N, K, seed=1000 + M, pairs=1500, extra_rows=rows)
+
+
+@pytest.mark.parametrize("M", [8, 40, 100])
+def test_linear_narrow_whole_tiles(M):
+    # more weight tiles than the counter region (4194 > 4096): small M runs whole narrow tiles
+    # strided over the CTAs; 4194 = 28 waves of 148 + 50 tiles, which at M = 100 (128-row
+    # tiles, one block per copy) run as two half-width runs each (16- to 64-row tiles fetch
+    # several blocks per copy and run them whole); a ragged last tile (N = 4194 x 128 - 37)
+    N, K = 4194 * 128 - 37, 256
+    path, ctas, _ = opq.plan(M, N, K)
+    assert path == 0 and ctas == 148
+    tail0 = 4144 * 128
+    rows = [0, 5, tail0 - 1, tail0, tail0 + 77, N - 90, N - 2, N - 1]
+    linear_parity_planes(M, N, K, seed=2000 + M, pairs=1500, extra_rows=rows)
+
+
 def test_linear_workspace_reuse_across_shapes():
     """One zero-filled workspace serves calls of different shapes in a row: every
     call leaves its arrival counters at zero for the next one."""

@@ -53,6 +53,19 @@ def student_t4(shape, std: float, gen: torch.Generator, device) -> torch.Tensor:
     return (t * (std / math.sqrt(2.0))).to(torch.bfloat16)
 
 
+def random_planes(N: int, K: int, seed: int):
+    """Packed planes of random bits for an N x K weight, as numpy arrays: codes uint32 [N, K/8]
+    (any nibble is a valid level), signs uint32 [N, K/32] and positive fp32 row maxima [N] in
+    [0.01, 0.1). Inputs for the linear at sizes where quantizing a weight first would take the
+    oracle too long; nothing of the method is computed here."""
+    import numpy as np
+    rng = np.random.default_rng(int(seed))
+    codes = rng.integers(0, 1 << 32, size=(N, K // 8), dtype=np.uint32)
+    signs = rng.integers(0, 1 << 32, size=(N, K // 32), dtype=np.uint32)
+    scales = (0.01 + 0.09 * rng.random(N)).astype(np.float32)
+    return codes, signs, scales
+
+
 def add_outlier_rows(w: torch.Tensor, frac: float, std: float, gen: torch.Generator) -> torch.Tensor:
     n, k = w.shape
     count = int(round(frac * n))
