@@ -147,9 +147,11 @@ def linear_bits_parity(x_cpu, w_cpu, bits, alpha, rows=None):
 
 
 @pytest.mark.parametrize("bits", [3, 5, 6])
-@pytest.mark.parametrize("M,N,K", [(1, 256, 512), (16, 384, 1024), (300, 131, 640), (700, 256, 384)])
+@pytest.mark.parametrize("M,N,K", [(1, 256, 512), (16, 384, 1024), (300, 131, 640), (700, 256, 384),
+                                   (512, 10240, 256)])
 def test_linear_bits(bits, M, N, K):
     # ragged activation and weight rows, several 128-K blocks; every M runs the 256-row tiles
+    # (512 x 10240 x 256: 160 tiles, the 12 past the first wave as two half-width runs each)
     lin = workloads.Linear("bits-lin", M, N, K, w_seed=M + N + K + bits, x_seed=7 * bits + M)
     x, w = lin.make("cpu")
     linear_bits_parity(x, w, bits, 0.73)

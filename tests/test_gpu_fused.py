@@ -35,7 +35,8 @@ def check(yg, yref, bound, b):
 
 @pytest.mark.parametrize("act", list(ACTS))
 @pytest.mark.parametrize("with_bias", [True, False])
-@pytest.mark.parametrize("M,N,K", [(1, 300, 512), (40, 1000, 640), (300, 130, 1280), (512, 10240, 1024)])
+@pytest.mark.parametrize("M,N,K", [(1, 300, 512), (40, 1000, 640), (300, 130, 1280), (512, 10240, 1024),
+                                   (512, 10240, 256)])
 def test_linear_fused(act, with_bias, M, N, K):
     lin = workloads.Linear("fused", M, N, K, w_seed=M + N, x_seed=K)
     x, w = lin.make("cpu")
