@@ -210,6 +210,7 @@ struct Plan {
     size_t counter_bytes;   // mode 1: the zero-between-calls arrival counters at the workspace start
     size_t ws_bytes;
     int launches;
+    bool unsupported;   // a shape no schedule serves: OPQ_ERR_UNSUPPORTED_SHAPE
 };
 
 // The schedule depends on the shape alone (a fixed 148-CTA budget), so the
@@ -242,8 +243,13 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, bool wide = false) {
     p.grp = p.bx <= 16 ? 4 : (p.bx <= 64 ? 2 : 1);
     p.ngroups = (p.kblocks + p.grp - 1) / p.grp;
     // stream-K (the kernel deals units in 32-bit arithmetic: units x CTAs below 2^31)
-    if (M <= 128 && !wide && p.n_tiles <= kCounterTiles &&
-        (int64_t)p.n_tiles * p.ngroups * kPlanSMs < ((int64_t)1 << 31)) {
+    const bool stream_k = M <= 128 && !wide && p.n_tiles <= kCounterTiles &&
+                          (int64_t)p.n_tiles * p.ngroups * kPlanSMs < ((int64_t)1 << 31);
+    // whole narrow tiles (past stream-K's range) only for whole 128-K blocks: with the sign
+    // words copied by cp.async, max-size tests of that schedule faulted (narrow tiles) or
+    // returned wrong sums for a few tiles (256-row tiles at M = 8); the entry points refuse it
+    p.unsupported = M <= 128 && !wide && !stream_k && K % 128 != 0;
+    if (stream_k) {
         p.mode = 1;
         const int64_t U = (int64_t)p.n_tiles * p.ngroups;
         p.grid = (int)(U < kPlanSMs ? U : kPlanSMs);
@@ -316,6 +322,8 @@ cudaError_t launch_linear(DeviceInfo *di, const Plan &plan, const CUtensorMap &x
     // half-width runs exist only for one block per copy (2-D x boxes); the plan never asks for
     // them otherwise, and a launch that did is refused here
     if (a.tail_split == 2 && C::GRP != 1) return cudaErrorInvalidConfiguration;
+    // whole-tile schedules of the narrow kernel only for whole 128-K blocks (signs by TMA)
+    if (a.mode == 0 && a.signs_tma == 0) return cudaErrorInvalidConfiguration;
     const int key = BX == 16 ? 0 : BX == 32 ? 1 : BX == 64 ? 2 : 3;
     if (!di->linear_attr[gs_index(GS)][key]) {
         cudaError_t e = cudaFuncSetAttribute(opqk::linear_kernel<BX, GS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -767,7 +775,9 @@ opq_status opq_linear_workspace_size(int64_t M, int64_t N, int64_t K, size_t *by
     opq_status s = check_sizes(N, K);
     if (s != OPQ_OK) return s;
     if (M > INT32_MAX) return OPQ_ERR_UNSUPPORTED_SHAPE;
-    *bytes = make_plan(M, N, K).ws_bytes;
+    const Plan p = make_plan(M, N, K);
+    if (p.unsupported) return OPQ_ERR_UNSUPPORTED_SHAPE;
+    *bytes = p.ws_bytes;
     return OPQ_OK;
 }
 
@@ -777,6 +787,7 @@ opq_status opq_linear_plan(int64_t M, int64_t N, int64_t K, int *path, int *ctas
     if (s != OPQ_OK) return s;
     if (M > INT32_MAX) return OPQ_ERR_UNSUPPORTED_SHAPE;
     const Plan p = make_plan(M, N, K);
+    if (p.unsupported) return OPQ_ERR_UNSUPPORTED_SHAPE;
     if (path) *path = p.mode;
     if (ctas) *ctas = p.grid;
     if (launches) *launches = p.launches;
@@ -816,6 +827,7 @@ static opq_status linear_impl(const uint16_t *x, int64_t M, int64_t K, const uin
         return s;
     if (bias && (s = check_ptrs({bias})) != OPQ_OK) return s;
     const Plan plan = make_plan(M, N, K);
+    if (plan.unsupported) return OPQ_ERR_UNSUPPORTED_SHAPE;
     if (plan.ws_bytes > 0) {
         if (workspace == nullptr || workspace_bytes < plan.ws_bytes) return OPQ_ERR_WORKSPACE;
         if ((s = check_ptrs({workspace})) != OPQ_OK) return s;
@@ -938,7 +950,9 @@ opq_status opq_linear_bits_workspace_size(int64_t M, int64_t N, int64_t K, int32
     if (!bytes) return OPQ_ERR_INVALID_ARG;
     opq_status s = check_bits_linear(M, N, K, bits);
     if (s != OPQ_OK) return s;
-    *bytes = bits == 4 ? make_plan(M, N, K).ws_bytes : make_plan(M, N, K, true).ws_bytes;
+    const Plan p = bits == 4 ? make_plan(M, N, K) : make_plan(M, N, K, true);
+    if (p.unsupported) return OPQ_ERR_UNSUPPORTED_SHAPE;
+    *bytes = p.ws_bytes;
     return OPQ_OK;
 }
 
@@ -1011,7 +1025,9 @@ opq_status opq_linear_grouped_workspace_size(int64_t M, int64_t N, int64_t K, in
     if (s != OPQ_OK) return s;
     if ((s = check_group(K, group_size)) != OPQ_OK) return s;
     if (M > INT32_MAX) return OPQ_ERR_UNSUPPORTED_SHAPE;
-    *bytes = make_plan(M, N, K).ws_bytes;
+    const Plan p = make_plan(M, N, K);
+    if (p.unsupported) return OPQ_ERR_UNSUPPORTED_SHAPE;
+    *bytes = p.ws_bytes;
     return OPQ_OK;
 }
 

@@ -258,7 +258,11 @@ opq_status opq_linear_workspace_size(int64_t M, int64_t N, int64_t K, size_t *by
  * opq_linear — y = x W'^T with W' decoded from the packed planes (the card's
  * OPQLinear forward: decode w' = sign * (q/15)^(1/alpha) * max, then matmul).
  *   x          bf16 [M, K] device, row-major (leading dimension K)
- *   M, K       activation rows and the reduction length (K % 32 == 0)
+ *   M, K       activation rows and the reduction length (K % 32 == 0). M <= 128 with
+ *              more than 4096 128-row weight tiles (N > 524288), or with
+ *              ceil(N/128) x (load groups per tile) x 148 >= 2^31, needs K % 128 == 0
+ *              (OPQ_ERR_UNSUPPORTED_SHAPE otherwise, also from the workspace size and
+ *              the plan)
  *   codes, signs, scales   packed W [N, K] (device)
  *   N          output features
  *   alpha      the power used to quantize

@@ -172,11 +172,22 @@ def test_plan_and_workspace_host_logic(lib):
         path, ctas, _ = opq.plan(1, 4096 * 128, K)
         assert path == (1 if units * 148 < 2 ** 31 else 0) and ctas == 148
         assert (opq.workspace_size(1, 4096 * 128, K) > 0) == (path == 1)
+    # small M past stream-K's range runs whole narrow tiles only for whole 128-K blocks; with
+    # K % 128 != 0 (sign words copied by cp.async) that schedule is refused, not run
+    sz = ctypes.c_size_t(0)
+    pth, cts, lau = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
+    for M, N, K in [(8, 4194 * 128 - 37, 160), (100, 4097 * 128, 96), (1, 4096 * 128, 128 * 4 * 3543 + 32)]:
+        assert lib.opq_linear_workspace_size(M, N, K, ctypes.byref(sz)) == 2
+        assert lib.opq_linear_plan(M, N, K, ctypes.byref(pth), ctypes.byref(cts), ctypes.byref(lau)) == 2
+        with pytest.raises(opq.OPQError):
+            opq.plan(M, N, K)
+    assert opq.plan(129, 4097 * 128, 96)[0] == 0          # M > 128: the 256-row tiles serve it
+    assert opq.plan(8, 4096 * 128, 160)[0] == 1           # within stream-K's range: served
     # large M: whole 128 x 256 tiles, one persistent CTA per SM. Tiles past the last whole wave,
     # when at most half as many as CTAs, run on two CTAs each; 256-row tiles of at least 8
     # 128-K blocks split K, and their fp32 partial sums (128 x 256 per tail tile) meet in the
     # workspace after the counter region; everything else needs no workspace
-    for M, N, K in [(129, 100, 32), (3072, 3840, 3840), (4096, 10240, 3840), (8, 4097 * 128, 64),
+    for M, N, K in [(129, 100, 32), (3072, 3840, 3840), (4096, 10240, 3840), (8, 4097 * 128, 128),
                     (512, 10240, 256), (512, 10240, 1024), (300, 9728, 160)]:
         path, ctas, launches = opq.plan(M, N, K)
         assert path == 0 and launches == 1

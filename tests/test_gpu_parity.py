@@ -368,29 +368,31 @@ def linear_parity_planes(M, N, K, seed, pairs, extra_rows):
     assert np.isfinite(got).all()
 
 
-@pytest.mark.parametrize("M", [1, 16])
-def test_linear_stream_k_most_tiles(M):
+@pytest.mark.parametrize("M,K", [(1, 1024), (16, 1024), (1, 1056)])
+def test_linear_stream_k_most_tiles(M, K):
     # the largest stream-K shape by weight tiles (4096: the arrival counters' whole region),
-    # K = 1024 (two load groups per tile, so CTA boundaries split tiles all along N)
-    N, K = 4096 * 128, 1024
+    # K = 1024 (two load groups per tile, so CTA boundaries split tiles all along N); K = 1056
+    # (not a whole number of 128-K blocks: 128-row tiles, one block per copy, signs by cp.async)
+    N = 4096 * 128
     path, ctas, _ = opq.plan(M, N, K)
     assert path == 1 and ctas == 148
     rows = [0, 1, 127, 128, N // 2, N - 129, N - 128, N - 2, N - 1]
-    linear_parity_planes(M, N, K, seed=1000 + M, pairs=1500, extra_rows=rows)
+    linear_parity_planes(M, N, K, seed=1000 + M + K, pairs=1500, extra_rows=rows)
 
 
-@pytest.mark.parametrize("M", [8, 40, 100])
-def test_linear_narrow_whole_tiles(M):
+@pytest.mark.parametrize("M,K", [(8, 256), (40, 256), (100, 256)])
+def test_linear_narrow_whole_tiles(M, K):
     # more weight tiles than the counter region (4194 > 4096): small M runs whole narrow tiles
     # strided over the CTAs; 4194 = 28 waves of 148 + 50 tiles, which at M = 100 (128-row
     # tiles, one block per copy) run as two half-width runs each (16- to 64-row tiles fetch
-    # several blocks per copy and run them whole); a ragged last tile (N = 4194 x 128 - 37)
-    N, K = 4194 * 128 - 37, 256
+    # several blocks per copy and run them whole); a ragged last tile (N = 4194 x 128 - 37).
+    # The same shapes with K % 128 != 0 are refused (test_abi)
+    N = 4194 * 128 - 37
     path, ctas, _ = opq.plan(M, N, K)
     assert path == 0 and ctas == 148
     tail0 = 4144 * 128
     rows = [0, 5, tail0 - 1, tail0, tail0 + 77, N - 90, N - 2, N - 1]
-    linear_parity_planes(M, N, K, seed=2000 + M, pairs=1500, extra_rows=rows)
+    linear_parity_planes(M, N, K, seed=2000 + M + K, pairs=1500, extra_rows=rows)
 
 
 def test_linear_workspace_reuse_across_shapes():
