@@ -188,6 +188,29 @@ def test_linear_grouped_tails(M, N, K, gs):
     grouped_linear_parity(x, w, gs, 0.73)
 
 
+@pytest.mark.parametrize("M,K,gs", [(16, 1024, 128), (40, 512, 64)])
+def test_linear_grouped_narrow_whole_tiles(M, K, gs):
+    # more weight tiles than the stream-K counters cover (4194 > 4096): small M runs whole narrow
+    # tiles with the group-wise decode; random packed planes and maxima, sampled outputs
+    N = 4194 * 128 - 37
+    assert opq.plan(M, N, K)[0] == 0
+    codes, signs, _ = workloads.random_planes(N, K, 11)
+    gmax = workloads.random_gmax(N, K // gs, 12)
+    x = workloads.Linear("grouped-whole", M, N, K, x_seed=13).make_x("cpu")
+    y = opq.linear_grouped(x.to(DEV), to_dev_u32(codes), to_dev_u32(signs),
+                           torch.from_numpy(gmax.view(np.int16)).to(DEV), 0.73)
+    torch.cuda.synchronize()
+    no_device_error()
+    rng = np.random.default_rng(14)
+    ms = np.concatenate([rng.integers(0, M, 3000), np.arange(M), np.arange(M)])
+    ns = np.concatenate([rng.integers(0, N, 3000), np.full(M, N - 1), np.zeros(M, np.int64)])
+    yref, bound = oracle.linear_grouped_pairs(x, codes, signs, gmax, 0.73, ms, ns)
+    got = (u16(y).astype(np.uint32) << 16).view(np.float32).astype(np.float64)[ms, ns]
+    err = np.abs(got - yref)
+    tol = 1e-2 * bound + 1e-3
+    assert not (err > tol).any(), f"{int((err > tol).sum())} outputs out of tolerance"
+
+
 def test_linear_grouped_full_size_sampled():
     lin = workloads.dit_attn_proj()
     x, w = lin.make("cpu")

@@ -66,6 +66,14 @@ def random_planes(N: int, K: int, seed: int):
     return codes, signs, scales
 
 
+def random_gmax(N: int, groups: int, seed: int):
+    """float16 group maxima [N, groups] in [0.01, 0.1), as their uint16 bit patterns (numpy): with
+    random_planes, the group-wise format's inputs for the linear at the largest sizes."""
+    import numpy as np
+    rng = np.random.default_rng(int(seed))
+    return (0.01 + 0.09 * rng.random((N, groups))).astype(np.float16).view(np.uint16)
+
+
 def add_outlier_rows(w: torch.Tensor, frac: float, std: float, gen: torch.Generator) -> torch.Tensor:
     n, k = w.shape
     count = int(round(frac * n))
